@@ -1,0 +1,393 @@
+"""CPU oracle for group-wise lookup-table (LUT) weight quantization and the
+dequantize-and-multiply product.
+
+TEST INFRASTRUCTURE ONLY.  This is the plain, slow reference that the CUDA
+library is checked against.  Only the test suite, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import it.  It shares no code with
+the CUDA library and imports nothing from it.
+
+What it follows (web pages, cited by title and section):
+
+* FLUTE abstract ("Daily Papers" listing, query "group-128"): weight-only
+  quantization onto a non-uniform lookup table, NormalFloat tables, group size
+  128, 3-bit (non-evenly-divisible) widths, and an offline restructuring of the
+  quantized matrix so that unpacking needs few bit operations.
+* BitMoD abstract (same listing): groups of 128 weights, the per-group partial
+  sum rescaled once by the group's scale.
+* Group-128 post-training-quantization study (same listing): round-to-nearest
+  (RTN) quantization at group size 128.
+* Log_bQuant abstract (catalyzex author page): a codebook spaced in
+  logarithmic space with an adjustable base.
+* "TurboQuant: A first-principles walkthrough": the Lloyd-Max algorithm for an
+  optimal scalar quantizer.
+
+The pages print no constants, packing layout or worked example.  Where they are
+silent the build's readings are used and stated at each function:
+
+* codebooks are computed in fp64 and rounded once to bf16 (round to nearest
+  even); NormalFloat uses the 8-positive / 7-negative / zero quantile
+  construction; the log codebook is +-b^-k, k = 0..7, b = 1.6; the 3-bit table is
+  the 8-level Lloyd-Max quantizer of N(0,1) normalised to max |level| = 1;
+* the group scale is the group's absolute maximum (exact in bf16);
+* RTN: v = fp32(w) / fp32(s) (IEEE divide), the code is the lowest index i
+  minimising the fp32 value |v - c_i|; an all-zero group uses v = 0;
+* the product is y[m, n] = sum_g s[n, g] * sum_{k in g} x[m, k] * c[q[n, k]]
+  accumulated in fp64 (every product is exact in fp64).
+
+Parity of every function here is pinned in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import math
+from typing import Tuple
+
+import numpy as np
+import scipy.special
+
+GROUP = 128          # weights per quantization group along K
+STRIP = 32           # rows per packing strip (layout V1)
+LAYOUT_VERSION = 1
+
+CODEBOOK_KINDS = ("nf4", "logb", "lloyd_max3", "uniform4")
+
+
+# --------------------------------------------------------------------------
+# bf16 helpers
+# --------------------------------------------------------------------------
+
+def bf16_round(values) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (ties to even), once.
+
+    bf16 keeps 8 significant bits.  For a normal value v = m * 2^e with
+    m in [1, 2), the result is round_half_even(m * 2^7) * 2^(e-7).
+    Returns fp64 values that are exactly representable in bf16.
+    """
+    v = np.asarray(values, dtype=np.float64)
+    out = np.zeros_like(v)
+    nz = v != 0.0
+    mant, expo = np.frexp(v[nz])            # v = mant * 2^expo, |mant| in [0.5, 1)
+    # 8 significant bits: scale |mant| in [0.5,1) by 2^8 -> [128, 256)
+    q = np.rint(mant * 256.0)               # numpy rint rounds half to even
+    out[nz] = np.ldexp(q, expo - 8)
+    return out
+
+
+def bf16_bits(values) -> np.ndarray:
+    """Bit patterns (uint16) of values that are exactly bf16-representable."""
+    f32 = np.asarray(values, dtype=np.float64).astype(np.float32)
+    if not np.array_equal(f32.astype(np.float64), np.asarray(values, dtype=np.float64)):
+        raise ValueError("value not representable in fp32")
+    bits = f32.view(np.uint32)
+    if np.any(bits & 0xFFFF):
+        raise ValueError("value not representable in bf16")
+    return (bits >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits) -> np.ndarray:
+    """uint16 bf16 bit patterns -> float32 values (exact)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32)
+
+
+# --------------------------------------------------------------------------
+# Codebooks (fp64), each normalised to max |level| = 1
+# --------------------------------------------------------------------------
+
+def nf4_levels() -> np.ndarray:
+    """16-level NormalFloat table (FLUTE abstract: "lookup table-based
+    NormalFloat quantization").
+
+    Reading: levels are standard-normal quantiles.  A table with an exact zero
+    and 16 entries cannot be symmetric, so it takes 8 positive quantiles, 7
+    negative ones and 0.  The outermost probability is
+    delta = ((1 - 1/30) + (1 - 1/32)) / 2.  Positive levels are Phi^-1(p) for
+    the 9 equally spaced p from delta down to 1/2, dropping 1/2; negative levels
+    are -Phi^-1(p) for the 8 equally spaced p from delta to 1/2, dropping 1/2.
+    The table is sorted and divided by Phi^-1(delta).
+    """
+    delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0))
+    p_pos = np.linspace(delta, 0.5, 9)[:-1]
+    p_neg = np.linspace(delta, 0.5, 8)[:-1]
+    pos = scipy.special.ndtri(p_pos)
+    neg = -scipy.special.ndtri(p_neg)
+    levels = np.sort(np.concatenate([neg, [0.0], pos]))
+    return levels / scipy.special.ndtri(delta)
+
+
+def logb_levels(base: float = 1.6, per_sign: int = 8) -> np.ndarray:
+    """Logarithmic table (Log_bQuant abstract: logarithmic space, adjustable
+    base).  Reading: +-base^-k for k = 0 .. per_sign-1, no zero level."""
+    mags = base ** (-np.arange(per_sign, dtype=np.float64))
+    return np.sort(np.concatenate([-mags, mags]))
+
+
+def _std_normal_pdf(t):
+    return np.exp(-0.5 * np.square(t)) / math.sqrt(2.0 * math.pi)
+
+
+def _std_normal_mass(a, b):
+    """P(a < Z < b) for Z ~ N(0,1), using the tail that avoids cancellation."""
+    if a >= 0.0:
+        return scipy.special.ndtr(-a) - scipy.special.ndtr(-b)
+    return scipy.special.ndtr(b) - scipy.special.ndtr(a)
+
+
+def lloyd_max_normal(n_levels: int = 8, tol: float = 1e-13,
+                     max_iter: int = 100000) -> Tuple[np.ndarray, np.ndarray]:
+    """Lloyd-Max quantizer of N(0,1) ("TurboQuant: A first-principles
+    walkthrough" names the Lloyd-Max algorithm).
+
+    Alternates the two optimality conditions until the levels move less than
+    ``tol``: thresholds are midpoints of adjacent levels; each level is the
+    conditional mean of Z over its cell, E[Z | a < Z < b] =
+    (pdf(a) - pdf(b)) / P(a < Z < b).  Returns (levels, thresholds), unnormalised.
+    """
+    y = np.linspace(-2.0, 2.0, n_levels)
+    for _ in range(max_iter):
+        t = np.concatenate([[-np.inf], 0.5 * (y[:-1] + y[1:]), [np.inf]])
+        y_new = np.empty_like(y)
+        for i in range(n_levels):
+            a, b = t[i], t[i + 1]
+            pa = 0.0 if np.isinf(a) else _std_normal_pdf(a)
+            pb = 0.0 if np.isinf(b) else _std_normal_pdf(b)
+            y_new[i] = (pa - pb) / _std_normal_mass(a, b)
+        step = np.max(np.abs(y_new - y))
+        y = y_new
+        if step < tol:
+            break
+    t = 0.5 * (y[:-1] + y[1:])
+    return y, t
+
+
+def lloyd_max3_levels() -> np.ndarray:
+    """8-level Lloyd-Max table for N(0,1), divided by its largest level."""
+    y, _ = lloyd_max_normal(8)
+    return y / np.max(np.abs(y))
+
+
+def uniform4_levels() -> np.ndarray:
+    """16 evenly spaced levels (2i - 15) / 15 (a uniform LUT, used by tests)."""
+    return (2.0 * np.arange(16) - 15.0) / 15.0
+
+
+def codebook(kind: str, bits: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Return (bf16 bit patterns uint16[2^bits], float32 values) for a kind."""
+    if kind == "nf4" and bits == 4:
+        lv = nf4_levels()
+    elif kind == "logb" and bits == 4:
+        lv = logb_levels()
+    elif kind == "lloyd_max3" and bits == 3:
+        lv = lloyd_max3_levels()
+    elif kind == "uniform4" and bits == 4:
+        lv = uniform4_levels()
+    else:
+        raise ValueError(f"no codebook {kind!r} with {bits} bits")
+    r = bf16_round(lv)
+    bits16 = bf16_bits(r)
+    return bits16, bf16_bits_to_f32(bits16)
+
+
+# --------------------------------------------------------------------------
+# RTN quantization (group absmax scale, nearest level)
+# --------------------------------------------------------------------------
+
+def quantize(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Quantize W[N, K] (values exactly bf16, given as float32) per group of 128.
+
+    s[n, g] = max_{k in g} |W[n, k]|   (a bf16 value, so stored exactly)
+    v = fp32(W) / fp32(s)              (IEEE division; 0 when s == 0)
+    q = lowest i minimising fp32 |v - c_i|, scanning i = 0 .. 2^bits - 1 and
+        replacing the best only on a strictly smaller distance.
+
+    Returns (codes uint8[N, K], scale bf16 bit patterns uint16[N, K/128]).
+    Raises ValueError on non-finite weights.
+    """
+    w = np.asarray(w, dtype=np.float32)
+    n, k = w.shape
+    if k % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    if not np.all(np.isfinite(w)):
+        raise ValueError("non-finite weight")
+    levels = np.asarray(levels_f32, dtype=np.float32)
+    if levels.shape != (1 << bits,):
+        raise ValueError("codebook size must be 2^bits")
+    g = k // GROUP
+    wg = w.reshape(n, g, GROUP)
+    s = np.max(np.abs(wg), axis=2)                          # float32, exact
+    s_b = np.broadcast_to(s[:, :, None], wg.shape)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s_b > 0, wg / s_b, np.float32(0.0)).astype(np.float32)
+    best_d = np.full(v.shape, np.inf, dtype=np.float32)
+    best_i = np.zeros(v.shape, dtype=np.uint8)
+    for i in range(levels.size):
+        d = np.abs(v - levels[i])                           # float32 subtract
+        take = d < best_d
+        best_i[take] = i
+        best_d[take] = d[take]
+    scale_bits = (s.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    return best_i.reshape(n, k), scale_bits
+
+
+# --------------------------------------------------------------------------
+# Packing, layout V1 (the offline restructuring of the FLUTE abstract)
+# --------------------------------------------------------------------------
+#
+# Rows come in strips of 32; groups are 128 codes along K.  The tile of
+# (strip s, group g) starts at byte (s * G + g) * T with T = 2048 (4-bit) or
+# 1536 (3-bit).  A tile is a sequence of 16-byte words; word w of row r (r in
+# 0..31 within the strip) sits at byte (32 * w + r) * 16 of the tile, so one
+# word index over a strip is 512 contiguous bytes.
+#
+# 4-bit: words w = 0..3 cover k = 128g + 32w + (0..31).  Byte i of the word
+#   holds the pair of codes (k0 + 2i, k0 + 2i + 1): even code in the low nibble.
+# 3-bit: a code q is split into lo2 = q & 3 and hi1 = q >> 2.  For a pair of
+#   codes (even e, odd o): lo2(pair) = lo2(e) | lo2(o) << 2 and
+#   hi2(pair) = hi1(e) | hi1(o) << 1.
+#   Words 0 and 1 ("lo planes") cover k0 = 128g + 64w, i.e. 32 pairs
+#   P = 0..31 with pair P = codes (k0 + 2P, k0 + 2P + 1).  Read as four
+#   little-endian u32 L_j (j = 0..3), byte b of L_j holds lo2(pair 8j + b) in
+#   its low nibble and lo2(pair 8j + 4 + b) in its high nibble.
+#   Word 2 ("hi plane") is four u32 H_j; byte b of H_j holds
+#     bits 1:0 = hi2(pair 8j + 4 + b of lo word 0)
+#     bits 3:2 = hi2(pair 8j + 4 + b of lo word 1)
+#     bits 5:4 = hi2(pair 8j + b     of lo word 0)
+#     bits 7:6 = hi2(pair 8j + b     of lo word 1)
+
+def packed_bytes(n: int, k: int, bits: int) -> int:
+    if bits == 4:
+        return n * k // 2
+    if bits == 3:
+        return 3 * n * k // 8
+    raise ValueError("bits must be 3 or 4")
+
+
+def _check_shape(n: int, k: int) -> None:
+    if n % STRIP or k % GROUP:
+        raise ValueError("N must be a multiple of 32 and K of 128")
+
+
+def pack(codes, bits: int) -> np.ndarray:
+    """codes uint8[N, K] -> packed uint8[packed_bytes(N, K, bits)] (layout V1)."""
+    q = np.asarray(codes, dtype=np.uint8)
+    n, k = q.shape
+    _check_shape(n, k)
+    if np.any(q >= (1 << bits)):
+        raise ValueError("code out of range")
+    ns, g = n // STRIP, k // GROUP
+    if bits == 4:
+        # index order of a code: row = 32 s + r, k = 128 g + 32 w + 2 i + e
+        t = q.reshape(ns, STRIP, g, 4, 16, 2)
+        byte = t[..., 0] | (t[..., 1] << 4)                 # [s, r, g, w, i]
+        tiles = byte.transpose(0, 2, 3, 1, 4)               # [s, g, w, r, i]
+        return np.ascontiguousarray(tiles).reshape(-1)
+    if bits == 3:
+        # k = 128 g + 64 w + 16 j + 8 h + 2 b + e  (h: low/high nibble half)
+        t = q.reshape(ns, STRIP, g, 2, 4, 2, 4, 2)
+        even, odd = t[..., 0], t[..., 1]                    # [s, r, g, w, j, h, b]
+        lo2 = (even & 3) | ((odd & 3) << 2)
+        hi2 = (even >> 2) | ((odd >> 2) << 1)
+        lo_byte = lo2[:, :, :, :, :, 0, :] | (lo2[:, :, :, :, :, 1, :] << 4)  # [s,r,g,w,j,b]
+        hi_byte = (hi2[:, :, :, 0, :, 1, :]
+                   | (hi2[:, :, :, 1, :, 1, :] << 2)
+                   | (hi2[:, :, :, 0, :, 0, :] << 4)
+                   | (hi2[:, :, :, 1, :, 0, :] << 6))                          # [s,r,g,j,b]
+        lo_words = lo_byte.reshape(ns, STRIP, g, 2, 16)     # byte 4j + b of word w
+        hi_words = hi_byte.reshape(ns, STRIP, g, 1, 16)
+        words = np.concatenate([lo_words, hi_words], axis=3)  # [s, r, g, 3, 16]
+        tiles = words.transpose(0, 2, 3, 1, 4)              # [s, g, w, r, 16]
+        return np.ascontiguousarray(tiles).reshape(-1).astype(np.uint8)
+    raise ValueError("bits must be 3 or 4")
+
+
+def unpack(packed, n: int, k: int, bits: int) -> np.ndarray:
+    """Inverse of :func:`pack`, written byte by byte from the layout text."""
+    p = np.asarray(packed, dtype=np.uint8)
+    _check_shape(n, k)
+    if p.size != packed_bytes(n, k, bits):
+        raise ValueError("packed size mismatch")
+    g = k // GROUP
+    q = np.zeros((n, k), dtype=np.uint8)
+    tile_bytes = 2048 if bits == 4 else 1536
+    for row in range(n):
+        s, r = divmod(row, STRIP)
+        for gi in range(g):
+            base = (s * g + gi) * tile_bytes
+            if bits == 4:
+                for w in range(4):
+                    word = p[base + (32 * w + r) * 16: base + (32 * w + r) * 16 + 16]
+                    for i in range(16):
+                        kk = GROUP * gi + 32 * w + 2 * i
+                        q[row, kk] = word[i] & 15
+                        q[row, kk + 1] = word[i] >> 4
+            else:
+                lo = [p[base + (32 * w + r) * 16: base + (32 * w + r) * 16 + 16] for w in (0, 1)]
+                hi = p[base + (64 + r) * 16: base + (64 + r) * 16 + 16]
+                for w in (0, 1):
+                    for j in range(4):
+                        for b in range(4):
+                            byte_lo = int(lo[w][4 * j + b])
+                            byte_hi = int(hi[4 * j + b])
+                            for h in (0, 1):
+                                pair = 8 * j + 4 * h + b
+                                l2 = (byte_lo >> (4 * h)) & 15
+                                shift = (2 * w) if h == 1 else (4 + 2 * w)
+                                h2 = (byte_hi >> shift) & 3
+                                kk = GROUP * gi + 64 * w + 2 * pair
+                                q[row, kk] = (l2 & 3) | ((h2 & 1) << 2)
+                                q[row, kk + 1] = ((l2 >> 2) & 3) | (((h2 >> 1) & 1) << 2)
+    return q
+
+
+# --------------------------------------------------------------------------
+# Dequantization and the product
+# --------------------------------------------------------------------------
+
+def dequant(codes, scale_bits, levels_f32) -> np.ndarray:
+    """W_hat[n, k] = s[n, k/128] * c[q[n, k]] in fp64 (exact: 8-bit x 8-bit
+    significands)."""
+    q = np.asarray(codes)
+    s = bf16_bits_to_f32(scale_bits).astype(np.float64)
+    c = np.asarray(levels_f32, dtype=np.float64)
+    n, k = q.shape
+    return (c[q].reshape(n, k // GROUP, GROUP) * s[:, :, None]).reshape(n, k)
+
+
+def gemv(x, codes, scale_bits, levels_f32) -> np.ndarray:
+    """y[m, n] = sum_g s[n, g] * (sum_{k in g} x[m, k] * c[q[n, k]]), fp64.
+
+    The inner sum is the per-group partial sum and the scale is applied once
+    per group (BitMoD abstract: rescale the per-group partial sum).
+    x is float32 (bf16-valued) [M, K]; returns float64 [M, N].
+    """
+    xf = np.asarray(x, dtype=np.float64)
+    q = np.asarray(codes)
+    n, k = q.shape
+    m = xf.shape[0]
+    g = k // GROUP
+    c = np.asarray(levels_f32, dtype=np.float64)
+    s = bf16_bits_to_f32(scale_bits).astype(np.float64)       # [N, G]
+    cq = c[q].reshape(n, g, GROUP).transpose(1, 2, 0)         # [G, 128, N]
+    xg = xf.reshape(m, g, GROUP).transpose(1, 0, 2)           # [G, M, 128]
+    partial = np.matmul(xg, cq)                                # [G, M, N]
+    return np.sum(partial * s.T[:, None, :], axis=0)
+
+
+def gemv_rows(x, w_rows, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Quantize a subset of rows and return (codes, scale bits, y[:, rows]).
+
+    Rows are independent in both quantization and the product, so checking a
+    sample of rows of a large layer needs only those rows."""
+    codes, sb = quantize(w_rows, levels_f32, bits)
+    return codes, sb, gemv(x, codes, sb, levels_f32)
+
+
+def rel_error_gate(y, y_ref, floor_frac: float = 1e-2) -> float:
+    """max |y - y_ref| / max(|y_ref|, floor_frac * rms of y_ref's row), the
+    error measure the 2e-3 tolerance applies to.  The floor keeps outputs
+    that cancel to near zero from dominating a relative measure."""
+    y = np.asarray(y, dtype=np.float64)
+    r = np.asarray(y_ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(np.square(r), axis=-1, keepdims=True))
+    den = np.maximum(np.abs(r), floor_frac * rms)
+    den = np.where(den > 0, den, 1.0)
+    return float(np.max(np.abs(y - r) / den)) if r.size else 0.0
