@@ -1,0 +1,387 @@
+"""Benchmark of the fused LUT-dequant GEMV (and the tensor-core GEMM) on B200.
+
+One step = one product call y = x * dequant(W)^T on one synthetic batch, the
+hot path of inference; quantization and packing are offline (once per layer)
+and run before the timed region.  Default workload: the Llama-3-8B-shaped
+down projection W[4096, 14336], 4-bit NormalFloat, group 128, batch 1.
+
+Timing: W warm-up steps, then exactly K steps between a barrier and
+torch.cuda.synchronize() on both sides, CUDA events on the launching stream,
+max over ranks.  The K launches are replayed from CUDA graphs.  The weights
+rotate over R device copies whose total exceeds 3x the L2 size, so no step
+finds its weights in L2.  `e2e` times the same steps through the public call
+with x copied from pinned host memory and y read back every step.
+
+`--impl reference` times the CPU oracle (test infrastructure) on the same
+workload, on a bounded sample of rows per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100000)
+    p.add_argument("--warmup", type=int, default=2000)
+    p.add_argument("--impl", default="lutq", choices=["lutq", "reference"])
+    p.add_argument("--workload", default="llama3_8b_w4_nf4")
+    p.add_argument("--layer", default="down")
+    p.add_argument("--codebook", default="nf4")
+    p.add_argument("--bits", type=int, default=4)
+    p.add_argument("--batch", type=int, default=1)
+    p.add_argument("--e2e-steps", type=int, default=5000)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def algorithmic_bytes(m, n, k, bits):
+    packed = n * k // 2 if bits == 4 else 3 * n * k // 8
+    return packed + n * (k // 128) * 2 + m * k * 2 + m * n * 4
+
+
+def kernel_source_sha():
+    src = os.path.join(ROOT, "dequant_gemv_group_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("lutq_common.cuh", "lutq_gemv.cu"):
+        h.update(open(os.path.join(src, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(kernel_key)
+    if not d or d.get("source_sha") != kernel_source_sha():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.tmp.flush()
+        rows = [ln.split(",") for ln in open(self.tmp.name).read().splitlines() if ln.strip()]
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(world, value):
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------- oracle arm
+
+def oracle_sample(lay, kind, bits, m, rows):
+    from oracle import lutq_oracle as O
+    w = lay.weights(seed=0)[:rows].float().numpy()
+    _, levels = O.codebook(kind, bits)
+    codes, sb = O.quantize(w, levels, bits)
+    x = workloads.activations(m, lay.k, seed=1).float().numpy()
+    return O, x, codes, sb, levels
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(lay, kind, bits, m, rows, seconds=None, calls=None):
+    O, x, codes, sb, levels = oracle_sample(lay, kind, bits, m, rows)
+    O.gemv(x, codes, sb, levels)
+    n_calls, t0 = 0, time.perf_counter()
+    while True:
+        O.gemv(x, codes, sb, levels)
+        n_calls += 1
+        el = time.perf_counter() - t0
+        if (calls is not None and n_calls >= calls) or (seconds is not None and el >= seconds):
+            break
+    per_call = el / n_calls
+    gbs = algorithmic_bytes(m, rows, lay.k, bits) / per_call / 1e9
+    return gbs, per_call, n_calls
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    lay = workloads.layer(args.workload, args.layer)
+    rows = 256
+    m = args.batch
+    O, x, codes, sb, levels = oracle_sample(lay, args.codebook, args.bits, m, rows)
+    for _ in range(args.warmup):
+        O.gemv(x, codes, sb, levels)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.gemv(x, codes, sb, levels)
+    el = time.perf_counter() - t0
+    gbs = algorithmic_bytes(m, rows, lay.k, args.bits) * args.steps / el / 1e9
+    sample = f"{rows} of {lay.n} rows of the layer per step (oracle-quantized), fp64 numpy"
+    cores = oracle_threads()
+    line = {
+        "impl": "reference", "metric": "dequant-fused GEMV HBM GB/s", "value": gbs,
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args, lay),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(args, lay):
+    return {"workload": f"{args.workload}/{lay.name} W[{lay.n},{lay.k}] {args.codebook} "
+                        f"W{args.bits} group128 batch{args.batch}",
+            "N": lay.n, "K": lay.k, "M": args.batch, "bits": args.bits,
+            "codebook": args.codebook, "group": 128}
+
+
+# ---------------------------------------------------------------------- lutq arm
+
+def capture(fn, count):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(count):
+            fn(i)
+    return g
+
+
+def run_lutq(args, world, rank, local):
+    import dequant_gemv_group_b200 as lq
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lay = workloads.layer(args.workload, args.layer)
+    n, k, m, bits = lay.n, lay.k, args.batch, args.bits
+
+    cb = lq.lutq_codebook(args.codebook, bits).to(dev)
+    w = lay.weights(seed=0).to(dev)
+    st = lq.new_status(dev)
+    codes, scales = lq.lutq_quantize(w, cb, bits, status=st)
+    packed = lq.lutq_pack(codes, bits, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    del w, codes
+
+    per_copy = packed.numel() + scales.numel() * 2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(2, int(np.ceil(3 * l2 / per_copy)) + 1)
+    packs = [packed] + [packed.clone() for _ in range(copies - 1)]
+    scs = [scales] + [scales.clone() for _ in range(copies - 1)]
+    x = workloads.activations(m, k, seed=1).to(dev)
+    y = torch.empty((m, n), dtype=torch.float32, device=dev)
+    ws = lq.new_workspace(m, n, k, bits, dev)
+    use_gemm = m > 16
+    call = lq.lutq_gemm if use_gemm else lq.lutq_gemv
+
+    def step(i):
+        j = i % copies
+        call(x, packs[j], scs[j], cb, bits, n, k, y=y, workspace=ws, status=st)
+
+    for i in range(8):  # eager warm-up (module load, attributes)
+        step(i)
+    torch.cuda.synchronize()
+
+    chunk = min(512, max(1, args.steps))
+    g_chunk = capture(step, chunk)
+    rem = args.steps % chunk
+    g_rem = capture(step, rem) if rem else None
+    w_graph = capture(step, args.warmup) if 0 < args.warmup <= 4096 else None
+
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    sampler.start()
+    if w_graph is not None:
+        w_graph.replay()
+    else:
+        for i in range(args.warmup):
+            step(i)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps // chunk):
+        g_chunk.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(world, ms)
+    assert int(st.item()) == 0
+
+    nbytes = algorithmic_bytes(m, n, k, bits)
+    per_step_s = ms / 1e3 / args.steps
+    gbs_rank = nbytes / per_step_s / 1e9
+    value = gbs_rank * world
+
+    # plain stream launches (no graph), for context
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    plain_steps = min(args.steps, 20000)
+    e0.record(stream)
+    for i in range(plain_steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    plain_gbs = nbytes / (e0.elapsed_time(e1) / 1e3 / plain_steps) / 1e9
+
+    # end to end through the public call with host buffers
+    x_host = workloads.activations(m, k, seed=1).pin_memory()
+    y_host = torch.empty((m, n), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_steps = min(args.steps, args.e2e_steps)
+    for i in range(20):
+        x_dev.copy_(x_host, non_blocking=True)
+        call(x_dev, packs[i % copies], scs[i % copies], cb, bits, n, k, y=y, workspace=ws)
+        y_host.copy_(y, non_blocking=True)
+        torch.cuda.synchronize()
+    barrier(world)
+    t0 = time.perf_counter()
+    for i in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        call(x_dev, packs[i % copies], scs[i % copies], cb, bits, n, k, y=y, workspace=ws)
+        y_host.copy_(y, non_blocking=True)
+        torch.cuda.synchronize()
+    e2e_s = max_over_ranks(world, time.perf_counter() - t0)
+    e2e_gbs = nbytes * e2e_steps / e2e_s / 1e9 * world
+
+    hbm_peak, tf_peak, peak_kind = peaks()
+    kernel_key = f"gemv_w{bits}_m{m}_{n}x{k}"
+    line = {
+        "metric": "dequant-fused GEMV HBM GB/s", "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(args, lay), parallelism=f"replicas{world}",
+                       launch="cuda_graph",
+                       l2=f"weights rotate over {copies} copies "
+                          f"({copies * per_copy / 1e6:.0f} MB > 3x L2 {l2 / 1e6:.0f} MB)"),
+        "roofline": {"bound": "hbm", "achieved": gbs_rank, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": gbs_rank / hbm_peak, "peak_source": peak_kind,
+                     "bytes_per_launch": nbytes, "traffic": ncu_traffic(kernel_key),
+                     "kernel": "lutq::gemv_kernel" if not use_gemm else "lutq::gemm_kernel"},
+        "pct_of_8TBs": gbs_rank / 8000.0,
+        "plain_launch_gbs": plain_gbs,
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": m * k * 2,
+                "d2h_bytes_per_step": m * n * 4, "steps": e2e_steps,
+                "note": "x H2D + product + y D2H + host sync per step"},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world >= 1:
+        rows = 512
+        gbs_cpu, per_call, calls = time_oracle(lay, args.codebook, bits, m, rows, seconds=10.0)
+        line["cpu_baseline"] = {
+            "value": gbs_cpu, "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{rows} of {n} rows (oracle-quantized), {calls} calls of the oracle "
+                      f"product, {per_call * 1e3:.1f} ms each"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_lutq(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,23 @@
+"""Group-wise lookup-table weight quantization and fused dequant GEMV/GEMM for
+NVIDIA B200 (sm_100a).
+
+The work is done by ``liblutq.so`` (CUDA kernels behind a C ABI, declared in
+``include/lutq.h``); this package only marshals torch tensors into it.
+"""
+from ._binding import (  # noqa: F401
+    CODEBOOK_KINDS,
+    LIB_PATH,
+    LutqError,
+    lib,
+    lutq_codebook,
+    lutq_gemm,
+    lutq_gemv,
+    lutq_layout_version,
+    lutq_pack,
+    lutq_packed_bytes,
+    lutq_quantize,
+    lutq_status_string,
+    lutq_workspace_bytes,
+    new_status,
+    new_workspace,
+)

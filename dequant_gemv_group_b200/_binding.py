@@ -1,0 +1,156 @@
+"""ctypes binding of liblutq (argument marshalling only).
+
+Every function here forwards to the C ABI function of the same name declared
+in ``include/lutq.h``; tensors are passed as raw device pointers, the stream is
+torch's current CUDA stream.  There is no fallback: if ``liblutq.so`` is
+missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblutq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m dequant_gemv_group_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_i32, _i64, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
+
+LUTQ_OK = 0
+STATUS_NAMES = {
+    0: "LUTQ_OK", 1: "LUTQ_ERR_INVALID_ARG", 2: "LUTQ_ERR_SHAPE", 3: "LUTQ_ERR_BITS",
+    4: "LUTQ_ERR_ALIGN", 5: "LUTQ_ERR_NONFINITE", 6: "LUTQ_ERR_CODE_RANGE",
+    7: "LUTQ_ERR_TIMEOUT", 8: "LUTQ_ERR_CUDA", 9: "LUTQ_ERR_WORKSPACE",
+}
+CODEBOOK_KINDS = {"nf4": 0, "logb": 1, "lloyd_max3": 2, "uniform4": 3}
+
+_SIGS = {
+    "lutq_status_string": (ctypes.c_char_p, [_i32]),
+    "lutq_layout_version": (_i32, []),
+    "lutq_packed_bytes": (_i64, [_i64, _i64, _i32]),
+    "lutq_codebook": (_i32, [_i32, _i32, _vp]),
+    "lutq_quantize": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "lutq_pack": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "lutq_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32]),
+    "lutq_gemv": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+    "lutq_gemm": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class LutqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lutq_status_string(status)}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != LUTQ_OK:
+        raise LutqError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def lutq_status_string(status: int) -> str:
+    return lib.lutq_status_string(int(status)).decode()
+
+
+def lutq_layout_version() -> int:
+    return lib.lutq_layout_version()
+
+
+def lutq_packed_bytes(n: int, k: int, bits: int) -> int:
+    return lib.lutq_packed_bytes(n, k, bits)
+
+
+def lutq_workspace_bytes(m: int, n: int, k: int, bits: int) -> int:
+    return lib.lutq_workspace_bytes(m, n, k, bits)
+
+
+def lutq_codebook(kind: str, bits: int) -> torch.Tensor:
+    """Host-built codebook as a CPU bf16 tensor of 2^bits ascending levels."""
+    out = torch.zeros(1 << bits, dtype=torch.int16)
+    _check(lib.lutq_codebook(CODEBOOK_KINDS[kind], bits, out.data_ptr()), "lutq_codebook")
+    return out.view(torch.bfloat16)
+
+
+def new_status(device=None) -> torch.Tensor:
+    """A zeroed int32 device status word."""
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def new_workspace(m: int, n: int, k: int, bits: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace of lutq_workspace_bytes(m, n, k, bits) bytes."""
+    nb = lutq_workspace_bytes(m, n, k, bits)
+    if nb < 0:
+        raise LutqError(2, "lutq_workspace_bytes")
+    return torch.zeros(max(nb, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def _need(t: torch.Tensor, dtype, name: str) -> None:
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor of {dtype}")
+
+
+def lutq_quantize(w: torch.Tensor, codebook: torch.Tensor, bits: int,
+                  status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    _need(w, torch.bfloat16, "W")
+    _need(codebook, torch.bfloat16, "codebook")
+    n, k = w.shape
+    codes = torch.empty((n, k), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((n, max(k // 128, 1)), dtype=torch.bfloat16, device=w.device)
+    _check(lib.lutq_quantize(w.data_ptr(), n, k, codebook.data_ptr(), bits, codes.data_ptr(),
+                             scales.data_ptr(), _ptr(status), _stream()), "lutq_quantize")
+    return codes, scales
+
+
+def lutq_pack(codes: torch.Tensor, bits: int,
+              status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(codes, torch.uint8, "codes")
+    n, k = codes.shape
+    nb = lutq_packed_bytes(n, k, bits)
+    if nb < 0:
+        raise LutqError(2, "lutq_packed_bytes")
+    packed = torch.empty(nb, dtype=torch.uint8, device=codes.device)
+    _check(lib.lutq_pack(codes.data_ptr(), n, k, bits, packed.data_ptr(), _ptr(status), _stream()),
+           "lutq_pack")
+    return packed
+
+
+def _product(fn, where, x, packed, scales, codebook, bits, n, k, y, workspace, status):
+    _need(x, torch.bfloat16, "x")
+    m = x.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    _check(fn(x.data_ptr(), m, packed.data_ptr(), scales.data_ptr(), codebook.data_ptr(), bits,
+              n, k, y.data_ptr(), ws_ptr, ws_bytes, _ptr(status), _stream()), where)
+    return y
+
+
+def lutq_gemv(x, packed, scales, codebook, bits, n, k, y=None, workspace=None, status=None):
+    """y[M, N] (fp32) for M = 1..16; see lutq_gemv in include/lutq.h."""
+    return _product(lib.lutq_gemv, "lutq_gemv", x, packed, scales, codebook, bits, n, k, y,
+                    workspace, status)
+
+
+def lutq_gemm(x, packed, scales, codebook, bits, n, k, y=None, workspace=None, status=None):
+    """y[M, N] (fp32) on the tensor cores; see lutq_gemm in include/lutq.h."""
+    return _product(lib.lutq_gemm, "lutq_gemm", x, packed, scales, codebook, bits, n, k, y,
+                    workspace, status)

@@ -1,0 +1,175 @@
+// C ABI of liblutq: argument checks and kernel launches.  Every argument error
+// is returned before anything is launched; device-side conditions go to the
+// caller's dev_status word.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "lutq.h"
+#include "lutq_common.cuh"
+
+namespace lutq {
+cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* codebook, int bits,
+                            uint8_t* codes, void* scales, int32_t* dev_status, int num_sms,
+                            cudaStream_t stream);
+cudaError_t launch_pack(const uint8_t* codes, int64_t N, int64_t K, int bits, void* packed,
+                        int32_t* dev_status, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* scales,
+                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
+                        void* workspace, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* scales,
+                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
+                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
+int64_t gemv_workspace_bytes(int64_t M, int64_t N);
+int64_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+}  // namespace lutq
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_num_sms[kMaxDevices] = {0};
+
+// Multiprocessor count of the current device (cached per device).
+lutq_status current_sms(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LUTQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LUTQ_ERR_CUDA;
+  if (g_num_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return LUTQ_ERR_CUDA;
+    g_num_sms[dev] = n;
+  }
+  *out = g_num_sms[dev];
+  return LUTQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lutq_status check_shape(int64_t N, int64_t K) {
+  if (N < lutq::kStrip || K < lutq::kGroup) return LUTQ_ERR_SHAPE;
+  if (N % lutq::kStrip != 0 || K % lutq::kGroup != 0) return LUTQ_ERR_SHAPE;
+  if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return LUTQ_ERR_SHAPE;
+  return LUTQ_OK;
+}
+
+lutq_status check_bits(int bits) { return (bits == 3 || bits == 4) ? LUTQ_OK : LUTQ_ERR_BITS; }
+
+lutq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LUTQ_OK : LUTQ_ERR_CUDA; }
+
+lutq_status check_product_args(const void* x, int64_t M, int64_t max_m, const void* packed,
+                               const void* scales, const void* codebook, int bits, int64_t N,
+                               int64_t K, const float* y, const void* workspace,
+                               int64_t workspace_bytes, int64_t need) {
+  if (!x || !packed || !scales || !codebook || !y) return LUTQ_ERR_INVALID_ARG;
+  lutq_status st = check_bits(bits);
+  if (st != LUTQ_OK) return st;
+  st = check_shape(N, K);
+  if (st != LUTQ_OK) return st;
+  if (M < 1 || M > max_m) return LUTQ_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(codebook) ||
+      !aligned16(y))
+    return LUTQ_ERR_ALIGN;
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need) return LUTQ_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return LUTQ_ERR_ALIGN;
+  }
+  return LUTQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lutq_status_string(int status) {
+  switch (status) {
+    case LUTQ_OK: return "LUTQ_OK";
+    case LUTQ_ERR_INVALID_ARG: return "LUTQ_ERR_INVALID_ARG: null pointer or invalid value";
+    case LUTQ_ERR_SHAPE: return "LUTQ_ERR_SHAPE: need N % 32 == 0, K % 128 == 0 and M in range";
+    case LUTQ_ERR_BITS: return "LUTQ_ERR_BITS: bits must be 3 or 4 (and match the codebook)";
+    case LUTQ_ERR_ALIGN: return "LUTQ_ERR_ALIGN: pointer not 16-byte aligned";
+    case LUTQ_ERR_NONFINITE: return "LUTQ_ERR_NONFINITE: non-finite weight";
+    case LUTQ_ERR_CODE_RANGE: return "LUTQ_ERR_CODE_RANGE: code >= 2^bits";
+    case LUTQ_ERR_TIMEOUT: return "LUTQ_ERR_TIMEOUT: bounded wait expired inside a kernel";
+    case LUTQ_ERR_CUDA: return "LUTQ_ERR_CUDA: CUDA runtime error";
+    case LUTQ_ERR_WORKSPACE: return "LUTQ_ERR_WORKSPACE: workspace missing or too small";
+    default: return "unknown lutq status";
+  }
+}
+
+int lutq_layout_version(void) { return 1; }
+
+int64_t lutq_packed_bytes(int64_t N, int64_t K, int bits) {
+  if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK) return -1;
+  return bits == 4 ? N * K / 2 : 3 * N * K / 8;
+}
+
+lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K, const void* codebook_bf16,
+                          int bits, uint8_t* codes, void* scales_bf16, int32_t* dev_status,
+                          void* stream) {
+  if (!W_bf16 || !codebook_bf16 || !codes || !scales_bf16) return LUTQ_ERR_INVALID_ARG;
+  lutq_status st = check_bits(bits);
+  if (st != LUTQ_OK) return st;
+  if ((st = check_shape(N, K)) != LUTQ_OK) return st;
+  if (!aligned16(W_bf16) || !aligned16(codebook_bf16) || !aligned16(codes) ||
+      !aligned16(scales_bf16))
+    return LUTQ_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16,
+                                         dev_status, sms, static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_pack(const uint8_t* codes, int64_t N, int64_t K, int bits, void* packed,
+                      int32_t* dev_status, void* stream) {
+  if (!codes || !packed) return LUTQ_ERR_INVALID_ARG;
+  lutq_status st = check_bits(bits);
+  if (st != LUTQ_OK) return st;
+  if ((st = check_shape(N, K)) != LUTQ_OK) return st;
+  if (!aligned16(codes) || !aligned16(packed)) return LUTQ_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_pack(codes, N, K, bits, packed, dev_status, sms,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
+  if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK || M < 1) return -1;
+  if (M <= 16) {
+    const int64_t a = lutq::gemv_workspace_bytes(M, N);
+    const int64_t b = lutq::gemm_workspace_bytes(M, N, K);
+    return a > b ? a : b;
+  }
+  return lutq::gemm_workspace_bytes(M, N, K);
+}
+
+lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed, const void* scales_bf16,
+                      const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
+                      void* workspace, int64_t workspace_bytes, int32_t* dev_status,
+                      void* stream) {
+  (void)dev_status;
+  lutq_status st = check_product_args(x_bf16, M, 16, packed, scales_bf16, codebook_bf16, bits, N,
+                                      K, y, workspace, workspace_bytes,
+                                      lutq_workspace_bytes(M, N, K, bits));
+  if (st != LUTQ_OK) return st;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_gemv(x_bf16, M, packed, scales_bf16, codebook_bf16, bits, N, K, y,
+                                     workspace, sms, static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed, const void* scales_bf16,
+                      const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
+                      void* workspace, int64_t workspace_bytes, int32_t* dev_status,
+                      void* stream) {
+  lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, scales_bf16,
+                                      codebook_bf16, bits, N, K, y, workspace, workspace_bytes,
+                                      lutq_workspace_bytes(M, N, K, bits));
+  if (st != LUTQ_OK) return st;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_gemm(x_bf16, M, packed, scales_bf16, codebook_bf16, bits, N, K, y,
+                                     workspace, dev_status, sms,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

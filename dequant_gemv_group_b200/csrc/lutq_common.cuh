@@ -1,0 +1,34 @@
+// Shared helpers for the liblutq kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "lutq.h"
+
+namespace lutq {
+
+constexpr int kGroup = 128;      // weights per quantization group along K
+constexpr int kStrip = 32;       // rows per packing strip (layout V1)
+constexpr int kWordBytes = 16;   // one packed word = one 16-byte vector load
+
+__host__ __device__ constexpr int tile_bytes(int bits) { return bits == 4 ? 2048 : 1536; }
+__host__ __device__ constexpr int words_per_row(int bits) { return bits == 4 ? 4 : 3; }
+
+// Record a device-side error: the first non-zero code wins.
+__device__ __forceinline__ void report(int32_t* dev_status, int code) {
+  if (dev_status != nullptr) atomicCAS(dev_status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// 16-byte streaming load that is not kept in L1 (each packed byte is used once).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+}  // namespace lutq

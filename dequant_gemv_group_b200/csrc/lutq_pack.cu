@@ -1,0 +1,117 @@
+// Offline restructuring of the codes into layout V1 (the FLUTE abstract,
+// "Daily Papers" listing: repack the quantized matrix offline so that the
+// product kernel needs few bit operations to unpack, including 3-bit widths).
+//
+// One thread writes one 16-byte output word; threads are numbered in output
+// order, so a warp writes 512 contiguous bytes.  Word id -> (tile, w, r):
+// r = id % 32, w = (id / 32) % words_per_row, tile = id / (32 * words_per_row),
+// tile = strip * G + g.  Codes >= 2^bits are reported and masked.
+#include "lutq_common.cuh"
+
+namespace lutq {
+
+__device__ __forceinline__ void load_codes(const uint8_t* p, uint8_t* out, int n) {
+  // n is a multiple of 16 and p is 16-byte aligned
+  for (int i = 0; i < n; i += 16) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) out[i + j] = uint8_t(w[j >> 2] >> (8 * (j & 3)));
+  }
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(256)
+pack_kernel(const uint8_t* __restrict__ codes, int64_t N, int64_t K, uint4* __restrict__ packed,
+            int32_t* dev_status) {
+  constexpr int WPR = words_per_row(BITS);
+  constexpr uint32_t kMask = (1u << BITS) - 1u;
+  const int64_t G = K / kGroup;
+  const int64_t words = (N / kStrip) * G * WPR * kStrip;
+  bool bad = false;
+  for (int64_t id = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; id < words;
+       id += int64_t(gridDim.x) * blockDim.x) {
+    const int r = int(id % kStrip);
+    const int w = int((id / kStrip) % WPR);
+    const int64_t tile = id / (kStrip * WPR);
+    const int64_t strip = tile / G, g = tile % G;
+    const uint8_t* row = codes + (strip * kStrip + r) * K + g * kGroup;
+    uint8_t out[16];
+    if (BITS == 4) {
+      uint8_t q[32];
+      load_codes(row + 32 * w, q, 32);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        bad |= q[i] > kMask;
+        q[i] &= kMask;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) out[i] = uint8_t(q[2 * i] | (q[2 * i + 1] << 4));
+    } else if (w < 2) {
+      // lo plane: 64 codes, 32 pairs; byte 4j+b = lo2(pair 8j+b) | lo2(pair 8j+4+b) << 4
+      uint8_t q[64];
+      load_codes(row + 64 * w, q, 64);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        bad |= q[i] > kMask;
+        q[i] &= kMask;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int p0 = 8 * j + b, p1 = 8 * j + 4 + b;
+          const uint32_t lo0 = (q[2 * p0] & 3u) | ((q[2 * p0 + 1] & 3u) << 2);
+          const uint32_t lo1 = (q[2 * p1] & 3u) | ((q[2 * p1 + 1] & 3u) << 2);
+          out[4 * j + b] = uint8_t(lo0 | (lo1 << 4));
+        }
+      }
+    } else {
+      // hi plane over both lo words: byte 4j+b =
+      //   hi2(w0, 8j+4+b) | hi2(w1, 8j+4+b) << 2 | hi2(w0, 8j+b) << 4 | hi2(w1, 8j+b) << 6
+      uint8_t q[128];
+      load_codes(row, q, 128);
+#pragma unroll
+      for (int i = 0; i < 128; ++i) q[i] &= kMask;  // range is checked by the lo-plane threads
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          uint32_t v = 0;
+          const int pairs[4] = {8 * j + 4 + b, 8 * j + 4 + b, 8 * j + b, 8 * j + b};
+#pragma unroll
+          for (int f = 0; f < 4; ++f) {
+            const int base = 64 * (f & 1) + 2 * pairs[f];
+            const uint32_t h2 = (q[base] >> 2) | ((q[base + 1] >> 2) << 1);
+            v |= h2 << (2 * f);
+          }
+          out[4 * j + b] = uint8_t(v);
+        }
+      }
+    }
+    uint4 o;
+    o.x = out[0] | (out[1] << 8) | (out[2] << 16) | (uint32_t(out[3]) << 24);
+    o.y = out[4] | (out[5] << 8) | (out[6] << 16) | (uint32_t(out[7]) << 24);
+    o.z = out[8] | (out[9] << 8) | (out[10] << 16) | (uint32_t(out[11]) << 24);
+    o.w = out[12] | (out[13] << 8) | (out[14] << 16) | (uint32_t(out[15]) << 24);
+    packed[id] = o;
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) report(dev_status, LUTQ_ERR_CODE_RANGE);
+}
+
+cudaError_t launch_pack(const uint8_t* codes, int64_t N, int64_t K, int bits, void* packed,
+                        int32_t* dev_status, int num_sms, cudaStream_t stream) {
+  const int64_t words = (N / kStrip) * (K / kGroup) * words_per_row(bits) * kStrip;
+  int64_t blocks = (words + 255) / 256;
+  const int64_t cap = int64_t(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (bits == 4)
+    pack_kernel<4><<<unsigned(blocks), 256, 0, stream>>>(codes, N, K, static_cast<uint4*>(packed),
+                                                        dev_status);
+  else
+    pack_kernel<3><<<unsigned(blocks), 256, 0, stream>>>(codes, N, K, static_cast<uint4*>(packed),
+                                                        dev_status);
+  return cudaGetLastError();
+}
+
+}  // namespace lutq

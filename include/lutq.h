@@ -1,0 +1,202 @@
+/*
+ * lutq.h - C ABI of liblutq: group-wise lookup-table (LUT) weight-only
+ * quantization and the fused dequantize-and-multiply product, for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operations follow the FLUTE abstract ("Daily Papers" listing, query
+ * "group-128"): weights are quantized offline onto a small non-uniform table of
+ * levels with one scale per group of 128 weights, the quantized matrix is
+ * restructured offline so that unpacking needs few bit operations, and a fused
+ * kernel dequantizes on the fly inside the matrix-vector product.
+ *
+ * Notation: W[N,K] bf16 weights (row n = output feature, K = reduction),
+ * G = K/128 groups per row, codebook c[0 .. 2^bits - 1] (bf16), codes
+ * q[N,K] (uint8), scales s[N,G] (bf16), x[M,K] bf16 activations, y[M,N] fp32.
+ * The dequantized weight is s[n, k/128] * c[q[n,k]].
+ *
+ * Conventions shared by every call:
+ *  - All matrices are dense and row-major.  Device pointers must point to
+ *    memory of the device that is current on the calling thread, and must be
+ *    16-byte aligned (LUTQ_ERR_ALIGN otherwise).
+ *  - The caller owns every buffer; the library allocates nothing per call and
+ *    keeps no state except a per-device cache of attributes.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL means the legacy default stream).  Argument errors are reported by
+ *    the return value before anything is launched.  Conditions found on the
+ *    device are written to `*dev_status` (an int32 in device memory, may be
+ *    NULL): the kernel stores the lutq_status code there if it was 0, so the
+ *    first error wins; the caller reads it after synchronizing.
+ *  - Inputs are never modified.
+ *  - Shape rules: N % 32 == 0, K % 128 == 0, N >= 32, K >= 128; bits is 3 or 4.
+ */
+#ifndef LUTQ_H_
+#define LUTQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LUTQ_OK = 0,
+  LUTQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, unknown enum value */
+  LUTQ_ERR_SHAPE = 2,       /* N % 32, K % 128 or M out of the supported range */
+  LUTQ_ERR_BITS = 3,        /* bits is not 3 or 4 / does not match the codebook */
+  LUTQ_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
+  LUTQ_ERR_NONFINITE = 5,   /* device: quantize met a NaN or infinite weight */
+  LUTQ_ERR_CODE_RANGE = 6,  /* device: pack met a code >= 2^bits */
+  LUTQ_ERR_TIMEOUT = 7,     /* device: a bounded wait inside a kernel expired */
+  LUTQ_ERR_CUDA = 8,        /* a CUDA runtime call failed */
+  LUTQ_ERR_WORKSPACE = 9    /* workspace missing or smaller than required */
+} lutq_status;
+
+/* Codebook kinds for lutq_codebook. */
+typedef enum {
+  LUTQ_CODEBOOK_NF4 = 0,        /* 16-level NormalFloat (4 bit) */
+  LUTQ_CODEBOOK_LOGB = 1,       /* 16-level logarithmic, base 1.6 (4 bit) */
+  LUTQ_CODEBOOK_LLOYD_MAX3 = 2, /* 8-level Lloyd-Max for N(0,1) (3 bit) */
+  LUTQ_CODEBOOK_UNIFORM4 = 3    /* 16 evenly spaced levels (4 bit) */
+} lutq_codebook_kind;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* lutq_status_string(int status);
+
+/* Version of the packed layout produced by lutq_pack and read by lutq_gemv /
+ * lutq_gemm.  Returns 1 for layout V1 (strips of 32 rows, 16-byte words
+ * interleaved across the rows of a strip; see lutq_pack). */
+int lutq_layout_version(void);
+
+/* Size in bytes of the packed codes of an N x K matrix: N*K/2 for 4 bits,
+ * 3*N*K/8 for 3 bits.  Returns -1 for an invalid shape or bit width. */
+int64_t lutq_packed_bytes(int64_t N, int64_t K, int bits);
+
+/*
+ * lutq_codebook - build a codebook on the HOST.
+ *
+ * Source: the FLUTE abstract (NormalFloat lookup table, 3-bit widths), the
+ * Log_bQuant abstract (catalyzex author page: levels spaced in logarithmic
+ * space with an adjustable base) and "TurboQuant: A first-principles
+ * walkthrough" (the Lloyd-Max algorithm).  Levels are computed in double
+ * precision, normalised to max |level| = 1, and rounded once to bf16 (round
+ * to nearest even), in ascending order:
+ *   NF4: 8 positive and 7 negative standard-normal quantiles plus 0, with the
+ *        outermost probability ((1-1/30)+(1-1/32))/2;
+ *   LOGB: +-1.6^-k, k = 0..7;
+ *   LLOYD_MAX3: the 8-level Lloyd-Max quantizer of N(0,1);
+ *   UNIFORM4: (2i-15)/15.
+ * out_bf16: host array of (1 << bits) uint16 bf16 bit patterns, written by the
+ * call.  Returns LUTQ_ERR_BITS if `bits` does not fit the kind.  No GPU use.
+ */
+lutq_status lutq_codebook(int kind, int bits, uint16_t* out_bf16);
+
+/*
+ * lutq_quantize - group-128 round-to-nearest quantization onto a codebook.
+ *
+ * Source: the group-128 post-training-quantization study and the FLUTE
+ * abstract (both "Daily Papers", query "group-128"): RTN weight-only
+ * quantization with one scale per group of 128 consecutive weights along K.
+ * For each row n and group g:
+ *   s[n,g] = max_{k in g} |W[n,k]|            (exact in bf16)
+ *   v      = float(W[n,k]) / float(s[n,g])     (IEEE fp32 divide; 0 if s == 0)
+ *   q[n,k] = lowest i minimising the fp32 value |v - c_i|.
+ * Subnormal weights are kept (no flush to zero); -0 behaves like +0.
+ *
+ * W_bf16   device, bf16 [N,K] row-major.
+ * codebook device, bf16 [1 << bits], ascending is not required.
+ * codes    device, uint8 [N,K] row-major, written.
+ * scales   device, bf16 [N,K/128] row-major, written.
+ * dev_status device int32 or NULL: LUTQ_ERR_NONFINITE if any weight is NaN or
+ *          infinite (codes and scales of that group are then unspecified).
+ */
+lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K,
+                          const void* codebook_bf16, int bits,
+                          uint8_t* codes, void* scales_bf16,
+                          int32_t* dev_status, void* stream);
+
+/*
+ * lutq_pack - offline restructuring of the codes into layout V1.
+ *
+ * Source: the FLUTE abstract ("offline restructuring of the quantized weight
+ * matrix to minimize bit manipulations associated with unpacking"; 3-bit,
+ * non-evenly-divisible widths).
+ *
+ * Layout V1.  Rows form strips of 32; G = K/128.  The tile of (strip s,
+ * group g) starts at byte (s*G + g)*T, T = 2048 (4 bit) or 1536 (3 bit).  A
+ * tile is made of 16-byte words; word w of row r (0..31 within the strip) is at
+ * byte (32*w + r)*16 of the tile, so one word index over a strip is 512
+ * contiguous bytes (one coalesced 16-byte load per lane of a warp).
+ *  4 bit: words 0..3 hold k = 128g + 32w + 0..31; byte i holds the codes
+ *         (k0+2i, k0+2i+1), the even one in the low nibble, so every byte is
+ *         directly an index into a 256-entry table of code pairs.
+ *  3 bit: a code splits into lo2 = q & 3 and hi1 = q >> 2; for a pair (even
+ *         e, odd o) lo2(pair) = lo2(e) | lo2(o) << 2, hi2(pair) = hi1(e) |
+ *         hi1(o) << 1.  Words 0 and 1 hold k0 = 128g + 64w, pairs P = 0..31;
+ *         as four little-endian u32 L_j, byte b has lo2(pair 8j+b) in the low
+ *         nibble and lo2(pair 8j+4+b) in the high nibble.  Word 2 is four u32
+ *         H_j; byte b holds hi2 of pair 8j+4+b of word 0 (bits 1:0) and of
+ *         word 1 (bits 3:2), and hi2 of pair 8j+b of word 0 (bits 5:4) and of
+ *         word 1 (bits 7:6).  One AND-OR of L_j with H_j (or H_j >> 2) then
+ *         yields four pair indices at once.
+ *
+ * codes  device, uint8 [N,K] (values < 2^bits).
+ * packed device, lutq_packed_bytes(N,K,bits) bytes, written.
+ * dev_status device int32 or NULL: LUTQ_ERR_CODE_RANGE if a code >= 2^bits.
+ */
+lutq_status lutq_pack(const uint8_t* codes, int64_t N, int64_t K, int bits,
+                      void* packed, int32_t* dev_status, void* stream);
+
+/*
+ * lutq_workspace_bytes - device scratch size needed by lutq_gemv / lutq_gemm
+ * for this problem (split-K partial sums and per-strip arrival counters).
+ * Returns -1 for an invalid argument.  The value does not depend on the device.
+ */
+int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
+
+/*
+ * lutq_gemv - fused dequantize-and-multiply for small batches, M = 1..16.
+ *
+ * Source: the FLUTE abstract (a kernel that fuses dequantization with the
+ * matmul; the bottleneck is moving weights from global memory; the lookup
+ * table is vectorized and duplicated to ease shared-memory bandwidth) and the
+ * BitMoD abstract (the per-group partial sum is rescaled once per group):
+ *   y[m,n] = sum_g s[n,g] * ( sum_{k in g} x[m,k] * c[q[n,k]] )
+ * Products are bf16 x bf16 (exact in fp32); sums are fp32.  The result is
+ * within 2e-3 (relative, floored at 1e-2 of the row's rms) of the exact sum.
+ *
+ * x        device bf16 [M,K] row-major.
+ * packed   device, layout V1 (lutq_pack).
+ * scales   device bf16 [N,K/128] row-major.
+ * codebook device bf16 [1 << bits].
+ * y        device fp32 [M,N] row-major, written (no accumulation into y).
+ * workspace device, at least lutq_workspace_bytes(M,N,K,bits) bytes, zero-
+ *          filled before its first use (e.g. cudaMemset); every call leaves
+ *          it zero-filled again.  Calls that may run at the same time on the
+ *          GPU must not share a workspace.  May be NULL only if the required
+ *          size is 0.
+ * Returns LUTQ_ERR_SHAPE if M is outside 1..16.
+ */
+lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
+                      const void* scales_bf16, const void* codebook_bf16,
+                      int bits, int64_t N, int64_t K, float* y,
+                      void* workspace, int64_t workspace_bytes,
+                      int32_t* dev_status, void* stream);
+
+/*
+ * lutq_gemm - the same product on the tensor cores (tcgen05), for batches
+ * where the problem is a dense contraction (tuned for M >= 32; any M >= 1 is
+ * accepted).  Arguments and numerics as lutq_gemv.  dev_status receives
+ * LUTQ_ERR_TIMEOUT if a pipeline wait inside the kernel exceeds its bound.
+ */
+lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
+                      const void* scales_bf16, const void* codebook_bf16,
+                      int bits, int64_t N, int64_t K, float* y,
+                      void* workspace, int64_t workspace_bytes,
+                      int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LUTQ_H_ */

@@ -1,0 +1,114 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/lutq.h declares, its host-only functions behave, and argument errors
+come back before anything touches the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import lutq_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"\b(lutq_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lq():
+    import dequant_gemv_group_b200 as m
+    return m
+
+
+def test_library_exports_every_declared_function(lq):
+    declared = _header_functions()
+    assert {"lutq_quantize", "lutq_pack", "lutq_gemv", "lutq_gemm"} <= declared
+    for name in sorted(declared):
+        assert hasattr(lq.lib, name), name
+
+
+def test_layout_version_and_sizes(lq):
+    assert lq.lutq_layout_version() == O.LAYOUT_VERSION == 1
+    for n, k, bits in [(4096, 14336, 4), (4096, 4096, 3), (32, 128, 4), (28672, 8192, 3)]:
+        assert lq.lutq_packed_bytes(n, k, bits) == O.packed_bytes(n, k, bits)
+    assert lq.lutq_packed_bytes(33, 128, 4) == -1
+    assert lq.lutq_packed_bytes(32, 100, 4) == -1
+    assert lq.lutq_packed_bytes(32, 128, 5) == -1
+    assert lq.lutq_workspace_bytes(1, 4096, 14336, 4) > 0
+    assert lq.lutq_workspace_bytes(0, 4096, 14336, 4) == -1
+
+
+def test_status_strings(lq):
+    for code in range(10):
+        assert lq.lutq_status_string(code).startswith(lq._binding.STATUS_NAMES[code])
+    assert "unknown" in lq.lutq_status_string(99)
+
+
+@pytest.mark.parametrize("kind,bits", [("nf4", 4), ("logb", 4), ("lloyd_max3", 3),
+                                       ("uniform4", 4)])
+def test_host_codebook_bit_exact_vs_oracle(lq, kind, bits):
+    import torch
+    ours = lq.lutq_codebook(kind, bits).view(torch.int16).numpy().view(np.uint16)
+    ref, _ = O.codebook(kind, bits)
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_codebook_bits_mismatch(lq):
+    with pytest.raises(lq.LutqError) as e:
+        lq.lutq_codebook("nf4", 3)
+    assert e.value.status == 3
+
+
+# Argument errors are decided on the host before any CUDA call, so fake (never
+# dereferenced) 16-byte-aligned addresses are enough here.
+A = 1 << 20
+
+
+def test_quantize_argument_errors(lq):
+    f = lq.lib.lutq_quantize
+    assert f(None, 32, 128, A, 4, A, A, None, None) == 1          # null W
+    assert f(A, 32, 128, A, 5, A, A, None, None) == 3             # bits
+    assert f(A, 33, 128, A, 4, A, A, None, None) == 2             # N % 32
+    assert f(A, 32, 130, A, 4, A, A, None, None) == 2             # K % 128
+    assert f(A, 0, 128, A, 4, A, A, None, None) == 2              # empty
+    assert f(A + 2, 32, 128, A, 4, A, A, None, None) == 4         # misaligned
+
+
+def test_pack_argument_errors(lq):
+    f = lq.lib.lutq_pack
+    assert f(None, 32, 128, 4, A, None, None) == 1
+    assert f(A, 32, 128, 2, A, None, None) == 3
+    assert f(A, 64, 64, 4, A, None, None) == 2
+    assert f(A, 32, 128, 4, A + 8, None, None) == 4
+
+
+@pytest.mark.parametrize("name", ["lutq_gemv", "lutq_gemm"])
+def test_product_argument_errors(lq, name):
+    f = getattr(lq.lib, name)
+    ws = lq.lutq_workspace_bytes(1, 64, 256, 4)
+    ok = dict(x=A, m=1, p=A, s=A, c=A, bits=4, n=64, k=256, y=A, ws=A, wsb=ws)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["x"], a["m"], a["p"], a["s"], a["c"], a["bits"], a["n"], a["k"], a["y"],
+                 a["ws"], a["wsb"], None, None)
+
+    assert call(x=None) == 1
+    assert call(bits=2) == 3
+    assert call(n=48) == 2
+    assert call(k=200) == 2
+    assert call(m=0) == 2
+    if name == "lutq_gemv":
+        assert call(m=17) == 2
+    assert call(y=A + 4) == 4
+    if ws > 0:
+        assert call(ws=None) == 9
+        assert call(wsb=ws - 1) == 9
