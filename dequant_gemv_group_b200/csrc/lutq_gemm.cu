@@ -1,14 +1,492 @@
-// Tensor-core (tcgen05) dequantize-and-multiply for batches that form a dense
-// contraction.  Not built yet: the entry point reports a CUDA error.
+// Dequantize-and-multiply on the 5th-generation tensor cores (tcgen05) for
+// batches where the product is a dense contraction (the FLUTE abstract,
+// "Daily Papers" listing, query "group-128": a kernel that fuses
+// dequantization with the matmul; the BitMoD abstract, same listing: the
+// per-group partial sum is rescaled once).
+//
+// Roles of the 10 warps of a CTA (one CTA per SM, persistent):
+//   warps 0-3  dequantize: lane r of warp w owns row 32 w + r of the 128-row
+//              tile; it decodes the row's 128 codes of one group through the
+//              lane-duplicated pair table into 64 bf16 pairs and stores them
+//              into tensor memory (lane = row, column j = codes 2j, 2j+1) as
+//              the A operand of the MMA (W is the M side: swap-AB).
+//   warps 4-7  promote: read the group's fp32 partial D[row, batch] from
+//              tensor memory, add s[row, g] * partial to registers, and write
+//              y (or a split partial) when the row tile's range ends.
+//   warp 8     loads: the tile's packed words (four contiguous 1-D bulk
+//              copies, one per 32-row strip) and the activations' 128-wide K
+//              slice (two 2-D tensor-map copies, 128-byte swizzle).
+//   warp 9     issues tcgen05.mma kind::f16 (A from tensor memory, B from
+//              shared memory, D fp32 in tensor memory), 8 MMAs of K = 16 per
+//              group into a fresh partial, and commits to the mbarriers.
+// Products are exact (bf16 x bf16) and every group's partial is rescaled in
+// fp32, so the result matches the fp32-accumulating GEMV up to summation order.
+//
+// Work split: units (batch tile, row tile, group) in that order; CTA c takes
+// units [floor(c U / C), floor((c+1) U / C)).  Row tiles split between CTAs are
+// finished per 32-row strip by the last contributor (warp-ordered sums), as
+// in the GEMV.  Every mbarrier wait is bounded; on expiry the kernel records
+// LUTQ_ERR_TIMEOUT, drains its own copies and MMAs, frees tensor memory and
+// returns.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstring>
+
 #include "lutq_common.cuh"
+#include "lutq_lut.cuh"
+#include "lutq_sm100.cuh"
 
 namespace lutq {
 
-int64_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+using namespace sm100;
 
-cudaError_t launch_gemm(const void*, int64_t, const void*, const void*, const void*, int, int64_t,
-                        int64_t, float*, void*, int32_t*, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kTileRows = 128;
+constexpr int kGemmMaxCtas = 256;            // bounds the workspace
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kTmemCols = 512;
+constexpr int kDCol = 128;                   // partial buffers start here; A uses 0..127
+
+template <int NT>
+struct GemmCfg {
+  static constexpr int XS = NT >= 128 ? 3 : 4;     // activation stages
+  static constexpr int PS = 6;                      // packed-tile stages
+  static constexpr int XSTAGE = 2 * NT * 128;       // two boxes of NT rows x 128 bytes
+  static constexpr int PG = NT >= 128 ? 2 : 1;      // promotion warp groups
+  static constexpr int NC = NT / PG;                // batch columns per promotion warp
+  static constexpr int WARPS = 4 + 4 * PG + 2;      // dequant, promote, load, MMA
+  static constexpr int THREADS = 32 * WARPS;
+};
+constexpr int kMaxPromoteGroups = 2;
+
+struct GemmArgs {
+  const uint8_t* packed;
+  const uint16_t* scales;
+  const uint16_t* codebook;
+  float* y;
+  float* part;        // [kGemmMaxCtas][2][4][NT][32]: (CTA, slot, strip, column, row)
+  int* counters;      // [BT * NTILES * 4 * kMaxPromoteGroups]
+  int32_t* dev_status;
+  int64_t N, G, M;
+  int64_t ntiles;     // row tiles, ceil(N / 128)
+  int64_t U;          // units
+  int C;              // CTAs
+};
+
+__device__ __forceinline__ int64_t g_unit_begin(int64_t c, int64_t U, int64_t C) { return (c * U) / C; }
+__device__ __forceinline__ int64_t g_unit_owner(int64_t u, int64_t U, int64_t C) {
+  return ((u + 1) * C - 1) / U;
+}
+
+// Bounded wait used after an abort: only the time limit ends it.
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+// Loads chunk_cols<NC>() consecutive columns (32, or 16 when a promotion warp
+// owns only 16 columns).
+template <int NC>
+__host__ __device__ constexpr int chunk_cols() { return NC >= 32 ? 32 : 16; }
+
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[32]) {
+  if (chunk_cols<NC>() == 32) {
+    tmem_ld_32x32b_x32(taddr, v);
+  } else {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+  }
+}
+
+// Write one finished 32-row strip of a row tile for batch tile bt; this warp
+// holds batch columns [c0, c0 + NC).
+template <int NT, int NC>
+__device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t seg, int64_t bt,
+                                  int64_t row, int sw, int pg, int64_t u0, int lane) {
+  const int c0 = pg * NC;
+  const int64_t seg_begin = seg * a.G, seg_end = seg_begin + a.G;
+  const int64_t mrem = a.M - bt * kTileRows;
+  const int mt = int(mrem < kTileRows ? mrem : kTileRows);
+  const int64_t c_lo = g_unit_owner(seg_begin, a.U, a.C), c_hi = g_unit_owner(seg_end - 1, a.U, a.C);
+  float* ycol = a.y + (bt * kTileRows + c0) * a.N + row;
+  if (c_lo == c_hi) {
+#pragma unroll
+    for (int j = 0; j < NC; ++j)
+      if (c0 + j < mt) ycol[int64_t(j) * a.N] = acc[j];
+    return;
+  }
+  const int64_t cta = blockIdx.x;
+  const int slot = (seg == u0 / a.G) ? 0 : 1;
+  float* mine = a.part + (((cta * 2 + slot) * 4 + sw) * NT + c0) * 32;
+#pragma unroll
+  for (int j = 0; j < NC; ++j) mine[j * 32 + lane] = acc[j];
+  __threadfence();
+  __syncwarp();
+  int arrived = 0;
+  int* counter = a.counters + (seg * 4 + sw) * kMaxPromoteGroups + pg;
+  if (lane == 0) arrived = atomicAdd(counter, 1);
+  arrived = __shfl_sync(0xffffffffu, arrived, 0);
+  if (arrived != int(c_hi - c_lo)) return;
+  __threadfence();
+#pragma unroll
+  for (int j = 0; j < NC; ++j) acc[j] = 0.0f;
+  for (int64_t c = c_lo; c <= c_hi; ++c) {
+    const int sl = (seg == g_unit_begin(c, a.U, a.C) / a.G) ? 0 : 1;
+    const float* src = a.part + (((c * 2 + sl) * 4 + sw) * NT + c0) * 32;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) acc[j] += __ldcg(src + j * 32 + lane);
+  }
+#pragma unroll
+  for (int j = 0; j < NC; ++j)
+    if (c0 + j < mt) ycol[int64_t(j) * a.N] = acc[j];
+  if (lane == 0) *counter = 0;
+}
+
+template <int BITS, int NT>
+__global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, GemmArgs a) {
+  using Cfg = GemmCfg<NT>;
+  constexpr int PG = Cfg::PG, NC = Cfg::NC;
+  constexpr int W_LOAD = 4 + 4 * PG, W_MMA = W_LOAD + 1;
+  constexpr int TB = tile_bytes(BITS);
+  constexpr int WPR = words_per_row(BITS);
+  constexpr int XS = Cfg::XS, PS = Cfg::PS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_sa = smem_addr(smem_raw);
+  const uint32_t base_sa = (raw_sa + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_sa - raw_sa);
+  uint8_t* lut = base;
+  const uint32_t lut_sa = base_sa;
+  const uint32_t xst_sa = base_sa + kLutBytes;
+  const uint32_t pst_sa = xst_sa + XS * Cfg::XSTAGE;
+  const uint32_t bar_sa = pst_sa + PS * 4 * TB;
+  // barrier ids
+  constexpr int B_XF = 0, B_XE = XS, B_PF = 2 * XS, B_PE = 2 * XS + PS, B_AF = 2 * XS + 2 * PS,
+                B_AE = B_AF + 2, B_DF = B_AE + 2, B_DE = B_DF + 2, NBAR = B_DE + 2;
+  auto bar = [&](int i) { return bar_sa + 8u * uint32_t(i); };
+  uint8_t* misc = base + (bar_sa - base_sa) + 8 * NBAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  uint16_t* cbs = reinterpret_cast<uint16_t*>(misc + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < XS; ++i) {
+      mbar_init(bar(B_XF + i), 1);
+      mbar_init(bar(B_XE + i), 1);
+    }
+    for (int i = 0; i < PS; ++i) {
+      mbar_init(bar(B_PF + i), 1);
+      mbar_init(bar(B_PE + i), 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_AF + i), 4);
+      mbar_init(bar(B_AE + i), 1);
+      mbar_init(bar(B_DF + i), 1);
+      mbar_init(bar(B_DE + i), 4 * PG);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
+  if (warp == W_MMA) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < kLutBytes / 16; c += blockDim.x) {
+    const uint32_t v = lut_entry<BITS>(cbs, c >> 4, (c >> 3) & 1);
+    reinterpret_cast<uint4*>(lut)[c] = make_uint4(v, v, v, v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int64_t u0 = g_unit_begin(blockIdx.x, a.U, a.C);
+  const int n = int(g_unit_begin(blockIdx.x + 1, a.U, a.C) - u0);
+  const int64_t per_bt = a.ntiles * a.G;
+
+  if (warp < 4) {
+    // ---------------------------------------------------------------- dequantize
+    const int sw = warp;
+    const uint32_t off_e = uint32_t(lane) * 4u, off_o = 128u + uint32_t(lane) * 4u;
+    for (int i = 0; i < n; ++i) {
+      const int64_t u = u0 + i;
+      const int64_t tau = (u % per_bt) / a.G;
+      const bool valid = tau * kTileRows + sw * 32 < a.N;
+      const int ps = i % PS;
+      bool ok = mbar_wait(bar(B_PF + ps), uint32_t(i / PS) & 1u, abort_flag, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      uint4 wd[4];
+      if (valid) {
+#pragma unroll
+        for (int j = 0; j < WPR; ++j)
+          wd[j] = lds128(pst_sa + uint32_t(ps * 4 * TB + sw * TB + (32 * j + lane) * 16));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_PE + ps));
+      uint32_t av[64];
+      if (valid) decode_group_row<BITS>(av, wd, lut_sa, off_e, off_o);
+      const int ab = i & 1;
+      ok = mbar_wait(bar(B_AE + ab), (uint32_t(i >> 1) & 1u) ^ 1u, abort_flag, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      if (valid) {
+        tmem_st_32x32b_x64(tmem + (uint32_t(sw * 32) << 16) + uint32_t(ab * 64), av);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_AF + ab));
+    }
+  } else if (warp < W_LOAD) {
+    // ---------------------------------------------------------------- promote
+    const int sw = warp & 3, pg = (warp - 4) >> 2;
+    float acc[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) acc[j] = 0.0f;
+    for (int i = 0; i < n; ++i) {
+      const int64_t u = u0 + i;
+      const int64_t bt = u / per_bt;
+      const int64_t rem = u - bt * per_bt;
+      const int64_t tau = rem / a.G, g = rem - tau * a.G;
+      const int64_t row = tau * kTileRows + sw * 32 + lane;
+      const bool valid = tau * kTileRows + sw * 32 < a.N;
+      const float s =
+          valid ? __uint_as_float(uint32_t(__ldg(a.scales + row * a.G + g)) << 16) : 0.0f;
+      const int db = i & 1;
+      const bool ok = mbar_wait(bar(B_DF + db), uint32_t(i >> 1) & 1u, abort_flag, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      constexpr int CH = chunk_cols<NC>();
+#pragma unroll
+      for (int c = 0; c < NC / CH; ++c) {
+        uint32_t v[32];
+        tmem_ld_cols<NC>(tmem + (uint32_t(sw * 32) << 16) +
+                             uint32_t(kDCol + db * NT + pg * NC + c * CH),
+                         v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < CH; ++j) acc[c * CH + j] = fmaf(s, __uint_as_float(v[j]), acc[c * CH + j]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_DE + db));
+      if (g == a.G - 1 || i == n - 1) {
+        if (valid) gemm_finish_strip<NT, NC>(a, acc, bt * a.ntiles + tau, bt, row, sw, pg, u0, lane);
+#pragma unroll
+        for (int j = 0; j < NC; ++j) acc[j] = 0.0f;
+      }
+    }
+  } else if (warp == W_LOAD) {
+    // ---------------------------------------------------------------- loads
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int64_t u = u0 + i;
+        const int64_t bt = u / per_bt;
+        const int64_t rem = u - bt * per_bt;
+        const int64_t tau = rem / a.G, g = rem - tau * a.G;
+        const int ps = i % PS;
+        if (!mbar_wait(bar(B_PE + ps), (uint32_t(i / PS) & 1u) ^ 1u, abort_flag, kWaitLimitNs))
+          break;
+        const int64_t srem = (a.N - tau * kTileRows) / 32;
+        const int vs = int(srem < 4 ? srem : 4);
+        mbar_expect_tx(bar(B_PF + ps), uint32_t(vs * TB));
+        for (int s = 0; s < vs; ++s)
+          bulk_g2s(pst_sa + uint32_t(ps * 4 * TB + s * TB),
+                   a.packed + ((tau * 4 + s) * a.G + g) * TB, TB, bar(B_PF + ps));
+        const int xs = i % XS;
+        if (!mbar_wait(bar(B_XE + xs), (uint32_t(i / XS) & 1u) ^ 1u, abort_flag, kWaitLimitNs)) {
+          issued = -(i + 1);  // packed stage i issued, activations not
+          break;
+        }
+        mbar_expect_tx(bar(B_XF + xs), uint32_t(Cfg::XSTAGE));
+        const uint32_t xd = xst_sa + uint32_t(xs * Cfg::XSTAGE);
+        tma_2d_g2s(xd, &tmap_x, int32_t(g * 128), int32_t(bt * kTileRows), bar(B_XF + xs));
+        tma_2d_g2s(xd + NT * 128, &tmap_x, int32_t(g * 128 + 64), int32_t(bt * kTileRows),
+                   bar(B_XF + xs));
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        // let the copies in flight land before the CTA can exit
+        const int np = issued >= 0 ? issued : -issued;
+        const int nx = issued >= 0 ? issued : -issued - 1;
+        for (int i = (np > PS ? np - PS : 0); i < np; ++i) mbar_drain(bar(B_PF + i % PS), uint32_t(i / PS) & 1u);
+        for (int i = (nx > XS ? nx - XS : 0); i < nx; ++i) mbar_drain(bar(B_XF + i % XS), uint32_t(i / XS) & 1u);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, NT);
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int xs = i % XS, ab = i & 1, db = i & 1;
+        if (!mbar_wait(bar(B_XF + xs), uint32_t(i / XS) & 1u, abort_flag, kWaitLimitNs)) break;
+        if (!mbar_wait(bar(B_AF + ab), uint32_t(i >> 1) & 1u, abort_flag, kWaitLimitNs)) break;
+        if (!mbar_wait(bar(B_DE + db), (uint32_t(i >> 1) & 1u) ^ 1u, abort_flag, kWaitLimitNs))
+          break;
+        tc_fence_after();
+        const uint32_t xb = xst_sa + uint32_t(xs * Cfg::XSTAGE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t b_sa = xb + uint32_t((kk >> 2) * (NT * 128) + (kk & 3) * 32);
+          mma_bf16_ts(tmem + uint32_t(kDCol + db * NT), tmem + uint32_t(ab * 64 + 8 * kk),
+                      smem_desc_k_sw128(b_sa), idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(B_DF + db));
+        mma_commit(bar(B_AE + ab));
+        mma_commit(bar(B_XE + xs));
+        issued = i + 1;
+      }
+      if (*abort_flag && issued > 0) {
+        const int i = issued - 1;
+        mbar_drain(bar(B_DF + (i & 1)), uint32_t(i >> 1) & 1u);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == W_MMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report(a.dev_status, LUTQ_ERR_TIMEOUT);
+}
+
+// --------------------------------------------------------------------------
+// host side
+// --------------------------------------------------------------------------
+
+static int gemm_nt(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  return 128;
+}
+
+int64_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)K;
+  const int nt = gemm_nt(M);
+  const int64_t bt = (M + kTileRows - 1) / kTileRows;
+  const int64_t ntiles = (N + kTileRows - 1) / kTileRows;
+  const int64_t counters = (bt * ntiles * 4 * kMaxPromoteGroups * 4 + 255) / 256 * 256;
+  return counters + int64_t(kGemmMaxCtas) * 2 * 4 * nt * 32 * 4;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// x[M, K] bf16 row-major; boxes of 64 (K) x nt (rows), 128-byte swizzle,
+// rows past M read as zero.
+static cudaError_t make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K, int nt) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(M)};
+  const cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+  const cuuint32_t box[2] = {64, cuuint32_t(nt)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int BITS, int NT>
+static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
+                             cudaStream_t stream) {
+  using Cfg = GemmCfg<NT>;
+  static int granted[64] = {0};
+  const int smem = 1024 + kLutBytes + Cfg::XS * Cfg::XSTAGE + Cfg::PS * 4 * tile_bytes(BITS) + 512;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (granted[dev] < smem) {
+    err = cudaFuncSetAttribute(gemm_kernel<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem);
+    if (err != cudaSuccess) return err;
+    granted[dev] = smem;
+  }
+  a.C = int(std::min<int64_t>(std::min<int64_t>(num_sms, kGemmMaxCtas), a.U));
+  gemm_kernel<BITS, NT><<<unsigned(a.C), Cfg::THREADS, smem, stream>>>(map, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* scales,
+                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
+                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream) {
+  const int nt = gemm_nt(M);
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof(map));
+  cudaError_t err = make_x_map(&map, x, M, K, nt);
+  if (err != cudaSuccess) return err;
+  GemmArgs a;
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.scales = static_cast<const uint16_t*>(scales);
+  a.codebook = static_cast<const uint16_t*>(codebook);
+  a.y = y;
+  a.dev_status = dev_status;
+  a.N = N;
+  a.G = K / kGroup;
+  a.M = M;
+  a.ntiles = (N + kTileRows - 1) / kTileRows;
+  const int64_t bt = (M + kTileRows - 1) / kTileRows;
+  a.U = bt * a.ntiles * a.G;
+  const int64_t counters = (bt * a.ntiles * 4 * kMaxPromoteGroups * 4 + 255) / 256 * 256;
+  a.counters = static_cast<int*>(workspace);
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + counters);
+  a.C = 0;
+  if (bits == 4) {
+    switch (nt) {
+      case 16: return launch_nt<4, 16>(map, a, num_sms, stream);
+      case 32: return launch_nt<4, 32>(map, a, num_sms, stream);
+      case 64: return launch_nt<4, 64>(map, a, num_sms, stream);
+      default: return launch_nt<4, 128>(map, a, num_sms, stream);
+    }
+  }
+  switch (nt) {
+    case 16: return launch_nt<3, 16>(map, a, num_sms, stream);
+    case 32: return launch_nt<3, 32>(map, a, num_sms, stream);
+    case 64: return launch_nt<3, 64>(map, a, num_sms, stream);
+    default: return launch_nt<3, 128>(map, a, num_sms, stream);
+  }
 }
 
 }  // namespace lutq

@@ -1,36 +1,50 @@
 // Fused dequantize-and-multiply GEMV for batches M = 1..16 on the CUDA cores
 // (the FLUTE abstract, "Daily Papers" listing, query "group-128": fuse
-// dequantization with the product, duplicate the lookup table against
-// shared-memory bandwidth limits; the BitMoD abstract, same listing: rescale
-// each group's partial sum once).
+// dequantization with the product; duplicate and vectorize the lookup table
+// against shared-memory bandwidth limits.  The BitMoD abstract, same listing:
+// rescale each group's partial sum once).
 //
-// Work split.  The packed matrix is a sequence of U = (N/32) * G units, one
-// unit = (strip of 32 rows, group of 128 codes) = 2048 (4-bit) or 1536 (3-bit)
-// contiguous bytes.  The W active warps of a persistent grid take contiguous,
-// equal-length unit ranges [floor(w U / W), floor((w+1) U / W)), so every warp
-// streams the same number of bytes.  Inside a unit, lane r owns row 32*strip+r
-// and reads its 16-byte words with coalesced 512-byte warp loads.
+// Work split (both kernels).  The packed matrix is a sequence of
+// U = (N/32) * G units, one unit = (strip of 32 rows, group of 128 codes) =
+// 2048 (4-bit) or 1536 (3-bit) contiguous bytes.  CTA c of a persistent grid
+// of C CTAs takes units [floor(c U / C), floor((c+1) U / C)); warp w of its NW
+// warps takes an equal share of that range, so every warp streams the same
+// number of bytes.  Sums are reduced in two deterministic levels:
+//  - a strip held whole by one warp is written by that warp;
+//  - otherwise each warp leaves its partial row sums of the strips at the two
+//    ends of its range in shared memory, and after a block barrier one warp
+//    per strip adds them in warp order;
+//  - a strip shared with other CTAs is finished by the last CTA to arrive
+//    (one atomic per contributor), which adds the CTAs' partials in CTA order
+//    and resets the strip's counter to zero for the next call.
+// Results therefore do not depend on timing.
 //
-// A strip whose units lie in one warp's range is finished by that warp.  A
-// strip split between warps is finished by the last contributor to arrive
-// (counted with one atomic per contributor): it adds the contributors'
-// partial sums in warp order, so the result does not depend on timing, and
-// resets the strip's counter to zero for the next call.
+// M = 1 kernel.  Lane t of a warp owns the k-chunk q = t & 3 (32 codes,
+// k = 128 g + 32 q ..) of the four rows (t >> 2) + 8 i, i = 0..3, of the
+// strip.  Its 32 activations stay in registers (fp32) and serve four rows;
+// each code pair costs one byte permute (forming the table address), one
+// conflict-free shared load, two bit operations (bf16 pair -> fp32 pair) and
+// one packed fp32x2 fused multiply-add.  The four lanes of a row add their
+// sums at the end of the strip.
 //
-// Lookup table.  Each shared-memory row of 256 bytes holds, for one 8-bit
-// pair index e, the code pair (c[even], c[odd]) as bf16x2, 32 times for the
-// "E" table and 32 times for the "O" table (3-bit only), one copy per lane,
-// so a warp-wide lookup never has a bank conflict.  A single byte permute
-// turns a packed byte into the lookup address: (byte << 8) | lane offset.
+// M = 2..16 kernel.  Lane r owns row 32 * strip + r and reads its 16-byte
+// words with coalesced 512-byte warp loads; activations come from global
+// memory through L1.  (Batches of more than one row are a small dense
+// contraction; the tensor-core kernel covers them too.)
+#include <algorithm>
+
 #include "lutq_common.cuh"
+#include "lutq_lut.cuh"
 
 namespace lutq {
 
-constexpr int kGemvWarps = 16;                       // warps per CTA
-constexpr int kGemvThreads = kGemvWarps * 32;
-constexpr int kLutBytes = 256 * 256;                 // 64 KB
-constexpr int kMaxWarpsTotal = 4096;                 // bounds the workspace
-constexpr int kXSmemMaxK = 40960;                    // fp32 x staged in shared memory if K <= this
+constexpr int kMaxCtas = 512;           // bounds the workspace
+#ifndef LUTQ_M1_WARPS
+#define LUTQ_M1_WARPS 20
+#endif
+constexpr int kM1Warps = LUTQ_M1_WARPS; // warps per CTA, M = 1 kernel
+constexpr int kGenWarps = 16;           // warps per CTA, generic kernel
+constexpr int kMaxSmemPerBlock = 227 * 1024;
 
 struct GemvArgs {
   const uint16_t* x;        // bf16 [M, K]
@@ -38,32 +52,104 @@ struct GemvArgs {
   const uint16_t* scales;   // bf16 [N, G]
   const uint16_t* codebook; // bf16 [2^bits]
   float* y;                 // fp32 [M, N]
-  float* part;              // [kMaxWarpsTotal][2][M][32] split-strip partial sums
+  float* part;              // [kMaxCtas][2][M][32]: CTA partials of strips shared between CTAs
   int* counters;            // [N/32] arrival counters (zero between calls)
   int64_t N, K, G, U;       // U = number of units
-  int W;                    // active warps
+  int C;                    // CTAs
 };
 
-__host__ __device__ inline int64_t unit_begin(int64_t w, int64_t U, int64_t W) { return (w * U) / W; }
-// The warp whose range holds unit u.
-__host__ __device__ inline int64_t unit_owner(int64_t u, int64_t U, int64_t W) { return ((u + 1) * W - 1) / U; }
-
-__device__ __forceinline__ uint32_t lut_addr(uint32_t word, uint32_t lane_off, int byte) {
-  // (byte `byte` of word) << 8 | lane_off  -- lane_off < 256
-  return __byte_perm(word, lane_off, 0x5504u | (uint32_t(byte) << 4));
+// Part i of `parts` equal shares of [0, total): [range_begin(i), range_begin(i+1)).
+__host__ __device__ inline int64_t range_begin(int64_t i, int64_t total, int64_t parts) {
+  return (i * total) / parts;
+}
+// The part holding element u (the last one whose range starts at or before u).
+__host__ __device__ inline int64_t range_owner(int64_t u, int64_t total, int64_t parts) {
+  return ((u + 1) * parts - 1) / total;
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t smem_addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr));
-  return v;
+__device__ __forceinline__ uint32_t sm_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ float4 lds128f(uint32_t smem_addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(smem_addr));
-  return v;
+// A warp has summed the strip `strip`.  vals[i][m] is the sum of row rows[i]
+// (within the strip) for batch row m, held by the lanes marked `writer`.
+// [u0, u1) is the warp's unit range; slots is its [2][M][32] shared area.
+template <int M, int R>
+__device__ __forceinline__ void deposit_strip(const GemvArgs& a, int64_t strip, int64_t u0,
+                                              int64_t u1, const float (&vals)[R][M],
+                                              const int (&rows)[R], bool writer, float* slots) {
+  if (!writer) return;
+  const int64_t lo = strip * a.G;
+  if (lo >= u0 && lo + a.G <= u1) {
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+      for (int m = 0; m < M; ++m) a.y[m * a.N + lo / a.G * kStrip + rows[i]] = vals[i][m];
+    return;
+  }
+  const int sl = (strip == u0 / a.G) ? 0 : 1;
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int m = 0; m < M; ++m) slots[(sl * M + m) * kStrip + rows[i]] = vals[i][m];
+}
+
+// After a block barrier: finish every strip of the CTA's range [cu0, cu1)
+// that no single warp held whole.  all_slots is [NW][2][M][32].
+template <int M, int NW>
+__device__ void cta_finish(const GemvArgs& a, const float* all_slots, int64_t cu0, int64_t cu1) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t L = cu1 - cu0;
+  const int64_t s_first = cu0 / a.G, s_last = (cu1 - 1) / a.G;
+  for (int64_t strip = s_first + warp; strip <= s_last; strip += NW) {
+    const int64_t lo = strip * a.G, hi = lo + a.G;
+    const int64_t vlo = (lo > cu0 ? lo : cu0) - cu0, vhi = (hi < cu1 ? hi : cu1) - cu0;
+    const int w_lo = int(range_owner(vlo, L, NW)), w_hi = int(range_owner(vhi - 1, L, NW));
+    if (w_lo == w_hi && range_begin(w_lo, L, NW) <= lo - cu0 &&
+        range_begin(w_lo + 1, L, NW) >= hi - cu0)
+      continue;  // written by its warp
+    float sum[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) sum[m] = 0.0f;
+    for (int w = w_lo; w <= w_hi; ++w) {
+      const int64_t b = range_begin(w, L, NW), e = range_begin(w + 1, L, NW);
+      if (b == e) continue;  // a warp without units
+      const int sl = (strip == (cu0 + b) / a.G) ? 0 : 1;
+      const float* src = all_slots + ((w * 2 + sl) * M) * kStrip;
+#pragma unroll
+      for (int m = 0; m < M; ++m) sum[m] += src[m * kStrip + lane];
+    }
+    float* yrow = a.y + strip * kStrip + lane;
+    if (lo >= cu0 && hi <= cu1) {
+#pragma unroll
+      for (int m = 0; m < M; ++m) yrow[m * a.N] = sum[m];
+      continue;
+    }
+    // shared with other CTAs
+    const int slot = (strip == s_first) ? 0 : 1;
+    float* mine = a.part + ((int64_t(blockIdx.x) * 2 + slot) * M) * kStrip;
+#pragma unroll
+    for (int m = 0; m < M; ++m) mine[m * kStrip + lane] = sum[m];
+    __threadfence();
+    __syncwarp();
+    const int64_t c_lo = range_owner(lo, a.U, a.C), c_hi = range_owner(hi - 1, a.U, a.C);
+    int arrived = 0;
+    if (lane == 0) arrived = atomicAdd(a.counters + strip, 1);
+    arrived = __shfl_sync(0xffffffffu, arrived, 0);
+    if (arrived != int(c_hi - c_lo)) continue;
+    __threadfence();
+#pragma unroll
+    for (int m = 0; m < M; ++m) sum[m] = 0.0f;
+    for (int64_t c = c_lo; c <= c_hi; ++c) {
+      const int sl = (strip == range_begin(c, a.U, a.C) / a.G) ? 0 : 1;
+      const float* src = a.part + ((c * 2 + sl) * M) * kStrip;
+#pragma unroll
+      for (int m = 0; m < M; ++m) sum[m] += __ldcg(src + m * kStrip + lane);
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m) yrow[m * a.N] = sum[m];
+    if (lane == 0) a.counters[strip] = 0;
+  }
 }
 
 // acc += (lo, hi) * (x0, x1) elementwise, one packed fp32x2 FMA.
@@ -76,80 +162,240 @@ __device__ __forceinline__ void ffma2(float2& acc, float lo, float hi, float x0,
   asm("mov.b64 {%0, %1}, %2;" : "=f"(acc.x), "=f"(acc.y) : "l"(a));
 }
 
-template <int BITS>
-__device__ __forceinline__ uint32_t lut_entry(const uint16_t* cb, int e, int half) {
-  uint32_t qe, qo;
-  if (BITS == 4) {
-    qe = e & 15;
-    qo = e >> 4;
-  } else if (half == 0) {  // E table: lo2 in bits 3:0, hi bits 4 (even) and 5 (odd)
-    qe = (e & 3) | (((e >> 4) & 1) << 2);
-    qo = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
-  } else {                 // O table: lo2 in bits 7:4, hi bits 0 (even) and 1 (odd)
-    qe = ((e >> 4) & 3) | ((e & 1) << 2);
-    qo = ((e >> 6) & 3) | (((e >> 1) & 1) << 2);
+// --------------------------------------------------------------------------
+// M = 1
+// --------------------------------------------------------------------------
+
+// One u32 of four pair indices against four activation pairs.  acc and each
+// x pair are fp32x2 values held in one 64-bit register (low half = even k).
+__device__ __forceinline__ void pairs4(uint64_t& acc, uint32_t idx, uint32_t lane_hi,
+                                       const uint64_t* x) {
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    // byte b -> bits 15:8; the lane offset (bits 7:0) and the table's 64 KB
+    // page (bits 23:16) come from lane_hi
+    const uint32_t lv = lds32(__byte_perm(idx, lane_hi, 0x6504u | (uint32_t(b) << 4)));
+    asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 w;\n\t"
+        "shl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xffff0000;\n\t"
+        "mov.b64 w, {lo, hi};\n\tfma.rn.f32x2 %0, w, %2, %0;\n\t}"
+        : "+l"(acc) : "r"(lv), "l"(x[b]));
   }
-  return uint32_t(cb[qe]) | (uint32_t(cb[qo]) << 16);
 }
 
-// Per-pair multiply-accumulate into the group partial sums.
-template <int M, bool XS>
-struct PairFma;
-
-template <>
-struct PairFma<1, true> {
-  // x in shared memory as fp32; one call handles the 4 pairs of one u32
-  // index word (8 consecutive k starting at k).
-  __device__ __forceinline__ static void run4(float2 (&part)[1], const uint32_t (&lv)[4],
-                                              uint32_t xs_addr, int k, const uint16_t*, int64_t) {
-    const float4 xa = lds128f(xs_addr + 4u * k);
-    const float4 xb = lds128f(xs_addr + 4u * (k + 4));
-    ffma2(part[0], bf16_lo_to_f32(lv[0]), bf16_hi_to_f32(lv[0]), xa.x, xa.y);
-    ffma2(part[0], bf16_lo_to_f32(lv[1]), bf16_hi_to_f32(lv[1]), xa.z, xa.w);
-    ffma2(part[0], bf16_lo_to_f32(lv[2]), bf16_hi_to_f32(lv[2]), xb.x, xb.y);
-    ffma2(part[0], bf16_lo_to_f32(lv[3]), bf16_hi_to_f32(lv[3]), xb.z, xb.w);
+// Per lane and unit: 4 rows x 32 codes.  wd[i] holds row i's 16 bytes for the
+// lane (4-bit: one word; 3-bit: 8 lo-plane bytes then 8 hi-plane bytes).
+template <int BITS>
+__device__ __forceinline__ void load_unit_m1(uint4 (&wd)[4], const uint8_t* tile, int lane) {
+  const int q = lane & 3, rq = lane >> 2;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = rq + 8 * i;
+    if (BITS == 4) {
+      wd[i] = ld_stream_v4(tile + (32 * q + r) * kWordBytes);
+    } else {
+      // lo word q >> 1, u32 2(q&1) and 2(q&1)+1; the hi word's u32 with the same index
+      const uint8_t* lo = tile + (32 * (q >> 1) + r) * kWordBytes + 8 * (q & 1);
+      const uint8_t* hi = tile + (64 + r) * kWordBytes + 8 * (q & 1);
+      uint32_t l0, l1, h0, h1;
+      asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                   : "=r"(l0), "=r"(l1) : "l"(lo));
+      asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(h0), "=r"(h1) : "l"(hi));
+      wd[i] = make_uint4(l0, l1, h0, h1);
+    }
   }
-};
+}
 
-template <int M>
-struct PairFma<M, false> {
-  // x read from global memory (bf16, L1-cached broadcast loads).
-  __device__ __forceinline__ static void run4(float2 (&part)[M], const uint32_t (&lv)[4],
-                                              uint32_t, int k, const uint16_t* x, int64_t K) {
+template <int BITS>
+__device__ __forceinline__ float row_partial_m1(const uint4& wd, uint32_t lane_e, uint32_t lane_o,
+                                                uint32_t hi_shift, const uint64_t (&x)[16]) {
+  uint64_t p = 0;
+  if (BITS == 4) {
+    pairs4(p, wd.x, lane_e, x + 0);
+    pairs4(p, wd.y, lane_e, x + 4);
+    pairs4(p, wd.z, lane_e, x + 8);
+    pairs4(p, wd.w, lane_e, x + 12);
+  } else {
+    // lo u32 j goes with hi u32 j; lo word 1 reads its hi fields two bits up
+    const uint32_t l[2] = {wd.x, wd.y}, h[2] = {wd.z >> hi_shift, wd.w >> hi_shift};
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + m * K + k));
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t e = (l[j] & 0x0F0F0F0Fu) | (h[j] & 0xF0F0F0F0u);
+      const uint32_t o = (l[j] & 0xF0F0F0F0u) | (h[j] & 0x0F0F0F0Fu);
+      pairs4(p, e, lane_e, x + 8 * j);
+      pairs4(p, o, lane_o, x + 8 * j + 4);
+    }
+  }
+  return __uint_as_float(uint32_t(p)) + __uint_as_float(uint32_t(p >> 32));
+}
+
+// Activations in shared memory: XF32 keeps fp32 values with 16 bytes of
+// padding after every 32 (so the four k-chunks of a group that the lanes of a
+// row read fall in different banks); otherwise bf16, widened when loaded.
+__host__ __device__ constexpr int x_pad_floats(int64_t k) { return int(k + k / 32 * 4); }
+
+template <bool XF32>
+__device__ __forceinline__ void load_x_m1(uint64_t (&x)[16], uint32_t xs_sa, int64_t g, int q) {
+  if (XF32) {
+    const uint32_t xa = xs_sa + uint32_t(x_pad_floats(g * kGroup + 32 * q)) * 4u;
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        ffma2(part[m], bf16_lo_to_f32(lv[p]), bf16_hi_to_f32(lv[p]), bf16_lo_to_f32(xw[p]),
-              bf16_hi_to_f32(xw[p]));
+    for (int v = 0; v < 8; ++v)
+      asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
+                   : "=l"(x[2 * v]), "=l"(x[2 * v + 1]) : "r"(xa + 16u * v));
+  } else {
+    const uint32_t xa = xs_sa + uint32_t(g * kGroup + 32 * q) * 2u;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint32_t r[4];
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(xa + 16u * v));
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        x[4 * v + t] = uint64_t(r[t] << 16) | (uint64_t(r[t] & 0xffff0000u) << 32);
+    }
+  }
+}
+
+template <int BITS, bool XF32>
+__global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ uint16_t cbs[16];
+  // The table sits on a 64 KB page of the shared window so that one byte
+  // permute produces its full address; activations and warp slots follow.
+  const uint32_t sbase = sm_addr(smem);
+  const uint32_t lut_sa = (sbase + 0xFFFFu) & ~0xFFFFu;
+  uint8_t* lut = smem + (lut_sa - sbase);
+  uint8_t* xs = lut + kLutBytes;
+  float* slots = reinterpret_cast<float*>(xs + (XF32 ? 4 * x_pad_floats(a.K) : 2 * a.K));
+
+  if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
+  {
+    const uint4* xg = reinterpret_cast<const uint4*>(a.x);
+    for (int64_t i = threadIdx.x; i < a.K / 8; i += blockDim.x) {
+      const uint4 v = __ldg(xg + i);
+      if (XF32) {
+        // 8 values k = 8i..8i+7 stay inside one 32-value chunk
+        float4* xd = reinterpret_cast<float4*>(reinterpret_cast<float*>(xs) + x_pad_floats(8 * i));
+        xd[0] = make_float4(bf16_lo_to_f32(v.x), bf16_hi_to_f32(v.x), bf16_lo_to_f32(v.y),
+                            bf16_hi_to_f32(v.y));
+        xd[1] = make_float4(bf16_lo_to_f32(v.z), bf16_hi_to_f32(v.z), bf16_lo_to_f32(v.w),
+                            bf16_hi_to_f32(v.w));
+      } else {
+        reinterpret_cast<uint4*>(xs)[i] = v;
       }
     }
   }
-};
+  __syncthreads();
+  // 16-byte chunk c of the table: row e = c >> 4, half (c >> 3) & 1, 4 lane copies.
+  for (int c = threadIdx.x; c < kLutBytes / 16; c += blockDim.x) {
+    const uint32_t v = lut_entry<BITS>(cbs, c >> 4, (c >> 3) & 1);
+    reinterpret_cast<uint4*>(lut)[c] = make_uint4(v, v, v, v);
+  }
+  __syncthreads();
 
-// Decode one 32-bit word of four pair indices into four bf16x2 code pairs.
-__device__ __forceinline__ void lookup4(uint32_t (&lv)[4], uint32_t idx, uint32_t lut_base,
-                                        uint32_t lane_off) {
+  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  const int64_t cu0 = range_begin(blockIdx.x, a.U, a.C), cu1 = range_begin(blockIdx.x + 1, a.U, a.C);
+  const int64_t u0 = cu0 + range_begin(wl, cu1 - cu0, kM1Warps);
+  const int64_t u1 = cu0 + range_begin(wl + 1, cu1 - cu0, kM1Warps);
+  const int q = lane & 3, rq = lane >> 2;
+  const uint32_t page = (lut_sa >> 16) << 8;
+  const uint32_t lane_e = page | uint32_t(lane) * 4u, lane_o = page | (128u + uint32_t(lane) * 4u);
+  const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
+  const uint32_t xs_sa = sm_addr(xs);
+  float* my_slots = slots + wl * 2 * kStrip;
+  constexpr int TB = tile_bytes(BITS);
+  int rows[4];
 #pragma unroll
-  for (int b = 0; b < 4; ++b) lv[b] = lds32(lut_base + lut_addr(idx, lane_off, b));
+  for (int i = 0; i < 4; ++i) rows[i] = rq + 8 * i;
+
+  if (u0 < u1) {
+    int64_t strip = u0 / a.G;
+    int64_t g = u0 - strip * a.G;
+    // scales of the current and the next unit: s[32 strip + rows[i], g]
+    const uint16_t* sc = a.scales + (strip * kStrip + rq) * a.G + g;
+    const int64_t s8 = 8 * a.G;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    uint4 cur[4], nxt[4];
+    uint16_t scur[4], snxt[4];
+    load_unit_m1<BITS>(cur, a.packed + u0 * TB, lane);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) scur[i] = __ldg(sc + i * s8);
+    for (int64_t u = u0; u < u1; ++u) {
+      const bool last_g = (g == a.G - 1);
+      if (u + 1 < u1) {
+        load_unit_m1<BITS>(nxt, a.packed + (u + 1) * TB, lane);
+        // the next unit is (strip, g + 1) or (strip + 1, 0)
+        const uint16_t* sn = last_g ? sc + kStrip * a.G - (a.G - 1) : sc + 1;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) snxt[i] = __ldg(sn + i * s8);
+      }
+      uint64_t x[16];
+      load_x_m1<XF32>(x, xs_sa, g, q);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float s = __uint_as_float(uint32_t(scur[i]) << 16);
+        acc[i] = fmaf(s, row_partial_m1<BITS>(cur[i], lane_e, lane_o, hi_shift, x), acc[i]);
+      }
+      if (last_g || u + 1 == u1) {
+        float vals[4][1];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float v = acc[i];
+          v += __shfl_xor_sync(0xffffffffu, v, 1);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          vals[i][0] = v;
+          acc[i] = 0.0f;
+        }
+        deposit_strip<1, 4>(a, strip, u0, u1, vals, rows, q == 0, my_slots);
+        sc += kStrip * a.G - (a.G - 1);
+        ++strip;
+        g = 0;
+      } else {
+        ++sc;
+        ++g;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        cur[i] = nxt[i];
+        scur[i] = snxt[i];
+      }
+    }
+  }
+  __syncthreads();
+  cta_finish<1, kM1Warps>(a, slots, cu0, cu1);
 }
 
-template <int BITS, int M, bool XS>
-__device__ __forceinline__ void unit_partial(float2 (&part)[M], const uint4 (&wd)[4],
-                                             uint32_t lut_base, uint32_t off_e, uint32_t off_o,
-                                             uint32_t xs_addr, int kg, const uint16_t* x,
-                                             int64_t K) {
+// --------------------------------------------------------------------------
+// M = 2..16 (thread per row)
+// --------------------------------------------------------------------------
+
+template <int M>
+__device__ __forceinline__ void run4_global_x(float2 (&part)[M], const uint32_t (&lv)[4], int k,
+                                              const uint16_t* x, int64_t K) {
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + m * K + k));
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+      ffma2(part[m], bf16_lo_to_f32(lv[p]), bf16_hi_to_f32(lv[p]), bf16_lo_to_f32(xw[p]),
+            bf16_hi_to_f32(xw[p]));
+  }
+}
+
+template <int BITS, int M>
+__device__ __forceinline__ void unit_partial_gen(float2 (&part)[M], const uint4 (&wd)[4],
+                                                 uint32_t lut_base, uint32_t off_e,
+                                                 uint32_t off_o, int kg, const uint16_t* x,
+                                                 int64_t K) {
+  uint32_t lv[4];
   if (BITS == 4) {
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const uint32_t v[4] = {wd[w].x, wd[w].y, wd[w].z, wd[w].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        uint32_t lv[4];
         lookup4(lv, v[j], lut_base, off_e);
-        PairFma<M, XS>::run4(part, lv, xs_addr, kg + 32 * w + 8 * j, x, K);
+        run4_global_x<M>(part, lv, kg + 32 * w + 8 * j, x, K);
       }
     }
   } else {
@@ -158,192 +404,163 @@ __device__ __forceinline__ void unit_partial(float2 (&part)[M], const uint4 (&wd
     const uint32_t H[4] = {wd[2].x, wd[2].y, wd[2].z, wd[2].w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t h2 = H[j] >> 2;
-      const uint32_t e0 = (L0[j] & 0x0F0F0F0Fu) | (H[j] & 0xF0F0F0F0u);
-      const uint32_t o0 = (L0[j] & 0xF0F0F0F0u) | (H[j] & 0x0F0F0F0Fu);
-      const uint32_t e1 = (L1[j] & 0x0F0F0F0Fu) | (h2 & 0xF0F0F0F0u);
-      const uint32_t o1 = (L1[j] & 0xF0F0F0F0u) | (h2 & 0x0F0F0F0Fu);
-      uint32_t lv[4];
-      lookup4(lv, e0, lut_base, off_e);
-      PairFma<M, XS>::run4(part, lv, xs_addr, kg + 16 * j, x, K);
-      lookup4(lv, o0, lut_base, off_o);
-      PairFma<M, XS>::run4(part, lv, xs_addr, kg + 16 * j + 8, x, K);
-      lookup4(lv, e1, lut_base, off_e);
-      PairFma<M, XS>::run4(part, lv, xs_addr, kg + 64 + 16 * j, x, K);
-      lookup4(lv, o1, lut_base, off_o);
-      PairFma<M, XS>::run4(part, lv, xs_addr, kg + 64 + 16 * j + 8, x, K);
+      const W3Index ix = w3_indices(L0[j], L1[j], H[j]);
+      lookup4(lv, ix.e0, lut_base, off_e);
+      run4_global_x<M>(part, lv, kg + 16 * j, x, K);
+      lookup4(lv, ix.o0, lut_base, off_o);
+      run4_global_x<M>(part, lv, kg + 16 * j + 8, x, K);
+      lookup4(lv, ix.e1, lut_base, off_e);
+      run4_global_x<M>(part, lv, kg + 64 + 16 * j, x, K);
+      lookup4(lv, ix.o1, lut_base, off_o);
+      run4_global_x<M>(part, lv, kg + 64 + 16 * j + 8, x, K);
     }
   }
 }
 
 template <int BITS>
-__device__ __forceinline__ void load_unit(uint4 (&wd)[4], const uint8_t* tile, int lane) {
+__device__ __forceinline__ void load_unit_row(uint4 (&wd)[4], const uint8_t* tile, int lane) {
   constexpr int WPR = words_per_row(BITS);
 #pragma unroll
   for (int w = 0; w < WPR; ++w) wd[w] = ld_stream_v4(tile + (32 * w + lane) * kWordBytes);
 }
 
-template <int M>
-__device__ void finish_strip(const GemvArgs& a, int64_t strip, int64_t warp, int64_t u0, int64_t u1,
-                             const float (&acc)[M], int lane) {
-  const int64_t row = strip * kStrip + lane;
-  const int64_t s_begin = strip * a.G, s_end = s_begin + a.G;
-  if (s_begin >= u0 && s_end <= u1) {  // the whole strip is ours
-#pragma unroll
-    for (int m = 0; m < M; ++m) a.y[m * a.N + row] = acc[m];
-    return;
-  }
-  const int slot = (strip == u0 / a.G) ? 0 : 1;
-  float* mine = a.part + ((warp * 2 + slot) * M) * kStrip;
-#pragma unroll
-  for (int m = 0; m < M; ++m) mine[m * kStrip + lane] = acc[m];
-  __threadfence();
-  __syncwarp();
-  const int64_t w_lo = unit_owner(s_begin, a.U, a.W);
-  const int64_t w_hi = unit_owner(s_end - 1, a.U, a.W);
-  int arrived = 0;
-  if (lane == 0) arrived = atomicAdd(a.counters + strip, 1);
-  arrived = __shfl_sync(0xffffffffu, arrived, 0);
-  if (arrived != int(w_hi - w_lo)) return;  // not the last contributor
-  __threadfence();
-  float sum[M];
-#pragma unroll
-  for (int m = 0; m < M; ++m) sum[m] = 0.0f;
-  for (int64_t w = w_lo; w <= w_hi; ++w) {
-    const int sl = (strip == unit_begin(w, a.U, a.W) / a.G) ? 0 : 1;
-    const float* src = a.part + ((w * 2 + sl) * M) * kStrip;
-#pragma unroll
-    for (int m = 0; m < M; ++m) sum[m] += __ldcg(src + m * kStrip + lane);
-  }
-#pragma unroll
-  for (int m = 0; m < M; ++m) a.y[m * a.N + row] = sum[m];
-  if (lane == 0) a.counters[strip] = 0;
-}
-
-template <int BITS, int M, bool XS>
-__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(GemvArgs a) {
+template <int BITS, int M>
+__global__ void __launch_bounds__(kGenWarps * 32, 1) gemv_kernel(GemvArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const int lane = threadIdx.x & 31;
-  const uint32_t lut_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-  const uint32_t xs_addr = lut_base + kLutBytes;
-
-  // Build the lane-duplicated pair table: word id -> (entry, half, copy).
-  for (int id = threadIdx.x; id < kLutBytes / 4; id += blockDim.x) {
-    const int e = id >> 6, half = (id >> 5) & 1;
-    reinterpret_cast<uint32_t*>(smem)[id] = lut_entry<BITS>(a.codebook, e, half);
-  }
-  if (XS) {
-    float* xs = reinterpret_cast<float*>(smem + kLutBytes);
-    const uint32_t* xw = reinterpret_cast<const uint32_t*>(a.x);
-    for (int64_t i = threadIdx.x; i < a.K / 2; i += blockDim.x) {
-      const uint32_t v = __ldg(xw + i);
-      xs[2 * i] = bf16_lo_to_f32(v);
-      xs[2 * i + 1] = bf16_hi_to_f32(v);
-    }
+  __shared__ uint16_t cbs[16];
+  float* slots = reinterpret_cast<float*>(smem + kLutBytes);  // [NW][2][M][32]
+  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  const uint32_t lut_base = sm_addr(smem);
+  if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
+  __syncthreads();
+  for (int c = threadIdx.x; c < kLutBytes / 16; c += blockDim.x) {
+    const uint32_t v = lut_entry<BITS>(cbs, c >> 4, (c >> 3) & 1);
+    reinterpret_cast<uint4*>(smem)[c] = make_uint4(v, v, v, v);
   }
   __syncthreads();
 
-  const int64_t warp = int64_t(blockIdx.x) * kGemvWarps + (threadIdx.x >> 5);
-  if (warp >= a.W) return;
-  const int64_t u0 = unit_begin(warp, a.U, a.W), u1 = unit_begin(warp + 1, a.U, a.W);
+  const int64_t cu0 = range_begin(blockIdx.x, a.U, a.C), cu1 = range_begin(blockIdx.x + 1, a.U, a.C);
+  const int64_t u0 = cu0 + range_begin(wl, cu1 - cu0, kGenWarps);
+  const int64_t u1 = cu0 + range_begin(wl + 1, cu1 - cu0, kGenWarps);
   const uint32_t off_e = uint32_t(lane) * 4u, off_o = 128u + uint32_t(lane) * 4u;
   constexpr int TB = tile_bytes(BITS);
+  const int rows[1] = {lane};
+  float* my_slots = slots + wl * 2 * M * kStrip;
 
-  int64_t strip = u0 / a.G;
-  int64_t g = u0 - strip * a.G;
-  float acc[M];
+  if (u0 < u1) {
+    int64_t strip = u0 / a.G;
+    int64_t g = u0 - strip * a.G;
+    float acc[1][M];
 #pragma unroll
-  for (int m = 0; m < M; ++m) acc[m] = 0.0f;
-
-  uint4 cur[4], nxt[4];
-  load_unit<BITS>(cur, a.packed + u0 * TB, lane);
-  for (int64_t u = u0; u < u1; ++u) {
-    if (u + 1 < u1) load_unit<BITS>(nxt, a.packed + (u + 1) * TB, lane);
-    const int64_t row = strip * kStrip + lane;
-    const float s = __uint_as_float(uint32_t(a.scales[row * a.G + g]) << 16);
-    float2 part[M];
+    for (int m = 0; m < M; ++m) acc[0][m] = 0.0f;
+    uint4 cur[4], nxt[4];
+    load_unit_row<BITS>(cur, a.packed + u0 * TB, lane);
+    for (int64_t u = u0; u < u1; ++u) {
+      if (u + 1 < u1) load_unit_row<BITS>(nxt, a.packed + (u + 1) * TB, lane);
+      const int64_t row = strip * kStrip + lane;
+      const float s = __uint_as_float(uint32_t(a.scales[row * a.G + g]) << 16);
+      float2 part[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) part[m] = make_float2(0.0f, 0.0f);
-    unit_partial<BITS, M, XS>(part, cur, lut_base, off_e, off_o, xs_addr, int(g * kGroup), a.x,
-                              a.K);
+      for (int m = 0; m < M; ++m) part[m] = make_float2(0.0f, 0.0f);
+      unit_partial_gen<BITS, M>(part, cur, lut_base, off_e, off_o, int(g * kGroup), a.x, a.K);
 #pragma unroll
-    for (int m = 0; m < M; ++m) acc[m] = fmaf(s, part[m].x + part[m].y, acc[m]);
-    if (g == a.G - 1 || u + 1 == u1) {
-      finish_strip<M>(a, strip, warp, u0, u1, acc, lane);
+      for (int m = 0; m < M; ++m) acc[0][m] = fmaf(s, part[m].x + part[m].y, acc[0][m]);
+      if (g == a.G - 1 || u + 1 == u1) {
+        deposit_strip<M, 1>(a, strip, u0, u1, acc, rows, true, my_slots);
 #pragma unroll
-      for (int m = 0; m < M; ++m) acc[m] = 0.0f;
-      ++strip;
-      g = 0;
-    } else {
-      ++g;
+        for (int m = 0; m < M; ++m) acc[0][m] = 0.0f;
+        ++strip;
+        g = 0;
+      } else {
+        ++g;
+      }
+#pragma unroll
+      for (int w = 0; w < 4; ++w) cur[w] = nxt[w];
     }
-#pragma unroll
-    for (int w = 0; w < 4; ++w) cur[w] = nxt[w];
   }
+  __syncthreads();
+  cta_finish<M, kGenWarps>(a, slots, cu0, cu1);
 }
+
+// --------------------------------------------------------------------------
+// host side
+// --------------------------------------------------------------------------
 
 int64_t gemv_workspace_bytes(int64_t M, int64_t N) {
   const int64_t counters = ((N / kStrip) * 4 + 255) / 256 * 256;
-  return counters + int64_t(kMaxWarpsTotal) * 2 * M * kStrip * 4;
+  return counters + int64_t(kMaxCtas) * 2 * M * kStrip * 4;
 }
 
 // Per device: the largest dynamic shared-memory size already granted to a
-// kernel instance, and its resident CTAs per SM at that size.
-struct LaunchCache {
-  int smem_set[64] = {0};
-  int per_sm[64] = {0};
+// kernel instance.
+struct SmemGrant {
+  int bytes[64] = {0};
 };
 
-template <int BITS, int M, bool XS>
-static cudaError_t launch_t(const GemvArgs& a0, int num_sms, cudaStream_t stream) {
-  static LaunchCache cache;
-  GemvArgs a = a0;
-  const int smem = kLutBytes + (XS ? int(a.K) * 4 : 0);
+template <typename Kernel>
+static cudaError_t grant_smem(Kernel k, SmemGrant& g, int smem) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (cache.smem_set[dev] < smem) {
-    err = cudaFuncSetAttribute(gemv_kernel<BITS, M, XS>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (g.bytes[dev] < smem) {
+    err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    cache.smem_set[dev] = smem;
-    cache.per_sm[dev] = 0;
+    g.bytes[dev] = smem;
   }
-  int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_kernel<BITS, M, XS>,
-                                                      kGemvThreads, smem);
+  return cudaSuccess;
+}
+
+static int m1_smem(int64_t K, bool xf32) {
+  // page-alignment slack (< 64 KB) + table + activations + warp slots
+  return 2 * kLutBytes + (xf32 ? 4 * x_pad_floats(K) : 2 * int(K)) + kM1Warps * 2 * kStrip * 4;
+}
+
+template <int BITS, bool XF32>
+static cudaError_t launch_m1(GemvArgs a, int num_sms, cudaStream_t stream) {
+  static SmemGrant grant;
+  const int smem = m1_smem(a.K, XF32);
+  cudaError_t err = grant_smem(gemv_m1_kernel<BITS, XF32>, grant, smem);
   if (err != cudaSuccess) return err;
-  if (per_sm < 1) per_sm = 1;
-  int64_t blocks = int64_t(num_sms) * per_sm;
-  if (blocks * kGemvWarps > kMaxWarpsTotal) blocks = kMaxWarpsTotal / kGemvWarps;
-  const int64_t need = (a.U + kGemvWarps - 1) / kGemvWarps;
-  if (blocks > need) blocks = need;
-  a.W = int(std::min<int64_t>(blocks * kGemvWarps, a.U));
-  gemv_kernel<BITS, M, XS><<<unsigned(blocks), kGemvThreads, smem, stream>>>(a);
+  a.C = int(std::min<int64_t>(std::min<int64_t>(num_sms, kMaxCtas), a.U));
+  gemv_m1_kernel<BITS, XF32><<<unsigned(a.C), kM1Warps * 32, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int BITS, int M>
+static cudaError_t launch_gen(GemvArgs a, int num_sms, cudaStream_t stream) {
+  static SmemGrant grant;
+  const int smem = kLutBytes + kGenWarps * 2 * M * kStrip * 4;
+  cudaError_t err = grant_smem(gemv_kernel<BITS, M>, grant, smem);
+  if (err != cudaSuccess) return err;
+  a.C = int(std::min<int64_t>(std::min<int64_t>(num_sms, kMaxCtas), a.U));
+  gemv_kernel<BITS, M><<<unsigned(a.C), kGenWarps * 32, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
 template <int BITS>
 static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream_t s) {
-  const bool xs = a.K <= kXSmemMaxK;
   switch (M) {
-    case 1: return xs ? launch_t<BITS, 1, true>(a, num_sms, s) : launch_t<BITS, 1, false>(a, num_sms, s);
-    case 2: return launch_t<BITS, 2, false>(a, num_sms, s);
-    case 3: return launch_t<BITS, 3, false>(a, num_sms, s);
-    case 4: return launch_t<BITS, 4, false>(a, num_sms, s);
-    case 5: return launch_t<BITS, 5, false>(a, num_sms, s);
-    case 6: return launch_t<BITS, 6, false>(a, num_sms, s);
-    case 7: return launch_t<BITS, 7, false>(a, num_sms, s);
-    case 8: return launch_t<BITS, 8, false>(a, num_sms, s);
-    case 9: return launch_t<BITS, 9, false>(a, num_sms, s);
-    case 10: return launch_t<BITS, 10, false>(a, num_sms, s);
-    case 11: return launch_t<BITS, 11, false>(a, num_sms, s);
-    case 12: return launch_t<BITS, 12, false>(a, num_sms, s);
-    case 13: return launch_t<BITS, 13, false>(a, num_sms, s);
-    case 14: return launch_t<BITS, 14, false>(a, num_sms, s);
-    case 15: return launch_t<BITS, 15, false>(a, num_sms, s);
-    case 16: return launch_t<BITS, 16, false>(a, num_sms, s);
+    case 1:
+      // the M = 1 kernel keeps all of x in shared memory next to the table
+      if (m1_smem(a.K, true) <= kMaxSmemPerBlock) return launch_m1<BITS, true>(a, num_sms, s);
+      if (m1_smem(a.K, false) <= kMaxSmemPerBlock) return launch_m1<BITS, false>(a, num_sms, s);
+      return launch_gen<BITS, 1>(a, num_sms, s);
+    case 2: return launch_gen<BITS, 2>(a, num_sms, s);
+    case 3: return launch_gen<BITS, 3>(a, num_sms, s);
+    case 4: return launch_gen<BITS, 4>(a, num_sms, s);
+    case 5: return launch_gen<BITS, 5>(a, num_sms, s);
+    case 6: return launch_gen<BITS, 6>(a, num_sms, s);
+    case 7: return launch_gen<BITS, 7>(a, num_sms, s);
+    case 8: return launch_gen<BITS, 8>(a, num_sms, s);
+    case 9: return launch_gen<BITS, 9>(a, num_sms, s);
+    case 10: return launch_gen<BITS, 10>(a, num_sms, s);
+    case 11: return launch_gen<BITS, 11>(a, num_sms, s);
+    case 12: return launch_gen<BITS, 12>(a, num_sms, s);
+    case 13: return launch_gen<BITS, 13>(a, num_sms, s);
+    case 14: return launch_gen<BITS, 14>(a, num_sms, s);
+    case 15: return launch_gen<BITS, 15>(a, num_sms, s);
+    case 16: return launch_gen<BITS, 16>(a, num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -364,7 +581,7 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   a.K = K;
   a.G = K / kGroup;
   a.U = (N / kStrip) * a.G;
-  a.W = 0;
+  a.C = 0;
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
                    : launch_bits<3>(a, int(M), num_sms, stream);
 }

@@ -1,0 +1,111 @@
+// The lane-duplicated pair lookup table shared by the GEMV and GEMM kernels.
+//
+// Shared-memory row e (256 bytes) holds, for the 8-bit pair index e, the code
+// pair (c[even], c[odd]) as bf16x2: 32 copies for the "E" table at bytes
+// 0..127 and 32 copies for the "O" table at bytes 128..255 (only 3-bit codes
+// use O).  Lane t reads copy t, so a warp-wide lookup never has a bank
+// conflict.  One byte permute forms the address (byte << 8) | lane offset.
+// This is the vectorized (two codes per lookup) and duplicated table of the
+// FLUTE abstract ("Daily Papers" listing, query "group-128").
+#pragma once
+
+#include <cstdint>
+
+namespace lutq {
+
+constexpr int kLutBytes = 256 * 256;  // 64 KB
+
+// Pair (c[even], c[odd]) for index e of table `half` (0 = E, 1 = O).
+//  4 bit: e = q_even | q_odd << 4.
+//  3 bit, E: bits 3:0 = lo2(even) | lo2(odd) << 2, bit 4 = hi1(even), bit 5 = hi1(odd).
+//  3 bit, O: bits 7:4 = lo2(even) | lo2(odd) << 2, bit 0 = hi1(even), bit 1 = hi1(odd).
+template <int BITS>
+__device__ __forceinline__ uint32_t lut_entry(const uint16_t* cb, int e, int half) {
+  uint32_t qe, qo;
+  if (BITS == 4) {
+    qe = e & 15;
+    qo = e >> 4;
+  } else if (half == 0) {
+    qe = (e & 3) | (((e >> 4) & 1) << 2);
+    qo = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
+  } else {
+    qe = ((e >> 4) & 3) | ((e & 1) << 2);
+    qo = ((e >> 6) & 3) | (((e >> 1) & 1) << 2);
+  }
+  return uint32_t(cb[qe]) | (uint32_t(cb[qo]) << 16);
+}
+
+// All threads of the block fill the table (callers synchronize afterwards).
+template <int BITS>
+__device__ __forceinline__ void build_lut(uint8_t* lut, const uint16_t* codebook) {
+  uint16_t cb[1 << BITS];
+#pragma unroll
+  for (int i = 0; i < (1 << BITS); ++i) cb[i] = __ldg(codebook + i);
+  for (int id = threadIdx.x; id < kLutBytes / 4; id += blockDim.x) {
+    const int e = id >> 6, half = (id >> 5) & 1;
+    reinterpret_cast<uint32_t*>(lut)[id] = lut_entry<BITS>(cb, e, half);
+  }
+}
+
+// (byte `byte` of word) << 8 | lane_off, with lane_off < 256.
+__device__ __forceinline__ uint32_t lut_addr(uint32_t word, uint32_t lane_off, int byte) {
+  return __byte_perm(word, lane_off, 0x5504u | (uint32_t(byte) << 4));
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t smem_addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr));
+  return v;
+}
+
+// Four pair indices (the bytes of idx) -> four bf16x2 code pairs.
+__device__ __forceinline__ void lookup4(uint32_t* lv, uint32_t idx, uint32_t lut_base,
+                                        uint32_t lane_off) {
+#pragma unroll
+  for (int b = 0; b < 4; ++b) lv[b] = lds32(lut_base + lut_addr(idx, lane_off, b));
+}
+
+// The four 32-bit index words of one 3-bit group row, j-th u32 of the two lo
+// planes and of the hi plane: E/O indices of lo word 0 and lo word 1.
+struct W3Index {
+  uint32_t e0, o0, e1, o1;
+};
+__device__ __forceinline__ W3Index w3_indices(uint32_t l0, uint32_t l1, uint32_t h) {
+  const uint32_t h2 = h >> 2;
+  W3Index r;
+  r.e0 = (l0 & 0x0F0F0F0Fu) | (h & 0xF0F0F0F0u);
+  r.o0 = (l0 & 0xF0F0F0F0u) | (h & 0x0F0F0F0Fu);
+  r.e1 = (l1 & 0x0F0F0F0Fu) | (h2 & 0xF0F0F0F0u);
+  r.o1 = (l1 & 0xF0F0F0F0u) | (h2 & 0x0F0F0F0Fu);
+  return r;
+}
+
+// Decode one row of one group (its packed words wd[0..WPR-1]) into the 64
+// bf16x2 pairs of k = 0..127 in order: out[p] = (c[q[2p]], c[q[2p+1]]).
+template <int BITS>
+__device__ __forceinline__ void decode_group_row(uint32_t (&out)[64], const uint4 (&wd)[4],
+                                                 uint32_t lut_base, uint32_t off_e,
+                                                 uint32_t off_o) {
+  if (BITS == 4) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t v[4] = {wd[w].x, wd[w].y, wd[w].z, wd[w].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) lookup4(out + 16 * w + 4 * j, v[j], lut_base, off_e);
+    }
+  } else {
+    const uint32_t L0[4] = {wd[0].x, wd[0].y, wd[0].z, wd[0].w};
+    const uint32_t L1[4] = {wd[1].x, wd[1].y, wd[1].z, wd[1].w};
+    const uint32_t H[4] = {wd[2].x, wd[2].y, wd[2].z, wd[2].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const W3Index ix = w3_indices(L0[j], L1[j], H[j]);
+      lookup4(out + 8 * j, ix.e0, lut_base, off_e);
+      lookup4(out + 8 * j + 4, ix.o0, lut_base, off_o);
+      lookup4(out + 32 + 8 * j, ix.e1, lut_base, off_e);
+      lookup4(out + 32 + 8 * j + 4, ix.o1, lut_base, off_o);
+    }
+  }
+}
+
+}  // namespace lutq
