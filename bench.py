@@ -51,6 +51,7 @@ def parse():
     p.add_argument("--batch", type=int, default=1)
     p.add_argument("--e2e-steps", type=int, default=5000)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-side", action="store_true", help="skip the GEMM and offline lines")
     return p.parse_args()
 
 
@@ -193,8 +194,12 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     lay = workloads.layer(args.workload, args.layer)
-    rows = 256
     m = args.batch
+    # rows per step sized so that warm-up + timed steps take about a minute
+    # (the oracle's product costs roughly 40 us per row of this layer per batch row)
+    per_step = 60.0 / max(1, args.steps + args.warmup)
+    rows = int(per_step / (40e-6 * m * lay.k / 14336)) // 32 * 32
+    rows = max(32, min(lay.n, rows))
     O, x, codes, sb, levels = oracle_sample(lay, args.codebook, args.bits, m, rows)
     for _ in range(args.warmup):
         O.gemv(x, codes, sb, levels)
@@ -233,6 +238,67 @@ def capture(fn, count):
         for i in range(count):
             fn(i)
     return g
+
+
+def time_events(fn, reps):
+    """Average device time of fn() over reps calls (CUDA events, current stream)."""
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(reps):
+        fn(i)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / reps
+
+
+def side_measurements(lq, dev, args):
+    """The rest of the metric and the offline steps, each on its own workload:
+    the tensor-core GEMM at batch 128 on the 70B-shaped gate/up layer (TFLOP/s
+    against the measured bf16 peak) and quantize + pack of the headline layer."""
+    out = {}
+    hbm_peak, tf_peak, peak_kind = peaks()
+    lay = workloads.layer("llama3_70b_mlp", "gate_up")
+    n, k, bits, m = lay.n, lay.k, 4, 128
+    cb = lq.lutq_codebook("nf4", bits).to(dev)
+    w = lay.weights(seed=0).to(dev)
+    st = lq.new_status(dev)
+    codes, scales = lq.lutq_quantize(w, cb, bits, status=st)
+    packed = lq.lutq_pack(codes, bits, status=st)
+    del w, codes
+    x = workloads.activations(m, k, seed=1).to(dev)
+    y = torch.empty((m, n), dtype=torch.float32, device=dev)
+    ws = lq.new_workspace(m, n, k, bits, dev)
+    call = lambda i: lq.lutq_gemm(x, packed, scales, cb, bits, n, k, y=y, workspace=ws, status=st)
+    for i in range(3):
+        call(i)
+    s = time_events(call, 20)
+    assert int(st.item()) == 0
+    tflops = 2.0 * m * n * k / s / 1e12
+    nbytes = packed.numel() + scales.numel() * 2 + m * k * 2 + m * n * 4
+    out["gemm"] = {"workload": f"llama3_70b_mlp/gate_up W[{n},{k}] nf4 W4 group128 batch{m}",
+                   "metric": "GEMM TFLOP/s at batch>=32", "value": tflops, "unit": "TFLOP/s",
+                   "us": s * 1e6, "hbm_gbs": nbytes / s / 1e9,
+                   "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_peak,
+                                "unit": "TFLOP/s", "frac": tflops / tf_peak,
+                                "peak_source": peak_kind + " (bf16 burst)"},
+                   "kernel": "lutq::gemm_kernel"}
+    del packed, scales, x, y, ws
+    # offline steps on the headline layer
+    lay = workloads.layer(args.workload, args.layer)
+    n, k, bits = lay.n, lay.k, args.bits
+    cb = lq.lutq_codebook(args.codebook, bits).to(dev)
+    w = lay.weights(seed=0).to(dev)
+    codes, scales = lq.lutq_quantize(w, cb, bits, status=st)
+    tq = time_events(lambda i: lq.lutq_quantize(w, cb, bits, status=st), 10)
+    tp = time_events(lambda i: lq.lutq_pack(codes, bits, status=st), 10)
+    assert int(st.item()) == 0
+    q_bytes = n * k * 2 + n * k + n * (k // 128) * 2
+    p_bytes = n * k + (n * k * bits) // 8
+    out["offline"] = {"quantize_gbs": q_bytes / tq / 1e9, "quantize_us": tq * 1e6,
+                      "pack_gbs": p_bytes / tp / 1e9, "pack_us": tp * 1e6,
+                      "note": "W bf16 -> codes u8 + scales; codes -> layout V1 (L2-warm)"}
+    return out
 
 
 def run_lutq(args, world, rank, local):
@@ -336,6 +402,8 @@ def run_lutq(args, world, rank, local):
     e2e_s = max_over_ranks(world, time.perf_counter() - t0)
     e2e_gbs = nbytes * e2e_steps / e2e_s / 1e9 * world
 
+    extra = side_measurements(lq, dev, args) if not args.no_side else {}
+
     hbm_peak, tf_peak, peak_kind = peaks()
     kernel_key = f"gemv_w{bits}_m{m}_{n}x{k}"
     line = {
@@ -359,6 +427,7 @@ def run_lutq(args, world, rank, local):
         "gpu_launches": args.steps,
         "clocks": clocks,
     }
+    line.update(extra)
     if rank == 0 and not args.no_cpu_baseline and world >= 1:
         rows = 512
         gbs_cpu, per_call, calls = time_oracle(lay, args.codebook, bits, m, rows, seconds=10.0)

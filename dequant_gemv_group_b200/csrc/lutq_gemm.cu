@@ -45,17 +45,21 @@ constexpr int kTileRows = 128;
 constexpr int kGemmMaxCtas = 256;            // bounds the workspace
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kTmemCols = 512;
-constexpr int kDCol = 128;                   // partial buffers start here; A uses 0..127
-
 template <int NT>
 struct GemmCfg {
-  static constexpr int XS = NT >= 128 ? 3 : 4;     // activation stages
-  static constexpr int PS = 6;                      // packed-tile stages
+  static constexpr int XS = NT >= 128 ? 3 : 4;     // activation stages (shared memory)
+  static constexpr int PS = 6;                      // packed-tile stages (shared memory)
   static constexpr int XSTAGE = 2 * NT * 128;       // two boxes of NT rows x 128 bytes
+  static constexpr int AS = 4;                      // A stages in tensor memory (64 columns each)
+  static constexpr int DS = NT >= 128 ? 2 : (NT >= 64 ? 3 : 4);  // partial stages (NT columns)
+  static constexpr int DW = NT >= 128 ? 4 : 8;      // dequant warps (8: two per lane quarter)
+  static constexpr int KC = 64 * 4 / DW;            // A columns written per dequant warp
   static constexpr int PG = NT >= 128 ? 2 : 1;      // promotion warp groups
   static constexpr int NC = NT / PG;                // batch columns per promotion warp
-  static constexpr int WARPS = 4 + 4 * PG + 2;      // dequant, promote, load, MMA
+  static constexpr int WARPS = DW + 4 * PG + 2;     // dequant, promote, load, MMA
   static constexpr int THREADS = 32 * WARPS;
+  static constexpr int DCOL = 64 * AS;              // first partial column
+  static_assert(DCOL + DS * NT <= kTmemCols, "tensor memory columns");
 };
 constexpr int kMaxPromoteGroups = 2;
 
@@ -97,7 +101,7 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
 // Loads chunk_cols<NC>() consecutive columns (32, or 16 when a promotion warp
 // owns only 16 columns).
 template <int NC>
-__host__ __device__ constexpr int chunk_cols() { return NC >= 32 ? 32 : 16; }
+__host__ __device__ constexpr int chunk_cols() { return NC == 32 ? 32 : 16; }
 
 template <int NC>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[32]) {
@@ -159,15 +163,48 @@ __device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t s
   if (lane == 0) *counter = 0;
 }
 
+// Position (batch tile, row tile, group) of consecutive units, advanced
+// without divisions.
+struct UnitPos {
+  int64_t bt, tau, g;
+  __device__ void init(int64_t u, int64_t per_bt, int64_t G) {
+    bt = u / per_bt;
+    tau = (u - bt * per_bt) / G;
+    g = u - bt * per_bt - tau * G;
+  }
+  __device__ void next(int64_t G, int64_t ntiles) {
+    if (++g == G) {
+      g = 0;
+      if (++tau == ntiles) {
+        tau = 0;
+        ++bt;
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ void tmem_st_cols32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
 template <int BITS, int NT>
 __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, GemmArgs a) {
   using Cfg = GemmCfg<NT>;
-  constexpr int PG = Cfg::PG, NC = Cfg::NC;
-  constexpr int W_LOAD = 4 + 4 * PG, W_MMA = W_LOAD + 1;
   constexpr int TB = tile_bytes(BITS);
   constexpr int WPR = words_per_row(BITS);
-  constexpr int XS = Cfg::XS, PS = Cfg::PS;
+  constexpr int XS = Cfg::XS, PS = Cfg::PS, AS = Cfg::AS, DS = Cfg::DS, DW = Cfg::DW;
+  constexpr int PG = Cfg::PG, NC = Cfg::NC;
+  constexpr int W_LOAD = DW + 4 * PG, W_MMA = W_LOAD + 1;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_sa = smem_addr(smem_raw);
   const uint32_t base_sa = (raw_sa + 1023u) & ~1023u;
@@ -179,7 +216,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   const uint32_t bar_sa = pst_sa + PS * 4 * TB;
   // barrier ids
   constexpr int B_XF = 0, B_XE = XS, B_PF = 2 * XS, B_PE = 2 * XS + PS, B_AF = 2 * XS + 2 * PS,
-                B_AE = B_AF + 2, B_DF = B_AE + 2, B_DE = B_DF + 2, NBAR = B_DE + 2;
+                B_AE = B_AF + AS, B_DF = B_AE + AS, B_DE = B_DF + DS, NBAR = B_DE + DS;
   auto bar = [&](int i) { return bar_sa + 8u * uint32_t(i); };
   uint8_t* misc = base + (bar_sa - base_sa) + 8 * NBAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
@@ -194,11 +231,13 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     }
     for (int i = 0; i < PS; ++i) {
       mbar_init(bar(B_PF + i), 1);
-      mbar_init(bar(B_PE + i), 4);
+      mbar_init(bar(B_PE + i), DW);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(B_AF + i), 4);
+    for (int i = 0; i < AS; ++i) {
+      mbar_init(bar(B_AF + i), DW);
       mbar_init(bar(B_AE + i), 1);
+    }
+    for (int i = 0; i < DS; ++i) {
       mbar_init(bar(B_DF + i), 1);
       mbar_init(bar(B_DE + i), 4 * PG);
     }
@@ -224,56 +263,88 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   const int n = int(g_unit_begin(blockIdx.x + 1, a.U, a.C) - u0);
   const int64_t per_bt = a.ntiles * a.G;
 
-  if (warp < 4) {
+  if (warp < DW) {
     // ---------------------------------------------------------------- dequantize
-    const int sw = warp;
+    const int sw = warp & 3, kh = DW == 8 ? (warp >> 2) : 0;
     const uint32_t off_e = uint32_t(lane) * 4u, off_o = 128u + uint32_t(lane) * 4u;
-    for (int i = 0; i < n; ++i) {
-      const int64_t u = u0 + i;
-      const int64_t tau = (u % per_bt) / a.G;
-      const bool valid = tau * kTileRows + sw * 32 < a.N;
+    UnitPos pos;
+    pos.init(u0, per_bt, a.G);
+    for (int i = 0; i < n; ++i, pos.next(a.G, a.ntiles)) {
+      const bool valid = pos.tau * kTileRows + sw * 32 < a.N;
       const int ps = i % PS;
       bool ok = mbar_wait(bar(B_PF + ps), uint32_t(i / PS) & 1u, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) break;
-      uint4 wd[4];
-      if (valid) {
+      const uint32_t src = pst_sa + uint32_t(ps * 4 * TB + sw * TB + lane * 16);
+      uint32_t av[Cfg::KC];
+      if (DW == 8) {
+        uint4 wd[2];
+        if (valid) {
+          // 4-bit: words 2kh, 2kh+1; 3-bit: lo word kh and the hi word
+          wd[0] = lds128(src + uint32_t((BITS == 4 ? 2 * kh : kh) * 512));
+          wd[1] = lds128(src + uint32_t((BITS == 4 ? 2 * kh + 1 : 2) * 512));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PE + ps));
+        if (valid) decode_group_half<BITS>(reinterpret_cast<uint32_t(&)[32]>(av), wd, kh, lut_sa,
+                                           off_e, off_o);
+      } else {
+        uint4 wd[4];
+        if (valid) {
 #pragma unroll
-        for (int j = 0; j < WPR; ++j)
-          wd[j] = lds128(pst_sa + uint32_t(ps * 4 * TB + sw * TB + (32 * j + lane) * 16));
+          for (int j = 0; j < WPR; ++j) wd[j] = lds128(src + uint32_t(j * 512));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PE + ps));
+        if (valid) decode_group_row<BITS>(reinterpret_cast<uint32_t(&)[64]>(av), wd, lut_sa, off_e,
+                                          off_o);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_PE + ps));
-      uint32_t av[64];
-      if (valid) decode_group_row<BITS>(av, wd, lut_sa, off_e, off_o);
-      const int ab = i & 1;
-      ok = mbar_wait(bar(B_AE + ab), (uint32_t(i >> 1) & 1u) ^ 1u, abort_flag, kWaitLimitNs);
+      const int as = i % AS;
+      ok = mbar_wait(bar(B_AE + as), (uint32_t(i / AS) & 1u) ^ 1u, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       if (valid) {
-        tmem_st_32x32b_x64(tmem + (uint32_t(sw * 32) << 16) + uint32_t(ab * 64), av);
+        const uint32_t ta = tmem + (uint32_t(sw * 32) << 16) + uint32_t(as * 64 + kh * 32);
+        if (DW == 8)
+          tmem_st_cols32(ta, reinterpret_cast<const uint32_t(&)[32]>(av));
+        else
+          tmem_st_32x32b_x64(ta, reinterpret_cast<const uint32_t(&)[64]>(av));
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_AF + ab));
+      if (lane == 0) mbar_arrive(bar(B_AF + as));
     }
   } else if (warp < W_LOAD) {
     // ---------------------------------------------------------------- promote
-    const int sw = warp & 3, pg = (warp - 4) >> 2;
+    const int sw = warp & 3, pg = (warp - DW) >> 2;
+    UnitPos cur;
+    cur.init(u0, per_bt, a.G);
+    // The group scales of the next SD units are loaded ahead.
+    constexpr int SD = 4;
+    uint32_t sq[SD];
+    UnitPos pf = cur;
+    auto scale_of = [&](const UnitPos& p) -> uint32_t {
+      const int64_t r0 = p.tau * kTileRows + sw * 32;
+      return r0 < a.N ? uint32_t(__ldg(a.scales + (r0 + lane) * a.G + p.g)) : 0u;
+    };
+#pragma unroll
+    for (int d = 0; d < SD; ++d) {
+      sq[d] = d < n ? scale_of(pf) : 0u;
+      pf.next(a.G, a.ntiles);
+    }
     float acc[NC];
 #pragma unroll
     for (int j = 0; j < NC; ++j) acc[j] = 0.0f;
     for (int i = 0; i < n; ++i) {
-      const int64_t u = u0 + i;
-      const int64_t bt = u / per_bt;
-      const int64_t rem = u - bt * per_bt;
-      const int64_t tau = rem / a.G, g = rem - tau * a.G;
-      const int64_t row = tau * kTileRows + sw * 32 + lane;
-      const bool valid = tau * kTileRows + sw * 32 < a.N;
-      const float s =
-          valid ? __uint_as_float(uint32_t(__ldg(a.scales + row * a.G + g)) << 16) : 0.0f;
-      const int db = i & 1;
-      const bool ok = mbar_wait(bar(B_DF + db), uint32_t(i >> 1) & 1u, abort_flag, kWaitLimitNs);
+      const int64_t row = cur.tau * kTileRows + sw * 32 + lane;
+      const bool valid = cur.tau * kTileRows + sw * 32 < a.N;
+      const float s = __uint_as_float(sq[0] << 16);
+#pragma unroll
+      for (int d = 0; d < SD - 1; ++d) sq[d] = sq[d + 1];
+      sq[SD - 1] = (i + SD < n) ? scale_of(pf) : 0u;
+      pf.next(a.G, a.ntiles);
+      const int ds = i % DS;
+      const bool ok = mbar_wait(bar(B_DF + ds), uint32_t(i / DS) & 1u, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       constexpr int CH = chunk_cols<NC>();
@@ -281,7 +352,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
       for (int c = 0; c < NC / CH; ++c) {
         uint32_t v[32];
         tmem_ld_cols<NC>(tmem + (uint32_t(sw * 32) << 16) +
-                             uint32_t(kDCol + db * NT + pg * NC + c * CH),
+                             uint32_t(Cfg::DCOL + ds * NT + pg * NC + c * CH),
                          v);
         tmem_wait_ld();
 #pragma unroll
@@ -289,49 +360,49 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_DE + db));
-      if (g == a.G - 1 || i == n - 1) {
-        if (valid) gemm_finish_strip<NT, NC>(a, acc, bt * a.ntiles + tau, bt, row, sw, pg, u0, lane);
+      if (lane == 0) mbar_arrive(bar(B_DE + ds));
+      if (cur.g == a.G - 1 || i == n - 1) {
+        if (valid)
+          gemm_finish_strip<NT, NC>(a, acc, cur.bt * a.ntiles + cur.tau, cur.bt, row, sw, pg, u0,
+                                    lane);
 #pragma unroll
         for (int j = 0; j < NC; ++j) acc[j] = 0.0f;
       }
+      cur.next(a.G, a.ntiles);
     }
   } else if (warp == W_LOAD) {
     // ---------------------------------------------------------------- loads
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < n; ++i) {
-        const int64_t u = u0 + i;
-        const int64_t bt = u / per_bt;
-        const int64_t rem = u - bt * per_bt;
-        const int64_t tau = rem / a.G, g = rem - tau * a.G;
+      int issued_p = 0, issued_x = 0;
+      UnitPos pos;
+      pos.init(u0, per_bt, a.G);
+      for (int i = 0; i < n; ++i, pos.next(a.G, a.ntiles)) {
         const int ps = i % PS;
         if (!mbar_wait(bar(B_PE + ps), (uint32_t(i / PS) & 1u) ^ 1u, abort_flag, kWaitLimitNs))
           break;
-        const int64_t srem = (a.N - tau * kTileRows) / 32;
+        const int64_t srem = (a.N - pos.tau * kTileRows) / 32;
         const int vs = int(srem < 4 ? srem : 4);
         mbar_expect_tx(bar(B_PF + ps), uint32_t(vs * TB));
         for (int s = 0; s < vs; ++s)
           bulk_g2s(pst_sa + uint32_t(ps * 4 * TB + s * TB),
-                   a.packed + ((tau * 4 + s) * a.G + g) * TB, TB, bar(B_PF + ps));
+                   a.packed + ((pos.tau * 4 + s) * a.G + pos.g) * TB, TB, bar(B_PF + ps));
+        issued_p = i + 1;
         const int xs = i % XS;
-        if (!mbar_wait(bar(B_XE + xs), (uint32_t(i / XS) & 1u) ^ 1u, abort_flag, kWaitLimitNs)) {
-          issued = -(i + 1);  // packed stage i issued, activations not
+        if (!mbar_wait(bar(B_XE + xs), (uint32_t(i / XS) & 1u) ^ 1u, abort_flag, kWaitLimitNs))
           break;
-        }
         mbar_expect_tx(bar(B_XF + xs), uint32_t(Cfg::XSTAGE));
         const uint32_t xd = xst_sa + uint32_t(xs * Cfg::XSTAGE);
-        tma_2d_g2s(xd, &tmap_x, int32_t(g * 128), int32_t(bt * kTileRows), bar(B_XF + xs));
-        tma_2d_g2s(xd + NT * 128, &tmap_x, int32_t(g * 128 + 64), int32_t(bt * kTileRows),
+        tma_2d_g2s(xd, &tmap_x, int32_t(pos.g * 128), int32_t(pos.bt * kTileRows), bar(B_XF + xs));
+        tma_2d_g2s(xd + NT * 128, &tmap_x, int32_t(pos.g * 128 + 64), int32_t(pos.bt * kTileRows),
                    bar(B_XF + xs));
-        issued = i + 1;
+        issued_x = i + 1;
       }
       if (*abort_flag) {
         // let the copies in flight land before the CTA can exit
-        const int np = issued >= 0 ? issued : -issued;
-        const int nx = issued >= 0 ? issued : -issued - 1;
-        for (int i = (np > PS ? np - PS : 0); i < np; ++i) mbar_drain(bar(B_PF + i % PS), uint32_t(i / PS) & 1u);
-        for (int i = (nx > XS ? nx - XS : 0); i < nx; ++i) mbar_drain(bar(B_XF + i % XS), uint32_t(i / XS) & 1u);
+        for (int i = (issued_p > PS ? issued_p - PS : 0); i < issued_p; ++i)
+          mbar_drain(bar(B_PF + i % PS), uint32_t(i / PS) & 1u);
+        for (int i = (issued_x > XS ? issued_x - XS : 0); i < issued_x; ++i)
+          mbar_drain(bar(B_XF + i % XS), uint32_t(i / XS) & 1u);
       }
     }
   } else {
@@ -340,27 +411,27 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, NT);
       int issued = 0;
       for (int i = 0; i < n; ++i) {
-        const int xs = i % XS, ab = i & 1, db = i & 1;
+        const int xs = i % XS, as = i % AS, ds = i % DS;
         if (!mbar_wait(bar(B_XF + xs), uint32_t(i / XS) & 1u, abort_flag, kWaitLimitNs)) break;
-        if (!mbar_wait(bar(B_AF + ab), uint32_t(i >> 1) & 1u, abort_flag, kWaitLimitNs)) break;
-        if (!mbar_wait(bar(B_DE + db), (uint32_t(i >> 1) & 1u) ^ 1u, abort_flag, kWaitLimitNs))
+        if (!mbar_wait(bar(B_AF + as), uint32_t(i / AS) & 1u, abort_flag, kWaitLimitNs)) break;
+        if (!mbar_wait(bar(B_DE + ds), (uint32_t(i / DS) & 1u) ^ 1u, abort_flag, kWaitLimitNs))
           break;
         tc_fence_after();
         const uint32_t xb = xst_sa + uint32_t(xs * Cfg::XSTAGE);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t b_sa = xb + uint32_t((kk >> 2) * (NT * 128) + (kk & 3) * 32);
-          mma_bf16_ts(tmem + uint32_t(kDCol + db * NT), tmem + uint32_t(ab * 64 + 8 * kk),
+          mma_bf16_ts(tmem + uint32_t(Cfg::DCOL + ds * NT), tmem + uint32_t(as * 64 + 8 * kk),
                       smem_desc_k_sw128(b_sa), idesc, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(B_DF + db));
-        mma_commit(bar(B_AE + ab));
+        mma_commit(bar(B_DF + ds));
+        mma_commit(bar(B_AE + as));
         mma_commit(bar(B_XE + xs));
         issued = i + 1;
       }
       if (*abort_flag && issued > 0) {
         const int i = issued - 1;
-        mbar_drain(bar(B_DF + (i & 1)), uint32_t(i >> 1) & 1u);
+        mbar_drain(bar(B_DF + i % DS), uint32_t(i / DS) & 1u);
       }
     }
   }

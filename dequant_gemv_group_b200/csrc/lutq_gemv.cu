@@ -19,9 +19,10 @@
 //    and resets the strip's counter to zero for the next call.
 // Results therefore do not depend on timing.
 //
-// M = 1 kernel.  Lane t of a warp owns the k-chunk q = t & 3 (32 codes,
-// k = 128 g + 32 q ..) of the four rows (t >> 2) + 8 i, i = 0..3, of the
-// strip.  Its 32 activations stay in registers (fp32) and serve four rows;
+// M = 1 kernel.  Lane t of a warp owns the k-chunk q = t >> 3 (32 codes,
+// k = 128 g + 32 q ..) of the four rows (t & 7) + 8 i, i = 0..3, of the
+// strip (the 8 lanes of a quarter-warp share q, so activation reads are
+// broadcasts).  Its 32 activations stay in registers (fp32) and serve four rows;
 // each code pair costs one byte permute (forming the table address), one
 // conflict-free shared load, two bit operations (bf16 pair -> fp32 pair) and
 // one packed fp32x2 fused multiply-add.  The four lanes of a row add their
@@ -40,7 +41,7 @@ namespace lutq {
 
 constexpr int kMaxCtas = 512;           // bounds the workspace
 #ifndef LUTQ_M1_WARPS
-#define LUTQ_M1_WARPS 20
+#define LUTQ_M1_WARPS 16
 #endif
 constexpr int kM1Warps = LUTQ_M1_WARPS; // warps per CTA, M = 1 kernel
 constexpr int kGenWarps = 16;           // warps per CTA, generic kernel
@@ -166,19 +167,30 @@ __device__ __forceinline__ void ffma2(float2& acc, float lo, float hi, float x0,
 // M = 1
 // --------------------------------------------------------------------------
 
-// One u32 of four pair indices against four activation pairs.  acc and each
-// x pair are fp32x2 values held in one 64-bit register (low half = even k).
-__device__ __forceinline__ void pairs4(uint64_t& acc, uint32_t idx, uint32_t lane_hi,
-                                       const uint64_t* x) {
+// acc (fp32x2 in one 64-bit register) += bf16 code pair lv (low half = even
+// k) * activation pair x (fp32x2, low half = even k).
+__device__ __forceinline__ void pair_fma(uint64_t& acc, uint32_t lv, uint64_t x) {
+  asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 w;\n\t"
+      "shl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xffff0000;\n\t"
+      "mov.b64 w, {lo, hi};\n\tfma.rn.f32x2 %0, w, %2, %0;\n\t}"
+      : "+l"(acc) : "r"(lv), "l"(x));
+}
+
+// The four rows' u32 index words idx[i] (four pair indices each) against the
+// four activation pairs x[0..3]; the rows are interleaved so that four
+// independent table loads and accumulator chains are in flight.
+__device__ __forceinline__ void quad4(uint64_t (&p)[4], const uint32_t (&idx)[4],
+                                      uint32_t lane_hi, const uint64_t* x) {
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
-    // byte b -> bits 15:8; the lane offset (bits 7:0) and the table's 64 KB
-    // page (bits 23:16) come from lane_hi
-    const uint32_t lv = lds32(__byte_perm(idx, lane_hi, 0x6504u | (uint32_t(b) << 4)));
-    asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 w;\n\t"
-        "shl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xffff0000;\n\t"
-        "mov.b64 w, {lo, hi};\n\tfma.rn.f32x2 %0, w, %2, %0;\n\t}"
-        : "+l"(acc) : "r"(lv), "l"(x[b]));
+    uint32_t lv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      // byte b -> bits 15:8; the lane offset (bits 7:0) and the table's 64 KB
+      // page (bits 23:16) come from lane_hi
+      lv[i] = lds32(__byte_perm(idx[i], lane_hi, 0x6504u | (uint32_t(b) << 4)));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pair_fma(p[i], lv[i], x[b]);
   }
 }
 
@@ -186,7 +198,7 @@ __device__ __forceinline__ void pairs4(uint64_t& acc, uint32_t idx, uint32_t lan
 // lane (4-bit: one word; 3-bit: 8 lo-plane bytes then 8 hi-plane bytes).
 template <int BITS>
 __device__ __forceinline__ void load_unit_m1(uint4 (&wd)[4], const uint8_t* tile, int lane) {
-  const int q = lane & 3, rq = lane >> 2;
+  const int q = lane >> 3, rq = lane & 7;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = rq + 8 * i;
@@ -205,27 +217,46 @@ __device__ __forceinline__ void load_unit_m1(uint4 (&wd)[4], const uint8_t* tile
   }
 }
 
+// Partial sums of the four rows of one unit: p[i] (fp32x2) for row i.
 template <int BITS>
-__device__ __forceinline__ float row_partial_m1(const uint4& wd, uint32_t lane_e, uint32_t lane_o,
+__device__ __forceinline__ void unit_partial_m1(uint64_t (&p)[4], const uint4 (&wd)[4],
+                                                uint32_t lane_e, uint32_t lane_o,
                                                 uint32_t hi_shift, const uint64_t (&x)[16]) {
-  uint64_t p = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = 0;
   if (BITS == 4) {
-    pairs4(p, wd.x, lane_e, x + 0);
-    pairs4(p, wd.y, lane_e, x + 4);
-    pairs4(p, wd.z, lane_e, x + 8);
-    pairs4(p, wd.w, lane_e, x + 12);
+    {
+      const uint32_t idx[4] = {wd[0].x, wd[1].x, wd[2].x, wd[3].x};
+      quad4(p, idx, lane_e, x + 0);
+    }
+    {
+      const uint32_t idx[4] = {wd[0].y, wd[1].y, wd[2].y, wd[3].y};
+      quad4(p, idx, lane_e, x + 4);
+    }
+    {
+      const uint32_t idx[4] = {wd[0].z, wd[1].z, wd[2].z, wd[3].z};
+      quad4(p, idx, lane_e, x + 8);
+    }
+    {
+      const uint32_t idx[4] = {wd[0].w, wd[1].w, wd[2].w, wd[3].w};
+      quad4(p, idx, lane_e, x + 12);
+    }
   } else {
     // lo u32 j goes with hi u32 j; lo word 1 reads its hi fields two bits up
-    const uint32_t l[2] = {wd.x, wd.y}, h[2] = {wd.z >> hi_shift, wd.w >> hi_shift};
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      const uint32_t e = (l[j] & 0x0F0F0F0Fu) | (h[j] & 0xF0F0F0F0u);
-      const uint32_t o = (l[j] & 0xF0F0F0F0u) | (h[j] & 0x0F0F0F0Fu);
-      pairs4(p, e, lane_e, x + 8 * j);
-      pairs4(p, o, lane_o, x + 8 * j + 4);
+      uint32_t e[4], o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t l = j == 0 ? wd[i].x : wd[i].y;
+        const uint32_t h = (j == 0 ? wd[i].z : wd[i].w) >> hi_shift;
+        e[i] = (l & 0x0F0F0F0Fu) | (h & 0xF0F0F0F0u);
+        o[i] = (l & 0xF0F0F0F0u) | (h & 0x0F0F0F0Fu);
+      }
+      quad4(p, e, lane_e, x + 8 * j);
+      quad4(p, o, lane_o, x + 8 * j + 4);
     }
   }
-  return __uint_as_float(uint32_t(p)) + __uint_as_float(uint32_t(p >> 32));
 }
 
 // Activations in shared memory: XF32 keeps fp32 values with 16 bytes of
@@ -296,7 +327,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   const int64_t cu0 = range_begin(blockIdx.x, a.U, a.C), cu1 = range_begin(blockIdx.x + 1, a.U, a.C);
   const int64_t u0 = cu0 + range_begin(wl, cu1 - cu0, kM1Warps);
   const int64_t u1 = cu0 + range_begin(wl + 1, cu1 - cu0, kM1Warps);
-  const int q = lane & 3, rq = lane >> 2;
+  const int q = lane >> 3, rq = lane & 7;
   const uint32_t page = (lut_sa >> 16) << 8;
   const uint32_t lane_e = page | uint32_t(lane) * 4u, lane_o = page | (128u + uint32_t(lane) * 4u);
   const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
@@ -308,56 +339,63 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   for (int i = 0; i < 4; ++i) rows[i] = rq + 8 * i;
 
   if (u0 < u1) {
-    int64_t strip = u0 / a.G;
-    int64_t g = u0 - strip * a.G;
-    // scales of the current and the next unit: s[32 strip + rows[i], g]
-    const uint16_t* sc = a.scales + (strip * kStrip + rq) * a.G + g;
+    // Units are prefetched two ahead into three rotating buffers; `fetch`
+    // walks (strip, group) of the next unit to load.
+    int64_t f_strip = u0 / a.G, f_g = u0 - f_strip * a.G;
     const int64_t s8 = 8 * a.G;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    uint4 cur[4], nxt[4];
-    uint16_t scur[4], snxt[4];
-    load_unit_m1<BITS>(cur, a.packed + u0 * TB, lane);
+    auto load = [&](uint4 (&wd)[4], uint16_t (&sv)[4], int64_t u) {
+      load_unit_m1<BITS>(wd, a.packed + u * TB, lane);
+      const uint16_t* sc = a.scales + (f_strip * kStrip + rq) * a.G + f_g;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) scur[i] = __ldg(sc + i * s8);
-    for (int64_t u = u0; u < u1; ++u) {
-      const bool last_g = (g == a.G - 1);
-      if (u + 1 < u1) {
-        load_unit_m1<BITS>(nxt, a.packed + (u + 1) * TB, lane);
-        // the next unit is (strip, g + 1) or (strip + 1, 0)
-        const uint16_t* sn = last_g ? sc + kStrip * a.G - (a.G - 1) : sc + 1;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) snxt[i] = __ldg(sn + i * s8);
+      for (int i = 0; i < 4; ++i) sv[i] = __ldg(sc + i * s8);
+      if (++f_g == a.G) {
+        f_g = 0;
+        ++f_strip;
       }
+    };
+    int64_t strip = f_strip, g = f_g;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    // consume one unit held in (wd, sv); refill that buffer with unit u + 3
+    auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], int64_t u) {
       uint64_t x[16];
       load_x_m1<XF32>(x, xs_sa, g, q);
+      uint64_t p[4];
+      unit_partial_m1<BITS>(p, wd, lane_e, lane_o, hi_shift, x);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float s = __uint_as_float(uint32_t(scur[i]) << 16);
-        acc[i] = fmaf(s, row_partial_m1<BITS>(cur[i], lane_e, lane_o, hi_shift, x), acc[i]);
+        const float s = __uint_as_float(uint32_t(sv[i]) << 16);
+        const float v = __uint_as_float(uint32_t(p[i])) + __uint_as_float(uint32_t(p[i] >> 32));
+        acc[i] = fmaf(s, v, acc[i]);
       }
-      if (last_g || u + 1 == u1) {
+      if (u + 3 < u1) load(wd, sv, u + 3);
+      if (g == a.G - 1 || u + 1 == u1) {
         float vals[4][1];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float v = acc[i];
-          v += __shfl_xor_sync(0xffffffffu, v, 1);
-          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
           vals[i][0] = v;
           acc[i] = 0.0f;
         }
         deposit_strip<1, 4>(a, strip, u0, u1, vals, rows, q == 0, my_slots);
-        sc += kStrip * a.G - (a.G - 1);
         ++strip;
         g = 0;
       } else {
-        ++sc;
         ++g;
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        cur[i] = nxt[i];
-        scur[i] = snxt[i];
-      }
+    };
+    uint4 b0[4], b1[4], b2[4];
+    uint16_t s0[4], s1[4], s2[4];
+    load(b0, s0, u0);
+    if (u0 + 1 < u1) load(b1, s1, u0 + 1);
+    if (u0 + 2 < u1) load(b2, s2, u0 + 2);
+    for (int64_t u = u0; u < u1; u += 3) {
+      step(b0, s0, u);
+      if (u + 1 >= u1) break;
+      step(b1, s1, u + 1);
+      if (u + 2 >= u1) break;
+      step(b2, s2, u + 2);
     }
   }
   __syncthreads();

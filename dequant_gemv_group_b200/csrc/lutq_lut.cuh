@@ -108,4 +108,30 @@ __device__ __forceinline__ void decode_group_row(uint32_t (&out)[64], const uint
   }
 }
 
+// Half of a group row: pairs 32 h .. 32 h + 31 (k = 64 h .. 64 h + 63) into
+// out[0..31].  4-bit: wd[0], wd[1] are words 2h, 2h+1.  3-bit: wd[0] is lo word
+// h and wd[1] the hi word.
+template <int BITS>
+__device__ __forceinline__ void decode_group_half(uint32_t (&out)[32], const uint4 (&wd)[2],
+                                                  int h, uint32_t lut_base, uint32_t off_e,
+                                                  uint32_t off_o) {
+  if (BITS == 4) {
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const uint32_t v[4] = {wd[w].x, wd[w].y, wd[w].z, wd[w].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) lookup4(out + 16 * w + 4 * j, v[j], lut_base, off_e);
+    }
+  } else {
+    const uint32_t L[4] = {wd[0].x, wd[0].y, wd[0].z, wd[0].w};
+    const uint32_t sh = 2u * uint32_t(h);
+    const uint32_t H[4] = {wd[1].x >> sh, wd[1].y >> sh, wd[1].z >> sh, wd[1].w >> sh};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      lookup4(out + 8 * j, (L[j] & 0x0F0F0F0Fu) | (H[j] & 0xF0F0F0F0u), lut_base, off_e);
+      lookup4(out + 8 * j + 4, (L[j] & 0xF0F0F0F0u) | (H[j] & 0x0F0F0F0Fu), lut_base, off_o);
+    }
+  }
+}
+
 }  // namespace lutq
