@@ -31,4 +31,13 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   return r;
 }
 
+// One acquire-release atomic add at GPU scope: publishes the calling warp's
+// earlier stores (ordered before it by __syncwarp) and, for the caller that
+// sees the final count, makes the other contributors' stores visible.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 }  // namespace lutq

@@ -48,7 +48,7 @@ constexpr int kTmemCols = 512;
 template <int NT>
 struct GemmCfg {
   static constexpr int XS = NT >= 128 ? 3 : 4;     // activation stages (shared memory)
-  static constexpr int PS = 6;                      // packed-tile stages (shared memory)
+  static constexpr int PS = NT >= 128 ? 4 : (NT >= 64 ? 8 : 12);  // packed-tile stages
   static constexpr int XSTAGE = 2 * NT * 128;       // two boxes of NT rows x 128 bytes
   static constexpr int AS = 4;                      // A stages in tensor memory (64 columns each)
   static constexpr int DS = NT >= 128 ? 2 : (NT >= 64 ? 3 : 4);  // partial stages (NT columns)
@@ -77,8 +77,12 @@ struct GemmArgs {
   int C;              // CTAs
 };
 
-__device__ __forceinline__ int64_t g_unit_begin(int64_t c, int64_t U, int64_t C) { return (c * U) / C; }
-__device__ __forceinline__ int64_t g_unit_owner(int64_t u, int64_t U, int64_t C) {
+// CTA c holds units [g_unit_begin(c), g_unit_begin(c+1)).  The host
+// guarantees U * C < 2^32, so the ranges use 32-bit unsigned arithmetic.
+__device__ __forceinline__ uint32_t g_unit_begin(uint32_t c, uint32_t U, uint32_t C) {
+  return (c * U) / C;
+}
+__device__ __forceinline__ uint32_t g_unit_owner(uint32_t u, uint32_t U, uint32_t C) {
   return ((u + 1) * C - 1) / U;
 }
 
@@ -123,12 +127,14 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[32]) 
 // holds batch columns [c0, c0 + NC).
 template <int NT, int NC>
 __device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t seg, int64_t bt,
-                                  int64_t row, int sw, int pg, int64_t u0, int lane) {
+                                  int64_t row, int sw, int pg, uint32_t u0, int lane) {
   const int c0 = pg * NC;
   const int64_t seg_begin = seg * a.G, seg_end = seg_begin + a.G;
   const int64_t mrem = a.M - bt * kTileRows;
   const int mt = int(mrem < kTileRows ? mrem : kTileRows);
-  const int64_t c_lo = g_unit_owner(seg_begin, a.U, a.C), c_hi = g_unit_owner(seg_end - 1, a.U, a.C);
+  const uint32_t U = uint32_t(a.U), C = uint32_t(a.C);
+  const uint32_t c_lo = g_unit_owner(uint32_t(seg_begin), U, C);
+  const uint32_t c_hi = g_unit_owner(uint32_t(seg_end - 1), U, C);
   float* ycol = a.y + (bt * kTileRows + c0) * a.N + row;
   if (c_lo == c_hi) {
 #pragma unroll
@@ -137,22 +143,21 @@ __device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t s
     return;
   }
   const int64_t cta = blockIdx.x;
-  const int slot = (seg == u0 / a.G) ? 0 : 1;
+  const int slot = (uint32_t(seg) == uint32_t(u0) / uint32_t(a.G)) ? 0 : 1;
   float* mine = a.part + (((cta * 2 + slot) * 4 + sw) * NT + c0) * 32;
 #pragma unroll
   for (int j = 0; j < NC; ++j) mine[j * 32 + lane] = acc[j];
-  __threadfence();
   __syncwarp();
   int arrived = 0;
   int* counter = a.counters + (seg * 4 + sw) * kMaxPromoteGroups + pg;
-  if (lane == 0) arrived = atomicAdd(counter, 1);
+  if (lane == 0) arrived = atom_add_acq_rel_gpu(counter, 1);
   arrived = __shfl_sync(0xffffffffu, arrived, 0);
   if (arrived != int(c_hi - c_lo)) return;
-  __threadfence();
+  __syncwarp();  // the other lanes' loads follow lane 0's acquire
 #pragma unroll
   for (int j = 0; j < NC; ++j) acc[j] = 0.0f;
-  for (int64_t c = c_lo; c <= c_hi; ++c) {
-    const int sl = (seg == g_unit_begin(c, a.U, a.C) / a.G) ? 0 : 1;
+  for (uint32_t c = c_lo; c <= c_hi; ++c) {
+    const int sl = (uint32_t(seg) == g_unit_begin(c, U, C) / uint32_t(a.G)) ? 0 : 1;
     const float* src = a.part + (((c * 2 + sl) * 4 + sw) * NT + c0) * 32;
 #pragma unroll
     for (int j = 0; j < NC; ++j) acc[j] += __ldcg(src + j * 32 + lane);
@@ -167,10 +172,11 @@ __device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t s
 // without divisions.
 struct UnitPos {
   int64_t bt, tau, g;
-  __device__ void init(int64_t u, int64_t per_bt, int64_t G) {
-    bt = u / per_bt;
-    tau = (u - bt * per_bt) / G;
-    g = u - bt * per_bt - tau * G;
+  __device__ void init(uint32_t u, uint32_t per_bt, uint32_t G) {
+    const uint32_t b = u / per_bt, r = u - b * per_bt, t = r / G;
+    bt = b;
+    tau = t;
+    g = r - t * G;
   }
   __device__ void next(int64_t G, int64_t ntiles) {
     if (++g == G) {
@@ -259,9 +265,9 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int64_t u0 = g_unit_begin(blockIdx.x, a.U, a.C);
-  const int n = int(g_unit_begin(blockIdx.x + 1, a.U, a.C) - u0);
-  const int64_t per_bt = a.ntiles * a.G;
+  const uint32_t u0 = g_unit_begin(blockIdx.x, uint32_t(a.U), uint32_t(a.C));
+  const int n = int(g_unit_begin(blockIdx.x + 1, uint32_t(a.U), uint32_t(a.C)) - u0);
+  const uint32_t per_bt = uint32_t(a.ntiles * a.G);
 
   if (warp < DW) {
     // ---------------------------------------------------------------- dequantize
@@ -372,8 +378,11 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     }
   } else if (warp == W_LOAD) {
     // ---------------------------------------------------------------- loads
+    // Lane 0 streams the packed tiles, lane 1 the activation tiles, each
+    // gated only by its own stages, so weight prefetch runs PS units ahead
+    // regardless of MMA progress.
     if (lane == 0) {
-      int issued_p = 0, issued_x = 0;
+      int issued = 0;
       UnitPos pos;
       pos.init(u0, per_bt, a.G);
       for (int i = 0; i < n; ++i, pos.next(a.G, a.ntiles)) {
@@ -386,7 +395,18 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         for (int s = 0; s < vs; ++s)
           bulk_g2s(pst_sa + uint32_t(ps * 4 * TB + s * TB),
                    a.packed + ((pos.tau * 4 + s) * a.G + pos.g) * TB, TB, bar(B_PF + ps));
-        issued_p = i + 1;
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        // let the copies in flight land before the CTA can exit
+        for (int i = (issued > PS ? issued - PS : 0); i < issued; ++i)
+          mbar_drain(bar(B_PF + i % PS), uint32_t(i / PS) & 1u);
+      }
+    } else if (lane == 1) {
+      int issued = 0;
+      UnitPos pos;
+      pos.init(u0, per_bt, a.G);
+      for (int i = 0; i < n; ++i, pos.next(a.G, a.ntiles)) {
         const int xs = i % XS;
         if (!mbar_wait(bar(B_XE + xs), (uint32_t(i / XS) & 1u) ^ 1u, abort_flag, kWaitLimitNs))
           break;
@@ -395,13 +415,10 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         tma_2d_g2s(xd, &tmap_x, int32_t(pos.g * 128), int32_t(pos.bt * kTileRows), bar(B_XF + xs));
         tma_2d_g2s(xd + NT * 128, &tmap_x, int32_t(pos.g * 128 + 64), int32_t(pos.bt * kTileRows),
                    bar(B_XF + xs));
-        issued_x = i + 1;
+        issued = i + 1;
       }
       if (*abort_flag) {
-        // let the copies in flight land before the CTA can exit
-        for (int i = (issued_p > PS ? issued_p - PS : 0); i < issued_p; ++i)
-          mbar_drain(bar(B_PF + i % PS), uint32_t(i / PS) & 1u);
-        for (int i = (issued_x > XS ? issued_x - XS : 0); i < issued_x; ++i)
+        for (int i = (issued > XS ? issued - XS : 0); i < issued; ++i)
           mbar_drain(bar(B_XF + i % XS), uint32_t(i / XS) & 1u);
       }
     }
@@ -540,6 +557,8 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
   a.ntiles = (N + kTileRows - 1) / kTileRows;
   const int64_t bt = (M + kTileRows - 1) / kTileRows;
   a.U = bt * a.ntiles * a.G;
+  // unit indices and range arithmetic are 32-bit (U * CTAs < 2^32)
+  if (a.U * kGemmMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   const int64_t counters = (bt * a.ntiles * 4 * kMaxPromoteGroups * 4 + 255) / 256 * 256;
   a.counters = static_cast<int*>(workspace);
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + counters);

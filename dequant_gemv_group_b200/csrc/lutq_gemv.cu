@@ -60,12 +60,30 @@ struct GemvArgs {
 };
 
 // Part i of `parts` equal shares of [0, total): [range_begin(i), range_begin(i+1)).
-__host__ __device__ inline int64_t range_begin(int64_t i, int64_t total, int64_t parts) {
+// The host guarantees total * parts < 2^32, so 32-bit unsigned arithmetic is
+// exact (integer division is a long instruction sequence; 64-bit even more so).
+__host__ __device__ inline uint32_t range_begin(uint32_t i, uint32_t total, uint32_t parts) {
   return (i * total) / parts;
 }
 // The part holding element u (the last one whose range starts at or before u).
-__host__ __device__ inline int64_t range_owner(int64_t u, int64_t total, int64_t parts) {
+__host__ __device__ inline uint32_t range_owner(uint32_t u, uint32_t total, uint32_t parts) {
   return ((u + 1) * parts - 1) / total;
+}
+
+// Per-CTA table of its warps' unit ranges, filled once in the prologue:
+// warp w holds units [cu0 + wb[w], cu0 + wb[w+1]); first strip ws[w].
+template <int NW>
+struct WarpTable {
+  uint32_t wb[NW + 1];
+  uint32_t ws[NW];
+};
+
+template <int NW>
+__device__ __forceinline__ void fill_warp_table(WarpTable<NW>& t, uint32_t cu0, uint32_t L,
+                                                uint32_t G) {
+  const int i = threadIdx.x;
+  if (i <= NW) t.wb[i] = range_begin(i, L, NW);
+  if (i < NW) t.ws[i] = (cu0 + range_begin(i, L, NW)) / G;
 }
 
 __device__ __forceinline__ uint32_t sm_addr(const void* p) {
@@ -74,21 +92,23 @@ __device__ __forceinline__ uint32_t sm_addr(const void* p) {
 
 // A warp has summed the strip `strip`.  vals[i][m] is the sum of row rows[i]
 // (within the strip) for batch row m, held by the lanes marked `writer`.
-// [u0, u1) is the warp's unit range; slots is its [2][M][32] shared area.
+// [u0, u1) is the warp's unit range, first_strip the strip of u0; slots is
+// its [2][M][32] shared area.
 template <int M, int R>
-__device__ __forceinline__ void deposit_strip(const GemvArgs& a, int64_t strip, int64_t u0,
-                                              int64_t u1, const float (&vals)[R][M],
-                                              const int (&rows)[R], bool writer, float* slots) {
+__device__ __forceinline__ void deposit_strip(const GemvArgs& a, uint32_t strip, uint32_t u0,
+                                              uint32_t u1, uint32_t first_strip,
+                                              const float (&vals)[R][M], const int (&rows)[R],
+                                              bool writer, float* slots) {
   if (!writer) return;
-  const int64_t lo = strip * a.G;
+  const uint32_t lo = strip * uint32_t(a.G);
   if (lo >= u0 && lo + a.G <= u1) {
 #pragma unroll
     for (int i = 0; i < R; ++i)
 #pragma unroll
-      for (int m = 0; m < M; ++m) a.y[m * a.N + lo / a.G * kStrip + rows[i]] = vals[i][m];
+      for (int m = 0; m < M; ++m) a.y[m * a.N + int64_t(strip) * kStrip + rows[i]] = vals[i][m];
     return;
   }
-  const int sl = (strip == u0 / a.G) ? 0 : 1;
+  const int sl = (strip == first_strip) ? 0 : 1;
 #pragma unroll
   for (int i = 0; i < R; ++i)
 #pragma unroll
@@ -98,52 +118,55 @@ __device__ __forceinline__ void deposit_strip(const GemvArgs& a, int64_t strip, 
 // After a block barrier: finish every strip of the CTA's range [cu0, cu1)
 // that no single warp held whole.  all_slots is [NW][2][M][32].
 template <int M, int NW>
-__device__ void cta_finish(const GemvArgs& a, const float* all_slots, int64_t cu0, int64_t cu1) {
+__device__ void cta_finish(const GemvArgs& a, const float* all_slots, const WarpTable<NW>& t,
+                           uint32_t cu0, uint32_t cu1) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t L = cu1 - cu0;
-  const int64_t s_first = cu0 / a.G, s_last = (cu1 - 1) / a.G;
-  for (int64_t strip = s_first + warp; strip <= s_last; strip += NW) {
-    const int64_t lo = strip * a.G, hi = lo + a.G;
-    const int64_t vlo = (lo > cu0 ? lo : cu0) - cu0, vhi = (hi < cu1 ? hi : cu1) - cu0;
-    const int w_lo = int(range_owner(vlo, L, NW)), w_hi = int(range_owner(vhi - 1, L, NW));
-    if (w_lo == w_hi && range_begin(w_lo, L, NW) <= lo - cu0 &&
-        range_begin(w_lo + 1, L, NW) >= hi - cu0)
-      continue;  // written by its warp
+  const uint32_t G = uint32_t(a.G);
+  const uint32_t s_first = t.ws[0];
+  const uint32_t s_last = (cu1 - 1) / G;
+  for (uint32_t strip = s_first + warp; strip <= s_last; strip += NW) {
+    const uint32_t lo = strip * G, hi = lo + G;
     float sum[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) sum[m] = 0.0f;
-    for (int w = w_lo; w <= w_hi; ++w) {
-      const int64_t b = range_begin(w, L, NW), e = range_begin(w + 1, L, NW);
-      if (b == e) continue;  // a warp without units
-      const int sl = (strip == (cu0 + b) / a.G) ? 0 : 1;
+    bool whole = false;
+    for (int w = 0; w < NW; ++w) {
+      const uint32_t b = cu0 + t.wb[w], e = cu0 + t.wb[w + 1];
+      if (b >= e || e <= lo || b >= hi) continue;   // no units of this strip
+      if (b <= lo && e >= hi) {                       // written by its warp
+        whole = true;
+        break;
+      }
+      const int sl = (strip == t.ws[w]) ? 0 : 1;
       const float* src = all_slots + ((w * 2 + sl) * M) * kStrip;
 #pragma unroll
       for (int m = 0; m < M; ++m) sum[m] += src[m * kStrip + lane];
     }
-    float* yrow = a.y + strip * kStrip + lane;
+    if (whole) continue;
+    float* yrow = a.y + int64_t(strip) * kStrip + lane;
     if (lo >= cu0 && hi <= cu1) {
 #pragma unroll
       for (int m = 0; m < M; ++m) yrow[m * a.N] = sum[m];
       continue;
     }
     // shared with other CTAs
+    const uint32_t U = uint32_t(a.U), C = uint32_t(a.C);
     const int slot = (strip == s_first) ? 0 : 1;
     float* mine = a.part + ((int64_t(blockIdx.x) * 2 + slot) * M) * kStrip;
 #pragma unroll
     for (int m = 0; m < M; ++m) mine[m * kStrip + lane] = sum[m];
-    __threadfence();
     __syncwarp();
-    const int64_t c_lo = range_owner(lo, a.U, a.C), c_hi = range_owner(hi - 1, a.U, a.C);
+    const uint32_t c_lo = range_owner(lo, U, C), c_hi = range_owner(hi - 1, U, C);
     int arrived = 0;
-    if (lane == 0) arrived = atomicAdd(a.counters + strip, 1);
+    if (lane == 0) arrived = atom_add_acq_rel_gpu(a.counters + strip, 1);
     arrived = __shfl_sync(0xffffffffu, arrived, 0);
     if (arrived != int(c_hi - c_lo)) continue;
-    __threadfence();
+    __syncwarp();  // the other lanes' loads follow lane 0's acquire
 #pragma unroll
     for (int m = 0; m < M; ++m) sum[m] = 0.0f;
-    for (int64_t c = c_lo; c <= c_hi; ++c) {
-      const int sl = (strip == range_begin(c, a.U, a.C) / a.G) ? 0 : 1;
-      const float* src = a.part + ((c * 2 + sl) * M) * kStrip;
+    for (uint32_t c = c_lo; c <= c_hi; ++c) {
+      const int sl = (strip == range_begin(c, U, C) / G) ? 0 : 1;
+      const float* src = a.part + ((int64_t(c) * 2 + sl) * M) * kStrip;
 #pragma unroll
       for (int m = 0; m < M; ++m) sum[m] += __ldcg(src + m * kStrip + lane);
     }
@@ -290,6 +313,8 @@ template <int BITS, bool XF32>
 __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ uint16_t cbs[16];
+  __shared__ uint32_t pairs[512];
+  __shared__ WarpTable<kM1Warps> wt;
   // The table sits on a 64 KB page of the shared window so that one byte
   // permute produces its full address; activations and warp slots follow.
   const uint32_t sbase = sm_addr(smem);
@@ -297,36 +322,56 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   uint8_t* lut = smem + (lut_sa - sbase);
   uint8_t* xs = lut + kLutBytes;
   float* slots = reinterpret_cast<float*>(xs + (XF32 ? 4 * x_pad_floats(a.K) : 2 * a.K));
+  const uint32_t cu0 = range_begin(blockIdx.x, uint32_t(a.U), uint32_t(a.C));
+  const uint32_t cu1 = range_begin(blockIdx.x + 1, uint32_t(a.U), uint32_t(a.C));
 
   if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
-  {
-    const uint4* xg = reinterpret_cast<const uint4*>(a.x);
-    for (int64_t i = threadIdx.x; i < a.K / 8; i += blockDim.x) {
-      const uint4 v = __ldg(xg + i);
-      if (XF32) {
-        // 8 values k = 8i..8i+7 stay inside one 32-value chunk
-        float4* xd = reinterpret_cast<float4*>(reinterpret_cast<float*>(xs) + x_pad_floats(8 * i));
-        xd[0] = make_float4(bf16_lo_to_f32(v.x), bf16_hi_to_f32(v.x), bf16_lo_to_f32(v.y),
-                            bf16_hi_to_f32(v.y));
-        xd[1] = make_float4(bf16_lo_to_f32(v.z), bf16_hi_to_f32(v.z), bf16_lo_to_f32(v.w),
-                            bf16_hi_to_f32(v.w));
-      } else {
-        reinterpret_cast<uint4*>(xs)[i] = v;
-      }
-    }
+  fill_warp_table<kM1Warps>(wt, cu0, cu1 - cu0, uint32_t(a.G));
+  // Activations: issue every load first, then build the table while they
+  // are in flight, then convert and store them.
+  constexpr int XPT = 8;  // x chunks (8 values) per thread, K <= 8 * XPT * threads
+  uint4 xv[XPT];
+  const int nx = int(a.K / 8);
+#pragma unroll
+  for (int r = 0; r < XPT; ++r) {
+    const int i = threadIdx.x + r * blockDim.x;
+    if (i < nx) xv[r] = __ldg(reinterpret_cast<const uint4*>(a.x) + i);
   }
   __syncthreads();
-  // 16-byte chunk c of the table: row e = c >> 4, half (c >> 3) & 1, 4 lane copies.
-  for (int c = threadIdx.x; c < kLutBytes / 16; c += blockDim.x) {
-    const uint32_t v = lut_entry<BITS>(cbs, c >> 4, (c >> 3) & 1);
-    reinterpret_cast<uint4*>(lut)[c] = make_uint4(v, v, v, v);
+  build_lut_copies<BITS>(lut, cbs, pairs);
+  // chunks beyond the unrolled loads (very long K) take a plain loop
+  for (int i = threadIdx.x + XPT * blockDim.x; i < nx; i += blockDim.x) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x) + i);
+    if (XF32) {
+      float4* xd = reinterpret_cast<float4*>(reinterpret_cast<float*>(xs) + x_pad_floats(8 * i));
+      xd[0] = make_float4(bf16_lo_to_f32(v.x), bf16_hi_to_f32(v.x), bf16_lo_to_f32(v.y),
+                          bf16_hi_to_f32(v.y));
+      xd[1] = make_float4(bf16_lo_to_f32(v.z), bf16_hi_to_f32(v.z), bf16_lo_to_f32(v.w),
+                          bf16_hi_to_f32(v.w));
+    } else {
+      reinterpret_cast<uint4*>(xs)[i] = v;
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < XPT; ++r) {
+    const int i = threadIdx.x + r * blockDim.x;
+    if (i >= nx) break;
+    const uint4 v = xv[r];
+    if (XF32) {
+      // 8 values k = 8i..8i+7 stay inside one 32-value chunk
+      float4* xd = reinterpret_cast<float4*>(reinterpret_cast<float*>(xs) + x_pad_floats(8 * i));
+      xd[0] = make_float4(bf16_lo_to_f32(v.x), bf16_hi_to_f32(v.x), bf16_lo_to_f32(v.y),
+                          bf16_hi_to_f32(v.y));
+      xd[1] = make_float4(bf16_lo_to_f32(v.z), bf16_hi_to_f32(v.z), bf16_lo_to_f32(v.w),
+                          bf16_hi_to_f32(v.w));
+    } else {
+      reinterpret_cast<uint4*>(xs)[i] = v;
+    }
   }
   __syncthreads();
 
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  const int64_t cu0 = range_begin(blockIdx.x, a.U, a.C), cu1 = range_begin(blockIdx.x + 1, a.U, a.C);
-  const int64_t u0 = cu0 + range_begin(wl, cu1 - cu0, kM1Warps);
-  const int64_t u1 = cu0 + range_begin(wl + 1, cu1 - cu0, kM1Warps);
+  const uint32_t u0 = cu0 + wt.wb[wl], u1 = cu0 + wt.wb[wl + 1];
   const int q = lane >> 3, rq = lane & 7;
   const uint32_t page = (lut_sa >> 16) << 8;
   const uint32_t lane_e = page | uint32_t(lane) * 4u, lane_o = page | (128u + uint32_t(lane) * 4u);
@@ -341,10 +386,11 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   if (u0 < u1) {
     // Units are prefetched two ahead into three rotating buffers; `fetch`
     // walks (strip, group) of the next unit to load.
-    int64_t f_strip = u0 / a.G, f_g = u0 - f_strip * a.G;
+    const uint32_t first_strip = wt.ws[wl];
+    int64_t f_strip = first_strip, f_g = int64_t(u0) - int64_t(first_strip) * a.G;
     const int64_t s8 = 8 * a.G;
-    auto load = [&](uint4 (&wd)[4], uint16_t (&sv)[4], int64_t u) {
-      load_unit_m1<BITS>(wd, a.packed + u * TB, lane);
+    auto load = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
+      load_unit_m1<BITS>(wd, a.packed + int64_t(u) * TB, lane);
       const uint16_t* sc = a.scales + (f_strip * kStrip + rq) * a.G + f_g;
 #pragma unroll
       for (int i = 0; i < 4; ++i) sv[i] = __ldg(sc + i * s8);
@@ -356,7 +402,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     int64_t strip = f_strip, g = f_g;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     // consume one unit held in (wd, sv); refill that buffer with unit u + 3
-    auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], int64_t u) {
+    auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
       uint64_t x[16];
       load_x_m1<XF32>(x, xs_sa, g, q);
       uint64_t p[4];
@@ -378,7 +424,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
           vals[i][0] = v;
           acc[i] = 0.0f;
         }
-        deposit_strip<1, 4>(a, strip, u0, u1, vals, rows, q == 0, my_slots);
+        deposit_strip<1, 4>(a, uint32_t(strip), u0, u1, first_strip, vals, rows, q == 0, my_slots);
         ++strip;
         g = 0;
       } else {
@@ -390,7 +436,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     load(b0, s0, u0);
     if (u0 + 1 < u1) load(b1, s1, u0 + 1);
     if (u0 + 2 < u1) load(b2, s2, u0 + 2);
-    for (int64_t u = u0; u < u1; u += 3) {
+    for (uint32_t u = u0; u < u1; u += 3) {
       step(b0, s0, u);
       if (u + 1 >= u1) break;
       step(b1, s1, u + 1);
@@ -399,7 +445,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     }
   }
   __syncthreads();
-  cta_finish<1, kM1Warps>(a, slots, cu0, cu1);
+  cta_finish<1, kM1Warps>(a, slots, wt, cu0, cu1);
 }
 
 // --------------------------------------------------------------------------
@@ -466,35 +512,36 @@ template <int BITS, int M>
 __global__ void __launch_bounds__(kGenWarps * 32, 1) gemv_kernel(GemvArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ uint16_t cbs[16];
+  __shared__ uint32_t pairs[512];
+  __shared__ WarpTable<kGenWarps> wt;
   float* slots = reinterpret_cast<float*>(smem + kLutBytes);  // [NW][2][M][32]
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const uint32_t lut_base = sm_addr(smem);
+  const uint32_t cu0 = range_begin(blockIdx.x, uint32_t(a.U), uint32_t(a.C));
+  const uint32_t cu1 = range_begin(blockIdx.x + 1, uint32_t(a.U), uint32_t(a.C));
   if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
+  fill_warp_table<kGenWarps>(wt, cu0, cu1 - cu0, uint32_t(a.G));
   __syncthreads();
-  for (int c = threadIdx.x; c < kLutBytes / 16; c += blockDim.x) {
-    const uint32_t v = lut_entry<BITS>(cbs, c >> 4, (c >> 3) & 1);
-    reinterpret_cast<uint4*>(smem)[c] = make_uint4(v, v, v, v);
-  }
+  build_lut_copies<BITS>(smem, cbs, pairs);
   __syncthreads();
 
-  const int64_t cu0 = range_begin(blockIdx.x, a.U, a.C), cu1 = range_begin(blockIdx.x + 1, a.U, a.C);
-  const int64_t u0 = cu0 + range_begin(wl, cu1 - cu0, kGenWarps);
-  const int64_t u1 = cu0 + range_begin(wl + 1, cu1 - cu0, kGenWarps);
+  const uint32_t u0 = cu0 + wt.wb[wl], u1 = cu0 + wt.wb[wl + 1];
   const uint32_t off_e = uint32_t(lane) * 4u, off_o = 128u + uint32_t(lane) * 4u;
   constexpr int TB = tile_bytes(BITS);
   const int rows[1] = {lane};
   float* my_slots = slots + wl * 2 * M * kStrip;
 
   if (u0 < u1) {
-    int64_t strip = u0 / a.G;
-    int64_t g = u0 - strip * a.G;
+    const uint32_t first_strip = wt.ws[wl];
+    int64_t strip = first_strip;
+    int64_t g = int64_t(u0) - strip * a.G;
     float acc[1][M];
 #pragma unroll
     for (int m = 0; m < M; ++m) acc[0][m] = 0.0f;
     uint4 cur[4], nxt[4];
-    load_unit_row<BITS>(cur, a.packed + u0 * TB, lane);
-    for (int64_t u = u0; u < u1; ++u) {
-      if (u + 1 < u1) load_unit_row<BITS>(nxt, a.packed + (u + 1) * TB, lane);
+    load_unit_row<BITS>(cur, a.packed + int64_t(u0) * TB, lane);
+    for (uint32_t u = u0; u < u1; ++u) {
+      if (u + 1 < u1) load_unit_row<BITS>(nxt, a.packed + int64_t(u + 1) * TB, lane);
       const int64_t row = strip * kStrip + lane;
       const float s = __uint_as_float(uint32_t(a.scales[row * a.G + g]) << 16);
       float2 part[M];
@@ -504,7 +551,7 @@ __global__ void __launch_bounds__(kGenWarps * 32, 1) gemv_kernel(GemvArgs a) {
 #pragma unroll
       for (int m = 0; m < M; ++m) acc[0][m] = fmaf(s, part[m].x + part[m].y, acc[0][m]);
       if (g == a.G - 1 || u + 1 == u1) {
-        deposit_strip<M, 1>(a, strip, u0, u1, acc, rows, true, my_slots);
+        deposit_strip<M, 1>(a, uint32_t(strip), u0, u1, first_strip, acc, rows, true, my_slots);
 #pragma unroll
         for (int m = 0; m < M; ++m) acc[0][m] = 0.0f;
         ++strip;
@@ -517,7 +564,7 @@ __global__ void __launch_bounds__(kGenWarps * 32, 1) gemv_kernel(GemvArgs a) {
     }
   }
   __syncthreads();
-  cta_finish<M, kGenWarps>(a, slots, cu0, cu1);
+  cta_finish<M, kGenWarps>(a, slots, wt, cu0, cu1);
 }
 
 // --------------------------------------------------------------------------
@@ -620,6 +667,8 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   a.G = K / kGroup;
   a.U = (N / kStrip) * a.G;
   a.C = 0;
+  // unit indices and range arithmetic are 32-bit (U * CTAs < 2^32)
+  if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
                    : launch_bits<3>(a, int(M), num_sms, stream);
 }

@@ -47,6 +47,25 @@ __device__ __forceinline__ void build_lut(uint8_t* lut, const uint16_t* codebook
   }
 }
 
+// Fill the lane-duplicated table at `lut` (needs a preceding barrier after
+// cbs is written; `pairs` is a 512-word scratch area).  The 256 (4-bit) or
+// 512 (3-bit: E and O) distinct pair values are computed once, then copied
+// 32 times with 16-byte stores.  4-bit codes use only the E half of each row.
+template <int BITS>
+__device__ __forceinline__ void build_lut_copies(uint8_t* lut, const uint16_t* cbs,
+                                                 uint32_t* pairs) {
+  constexpr int NV = BITS == 4 ? 256 : 512;
+  for (int v = threadIdx.x; v < NV; v += blockDim.x) pairs[v] = lut_entry<BITS>(cbs, v & 255, v >> 8);
+  __syncthreads();
+  constexpr int HALVES = BITS == 4 ? 1 : 2;
+  // chunk j of row e, half h: 8 chunks of 16 bytes per half
+  for (int c = threadIdx.x; c < 256 * HALVES * 8; c += blockDim.x) {
+    const int e = c / (HALVES * 8), h = (c / 8) % HALVES, j = c & 7;
+    const uint32_t v = pairs[e + 256 * h];
+    reinterpret_cast<uint4*>(lut)[e * 16 + h * 8 + j] = make_uint4(v, v, v, v);
+  }
+}
+
 // (byte `byte` of word) << 8 | lane_off, with lane_off < 256.
 __device__ __forceinline__ uint32_t lut_addr(uint32_t word, uint32_t lane_off, int byte) {
   return __byte_perm(word, lane_off, 0x5504u | (uint32_t(byte) << 4));
