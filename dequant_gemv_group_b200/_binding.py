@@ -41,6 +41,7 @@ _SIGS = {
     "lutq_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32]),
     "lutq_gemv": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "lutq_gemm": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+    "lutq_gemv_noalloc": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -148,6 +149,19 @@ def lutq_gemv(x, packed, scales, codebook, bits, n, k, y=None, workspace=None, s
     """y[M, N] (fp32) for M = 1..16; see lutq_gemv in include/lutq.h."""
     return _product(lib.lutq_gemv, "lutq_gemv", x, packed, scales, codebook, bits, n, k, y,
                     workspace, status)
+
+
+def lutq_gemv_noalloc(x, packed, scales, codebook, bits, n, k, y=None, status=None):
+    """lutq_gemv with the library's fixed scratch array instead of a workspace
+    (for callers that cannot allocate device memory; see include/lutq.h)."""
+    _need(x, torch.bfloat16, "x")
+    m = x.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    _check(lib.lutq_gemv_noalloc(x.data_ptr(), m, packed.data_ptr(), scales.data_ptr(),
+                                 codebook.data_ptr(), bits, n, k, y.data_ptr(), _ptr(status),
+                                 _stream()), "lutq_gemv_noalloc")
+    return y
 
 
 def lutq_gemm(x, packed, scales, codebook, bits, n, k, y=None, workspace=None, status=None):

@@ -23,7 +23,8 @@ COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE
 PER_FILE = {
     "lutq_quantize.cu": ["-fmad=false", "-ftz=false", "-prec-div=true", "-prec-sqrt=true"],
 }
-SOURCES = ["lutq_api.cu", "lutq_quantize.cu", "lutq_pack.cu", "lutq_gemv.cu", "lutq_gemm.cu"]
+SOURCES = ["lutq_api.cu", "lutq_quantize.cu", "lutq_pack.cu", "lutq_gemv.cu", "lutq_gemm.cu",
+           "lutq_noalloc.cu"]
 HOST_SOURCES = ["lutq_codebook.cpp"]
 
 

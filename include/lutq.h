@@ -184,6 +184,33 @@ lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
                       int32_t* dev_status, void* stream);
 
 /*
+ * lutq_gemv_noalloc - lutq_gemv without a caller-provided workspace.
+ *
+ * No counterpart in the paper: this is a calling convention of the library.
+ * It serves callers that cannot allocate device memory where they run the
+ * product: code recording CUDA graphs in a capture mode where cudaMalloc is
+ * illegal, latency-critical loops that must not call cudaMalloc (it can block
+ * and synchronize the device), and plug-in hosts that give a library no
+ * allocator.  The scratch that lutq_gemv takes from `workspace` lives here in
+ * a fixed library-owned device array of 4 MiB, which every GPU that loads the
+ * library holds until the process exits; the call allocates nothing.
+ * Arguments other than the workspace, numerics and results are those of
+ * lutq_gemv (M = 1..16).
+ *  - The first call on a device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls share the array: calls that may overlap on the GPU (other
+ *    streams, other threads) race and must be serialized by the caller.  Each
+ *    call first clears the array's arrival counters (an asynchronous memset
+ *    on `stream`), so a call never depends on what an earlier one left.
+ *  - Returns LUTQ_ERR_WORKSPACE, launching nothing, if the problem's scratch
+ *    (N/8 bytes rounded up to 256, plus 128 KiB per batch row) exceeds 4 MiB.
+ */
+lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const void* packed,
+                              const void* scales_bf16, const void* codebook_bf16,
+                              int bits, int64_t N, int64_t K, float* y,
+                              int32_t* dev_status, void* stream);
+
+/*
  * lutq_gemm - the same product on the tensor cores (tcgen05), for batches
  * where the problem is a dense contraction (tuned for M >= 32; any M >= 1 is
  * accepted).  Arguments and numerics as lutq_gemv.  dev_status receives
