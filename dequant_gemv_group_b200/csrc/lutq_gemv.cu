@@ -324,6 +324,32 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   float* slots = reinterpret_cast<float*>(xs + (XF32 ? 4 * x_pad_floats(a.K) : 2 * a.K));
   const uint32_t cu0 = range_begin(blockIdx.x, uint32_t(a.U), uint32_t(a.C));
   const uint32_t cu1 = range_begin(blockIdx.x + 1, uint32_t(a.U), uint32_t(a.C));
+  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  const uint32_t u0 = cu0 + range_begin(wl, cu1 - cu0, kM1Warps);
+  const uint32_t u1 = cu0 + range_begin(wl + 1, cu1 - cu0, kM1Warps);
+  const uint32_t first_strip = u0 / uint32_t(a.G);
+  const int q = lane >> 3, rq = lane & 7;
+  constexpr int TB = tile_bytes(BITS);
+
+  // The warp's first three units are requested before the prologue so that
+  // their latency overlaps the table build.
+  uint32_t f_strip = first_strip, f_g = u0 - first_strip * uint32_t(a.G);
+  const int64_t s8 = 8 * a.G;
+  auto load = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
+    load_unit_m1<BITS>(wd, a.packed + int64_t(u) * TB, lane);
+    const uint16_t* sc = a.scales + (int64_t(f_strip) * kStrip + rq) * a.G + f_g;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sv[i] = __ldg(sc + i * s8);
+    if (++f_g == uint32_t(a.G)) {
+      f_g = 0;
+      ++f_strip;
+    }
+  };
+  uint4 b0[4], b1[4], b2[4];
+  uint16_t s0[4], s1[4], s2[4];
+  if (u0 < u1) load(b0, s0, u0);
+  if (u0 + 1 < u1) load(b1, s1, u0 + 1);
+  if (u0 + 2 < u1) load(b2, s2, u0 + 2);
 
   if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
   fill_warp_table<kM1Warps>(wt, cu0, cu1 - cu0, uint32_t(a.G));
@@ -370,36 +396,18 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   }
   __syncthreads();
 
-  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  const uint32_t u0 = cu0 + wt.wb[wl], u1 = cu0 + wt.wb[wl + 1];
-  const int q = lane >> 3, rq = lane & 7;
   const uint32_t page = (lut_sa >> 16) << 8;
   const uint32_t lane_e = page | uint32_t(lane) * 4u, lane_o = page | (128u + uint32_t(lane) * 4u);
   const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
   const uint32_t xs_sa = sm_addr(xs);
   float* my_slots = slots + wl * 2 * kStrip;
-  constexpr int TB = tile_bytes(BITS);
   int rows[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) rows[i] = rq + 8 * i;
 
   if (u0 < u1) {
-    // Units are prefetched two ahead into three rotating buffers; `fetch`
-    // walks (strip, group) of the next unit to load.
-    const uint32_t first_strip = wt.ws[wl];
-    int64_t f_strip = first_strip, f_g = int64_t(u0) - int64_t(first_strip) * a.G;
-    const int64_t s8 = 8 * a.G;
-    auto load = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
-      load_unit_m1<BITS>(wd, a.packed + int64_t(u) * TB, lane);
-      const uint16_t* sc = a.scales + (f_strip * kStrip + rq) * a.G + f_g;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sv[i] = __ldg(sc + i * s8);
-      if (++f_g == a.G) {
-        f_g = 0;
-        ++f_strip;
-      }
-    };
-    int64_t strip = f_strip, g = f_g;
+    // Units are prefetched two ahead into three rotating buffers.
+    int64_t strip = first_strip, g = int64_t(u0) - int64_t(first_strip) * a.G;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     // consume one unit held in (wd, sv); refill that buffer with unit u + 3
     auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
@@ -431,11 +439,6 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
         ++g;
       }
     };
-    uint4 b0[4], b1[4], b2[4];
-    uint16_t s0[4], s1[4], s2[4];
-    load(b0, s0, u0);
-    if (u0 + 1 < u1) load(b1, s1, u0 + 1);
-    if (u0 + 2 < u1) load(b2, s2, u0 + 2);
     for (uint32_t u = u0; u < u1; u += 3) {
       step(b0, s0, u);
       if (u + 1 >= u1) break;
@@ -596,6 +599,25 @@ static cudaError_t grant_smem(Kernel k, SmemGrant& g, int smem) {
   return cudaSuccess;
 }
 
+// Number of CTAs.  Equal unit ranges (one CTA per SM) balance the bytes
+// exactly but split strips between CTAs, whose partial sums then meet through
+// global memory at the end (a few microseconds of latency, ~kFixupUnits units
+// of streaming).  When the strips can be dealt out whole to a divisor of the
+// strip count that costs less, no strip is shared and that step disappears.
+constexpr int64_t kFixupUnits = 32;
+
+static int choose_ctas(int64_t strips, int64_t G, int64_t U, int num_sms) {
+  const int64_t cap = std::min<int64_t>(num_sms, kMaxCtas);
+  const int64_t c_split = std::min<int64_t>(cap, U);
+  const int64_t t_split = (U + c_split - 1) / c_split + kFixupUnits;
+  for (int64_t d = 1; d <= strips; ++d) {
+    if (strips % d != 0 || strips / d > cap) continue;
+    const int64_t t_whole = d * G;
+    return int(t_whole <= t_split ? strips / d : c_split);
+  }
+  return int(c_split);
+}
+
 static int m1_smem(int64_t K, bool xf32) {
   // page-alignment slack (< 64 KB) + table + activations + warp slots
   return 2 * kLutBytes + (xf32 ? 4 * x_pad_floats(K) : 2 * int(K)) + kM1Warps * 2 * kStrip * 4;
@@ -607,7 +629,7 @@ static cudaError_t launch_m1(GemvArgs a, int num_sms, cudaStream_t stream) {
   const int smem = m1_smem(a.K, XF32);
   cudaError_t err = grant_smem(gemv_m1_kernel<BITS, XF32>, grant, smem);
   if (err != cudaSuccess) return err;
-  a.C = int(std::min<int64_t>(std::min<int64_t>(num_sms, kMaxCtas), a.U));
+  a.C = choose_ctas(a.N / kStrip, a.G, a.U, num_sms);
   gemv_m1_kernel<BITS, XF32><<<unsigned(a.C), kM1Warps * 32, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -618,7 +640,7 @@ static cudaError_t launch_gen(GemvArgs a, int num_sms, cudaStream_t stream) {
   const int smem = kLutBytes + kGenWarps * 2 * M * kStrip * 4;
   cudaError_t err = grant_smem(gemv_kernel<BITS, M>, grant, smem);
   if (err != cudaSuccess) return err;
-  a.C = int(std::min<int64_t>(std::min<int64_t>(num_sms, kMaxCtas), a.U));
+  a.C = choose_ctas(a.N / kStrip, a.G, a.U, num_sms);
   gemv_kernel<BITS, M><<<unsigned(a.C), kGenWarps * 32, smem, stream>>>(a);
   return cudaGetLastError();
 }
