@@ -428,7 +428,7 @@ def run_lutq(args, world, rank, local):
         "clocks": clocks,
     }
     line.update(extra)
-    if rank == 0 and not args.no_cpu_baseline and world >= 1:
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
         rows = 512
         gbs_cpu, per_call, calls = time_oracle(lay, args.codebook, bits, m, rows, seconds=10.0)
         line["cpu_baseline"] = {

@@ -56,7 +56,7 @@ struct GemmCfg {
   static constexpr int KC = 64 * 4 / DW;            // A columns written per dequant warp
   static constexpr int PG = NT >= 128 ? 2 : 1;      // promotion warp groups
   static constexpr int NC = NT / PG;                // batch columns per promotion warp
-  static constexpr int WARPS = DW + 4 * PG + 2;     // dequant, promote, load, MMA
+  static constexpr int WARPS = DW + 4 * PG + 3;     // dequant, promote, 2 load, MMA
   static constexpr int THREADS = 32 * WARPS;
   static constexpr int DCOL = 64 * AS;              // first partial column
   static_assert(DCOL + DS * NT <= kTmemCols, "tensor memory columns");
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   constexpr int WPR = words_per_row(BITS);
   constexpr int XS = Cfg::XS, PS = Cfg::PS, AS = Cfg::AS, DS = Cfg::DS, DW = Cfg::DW;
   constexpr int PG = Cfg::PG, NC = Cfg::NC;
-  constexpr int W_LOAD = DW + 4 * PG, W_MMA = W_LOAD + 1;
+  constexpr int W_LOAD = DW + 4 * PG, W_XLOAD = W_LOAD + 1, W_MMA = W_LOAD + 2;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_sa = smem_addr(smem_raw);
   const uint32_t base_sa = (raw_sa + 1023u) & ~1023u;
@@ -378,9 +378,10 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     }
   } else if (warp == W_LOAD) {
     // ---------------------------------------------------------------- loads
-    // Lane 0 streams the packed tiles, lane 1 the activation tiles, each
-    // gated only by its own stages, so weight prefetch runs PS units ahead
-    // regardless of MMA progress.
+    // One warp streams the packed tiles and another the activation tiles,
+    // each gated only by its own stages, so weight prefetch runs PS units
+    // ahead regardless of MMA progress (two lanes of one warp would
+    // serialize on each other's waits).
     if (lane == 0) {
       int issued = 0;
       UnitPos pos;
@@ -402,7 +403,9 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         for (int i = (issued > PS ? issued - PS : 0); i < issued; ++i)
           mbar_drain(bar(B_PF + i % PS), uint32_t(i / PS) & 1u);
       }
-    } else if (lane == 1) {
+    }
+  } else if (warp == W_XLOAD) {
+    if (lane == 0) {
       int issued = 0;
       UnitPos pos;
       pos.init(u0, per_bt, a.G);
