@@ -68,22 +68,26 @@ def algorithmic_bytes(m, n, k, bits):
     return packed + n * (k // 128) * 2 + m * k * 2 + m * n * 4
 
 
-def kernel_source_sha():
+GEMV_SOURCES = ("lutq_common.cuh", "lutq_lut.cuh", "lutq_gemv.cu")
+GEMM_SOURCES = ("lutq_common.cuh", "lutq_lut.cuh", "lutq_sm100.cuh", "lutq_gemm.cu")
+
+
+def kernel_source_sha(files):
     src = os.path.join(ROOT, "dequant_gemv_group_b200", "csrc")
     h = hashlib.sha256()
-    for f in ("lutq_common.cuh", "lutq_gemv.cu"):
+    for f in files:
         h.update(open(os.path.join(src, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key):
+def ncu_traffic(kernel_key, files):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    the current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     d = json.load(open(path)).get(kernel_key)
-    if not d or d.get("source_sha") != kernel_source_sha():
+    if not d or d.get("source_sha") != kernel_source_sha(files):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -195,11 +199,11 @@ def run_reference(args, world, rank):
         return
     lay = workloads.layer(args.workload, args.layer)
     m = args.batch
-    # rows per step sized so that warm-up + timed steps take about a minute
-    # (the oracle's product costs roughly 40 us per row of this layer per batch row)
+    # rows per step sized so that warm-up + timed steps take about a minute:
+    # the cost of one row is calibrated on a 64-row sample first
+    _, per_call, _ = time_oracle(lay, args.codebook, args.bits, m, 64, calls=3)
     per_step = 60.0 / max(1, args.steps + args.warmup)
-    rows = int(per_step / (40e-6 * m * lay.k / 14336)) // 32 * 32
-    rows = max(32, min(lay.n, rows))
+    rows = max(1, min(lay.n, int(per_step / (per_call / 64))))
     O, x, codes, sb, levels = oracle_sample(lay, args.codebook, args.bits, m, rows)
     for _ in range(args.warmup):
         O.gemv(x, codes, sb, levels)
@@ -281,7 +285,8 @@ def side_measurements(lq, dev, args):
                    "us": s * 1e6, "hbm_gbs": nbytes / s / 1e9,
                    "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_peak,
                                 "unit": "TFLOP/s", "frac": tflops / tf_peak,
-                                "peak_source": peak_kind + " (bf16 burst)"},
+                                "peak_source": peak_kind + " (bf16 burst)",
+                                "traffic": ncu_traffic(f"gemm_w4_m{m}_{n}x{k}", GEMM_SOURCES)},
                    "kernel": "lutq::gemm_kernel"}
     del packed, scales, x, y, ws
     # offline steps on the headline layer
@@ -417,7 +422,8 @@ def run_lutq(args, world, rank, local):
                           f"({copies * per_copy / 1e6:.0f} MB > 3x L2 {l2 / 1e6:.0f} MB)"),
         "roofline": {"bound": "hbm", "achieved": gbs_rank, "peak": hbm_peak, "unit": "GB/s",
                      "frac": gbs_rank / hbm_peak, "peak_source": peak_kind,
-                     "bytes_per_launch": nbytes, "traffic": ncu_traffic(kernel_key),
+                     "bytes_per_launch": nbytes, "traffic": ncu_traffic(kernel_key,
+                                                                    GEMM_SOURCES if use_gemm else GEMV_SOURCES),
                      "kernel": "lutq::gemv_kernel" if not use_gemm else "lutq::gemm_kernel"},
         "pct_of_8TBs": gbs_rank / 8000.0,
         "plain_launch_gbs": plain_gbs,
