@@ -199,9 +199,19 @@ __device__ __forceinline__ void pair_fma(uint64_t& acc, uint32_t lv, uint64_t x)
       : "+l"(acc) : "r"(lv), "l"(x));
 }
 
+// acc = lv * x (the first pair of a chain; no zeroed accumulator needed).
+__device__ __forceinline__ void pair_mul(uint64_t& acc, uint32_t lv, uint64_t x) {
+  asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 w;\n\t"
+      "shl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xffff0000;\n\t"
+      "mov.b64 w, {lo, hi};\n\tmul.rn.f32x2 %0, w, %2;\n\t}"
+      : "=l"(acc) : "r"(lv), "l"(x));
+}
+
 // The four rows' u32 index words idx[i] (four pair indices each) against the
 // four activation pairs x[0..3]; the rows are interleaved so that four
-// independent table loads and accumulator chains are in flight.
+// independent table loads and accumulator chains are in flight.  FIRST starts
+// the chains (p[i] is not read).
+template <bool FIRST>
 __device__ __forceinline__ void quad4(uint64_t (&p)[4], const uint32_t (&idx)[4],
                                       uint32_t lane_hi, const uint64_t* x) {
 #pragma unroll
@@ -213,28 +223,43 @@ __device__ __forceinline__ void quad4(uint64_t (&p)[4], const uint32_t (&idx)[4]
       // page (bits 23:16) come from lane_hi
       lv[i] = lds32(__byte_perm(idx[i], lane_hi, 0x6504u | (uint32_t(b) << 4)));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) pair_fma(p[i], lv[i], x[b]);
+    for (int i = 0; i < 4; ++i) {
+      if (FIRST && b == 0)
+        pair_mul(p[i], lv[i], x[b]);
+      else
+        pair_fma(p[i], lv[i], x[b]);
+    }
   }
 }
 
-// Per lane and unit: 4 rows x 32 codes.  wd[i] holds row i's 16 bytes for the
-// lane (4-bit: one word; 3-bit: 8 lo-plane bytes then 8 hi-plane bytes).
+// Byte offset, inside a tile, of the lane's packed bytes of row rq; rows
+// rq + 8 i follow at +128 i.  4-bit: word q.  3-bit: u32 pair 2 (q & 1) of lo
+// word q >> 1 (its hi-plane bytes are lane_hi_delta(q) further on).
 template <int BITS>
-__device__ __forceinline__ void load_unit_m1(uint4 (&wd)[4], const uint8_t* tile, int lane) {
-  const int q = lane >> 3, rq = lane & 7;
+__device__ __forceinline__ uint32_t lane_tile_offset(int q, int rq) {
+  return BITS == 4 ? uint32_t((32 * q + rq) * kWordBytes)
+                   : uint32_t((32 * (q >> 1) + rq) * kWordBytes + 8 * (q & 1));
+}
+__device__ __forceinline__ uint32_t lane_hi_delta(int q) {
+  return uint32_t((64 - 32 * (q >> 1)) * kWordBytes);
+}
+
+// Per lane and unit: 4 rows x 32 codes.  wd[i] holds row i's 16 bytes for the
+// lane (4-bit: one word; 3-bit: 8 lo-plane bytes then 8 hi-plane bytes); p is
+// the lane's bytes in the tile (lane_tile_offset).
+template <int BITS>
+__device__ __forceinline__ void load_unit_m1(uint4 (&wd)[4], const uint8_t* p,
+                                             uint32_t hi_delta) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = rq + 8 * i;
     if (BITS == 4) {
-      wd[i] = ld_stream_v4(tile + (32 * q + r) * kWordBytes);
+      wd[i] = ld_stream_v4(p + 128 * i);
     } else {
-      // lo word q >> 1, u32 2(q&1) and 2(q&1)+1; the hi word's u32 with the same index
-      const uint8_t* lo = tile + (32 * (q >> 1) + r) * kWordBytes + 8 * (q & 1);
-      const uint8_t* hi = tile + (64 + r) * kWordBytes + 8 * (q & 1);
       uint32_t l0, l1, h0, h1;
       asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
-                   : "=r"(l0), "=r"(l1) : "l"(lo));
-      asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(h0), "=r"(h1) : "l"(hi));
+                   : "=r"(l0), "=r"(l1) : "l"(p + 128 * i));
+      asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];"
+                   : "=r"(h0), "=r"(h1) : "l"(p + hi_delta + 128 * i));
       wd[i] = make_uint4(l0, l1, h0, h1);
     }
   }
@@ -245,24 +270,22 @@ template <int BITS>
 __device__ __forceinline__ void unit_partial_m1(uint64_t (&p)[4], const uint4 (&wd)[4],
                                                 uint32_t lane_e, uint32_t lane_o,
                                                 uint32_t hi_shift, const uint64_t (&x)[16]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) p[i] = 0;
   if (BITS == 4) {
     {
       const uint32_t idx[4] = {wd[0].x, wd[1].x, wd[2].x, wd[3].x};
-      quad4(p, idx, lane_e, x + 0);
+      quad4<true>(p, idx, lane_e, x + 0);
     }
     {
       const uint32_t idx[4] = {wd[0].y, wd[1].y, wd[2].y, wd[3].y};
-      quad4(p, idx, lane_e, x + 4);
+      quad4<false>(p, idx, lane_e, x + 4);
     }
     {
       const uint32_t idx[4] = {wd[0].z, wd[1].z, wd[2].z, wd[3].z};
-      quad4(p, idx, lane_e, x + 8);
+      quad4<false>(p, idx, lane_e, x + 8);
     }
     {
       const uint32_t idx[4] = {wd[0].w, wd[1].w, wd[2].w, wd[3].w};
-      quad4(p, idx, lane_e, x + 12);
+      quad4<false>(p, idx, lane_e, x + 12);
     }
   } else {
     // lo u32 j goes with hi u32 j; lo word 1 reads its hi fields two bits up
@@ -276,8 +299,11 @@ __device__ __forceinline__ void unit_partial_m1(uint64_t (&p)[4], const uint4 (&
         e[i] = (l & 0x0F0F0F0Fu) | (h & 0xF0F0F0F0u);
         o[i] = (l & 0xF0F0F0F0u) | (h & 0x0F0F0F0Fu);
       }
-      quad4(p, e, lane_e, x + 8 * j);
-      quad4(p, o, lane_o, x + 8 * j + 4);
+      if (j == 0)
+        quad4<true>(p, e, lane_e, x + 0);
+      else
+        quad4<false>(p, e, lane_e, x + 8);
+      quad4<false>(p, o, lane_o, x + 8 * j + 4);
     }
   }
 }
@@ -286,17 +312,21 @@ __device__ __forceinline__ void unit_partial_m1(uint64_t (&p)[4], const uint4 (&
 // padding after every 32 (so the four k-chunks of a group that the lanes of a
 // row read fall in different banks); otherwise bf16, widened when loaded.
 __host__ __device__ constexpr int x_pad_floats(int64_t k) { return int(k + k / 32 * 4); }
-
+// Shared-memory bytes per group and lane offset of chunk q.
 template <bool XF32>
-__device__ __forceinline__ void load_x_m1(uint64_t (&x)[16], uint32_t xs_sa, int64_t g, int q) {
+__host__ __device__ constexpr uint32_t x_group_bytes() { return XF32 ? 576u : 256u; }
+template <bool XF32>
+__host__ __device__ constexpr uint32_t x_chunk_bytes() { return XF32 ? 144u : 64u; }
+
+// The lane's 32 activations of one group, as 16 fp32 pairs, from address xa.
+template <bool XF32>
+__device__ __forceinline__ void load_x_m1(uint64_t (&x)[16], uint32_t xa) {
   if (XF32) {
-    const uint32_t xa = xs_sa + uint32_t(x_pad_floats(g * kGroup + 32 * q)) * 4u;
 #pragma unroll
     for (int v = 0; v < 8; ++v)
       asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
                    : "=l"(x[2 * v]), "=l"(x[2 * v + 1]) : "r"(xa + 16u * v));
   } else {
-    const uint32_t xa = xs_sa + uint32_t(g * kGroup + 32 * q) * 2u;
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       uint32_t r[4];
@@ -309,11 +339,24 @@ __device__ __forceinline__ void load_x_m1(uint64_t (&x)[16], uint32_t xs_sa, int
   }
 }
 
+// Activations: bf16 global -> shared (fp32 padded or bf16), 8 values per chunk.
+template <bool XF32>
+__device__ __forceinline__ void store_x_chunk(uint8_t* xs, int i, uint4 v) {
+  if (XF32) {
+    // values k = 8i..8i+7 stay inside one 32-value chunk
+    float4* xd = reinterpret_cast<float4*>(reinterpret_cast<float*>(xs) + x_pad_floats(8 * i));
+    xd[0] = make_float4(bf16_lo_to_f32(v.x), bf16_hi_to_f32(v.x), bf16_lo_to_f32(v.y),
+                        bf16_hi_to_f32(v.y));
+    xd[1] = make_float4(bf16_lo_to_f32(v.z), bf16_hi_to_f32(v.z), bf16_lo_to_f32(v.w),
+                        bf16_hi_to_f32(v.w));
+  } else {
+    reinterpret_cast<uint4*>(xs)[i] = v;
+  }
+}
+
 template <int BITS, bool XF32>
 __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ uint16_t cbs[16];
-  __shared__ uint32_t pairs[512];
   __shared__ WarpTable<kM1Warps> wt;
   // The table sits on a 64 KB page of the shared window so that one byte
   // permute produces its full address; activations and warp slots follow.
@@ -322,40 +365,51 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   uint8_t* lut = smem + (lut_sa - sbase);
   uint8_t* xs = lut + kLutBytes;
   float* slots = reinterpret_cast<float*>(xs + (XF32 ? 4 * x_pad_floats(a.K) : 2 * a.K));
+  const uint32_t G = uint32_t(a.G);
   const uint32_t cu0 = range_begin(blockIdx.x, uint32_t(a.U), uint32_t(a.C));
   const uint32_t cu1 = range_begin(blockIdx.x + 1, uint32_t(a.U), uint32_t(a.C));
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const uint32_t u0 = cu0 + range_begin(wl, cu1 - cu0, kM1Warps);
   const uint32_t u1 = cu0 + range_begin(wl + 1, cu1 - cu0, kM1Warps);
-  const uint32_t first_strip = u0 / uint32_t(a.G);
+  const uint32_t first_strip = u0 / G;
+  const uint32_t g_first = u0 - first_strip * G;
   const int q = lane >> 3, rq = lane & 7;
   constexpr int TB = tile_bytes(BITS);
 
-  // The warp's first three units are requested before the prologue so that
-  // their latency overlaps the table build.
-  uint32_t f_strip = first_strip, f_g = u0 - first_strip * uint32_t(a.G);
-  const int64_t s8 = 8 * a.G;
-  auto load = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
-    load_unit_m1<BITS>(wd, a.packed + int64_t(u) * TB, lane);
-    const uint16_t* sc = a.scales + (int64_t(f_strip) * kStrip + rq) * a.G + f_g;
+  // Fetch cursor: the lane's bytes of the next tile to load, the scale of
+  // its row rq for that tile's group (rows rq + 8 i are 16 G bytes apart),
+  // and that group.  Tiles are loaded in order u0, u0 + 1, ...
+  const uint32_t hi_delta = BITS == 3 ? lane_hi_delta(q) : 0u;
+  const uint8_t* fw = a.packed + uint64_t(u0) * TB + lane_tile_offset<BITS>(q, rq);
+  const uint16_t* fs = a.scales + (uint64_t(first_strip) * kStrip + rq) * G + g_first;
+  uint32_t fg = g_first;
+  const uint32_t s8b = 16u * G;
+  const uint32_t s_wrap = 31u * G + 1u;  // last group of row r -> group 0 of row r, next strip
+  auto fetch = [&](uint4 (&wd)[4], uint16_t (&sv)[4]) {
+    load_unit_m1<BITS>(wd, fw, hi_delta);
+    const uint8_t* sb = reinterpret_cast<const uint8_t*>(fs);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sv[i] = __ldg(sc + i * s8);
-    if (++f_g == uint32_t(a.G)) {
-      f_g = 0;
-      ++f_strip;
-    }
+    for (int i = 0; i < 4; ++i) sv[i] = __ldg(reinterpret_cast<const uint16_t*>(sb + i * s8b));
+    fw += TB;
+    const bool wrap = fg + 1 == G;
+    fs += wrap ? s_wrap : 1u;
+    fg = wrap ? 0u : fg + 1u;
   };
+
+  // The warp's first three tiles are requested before the prologue so that
+  // their latency overlaps the table build.
   uint4 b0[4], b1[4], b2[4];
   uint16_t s0[4], s1[4], s2[4];
-  if (u0 < u1) load(b0, s0, u0);
-  if (u0 + 1 < u1) load(b1, s1, u0 + 1);
-  if (u0 + 2 < u1) load(b2, s2, u0 + 2);
+  if (u0 < u1) fetch(b0, s0);
+  if (u0 + 1 < u1) fetch(b1, s1);
+  if (u0 + 2 < u1) fetch(b2, s2);
 
-  if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
-  fill_warp_table<kM1Warps>(wt, cu0, cu1 - cu0, uint32_t(a.G));
-  // Activations: issue every load first, then build the table while they
-  // are in flight, then convert and store them.
-  constexpr int XPT = 8;  // x chunks (8 values) per thread, K <= 8 * XPT * threads
+  // Lane t holds codebook[t mod 2^BITS]; the table is built from it with
+  // shuffles, so no shared staging (and no barrier) precedes the build.
+  const uint32_t cbv = __ldg(a.codebook + (lane & ((1 << BITS) - 1)));
+  // Activations: issue every load first, build the table while they are in
+  // flight, then convert and store them.
+  constexpr int XPT = 8;  // x chunks (8 values) per thread held in registers
   uint4 xv[XPT];
   const int nx = int(a.K / 8);
 #pragma unroll
@@ -363,56 +417,36 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     const int i = threadIdx.x + r * blockDim.x;
     if (i < nx) xv[r] = __ldg(reinterpret_cast<const uint4*>(a.x) + i);
   }
-  __syncthreads();
-  build_lut_copies<BITS>(lut, cbs, pairs);
-  // chunks beyond the unrolled loads (very long K) take a plain loop
-  for (int i = threadIdx.x + XPT * blockDim.x; i < nx; i += blockDim.x) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x) + i);
-    if (XF32) {
-      float4* xd = reinterpret_cast<float4*>(reinterpret_cast<float*>(xs) + x_pad_floats(8 * i));
-      xd[0] = make_float4(bf16_lo_to_f32(v.x), bf16_hi_to_f32(v.x), bf16_lo_to_f32(v.y),
-                          bf16_hi_to_f32(v.y));
-      xd[1] = make_float4(bf16_lo_to_f32(v.z), bf16_hi_to_f32(v.z), bf16_lo_to_f32(v.w),
-                          bf16_hi_to_f32(v.w));
-    } else {
-      reinterpret_cast<uint4*>(xs)[i] = v;
-    }
-  }
+  fill_warp_table<kM1Warps>(wt, cu0, cu1 - cu0, G);
+  build_lut_shfl<BITS>(lut, cbv);
+  // chunks beyond the ones held in registers (very long K) take a plain loop
+  for (int i = threadIdx.x + XPT * blockDim.x; i < nx; i += blockDim.x)
+    store_x_chunk<XF32>(xs, i, __ldg(reinterpret_cast<const uint4*>(a.x) + i));
 #pragma unroll
   for (int r = 0; r < XPT; ++r) {
     const int i = threadIdx.x + r * blockDim.x;
-    if (i >= nx) break;
-    const uint4 v = xv[r];
-    if (XF32) {
-      // 8 values k = 8i..8i+7 stay inside one 32-value chunk
-      float4* xd = reinterpret_cast<float4*>(reinterpret_cast<float*>(xs) + x_pad_floats(8 * i));
-      xd[0] = make_float4(bf16_lo_to_f32(v.x), bf16_hi_to_f32(v.x), bf16_lo_to_f32(v.y),
-                          bf16_hi_to_f32(v.y));
-      xd[1] = make_float4(bf16_lo_to_f32(v.z), bf16_hi_to_f32(v.z), bf16_lo_to_f32(v.w),
-                          bf16_hi_to_f32(v.w));
-    } else {
-      reinterpret_cast<uint4*>(xs)[i] = v;
-    }
+    if (i < nx) store_x_chunk<XF32>(xs, i, xv[r]);
   }
   __syncthreads();
 
   const uint32_t page = (lut_sa >> 16) << 8;
   const uint32_t lane_e = page | uint32_t(lane) * 4u, lane_o = page | (128u + uint32_t(lane) * 4u);
   const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
-  const uint32_t xs_sa = sm_addr(xs);
+  const uint32_t xa0 = sm_addr(xs) + uint32_t(q) * x_chunk_bytes<XF32>();
   float* my_slots = slots + wl * 2 * kStrip;
   int rows[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) rows[i] = rq + 8 * i;
 
   if (u0 < u1) {
-    // Units are prefetched two ahead into three rotating buffers.
-    int64_t strip = first_strip, g = int64_t(u0) - int64_t(first_strip) * a.G;
+    // Tiles are prefetched two ahead into three rotating buffers.
+    uint32_t strip = first_strip, g = g_first;
+    uint32_t xa = xa0 + g_first * x_group_bytes<XF32>();
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    // consume one unit held in (wd, sv); refill that buffer with unit u + 3
+    // consume the tile u held in (wd, sv); refill that buffer with tile u + 3
     auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
       uint64_t x[16];
-      load_x_m1<XF32>(x, xs_sa, g, q);
+      load_x_m1<XF32>(x, xa);
       uint64_t p[4];
       unit_partial_m1<BITS>(p, wd, lane_e, lane_o, hi_shift, x);
 #pragma unroll
@@ -421,8 +455,8 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
         const float v = __uint_as_float(uint32_t(p[i])) + __uint_as_float(uint32_t(p[i] >> 32));
         acc[i] = fmaf(s, v, acc[i]);
       }
-      if (u + 3 < u1) load(wd, sv, u + 3);
-      if (g == a.G - 1 || u + 1 == u1) {
+      if (u + 3 < u1) fetch(wd, sv);
+      if (g + 1 == G || u + 1 == u1) {
         float vals[4][1];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -432,11 +466,13 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
           vals[i][0] = v;
           acc[i] = 0.0f;
         }
-        deposit_strip<1, 4>(a, uint32_t(strip), u0, u1, first_strip, vals, rows, q == 0, my_slots);
+        deposit_strip<1, 4>(a, strip, u0, u1, first_strip, vals, rows, q == 0, my_slots);
         ++strip;
         g = 0;
+        xa = xa0;
       } else {
         ++g;
+        xa += x_group_bytes<XF32>();
       }
     };
     for (uint32_t u = u0; u < u1; u += 3) {

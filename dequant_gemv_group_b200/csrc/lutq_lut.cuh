@@ -66,6 +66,37 @@ __device__ __forceinline__ void build_lut_copies(uint8_t* lut, const uint16_t* c
   }
 }
 
+// Fill the lane-duplicated table from a codebook held in registers: lane t of
+// every warp passes cbv = codebook[t mod 2^BITS], and each pair value is
+// assembled with two shuffles, so no shared staging or barrier comes before
+// the build (callers synchronize after it).  Thread i writes the 16-byte
+// chunks i, i + blockDim.x, ...; blockDim.x is a multiple of 32, so all lanes
+// of a warp take the same number of turns, as the shuffles require.
+template <int BITS>
+__device__ __forceinline__ void build_lut_shfl(uint8_t* lut, uint32_t cbv) {
+  constexpr int HALVES = BITS == 4 ? 1 : 2;
+  constexpr int CHUNKS = 256 * HALVES * 8;  // 8 chunks of 16 bytes per half row
+  static_assert(CHUNKS % 32 == 0, "whole warps");
+  for (int c = threadIdx.x; c < CHUNKS; c += blockDim.x) {
+    const int e = c / (HALVES * 8), h = (c / 8) % HALVES;
+    uint32_t qe, qo;
+    if (BITS == 4) {
+      qe = e & 15;
+      qo = e >> 4;
+    } else if (h == 0) {
+      qe = (e & 3) | (((e >> 4) & 1) << 2);
+      qo = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
+    } else {
+      qe = ((e >> 4) & 3) | ((e & 1) << 2);
+      qo = ((e >> 6) & 3) | (((e >> 1) & 1) << 2);
+    }
+    const uint32_t ve = __shfl_sync(0xffffffffu, cbv, int(qe));
+    const uint32_t vo = __shfl_sync(0xffffffffu, cbv, int(qo));
+    const uint32_t v = (ve & 0xffffu) | (vo << 16);
+    reinterpret_cast<uint4*>(lut)[e * 16 + h * 8 + (c & 7)] = make_uint4(v, v, v, v);
+  }
+}
+
 // (byte `byte` of word) << 8 | lane_off, with lane_off < 256.
 __device__ __forceinline__ uint32_t lut_addr(uint32_t word, uint32_t lane_off, int byte) {
   return __byte_perm(word, lane_off, 0x5504u | (uint32_t(byte) << 4));
