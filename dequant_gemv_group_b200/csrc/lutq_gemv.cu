@@ -22,11 +22,12 @@
 // M = 1 kernel.  Lane t of a warp owns the k-chunk q = t >> 3 (32 codes,
 // k = 128 g + 32 q ..) of the four rows (t & 7) + 8 i, i = 0..3, of the
 // strip (the 8 lanes of a quarter-warp share q, so activation reads are
-// broadcasts).  Its 32 activations stay in registers (fp32) and serve four rows;
-// each code pair costs one byte permute (forming the table address), one
-// conflict-free shared load, two bit operations (bf16 pair -> fp32 pair) and
-// one packed fp32x2 fused multiply-add.  The four lanes of a row add their
-// sums at the end of the strip.
+// broadcasts).  Its 32 activations stay in registers (bf16 pairs) and serve
+// four rows; each code pair costs one byte permute (forming the table
+// address), one conflict-free shared load and two fused multiply-adds with
+// bf16 multiplicands and fp32 accumulators (a bf16 x bf16 product is exact in
+// fp32, so this is the fp32 product of the widened values).  The four lanes
+// of a row add their sums at the end of the strip.
 //
 // M = 2..16 kernel.  Lane r owns row 32 * strip + r and reads its 16-byte
 // words with coalesced 512-byte warp loads; activations come from global
@@ -129,18 +130,19 @@ __device__ void cta_finish(const GemvArgs& a, const float* all_slots, const Warp
     float sum[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) sum[m] = 0.0f;
+    // Unrolled over the warps, so that the slot reads do not wait on one
+    // another; the sum still runs in warp order.  A strip held whole by one
+    // warp has no other contributor (the warps' ranges are disjoint).
     bool whole = false;
+#pragma unroll
     for (int w = 0; w < NW; ++w) {
       const uint32_t b = cu0 + t.wb[w], e = cu0 + t.wb[w + 1];
-      if (b >= e || e <= lo || b >= hi) continue;   // no units of this strip
-      if (b <= lo && e >= hi) {                       // written by its warp
-        whole = true;
-        break;
-      }
+      const bool some = b < e && e > lo && b < hi;   // has units of this strip
+      whole |= some && b <= lo && e >= hi;           // ... all of them
       const int sl = (strip == t.ws[w]) ? 0 : 1;
       const float* src = all_slots + ((w * 2 + sl) * M) * kStrip;
 #pragma unroll
-      for (int m = 0; m < M; ++m) sum[m] += src[m * kStrip + lane];
+      for (int m = 0; m < M; ++m) sum[m] += some ? src[m * kStrip + lane] : 0.0f;
     }
     if (whole) continue;
     float* yrow = a.y + int64_t(strip) * kStrip + lane;
@@ -190,30 +192,24 @@ __device__ __forceinline__ void ffma2(float2& acc, float lo, float hi, float x0,
 // M = 1
 // --------------------------------------------------------------------------
 
-// acc (fp32x2 in one 64-bit register) += bf16 code pair lv (low half = even
-// k) * activation pair x (fp32x2, low half = even k).
-__device__ __forceinline__ void pair_fma(uint64_t& acc, uint32_t lv, uint64_t x) {
-  asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 w;\n\t"
-      "shl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xffff0000;\n\t"
-      "mov.b64 w, {lo, hi};\n\tfma.rn.f32x2 %0, w, %2, %0;\n\t}"
-      : "+l"(acc) : "r"(lv), "l"(x));
+// ae += c_even * x_even and ao += c_odd * x_odd, with lv = (c_even, c_odd) and
+// xw = (x_even, x_odd) bf16x2 words (low half = even k): two fused
+// multiply-adds with bf16 multiplicands and an fp32 addend.  The product of
+// two bf16 values is exact in fp32, so each step rounds once, exactly as an
+// fp32 fma on the widened operands would; no instruction widens anything.
+__device__ __forceinline__ void pair_fma(float& ae, float& ao, uint32_t lv, uint32_t xw) {
+  asm("{\n\t.reg .b16 c0, c1, x0, x1;\n\t"
+      "mov.b32 {c0, c1}, %2;\n\tmov.b32 {x0, x1}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, c0, x0, %0;\n\tfma.rn.f32.bf16 %1, c1, x1, %1;\n\t}"
+      : "+f"(ae), "+f"(ao) : "r"(lv), "r"(xw));
 }
 
-// acc = lv * x (the first pair of a chain; no zeroed accumulator needed).
-__device__ __forceinline__ void pair_mul(uint64_t& acc, uint32_t lv, uint64_t x) {
-  asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 w;\n\t"
-      "shl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xffff0000;\n\t"
-      "mov.b64 w, {lo, hi};\n\tmul.rn.f32x2 %0, w, %2;\n\t}"
-      : "=l"(acc) : "r"(lv), "l"(x));
-}
-
-// The four rows' u32 index words idx[i] (four pair indices each) against the
-// four activation pairs x[0..3]; the rows are interleaved so that four
-// independent table loads and accumulator chains are in flight.  FIRST starts
-// the chains (p[i] is not read).
-template <bool FIRST>
-__device__ __forceinline__ void quad4(uint64_t (&p)[4], const uint32_t (&idx)[4],
-                                      uint32_t lane_hi, const uint64_t* x) {
+// Row sums of one unit, split by k parity: se[i] (even k) and so[i] (odd k)
+// of row i.  The four rows' u32 index words idx[i] (four pair indices each)
+// go against the four activation words xw[0..3]; the rows are interleaved so
+// that four independent table loads and accumulator chains are in flight.
+__device__ __forceinline__ void quad4(float (&se)[4], float (&so)[4], const uint32_t (&idx)[4],
+                                      uint32_t lane_hi, const uint32_t* xw) {
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     uint32_t lv[4];
@@ -223,12 +219,7 @@ __device__ __forceinline__ void quad4(uint64_t (&p)[4], const uint32_t (&idx)[4]
       // page (bits 23:16) come from lane_hi
       lv[i] = lds32(__byte_perm(idx[i], lane_hi, 0x6504u | (uint32_t(b) << 4)));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (FIRST && b == 0)
-        pair_mul(p[i], lv[i], x[b]);
-      else
-        pair_fma(p[i], lv[i], x[b]);
-    }
+    for (int i = 0; i < 4; ++i) pair_fma(se[i], so[i], lv[i], xw[b]);
   }
 }
 
@@ -265,27 +256,30 @@ __device__ __forceinline__ void load_unit_m1(uint4 (&wd)[4], const uint8_t* p,
   }
 }
 
-// Partial sums of the four rows of one unit: p[i] (fp32x2) for row i.
+// Row sums of one unit for the lane's four rows, split by k parity.
 template <int BITS>
-__device__ __forceinline__ void unit_partial_m1(uint64_t (&p)[4], const uint4 (&wd)[4],
-                                                uint32_t lane_e, uint32_t lane_o,
-                                                uint32_t hi_shift, const uint64_t (&x)[16]) {
+__device__ __forceinline__ void unit_partial_m1(float (&se)[4], float (&so)[4],
+                                                const uint4 (&wd)[4], uint32_t lane_e,
+                                                uint32_t lane_o, uint32_t hi_shift,
+                                                const uint32_t (&xw)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) se[i] = so[i] = 0.0f;
   if (BITS == 4) {
     {
       const uint32_t idx[4] = {wd[0].x, wd[1].x, wd[2].x, wd[3].x};
-      quad4<true>(p, idx, lane_e, x + 0);
+      quad4(se, so, idx, lane_e, xw + 0);
     }
     {
       const uint32_t idx[4] = {wd[0].y, wd[1].y, wd[2].y, wd[3].y};
-      quad4<false>(p, idx, lane_e, x + 4);
+      quad4(se, so, idx, lane_e, xw + 4);
     }
     {
       const uint32_t idx[4] = {wd[0].z, wd[1].z, wd[2].z, wd[3].z};
-      quad4<false>(p, idx, lane_e, x + 8);
+      quad4(se, so, idx, lane_e, xw + 8);
     }
     {
       const uint32_t idx[4] = {wd[0].w, wd[1].w, wd[2].w, wd[3].w};
-      quad4<false>(p, idx, lane_e, x + 12);
+      quad4(se, so, idx, lane_e, xw + 12);
     }
   } else {
     // lo u32 j goes with hi u32 j; lo word 1 reads its hi fields two bits up
@@ -299,62 +293,34 @@ __device__ __forceinline__ void unit_partial_m1(uint64_t (&p)[4], const uint4 (&
         e[i] = (l & 0x0F0F0F0Fu) | (h & 0xF0F0F0F0u);
         o[i] = (l & 0xF0F0F0F0u) | (h & 0x0F0F0F0Fu);
       }
-      if (j == 0)
-        quad4<true>(p, e, lane_e, x + 0);
-      else
-        quad4<false>(p, e, lane_e, x + 8);
-      quad4<false>(p, o, lane_o, x + 8 * j + 4);
+      quad4(se, so, e, lane_e, xw + 8 * j);
+      quad4(se, so, o, lane_o, xw + 8 * j + 4);
     }
   }
 }
 
-// Activations in shared memory: XF32 keeps fp32 values with 16 bytes of
-// padding after every 32 (so the four k-chunks of a group that the lanes of a
-// row read fall in different banks); otherwise bf16, widened when loaded.
-__host__ __device__ constexpr int x_pad_floats(int64_t k) { return int(k + k / 32 * 4); }
-// Shared-memory bytes per group and lane offset of chunk q.
-template <bool XF32>
-__host__ __device__ constexpr uint32_t x_group_bytes() { return XF32 ? 576u : 256u; }
-template <bool XF32>
-__host__ __device__ constexpr uint32_t x_chunk_bytes() { return XF32 ? 144u : 64u; }
+// Activations in shared memory stay bf16, in chunks of 32 values (64 bytes)
+// followed by 16 bytes of padding, so that the four chunks of a group that
+// the quarter-warps read at once fall in different banks.
+constexpr uint32_t kXChunkBytes = 80;
+constexpr uint32_t kXGroupBytes = 4 * kXChunkBytes;
+__host__ __device__ constexpr int64_t x_smem_bytes(int64_t k) { return k / 32 * kXChunkBytes; }
 
-// The lane's 32 activations of one group, as 16 fp32 pairs, from address xa.
-template <bool XF32>
-__device__ __forceinline__ void load_x_m1(uint64_t (&x)[16], uint32_t xa) {
-  if (XF32) {
+// The lane's 32 activations of one group (16 bf16x2 words) from address xa.
+__device__ __forceinline__ void load_x_m1(uint32_t (&xw)[16], uint32_t xa) {
 #pragma unroll
-    for (int v = 0; v < 8; ++v)
-      asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];"
-                   : "=l"(x[2 * v]), "=l"(x[2 * v + 1]) : "r"(xa + 16u * v));
-  } else {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      uint32_t r[4];
-      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(xa + 16u * v));
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-        x[4 * v + t] = uint64_t(r[t] << 16) | (uint64_t(r[t] & 0xffff0000u) << 32);
-    }
-  }
+  for (int v = 0; v < 4; ++v)
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(xw[4 * v]), "=r"(xw[4 * v + 1]), "=r"(xw[4 * v + 2]), "=r"(xw[4 * v + 3])
+                 : "r"(xa + 16u * v));
 }
 
-// Activations: bf16 global -> shared (fp32 padded or bf16), 8 values per chunk.
-template <bool XF32>
+// Activation chunk i (8 bf16 values, k = 8 i ..) into the padded layout.
 __device__ __forceinline__ void store_x_chunk(uint8_t* xs, int i, uint4 v) {
-  if (XF32) {
-    // values k = 8i..8i+7 stay inside one 32-value chunk
-    float4* xd = reinterpret_cast<float4*>(reinterpret_cast<float*>(xs) + x_pad_floats(8 * i));
-    xd[0] = make_float4(bf16_lo_to_f32(v.x), bf16_hi_to_f32(v.x), bf16_lo_to_f32(v.y),
-                        bf16_hi_to_f32(v.y));
-    xd[1] = make_float4(bf16_lo_to_f32(v.z), bf16_hi_to_f32(v.z), bf16_lo_to_f32(v.w),
-                        bf16_hi_to_f32(v.w));
-  } else {
-    reinterpret_cast<uint4*>(xs)[i] = v;
-  }
+  *reinterpret_cast<uint4*>(xs + (i >> 2) * kXChunkBytes + (i & 3) * 16) = v;
 }
 
-template <int BITS, bool XF32>
+template <int BITS>
 __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ WarpTable<kM1Warps> wt;
@@ -364,7 +330,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   const uint32_t lut_sa = (sbase + 0xFFFFu) & ~0xFFFFu;
   uint8_t* lut = smem + (lut_sa - sbase);
   uint8_t* xs = lut + kLutBytes;
-  float* slots = reinterpret_cast<float*>(xs + (XF32 ? 4 * x_pad_floats(a.K) : 2 * a.K));
+  float* slots = reinterpret_cast<float*>(xs + x_smem_bytes(a.K));
   const uint32_t G = uint32_t(a.G);
   const uint32_t cu0 = range_begin(blockIdx.x, uint32_t(a.U), uint32_t(a.C));
   const uint32_t cu1 = range_begin(blockIdx.x + 1, uint32_t(a.U), uint32_t(a.C));
@@ -396,19 +362,11 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     fg = wrap ? 0u : fg + 1u;
   };
 
-  // The warp's first three tiles are requested before the prologue so that
-  // their latency overlaps the table build.
-  uint4 b0[4], b1[4], b2[4];
-  uint16_t s0[4], s1[4], s2[4];
-  if (u0 < u1) fetch(b0, s0);
-  if (u0 + 1 < u1) fetch(b1, s1);
-  if (u0 + 2 < u1) fetch(b2, s2);
-
   // Lane t holds codebook[t mod 2^BITS]; the table is built from it with
   // shuffles, so no shared staging (and no barrier) precedes the build.
   const uint32_t cbv = __ldg(a.codebook + (lane & ((1 << BITS) - 1)));
   // Activations: issue every load first, build the table while they are in
-  // flight, then convert and store them.
+  // flight, then store them.
   constexpr int XPT = 8;  // x chunks (8 values) per thread held in registers
   uint4 xv[XPT];
   const int nx = int(a.K / 8);
@@ -421,18 +379,29 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   build_lut_shfl<BITS>(lut, cbv);
   // chunks beyond the ones held in registers (very long K) take a plain loop
   for (int i = threadIdx.x + XPT * blockDim.x; i < nx; i += blockDim.x)
-    store_x_chunk<XF32>(xs, i, __ldg(reinterpret_cast<const uint4*>(a.x) + i));
+    store_x_chunk(xs, i, __ldg(reinterpret_cast<const uint4*>(a.x) + i));
 #pragma unroll
   for (int r = 0; r < XPT; ++r) {
     const int i = threadIdx.x + r * blockDim.x;
-    if (i < nx) store_x_chunk<XF32>(xs, i, xv[r]);
+    if (i < nx) store_x_chunk(xs, i, xv[r]);
   }
+  // Only now, with the codebook and the activations in, are the warp's first
+  // three tiles requested: issued earlier, the weight stream would fill the
+  // memory pipeline ahead of those small loads and hold up the prologue.  The
+  // tiles arrive while the block waits at the barrier.
+  asm volatile("" ::: "memory");
+  __syncwarp();
+  uint4 b0[4], b1[4], b2[4];
+  uint16_t s0[4], s1[4], s2[4];
+  if (u0 < u1) fetch(b0, s0);
+  if (u0 + 1 < u1) fetch(b1, s1);
+  if (u0 + 2 < u1) fetch(b2, s2);
   __syncthreads();
 
   const uint32_t page = (lut_sa >> 16) << 8;
   const uint32_t lane_e = page | uint32_t(lane) * 4u, lane_o = page | (128u + uint32_t(lane) * 4u);
   const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
-  const uint32_t xa0 = sm_addr(xs) + uint32_t(q) * x_chunk_bytes<XF32>();
+  const uint32_t xa0 = sm_addr(xs) + uint32_t(q) * kXChunkBytes;
   float* my_slots = slots + wl * 2 * kStrip;
   int rows[4];
 #pragma unroll
@@ -441,19 +410,18 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   if (u0 < u1) {
     // Tiles are prefetched two ahead into three rotating buffers.
     uint32_t strip = first_strip, g = g_first;
-    uint32_t xa = xa0 + g_first * x_group_bytes<XF32>();
+    uint32_t xa = xa0 + g_first * kXGroupBytes;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     // consume the tile u held in (wd, sv); refill that buffer with tile u + 3
     auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
-      uint64_t x[16];
-      load_x_m1<XF32>(x, xa);
-      uint64_t p[4];
-      unit_partial_m1<BITS>(p, wd, lane_e, lane_o, hi_shift, x);
+      uint32_t xw[16];
+      load_x_m1(xw, xa);
+      float se[4], so[4];
+      unit_partial_m1<BITS>(se, so, wd, lane_e, lane_o, hi_shift, xw);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float s = __uint_as_float(uint32_t(sv[i]) << 16);
-        const float v = __uint_as_float(uint32_t(p[i])) + __uint_as_float(uint32_t(p[i] >> 32));
-        acc[i] = fmaf(s, v, acc[i]);
+        acc[i] = fmaf(s, se[i] + so[i], acc[i]);
       }
       if (u + 3 < u1) fetch(wd, sv);
       if (g + 1 == G || u + 1 == u1) {
@@ -472,7 +440,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
         xa = xa0;
       } else {
         ++g;
-        xa += x_group_bytes<XF32>();
+        xa += kXGroupBytes;
       }
     };
     for (uint32_t u = u0; u < u1; u += 3) {
@@ -654,19 +622,19 @@ static int choose_ctas(int64_t strips, int64_t G, int64_t U, int num_sms) {
   return int(c_split);
 }
 
-static int m1_smem(int64_t K, bool xf32) {
+static int64_t m1_smem(int64_t K) {
   // page-alignment slack (< 64 KB) + table + activations + warp slots
-  return 2 * kLutBytes + (xf32 ? 4 * x_pad_floats(K) : 2 * int(K)) + kM1Warps * 2 * kStrip * 4;
+  return 2 * kLutBytes + x_smem_bytes(K) + kM1Warps * 2 * kStrip * 4;
 }
 
-template <int BITS, bool XF32>
+template <int BITS>
 static cudaError_t launch_m1(GemvArgs a, int num_sms, cudaStream_t stream) {
   static SmemGrant grant;
-  const int smem = m1_smem(a.K, XF32);
-  cudaError_t err = grant_smem(gemv_m1_kernel<BITS, XF32>, grant, smem);
+  const int smem = int(m1_smem(a.K));
+  cudaError_t err = grant_smem(gemv_m1_kernel<BITS>, grant, smem);
   if (err != cudaSuccess) return err;
   a.C = choose_ctas(a.N / kStrip, a.G, a.U, num_sms);
-  gemv_m1_kernel<BITS, XF32><<<unsigned(a.C), kM1Warps * 32, smem, stream>>>(a);
+  gemv_m1_kernel<BITS><<<unsigned(a.C), kM1Warps * 32, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -686,8 +654,7 @@ static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream
   switch (M) {
     case 1:
       // the M = 1 kernel keeps all of x in shared memory next to the table
-      if (m1_smem(a.K, true) <= kMaxSmemPerBlock) return launch_m1<BITS, true>(a, num_sms, s);
-      if (m1_smem(a.K, false) <= kMaxSmemPerBlock) return launch_m1<BITS, false>(a, num_sms, s);
+      if (m1_smem(a.K) <= kMaxSmemPerBlock) return launch_m1<BITS>(a, num_sms, s);
       return launch_gen<BITS, 1>(a, num_sms, s);
     case 2: return launch_gen<BITS, 2>(a, num_sms, s);
     case 3: return launch_gen<BITS, 3>(a, num_sms, s);
