@@ -204,10 +204,21 @@ __device__ __forceinline__ void pair_fma(float& ae, float& ao, uint32_t lv, uint
       : "+f"(ae), "+f"(ao) : "r"(lv), "r"(xw));
 }
 
+// The same with a zero addend: se = c_even * x_even, so = c_odd * x_odd (the
+// first pair of a chain; no zeroed accumulator needs setting up).
+__device__ __forceinline__ void pair_first(float& ae, float& ao, uint32_t lv, uint32_t xw) {
+  asm("{\n\t.reg .b16 c0, c1, x0, x1;\n\t"
+      "mov.b32 {c0, c1}, %2;\n\tmov.b32 {x0, x1}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, c0, x0, 0f00000000;\n\tfma.rn.f32.bf16 %1, c1, x1, 0f00000000;\n\t}"
+      : "=f"(ae), "=f"(ao) : "r"(lv), "r"(xw));
+}
+
 // Row sums of one unit, split by k parity: se[i] (even k) and so[i] (odd k)
 // of row i.  The four rows' u32 index words idx[i] (four pair indices each)
 // go against the four activation words xw[0..3]; the rows are interleaved so
 // that four independent table loads and accumulator chains are in flight.
+// FIRST starts the chains (se, so are not read).
+template <bool FIRST>
 __device__ __forceinline__ void quad4(float (&se)[4], float (&so)[4], const uint32_t (&idx)[4],
                                       uint32_t lane_hi, const uint32_t* xw) {
 #pragma unroll
@@ -219,7 +230,12 @@ __device__ __forceinline__ void quad4(float (&se)[4], float (&so)[4], const uint
       // page (bits 23:16) come from lane_hi
       lv[i] = lds32(__byte_perm(idx[i], lane_hi, 0x6504u | (uint32_t(b) << 4)));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) pair_fma(se[i], so[i], lv[i], xw[b]);
+    for (int i = 0; i < 4; ++i) {
+      if (FIRST && b == 0)
+        pair_first(se[i], so[i], lv[i], xw[b]);
+      else
+        pair_fma(se[i], so[i], lv[i], xw[b]);
+    }
   }
 }
 
@@ -262,24 +278,22 @@ __device__ __forceinline__ void unit_partial_m1(float (&se)[4], float (&so)[4],
                                                 const uint4 (&wd)[4], uint32_t lane_e,
                                                 uint32_t lane_o, uint32_t hi_shift,
                                                 const uint32_t (&xw)[16]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) se[i] = so[i] = 0.0f;
   if (BITS == 4) {
     {
       const uint32_t idx[4] = {wd[0].x, wd[1].x, wd[2].x, wd[3].x};
-      quad4(se, so, idx, lane_e, xw + 0);
+      quad4<true>(se, so, idx, lane_e, xw + 0);
     }
     {
       const uint32_t idx[4] = {wd[0].y, wd[1].y, wd[2].y, wd[3].y};
-      quad4(se, so, idx, lane_e, xw + 4);
+      quad4<false>(se, so, idx, lane_e, xw + 4);
     }
     {
       const uint32_t idx[4] = {wd[0].z, wd[1].z, wd[2].z, wd[3].z};
-      quad4(se, so, idx, lane_e, xw + 8);
+      quad4<false>(se, so, idx, lane_e, xw + 8);
     }
     {
       const uint32_t idx[4] = {wd[0].w, wd[1].w, wd[2].w, wd[3].w};
-      quad4(se, so, idx, lane_e, xw + 12);
+      quad4<false>(se, so, idx, lane_e, xw + 12);
     }
   } else {
     // lo u32 j goes with hi u32 j; lo word 1 reads its hi fields two bits up
@@ -293,8 +307,11 @@ __device__ __forceinline__ void unit_partial_m1(float (&se)[4], float (&so)[4],
         e[i] = (l & 0x0F0F0F0Fu) | (h & 0xF0F0F0F0u);
         o[i] = (l & 0xF0F0F0F0u) | (h & 0x0F0F0F0Fu);
       }
-      quad4(se, so, e, lane_e, xw + 8 * j);
-      quad4(se, so, o, lane_o, xw + 8 * j + 4);
+      if (j == 0)
+        quad4<true>(se, so, e, lane_e, xw);
+      else
+        quad4<false>(se, so, e, lane_e, xw + 8);
+      quad4<false>(se, so, o, lane_o, xw + 8 * j + 4);
     }
   }
 }
@@ -375,6 +392,11 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     const int i = threadIdx.x + r * blockDim.x;
     if (i < nx) xv[r] = __ldg(reinterpret_cast<const uint4*>(a.x) + i);
   }
+  // The first tile follows right behind those loads: one 2 KB tile per warp
+  // does not crowd them out, and its latency overlaps theirs.
+  uint4 b0[4], b1[4], b2[4];
+  uint16_t s0[4], s1[4], s2[4];
+  if (u0 < u1) fetch(b0, s0);
   fill_warp_table<kM1Warps>(wt, cu0, cu1 - cu0, G);
   build_lut_shfl<BITS>(lut, cbv);
   // chunks beyond the ones held in registers (very long K) take a plain loop
@@ -385,15 +407,11 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     const int i = threadIdx.x + r * blockDim.x;
     if (i < nx) store_x_chunk(xs, i, xv[r]);
   }
-  // Only now, with the codebook and the activations in, are the warp's first
-  // three tiles requested: issued earlier, the weight stream would fill the
-  // memory pipeline ahead of those small loads and hold up the prologue.  The
-  // tiles arrive while the block waits at the barrier.
+  // Only now, with the codebook and the activations in, are the next two
+  // tiles requested: issued earlier, the weight stream would fill the memory
+  // pipeline ahead of those small loads and hold up the prologue.
   asm volatile("" ::: "memory");
   __syncwarp();
-  uint4 b0[4], b1[4], b2[4];
-  uint16_t s0[4], s1[4], s2[4];
-  if (u0 < u1) fetch(b0, s0);
   if (u0 + 1 < u1) fetch(b1, s1);
   if (u0 + 2 < u1) fetch(b2, s2);
   __syncthreads();
