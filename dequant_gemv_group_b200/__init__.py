@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     lutq_gemm,
     lutq_gemv,
     lutq_gemv_noalloc,
+    lutq_gemv_plan,
     lutq_layout_version,
     lutq_pack,
     lutq_packed_bytes,

@@ -42,6 +42,7 @@ _SIGS = {
     "lutq_gemv": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "lutq_gemm": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "lutq_gemv_noalloc": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
+    "lutq_gemv_plan": (_i32, [_i64, _i64, _i32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -82,6 +83,13 @@ def lutq_packed_bytes(n: int, k: int, bits: int) -> int:
 
 def lutq_workspace_bytes(m: int, n: int, k: int, bits: int) -> int:
     return lib.lutq_workspace_bytes(m, n, k, bits)
+
+
+def lutq_gemv_plan(n: int, k: int, num_sms: int) -> dict:
+    """How lutq_gemv divides an n x k problem among thread blocks (host only)."""
+    out = (ctypes.c_int32 * 6)()
+    _check(lib.lutq_gemv_plan(n, k, num_sms, out), "lutq_gemv_plan")
+    return dict(zip(("C", "kind", "align", "Cm", "T", "nh"), list(out)))
 
 
 def lutq_codebook(kind: str, bits: int) -> torch.Tensor:

@@ -20,6 +20,7 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
                         const void* codebook, int bits, int64_t N, int64_t K, float* y,
                         void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
 int64_t gemv_workspace_bytes(int64_t M, int64_t N);
+void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out);
 int64_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 }  // namespace lutq
 
@@ -130,6 +131,14 @@ lutq_status lutq_pack(const uint8_t* codes, int64_t N, int64_t K, int bits, void
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_pack(codes, N, K, bits, packed, dev_status, sms,
                                      static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan) {
+  if (plan == nullptr || num_sms < 1) return LUTQ_ERR_INVALID_ARG;
+  lutq_status st;
+  if ((st = check_shape(N, K)) != LUTQ_OK) return st;
+  lutq::gemv_plan(N, K, num_sms, plan);
+  return LUTQ_OK;
 }
 
 int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {

@@ -6,17 +6,20 @@
 //
 // Work split (both kernels).  The packed matrix is a sequence of
 // U = (N/32) * G units, one unit = (strip of 32 rows, group of 128 codes) =
-// 2048 (4-bit) or 1536 (3-bit) contiguous bytes.  CTA c of a persistent grid
-// of C CTAs takes units [floor(c U / C), floor((c+1) U / C)); warp w of its NW
-// warps takes an equal share of that range, so every warp streams the same
-// number of bytes.  Sums are reduced in two deterministic levels:
+// 2048 (4-bit) or 1536 (3-bit) contiguous bytes.  A plan (choose_plan) gives
+// each CTA of a grid of at most one CTA per SM a run of units: whole strips,
+// an equal share of the unit sequence, or (for few, deep strips) the first or
+// the last groups of strips; warp w of its NW warps takes an equal share of
+// that run, so every warp streams the same number of bytes.  Sums are reduced
+// in deterministic steps:
 //  - a strip held whole by one warp is written by that warp;
 //  - otherwise each warp leaves its partial row sums of the strips at the two
-//    ends of its range in shared memory, and after a block barrier one warp
-//    per strip adds them in warp order;
-//  - a strip shared with other CTAs is finished by the last CTA to arrive
-//    (one atomic per contributor), which adds the CTAs' partials in CTA order
-//    and resets the strip's counter to zero for the next call.
+//    ends of its run in shared memory, and after a block barrier one warp per
+//    strip adds them in warp order;
+//  - a strip that the plan splits between two CTAs (never more) is finished
+//    by whichever of the two arrives second, through one 64-bit atomic
+//    exchange per row (exchange_half); a sum of two commutes, so the result
+//    does not depend on which.
 // Results therefore do not depend on timing.
 //
 // M = 1 kernel.  Lane t of a warp owns the k-chunk q = t >> 3 (32 codes,
@@ -54,10 +57,13 @@ struct GemvArgs {
   const uint16_t* scales;   // bf16 [N, G]
   const uint16_t* codebook; // bf16 [2^bits]
   float* y;                 // fp32 [M, N]
-  float* part;              // [kMaxCtas][2][M][32]: CTA partials of strips shared between CTAs
-  int* counters;            // [N/32] arrival counters (zero between calls)
+  unsigned long long* xch;  // [M][N] exchange slots of strips split between two CTAs (zero between calls)
   int64_t N, K, G, U;       // U = number of units
   int C;                    // CTAs
+  // work plan (choose_plan): kind 0 = ranges of the unit sequence, strip-
+  // aligned if `align`; kind 1 = the first Cm CTAs take groups [0, G - T) of
+  // one strip each, the others groups [G - T, G) of nh strips each
+  uint32_t kind, align, Cm, T, nh;
 };
 
 // Part i of `parts` equal shares of [0, total): [range_begin(i), range_begin(i+1)).
@@ -66,13 +72,48 @@ struct GemvArgs {
 __host__ __device__ inline uint32_t range_begin(uint32_t i, uint32_t total, uint32_t parts) {
   return (i * total) / parts;
 }
-// The part holding element u (the last one whose range starts at or before u).
-__host__ __device__ inline uint32_t range_owner(uint32_t u, uint32_t total, uint32_t parts) {
-  return ((u + 1) * parts - 1) / total;
+
+// The units of one CTA, in the order it takes them: strips s0, s0 + 1, ...,
+// each contributing its W groups ga .. ga + W - 1; the CTA takes positions
+// [v0, v1) of that sequence, position v being unit (s0 + v / W, ga + v % W).
+// Every plan leaves a strip either whole in one CTA (only when W = G) or
+// split between exactly two CTAs.
+struct Span {
+  uint32_t s0, ga, W, v0, v1;
+};
+
+__device__ __forceinline__ Span cta_span(const GemvArgs& a, uint32_t c) {
+  Span p;
+  const uint32_t G = uint32_t(a.G), S = uint32_t(a.N / kStrip), C = uint32_t(a.C);
+  if (a.kind == 0) {
+    p.s0 = 0;
+    p.ga = 0;
+    p.W = G;
+    if (a.align) {
+      p.v0 = G * range_begin(c, S, C);
+      p.v1 = G * range_begin(c + 1, S, C);
+    } else {
+      p.v0 = range_begin(c, uint32_t(a.U), C);
+      p.v1 = range_begin(c + 1, uint32_t(a.U), C);
+    }
+  } else if (c < a.Cm) {
+    p.s0 = c;
+    p.ga = 0;
+    p.W = G - a.T;
+    p.v0 = 0;
+    p.v1 = p.W;
+  } else {
+    p.s0 = (c - a.Cm) * a.nh;
+    p.ga = G - a.T;
+    p.W = a.T;
+    p.v0 = 0;
+    p.v1 = p.s0 < S ? (S - p.s0 < a.nh ? S - p.s0 : a.nh) * a.T : 0u;
+  }
+  return p;
 }
 
-// Per-CTA table of its warps' unit ranges, filled once in the prologue:
-// warp w holds units [cu0 + wb[w], cu0 + wb[w+1]); first strip ws[w].
+// Per-CTA table of its warps' position ranges, filled once in the prologue:
+// warp w holds positions [v0 + wb[w], v0 + wb[w+1]); its first strip is ws[w].
 template <int NW>
 struct WarpTable {
   uint32_t wb[NW + 1];
@@ -80,29 +121,30 @@ struct WarpTable {
 };
 
 template <int NW>
-__device__ __forceinline__ void fill_warp_table(WarpTable<NW>& t, uint32_t cu0, uint32_t L,
-                                                uint32_t G) {
+__device__ __forceinline__ void fill_warp_table(WarpTable<NW>& t, const Span& p) {
   const int i = threadIdx.x;
+  const uint32_t L = p.v1 - p.v0;
   if (i <= NW) t.wb[i] = range_begin(i, L, NW);
-  if (i < NW) t.ws[i] = (cu0 + range_begin(i, L, NW)) / G;
+  if (i < NW) t.ws[i] = p.s0 + (p.v0 + range_begin(i, L, NW)) / p.W;
 }
 
 __device__ __forceinline__ uint32_t sm_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// A warp has summed the strip `strip`.  vals[i][m] is the sum of row rows[i]
-// (within the strip) for batch row m, held by the lanes marked `writer`.
-// [u0, u1) is the warp's unit range, first_strip the strip of u0; slots is
-// its [2][M][32] shared area.
+// A warp has summed its units of strip `strip`.  vals[i][m] is the sum of
+// row rows[i] (within the strip) for batch row m, held by the lanes marked
+// `writer`.  [w0, w1) are the warp's positions, first_strip the strip of w0;
+// slots is its [2][M][32] shared area.  A strip held whole by the warp (which
+// needs W = G) is written out; otherwise the sums wait in the slots.
 template <int M, int R>
-__device__ __forceinline__ void deposit_strip(const GemvArgs& a, uint32_t strip, uint32_t u0,
-                                              uint32_t u1, uint32_t first_strip,
+__device__ __forceinline__ void deposit_strip(const GemvArgs& a, const Span& p, uint32_t strip,
+                                              uint32_t w0, uint32_t w1, uint32_t first_strip,
                                               const float (&vals)[R][M], const int (&rows)[R],
                                               bool writer, float* slots) {
   if (!writer) return;
-  const uint32_t lo = strip * uint32_t(a.G);
-  if (lo >= u0 && lo + a.G <= u1) {
+  const uint32_t lo = (strip - p.s0) * p.W;
+  if (p.W == uint32_t(a.G) && lo >= w0 && lo + p.W <= w1) {
 #pragma unroll
     for (int i = 0; i < R; ++i)
 #pragma unroll
@@ -116,17 +158,34 @@ __device__ __forceinline__ void deposit_strip(const GemvArgs& a, uint32_t strip,
     for (int m = 0; m < M; ++m) slots[(sl * M + m) * kStrip + rows[i]] = vals[i][m];
 }
 
-// After a block barrier: finish every strip of the CTA's range [cu0, cu1)
-// that no single warp held whole.  all_slots is [NW][2][M][32].
+// One of the two halves of a split row value meets the other: the first to
+// arrive leaves its value (tagged in the high word) in the slot; the second
+// takes it, writes the sum and clears the slot for the next call.  Both
+// orders give the same fp32 sum (addition of two values commutes), so the
+// result does not depend on timing.
+__device__ __forceinline__ void exchange_half(unsigned long long* slot, float v, float* y) {
+  const unsigned long long mine = (1ull << 32) | __float_as_uint(v);
+  const unsigned long long other = atomicExch(slot, mine);
+  if (other != 0ull) {
+    *y = v + __uint_as_float(uint32_t(other));
+    *slot = 0ull;
+  }
+}
+
+// After a block barrier: finish every strip of the CTA's span that no single
+// warp wrote out.  all_slots is [NW][2][M][32].  One warp per strip adds the
+// warps' sums in warp order; a strip whole in this CTA is written, a strip
+// split with the other CTA goes through exchange_half.
 template <int M, int NW>
-__device__ void cta_finish(const GemvArgs& a, const float* all_slots, const WarpTable<NW>& t,
-                           uint32_t cu0, uint32_t cu1) {
+__device__ void cta_finish(const GemvArgs& a, const Span& p, const float* all_slots,
+                           const WarpTable<NW>& t) {
+  if (p.v0 >= p.v1) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t G = uint32_t(a.G);
+  const bool full = p.W == uint32_t(a.G);
   const uint32_t s_first = t.ws[0];
-  const uint32_t s_last = (cu1 - 1) / G;
+  const uint32_t s_last = p.s0 + (p.v1 - 1) / p.W;
   for (uint32_t strip = s_first + warp; strip <= s_last; strip += NW) {
-    const uint32_t lo = strip * G, hi = lo + G;
+    const uint32_t lo = (strip - p.s0) * p.W, hi = lo + p.W;
     float sum[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) sum[m] = 0.0f;
@@ -136,7 +195,7 @@ __device__ void cta_finish(const GemvArgs& a, const float* all_slots, const Warp
     bool whole = false;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      const uint32_t b = cu0 + t.wb[w], e = cu0 + t.wb[w + 1];
+      const uint32_t b = p.v0 + t.wb[w], e = p.v0 + t.wb[w + 1];
       const bool some = b < e && e > lo && b < hi;   // has units of this strip
       whole |= some && b <= lo && e >= hi;           // ... all of them
       const int sl = (strip == t.ws[w]) ? 0 : 1;
@@ -144,37 +203,16 @@ __device__ void cta_finish(const GemvArgs& a, const float* all_slots, const Warp
 #pragma unroll
       for (int m = 0; m < M; ++m) sum[m] += some ? src[m * kStrip + lane] : 0.0f;
     }
-    if (whole) continue;
+    if (full && whole) continue;  // written by its warp
     float* yrow = a.y + int64_t(strip) * kStrip + lane;
-    if (lo >= cu0 && hi <= cu1) {
+    if (full && lo >= p.v0 && hi <= p.v1) {
 #pragma unroll
       for (int m = 0; m < M; ++m) yrow[m * a.N] = sum[m];
       continue;
     }
-    // shared with other CTAs
-    const uint32_t U = uint32_t(a.U), C = uint32_t(a.C);
-    const int slot = (strip == s_first) ? 0 : 1;
-    float* mine = a.part + ((int64_t(blockIdx.x) * 2 + slot) * M) * kStrip;
+    unsigned long long* xrow = a.xch + int64_t(strip) * kStrip + lane;
 #pragma unroll
-    for (int m = 0; m < M; ++m) mine[m * kStrip + lane] = sum[m];
-    __syncwarp();
-    const uint32_t c_lo = range_owner(lo, U, C), c_hi = range_owner(hi - 1, U, C);
-    int arrived = 0;
-    if (lane == 0) arrived = atom_add_acq_rel_gpu(a.counters + strip, 1);
-    arrived = __shfl_sync(0xffffffffu, arrived, 0);
-    if (arrived != int(c_hi - c_lo)) continue;
-    __syncwarp();  // the other lanes' loads follow lane 0's acquire
-#pragma unroll
-    for (int m = 0; m < M; ++m) sum[m] = 0.0f;
-    for (uint32_t c = c_lo; c <= c_hi; ++c) {
-      const int sl = (strip == range_begin(c, U, C) / G) ? 0 : 1;
-      const float* src = a.part + ((int64_t(c) * 2 + sl) * M) * kStrip;
-#pragma unroll
-      for (int m = 0; m < M; ++m) sum[m] += __ldcg(src + m * kStrip + lane);
-    }
-#pragma unroll
-    for (int m = 0; m < M; ++m) yrow[m * a.N] = sum[m];
-    if (lane == 0) a.counters[strip] = 0;
+    for (int m = 0; m < M; ++m) exchange_half(xrow + m * a.N, sum[m], yrow + m * a.N);
   }
 }
 
@@ -349,32 +387,37 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   uint8_t* xs = lut + kLutBytes;
   float* slots = reinterpret_cast<float*>(xs + x_smem_bytes(a.K));
   const uint32_t G = uint32_t(a.G);
-  const uint32_t cu0 = range_begin(blockIdx.x, uint32_t(a.U), uint32_t(a.C));
-  const uint32_t cu1 = range_begin(blockIdx.x + 1, uint32_t(a.U), uint32_t(a.C));
+  const Span sp = cta_span(a, blockIdx.x);
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  const uint32_t u0 = cu0 + range_begin(wl, cu1 - cu0, kM1Warps);
-  const uint32_t u1 = cu0 + range_begin(wl + 1, cu1 - cu0, kM1Warps);
-  const uint32_t first_strip = u0 / G;
-  const uint32_t g_first = u0 - first_strip * G;
+  // the warp's positions [u0, u1) of the CTA's unit sequence
+  const uint32_t u0 = sp.v0 + range_begin(wl, sp.v1 - sp.v0, kM1Warps);
+  const uint32_t u1 = sp.v0 + range_begin(wl + 1, sp.v1 - sp.v0, kM1Warps);
+  const uint32_t first_strip = sp.s0 + u0 / sp.W;
+  const uint32_t g_first = u0 % sp.W;  // within the window: group sp.ga + g_first
   const int q = lane >> 3, rq = lane & 7;
   constexpr int TB = tile_bytes(BITS);
 
   // Fetch cursor: the lane's bytes of the next tile to load, the scale of
   // its row rq for that tile's group (rows rq + 8 i are 16 G bytes apart),
-  // and that group.  Tiles are loaded in order u0, u0 + 1, ...
+  // and that group's place in the window.  Tiles are loaded in the order of
+  // the positions; after the last group of the window comes group sp.ga of
+  // the next strip.
   const uint32_t hi_delta = BITS == 3 ? lane_hi_delta(q) : 0u;
-  const uint8_t* fw = a.packed + uint64_t(u0) * TB + lane_tile_offset<BITS>(q, rq);
-  const uint16_t* fs = a.scales + (uint64_t(first_strip) * kStrip + rq) * G + g_first;
+  const uint8_t* fw = a.packed + (uint64_t(first_strip) * G + sp.ga + g_first) * TB +
+                      lane_tile_offset<BITS>(q, rq);
+  const uint16_t* fs =
+      a.scales + (uint64_t(first_strip) * kStrip + rq) * G + sp.ga + g_first;
   uint32_t fg = g_first;
   const uint32_t s8b = 16u * G;
-  const uint32_t s_wrap = 31u * G + 1u;  // last group of row r -> group 0 of row r, next strip
+  const uint64_t w_wrap = uint64_t(G - sp.W + 1) * TB;  // tile after the window's last one
+  const uint32_t s_wrap = 32u * G - sp.W + 1u;           // likewise for the scale of row r
   auto fetch = [&](uint4 (&wd)[4], uint16_t (&sv)[4]) {
     load_unit_m1<BITS>(wd, fw, hi_delta);
     const uint8_t* sb = reinterpret_cast<const uint8_t*>(fs);
 #pragma unroll
     for (int i = 0; i < 4; ++i) sv[i] = __ldg(reinterpret_cast<const uint16_t*>(sb + i * s8b));
-    fw += TB;
-    const bool wrap = fg + 1 == G;
+    const bool wrap = fg + 1 == sp.W;
+    fw += wrap ? w_wrap : uint64_t(TB);
     fs += wrap ? s_wrap : 1u;
     fg = wrap ? 0u : fg + 1u;
   };
@@ -397,7 +440,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   uint4 b0[4], b1[4], b2[4];
   uint16_t s0[4], s1[4], s2[4];
   if (u0 < u1) fetch(b0, s0);
-  fill_warp_table<kM1Warps>(wt, cu0, cu1 - cu0, G);
+  fill_warp_table<kM1Warps>(wt, sp);
   build_lut_shfl<BITS>(lut, cbv);
   // chunks beyond the ones held in registers (very long K) take a plain loop
   for (int i = threadIdx.x + XPT * blockDim.x; i < nx; i += blockDim.x)
@@ -428,7 +471,8 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   if (u0 < u1) {
     // Tiles are prefetched two ahead into three rotating buffers.
     uint32_t strip = first_strip, g = g_first;
-    uint32_t xa = xa0 + g_first * kXGroupBytes;
+    const uint32_t xa_w = xa0 + sp.ga * kXGroupBytes;  // first group of the window
+    uint32_t xa = xa_w + g_first * kXGroupBytes;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     // consume the tile u held in (wd, sv); refill that buffer with tile u + 3
     auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
@@ -442,7 +486,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
         acc[i] = fmaf(s, se[i] + so[i], acc[i]);
       }
       if (u + 3 < u1) fetch(wd, sv);
-      if (g + 1 == G || u + 1 == u1) {
+      if (g + 1 == sp.W || u + 1 == u1) {
         float vals[4][1];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -452,10 +496,10 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
           vals[i][0] = v;
           acc[i] = 0.0f;
         }
-        deposit_strip<1, 4>(a, strip, u0, u1, first_strip, vals, rows, q == 0, my_slots);
+        deposit_strip<1, 4>(a, sp, strip, u0, u1, first_strip, vals, rows, q == 0, my_slots);
         ++strip;
         g = 0;
-        xa = xa0;
+        xa = xa_w;
       } else {
         ++g;
         xa += kXGroupBytes;
@@ -470,7 +514,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     }
   }
   __syncthreads();
-  cta_finish<1, kM1Warps>(a, slots, wt, cu0, cu1);
+  cta_finish<1, kM1Warps>(a, sp, slots, wt);
 }
 
 // --------------------------------------------------------------------------
@@ -542,15 +586,15 @@ __global__ void __launch_bounds__(kGenWarps * 32, 1) gemv_kernel(GemvArgs a) {
   float* slots = reinterpret_cast<float*>(smem + kLutBytes);  // [NW][2][M][32]
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const uint32_t lut_base = sm_addr(smem);
-  const uint32_t cu0 = range_begin(blockIdx.x, uint32_t(a.U), uint32_t(a.C));
-  const uint32_t cu1 = range_begin(blockIdx.x + 1, uint32_t(a.U), uint32_t(a.C));
+  const Span sp = cta_span(a, blockIdx.x);
   if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
-  fill_warp_table<kGenWarps>(wt, cu0, cu1 - cu0, uint32_t(a.G));
+  fill_warp_table<kGenWarps>(wt, sp);
   __syncthreads();
   build_lut_copies<BITS>(smem, cbs, pairs);
   __syncthreads();
 
-  const uint32_t u0 = cu0 + wt.wb[wl], u1 = cu0 + wt.wb[wl + 1];
+  // the warp's positions [u0, u1) of the CTA's unit sequence
+  const uint32_t u0 = sp.v0 + wt.wb[wl], u1 = sp.v0 + wt.wb[wl + 1];
   const uint32_t off_e = uint32_t(lane) * 4u, off_o = 128u + uint32_t(lane) * 4u;
   constexpr int TB = tile_bytes(BITS);
   const int rows[1] = {lane};
@@ -559,24 +603,30 @@ __global__ void __launch_bounds__(kGenWarps * 32, 1) gemv_kernel(GemvArgs a) {
   if (u0 < u1) {
     const uint32_t first_strip = wt.ws[wl];
     int64_t strip = first_strip;
-    int64_t g = int64_t(u0) - strip * a.G;
+    int64_t g = u0 % sp.W;  // place in the window: group sp.ga + g
     float acc[1][M];
 #pragma unroll
     for (int m = 0; m < M; ++m) acc[0][m] = 0.0f;
     uint4 cur[4], nxt[4];
-    load_unit_row<BITS>(cur, a.packed + int64_t(u0) * TB, lane);
+    // tile of (strip, window place) and the one after it in the sequence
+    auto tile = [&](int64_t st, int64_t gw) { return a.packed + (st * a.G + sp.ga + gw) * TB; };
+    load_unit_row<BITS>(cur, tile(strip, g), lane);
     for (uint32_t u = u0; u < u1; ++u) {
-      if (u + 1 < u1) load_unit_row<BITS>(nxt, a.packed + int64_t(u + 1) * TB, lane);
+      const bool last_in_window = g + 1 == sp.W;
+      if (u + 1 < u1)
+        load_unit_row<BITS>(nxt, last_in_window ? tile(strip + 1, 0) : tile(strip, g + 1), lane);
       const int64_t row = strip * kStrip + lane;
-      const float s = __uint_as_float(uint32_t(a.scales[row * a.G + g]) << 16);
+      const float s = __uint_as_float(uint32_t(a.scales[row * a.G + sp.ga + g]) << 16);
       float2 part[M];
 #pragma unroll
       for (int m = 0; m < M; ++m) part[m] = make_float2(0.0f, 0.0f);
-      unit_partial_gen<BITS, M>(part, cur, lut_base, off_e, off_o, int(g * kGroup), a.x, a.K);
+      unit_partial_gen<BITS, M>(part, cur, lut_base, off_e, off_o, int((sp.ga + g) * kGroup),
+                                a.x, a.K);
 #pragma unroll
       for (int m = 0; m < M; ++m) acc[0][m] = fmaf(s, part[m].x + part[m].y, acc[0][m]);
-      if (g == a.G - 1 || u + 1 == u1) {
-        deposit_strip<M, 1>(a, uint32_t(strip), u0, u1, first_strip, acc, rows, true, my_slots);
+      if (last_in_window || u + 1 == u1) {
+        deposit_strip<M, 1>(a, sp, uint32_t(strip), u0, u1, first_strip, acc, rows, true,
+                            my_slots);
 #pragma unroll
         for (int m = 0; m < M; ++m) acc[0][m] = 0.0f;
         ++strip;
@@ -589,17 +639,15 @@ __global__ void __launch_bounds__(kGenWarps * 32, 1) gemv_kernel(GemvArgs a) {
     }
   }
   __syncthreads();
-  cta_finish<M, kGenWarps>(a, slots, wt, cu0, cu1);
+  cta_finish<M, kGenWarps>(a, sp, slots, wt);
 }
 
 // --------------------------------------------------------------------------
 // host side
 // --------------------------------------------------------------------------
 
-int64_t gemv_workspace_bytes(int64_t M, int64_t N) {
-  const int64_t counters = ((N / kStrip) * 4 + 255) / 256 * 256;
-  return counters + int64_t(kMaxCtas) * 2 * M * kStrip * 4;
-}
+// One 8-byte exchange slot per output value (exchange_half).
+int64_t gemv_workspace_bytes(int64_t M, int64_t N) { return (M * N * 8 + 255) / 256 * 256; }
 
 // Per device: the largest dynamic shared-memory size already granted to a
 // kernel instance.
@@ -621,23 +669,79 @@ static cudaError_t grant_smem(Kernel k, SmemGrant& g, int smem) {
   return cudaSuccess;
 }
 
-// Number of CTAs.  Equal unit ranges (one CTA per SM) balance the bytes
-// exactly but split strips between CTAs, whose partial sums then meet through
-// global memory at the end (a few microseconds of latency, ~kFixupUnits units
-// of streaming).  When the strips can be dealt out whole to a divisor of the
-// strip count that costs less, no strip is shared and that step disappears.
-constexpr int64_t kFixupUnits = 32;
+// The work plan (see cta_span).  Costs are in units per CTA, the longest CTA
+// deciding; a plan that splits strips between two CTAs pays kExchangeUnits
+// more for the exchange of the split halves at the end (one atomic round
+// trip to L2, about a unit's worth of streaming per warp).
+//  - whole strips, dealt out in equal runs to min(SMs, strips) CTAs;
+//  - equal unit ranges, one CTA per SM, when there are at least as many
+//    strips as CTAs (each range then spans a strip or more, so a strip is
+//    split between two CTAs at most);
+//  - otherwise, main and helper CTAs: one CTA per strip takes its first
+//    G - T groups, and each of the remaining CTAs the last T groups of nh
+//    strips, T balancing the two.
+constexpr int64_t kExchangeUnits = 16;
 
-static int choose_ctas(int64_t strips, int64_t G, int64_t U, int num_sms) {
+struct Plan {
+  int C;
+  uint32_t kind, align, Cm, T, nh;
+};
+
+static Plan choose_plan(int64_t S, int64_t G, int num_sms) {
   const int64_t cap = std::min<int64_t>(num_sms, kMaxCtas);
-  const int64_t c_split = std::min<int64_t>(cap, U);
-  const int64_t t_split = (U + c_split - 1) / c_split + kFixupUnits;
-  for (int64_t d = 1; d <= strips; ++d) {
-    if (strips % d != 0 || strips / d > cap) continue;
-    const int64_t t_whole = d * G;
-    return int(t_whole <= t_split ? strips / d : c_split);
+  const int64_t U = S * G;
+  Plan best;
+  // whole strips
+  best.C = int(std::min<int64_t>(cap, S));
+  best.kind = 0;
+  best.align = 1;
+  best.Cm = best.T = best.nh = 0;
+  int64_t t_best = (S + best.C - 1) / best.C * G;
+  if (S >= cap) {
+    const int64_t t = (U + cap - 1) / cap + kExchangeUnits;
+    if (t < t_best) {
+      t_best = t;
+      best.C = int(cap);
+      best.align = 0;
+    }
+  } else if (G >= 2) {
+    const int64_t H = cap - S;
+    const int64_t nh = (S + H - 1) / H;
+    int64_t T = (G + nh) / (nh + 1);  // G / (nh + 1), rounded
+    T = std::max<int64_t>(1, std::min<int64_t>(T, G - 1));
+    const int64_t t = std::max<int64_t>(G - T, nh * T) + kExchangeUnits;
+    if (t < t_best) {
+      t_best = t;
+      best.C = int(S + (S + nh - 1) / nh);
+      best.kind = 1;
+      best.align = 0;
+      best.Cm = uint32_t(S);
+      best.T = uint32_t(T);
+      best.nh = uint32_t(nh);
+    }
   }
-  return int(c_split);
+  return best;
+}
+
+// The plan as six integers {C, kind, align, Cm, T, nh} (for inspection).
+void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out) {
+  const Plan pl = choose_plan(N / kStrip, K / kGroup, num_sms);
+  out[0] = pl.C;
+  out[1] = int32_t(pl.kind);
+  out[2] = int32_t(pl.align);
+  out[3] = int32_t(pl.Cm);
+  out[4] = int32_t(pl.T);
+  out[5] = int32_t(pl.nh);
+}
+
+static void apply_plan(GemvArgs& a, int num_sms) {
+  const Plan pl = choose_plan(a.N / kStrip, a.G, num_sms);
+  a.C = pl.C;
+  a.kind = pl.kind;
+  a.align = pl.align;
+  a.Cm = pl.Cm;
+  a.T = pl.T;
+  a.nh = pl.nh;
 }
 
 static int64_t m1_smem(int64_t K) {
@@ -651,7 +755,7 @@ static cudaError_t launch_m1(GemvArgs a, int num_sms, cudaStream_t stream) {
   const int smem = int(m1_smem(a.K));
   cudaError_t err = grant_smem(gemv_m1_kernel<BITS>, grant, smem);
   if (err != cudaSuccess) return err;
-  a.C = choose_ctas(a.N / kStrip, a.G, a.U, num_sms);
+  apply_plan(a, num_sms);
   gemv_m1_kernel<BITS><<<unsigned(a.C), kM1Warps * 32, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -662,7 +766,7 @@ static cudaError_t launch_gen(GemvArgs a, int num_sms, cudaStream_t stream) {
   const int smem = kLutBytes + kGenWarps * 2 * M * kStrip * 4;
   cudaError_t err = grant_smem(gemv_kernel<BITS, M>, grant, smem);
   if (err != cudaSuccess) return err;
-  a.C = choose_ctas(a.N / kStrip, a.G, a.U, num_sms);
+  apply_plan(a, num_sms);
   gemv_kernel<BITS, M><<<unsigned(a.C), kGenWarps * 32, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -702,9 +806,7 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   a.scales = static_cast<const uint16_t*>(scales);
   a.codebook = static_cast<const uint16_t*>(codebook);
   a.y = y;
-  const int64_t counters = ((N / kStrip) * 4 + 255) / 256 * 256;
-  a.counters = static_cast<int*>(workspace);
-  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + counters);
+  a.xch = static_cast<unsigned long long*>(workspace);
   a.N = N;
   a.K = K;
   a.G = K / kGroup;

@@ -8,8 +8,8 @@
 // library no allocator of its own.  This entry point lets them call the
 // product with only their inputs and outputs.
 //
-// The scratch (the split-strip partial sums and the per-strip arrival
-// counters of lutq_gemv) lives in g_noalloc_scratch below: a file-scope
+// The scratch (the exchange slots where lutq_gemv meets the two halves of a
+// strip split between two CTAs) lives in g_noalloc_scratch below: a file-scope
 // __device__ array of kNoallocScratchBytes (4 MiB).  Every GPU that loads the
 // library holds that array until the process exits.  In host code the
 // array's name is only a stand-in for a device symbol, so its device address
@@ -76,10 +76,9 @@ extern "C" lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const vo
     g_scratch_addr[dev] = addr;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's contents; the arrival counters at its
-  // start must begin at zero.
-  const int64_t counter_bytes = ((N / lutq::kStrip) * 4 + 255) / 256 * 256;
-  if (cudaMemsetAsync(g_scratch_addr[dev], 0, size_t(counter_bytes), s) != cudaSuccess)
+  // The array keeps the previous call's contents; the exchange slots this
+  // problem uses must begin at zero.
+  if (cudaMemsetAsync(g_scratch_addr[dev], 0, size_t(need), s) != cudaSuccess)
     return LUTQ_ERR_CUDA;
   const cudaError_t err = lutq::launch_gemv(x_bf16, M, packed, scales_bf16, codebook_bf16, bits,
                                             N, K, y, g_scratch_addr[dev], g_scratch_sms[dev], s);

@@ -149,7 +149,9 @@ lutq_status lutq_pack(const uint8_t* codes, int64_t N, int64_t K, int bits,
 
 /*
  * lutq_workspace_bytes - device scratch size needed by lutq_gemv / lutq_gemm
- * for this problem (split-K partial sums and per-strip arrival counters).
+ * for this problem (lutq_gemv: one 8-byte exchange slot per output value,
+ * where the two halves of a row split between two thread blocks meet;
+ * lutq_gemm: split-K partial sums and per-tile arrival counters).
  * Returns -1 for an invalid argument.  The value does not depend on the device.
  */
 int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
@@ -200,15 +202,34 @@ lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
  *    that device current; make that first call before any stream capture.
  *  - All calls share the array: calls that may overlap on the GPU (other
  *    streams, other threads) race and must be serialized by the caller.  Each
- *    call first clears the array's arrival counters (an asynchronous memset
+ *    call first clears the part of the array it uses (an asynchronous memset
  *    on `stream`), so a call never depends on what an earlier one left.
  *  - Returns LUTQ_ERR_WORKSPACE, launching nothing, if the problem's scratch
- *    (N/8 bytes rounded up to 256, plus 128 KiB per batch row) exceeds 4 MiB.
+ *    (8 * M * N bytes, rounded up to 256) exceeds 4 MiB.
  */
 lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const void* packed,
                               const void* scales_bf16, const void* codebook_bf16,
                               int bits, int64_t N, int64_t K, float* y,
                               int32_t* dev_status, void* stream);
+
+/*
+ * lutq_gemv_plan - how lutq_gemv divides an N x K problem among thread blocks
+ * on a GPU with num_sms multiprocessors (host only; for inspection and tests).
+ *
+ * No counterpart in the paper: the FLUTE abstract asks for a kernel that
+ * keeps every multiprocessor streaming weights; this reports the division
+ * that does so.  The packed matrix is a sequence of units (strip of 32 rows,
+ * group of 128 codes), strip-major.  plan[6] receives {C, kind, align, Cm, T,
+ * nh}: C thread blocks; kind 0 gives block c the units
+ * [G*floor(c*S/C), G*floor((c+1)*S/C)) when align = 1 (whole strips) or
+ * [floor(c*U/C), floor((c+1)*U/C)) when align = 0 (S = N/32 strips, G = K/128
+ * groups, U = S*G units); kind 1 gives block c < Cm groups [0, G-T) of strip
+ * c and block Cm + h groups [G-T, G) of strips h*nh .. h*nh+nh-1 (those that
+ * exist).  Every strip is then whole in one block or split between two.
+ * Returns LUTQ_ERR_SHAPE for N, K as lutq_gemv rejects them,
+ * LUTQ_ERR_INVALID_ARG for a NULL plan or num_sms < 1.
+ */
+lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan);
 
 /*
  * lutq_gemm - the same product on the tensor cores (tcgen05), for batches

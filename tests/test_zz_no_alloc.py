@@ -55,7 +55,7 @@ def test_noalloc_matches_workspace_gemv_twice(lq, n, k, bits, kind, m):
 
 
 def test_noalloc_rejects_problems_beyond_its_array(lq):
-    # 2^26 rows need N/8 = 8 MiB of counters: more than the 4 MiB array.  The
+    # 2^26 rows need 8 N = 512 MiB of exchange slots: more than the 4 MiB array.  The
     # size check comes before any device work, so aligned placeholder
     # addresses are never touched.
     a = 1 << 20
