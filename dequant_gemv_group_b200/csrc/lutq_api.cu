@@ -15,7 +15,7 @@ cudaError_t launch_pack(const uint8_t* codes, int64_t N, int64_t K, int bits, vo
                         int32_t* dev_status, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* scales,
                         const void* codebook, int bits, int64_t N, int64_t K, float* y,
-                        void* workspace, int num_sms, cudaStream_t stream);
+                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* scales,
                         const void* codebook, int bits, int64_t N, int64_t K, float* y,
                         void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
@@ -155,7 +155,6 @@ lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed, const v
                       const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
                       void* workspace, int64_t workspace_bytes, int32_t* dev_status,
                       void* stream) {
-  (void)dev_status;
   lutq_status st = check_product_args(x_bf16, M, 16, packed, scales_bf16, codebook_bf16, bits, N,
                                       K, y, workspace, workspace_bytes,
                                       lutq_workspace_bytes(M, N, K, bits));
@@ -163,7 +162,8 @@ lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed, const v
   int sms = 0;
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_gemv(x_bf16, M, packed, scales_bf16, codebook_bf16, bits, N, K, y,
-                                     workspace, sms, static_cast<cudaStream_t>(stream)));
+                                     workspace, dev_status, sms,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed, const void* scales_bf16,

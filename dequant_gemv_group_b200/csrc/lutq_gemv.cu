@@ -40,6 +40,7 @@
 
 #include "lutq_common.cuh"
 #include "lutq_lut.cuh"
+#include "lutq_sm100.cuh"
 
 namespace lutq {
 
@@ -58,6 +59,7 @@ struct GemvArgs {
   const uint16_t* codebook; // bf16 [2^bits]
   float* y;                 // fp32 [M, N]
   unsigned long long* xch;  // [M][N] exchange slots of strips split between two CTAs (zero between calls)
+  int32_t* status;          // caller's device status word or null
   int64_t N, K, G, U;       // U = number of units
   int C;                    // CTAs
   // work plan (choose_plan): kind 0 = ranges of the unit sequence, strip-
@@ -354,12 +356,11 @@ __device__ __forceinline__ void unit_partial_m1(float (&se)[4], float (&so)[4],
   }
 }
 
-// Activations in shared memory stay bf16, in chunks of 32 values (64 bytes)
-// followed by 16 bytes of padding, so that the four chunks of a group that
-// the quarter-warps read at once fall in different banks.
-constexpr uint32_t kXChunkBytes = 80;
+// Activations in shared memory stay bf16, in order: a group's four chunks of
+// 32 values (64 bytes each) are contiguous, so that one bulk copy brings a
+// whole run of them.
+constexpr uint32_t kXChunkBytes = 64;
 constexpr uint32_t kXGroupBytes = 4 * kXChunkBytes;
-__host__ __device__ constexpr int64_t x_smem_bytes(int64_t k) { return k / 32 * kXChunkBytes; }
 
 // The lane's 32 activations of one group (16 bf16x2 words) from address xa.
 __device__ __forceinline__ void load_x_m1(uint32_t (&xw)[16], uint32_t xa) {
@@ -370,32 +371,83 @@ __device__ __forceinline__ void load_x_m1(uint32_t (&xw)[16], uint32_t xa) {
                  : "r"(xa + 16u * v));
 }
 
-// Activation chunk i (8 bf16 values, k = 8 i ..) into the padded layout.
-__device__ __forceinline__ void store_x_chunk(uint8_t* xs, int i, uint4 v) {
-  *reinterpret_cast<uint4*>(xs + (i >> 2) * kXChunkBytes + (i & 3) * 16) = v;
+
+// Shared-window layout of the M = 1 kernel, in addresses of the CTA's shared
+// window (the block's own static shared memory and the system's reserved
+// bytes lie below kSbaseMax, where dynamic shared memory begins):
+//   [kSlotsAt, kXLoAt)           warp slots, [NW][2][32] fp32
+//   [kXLoAt, kPageAt)            activations of groups [0, gb)
+//   [kPageAt, kAboveAt)          the lookup table, on its own 64 KB page
+//   [kAboveAt, ...)              activations of groups [gb, G), then each
+//                                warp's first tile, copied in by the bulk
+//                                copy engine
+// The dynamic size kAboveAt + m1_above_bytes therefore covers the window up
+// to the end of the staging area whatever the exact start (<= kSbaseMax).
+constexpr uint32_t kSbaseMax = 4096;
+constexpr uint32_t kSlotsAt = kSbaseMax;
+constexpr uint32_t kXLoAt = kSlotsAt + kM1Warps * 2 * kStrip * 4;
+constexpr uint32_t kPageAt = 0x10000;
+constexpr uint32_t kAboveAt = 0x20000;
+constexpr uint64_t kM1WaitNs = 2000000000ull;  // bounded waits: 2 s
+
+__host__ __device__ constexpr uint32_t x_groups_below(uint32_t G) {
+  return G < (kPageAt - kXLoAt) / kXGroupBytes ? G : (kPageAt - kXLoAt) / kXGroupBytes;
+}
+__host__ __device__ constexpr uint32_t m1_above_bytes(uint32_t G, int bits) {
+  return (G - x_groups_below(G)) * kXGroupBytes + kM1Warps * uint32_t(tile_bytes(bits));
 }
 
 template <int BITS>
 __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ WarpTable<kM1Warps> wt;
-  // The table sits on a 64 KB page of the shared window so that one byte
-  // permute produces its full address; activations and warp slots follow.
+  __shared__ __align__(8) uint64_t bars[1 + kM1Warps];  // activations, then one per warp's tile
+  __shared__ int abort_flag;
   const uint32_t sbase = sm_addr(smem);
-  const uint32_t lut_sa = (sbase + 0xFFFFu) & ~0xFFFFu;
-  uint8_t* lut = smem + (lut_sa - sbase);
-  uint8_t* xs = lut + kLutBytes;
-  float* slots = reinterpret_cast<float*>(xs + x_smem_bytes(a.K));
   const uint32_t G = uint32_t(a.G);
-  const Span sp = cta_span(a, blockIdx.x);
+  const uint32_t gb = x_groups_below(G);
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  // The layout needs dynamic shared memory to begin below kSbaseMax; the
+  // host allocates for that.  Should it not, nothing is touched.
+  if (sbase > kSbaseMax) {
+    if (threadIdx.x == 0) report(a.status, LUTQ_ERR_CUDA);
+    return;
+  }
+  float* slots = reinterpret_cast<float*>(smem + (kSlotsAt - sbase));
+  uint8_t* lut = smem + (kPageAt - sbase);
+  constexpr int TB = tile_bytes(BITS);
+  const uint32_t stage_at = kAboveAt + (G - gb) * kXGroupBytes + uint32_t(wl) * TB;
+  const uint32_t xbar = sm_addr(&bars[0]), tbar = sm_addr(&bars[1 + wl]);
+
+  const Span sp = cta_span(a, blockIdx.x);
   // the warp's positions [u0, u1) of the CTA's unit sequence
   const uint32_t u0 = sp.v0 + range_begin(wl, sp.v1 - sp.v0, kM1Warps);
   const uint32_t u1 = sp.v0 + range_begin(wl + 1, sp.v1 - sp.v0, kM1Warps);
   const uint32_t first_strip = sp.s0 + u0 / sp.W;
   const uint32_t g_first = u0 % sp.W;  // within the window: group sp.ga + g_first
   const int q = lane >> 3, rq = lane & 7;
-  constexpr int TB = tile_bytes(BITS);
+  const uint8_t* tile0 = a.packed + (uint64_t(first_strip) * G + sp.ga + g_first) * TB;
+
+  // Activations and each warp's first tile come in through the bulk copy
+  // engine (no load instructions, so the table build below does not queue
+  // behind them): the activations in one or two runs (below and above the
+  // table's page), counted in bytes on bars[0]; the tile whole into the
+  // warp's staging area on its own barrier.
+  if (threadIdx.x == 0) abort_flag = 0;
+  if (lane == 0) {
+    if (wl == 0) sm100::mbar_init(xbar, 1);
+    sm100::mbar_init(tbar, 1);
+    sm100::mbar_fence_init();
+    if (wl == 0) sm100::mbar_expect_tx(xbar, uint32_t(a.K) * 2u);
+    if (u0 < u1) {
+      sm100::mbar_expect_tx(tbar, uint32_t(TB));
+      sm100::bulk_g2s(stage_at, tile0, uint32_t(TB), tbar);
+    }
+  }
+  if (threadIdx.x == 0) {
+    sm100::bulk_g2s(kXLoAt, a.x, gb * kXGroupBytes, xbar);
+    if (gb < G) sm100::bulk_g2s(kAboveAt, a.x + uint64_t(gb) * kGroup, (G - gb) * kXGroupBytes, xbar);
+  }
 
   // Fetch cursor: the lane's bytes of the next tile to load, the scale of
   // its row rq for that tile's group (rows rq + 8 i are 16 G bytes apart),
@@ -403,76 +455,91 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   // the positions; after the last group of the window comes group sp.ga of
   // the next strip.
   const uint32_t hi_delta = BITS == 3 ? lane_hi_delta(q) : 0u;
-  const uint8_t* fw = a.packed + (uint64_t(first_strip) * G + sp.ga + g_first) * TB +
-                      lane_tile_offset<BITS>(q, rq);
+  const uint32_t lane_off = lane_tile_offset<BITS>(q, rq);
+  const uint8_t* fw = tile0 + lane_off;
   const uint16_t* fs =
       a.scales + (uint64_t(first_strip) * kStrip + rq) * G + sp.ga + g_first;
   uint32_t fg = g_first;
   const uint32_t s8b = 16u * G;
   const uint64_t w_wrap = uint64_t(G - sp.W + 1) * TB;  // tile after the window's last one
   const uint32_t s_wrap = 32u * G - sp.W + 1u;           // likewise for the scale of row r
-  auto fetch = [&](uint4 (&wd)[4], uint16_t (&sv)[4]) {
-    load_unit_m1<BITS>(wd, fw, hi_delta);
+  auto fetch_scales = [&](uint16_t (&sv)[4]) {
     const uint8_t* sb = reinterpret_cast<const uint8_t*>(fs);
 #pragma unroll
     for (int i = 0; i < 4; ++i) sv[i] = __ldg(reinterpret_cast<const uint16_t*>(sb + i * s8b));
+  };
+  auto advance = [&]() {
     const bool wrap = fg + 1 == sp.W;
     fw += wrap ? w_wrap : uint64_t(TB);
     fs += wrap ? s_wrap : 1u;
     fg = wrap ? 0u : fg + 1u;
   };
+  auto fetch = [&](uint4 (&wd)[4], uint16_t (&sv)[4]) {
+    load_unit_m1<BITS>(wd, fw, hi_delta);
+    fetch_scales(sv);
+    advance();
+  };
 
   // Lane t holds codebook[t mod 2^BITS]; the table is built from it with
   // shuffles, so no shared staging (and no barrier) precedes the build.
   const uint32_t cbv = __ldg(a.codebook + (lane & ((1 << BITS) - 1)));
-  // Activations: issue every load first, build the table while they are in
-  // flight, then store them.
-  constexpr int XPT = 8;  // x chunks (8 values) per thread held in registers
-  uint4 xv[XPT];
-  const int nx = int(a.K / 8);
-#pragma unroll
-  for (int r = 0; r < XPT; ++r) {
-    const int i = threadIdx.x + r * blockDim.x;
-    if (i < nx) xv[r] = __ldg(reinterpret_cast<const uint4*>(a.x) + i);
-  }
-  // The first tile follows right behind those loads: one 2 KB tile per warp
-  // does not crowd them out, and its latency overlaps theirs.
   uint4 b0[4], b1[4], b2[4];
   uint16_t s0[4], s1[4], s2[4];
-  if (u0 < u1) fetch(b0, s0);
+  if (u0 < u1) {
+    fetch_scales(s0);  // the words of tile u0 are on their way to the staging area
+    advance();
+  }
   fill_warp_table<kM1Warps>(wt, sp);
   build_lut_shfl<BITS>(lut, cbv);
-  // chunks beyond the ones held in registers (very long K) take a plain loop
-  for (int i = threadIdx.x + XPT * blockDim.x; i < nx; i += blockDim.x)
-    store_x_chunk(xs, i, __ldg(reinterpret_cast<const uint4*>(a.x) + i));
-#pragma unroll
-  for (int r = 0; r < XPT; ++r) {
-    const int i = threadIdx.x + r * blockDim.x;
-    if (i < nx) store_x_chunk(xs, i, xv[r]);
-  }
-  // Only now, with the codebook and the activations in, are the next two
-  // tiles requested: issued earlier, the weight stream would fill the memory
-  // pipeline ahead of those small loads and hold up the prologue.
-  asm volatile("" ::: "memory");
-  __syncwarp();
+  // the next two tiles go straight to registers
   if (u0 + 1 < u1) fetch(b1, s1);
   if (u0 + 2 < u1) fetch(b2, s2);
-  __syncthreads();
+  __syncthreads();  // table, warp table, barrier initialisation
 
-  const uint32_t page = (lut_sa >> 16) << 8;
+  // Activations and the first tile in; a wait that runs out marks the call
+  // failed, and the warps skip their work.
+  if (!sm100::mbar_wait(xbar, 0, &abort_flag, kM1WaitNs)) report(a.status, LUTQ_ERR_TIMEOUT);
+  bool ok = true;
+  if (u0 < u1) {
+    ok = sm100::mbar_wait(tbar, 0, &abort_flag, kM1WaitNs);
+    if (!ok) report(a.status, LUTQ_ERR_TIMEOUT);
+    // the staged words of tile u0, at the offsets a global load would use
+    const uint32_t t = stage_at + lane_off;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (BITS == 4) {
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(b0[i].x), "=r"(b0[i].y), "=r"(b0[i].z), "=r"(b0[i].w)
+                     : "r"(t + 128u * i));
+      } else {
+        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
+                     : "=r"(b0[i].x), "=r"(b0[i].y) : "r"(t + 128u * i));
+        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
+                     : "=r"(b0[i].z), "=r"(b0[i].w) : "r"(t + hi_delta + 128u * i));
+      }
+    }
+  }
+  ok = ok && !*reinterpret_cast<volatile int*>(&abort_flag);
+
+  const uint32_t page = (kPageAt >> 16) << 8;
   const uint32_t lane_e = page | uint32_t(lane) * 4u, lane_o = page | (128u + uint32_t(lane) * 4u);
   const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
-  const uint32_t xa0 = sm_addr(xs) + uint32_t(q) * kXChunkBytes;
   float* my_slots = slots + wl * 2 * kStrip;
   int rows[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) rows[i] = rq + 8 * i;
+  // activation address of (group g, chunk q): below the page for g < gb
+  const uint32_t xq = uint32_t(q) * kXChunkBytes;
+  auto x_at = [&](uint32_t g) {
+    return (g < gb ? kXLoAt + g * kXGroupBytes : kAboveAt + (g - gb) * kXGroupBytes) + xq;
+  };
 
-  if (u0 < u1) {
+  if (u0 < u1 && ok) {
     // Tiles are prefetched two ahead into three rotating buffers.
     uint32_t strip = first_strip, g = g_first;
-    const uint32_t xa_w = xa0 + sp.ga * kXGroupBytes;  // first group of the window
-    uint32_t xa = xa_w + g_first * kXGroupBytes;
+    const uint32_t xa_w = x_at(sp.ga);  // first group of the window
+    uint32_t xa = x_at(sp.ga + g_first);
+    const uint32_t xa_hi = x_at(gb);    // first group above the page
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     // consume the tile u held in (wd, sv); refill that buffer with tile u + 3
     auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
@@ -502,7 +569,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
         xa = xa_w;
       } else {
         ++g;
-        xa += kXGroupBytes;
+        xa = sp.ga + g == gb ? xa_hi : xa + kXGroupBytes;
       }
     };
     for (uint32_t u = u0; u < u1; u += 3) {
@@ -514,6 +581,14 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     }
   }
   __syncthreads();
+  if (*reinterpret_cast<volatile int*>(&abort_flag)) {
+    // A wait ran out: let this block's own copies land (bounded again)
+    // before the shared memory is released, and leave y to the error.
+    volatile int again = 0;
+    if (lane == 0 && u0 < u1) sm100::mbar_wait(tbar, 0, &again, kM1WaitNs);
+    if (threadIdx.x == 0) sm100::mbar_wait(xbar, 0, &again, kM1WaitNs);
+    return;
+  }
   cta_finish<1, kM1Warps>(a, sp, slots, wt);
 }
 
@@ -744,15 +819,14 @@ static void apply_plan(GemvArgs& a, int num_sms) {
   a.nh = pl.nh;
 }
 
-static int64_t m1_smem(int64_t K) {
-  // page-alignment slack (< 64 KB) + table + activations + warp slots
-  return 2 * kLutBytes + x_smem_bytes(K) + kM1Warps * 2 * kStrip * 4;
+static int64_t m1_smem(int64_t K, int bits) {
+  return int64_t(kAboveAt) + m1_above_bytes(uint32_t(K / kGroup), bits);
 }
 
 template <int BITS>
 static cudaError_t launch_m1(GemvArgs a, int num_sms, cudaStream_t stream) {
   static SmemGrant grant;
-  const int smem = int(m1_smem(a.K));
+  const int smem = int(m1_smem(a.K, BITS));
   cudaError_t err = grant_smem(gemv_m1_kernel<BITS>, grant, smem);
   if (err != cudaSuccess) return err;
   apply_plan(a, num_sms);
@@ -776,7 +850,7 @@ static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream
   switch (M) {
     case 1:
       // the M = 1 kernel keeps all of x in shared memory next to the table
-      if (m1_smem(a.K) <= kMaxSmemPerBlock) return launch_m1<BITS>(a, num_sms, s);
+      if (m1_smem(a.K, BITS) <= kMaxSmemPerBlock - 1024) return launch_m1<BITS>(a, num_sms, s);
       return launch_gen<BITS, 1>(a, num_sms, s);
     case 2: return launch_gen<BITS, 2>(a, num_sms, s);
     case 3: return launch_gen<BITS, 3>(a, num_sms, s);
@@ -799,7 +873,7 @@ static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream
 
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* scales,
                         const void* codebook, int bits, int64_t N, int64_t K, float* y,
-                        void* workspace, int num_sms, cudaStream_t stream) {
+                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream) {
   GemvArgs a;
   a.x = static_cast<const uint16_t*>(x);
   a.packed = static_cast<const uint8_t*>(packed);
@@ -807,6 +881,7 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   a.codebook = static_cast<const uint16_t*>(codebook);
   a.y = y;
   a.xch = static_cast<unsigned long long*>(workspace);
+  a.status = dev_status;
   a.N = N;
   a.K = K;
   a.G = K / kGroup;

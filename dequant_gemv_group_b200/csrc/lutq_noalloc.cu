@@ -24,7 +24,7 @@
 namespace lutq {
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* scales,
                         const void* codebook, int bits, int64_t N, int64_t K, float* y,
-                        void* workspace, int num_sms, cudaStream_t stream);
+                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
 int64_t gemv_workspace_bytes(int64_t M, int64_t N);
 }  // namespace lutq
 
@@ -47,7 +47,6 @@ extern "C" lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const vo
                                          const void* scales_bf16, const void* codebook_bf16,
                                          int bits, int64_t N, int64_t K, float* y,
                                          int32_t* dev_status, void* stream) {
-  (void)dev_status;
   if (!x_bf16 || !packed || !scales_bf16 || !codebook_bf16 || !y) return LUTQ_ERR_INVALID_ARG;
   if (bits != 3 && bits != 4) return LUTQ_ERR_BITS;
   if (N < lutq::kStrip || K < lutq::kGroup || N % lutq::kStrip != 0 || K % lutq::kGroup != 0 ||
@@ -80,7 +79,8 @@ extern "C" lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const vo
   // problem uses must begin at zero.
   if (cudaMemsetAsync(g_scratch_addr[dev], 0, size_t(need), s) != cudaSuccess)
     return LUTQ_ERR_CUDA;
-  const cudaError_t err = lutq::launch_gemv(x_bf16, M, packed, scales_bf16, codebook_bf16, bits,
-                                            N, K, y, g_scratch_addr[dev], g_scratch_sms[dev], s);
+  const cudaError_t err =
+      lutq::launch_gemv(x_bf16, M, packed, scales_bf16, codebook_bf16, bits, N, K, y,
+                        g_scratch_addr[dev], dev_status, g_scratch_sms[dev], s);
   return err == cudaSuccess ? LUTQ_OK : LUTQ_ERR_CUDA;
 }
