@@ -232,35 +232,35 @@ __device__ __forceinline__ void ffma2(float2& acc, float lo, float hi, float x0,
 // M = 1
 // --------------------------------------------------------------------------
 
-// ae += c_even * x_even and ao += c_odd * x_odd, with lv = (c_even, c_odd) and
+// acc += c_even * x_even + c_odd * x_odd, with lv = (c_even, c_odd) and
 // xw = (x_even, x_odd) bf16x2 words (low half = even k): two fused
-// multiply-adds with bf16 multiplicands and an fp32 addend.  The product of
-// two bf16 values is exact in fp32, so each step rounds once, exactly as an
-// fp32 fma on the widened operands would; no instruction widens anything.
-__device__ __forceinline__ void pair_fma(float& ae, float& ao, uint32_t lv, uint32_t xw) {
+// multiply-adds with bf16 multiplicands and an fp32 addend, one after the
+// other.  The product of two bf16 values is exact in fp32, so each step
+// rounds once, exactly as an fp32 fma on the widened operands would; no
+// instruction widens anything.
+__device__ __forceinline__ void pair_fma(float& acc, uint32_t lv, uint32_t xw) {
   asm("{\n\t.reg .b16 c0, c1, x0, x1;\n\t"
-      "mov.b32 {c0, c1}, %2;\n\tmov.b32 {x0, x1}, %3;\n\t"
-      "fma.rn.f32.bf16 %0, c0, x0, %0;\n\tfma.rn.f32.bf16 %1, c1, x1, %1;\n\t}"
-      : "+f"(ae), "+f"(ao) : "r"(lv), "r"(xw));
+      "mov.b32 {c0, c1}, %1;\n\tmov.b32 {x0, x1}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, c0, x0, %0;\n\tfma.rn.f32.bf16 %0, c1, x1, %0;\n\t}"
+      : "+f"(acc) : "r"(lv), "r"(xw));
 }
 
-// The same with a zero addend: se = c_even * x_even, so = c_odd * x_odd (the
-// first pair of a chain; no zeroed accumulator needs setting up).
-__device__ __forceinline__ void pair_first(float& ae, float& ao, uint32_t lv, uint32_t xw) {
+// The same starting from zero (the first pair of a chain).
+__device__ __forceinline__ void pair_first(float& acc, uint32_t lv, uint32_t xw) {
   asm("{\n\t.reg .b16 c0, c1, x0, x1;\n\t"
-      "mov.b32 {c0, c1}, %2;\n\tmov.b32 {x0, x1}, %3;\n\t"
-      "fma.rn.f32.bf16 %0, c0, x0, 0f00000000;\n\tfma.rn.f32.bf16 %1, c1, x1, 0f00000000;\n\t}"
-      : "=f"(ae), "=f"(ao) : "r"(lv), "r"(xw));
+      "mov.b32 {c0, c1}, %1;\n\tmov.b32 {x0, x1}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, c0, x0, 0f00000000;\n\tfma.rn.f32.bf16 %0, c1, x1, %0;\n\t}"
+      : "=f"(acc) : "r"(lv), "r"(xw));
 }
 
-// Row sums of one unit, split by k parity: se[i] (even k) and so[i] (odd k)
-// of row i.  The four rows' u32 index words idx[i] (four pair indices each)
-// go against the four activation words xw[0..3]; the rows are interleaved so
-// that four independent table loads and accumulator chains are in flight.
-// FIRST starts the chains (se, so are not read).
+// Row sums of one unit: su[i] for row i.  The four rows' u32 index words
+// idx[i] (four pair indices each) go against the four activation words
+// xw[0..3]; the rows are interleaved so that four independent table loads
+// and accumulator chains are in flight.  FIRST starts the chains (su is not
+// read).
 template <bool FIRST>
-__device__ __forceinline__ void quad4(float (&se)[4], float (&so)[4], const uint32_t (&idx)[4],
-                                      uint32_t lane_hi, const uint32_t* xw) {
+__device__ __forceinline__ void quad4(float (&su)[4], const uint32_t (&idx)[4], uint32_t lane_hi,
+                                      const uint32_t* xw) {
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     uint32_t lv[4];
@@ -272,9 +272,9 @@ __device__ __forceinline__ void quad4(float (&se)[4], float (&so)[4], const uint
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       if (FIRST && b == 0)
-        pair_first(se[i], so[i], lv[i], xw[b]);
+        pair_first(su[i], lv[i], xw[b]);
       else
-        pair_fma(se[i], so[i], lv[i], xw[b]);
+        pair_fma(su[i], lv[i], xw[b]);
     }
   }
 }
@@ -312,28 +312,27 @@ __device__ __forceinline__ void load_unit_m1(uint4 (&wd)[4], const uint8_t* p,
   }
 }
 
-// Row sums of one unit for the lane's four rows, split by k parity.
+// Row sums of one unit for the lane's four rows.
 template <int BITS>
-__device__ __forceinline__ void unit_partial_m1(float (&se)[4], float (&so)[4],
-                                                const uint4 (&wd)[4], uint32_t lane_e,
-                                                uint32_t lane_o, uint32_t hi_shift,
-                                                const uint32_t (&xw)[16]) {
+__device__ __forceinline__ void unit_partial_m1(float (&su)[4], const uint4 (&wd)[4],
+                                                uint32_t lane_e, uint32_t lane_o,
+                                                uint32_t hi_shift, const uint32_t (&xw)[16]) {
   if (BITS == 4) {
     {
       const uint32_t idx[4] = {wd[0].x, wd[1].x, wd[2].x, wd[3].x};
-      quad4<true>(se, so, idx, lane_e, xw + 0);
+      quad4<true>(su, idx, lane_e, xw + 0);
     }
     {
       const uint32_t idx[4] = {wd[0].y, wd[1].y, wd[2].y, wd[3].y};
-      quad4<false>(se, so, idx, lane_e, xw + 4);
+      quad4<false>(su, idx, lane_e, xw + 4);
     }
     {
       const uint32_t idx[4] = {wd[0].z, wd[1].z, wd[2].z, wd[3].z};
-      quad4<false>(se, so, idx, lane_e, xw + 8);
+      quad4<false>(su, idx, lane_e, xw + 8);
     }
     {
       const uint32_t idx[4] = {wd[0].w, wd[1].w, wd[2].w, wd[3].w};
-      quad4<false>(se, so, idx, lane_e, xw + 12);
+      quad4<false>(su, idx, lane_e, xw + 12);
     }
   } else {
     // lo u32 j goes with hi u32 j; lo word 1 reads its hi fields two bits up
@@ -348,10 +347,10 @@ __device__ __forceinline__ void unit_partial_m1(float (&se)[4], float (&so)[4],
         o[i] = (l & 0xF0F0F0F0u) | (h & 0x0F0F0F0Fu);
       }
       if (j == 0)
-        quad4<true>(se, so, e, lane_e, xw);
+        quad4<true>(su, e, lane_e, xw);
       else
-        quad4<false>(se, so, e, lane_e, xw + 8);
-      quad4<false>(se, so, o, lane_o, xw + 8 * j + 4);
+        quad4<false>(su, e, lane_e, xw + 8);
+      quad4<false>(su, o, lane_o, xw + 8 * j + 4);
     }
   }
 }
@@ -433,6 +432,13 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   // behind them): the activations in one or two runs (below and above the
   // table's page), counted in bytes on bars[0]; the tile whole into the
   // warp's staging area on its own barrier.
+  // Everything above reads only the launch parameters.  The kernel is
+  // launched as a programmatic dependent of the work before it on the
+  // stream, so it may start while that work finishes; global memory is
+  // touched only from here on, once that work is complete.  The next launch
+  // may likewise start early (it waits the same way).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) abort_flag = 0;
   if (lane == 0) {
     if (wl == 0) sm100::mbar_init(xbar, 1);
@@ -469,10 +475,13 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     for (int i = 0; i < 4; ++i) sv[i] = __ldg(reinterpret_cast<const uint16_t*>(sb + i * s8b));
   };
   auto advance = [&]() {
-    const bool wrap = fg + 1 == sp.W;
-    fw += wrap ? w_wrap : uint64_t(TB);
-    fs += wrap ? s_wrap : 1u;
-    fg = wrap ? 0u : fg + 1u;
+    fw += TB;
+    ++fs;
+    if (++fg == sp.W) {  // rare: on to the next strip
+      fg = 0;
+      fw += w_wrap - TB;
+      fs += s_wrap - 1u;
+    }
   };
   auto fetch = [&](uint4 (&wd)[4], uint16_t (&sv)[4]) {
     load_unit_m1<BITS>(wd, fw, hi_delta);
@@ -545,13 +554,10 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
       uint32_t xw[16];
       load_x_m1(xw, xa);
-      float se[4], so[4];
-      unit_partial_m1<BITS>(se, so, wd, lane_e, lane_o, hi_shift, xw);
+      float su[4];
+      unit_partial_m1<BITS>(su, wd, lane_e, lane_o, hi_shift, xw);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float s = __uint_as_float(uint32_t(sv[i]) << 16);
-        acc[i] = fmaf(s, se[i] + so[i], acc[i]);
-      }
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(__uint_as_float(uint32_t(sv[i]) << 16), su[i], acc[i]);
       if (u + 3 < u1) fetch(wd, sv);
       if (g + 1 == sp.W || u + 1 == u1) {
         float vals[4][1];
@@ -830,8 +836,19 @@ static cudaError_t launch_m1(GemvArgs a, int num_sms, cudaStream_t stream) {
   cudaError_t err = grant_smem(gemv_m1_kernel<BITS>, grant, smem);
   if (err != cudaSuccess) return err;
   apply_plan(a, num_sms);
-  gemv_m1_kernel<BITS><<<unsigned(a.C), kM1Warps * 32, smem, stream>>>(a);
-  return cudaGetLastError();
+  // programmatic dependent launch: the kernel's prologue (launch parameters,
+  // work split) may overlap the end of the preceding kernel on the stream
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(a.C));
+  cfg.blockDim = dim3(kM1Warps * 32);
+  cfg.dynamicSmemBytes = size_t(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_m1_kernel<BITS>, a);
 }
 
 template <int BITS, int M>
