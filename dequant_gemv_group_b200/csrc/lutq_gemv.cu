@@ -253,14 +253,15 @@ __device__ __forceinline__ void pair_first(float& acc, uint32_t lv, uint32_t xw)
       : "=f"(acc) : "r"(lv), "r"(xw));
 }
 
-// Row sums of one unit: su[i] for row i.  The four rows' u32 index words
-// idx[i] (four pair indices each) go against the four activation words
-// xw[0..3]; the rows are interleaved so that four independent table loads
-// and accumulator chains are in flight.  FIRST starts the chains (su is not
+// Row sums of one unit, su[i][m] for row i and batch row m.  The four rows'
+// u32 index words idx[i] (four pair indices each) go against the activation
+// words xq[m][0..3] of each batch row; the rows are interleaved so that four
+// independent table loads and accumulator chains are in flight, and each
+// table load serves all M batch rows.  FIRST starts the chains (su is not
 // read).
-template <bool FIRST>
-__device__ __forceinline__ void quad4(float (&su)[4], const uint32_t (&idx)[4], uint32_t lane_hi,
-                                      const uint32_t* xw) {
+template <bool FIRST, int M>
+__device__ __forceinline__ void quad4(float (&su)[4][M], const uint32_t (&idx)[4],
+                                      uint32_t lane_hi, const uint32_t (&xq)[M][4]) {
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     uint32_t lv[4];
@@ -270,13 +271,26 @@ __device__ __forceinline__ void quad4(float (&su)[4], const uint32_t (&idx)[4], 
       // page (bits 23:16) come from lane_hi
       lv[i] = lds32(__byte_perm(idx[i], lane_hi, 0x6504u | (uint32_t(b) << 4)));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (FIRST && b == 0)
-        pair_first(su[i], lv[i], xw[b]);
-      else
-        pair_fma(su[i], lv[i], xw[b]);
-    }
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        if (FIRST && b == 0)
+          pair_first(su[i][m], lv[i], xq[m][b]);
+        else
+          pair_fma(su[i][m], lv[i], xq[m][b]);
+      }
   }
+}
+
+// Four activation words (8 bf16 values) of each batch row: batch row m's
+// run of the current group starts at xa + m * xstride.
+template <int M>
+__device__ __forceinline__ void load_xq(uint32_t (&xq)[M][4], uint32_t xa, uint32_t xstride) {
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(xq[m][0]), "=r"(xq[m][1]), "=r"(xq[m][2]), "=r"(xq[m][3])
+                 : "r"(xa + uint32_t(m) * xstride));
 }
 
 // Byte offset, inside a tile, of the lane's packed bytes of row rq; rows
@@ -312,27 +326,25 @@ __device__ __forceinline__ void load_unit_m1(uint4 (&wd)[4], const uint8_t* p,
   }
 }
 
-// Row sums of one unit for the lane's four rows.
-template <int BITS>
-__device__ __forceinline__ void unit_partial_m1(float (&su)[4], const uint4 (&wd)[4],
-                                                uint32_t lane_e, uint32_t lane_o,
-                                                uint32_t hi_shift, const uint32_t (&xw)[16]) {
+// Row sums of one unit for the lane's four rows and the M batch rows; xa is
+// the address of the lane's 32 activations of the group for batch row 0.
+template <int BITS, int M>
+__device__ __forceinline__ void unit_partial(float (&su)[4][M], const uint4 (&wd)[4],
+                                             uint32_t lane_e, uint32_t lane_o, uint32_t hi_shift,
+                                             uint32_t xa, uint32_t xstride) {
+  uint32_t xq[M][4];
   if (BITS == 4) {
-    {
-      const uint32_t idx[4] = {wd[0].x, wd[1].x, wd[2].x, wd[3].x};
-      quad4<true>(su, idx, lane_e, xw + 0);
-    }
-    {
-      const uint32_t idx[4] = {wd[0].y, wd[1].y, wd[2].y, wd[3].y};
-      quad4<false>(su, idx, lane_e, xw + 4);
-    }
-    {
-      const uint32_t idx[4] = {wd[0].z, wd[1].z, wd[2].z, wd[3].z};
-      quad4<false>(su, idx, lane_e, xw + 8);
-    }
-    {
-      const uint32_t idx[4] = {wd[0].w, wd[1].w, wd[2].w, wd[3].w};
-      quad4<false>(su, idx, lane_e, xw + 12);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      load_xq<M>(xq, xa + 16u * j, xstride);
+      const uint32_t idx[4] = {j == 0 ? wd[0].x : j == 1 ? wd[0].y : j == 2 ? wd[0].z : wd[0].w,
+                               j == 0 ? wd[1].x : j == 1 ? wd[1].y : j == 2 ? wd[1].z : wd[1].w,
+                               j == 0 ? wd[2].x : j == 1 ? wd[2].y : j == 2 ? wd[2].z : wd[2].w,
+                               j == 0 ? wd[3].x : j == 1 ? wd[3].y : j == 2 ? wd[3].z : wd[3].w};
+      if (j == 0)
+        quad4<true, M>(su, idx, lane_e, xq);
+      else
+        quad4<false, M>(su, idx, lane_e, xq);
     }
   } else {
     // lo u32 j goes with hi u32 j; lo word 1 reads its hi fields two bits up
@@ -346,11 +358,13 @@ __device__ __forceinline__ void unit_partial_m1(float (&su)[4], const uint4 (&wd
         e[i] = (l & 0x0F0F0F0Fu) | (h & 0xF0F0F0F0u);
         o[i] = (l & 0xF0F0F0F0u) | (h & 0x0F0F0F0Fu);
       }
+      load_xq<M>(xq, xa + 32u * j, xstride);
       if (j == 0)
-        quad4<true>(su, e, lane_e, xw);
+        quad4<true, M>(su, e, lane_e, xq);
       else
-        quad4<false>(su, e, lane_e, xw + 8);
-      quad4<false>(su, o, lane_o, xw + 8 * j + 4);
+        quad4<false, M>(su, e, lane_e, xq);
+      load_xq<M>(xq, xa + 32u * j + 16u, xstride);
+      quad4<false, M>(su, o, lane_o, xq);
     }
   }
 }
@@ -361,50 +375,53 @@ __device__ __forceinline__ void unit_partial_m1(float (&su)[4], const uint4 (&wd
 constexpr uint32_t kXChunkBytes = 64;
 constexpr uint32_t kXGroupBytes = 4 * kXChunkBytes;
 
-// The lane's 32 activations of one group (16 bf16x2 words) from address xa.
-__device__ __forceinline__ void load_x_m1(uint32_t (&xw)[16], uint32_t xa) {
-#pragma unroll
-  for (int v = 0; v < 4; ++v)
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(xw[4 * v]), "=r"(xw[4 * v + 1]), "=r"(xw[4 * v + 2]), "=r"(xw[4 * v + 3])
-                 : "r"(xa + 16u * v));
-}
-
-
-// Shared-window layout of the M = 1 kernel, in addresses of the CTA's shared
-// window (the block's own static shared memory and the system's reserved
-// bytes lie below kSbaseMax, where dynamic shared memory begins):
-//   [kSlotsAt, kXLoAt)           warp slots, [NW][2][32] fp32
-//   [kXLoAt, kPageAt)            activations of groups [0, gb)
+// Shared-window layout of the small-batch kernel, in addresses of the CTA's
+// shared window (the block's own static shared memory and the system's
+// reserved bytes lie below kSbaseMax, where dynamic shared memory begins):
+//   [kSlotsAt, xlo_at(M))        warp slots, [NW][2][M][32] fp32
+//   [xlo_at(M), kPageAt)         activations of groups [0, gb), batch row by
+//                                batch row (gb groups each)
 //   [kPageAt, kAboveAt)          the lookup table, on its own 64 KB page
-//   [kAboveAt, ...)              activations of groups [gb, G), then each
-//                                warp's first tile, copied in by the bulk
-//                                copy engine
-// The dynamic size kAboveAt + m1_above_bytes therefore covers the window up
-// to the end of the staging area whatever the exact start (<= kSbaseMax).
+//   [kAboveAt, ...)              activations of groups [gb, G), batch row by
+//                                batch row, then each warp's first tile, all
+//                                copied in by the bulk copy engine
+// The dynamic size kAboveAt + small_above_bytes therefore covers the window
+// up to the end of the staging area whatever the exact start (<= kSbaseMax).
 constexpr uint32_t kSbaseMax = 4096;
 constexpr uint32_t kSlotsAt = kSbaseMax;
-constexpr uint32_t kXLoAt = kSlotsAt + kM1Warps * 2 * kStrip * 4;
 constexpr uint32_t kPageAt = 0x10000;
 constexpr uint32_t kAboveAt = 0x20000;
 constexpr uint64_t kM1WaitNs = 2000000000ull;  // bounded waits: 2 s
 
-__host__ __device__ constexpr uint32_t x_groups_below(uint32_t G) {
-  return G < (kPageAt - kXLoAt) / kXGroupBytes ? G : (kPageAt - kXLoAt) / kXGroupBytes;
+__host__ __device__ constexpr uint32_t xlo_at(int M) {
+  return kSlotsAt + uint32_t(kM1Warps * 2 * M * kStrip * 4);
 }
-__host__ __device__ constexpr uint32_t m1_above_bytes(uint32_t G, int bits) {
-  return (G - x_groups_below(G)) * kXGroupBytes + kM1Warps * uint32_t(tile_bytes(bits));
+__host__ __device__ constexpr uint32_t x_groups_below(uint32_t G, int M) {
+  return G < (kPageAt - xlo_at(M)) / (kXGroupBytes * M) ? G
+                                                        : (kPageAt - xlo_at(M)) / (kXGroupBytes * M);
+}
+__host__ __device__ constexpr uint32_t small_above_bytes(uint32_t G, int M, int bits) {
+  return (G - x_groups_below(G, M)) * kXGroupBytes * M + kM1Warps * uint32_t(tile_bytes(bits));
 }
 
-template <int BITS>
-__global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
+// Prefetch depth: tiles in registers ahead of the one being consumed.  Three
+// rotating buffers for M <= 2; two for larger batches, whose accumulators
+// need the registers.
+template <int M>
+struct SmallCfg {
+  static constexpr int NB = M <= 2 ? 3 : 2;
+};
+
+template <int BITS, int M>
+__global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a) {
+  constexpr int NB = SmallCfg<M>::NB;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ WarpTable<kM1Warps> wt;
   __shared__ __align__(8) uint64_t bars[1 + kM1Warps];  // activations, then one per warp's tile
   __shared__ int abort_flag;
   const uint32_t sbase = sm_addr(smem);
   const uint32_t G = uint32_t(a.G);
-  const uint32_t gb = x_groups_below(G);
+  const uint32_t gb = x_groups_below(G, M);
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   // The layout needs dynamic shared memory to begin below kSbaseMax; the
   // host allocates for that.  Should it not, nothing is touched.
@@ -415,7 +432,9 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   float* slots = reinterpret_cast<float*>(smem + (kSlotsAt - sbase));
   uint8_t* lut = smem + (kPageAt - sbase);
   constexpr int TB = tile_bytes(BITS);
-  const uint32_t stage_at = kAboveAt + (G - gb) * kXGroupBytes + uint32_t(wl) * TB;
+  const uint32_t x_lo = xlo_at(M), x_lo_stride = gb * kXGroupBytes;
+  const uint32_t x_hi_stride = (G - gb) * kXGroupBytes;
+  const uint32_t stage_at = kAboveAt + x_hi_stride * M + uint32_t(wl) * TB;
   const uint32_t xbar = sm_addr(&bars[0]), tbar = sm_addr(&bars[1 + wl]);
 
   const Span sp = cta_span(a, blockIdx.x);
@@ -427,11 +446,6 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   const int q = lane >> 3, rq = lane & 7;
   const uint8_t* tile0 = a.packed + (uint64_t(first_strip) * G + sp.ga + g_first) * TB;
 
-  // Activations and each warp's first tile come in through the bulk copy
-  // engine (no load instructions, so the table build below does not queue
-  // behind them): the activations in one or two runs (below and above the
-  // table's page), counted in bytes on bars[0]; the tile whole into the
-  // warp's staging area on its own barrier.
   // Everything above reads only the launch parameters.  The kernel is
   // launched as a programmatic dependent of the work before it on the
   // stream, so it may start while that work finishes; global memory is
@@ -439,20 +453,32 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   // may likewise start early (it waits the same way).
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // Activations and each warp's first tile come in through the bulk copy
+  // engine (no load instructions, so the table build below does not queue
+  // behind them): each batch row's activations in one or two runs (below and
+  // above the table's page), counted in bytes on bars[0]; the tile whole into
+  // the warp's staging area on its own barrier.
   if (threadIdx.x == 0) abort_flag = 0;
   if (lane == 0) {
     if (wl == 0) sm100::mbar_init(xbar, 1);
     sm100::mbar_init(tbar, 1);
     sm100::mbar_fence_init();
-    if (wl == 0) sm100::mbar_expect_tx(xbar, uint32_t(a.K) * 2u);
+    if (wl == 0) sm100::mbar_expect_tx(xbar, uint32_t(M) * uint32_t(a.K) * 2u);
     if (u0 < u1) {
       sm100::mbar_expect_tx(tbar, uint32_t(TB));
       sm100::bulk_g2s(stage_at, tile0, uint32_t(TB), tbar);
     }
   }
   if (threadIdx.x == 0) {
-    sm100::bulk_g2s(kXLoAt, a.x, gb * kXGroupBytes, xbar);
-    if (gb < G) sm100::bulk_g2s(kAboveAt, a.x + uint64_t(gb) * kGroup, (G - gb) * kXGroupBytes, xbar);
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const uint16_t* xm = a.x + uint64_t(m) * a.K;
+      sm100::bulk_g2s(x_lo + uint32_t(m) * x_lo_stride, xm, x_lo_stride, xbar);
+      if (gb < G)
+        sm100::bulk_g2s(kAboveAt + uint32_t(m) * x_hi_stride, xm + uint64_t(gb) * kGroup,
+                        x_hi_stride, xbar);
+    }
   }
 
   // Fetch cursor: the lane's bytes of the next tile to load, the scale of
@@ -492,17 +518,18 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   // Lane t holds codebook[t mod 2^BITS]; the table is built from it with
   // shuffles, so no shared staging (and no barrier) precedes the build.
   const uint32_t cbv = __ldg(a.codebook + (lane & ((1 << BITS) - 1)));
-  uint4 b0[4], b1[4], b2[4];
-  uint16_t s0[4], s1[4], s2[4];
+  uint4 buf[NB][4];
+  uint16_t sbuf[NB][4];
   if (u0 < u1) {
-    fetch_scales(s0);  // the words of tile u0 are on their way to the staging area
+    fetch_scales(sbuf[0]);  // the words of tile u0 are on their way to the staging area
     advance();
   }
   fill_warp_table<kM1Warps>(wt, sp);
   build_lut_shfl<BITS>(lut, cbv);
-  // the next two tiles go straight to registers
-  if (u0 + 1 < u1) fetch(b1, s1);
-  if (u0 + 2 < u1) fetch(b2, s2);
+  // the next tiles go straight to registers
+#pragma unroll
+  for (int t = 1; t < NB; ++t)
+    if (u0 + t < u1) fetch(buf[t], sbuf[t]);
   __syncthreads();  // table, warp table, barrier initialisation
 
   // Activations and the first tile in; a wait that runs out marks the call
@@ -518,13 +545,13 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     for (int i = 0; i < 4; ++i) {
       if (BITS == 4) {
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(b0[i].x), "=r"(b0[i].y), "=r"(b0[i].z), "=r"(b0[i].w)
+                     : "=r"(buf[0][i].x), "=r"(buf[0][i].y), "=r"(buf[0][i].z), "=r"(buf[0][i].w)
                      : "r"(t + 128u * i));
       } else {
         asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                     : "=r"(b0[i].x), "=r"(b0[i].y) : "r"(t + 128u * i));
+                     : "=r"(buf[0][i].x), "=r"(buf[0][i].y) : "r"(t + 128u * i));
         asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                     : "=r"(b0[i].z), "=r"(b0[i].w) : "r"(t + hi_delta + 128u * i));
+                     : "=r"(buf[0][i].z), "=r"(buf[0][i].w) : "r"(t + hi_delta + 128u * i));
       }
     }
   }
@@ -533,57 +560,73 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
   const uint32_t page = (kPageAt >> 16) << 8;
   const uint32_t lane_e = page | uint32_t(lane) * 4u, lane_o = page | (128u + uint32_t(lane) * 4u);
   const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
-  float* my_slots = slots + wl * 2 * kStrip;
+  float* my_slots = slots + wl * 2 * M * kStrip;
   int rows[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) rows[i] = rq + 8 * i;
-  // activation address of (group g, chunk q): below the page for g < gb
+  // activation address of (group g, chunk q) for batch row 0, and the step
+  // to the next batch row: below the page for g < gb, above it otherwise
   const uint32_t xq = uint32_t(q) * kXChunkBytes;
   auto x_at = [&](uint32_t g) {
-    return (g < gb ? kXLoAt + g * kXGroupBytes : kAboveAt + (g - gb) * kXGroupBytes) + xq;
+    return (g < gb ? x_lo + g * kXGroupBytes : kAboveAt + (g - gb) * kXGroupBytes) + xq;
   };
 
   if (u0 < u1 && ok) {
-    // Tiles are prefetched two ahead into three rotating buffers.
     uint32_t strip = first_strip, g = g_first;
     const uint32_t xa_w = x_at(sp.ga);  // first group of the window
+    const uint32_t xs_w = sp.ga < gb ? x_lo_stride : x_hi_stride;
     uint32_t xa = x_at(sp.ga + g_first);
-    const uint32_t xa_hi = x_at(gb);    // first group above the page
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    // consume the tile u held in (wd, sv); refill that buffer with tile u + 3
+    uint32_t xs = sp.ga + g_first < gb ? x_lo_stride : x_hi_stride;
+    const uint32_t xa_hi = x_at(gb);     // first group above the page
+    float acc[4][M];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int m = 0; m < M; ++m) acc[i][m] = 0.0f;
+    // consume the tile u held in (wd, sv); refill that buffer with tile u + NB
     auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
-      uint32_t xw[16];
-      load_x_m1(xw, xa);
-      float su[4];
-      unit_partial_m1<BITS>(su, wd, lane_e, lane_o, hi_shift, xw);
+      float su[4][M];
+      unit_partial<BITS, M>(su, wd, lane_e, lane_o, hi_shift, xa, xs);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = fmaf(__uint_as_float(uint32_t(sv[i]) << 16), su[i], acc[i]);
-      if (u + 3 < u1) fetch(wd, sv);
+      for (int i = 0; i < 4; ++i) {
+        const float s = __uint_as_float(uint32_t(sv[i]) << 16);
+#pragma unroll
+        for (int m = 0; m < M; ++m) acc[i][m] = fmaf(s, su[i][m], acc[i][m]);
+      }
+      if (u + NB < u1) fetch(wd, sv);
       if (g + 1 == sp.W || u + 1 == u1) {
-        float vals[4][1];
+        float vals[4][M];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float v = acc[i];
-          v += __shfl_xor_sync(0xffffffffu, v, 8);
-          v += __shfl_xor_sync(0xffffffffu, v, 16);
-          vals[i][0] = v;
-          acc[i] = 0.0f;
-        }
-        deposit_strip<1, 4>(a, sp, strip, u0, u1, first_strip, vals, rows, q == 0, my_slots);
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            float v = acc[i][m];
+            v += __shfl_xor_sync(0xffffffffu, v, 8);
+            v += __shfl_xor_sync(0xffffffffu, v, 16);
+            vals[i][m] = v;
+            acc[i][m] = 0.0f;
+          }
+        deposit_strip<M, 4>(a, sp, strip, u0, u1, first_strip, vals, rows, q == 0, my_slots);
         ++strip;
         g = 0;
         xa = xa_w;
+        xs = xs_w;
       } else {
         ++g;
-        xa = sp.ga + g == gb ? xa_hi : xa + kXGroupBytes;
+        if (sp.ga + g == gb) {
+          xa = xa_hi;
+          xs = x_hi_stride;
+        } else {
+          xa += kXGroupBytes;
+        }
       }
     };
-    for (uint32_t u = u0; u < u1; u += 3) {
-      step(b0, s0, u);
-      if (u + 1 >= u1) break;
-      step(b1, s1, u + 1);
-      if (u + 2 >= u1) break;
-      step(b2, s2, u + 2);
+    for (uint32_t u = u0; u < u1; u += NB) {
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+        if (t > 0 && u + t >= u1) break;
+        step(buf[t], sbuf[t], u + t);
+      }
     }
   }
   __syncthreads();
@@ -595,7 +638,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_m1_kernel(GemvArgs a) {
     if (threadIdx.x == 0) sm100::mbar_wait(xbar, 0, &again, kM1WaitNs);
     return;
   }
-  cta_finish<1, kM1Warps>(a, sp, slots, wt);
+  cta_finish<M, kM1Warps>(a, sp, slots, wt);
 }
 
 // --------------------------------------------------------------------------
@@ -825,15 +868,26 @@ static void apply_plan(GemvArgs& a, int num_sms) {
   a.nh = pl.nh;
 }
 
-static int64_t m1_smem(int64_t K, int bits) {
-  return int64_t(kAboveAt) + m1_above_bytes(uint32_t(K / kGroup), bits);
+template <int BITS, int M>
+static cudaError_t launch_gen(GemvArgs a, int num_sms, cudaStream_t stream) {
+  static SmemGrant grant;
+  const int smem = kLutBytes + kGenWarps * 2 * M * kStrip * 4;
+  cudaError_t err = grant_smem(gemv_kernel<BITS, M>, grant, smem);
+  if (err != cudaSuccess) return err;
+  apply_plan(a, num_sms);
+  gemv_kernel<BITS, M><<<unsigned(a.C), kGenWarps * 32, smem, stream>>>(a);
+  return cudaGetLastError();
 }
 
-template <int BITS>
-static cudaError_t launch_m1(GemvArgs a, int num_sms, cudaStream_t stream) {
+static int64_t small_smem(int64_t K, int M, int bits) {
+  return int64_t(kAboveAt) + small_above_bytes(uint32_t(K / kGroup), M, bits);
+}
+
+template <int BITS, int M>
+static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
   static SmemGrant grant;
-  const int smem = int(m1_smem(a.K, BITS));
-  cudaError_t err = grant_smem(gemv_m1_kernel<BITS>, grant, smem);
+  const int smem = int(small_smem(a.K, M, BITS));
+  cudaError_t err = grant_smem(gemv_small_kernel<BITS, M>, grant, smem);
   if (err != cudaSuccess) return err;
   apply_plan(a, num_sms);
   // programmatic dependent launch: the kernel's prologue (launch parameters,
@@ -848,30 +902,26 @@ static cudaError_t launch_m1(GemvArgs a, int num_sms, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_m1_kernel<BITS>, a);
+  return cudaLaunchKernelEx(&cfg, gemv_small_kernel<BITS, M>, a);
 }
 
+// The small-batch kernel when its shared-memory layout fits, else the
+// thread-per-row kernel.
 template <int BITS, int M>
-static cudaError_t launch_gen(GemvArgs a, int num_sms, cudaStream_t stream) {
-  static SmemGrant grant;
-  const int smem = kLutBytes + kGenWarps * 2 * M * kStrip * 4;
-  cudaError_t err = grant_smem(gemv_kernel<BITS, M>, grant, smem);
-  if (err != cudaSuccess) return err;
-  apply_plan(a, num_sms);
-  gemv_kernel<BITS, M><<<unsigned(a.C), kGenWarps * 32, smem, stream>>>(a);
-  return cudaGetLastError();
+static cudaError_t launch_m(const GemvArgs& a, int num_sms, cudaStream_t s) {
+  if (small_smem(a.K, M, BITS) <= kMaxSmemPerBlock - 1024) return launch_small<BITS, M>(a, num_sms, s);
+  return launch_gen<BITS, M>(a, num_sms, s);
 }
+
 
 template <int BITS>
 static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream_t s) {
   switch (M) {
-    case 1:
-      // the M = 1 kernel keeps all of x in shared memory next to the table
-      if (m1_smem(a.K, BITS) <= kMaxSmemPerBlock - 1024) return launch_m1<BITS>(a, num_sms, s);
-      return launch_gen<BITS, 1>(a, num_sms, s);
-    case 2: return launch_gen<BITS, 2>(a, num_sms, s);
-    case 3: return launch_gen<BITS, 3>(a, num_sms, s);
-    case 4: return launch_gen<BITS, 4>(a, num_sms, s);
+    // the small-batch kernel keeps all of x in shared memory next to the table
+    case 1: return launch_m<BITS, 1>(a, num_sms, s);
+    case 2: return launch_m<BITS, 2>(a, num_sms, s);
+    case 3: return launch_m<BITS, 3>(a, num_sms, s);
+    case 4: return launch_m<BITS, 4>(a, num_sms, s);
     case 5: return launch_gen<BITS, 5>(a, num_sms, s);
     case 6: return launch_gen<BITS, 6>(a, num_sms, s);
     case 7: return launch_gen<BITS, 7>(a, num_sms, s);
