@@ -22,20 +22,16 @@
 //    does not depend on which.
 // Results therefore do not depend on timing.
 //
-// M = 1 kernel.  Lane t of a warp owns the k-chunk q = t >> 3 (32 codes,
-// k = 128 g + 32 q ..) of the four rows (t & 7) + 8 i, i = 0..3, of the
-// strip (the 8 lanes of a quarter-warp share q, so activation reads are
-// broadcasts).  Its 32 activations stay in registers (bf16 pairs) and serve
-// four rows; each code pair costs one byte permute (forming the table
-// address), one conflict-free shared load and two fused multiply-adds with
-// bf16 multiplicands and fp32 accumulators (a bf16 x bf16 product is exact in
+// Small-batch kernel (M = 1..4).  Lane t of a warp owns the k-chunk
+// q = t >> 3 (32 codes, k = 128 g + 32 q ..) of the four rows (t & 7) + 8 i,
+// i = 0..3, of the strip (the 8 lanes of a quarter-warp share q, so
+// activation reads are broadcasts).  Each code pair costs one byte permute
+// (forming the table address) and one conflict-free shared load, shared by
+// the M batch rows, then two fused multiply-adds per batch row with bf16
+// multiplicands and an fp32 accumulator (a bf16 x bf16 product is exact in
 // fp32, so this is the fp32 product of the widened values).  The four lanes
-// of a row add their sums at the end of the strip.
-//
-// M = 2..16 kernel.  Lane r owns row 32 * strip + r and reads its 16-byte
-// words with coalesced 512-byte warp loads; activations come from global
-// memory through L1.  (Batches of more than one row are a small dense
-// contraction; the tensor-core kernel covers them too.)
+// of a row add their sums at the end of the strip.  Larger batches go to the
+// tensor-core kernel (launch_gemv).
 #include <algorithm>
 
 #include "lutq_common.cuh"
@@ -49,7 +45,6 @@ constexpr int kMaxCtas = 512;           // bounds the workspace
 #define LUTQ_M1_WARPS 16
 #endif
 constexpr int kM1Warps = LUTQ_M1_WARPS; // warps per CTA, M = 1 kernel
-constexpr int kGenWarps = 16;           // warps per CTA, generic kernel
 constexpr int kMaxSmemPerBlock = 227 * 1024;
 
 struct GemvArgs {
@@ -218,15 +213,6 @@ __device__ void cta_finish(const GemvArgs& a, const Span& p, const float* all_sl
   }
 }
 
-// acc += (lo, hi) * (x0, x1) elementwise, one packed fp32x2 FMA.
-__device__ __forceinline__ void ffma2(float2& acc, float lo, float hi, float x0, float x1) {
-  uint64_t a, w, xv;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(acc.x), "f"(acc.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(w) : "f"(lo), "f"(hi));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(x0), "f"(x1));
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(w), "l"(xv));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(acc.x), "=f"(acc.y) : "l"(a));
-}
 
 // --------------------------------------------------------------------------
 // M = 1
@@ -642,131 +628,6 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 }
 
 // --------------------------------------------------------------------------
-// M = 2..16 (thread per row)
-// --------------------------------------------------------------------------
-
-template <int M>
-__device__ __forceinline__ void run4_global_x(float2 (&part)[M], const uint32_t (&lv)[4], int k,
-                                              const uint16_t* x, int64_t K) {
-#pragma unroll
-  for (int m = 0; m < M; ++m) {
-    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + m * K + k));
-    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-      ffma2(part[m], bf16_lo_to_f32(lv[p]), bf16_hi_to_f32(lv[p]), bf16_lo_to_f32(xw[p]),
-            bf16_hi_to_f32(xw[p]));
-  }
-}
-
-template <int BITS, int M>
-__device__ __forceinline__ void unit_partial_gen(float2 (&part)[M], const uint4 (&wd)[4],
-                                                 uint32_t lut_base, uint32_t off_e,
-                                                 uint32_t off_o, int kg, const uint16_t* x,
-                                                 int64_t K) {
-  uint32_t lv[4];
-  if (BITS == 4) {
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const uint32_t v[4] = {wd[w].x, wd[w].y, wd[w].z, wd[w].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        lookup4(lv, v[j], lut_base, off_e);
-        run4_global_x<M>(part, lv, kg + 32 * w + 8 * j, x, K);
-      }
-    }
-  } else {
-    const uint32_t L0[4] = {wd[0].x, wd[0].y, wd[0].z, wd[0].w};
-    const uint32_t L1[4] = {wd[1].x, wd[1].y, wd[1].z, wd[1].w};
-    const uint32_t H[4] = {wd[2].x, wd[2].y, wd[2].z, wd[2].w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const W3Index ix = w3_indices(L0[j], L1[j], H[j]);
-      lookup4(lv, ix.e0, lut_base, off_e);
-      run4_global_x<M>(part, lv, kg + 16 * j, x, K);
-      lookup4(lv, ix.o0, lut_base, off_o);
-      run4_global_x<M>(part, lv, kg + 16 * j + 8, x, K);
-      lookup4(lv, ix.e1, lut_base, off_e);
-      run4_global_x<M>(part, lv, kg + 64 + 16 * j, x, K);
-      lookup4(lv, ix.o1, lut_base, off_o);
-      run4_global_x<M>(part, lv, kg + 64 + 16 * j + 8, x, K);
-    }
-  }
-}
-
-template <int BITS>
-__device__ __forceinline__ void load_unit_row(uint4 (&wd)[4], const uint8_t* tile, int lane) {
-  constexpr int WPR = words_per_row(BITS);
-#pragma unroll
-  for (int w = 0; w < WPR; ++w) wd[w] = ld_stream_v4(tile + (32 * w + lane) * kWordBytes);
-}
-
-template <int BITS, int M>
-__global__ void __launch_bounds__(kGenWarps * 32, 1) gemv_kernel(GemvArgs a) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ uint16_t cbs[16];
-  __shared__ uint32_t pairs[512];
-  __shared__ WarpTable<kGenWarps> wt;
-  float* slots = reinterpret_cast<float*>(smem + kLutBytes);  // [NW][2][M][32]
-  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  const uint32_t lut_base = sm_addr(smem);
-  const Span sp = cta_span(a, blockIdx.x);
-  if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
-  fill_warp_table<kGenWarps>(wt, sp);
-  __syncthreads();
-  build_lut_copies<BITS>(smem, cbs, pairs);
-  __syncthreads();
-
-  // the warp's positions [u0, u1) of the CTA's unit sequence
-  const uint32_t u0 = sp.v0 + wt.wb[wl], u1 = sp.v0 + wt.wb[wl + 1];
-  const uint32_t off_e = uint32_t(lane) * 4u, off_o = 128u + uint32_t(lane) * 4u;
-  constexpr int TB = tile_bytes(BITS);
-  const int rows[1] = {lane};
-  float* my_slots = slots + wl * 2 * M * kStrip;
-
-  if (u0 < u1) {
-    const uint32_t first_strip = wt.ws[wl];
-    int64_t strip = first_strip;
-    int64_t g = u0 % sp.W;  // place in the window: group sp.ga + g
-    float acc[1][M];
-#pragma unroll
-    for (int m = 0; m < M; ++m) acc[0][m] = 0.0f;
-    uint4 cur[4], nxt[4];
-    // tile of (strip, window place) and the one after it in the sequence
-    auto tile = [&](int64_t st, int64_t gw) { return a.packed + (st * a.G + sp.ga + gw) * TB; };
-    load_unit_row<BITS>(cur, tile(strip, g), lane);
-    for (uint32_t u = u0; u < u1; ++u) {
-      const bool last_in_window = g + 1 == sp.W;
-      if (u + 1 < u1)
-        load_unit_row<BITS>(nxt, last_in_window ? tile(strip + 1, 0) : tile(strip, g + 1), lane);
-      const int64_t row = strip * kStrip + lane;
-      const float s = __uint_as_float(uint32_t(a.scales[row * a.G + sp.ga + g]) << 16);
-      float2 part[M];
-#pragma unroll
-      for (int m = 0; m < M; ++m) part[m] = make_float2(0.0f, 0.0f);
-      unit_partial_gen<BITS, M>(part, cur, lut_base, off_e, off_o, int((sp.ga + g) * kGroup),
-                                a.x, a.K);
-#pragma unroll
-      for (int m = 0; m < M; ++m) acc[0][m] = fmaf(s, part[m].x + part[m].y, acc[0][m]);
-      if (last_in_window || u + 1 == u1) {
-        deposit_strip<M, 1>(a, sp, uint32_t(strip), u0, u1, first_strip, acc, rows, true,
-                            my_slots);
-#pragma unroll
-        for (int m = 0; m < M; ++m) acc[0][m] = 0.0f;
-        ++strip;
-        g = 0;
-      } else {
-        ++g;
-      }
-#pragma unroll
-      for (int w = 0; w < 4; ++w) cur[w] = nxt[w];
-    }
-  }
-  __syncthreads();
-  cta_finish<M, kGenWarps>(a, sp, slots, wt);
-}
-
-// --------------------------------------------------------------------------
 // host side
 // --------------------------------------------------------------------------
 
@@ -868,16 +729,6 @@ static void apply_plan(GemvArgs& a, int num_sms) {
   a.nh = pl.nh;
 }
 
-template <int BITS, int M>
-static cudaError_t launch_gen(GemvArgs a, int num_sms, cudaStream_t stream) {
-  static SmemGrant grant;
-  const int smem = kLutBytes + kGenWarps * 2 * M * kStrip * 4;
-  cudaError_t err = grant_smem(gemv_kernel<BITS, M>, grant, smem);
-  if (err != cudaSuccess) return err;
-  apply_plan(a, num_sms);
-  gemv_kernel<BITS, M><<<unsigned(a.C), kGenWarps * 32, smem, stream>>>(a);
-  return cudaGetLastError();
-}
 
 static int64_t small_smem(int64_t K, int M, int bits) {
   return int64_t(kAboveAt) + small_above_bytes(uint32_t(K / kGroup), M, bits);
@@ -905,36 +756,29 @@ static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, gemv_small_kernel<BITS, M>, a);
 }
 
-// The small-batch kernel when its shared-memory layout fits, else the
-// thread-per-row kernel.
-template <int BITS, int M>
-static cudaError_t launch_m(const GemvArgs& a, int num_sms, cudaStream_t s) {
-  if (small_smem(a.K, M, BITS) <= kMaxSmemPerBlock - 1024) return launch_small<BITS, M>(a, num_sms, s);
-  return launch_gen<BITS, M>(a, num_sms, s);
-}
+cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* scales,
+                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
+                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
 
+// Batches up to kMaxSmallBatch run on the CUDA cores when their activations
+// fit the small-batch kernel's shared memory.  Larger batches are a dense
+// contraction for the CUDA cores (each table lookup feeds 2M multiply-adds;
+// from M = 5 on that costs more than the tensor-core kernel's whole pass),
+// so they, and over-long rows, take the tcgen05 kernel of lutq_gemm.
+constexpr int kMaxSmallBatch = 4;
+
+template <int BITS>
+static bool small_fits(int64_t M, int64_t K) {
+  return M >= 1 && M <= kMaxSmallBatch && small_smem(K, int(M), BITS) <= kMaxSmemPerBlock - 1024;
+}
 
 template <int BITS>
 static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream_t s) {
   switch (M) {
-    // the small-batch kernel keeps all of x in shared memory next to the table
-    case 1: return launch_m<BITS, 1>(a, num_sms, s);
-    case 2: return launch_m<BITS, 2>(a, num_sms, s);
-    case 3: return launch_m<BITS, 3>(a, num_sms, s);
-    case 4: return launch_m<BITS, 4>(a, num_sms, s);
-    case 5: return launch_gen<BITS, 5>(a, num_sms, s);
-    case 6: return launch_gen<BITS, 6>(a, num_sms, s);
-    case 7: return launch_gen<BITS, 7>(a, num_sms, s);
-    case 8: return launch_gen<BITS, 8>(a, num_sms, s);
-    case 9: return launch_gen<BITS, 9>(a, num_sms, s);
-    case 10: return launch_gen<BITS, 10>(a, num_sms, s);
-    case 11: return launch_gen<BITS, 11>(a, num_sms, s);
-    case 12: return launch_gen<BITS, 12>(a, num_sms, s);
-    case 13: return launch_gen<BITS, 13>(a, num_sms, s);
-    case 14: return launch_gen<BITS, 14>(a, num_sms, s);
-    case 15: return launch_gen<BITS, 15>(a, num_sms, s);
-    case 16: return launch_gen<BITS, 16>(a, num_sms, s);
-    default: return cudaErrorInvalidValue;
+    case 1: return launch_small<BITS, 1>(a, num_sms, s);
+    case 2: return launch_small<BITS, 2>(a, num_sms, s);
+    case 3: return launch_small<BITS, 3>(a, num_sms, s);
+    default: return launch_small<BITS, 4>(a, num_sms, s);
   }
 }
 
@@ -956,6 +800,10 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   a.C = 0;
   // unit indices and range arithmetic are 32-bit (U * CTAs < 2^32)
   if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
+  const bool small = bits == 4 ? small_fits<4>(M, K) : small_fits<3>(M, K);
+  if (!small)
+    return launch_gemm(x, M, packed, scales, codebook, bits, N, K, y, workspace, dev_status,
+                       num_sms, stream);
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
                    : launch_bits<3>(a, int(M), num_sms, stream);
 }

