@@ -424,7 +424,7 @@ def run_lutq(args, world, rank, local):
                      "frac": gbs_rank / hbm_peak, "peak_source": peak_kind,
                      "bytes_per_launch": nbytes, "traffic": ncu_traffic(kernel_key,
                                                                     GEMM_SOURCES if use_gemm else GEMV_SOURCES),
-                     "kernel": "lutq::gemv_kernel" if not use_gemm else "lutq::gemm_kernel"},
+                     "kernel": "lutq::gemv_small_kernel" if not use_gemm else "lutq::gemm_kernel"},
         "pct_of_8TBs": gbs_rank / 8000.0,
         "plain_launch_gbs": plain_gbs,
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": m * k * 2,
