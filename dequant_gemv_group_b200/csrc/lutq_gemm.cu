@@ -13,9 +13,9 @@
 //   warps 4-7  promote: read the group's fp32 partial D[row, batch] from
 //              tensor memory, add s[row, g] * partial to registers, and write
 //              y (or a split partial) when the row tile's range ends.
-//   warp 8     loads: the tile's packed words (four contiguous 1-D bulk
-//              copies, one per 32-row strip) and the activations' 128-wide K
-//              slice (two 2-D tensor-map copies, 128-byte swizzle).
+//   warp 8     loads the activations' 128-wide K slice (two 2-D tensor-map
+//              copies, 128-byte swizzle); the dequantize warps load their
+//              rows' packed words themselves, straight into registers.
 //   warp 9     issues tcgen05.mma kind::f16 (A from tensor memory, B from
 //              shared memory, D fp32 in tensor memory), 8 MMAs of K = 16 per
 //              group into a fresh partial, and commits to the mbarriers.
@@ -48,15 +48,15 @@ constexpr int kTmemCols = 512;
 template <int NT>
 struct GemmCfg {
   static constexpr int XS = NT >= 128 ? 3 : 4;     // activation stages (shared memory)
-  static constexpr int PS = NT >= 128 ? 4 : (NT >= 64 ? 8 : 12);  // packed-tile stages
   static constexpr int XSTAGE = 2 * NT * 128;       // two boxes of NT rows x 128 bytes
   static constexpr int AS = 4;                      // A stages in tensor memory (64 columns each)
   static constexpr int DS = NT >= 128 ? 2 : (NT >= 64 ? 3 : 4);  // partial stages (NT columns)
   static constexpr int DW = NT >= 128 ? 4 : 8;      // dequant warps (8: two per lane quarter)
+  static constexpr int NB = DW == 8 ? 4 : 2;        // units of packed words in flight per lane
   static constexpr int KC = 64 * 4 / DW;            // A columns written per dequant warp
   static constexpr int PG = NT >= 128 ? 2 : 1;      // promotion warp groups
   static constexpr int NC = NT / PG;                // batch columns per promotion warp
-  static constexpr int WARPS = DW + 4 * PG + 3;     // dequant, promote, 2 load, MMA
+  static constexpr int WARPS = DW + 4 * PG + 2;     // dequant, promote, activation load, MMA
   static constexpr int THREADS = 32 * WARPS;
   static constexpr int DCOL = 64 * AS;              // first partial column
   static_assert(DCOL + DS * NT <= kTmemCols, "tensor memory columns");
@@ -208,9 +208,9 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   using Cfg = GemmCfg<NT>;
   constexpr int TB = tile_bytes(BITS);
   constexpr int WPR = words_per_row(BITS);
-  constexpr int XS = Cfg::XS, PS = Cfg::PS, AS = Cfg::AS, DS = Cfg::DS, DW = Cfg::DW;
-  constexpr int PG = Cfg::PG, NC = Cfg::NC;
-  constexpr int W_LOAD = DW + 4 * PG, W_XLOAD = W_LOAD + 1, W_MMA = W_LOAD + 2;
+  constexpr int XS = Cfg::XS, AS = Cfg::AS, DS = Cfg::DS, DW = Cfg::DW;
+  constexpr int PG = Cfg::PG, NC = Cfg::NC, NB = Cfg::NB;
+  constexpr int W_XLOAD = DW + 4 * PG, W_MMA = W_XLOAD + 1;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_sa = smem_addr(smem_raw);
   const uint32_t base_sa = (raw_sa + 1023u) & ~1023u;
@@ -218,11 +218,10 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   uint8_t* lut = base;
   const uint32_t lut_sa = base_sa;
   const uint32_t xst_sa = base_sa + kLutBytes;
-  const uint32_t pst_sa = xst_sa + XS * Cfg::XSTAGE;
-  const uint32_t bar_sa = pst_sa + PS * 4 * TB;
+  const uint32_t bar_sa = xst_sa + XS * Cfg::XSTAGE;
   // barrier ids
-  constexpr int B_XF = 0, B_XE = XS, B_PF = 2 * XS, B_PE = 2 * XS + PS, B_AF = 2 * XS + 2 * PS,
-                B_AE = B_AF + AS, B_DF = B_AE + AS, B_DE = B_DF + DS, NBAR = B_DE + DS;
+  constexpr int B_XF = 0, B_XE = XS, B_AF = 2 * XS, B_AE = B_AF + AS, B_DF = B_AE + AS,
+                B_DE = B_DF + DS, NBAR = B_DE + DS;
   auto bar = [&](int i) { return bar_sa + 8u * uint32_t(i); };
   uint8_t* misc = base + (bar_sa - base_sa) + 8 * NBAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
@@ -234,10 +233,6 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     for (int i = 0; i < XS; ++i) {
       mbar_init(bar(B_XF + i), 1);
       mbar_init(bar(B_XE + i), 1);
-    }
-    for (int i = 0; i < PS; ++i) {
-      mbar_init(bar(B_PF + i), 1);
-      mbar_init(bar(B_PE + i), DW);
     }
     for (int i = 0; i < AS; ++i) {
       mbar_init(bar(B_AF + i), DW);
@@ -271,42 +266,54 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
 
   if (warp < DW) {
     // ---------------------------------------------------------------- dequantize
+    // Lane r of warp w loads its row's packed words itself, NB units ahead,
+    // straight into registers (16-byte loads, 512 contiguous bytes per warp
+    // instruction): a 2 KB bulk copy per strip and unit costs the copy
+    // engine about as much as 16 KB of data, and would hold the kernel to
+    // about a quarter of the HBM bandwidth.
     const int sw = warp & 3, kh = DW == 8 ? (warp >> 2) : 0;
     const uint32_t off_e = uint32_t(lane) * 4u, off_o = 128u + uint32_t(lane) * 4u;
+    constexpr int NWL = DW == 8 ? 2 : WPR;  // 16-byte words per lane and unit
+    // word j of the lane's words: 4-bit, words 2kh, 2kh+1 (DW = 8) or all;
+    // 3-bit, lo word kh and the hi word (DW = 8) or all three
+    auto word_of = [&](int j) { return DW == 8 ? (BITS == 4 ? 2 * kh + j : (j == 0 ? kh : 2)) : j; };
+    UnitPos fp;  // the next unit to fetch
+    fp.init(u0, per_bt, a.G);
+    int fetched = 0;
+    auto fetch = [&](uint4 (&wd)[NWL]) {
+      if (fetched < n && fp.tau * kTileRows + sw * 32 < a.N) {
+        const uint8_t* t = a.packed + ((fp.tau * 4 + sw) * a.G + fp.g) * TB + lane * 16;
+#pragma unroll
+        for (int j = 0; j < NWL; ++j) wd[j] = ld_stream_v4(t + word_of(j) * 512);
+      }
+      ++fetched;
+      fp.next(a.G, a.ntiles);
+    };
+    uint4 ring[NB][NWL];
+#pragma unroll
+    for (int t = 0; t < NB; ++t) fetch(ring[t]);
     UnitPos pos;
     pos.init(u0, per_bt, a.G);
-    for (int i = 0; i < n; ++i, pos.next(a.G, a.ntiles)) {
+    bool ok = true;
+    // decode unit i from wd, refill wd with unit i + NB, hand the tile to the MMA
+    auto step = [&](uint4 (&wd)[NWL], int i) {
       const bool valid = pos.tau * kTileRows + sw * 32 < a.N;
-      const int ps = i % PS;
-      bool ok = mbar_wait(bar(B_PF + ps), uint32_t(i / PS) & 1u, abort_flag, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      const uint32_t src = pst_sa + uint32_t(ps * 4 * TB + sw * TB + lane * 16);
       uint32_t av[Cfg::KC];
-      if (DW == 8) {
-        uint4 wd[2];
-        if (valid) {
-          // 4-bit: words 2kh, 2kh+1; 3-bit: lo word kh and the hi word
-          wd[0] = lds128(src + uint32_t((BITS == 4 ? 2 * kh : kh) * 512));
-          wd[1] = lds128(src + uint32_t((BITS == 4 ? 2 * kh + 1 : 2) * 512));
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_PE + ps));
-        if (valid) decode_group_half<BITS>(reinterpret_cast<uint32_t(&)[32]>(av), wd, kh, lut_sa,
-                                           off_e, off_o);
-      } else {
-        uint4 wd[4];
-        if (valid) {
-#pragma unroll
-          for (int j = 0; j < WPR; ++j) wd[j] = lds128(src + uint32_t(j * 512));
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_PE + ps));
-        if (valid) decode_group_row<BITS>(reinterpret_cast<uint32_t(&)[64]>(av), wd, lut_sa, off_e,
-                                          off_o);
+      if (valid) {
+        if (DW == 8)
+          decode_group_half<BITS>(reinterpret_cast<uint32_t(&)[32]>(av),
+                                  reinterpret_cast<const uint4(&)[2]>(wd), kh, lut_sa, off_e, off_o);
+        else
+          decode_group_row<BITS>(reinterpret_cast<uint32_t(&)[64]>(av),
+                                 reinterpret_cast<const uint4(&)[4]>(wd), lut_sa, off_e, off_o);
       }
+      fetch(wd);
       const int as = i % AS;
       ok = mbar_wait(bar(B_AE + as), (uint32_t(i / AS) & 1u) ^ 1u, abort_flag, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        return;
+      }
       tc_fence_after();
       if (valid) {
         const uint32_t ta = tmem + (uint32_t(sw * 32) << 16) + uint32_t(as * 64 + kh * 32);
@@ -319,8 +326,16 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_AF + as));
+      pos.next(a.G, a.ntiles);
+    };
+    for (int i = 0; i < n && ok; i += NB) {
+#pragma unroll
+      for (int t = 0; t < NB; ++t) {
+        if (i + t >= n || !ok) break;
+        step(ring[t], i + t);
+      }
     }
-  } else if (warp < W_LOAD) {
+  } else if (warp < W_XLOAD) {
     // ---------------------------------------------------------------- promote
     const int sw = warp & 3, pg = (warp - DW) >> 2;
     UnitPos cur;
@@ -375,34 +390,6 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         for (int j = 0; j < NC; ++j) acc[j] = 0.0f;
       }
       cur.next(a.G, a.ntiles);
-    }
-  } else if (warp == W_LOAD) {
-    // ---------------------------------------------------------------- loads
-    // One warp streams the packed tiles and another the activation tiles,
-    // each gated only by its own stages, so weight prefetch runs PS units
-    // ahead regardless of MMA progress (two lanes of one warp would
-    // serialize on each other's waits).
-    if (lane == 0) {
-      int issued = 0;
-      UnitPos pos;
-      pos.init(u0, per_bt, a.G);
-      for (int i = 0; i < n; ++i, pos.next(a.G, a.ntiles)) {
-        const int ps = i % PS;
-        if (!mbar_wait(bar(B_PE + ps), (uint32_t(i / PS) & 1u) ^ 1u, abort_flag, kWaitLimitNs))
-          break;
-        const int64_t srem = (a.N - pos.tau * kTileRows) / 32;
-        const int vs = int(srem < 4 ? srem : 4);
-        mbar_expect_tx(bar(B_PF + ps), uint32_t(vs * TB));
-        for (int s = 0; s < vs; ++s)
-          bulk_g2s(pst_sa + uint32_t(ps * 4 * TB + s * TB),
-                   a.packed + ((pos.tau * 4 + s) * a.G + pos.g) * TB, TB, bar(B_PF + ps));
-        issued = i + 1;
-      }
-      if (*abort_flag) {
-        // let the copies in flight land before the CTA can exit
-        for (int i = (issued > PS ? issued - PS : 0); i < issued; ++i)
-          mbar_drain(bar(B_PF + i % PS), uint32_t(i / PS) & 1u);
-      }
     }
   } else if (warp == W_XLOAD) {
     if (lane == 0) {
@@ -524,7 +511,7 @@ static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
                              cudaStream_t stream) {
   using Cfg = GemmCfg<NT>;
   static int granted[64] = {0};
-  const int smem = 1024 + kLutBytes + Cfg::XS * Cfg::XSTAGE + Cfg::PS * 4 * tile_bytes(BITS) + 512;
+  const int smem = 1024 + kLutBytes + Cfg::XS * Cfg::XSTAGE + 512;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
