@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     lutq_pack,
     lutq_packed_bytes,
     lutq_quantize,
+    lutq_selftest_wait_timeout,
     lutq_status_string,
     lutq_workspace_bytes,
     new_status,

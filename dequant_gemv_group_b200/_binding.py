@@ -43,6 +43,7 @@ _SIGS = {
     "lutq_gemm": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "lutq_gemv_noalloc": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
     "lutq_gemv_plan": (_i32, [_i64, _i64, _i32, _vp]),
+    "lutq_selftest_wait_timeout": (_i32, [_vp, _i64, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -90,6 +91,13 @@ def lutq_gemv_plan(n: int, k: int, num_sms: int) -> dict:
     out = (ctypes.c_int32 * 6)()
     _check(lib.lutq_gemv_plan(n, k, num_sms, out), "lutq_gemv_plan")
     return dict(zip(("C", "kind", "align", "Cm", "T", "nh"), list(out)))
+
+
+def lutq_selftest_wait_timeout(status: torch.Tensor, limit_ns: int) -> None:
+    """Run the kernels' bounded pipeline wait on a barrier nothing completes."""
+    _need(status, torch.int32, "status")
+    _check(lib.lutq_selftest_wait_timeout(status.data_ptr(), int(limit_ns), _stream()),
+           "lutq_selftest_wait_timeout")
 
 
 def lutq_codebook(kind: str, bits: int) -> torch.Tensor:

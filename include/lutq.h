@@ -238,6 +238,20 @@ lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const void* packed,
 lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan);
 
 /*
+ * lutq_selftest_wait_timeout - checks the bound on the kernels' pipeline waits.
+ *
+ * No counterpart in the paper: every mbarrier wait inside lutq_gemv and
+ * lutq_gemm gives up after a time limit (2 s) and reports LUTQ_ERR_TIMEOUT
+ * instead of hanging the GPU.  This call runs that same wait, for limit_ns
+ * nanoseconds, on a barrier that nothing completes: afterwards *dev_status
+ * (device int32, required) holds LUTQ_ERR_TIMEOUT unless it already held an
+ * error, and the stream and context remain usable.  Asynchronous on `stream`.
+ * Returns LUTQ_ERR_INVALID_ARG for a NULL dev_status or limit_ns outside
+ * 1 .. 1e9.
+ */
+lutq_status lutq_selftest_wait_timeout(int32_t* dev_status, int64_t limit_ns, void* stream);
+
+/*
  * lutq_gemm - the same product on the tensor cores (tcgen05), for batches
  * where the problem is a dense contraction (tuned for M >= 32; any M >= 1 is
  * accepted).  Arguments and numerics as lutq_gemv.  dev_status receives
