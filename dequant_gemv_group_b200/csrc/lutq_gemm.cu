@@ -16,7 +16,8 @@
 //   warp 8     loads the activations' 128-wide K slice (two 2-D tensor-map
 //              copies, 128-byte swizzle); the dequantize warps load their
 //              rows' packed words themselves, straight into registers.
-//   warp 9     issues tcgen05.mma kind::f16 (A from tensor memory, B from
+//   warp 9     issues tcgen05.mma (for batch tiles of 16 or 32, warps 9 and
+//              10 take alternate units) kind::f16 (A from tensor memory, B from
 //              shared memory, D fp32 in tensor memory), 8 MMAs of K = 16 per
 //              group into a fresh partial, and commits to the mbarriers.
 // Products are exact (bf16 x bf16) and every group's partial is rescaled in
@@ -56,7 +57,8 @@ struct GemmCfg {
   static constexpr int KC = 64 * 4 / DW;            // A columns written per dequant warp
   static constexpr int PG = NT >= 128 ? 2 : 1;      // promotion warp groups
   static constexpr int NC = NT / PG;                // batch columns per promotion warp
-  static constexpr int WARPS = DW + 4 * PG + 2;     // dequant, promote, activation load, MMA
+  static constexpr int MW = NT <= 32 ? 2 : 1;      // MMA-issuing warps (see the MMA role)
+  static constexpr int WARPS = DW + 4 * PG + 1 + MW;  // dequant, promote, activation load, MMA
   static constexpr int THREADS = 32 * WARPS;
   static constexpr int DCOL = 64 * AS;              // first partial column
   static_assert(DCOL + DS * NT <= kTmemCols, "tensor memory columns");
@@ -210,7 +212,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   constexpr int WPR = words_per_row(BITS);
   constexpr int XS = Cfg::XS, AS = Cfg::AS, DS = Cfg::DS, DW = Cfg::DW;
   constexpr int PG = Cfg::PG, NC = Cfg::NC, NB = Cfg::NB;
-  constexpr int W_XLOAD = DW + 4 * PG, W_MMA = W_XLOAD + 1;
+  constexpr int W_XLOAD = DW + 4 * PG, W_MMA = W_XLOAD + 1;  // MMA warps: W_MMA .. W_MMA + MW - 1
+  constexpr int MW = Cfg::MW;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_sa = smem_addr(smem_raw);
   const uint32_t base_sa = (raw_sa + 1023u) & ~1023u;
@@ -414,10 +417,16 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- MMA
+    // For small batches two warps issue the MMAs, for the even and the odd
+    // units: each waits for its unit's operands and stage while the other's
+    // MMAs run, so the barrier waits (slow while the table lookups load
+    // shared memory) do not leave the tensor pipe idle (16% faster at
+    // N_tile = 16; at 64 and above, where each MMA is long, one warp is
+    // faster).  Each commits its own MMAs.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, NT);
-      int issued = 0;
-      for (int i = 0; i < n; ++i) {
+      int issued = -1;
+      for (int i = warp - W_MMA; i < n; i += MW) {
         const int xs = i % XS, as = i % AS, ds = i % DS;
         if (!mbar_wait(bar(B_XF + xs), uint32_t(i / XS) & 1u, abort_flag, kWaitLimitNs)) break;
         if (!mbar_wait(bar(B_AF + as), uint32_t(i / AS) & 1u, abort_flag, kWaitLimitNs)) break;
@@ -434,12 +443,9 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         mma_commit(bar(B_DF + ds));
         mma_commit(bar(B_AE + as));
         mma_commit(bar(B_XE + xs));
-        issued = i + 1;
+        issued = i;
       }
-      if (*abort_flag && issued > 0) {
-        const int i = issued - 1;
-        mbar_drain(bar(B_DF + i % DS), uint32_t(i / DS) & 1u);
-      }
+      if (*abort_flag && issued >= 0) mbar_drain(bar(B_DF + issued % DS), uint32_t(issued / DS) & 1u);
     }
   }
 
