@@ -656,8 +656,9 @@ static cudaError_t grant_smem(Kernel k, SmemGrant& g, int smem) {
 
 // The work plan (see cta_span).  Costs are in units per CTA, the longest CTA
 // deciding; a plan that splits strips between two CTAs pays kExchangeUnits
-// more for the exchange of the split halves at the end (one atomic round
-// trip to L2, about a unit's worth of streaming per warp).
+// more for the exchange of the split halves at the end and the extra strip
+// ends (measured: main/helper CTAs of 98 units run as fast as whole strips
+// of 112, and 16 + 15 units beat 32 whole ones).
 //  - whole strips, dealt out in equal runs to min(SMs, strips) CTAs;
 //  - equal unit ranges, one CTA per SM, when there are at least as many
 //    strips as CTAs (each range then spans a strip or more, so a strip is
@@ -665,7 +666,7 @@ static cudaError_t grant_smem(Kernel k, SmemGrant& g, int smem) {
 //  - otherwise, main and helper CTAs: one CTA per strip takes its first
 //    G - T groups, and each of the remaining CTAs the last T groups of nh
 //    strips, T balancing the two.
-constexpr int64_t kExchangeUnits = 16;
+constexpr int64_t kExchangeUnits = 15;
 
 struct Plan {
   int C;
