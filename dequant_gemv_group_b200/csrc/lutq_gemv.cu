@@ -32,6 +32,17 @@
 // fp32, so this is the fp32 product of the widened values).  The four lanes
 // of a row add their sums at the end of the strip.  Larger batches go to the
 // tensor-core kernel (launch_gemv).
+//
+// Pipeline.  The kernel is a programmatic dependent of the work before it on
+// the stream.  Its blocks start as multiprocessors free up and, before
+// waiting for that work, compute their split and (the weights are read-only)
+// bring weights into L2: when the plan leaves multiprocessors free, the grid
+// begins with that many prefetching blocks, which land on them while the
+// preceding kernel still runs and prefetch the whole matrix line by line;
+// otherwise each warp prefetches its first tiles.  After the wait each block
+// loads the activations into shared memory and builds the lookup table,
+// and each warp keeps NB tiles (codes and scales) in flight in registers,
+// loaded under one predicate so that the loop has no branch per load.
 #include <algorithm>
 
 #include "lutq_common.cuh"
@@ -61,6 +72,9 @@ struct GemvArgs {
   // aligned if `align`; kind 1 = the first Cm CTAs take groups [0, G - T) of
   // one strip each, the others groups [G - T, G) of nh strips each
   uint32_t kind, align, Cm, T, nh;
+  // The grid's first pf_ctas CTAs only bring the packed matrix and the
+  // scales into L2 (the work goes to CTAs pf_ctas .. pf_ctas + C - 1)
+  uint32_t pf_ctas;
 };
 
 // Part i of `parts` equal shares of [0, total): [range_begin(i), range_begin(i+1)).
@@ -215,8 +229,39 @@ __device__ void cta_finish(const GemvArgs& a, const Span& p, const float* all_sl
 
 
 // --------------------------------------------------------------------------
-// M = 1
+// Small-batch kernel (M = 1..4)
 // --------------------------------------------------------------------------
+
+// Shared-window layout of the small-batch kernel, in addresses of the CTA's
+// shared window (the block's own static shared memory and the system's
+// reserved bytes lie below kSbaseMax, where dynamic shared memory begins):
+//   [kLutAt, kXAt)                 the lookup table, 256 rows of 256 bytes
+//   [kXAt, slots_at(K, M))         activations, bf16 in order, batch row by
+//                                  batch row: a group's four chunks of 32
+//                                  values (64 bytes each) are contiguous
+//   [slots_at(K, M), small_end)    warp slots, [NW][2][M][32] fp32
+// The dynamic size small_end(K, M) therefore covers the window up to the end
+// of the slots whatever the exact start (<= kSbaseMax).  A table address is
+// formed as (row << 8 | column); kLutAt goes into the load's offset.
+constexpr uint32_t kSbaseMax = 4096;
+constexpr uint32_t kLutAt = kSbaseMax;
+constexpr uint32_t kXAt = kLutAt + 0x10000;
+constexpr uint32_t kXChunkBytes = 64;
+constexpr uint32_t kXGroupBytes = 4 * kXChunkBytes;
+
+__host__ __device__ constexpr uint32_t slots_at(uint32_t K, int M) {
+  return kXAt + uint32_t(M) * K * 2u;  // K * 2 is a multiple of 256
+}
+__host__ __device__ constexpr uint32_t small_end(uint32_t K, int M) {
+  return slots_at(K, M) + uint32_t(kM1Warps * 2 * M * kStrip * 4);
+}
+
+// The table entry (a bf16x2 pair of levels) at table address t.
+__device__ __forceinline__ uint32_t lut_ld(uint32_t t) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(t), "n"(kLutAt));
+  return v;
+}
 
 // acc += c_even * x_even + c_odd * x_odd, with lv = (c_even, c_odd) and
 // xw = (x_even, x_odd) bf16x2 words (low half = even k): two fused
@@ -247,15 +292,15 @@ __device__ __forceinline__ void pair_first(float& acc, uint32_t lv, uint32_t xw)
 // read).
 template <bool FIRST, int M>
 __device__ __forceinline__ void quad4(float (&su)[4][M], const uint32_t (&idx)[4],
-                                      uint32_t lane_hi, const uint32_t (&xq)[M][4]) {
+                                      uint32_t lane_col, const uint32_t (&xq)[M][4]) {
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     uint32_t lv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      // byte b -> bits 15:8; the lane offset (bits 7:0) and the table's 64 KB
-      // page (bits 23:16) come from lane_hi
-      lv[i] = lds32(__byte_perm(idx[i], lane_hi, 0x6504u | (uint32_t(b) << 4)));
+      // row = byte b of the index word (bits 15:8), column = the lane's
+      // (bits 7:0; lane_col < 256, so bits 31:16 are zero)
+      lv[i] = lut_ld(__byte_perm(idx[i], lane_col, 0x6504u | (uint32_t(b) << 4)));
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -291,24 +336,48 @@ __device__ __forceinline__ uint32_t lane_hi_delta(int q) {
   return uint32_t((64 - 32 * (q >> 1)) * kWordBytes);
 }
 
-// Per lane and unit: 4 rows x 32 codes.  wd[i] holds row i's 16 bytes for the
-// lane (4-bit: one word; 3-bit: 8 lo-plane bytes then 8 hi-plane bytes); p is
-// the lane's bytes in the tile (lane_tile_offset).
+// The lane's share of one unit, loaded only if live > 0 (otherwise nothing is
+// read and the registers are left as they are): row i's 16 bytes of the tile
+// at p (4-bit: one word; 3-bit: 8 lo-plane bytes, then the 8 hi-plane bytes
+// hi_delta further on) into wd[i], row i's scale s[i][0] into sv[i].  One
+// predicate serves all eight loads.
 template <int BITS>
-__device__ __forceinline__ void load_unit_m1(uint4 (&wd)[4], const uint8_t* p,
-                                             uint32_t hi_delta) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (BITS == 4) {
-      wd[i] = ld_stream_v4(p + 128 * i);
-    } else {
-      uint32_t l0, l1, h0, h1;
-      asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
-                   : "=r"(l0), "=r"(l1) : "l"(p + 128 * i));
-      asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];"
-                   : "=r"(h0), "=r"(h1) : "l"(p + hi_delta + 128 * i));
-      wd[i] = make_uint4(l0, l1, h0, h1);
-    }
+__device__ __forceinline__ void fetch_unit(uint4 (&wd)[4], uint32_t (&sv)[4], const uint8_t* p,
+                                           uint32_t hi_delta, const uint16_t* s0,
+                                           const uint16_t* s1, const uint16_t* s2,
+                                           const uint16_t* s3, int live) {
+  if (BITS == 4) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.gt.s32 p, %25, 0;\n\t"
+        "@p ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%20];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v4.u32 {%4, %5, %6, %7}, [%20+128];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v4.u32 {%8, %9, %10, %11}, [%20+256];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v4.u32 {%12, %13, %14, %15}, [%20+384];\n\t"
+        "@p ld.global.nc.u16 %16, [%21];\n\t@p ld.global.nc.u16 %17, [%22];\n\t"
+        "@p ld.global.nc.u16 %18, [%23];\n\t@p ld.global.nc.u16 %19, [%24];\n\t}"
+        : "=r"(wd[0].x), "=r"(wd[0].y), "=r"(wd[0].z), "=r"(wd[0].w), "=r"(wd[1].x),
+          "=r"(wd[1].y), "=r"(wd[1].z), "=r"(wd[1].w), "=r"(wd[2].x), "=r"(wd[2].y),
+          "=r"(wd[2].z), "=r"(wd[2].w), "=r"(wd[3].x), "=r"(wd[3].y), "=r"(wd[3].z),
+          "=r"(wd[3].w), "=r"(sv[0]), "=r"(sv[1]), "=r"(sv[2]), "=r"(sv[3])
+        : "l"(p), "l"(s0), "l"(s1), "l"(s2), "l"(s3), "r"(live));
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.gt.s32 p, %26, 0;\n\t"
+        "@p ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%20];\n\t"
+        "@p ld.global.nc.v2.u32 {%2, %3}, [%21];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v2.u32 {%4, %5}, [%20+128];\n\t"
+        "@p ld.global.nc.v2.u32 {%6, %7}, [%21+128];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v2.u32 {%8, %9}, [%20+256];\n\t"
+        "@p ld.global.nc.v2.u32 {%10, %11}, [%21+256];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v2.u32 {%12, %13}, [%20+384];\n\t"
+        "@p ld.global.nc.v2.u32 {%14, %15}, [%21+384];\n\t"
+        "@p ld.global.nc.u16 %16, [%22];\n\t@p ld.global.nc.u16 %17, [%23];\n\t"
+        "@p ld.global.nc.u16 %18, [%24];\n\t@p ld.global.nc.u16 %19, [%25];\n\t}"
+        : "=r"(wd[0].x), "=r"(wd[0].y), "=r"(wd[0].z), "=r"(wd[0].w), "=r"(wd[1].x),
+          "=r"(wd[1].y), "=r"(wd[1].z), "=r"(wd[1].w), "=r"(wd[2].x), "=r"(wd[2].y),
+          "=r"(wd[2].z), "=r"(wd[2].w), "=r"(wd[3].x), "=r"(wd[3].y), "=r"(wd[3].z),
+          "=r"(wd[3].w), "=r"(sv[0]), "=r"(sv[1]), "=r"(sv[2]), "=r"(sv[3])
+        : "l"(p), "l"(p + hi_delta), "l"(s0), "l"(s1), "l"(s2), "l"(s3), "r"(live));
   }
 }
 
@@ -355,275 +424,244 @@ __device__ __forceinline__ void unit_partial(float (&su)[4][M], const uint4 (&wd
   }
 }
 
-// Activations in shared memory stay bf16, in order: a group's four chunks of
-// 32 values (64 bytes each) are contiguous, so that one bulk copy brings a
-// whole run of them.
-constexpr uint32_t kXChunkBytes = 64;
-constexpr uint32_t kXGroupBytes = 4 * kXChunkBytes;
-
-// Shared-window layout of the small-batch kernel, in addresses of the CTA's
-// shared window (the block's own static shared memory and the system's
-// reserved bytes lie below kSbaseMax, where dynamic shared memory begins):
-//   [kSlotsAt, xlo_at(M))        warp slots, [NW][2][M][32] fp32
-//   [xlo_at(M), kPageAt)         activations of groups [0, gb), batch row by
-//                                batch row (gb groups each)
-//   [kPageAt, kAboveAt)          the lookup table, on its own 64 KB page
-//   [kAboveAt, ...)              activations of groups [gb, G), batch row by
-//                                batch row, then each warp's first tile, all
-//                                copied in by the bulk copy engine
-// The dynamic size kAboveAt + small_above_bytes therefore covers the window
-// up to the end of the staging area whatever the exact start (<= kSbaseMax).
-constexpr uint32_t kSbaseMax = 4096;
-constexpr uint32_t kSlotsAt = kSbaseMax;
-constexpr uint32_t kPageAt = 0x10000;
-constexpr uint32_t kAboveAt = 0x20000;
-constexpr uint64_t kM1WaitNs = 2000000000ull;  // bounded waits: 2 s
-
-__host__ __device__ constexpr uint32_t xlo_at(int M) {
-  return kSlotsAt + uint32_t(kM1Warps * 2 * M * kStrip * 4);
-}
-__host__ __device__ constexpr uint32_t x_groups_below(uint32_t G, int M) {
-  return G < (kPageAt - xlo_at(M)) / (kXGroupBytes * M) ? G
-                                                        : (kPageAt - xlo_at(M)) / (kXGroupBytes * M);
-}
-__host__ __device__ constexpr uint32_t small_above_bytes(uint32_t G, int M, int bits) {
-  return (G - x_groups_below(G, M)) * kXGroupBytes * M + kM1Warps * uint32_t(tile_bytes(bits));
-}
-
-// Prefetch depth: tiles in registers ahead of the one being consumed.  Three
-// rotating buffers for M <= 2; two for larger batches, whose accumulators
-// need the registers.
-template <int M>
+// Prefetch depth NB: tiles in registers, the one being consumed and the next
+// (a third buffer measured 2% slower on the 4096 x 14336 layer once the
+// weights come from L2).  kFourBases: the four scale rows of a lane get a
+// base address each (one fewer add per load, eight more registers).
+template <int BITS, int M>
 struct SmallCfg {
-  static constexpr int NB = M <= 2 ? 3 : 2;
+  static constexpr int NB = 2;
+  static constexpr bool kFourBases = M == 1 || (BITS == 4 && M >= 3);
 };
+
+// base + i * scale as one wide multiply-add (i, scale 32-bit).
+template <typename T>
+__device__ __forceinline__ const T* wide_addr(const T* base, uint32_t i, uint32_t scale) {
+  uint64_t r;
+  asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(r) : "r"(i), "r"(scale), "l"(base));
+  return reinterpret_cast<const T*>(r);
+}
+
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_cg_u16(const uint16_t* p) {
+  uint32_t r;
+  asm volatile("ld.global.cg.u16 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 
 template <int BITS, int M>
 __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a) {
-  constexpr int NB = SmallCfg<M>::NB;
+  constexpr int NB = SmallCfg<BITS, M>::NB;
+  constexpr int TB = tile_bytes(BITS);
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ WarpTable<kM1Warps> wt;
-  __shared__ __align__(8) uint64_t bars[1 + kM1Warps];  // activations, then one per warp's tile
-  __shared__ int abort_flag;
   const uint32_t sbase = sm_addr(smem);
-  const uint32_t G = uint32_t(a.G);
-  const uint32_t gb = x_groups_below(G, M);
+  const uint32_t G = uint32_t(a.G), K = uint32_t(a.K);
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  // The layout needs dynamic shared memory to begin below kSbaseMax; the
-  // host allocates for that.  Should it not, nothing is touched.
-  if (sbase > kSbaseMax) {
-    if (threadIdx.x == 0) report(a.status, LUTQ_ERR_CUDA);
+
+  // A grid smaller than the GPU starts with pf_ctas CTAs that find free
+  // multiprocessors while the preceding kernel on the stream still runs:
+  // they bring the whole packed matrix and the scales into L2, line by line,
+  // and leave (a prefetch reads nothing into the kernel, so it needs no wait
+  // for the preceding kernel).
+  if (blockIdx.x < a.pf_ctas) {
+    const uint32_t pk_lines = uint32_t(a.U) * uint32_t(TB / 128);
+    const uint32_t sc_lines = uint32_t((uint64_t(a.N) * G * 2u + 127u) / 128u);
+    const uint8_t* const sc = reinterpret_cast<const uint8_t*>(a.scales);
+    for (uint32_t j = blockIdx.x * blockDim.x + threadIdx.x; j < pk_lines + sc_lines;
+         j += a.pf_ctas * blockDim.x)
+      prefetch_l2(j < pk_lines ? a.packed + uint64_t(j) * 128u
+                               : sc + uint64_t(j - pk_lines) * 128u);
     return;
   }
-  float* slots = reinterpret_cast<float*>(smem + (kSlotsAt - sbase));
-  uint8_t* lut = smem + (kPageAt - sbase);
-  constexpr int TB = tile_bytes(BITS);
-  const uint32_t x_lo = xlo_at(M), x_lo_stride = gb * kXGroupBytes;
-  const uint32_t x_hi_stride = (G - gb) * kXGroupBytes;
-  const uint32_t stage_at = kAboveAt + x_hi_stride * M + uint32_t(wl) * TB;
-  const uint32_t xbar = sm_addr(&bars[0]), tbar = sm_addr(&bars[1 + wl]);
-
-  const Span sp = cta_span(a, blockIdx.x);
+  const Span sp = cta_span(a, blockIdx.x - a.pf_ctas);
   // the warp's positions [u0, u1) of the CTA's unit sequence
   const uint32_t u0 = sp.v0 + range_begin(wl, sp.v1 - sp.v0, kM1Warps);
   const uint32_t u1 = sp.v0 + range_begin(wl + 1, sp.v1 - sp.v0, kM1Warps);
   const uint32_t first_strip = sp.s0 + u0 / sp.W;
   const uint32_t g_first = u0 % sp.W;  // within the window: group sp.ga + g_first
   const int q = lane >> 3, rq = lane & 7;
-  const uint8_t* tile0 = a.packed + (uint64_t(first_strip) * G + sp.ga + g_first) * TB;
 
-  // Everything above reads only the launch parameters.  The kernel is
-  // launched as a programmatic dependent of the work before it on the
-  // stream, so it may start while that work finishes; global memory is
-  // touched only from here on, once that work is complete.  The next launch
-  // may likewise start early (it waits the same way).
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-  // Activations and each warp's first tile come in through the bulk copy
-  // engine (no load instructions, so the table build below does not queue
-  // behind them): each batch row's activations in one or two runs (below and
-  // above the table's page), counted in bytes on bars[0]; the tile whole into
-  // the warp's staging area on its own barrier.
-  if (threadIdx.x == 0) abort_flag = 0;
-  if (lane == 0) {
-    if (wl == 0) sm100::mbar_init(xbar, 1);
-    sm100::mbar_init(tbar, 1);
-    sm100::mbar_fence_init();
-    if (wl == 0) sm100::mbar_expect_tx(xbar, uint32_t(M) * uint32_t(a.K) * 2u);
-    if (u0 < u1) {
-      sm100::mbar_expect_tx(tbar, uint32_t(TB));
-      sm100::bulk_g2s(stage_at, tile0, uint32_t(TB), tbar);
-    }
-  }
-  if (threadIdx.x == 0) {
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-      const uint16_t* xm = a.x + uint64_t(m) * a.K;
-      sm100::bulk_g2s(x_lo + uint32_t(m) * x_lo_stride, xm, x_lo_stride, xbar);
-      if (gb < G)
-        sm100::bulk_g2s(kAboveAt + uint32_t(m) * x_hi_stride, xm + uint64_t(gb) * kGroup,
-                        x_hi_stride, xbar);
-    }
-  }
-
-  // Fetch cursor: the lane's bytes of the next tile to load, the scale of
-  // its row rq for that tile's group (rows rq + 8 i are 16 G bytes apart),
-  // and that group's place in the window.  Tiles are loaded in the order of
-  // the positions; after the last group of the window comes group sp.ga of
-  // the next strip.
-  const uint32_t hi_delta = BITS == 3 ? lane_hi_delta(q) : 0u;
+  // Fetch cursor, in the order of the positions: tile index ft (strip * G +
+  // group) and scale index fs (strip * 32 G + group) of the next unit to
+  // load; fleft units until the end of the window in that strip (the window's
+  // first group of the next strip follows); fn units still to load.
+  uint32_t ft = first_strip * G + sp.ga + g_first;
+  uint32_t fs = first_strip * uint32_t(kStrip) * G + sp.ga + g_first;
+  uint32_t fleft = sp.W - g_first;
+  int fn = int(u1 - u0);
   const uint32_t lane_off = lane_tile_offset<BITS>(q, rq);
-  const uint8_t* fw = tile0 + lane_off;
-  const uint16_t* fs =
-      a.scales + (uint64_t(first_strip) * kStrip + rq) * G + sp.ga + g_first;
-  uint32_t fg = g_first;
-  const uint32_t s8b = 16u * G;
-  const uint64_t w_wrap = uint64_t(G - sp.W + 1) * TB;  // tile after the window's last one
-  const uint32_t s_wrap = 32u * G - sp.W + 1u;           // likewise for the scale of row r
-  auto fetch_scales = [&](uint16_t (&sv)[4]) {
-    const uint8_t* sb = reinterpret_cast<const uint8_t*>(fs);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sv[i] = __ldg(reinterpret_cast<const uint16_t*>(sb + i * s8b));
-  };
-  auto advance = [&]() {
-    fw += TB;
-    ++fs;
-    if (++fg == sp.W) {  // rare: on to the next strip
-      fg = 0;
-      fw += w_wrap - TB;
-      fs += s_wrap - 1u;
-    }
-  };
-  auto fetch = [&](uint4 (&wd)[4], uint16_t (&sv)[4]) {
-    load_unit_m1<BITS>(wd, fw, hi_delta);
-    fetch_scales(sv);
-    advance();
-  };
+  const uint32_t hi_delta = BITS == 3 ? lane_hi_delta(q) : 0u;
+  const uint8_t* const pk = a.packed + lane_off;
+  // the lane's rows rq + 8 i are 8 G scales apart; with many accumulators
+  // live, the four addresses are formed from one base (fewer registers)
+  constexpr bool kFourBases = SmallCfg<BITS, M>::kFourBases;
+  const uint16_t* const sc0 = a.scales + uint64_t(rq) * G;
+  const uint16_t* const sc1 = kFourBases ? sc0 + 8u * G : sc0;
+  const uint16_t* const sc2 = kFourBases ? sc1 + 8u * G : sc0;
+  const uint16_t* const sc3 = kFourBases ? sc2 + 8u * G : sc0;
+  const uint32_t g8 = kFourBases ? 0u : 8u * G;
 
-  // Lane t holds codebook[t mod 2^BITS]; the table is built from it with
-  // shuffles, so no shared staging (and no barrier) precedes the build.
-  const uint32_t cbv = __ldg(a.codebook + (lane & ((1 << BITS) - 1)));
-  uint4 buf[NB][4];
-  uint16_t sbuf[NB][4];
-  if (u0 < u1) {
-    fetch_scales(sbuf[0]);  // the words of tile u0 are on their way to the staging area
-    advance();
-  }
-  fill_warp_table<kM1Warps>(wt, sp);
-  build_lut_shfl<BITS>(lut, cbv);
-  // the next tiles go straight to registers
+  // Before the preceding kernel on the stream is complete (this kernel is
+  // its programmatic dependent) nothing is read.  Without prefetching CTAs,
+  // the warp's first tiles and scales are brought into L2 (which keeps no
+  // stale copy) meanwhile; the values are loaded after the wait below.
+  if (a.pf_ctas == 0 && u0 < u1) {
+    uint32_t t = ft, l = fleft;
 #pragma unroll
-  for (int t = 1; t < NB; ++t)
-    if (u0 + t < u1) fetch(buf[t], sbuf[t]);
-  __syncthreads();  // table, warp table, barrier initialisation
-
-  // Activations and the first tile in; a wait that runs out marks the call
-  // failed, and the warps skip their work.
-  if (!sm100::mbar_wait(xbar, 0, &abort_flag, kM1WaitNs)) report(a.status, LUTQ_ERR_TIMEOUT);
-  bool ok = true;
-  if (u0 < u1) {
-    ok = sm100::mbar_wait(tbar, 0, &abort_flag, kM1WaitNs);
-    if (!ok) report(a.status, LUTQ_ERR_TIMEOUT);
-    // the staged words of tile u0, at the offsets a global load would use
-    const uint32_t t = stage_at + lane_off;
+    for (int j = 0; j < NB; ++j) {
+      if (u0 + j < u1) {
+        const uint8_t* p = wide_addr(pk, t, uint32_t(TB));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (BITS == 4) {
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(buf[0][i].x), "=r"(buf[0][i].y), "=r"(buf[0][i].z), "=r"(buf[0][i].w)
-                     : "r"(t + 128u * i));
-      } else {
-        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                     : "=r"(buf[0][i].x), "=r"(buf[0][i].y) : "r"(t + 128u * i));
-        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                     : "=r"(buf[0][i].z), "=r"(buf[0][i].w) : "r"(t + hi_delta + 128u * i));
+        for (int i = 0; i < 4; ++i) prefetch_l2(p + 128 * i);
+      }
+      ++t;
+      if (--l == 0) {
+        t += G - sp.W;
+        l = sp.W;
       }
     }
+    if (q == 0) {
+      prefetch_l2(sc0 + fs);
+      prefetch_l2(sc1 + (fs + g8));
+      prefetch_l2(sc2 + (fs + 2u * g8));
+      prefetch_l2(sc3 + (fs + 3u * g8));
+    }
   }
-  ok = ok && !*reinterpret_cast<volatile int*>(&abort_flag);
+  if (threadIdx.x == 0) prefetch_l2(a.codebook);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // The layout needs dynamic shared memory to begin below kSbaseMax; the
+  // host allocates for that.  Should it not, nothing is touched.
+  if (sbase > kSbaseMax) {
+    if (threadIdx.x == 0) report(a.status, LUTQ_ERR_CUDA);
+    return;
+  }
 
-  const uint32_t page = (kPageAt >> 16) << 8;
-  const uint32_t lane_e = page | uint32_t(lane) * 4u, lane_o = page | (128u + uint32_t(lane) * 4u);
+  auto fetch = [&](uint4 (&wd)[4], uint32_t (&sv)[4]) {
+    fetch_unit<BITS>(wd, sv, wide_addr(pk, ft, TB), hi_delta, wide_addr(sc0, fs, 2u),
+                     wide_addr(sc1, fs + g8, 2u), wide_addr(sc2, fs + 2u * g8, 2u),
+                     wide_addr(sc3, fs + 3u * g8, 2u), fn);
+    --fn;
+    ++ft;
+    ++fs;
+    if (--fleft == 0) {  // on to the window's first group of the next strip
+      ft += G - sp.W;
+      fs += uint32_t(kStrip) * G - sp.W;
+      fleft = sp.W;
+    }
+  };
+
+  // The activations first (all threads, 16 bytes at a time, through L2:
+  // the preceding kernel may have written them), the codebook (lane t holds
+  // codebook[t mod 2^BITS], and the table is built from it with shuffles)
+  // and the first tile; the other NB - 1 tiles once the activations are in.
+  uint4 buf[NB][4];
+  uint32_t sbuf[NB][4];
+  uint32_t cbv;
+  {
+    constexpr uint32_t kStep = kM1Warps * 32 * 16;
+    const uint32_t xbytes = uint32_t(M) * K * 2u;
+    const uint8_t* xg = reinterpret_cast<const uint8_t*>(a.x);
+    uint8_t* xs = smem + (kXAt - sbase);
+    uint32_t o = threadIdx.x * 16u;
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (o + j * kStep < xbytes) v[j] = ld_cg_v4(xg + o + j * kStep);
+    cbv = ld_cg_u16(a.codebook + (lane & ((1 << BITS) - 1)));
+    fetch(buf[0], sbuf[0]);
+    for (;;) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (o + j * kStep < xbytes) *reinterpret_cast<uint4*>(xs + o + j * kStep) = v[j];
+      o += 4 * kStep;
+      if (o >= xbytes) break;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (o + j * kStep < xbytes) v[j] = ld_cg_v4(xg + o + j * kStep);
+    }
+  }
+  build_lut_shfl<BITS>(smem + (kLutAt - sbase), cbv);
+#pragma unroll
+  for (int t = 1; t < NB; ++t) fetch(buf[t], sbuf[t]);
+  __syncthreads();  // table, activations
+
+  const uint32_t lane_e = uint32_t(lane) * 4u, lane_o = 128u + uint32_t(lane) * 4u;
   const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
-  float* my_slots = slots + wl * 2 * M * kStrip;
+  float* const slots = reinterpret_cast<float*>(smem + (slots_at(K, M) - sbase));
+  float* const my_slots = slots + wl * 2 * M * kStrip;
   int rows[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) rows[i] = rq + 8 * i;
-  // activation address of (group g, chunk q) for batch row 0, and the step
-  // to the next batch row: below the page for g < gb, above it otherwise
-  const uint32_t xq = uint32_t(q) * kXChunkBytes;
-  auto x_at = [&](uint32_t g) {
-    return (g < gb ? x_lo + g * kXGroupBytes : kAboveAt + (g - gb) * kXGroupBytes) + xq;
-  };
+  const uint32_t xstride = K * 2u;
+  // the lane's activations of the window's first group, batch row 0
+  const uint32_t xa_w = kXAt + sp.ga * kXGroupBytes + uint32_t(q) * kXChunkBytes;
 
-  if (u0 < u1 && ok) {
-    uint32_t strip = first_strip, g = g_first;
-    const uint32_t xa_w = x_at(sp.ga);  // first group of the window
-    const uint32_t xs_w = sp.ga < gb ? x_lo_stride : x_hi_stride;
-    uint32_t xa = x_at(sp.ga + g_first);
-    uint32_t xs = sp.ga + g_first < gb ? x_lo_stride : x_hi_stride;
-    const uint32_t xa_hi = x_at(gb);     // first group above the page
+  if (u0 < u1) {
+    uint32_t strip = first_strip;
+    uint32_t xa = xa_w + g_first * kXGroupBytes;
+    // cleft: units of the current strip still to consume; rest: units of
+    // the range after the current strip's
+    uint32_t cleft = min(sp.W - g_first, u1 - u0);
+    uint32_t rest = (u1 - u0) - cleft;
     float acc[4][M];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int m = 0; m < M; ++m) acc[i][m] = 0.0f;
-    // consume the tile u held in (wd, sv); refill that buffer with tile u + NB
-    auto step = [&](uint4 (&wd)[4], uint16_t (&sv)[4], uint32_t u) {
+    // Consume the unit held in (wd, sv); true once the range is done.
+    auto step = [&](const uint4 (&wd)[4], const uint32_t (&sv)[4]) -> bool {
       float su[4][M];
-      unit_partial<BITS, M>(su, wd, lane_e, lane_o, hi_shift, xa, xs);
+      unit_partial<BITS, M>(su, wd, lane_e, lane_o, hi_shift, xa, xstride);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float s = __uint_as_float(uint32_t(sv[i]) << 16);
+        const float s = __uint_as_float(sv[i] << 16);
 #pragma unroll
         for (int m = 0; m < M; ++m) acc[i][m] = fmaf(s, su[i][m], acc[i][m]);
       }
-      if (u + NB < u1) fetch(wd, sv);
-      if (g + 1 == sp.W || u + 1 == u1) {
-        float vals[4][M];
+      xa += kXGroupBytes;
+      if (--cleft != 0) return false;
+      // the warp's units of this strip are summed: the four lanes of a row
+      // add theirs, and the strip's sums are written or left in the slots
+      float vals[4][M];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int m = 0; m < M; ++m) {
-            float v = acc[i][m];
-            v += __shfl_xor_sync(0xffffffffu, v, 8);
-            v += __shfl_xor_sync(0xffffffffu, v, 16);
-            vals[i][m] = v;
-            acc[i][m] = 0.0f;
-          }
-        deposit_strip<M, 4>(a, sp, strip, u0, u1, first_strip, vals, rows, q == 0, my_slots);
-        ++strip;
-        g = 0;
-        xa = xa_w;
-        xs = xs_w;
-      } else {
-        ++g;
-        if (sp.ga + g == gb) {
-          xa = xa_hi;
-          xs = x_hi_stride;
-        } else {
-          xa += kXGroupBytes;
+        for (int m = 0; m < M; ++m) {
+          float v = acc[i][m];
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
+          vals[i][m] = v;
+          acc[i][m] = 0.0f;
         }
-      }
+      deposit_strip<M, 4>(a, sp, strip, u0, u1, first_strip, vals, rows, q == 0, my_slots);
+      if (rest == 0) return true;
+      ++strip;
+      xa = xa_w;
+      cleft = min(sp.W, rest);
+      rest -= cleft;
+      return false;
     };
-    for (uint32_t u = u0; u < u1; u += NB) {
+    for (;;) {
 #pragma unroll
       for (int t = 0; t < NB; ++t) {
-        if (t > 0 && u + t >= u1) break;
-        step(buf[t], sbuf[t], u + t);
+        if (step(buf[t], sbuf[t])) goto range_done;
+        fetch(buf[t], sbuf[t]);
       }
     }
+  range_done:;
   }
+  fill_warp_table<kM1Warps>(wt, sp);
   __syncthreads();
-  if (*reinterpret_cast<volatile int*>(&abort_flag)) {
-    // A wait ran out: let this block's own copies land (bounded again)
-    // before the shared memory is released, and leave y to the error.
-    volatile int again = 0;
-    if (lane == 0 && u0 < u1) sm100::mbar_wait(tbar, 0, &again, kM1WaitNs);
-    if (threadIdx.x == 0) sm100::mbar_wait(xbar, 0, &again, kM1WaitNs);
-    return;
-  }
   cta_finish<M, kM1Warps>(a, sp, slots, wt);
 }
 
@@ -720,7 +758,12 @@ void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out) {
   out[5] = int32_t(pl.nh);
 }
 
-static void apply_plan(GemvArgs& a, int num_sms) {
+// A matrix (packed bytes and scales) up to this size is brought into L2
+// ahead of the loads by prefetching CTAs on the multiprocessors the plan
+// leaves free.
+constexpr int64_t kPrefetchBytes = int64_t(64) << 20;
+
+static void apply_plan(GemvArgs& a, int num_sms, int bits) {
   const Plan pl = choose_plan(a.N / kStrip, a.G, num_sms);
   a.C = pl.C;
   a.kind = pl.kind;
@@ -728,24 +771,26 @@ static void apply_plan(GemvArgs& a, int num_sms) {
   a.Cm = pl.Cm;
   a.T = pl.T;
   a.nh = pl.nh;
+  const int64_t bytes = a.U * tile_bytes(bits) + a.N * a.G * 2;
+  a.pf_ctas = pl.C < num_sms && bytes <= kPrefetchBytes ? uint32_t(num_sms - pl.C) : 0u;
 }
 
 
-static int64_t small_smem(int64_t K, int M, int bits) {
-  return int64_t(kAboveAt) + small_above_bytes(uint32_t(K / kGroup), M, bits);
+static int64_t small_smem(int64_t K, int M) {
+  return K < (int64_t(1) << 20) ? int64_t(small_end(uint32_t(K), M)) : int64_t(1) << 30;
 }
 
 template <int BITS, int M>
 static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
   static SmemGrant grant;
-  const int smem = int(small_smem(a.K, M, BITS));
+  const int smem = int(small_smem(a.K, M));
   cudaError_t err = grant_smem(gemv_small_kernel<BITS, M>, grant, smem);
   if (err != cudaSuccess) return err;
-  apply_plan(a, num_sms);
-  // programmatic dependent launch: the kernel's prologue (launch parameters,
-  // work split) may overlap the end of the preceding kernel on the stream
+  apply_plan(a, num_sms, BITS);
+  // programmatic dependent launch: the prefetching blocks and the work
+  // blocks' set-up may overlap the end of the preceding kernel on the stream
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(a.C));
+  cfg.gridDim = dim3(unsigned(a.C) + a.pf_ctas);
   cfg.blockDim = dim3(kM1Warps * 32);
   cfg.dynamicSmemBytes = size_t(smem);
   cfg.stream = stream;
@@ -770,7 +815,7 @@ constexpr int kMaxSmallBatch = 4;
 
 template <int BITS>
 static bool small_fits(int64_t M, int64_t K) {
-  return M >= 1 && M <= kMaxSmallBatch && small_smem(K, int(M), BITS) <= kMaxSmemPerBlock - 1024;
+  return M >= 1 && M <= kMaxSmallBatch && small_smem(K, int(M)) <= kMaxSmemPerBlock - 1024;
 }
 
 template <int BITS>

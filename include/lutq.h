@@ -168,9 +168,17 @@ int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
  * within 2e-3 (relative, floored at 1e-2 of the row's rms) of the exact sum.
  * M = 1..4 run on the CUDA cores (each table lookup serves the M batch rows);
  * larger batches, whose product is a dense contraction for the CUDA cores,
- * and rows whose activations do not fit the kernel's shared memory (K above
- * about 60000 / M) run on the tensor cores exactly as lutq_gemm.  Either way
- * the result does not depend on timing.
+ * and rows whose activations do not fit the kernel's shared memory
+ * (M * (K + 2048) > 80896: K above 78848 at M = 1, above 18176 at M = 4) run
+ * on the tensor cores exactly as lutq_gemm.  Either way the result does not
+ * depend on timing.
+ * The CUDA-core kernel is launched as a programmatic dependent of the work
+ * before it on `stream`: its set-up overlaps the end of that work, and when
+ * its plan leaves multiprocessors free and the matrix (packed bytes and
+ * scales) is at most 64 MiB, extra thread blocks on those multiprocessors
+ * bring the matrix into L2 meanwhile.  Nothing is read into the kernel
+ * before the preceding work is complete, so the caller need not order
+ * anything.
  *
  * x        device bf16 [M,K] row-major.
  * packed   device, layout V1 (lutq_pack).

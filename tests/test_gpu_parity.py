@@ -254,3 +254,28 @@ def test_gemv_split_strips(lq, kind, bits, n, k, want_kind, want_align):
         assert int(ws.count_nonzero().item()) == 0
         y2, _ = _gemv(lq, x, packed, scales, cb, bits, n, k, ws=ws)
         np.testing.assert_array_equal(y, y2)
+
+
+# ------------------------------------------------------------------ runs over many strips
+
+@pytest.mark.parametrize("kind,bits", [("nf4", 4), ("lloyd_max3", 3)])
+def test_gemv_warp_runs_span_strips(lq, kind, bits):
+    """Two groups per row and 4096 strips: every block takes ~28 whole strips,
+    so each warp's run of units crosses from strip to strip (its partial sums
+    go through the block's slots at every strip end)."""
+    n, k = 131072, 256
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plan = lq.lutq_gemv_plan(n, k, sms)
+    assert plan["kind"] == 0 and plan["align"] == 1 and plan["C"] == min(sms, n // 32)
+    w = workloads.normal_weights(n, k, 0.02, seed=41)
+    cb, levels, codes, scales, packed = _quantize_pack(lq, w, kind, bits)
+    strips = _sample_strips(n, count=8, seed=3)
+    rows = np.concatenate([np.arange(32 * s, 32 * s + 32) for s in strips])
+    ref_codes, ref_sb = O.quantize(_f32(w[rows]), levels, bits)
+    np.testing.assert_array_equal(codes[rows].cpu().numpy(), ref_codes)
+    ws = lq.new_workspace(4, n, k, bits)
+    for m in (1, 2, 4):
+        x = workloads.activations(m, k, seed=51 + m)
+        y, _ = _gemv(lq, x, packed, scales, cb, bits, n, k, ws=ws)
+        y_ref = O.gemv(_f32(x), ref_codes, ref_sb, levels)
+        assert O.rel_error_gate(y[:, rows], y_ref) <= TOL, (m,)
