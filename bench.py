@@ -268,18 +268,18 @@ def side_measurements(lq, dev, args):
     w = lay.weights(seed=0).to(dev)
     st = lq.new_status(dev)
     codes, scales = lq.lutq_quantize(w, cb, bits, status=st)
-    packed = lq.lutq_pack(codes, bits, status=st)
-    del w, codes
+    packed = lq.lutq_pack(codes, scales, bits, status=st)
+    del w, codes, scales
     x = workloads.activations(m, k, seed=1).to(dev)
     y = torch.empty((m, n), dtype=torch.float32, device=dev)
     ws = lq.new_workspace(m, n, k, bits, dev)
-    call = lambda i: lq.lutq_gemm(x, packed, scales, cb, bits, n, k, y=y, workspace=ws, status=st)
+    call = lambda i: lq.lutq_gemm(x, packed, cb, bits, n, k, y=y, workspace=ws, status=st)
     for i in range(3):
         call(i)
     s = time_events(call, 20)
     assert int(st.item()) == 0
     tflops = 2.0 * m * n * k / s / 1e12
-    nbytes = packed.numel() + scales.numel() * 2 + m * k * 2 + m * n * 4
+    nbytes = packed.numel() + m * k * 2 + m * n * 4
     out["gemm"] = {"workload": f"llama3_70b_mlp/gate_up W[{n},{k}] nf4 W4 group128 batch{m}",
                    "metric": "GEMM TFLOP/s at batch>=32", "value": tflops, "unit": "TFLOP/s",
                    "us": s * 1e6, "hbm_gbs": nbytes / s / 1e9,
@@ -288,7 +288,7 @@ def side_measurements(lq, dev, args):
                                 "peak_source": peak_kind + " (bf16 burst)",
                                 "traffic": ncu_traffic(f"gemm_w4_m{m}_{n}x{k}", GEMM_SOURCES)},
                    "kernel": "lutq::gemm_kernel"}
-    del packed, scales, x, y, ws
+    del packed, x, y, ws
     # offline steps on the headline layer
     lay = workloads.layer(args.workload, args.layer)
     n, k, bits = lay.n, lay.k, args.bits
@@ -296,13 +296,13 @@ def side_measurements(lq, dev, args):
     w = lay.weights(seed=0).to(dev)
     codes, scales = lq.lutq_quantize(w, cb, bits, status=st)
     tq = time_events(lambda i: lq.lutq_quantize(w, cb, bits, status=st), 10)
-    tp = time_events(lambda i: lq.lutq_pack(codes, bits, status=st), 10)
+    tp = time_events(lambda i: lq.lutq_pack(codes, scales, bits, status=st), 10)
     assert int(st.item()) == 0
     q_bytes = n * k * 2 + n * k + n * (k // 128) * 2
-    p_bytes = n * k + (n * k * bits) // 8
+    p_bytes = n * k + (n * k * bits) // 8 + 2 * n * (k // 128) * 2
     out["offline"] = {"quantize_gbs": q_bytes / tq / 1e9, "quantize_us": tq * 1e6,
                       "pack_gbs": p_bytes / tp / 1e9, "pack_us": tp * 1e6,
-                      "note": "W bf16 -> codes u8 + scales; codes -> layout V1 (L2-warm)"}
+                      "note": "W bf16 -> codes u8 + scales; codes + scales -> layout V2 (L2-warm)"}
     return out
 
 
@@ -317,16 +317,15 @@ def run_lutq(args, world, rank, local):
     w = lay.weights(seed=0).to(dev)
     st = lq.new_status(dev)
     codes, scales = lq.lutq_quantize(w, cb, bits, status=st)
-    packed = lq.lutq_pack(codes, bits, status=st)
+    packed = lq.lutq_pack(codes, scales, bits, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    del w, codes
+    del w, codes, scales
 
-    per_copy = packed.numel() + scales.numel() * 2
+    per_copy = packed.numel()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     copies = max(2, int(np.ceil(3 * l2 / per_copy)) + 1)
     packs = [packed] + [packed.clone() for _ in range(copies - 1)]
-    scs = [scales] + [scales.clone() for _ in range(copies - 1)]
     x = workloads.activations(m, k, seed=1).to(dev)
     y = torch.empty((m, n), dtype=torch.float32, device=dev)
     ws = lq.new_workspace(m, n, k, bits, dev)
@@ -335,7 +334,7 @@ def run_lutq(args, world, rank, local):
 
     def step(i):
         j = i % copies
-        call(x, packs[j], scs[j], cb, bits, n, k, y=y, workspace=ws, status=st)
+        call(x, packs[j], cb, bits, n, k, y=y, workspace=ws, status=st)
 
     for i in range(8):  # eager warm-up (module load, attributes)
         step(i)
@@ -394,14 +393,14 @@ def run_lutq(args, world, rank, local):
     e2e_steps = min(args.steps, args.e2e_steps)
     for i in range(20):
         x_dev.copy_(x_host, non_blocking=True)
-        call(x_dev, packs[i % copies], scs[i % copies], cb, bits, n, k, y=y, workspace=ws)
+        call(x_dev, packs[i % copies], cb, bits, n, k, y=y, workspace=ws)
         y_host.copy_(y, non_blocking=True)
         torch.cuda.synchronize()
     barrier(world)
     t0 = time.perf_counter()
     for i in range(e2e_steps):
         x_dev.copy_(x_host, non_blocking=True)
-        call(x_dev, packs[i % copies], scs[i % copies], cb, bits, n, k, y=y, workspace=ws)
+        call(x_dev, packs[i % copies], cb, bits, n, k, y=y, workspace=ws)
         y_host.copy_(y, non_blocking=True)
         torch.cuda.synchronize()
     e2e_s = max_over_ranks(world, time.perf_counter() - t0)

@@ -37,11 +37,11 @@ _SIGS = {
     "lutq_packed_bytes": (_i64, [_i64, _i64, _i32]),
     "lutq_codebook": (_i32, [_i32, _i32, _vp]),
     "lutq_quantize": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
-    "lutq_pack": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "lutq_pack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "lutq_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32]),
-    "lutq_gemv": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
-    "lutq_gemm": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
-    "lutq_gemv_noalloc": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
+    "lutq_gemv": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+    "lutq_gemm": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+    "lutq_gemv_noalloc": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
     "lutq_gemv_plan": (_i32, [_i64, _i64, _i32, _vp]),
     "lutq_selftest_wait_timeout": (_i32, [_vp, _i64, _vp]),
 }
@@ -137,50 +137,55 @@ def lutq_quantize(w: torch.Tensor, codebook: torch.Tensor, bits: int,
     return codes, scales
 
 
-def lutq_pack(codes: torch.Tensor, bits: int,
+def lutq_pack(codes: torch.Tensor, scales: torch.Tensor, bits: int,
               status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """codes uint8 [N, K] and scales bf16 [N, K/128] -> the packed matrix
+    (layout V2, codes and scales); see lutq_pack in include/lutq.h."""
     _need(codes, torch.uint8, "codes")
+    _need(scales, torch.bfloat16, "scales")
     n, k = codes.shape
+    if tuple(scales.shape) != (n, k // 128):
+        raise LutqError(2, "lutq_pack: scales shape")
     nb = lutq_packed_bytes(n, k, bits)
     if nb < 0:
         raise LutqError(2, "lutq_packed_bytes")
     packed = torch.empty(nb, dtype=torch.uint8, device=codes.device)
-    _check(lib.lutq_pack(codes.data_ptr(), n, k, bits, packed.data_ptr(), _ptr(status), _stream()),
-           "lutq_pack")
+    _check(lib.lutq_pack(codes.data_ptr(), scales.data_ptr(), n, k, bits, packed.data_ptr(),
+                         _ptr(status), _stream()), "lutq_pack")
     return packed
 
 
-def _product(fn, where, x, packed, scales, codebook, bits, n, k, y, workspace, status):
+def _product(fn, where, x, packed, codebook, bits, n, k, y, workspace, status):
     _need(x, torch.bfloat16, "x")
     m = x.shape[0]
     if y is None:
         y = torch.empty((m, n), dtype=torch.float32, device=x.device)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
-    _check(fn(x.data_ptr(), m, packed.data_ptr(), scales.data_ptr(), codebook.data_ptr(), bits,
-              n, k, y.data_ptr(), ws_ptr, ws_bytes, _ptr(status), _stream()), where)
+    _check(fn(x.data_ptr(), m, packed.data_ptr(), codebook.data_ptr(), bits, n, k, y.data_ptr(),
+              ws_ptr, ws_bytes, _ptr(status), _stream()), where)
     return y
 
 
-def lutq_gemv(x, packed, scales, codebook, bits, n, k, y=None, workspace=None, status=None):
+def lutq_gemv(x, packed, codebook, bits, n, k, y=None, workspace=None, status=None):
     """y[M, N] (fp32) for M = 1..16; see lutq_gemv in include/lutq.h."""
-    return _product(lib.lutq_gemv, "lutq_gemv", x, packed, scales, codebook, bits, n, k, y,
-                    workspace, status)
+    return _product(lib.lutq_gemv, "lutq_gemv", x, packed, codebook, bits, n, k, y, workspace,
+                    status)
 
 
-def lutq_gemv_noalloc(x, packed, scales, codebook, bits, n, k, y=None, status=None):
+def lutq_gemv_noalloc(x, packed, codebook, bits, n, k, y=None, status=None):
     """lutq_gemv with the library's fixed scratch array instead of a workspace
     (for callers that cannot allocate device memory; see include/lutq.h)."""
     _need(x, torch.bfloat16, "x")
     m = x.shape[0]
     if y is None:
         y = torch.empty((m, n), dtype=torch.float32, device=x.device)
-    _check(lib.lutq_gemv_noalloc(x.data_ptr(), m, packed.data_ptr(), scales.data_ptr(),
-                                 codebook.data_ptr(), bits, n, k, y.data_ptr(), _ptr(status),
-                                 _stream()), "lutq_gemv_noalloc")
+    _check(lib.lutq_gemv_noalloc(x.data_ptr(), m, packed.data_ptr(), codebook.data_ptr(), bits,
+                                 n, k, y.data_ptr(), _ptr(status), _stream()),
+           "lutq_gemv_noalloc")
     return y
 
 
-def lutq_gemm(x, packed, scales, codebook, bits, n, k, y=None, workspace=None, status=None):
+def lutq_gemm(x, packed, codebook, bits, n, k, y=None, workspace=None, status=None):
     """y[M, N] (fp32) on the tensor cores; see lutq_gemm in include/lutq.h."""
-    return _product(lib.lutq_gemm, "lutq_gemm", x, packed, scales, codebook, bits, n, k, y,
-                    workspace, status)
+    return _product(lib.lutq_gemm, "lutq_gemm", x, packed, codebook, bits, n, k, y, workspace,
+                    status)

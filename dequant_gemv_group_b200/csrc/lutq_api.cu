@@ -11,14 +11,15 @@ namespace lutq {
 cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* codebook, int bits,
                             uint8_t* codes, void* scales, int32_t* dev_status, int num_sms,
                             cudaStream_t stream);
-cudaError_t launch_pack(const uint8_t* codes, int64_t N, int64_t K, int bits, void* packed,
+cudaError_t launch_pack(const uint8_t* codes, const void* scales, int64_t N, int64_t K,
+                        int bits, void* packed, int32_t* dev_status, int num_sms,
+                        cudaStream_t stream);
+cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
+                        int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream);
-cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* scales,
-                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
-                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
-cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* scales,
-                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
-                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
+                        int bits, int64_t N, int64_t K, float* y, void* workspace,
+                        int32_t* dev_status, int num_sms, cudaStream_t stream);
 int64_t gemv_workspace_bytes(int64_t M, int64_t N);
 void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out);
 int64_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
@@ -58,17 +59,16 @@ lutq_status check_bits(int bits) { return (bits == 3 || bits == 4) ? LUTQ_OK : L
 lutq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LUTQ_OK : LUTQ_ERR_CUDA; }
 
 lutq_status check_product_args(const void* x, int64_t M, int64_t max_m, const void* packed,
-                               const void* scales, const void* codebook, int bits, int64_t N,
-                               int64_t K, const float* y, const void* workspace,
-                               int64_t workspace_bytes, int64_t need) {
-  if (!x || !packed || !scales || !codebook || !y) return LUTQ_ERR_INVALID_ARG;
+                               const void* codebook, int bits, int64_t N, int64_t K,
+                               const float* y, const void* workspace, int64_t workspace_bytes,
+                               int64_t need) {
+  if (!x || !packed || !codebook || !y) return LUTQ_ERR_INVALID_ARG;
   lutq_status st = check_bits(bits);
   if (st != LUTQ_OK) return st;
   st = check_shape(N, K);
   if (st != LUTQ_OK) return st;
   if (M < 1 || M > max_m) return LUTQ_ERR_SHAPE;
-  if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(codebook) ||
-      !aligned16(y))
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(codebook) || !aligned16(y))
     return LUTQ_ERR_ALIGN;
   if (need > 0) {
     if (workspace == nullptr || workspace_bytes < need) return LUTQ_ERR_WORKSPACE;
@@ -97,11 +97,11 @@ const char* lutq_status_string(int status) {
   }
 }
 
-int lutq_layout_version(void) { return 1; }
+int lutq_layout_version(void) { return 2; }
 
 int64_t lutq_packed_bytes(int64_t N, int64_t K, int bits) {
   if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK) return -1;
-  return bits == 4 ? N * K / 2 : 3 * N * K / 8;
+  return (N / lutq::kStrip) * (K / lutq::kGroup) * (lutq::tile_bytes(bits) + lutq::kScaleBytes);
 }
 
 lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K, const void* codebook_bf16,
@@ -120,16 +120,16 @@ lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K, const void* 
                                          dev_status, sms, static_cast<cudaStream_t>(stream)));
 }
 
-lutq_status lutq_pack(const uint8_t* codes, int64_t N, int64_t K, int bits, void* packed,
-                      int32_t* dev_status, void* stream) {
-  if (!codes || !packed) return LUTQ_ERR_INVALID_ARG;
+lutq_status lutq_pack(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
+                      int bits, void* packed, int32_t* dev_status, void* stream) {
+  if (!codes || !scales_bf16 || !packed) return LUTQ_ERR_INVALID_ARG;
   lutq_status st = check_bits(bits);
   if (st != LUTQ_OK) return st;
   if ((st = check_shape(N, K)) != LUTQ_OK) return st;
-  if (!aligned16(codes) || !aligned16(packed)) return LUTQ_ERR_ALIGN;
+  if (!aligned16(codes) || !aligned16(scales_bf16) || !aligned16(packed)) return LUTQ_ERR_ALIGN;
   int sms = 0;
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
-  return from_cuda(lutq::launch_pack(codes, N, K, bits, packed, dev_status, sms,
+  return from_cuda(lutq::launch_pack(codes, scales_bf16, N, K, bits, packed, dev_status, sms,
                                      static_cast<cudaStream_t>(stream)));
 }
 
@@ -151,34 +151,32 @@ int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
   return lutq::gemm_workspace_bytes(M, N, K);
 }
 
-lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed, const void* scales_bf16,
+lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
                       const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
                       void* workspace, int64_t workspace_bytes, int32_t* dev_status,
                       void* stream) {
-  lutq_status st = check_product_args(x_bf16, M, 16, packed, scales_bf16, codebook_bf16, bits, N,
-                                      K, y, workspace, workspace_bytes,
+  lutq_status st = check_product_args(x_bf16, M, 16, packed, codebook_bf16, bits, N, K, y,
+                                      workspace, workspace_bytes,
                                       lutq_workspace_bytes(M, N, K, bits));
   if (st != LUTQ_OK) return st;
   int sms = 0;
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
-  return from_cuda(lutq::launch_gemv(x_bf16, M, packed, scales_bf16, codebook_bf16, bits, N, K, y,
-                                     workspace, dev_status, sms,
-                                     static_cast<cudaStream_t>(stream)));
+  return from_cuda(lutq::launch_gemv(x_bf16, M, packed, codebook_bf16, bits, N, K, y, workspace,
+                                     dev_status, sms, static_cast<cudaStream_t>(stream)));
 }
 
-lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed, const void* scales_bf16,
+lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
                       const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
                       void* workspace, int64_t workspace_bytes, int32_t* dev_status,
                       void* stream) {
-  lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, scales_bf16,
-                                      codebook_bf16, bits, N, K, y, workspace, workspace_bytes,
+  lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, codebook_bf16, bits,
+                                      N, K, y, workspace, workspace_bytes,
                                       lutq_workspace_bytes(M, N, K, bits));
   if (st != LUTQ_OK) return st;
   int sms = 0;
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
-  return from_cuda(lutq::launch_gemm(x_bf16, M, packed, scales_bf16, codebook_bf16, bits, N, K, y,
-                                     workspace, dev_status, sms,
-                                     static_cast<cudaStream_t>(stream)));
+  return from_cuda(lutq::launch_gemm(x_bf16, M, packed, codebook_bf16, bits, N, K, y, workspace,
+                                     dev_status, sms, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

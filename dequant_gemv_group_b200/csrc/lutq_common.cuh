@@ -9,10 +9,15 @@
 namespace lutq {
 
 constexpr int kGroup = 128;      // weights per quantization group along K
-constexpr int kStrip = 32;       // rows per packing strip (layout V1)
+constexpr int kStrip = 32;       // rows per packing strip (layout V2)
 constexpr int kWordBytes = 16;   // one packed word = one 16-byte vector load
+constexpr int kScaleBytes = 64;  // one unit's 32 row scales
 
+// Layout V2: unit t (strip of 32 rows, group of 128 codes) has tile_bytes of
+// codes at t * tile_bytes and its scales at U * tile_bytes + t * 64, row r's
+// at byte scale_slot(r) of those 64.
 __host__ __device__ constexpr int tile_bytes(int bits) { return bits == 4 ? 2048 : 1536; }
+__host__ __device__ constexpr int scale_slot(int r) { return 2 * (4 * (r & 7) + (r >> 3)); }
 __host__ __device__ constexpr int words_per_row(int bits) { return bits == 4 ? 4 : 3; }
 
 // Record a device-side error: the first non-zero code wins.

@@ -67,7 +67,7 @@ constexpr int kMaxPromoteGroups = 2;
 
 struct GemmArgs {
   const uint8_t* packed;
-  const uint16_t* scales;
+  const uint8_t* scales;    // the packed matrix's scale blocks (layout V2)
   const uint16_t* codebook;
   float* y;
   float* part;        // [kGemmMaxCtas][2][4][NT][32]: (CTA, slot, strip, column, row)
@@ -349,7 +349,9 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     UnitPos pf = cur;
     auto scale_of = [&](const UnitPos& p) -> uint32_t {
       const int64_t r0 = p.tau * kTileRows + sw * 32;
-      return r0 < a.N ? uint32_t(__ldg(a.scales + (r0 + lane) * a.G + p.g)) : 0u;
+      if (r0 >= a.N) return 0u;
+      const uint8_t* b = a.scales + ((r0 / kStrip) * a.G + p.g) * kScaleBytes + scale_slot(lane);
+      return uint32_t(__ldg(reinterpret_cast<const uint16_t*>(b)));
     };
 #pragma unroll
     for (int d = 0; d < SD; ++d) {
@@ -533,9 +535,9 @@ static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* scales,
-                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
-                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream) {
+cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
+                        int bits, int64_t N, int64_t K, float* y, void* workspace,
+                        int32_t* dev_status, int num_sms, cudaStream_t stream) {
   const int nt = gemm_nt(M);
   CUtensorMap map;
   std::memset(&map, 0, sizeof(map));
@@ -543,7 +545,7 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
   if (err != cudaSuccess) return err;
   GemmArgs a;
   a.packed = static_cast<const uint8_t*>(packed);
-  a.scales = static_cast<const uint16_t*>(scales);
+  a.scales = a.packed + (N / kStrip) * (K / kGroup) * tile_bytes(bits);
   a.codebook = static_cast<const uint16_t*>(codebook);
   a.y = y;
   a.dev_status = dev_status;

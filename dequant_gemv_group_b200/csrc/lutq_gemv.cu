@@ -60,8 +60,7 @@ constexpr int kMaxSmemPerBlock = 227 * 1024;
 
 struct GemvArgs {
   const uint16_t* x;        // bf16 [M, K]
-  const uint8_t* packed;    // layout V1
-  const uint16_t* scales;   // bf16 [N, G]
+  const uint8_t* packed;    // layout V2 (codes and scales)
   const uint16_t* codebook; // bf16 [2^bits]
   float* y;                 // fp32 [M, N]
   unsigned long long* xch;  // [M][N] exchange slots of strips split between two CTAs (zero between calls)
@@ -72,8 +71,8 @@ struct GemvArgs {
   // aligned if `align`; kind 1 = the first Cm CTAs take groups [0, G - T) of
   // one strip each, the others groups [G - T, G) of nh strips each
   uint32_t kind, align, Cm, T, nh;
-  // The grid's first pf_ctas CTAs only bring the packed matrix and the
-  // scales into L2 (the work goes to CTAs pf_ctas .. pf_ctas + C - 1)
+  // The grid's first pf_ctas CTAs only bring the packed matrix into L2
+  // (the work goes to CTAs pf_ctas .. pf_ctas + C - 1)
   uint32_t pf_ctas;
 };
 
@@ -339,45 +338,41 @@ __device__ __forceinline__ uint32_t lane_hi_delta(int q) {
 // The lane's share of one unit, loaded only if live > 0 (otherwise nothing is
 // read and the registers are left as they are): row i's 16 bytes of the tile
 // at p (4-bit: one word; 3-bit: 8 lo-plane bytes, then the 8 hi-plane bytes
-// hi_delta further on) into wd[i], row i's scale s[i][0] into sv[i].  One
-// predicate serves all eight loads.
+// hi_delta further on) into wd[i], and the scales of rows 0..3 (bf16 pairs:
+// rows 0, 1 and rows 2, 3) from ps into sv.  One predicate serves all loads.
 template <int BITS>
-__device__ __forceinline__ void fetch_unit(uint4 (&wd)[4], uint32_t (&sv)[4], const uint8_t* p,
-                                           uint32_t hi_delta, const uint16_t* s0,
-                                           const uint16_t* s1, const uint16_t* s2,
-                                           const uint16_t* s3, int live) {
+__device__ __forceinline__ void fetch_unit(uint4 (&wd)[4], uint32_t (&sv)[2], const uint8_t* p,
+                                           uint32_t hi_delta, const uint8_t* ps, int live) {
   if (BITS == 4) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.gt.s32 p, %25, 0;\n\t"
-        "@p ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%20];\n\t"
-        "@p ld.global.nc.L1::no_allocate.v4.u32 {%4, %5, %6, %7}, [%20+128];\n\t"
-        "@p ld.global.nc.L1::no_allocate.v4.u32 {%8, %9, %10, %11}, [%20+256];\n\t"
-        "@p ld.global.nc.L1::no_allocate.v4.u32 {%12, %13, %14, %15}, [%20+384];\n\t"
-        "@p ld.global.nc.u16 %16, [%21];\n\t@p ld.global.nc.u16 %17, [%22];\n\t"
-        "@p ld.global.nc.u16 %18, [%23];\n\t@p ld.global.nc.u16 %19, [%24];\n\t}"
+        "{\n\t.reg .pred p;\n\tsetp.gt.s32 p, %20, 0;\n\t"
+        "@p ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%18];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v4.u32 {%4, %5, %6, %7}, [%18+128];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v4.u32 {%8, %9, %10, %11}, [%18+256];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v4.u32 {%12, %13, %14, %15}, [%18+384];\n\t"
+        "@p ld.global.nc.v2.u32 {%16, %17}, [%19];\n\t}"
         : "=r"(wd[0].x), "=r"(wd[0].y), "=r"(wd[0].z), "=r"(wd[0].w), "=r"(wd[1].x),
           "=r"(wd[1].y), "=r"(wd[1].z), "=r"(wd[1].w), "=r"(wd[2].x), "=r"(wd[2].y),
           "=r"(wd[2].z), "=r"(wd[2].w), "=r"(wd[3].x), "=r"(wd[3].y), "=r"(wd[3].z),
-          "=r"(wd[3].w), "=r"(sv[0]), "=r"(sv[1]), "=r"(sv[2]), "=r"(sv[3])
-        : "l"(p), "l"(s0), "l"(s1), "l"(s2), "l"(s3), "r"(live));
+          "=r"(wd[3].w), "=r"(sv[0]), "=r"(sv[1])
+        : "l"(p), "l"(ps), "r"(live));
   } else {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.gt.s32 p, %26, 0;\n\t"
-        "@p ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%20];\n\t"
-        "@p ld.global.nc.v2.u32 {%2, %3}, [%21];\n\t"
-        "@p ld.global.nc.L1::no_allocate.v2.u32 {%4, %5}, [%20+128];\n\t"
-        "@p ld.global.nc.v2.u32 {%6, %7}, [%21+128];\n\t"
-        "@p ld.global.nc.L1::no_allocate.v2.u32 {%8, %9}, [%20+256];\n\t"
-        "@p ld.global.nc.v2.u32 {%10, %11}, [%21+256];\n\t"
-        "@p ld.global.nc.L1::no_allocate.v2.u32 {%12, %13}, [%20+384];\n\t"
-        "@p ld.global.nc.v2.u32 {%14, %15}, [%21+384];\n\t"
-        "@p ld.global.nc.u16 %16, [%22];\n\t@p ld.global.nc.u16 %17, [%23];\n\t"
-        "@p ld.global.nc.u16 %18, [%24];\n\t@p ld.global.nc.u16 %19, [%25];\n\t}"
+        "{\n\t.reg .pred p;\n\tsetp.gt.s32 p, %21, 0;\n\t"
+        "@p ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%18];\n\t"
+        "@p ld.global.nc.v2.u32 {%2, %3}, [%19];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v2.u32 {%4, %5}, [%18+128];\n\t"
+        "@p ld.global.nc.v2.u32 {%6, %7}, [%19+128];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v2.u32 {%8, %9}, [%18+256];\n\t"
+        "@p ld.global.nc.v2.u32 {%10, %11}, [%19+256];\n\t"
+        "@p ld.global.nc.L1::no_allocate.v2.u32 {%12, %13}, [%18+384];\n\t"
+        "@p ld.global.nc.v2.u32 {%14, %15}, [%19+384];\n\t"
+        "@p ld.global.nc.v2.u32 {%16, %17}, [%20];\n\t}"
         : "=r"(wd[0].x), "=r"(wd[0].y), "=r"(wd[0].z), "=r"(wd[0].w), "=r"(wd[1].x),
           "=r"(wd[1].y), "=r"(wd[1].z), "=r"(wd[1].w), "=r"(wd[2].x), "=r"(wd[2].y),
           "=r"(wd[2].z), "=r"(wd[2].w), "=r"(wd[3].x), "=r"(wd[3].y), "=r"(wd[3].z),
-          "=r"(wd[3].w), "=r"(sv[0]), "=r"(sv[1]), "=r"(sv[2]), "=r"(sv[3])
-        : "l"(p), "l"(p + hi_delta), "l"(s0), "l"(s1), "l"(s2), "l"(s3), "r"(live));
+          "=r"(wd[3].w), "=r"(sv[0]), "=r"(sv[1])
+        : "l"(p), "l"(p + hi_delta), "l"(ps), "r"(live));
   }
 }
 
@@ -426,12 +421,10 @@ __device__ __forceinline__ void unit_partial(float (&su)[4][M], const uint4 (&wd
 
 // Prefetch depth NB: tiles in registers, the one being consumed and the next
 // (a third buffer measured 2% slower on the 4096 x 14336 layer once the
-// weights come from L2).  kFourBases: the four scale rows of a lane get a
-// base address each (one fewer add per load, eight more registers).
+// weights come from L2).
 template <int BITS, int M>
 struct SmallCfg {
   static constexpr int NB = 2;
-  static constexpr bool kFourBases = M == 1 || (BITS == 4 && M >= 3);
 };
 
 // base + i * scale as one wide multiply-add (i, scale 32-bit).
@@ -469,17 +462,14 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 
   // A grid smaller than the GPU starts with pf_ctas CTAs that find free
   // multiprocessors while the preceding kernel on the stream still runs:
-  // they bring the whole packed matrix and the scales into L2, line by line,
-  // and leave (a prefetch reads nothing into the kernel, so it needs no wait
-  // for the preceding kernel).
+  // they bring the whole packed matrix into L2, line by line, and leave (a
+  // prefetch reads nothing into the kernel, so it needs no wait for the
+  // preceding kernel).
   if (blockIdx.x < a.pf_ctas) {
-    const uint32_t pk_lines = uint32_t(a.U) * uint32_t(TB / 128);
-    const uint32_t sc_lines = uint32_t((uint64_t(a.N) * G * 2u + 127u) / 128u);
-    const uint8_t* const sc = reinterpret_cast<const uint8_t*>(a.scales);
-    for (uint32_t j = blockIdx.x * blockDim.x + threadIdx.x; j < pk_lines + sc_lines;
+    const uint32_t lines = uint32_t((uint64_t(a.U) * (TB + kScaleBytes) + 127u) / 128u);
+    for (uint32_t j = blockIdx.x * blockDim.x + threadIdx.x; j < lines;
          j += a.pf_ctas * blockDim.x)
-      prefetch_l2(j < pk_lines ? a.packed + uint64_t(j) * 128u
-                               : sc + uint64_t(j - pk_lines) * 128u);
+      prefetch_l2(a.packed + uint64_t(j) * 128u);
     return;
   }
   const Span sp = cta_span(a, blockIdx.x - a.pf_ctas);
@@ -491,29 +481,22 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
   const int q = lane >> 3, rq = lane & 7;
 
   // Fetch cursor, in the order of the positions: tile index ft (strip * G +
-  // group) and scale index fs (strip * 32 G + group) of the next unit to
-  // load; fleft units until the end of the window in that strip (the window's
-  // first group of the next strip follows); fn units still to load.
+  // group) of the next unit to load; fleft units until the end of the window
+  // in that strip (the window's first group of the next strip follows); fn
+  // units still to load.
   uint32_t ft = first_strip * G + sp.ga + g_first;
-  uint32_t fs = first_strip * uint32_t(kStrip) * G + sp.ga + g_first;
   uint32_t fleft = sp.W - g_first;
   int fn = int(u1 - u0);
   const uint32_t lane_off = lane_tile_offset<BITS>(q, rq);
   const uint32_t hi_delta = BITS == 3 ? lane_hi_delta(q) : 0u;
   const uint8_t* const pk = a.packed + lane_off;
-  // the lane's rows rq + 8 i are 8 G scales apart; with many accumulators
-  // live, the four addresses are formed from one base (fewer registers)
-  constexpr bool kFourBases = SmallCfg<BITS, M>::kFourBases;
-  const uint16_t* const sc0 = a.scales + uint64_t(rq) * G;
-  const uint16_t* const sc1 = kFourBases ? sc0 + 8u * G : sc0;
-  const uint16_t* const sc2 = kFourBases ? sc1 + 8u * G : sc0;
-  const uint16_t* const sc3 = kFourBases ? sc2 + 8u * G : sc0;
-  const uint32_t g8 = kFourBases ? 0u : 8u * G;
+  // the scales of the lane's rows rq + 8 i, i = 0..3: 8 bytes of each unit's 64
+  const uint8_t* const psc = a.packed + uint64_t(a.U) * TB + scale_slot(rq);
 
   // Before the preceding kernel on the stream is complete (this kernel is
   // its programmatic dependent) nothing is read.  Without prefetching CTAs,
-  // the warp's first tiles and scales are brought into L2 (which keeps no
-  // stale copy) meanwhile; the values are loaded after the wait below.
+  // the warp's first tiles are brought into L2 (which keeps no stale copy)
+  // meanwhile; the values are loaded after the wait below.
   if (a.pf_ctas == 0 && u0 < u1) {
     uint32_t t = ft, l = fleft;
 #pragma unroll
@@ -522,18 +505,13 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
         const uint8_t* p = wide_addr(pk, t, uint32_t(TB));
 #pragma unroll
         for (int i = 0; i < 4; ++i) prefetch_l2(p + 128 * i);
+        if (lane == 0) prefetch_l2(wide_addr(psc, t, uint32_t(kScaleBytes)));
       }
       ++t;
       if (--l == 0) {
         t += G - sp.W;
         l = sp.W;
       }
-    }
-    if (q == 0) {
-      prefetch_l2(sc0 + fs);
-      prefetch_l2(sc1 + (fs + g8));
-      prefetch_l2(sc2 + (fs + 2u * g8));
-      prefetch_l2(sc3 + (fs + 3u * g8));
     }
   }
   if (threadIdx.x == 0) prefetch_l2(a.codebook);
@@ -546,16 +524,13 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
     return;
   }
 
-  auto fetch = [&](uint4 (&wd)[4], uint32_t (&sv)[4]) {
-    fetch_unit<BITS>(wd, sv, wide_addr(pk, ft, TB), hi_delta, wide_addr(sc0, fs, 2u),
-                     wide_addr(sc1, fs + g8, 2u), wide_addr(sc2, fs + 2u * g8, 2u),
-                     wide_addr(sc3, fs + 3u * g8, 2u), fn);
+  auto fetch = [&](uint4 (&wd)[4], uint32_t (&sv)[2]) {
+    fetch_unit<BITS>(wd, sv, wide_addr(pk, ft, TB), hi_delta,
+                     wide_addr(psc, ft, uint32_t(kScaleBytes)), fn);
     --fn;
     ++ft;
-    ++fs;
     if (--fleft == 0) {  // on to the window's first group of the next strip
       ft += G - sp.W;
-      fs += uint32_t(kStrip) * G - sp.W;
       fleft = sp.W;
     }
   };
@@ -565,7 +540,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
   // codebook[t mod 2^BITS], and the table is built from it with shuffles)
   // and the first tile; the other NB - 1 tiles once the activations are in.
   uint4 buf[NB][4];
-  uint32_t sbuf[NB][4];
+  uint32_t sbuf[NB][2];
   uint32_t cbv;
   {
     constexpr uint32_t kStep = kM1Warps * 32 * 16;
@@ -619,12 +594,12 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 #pragma unroll
       for (int m = 0; m < M; ++m) acc[i][m] = 0.0f;
     // Consume the unit held in (wd, sv); true once the range is done.
-    auto step = [&](const uint4 (&wd)[4], const uint32_t (&sv)[4]) -> bool {
+    auto step = [&](const uint4 (&wd)[4], const uint32_t (&sv)[2]) -> bool {
       float su[4][M];
       unit_partial<BITS, M>(su, wd, lane_e, lane_o, hi_shift, xa, xstride);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float s = __uint_as_float(sv[i] << 16);
+        const float s = (i & 1) ? bf16_hi_to_f32(sv[i >> 1]) : bf16_lo_to_f32(sv[i >> 1]);
 #pragma unroll
         for (int m = 0; m < M; ++m) acc[i][m] = fmaf(s, su[i][m], acc[i][m]);
       }
@@ -758,7 +733,7 @@ void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out) {
   out[5] = int32_t(pl.nh);
 }
 
-// A matrix (packed bytes and scales) up to this size is brought into L2
+// A packed matrix up to this size is brought into L2
 // ahead of the loads by prefetching CTAs on the multiprocessors the plan
 // leaves free.
 constexpr int64_t kPrefetchBytes = int64_t(64) << 20;
@@ -771,7 +746,7 @@ static void apply_plan(GemvArgs& a, int num_sms, int bits) {
   a.Cm = pl.Cm;
   a.T = pl.T;
   a.nh = pl.nh;
-  const int64_t bytes = a.U * tile_bytes(bits) + a.N * a.G * 2;
+  const int64_t bytes = a.U * (tile_bytes(bits) + kScaleBytes);
   a.pf_ctas = pl.C < num_sms && bytes <= kPrefetchBytes ? uint32_t(num_sms - pl.C) : 0u;
 }
 
@@ -802,9 +777,9 @@ static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, gemv_small_kernel<BITS, M>, a);
 }
 
-cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* scales,
-                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
-                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
+                        int bits, int64_t N, int64_t K, float* y, void* workspace,
+                        int32_t* dev_status, int num_sms, cudaStream_t stream);
 
 // Batches up to kMaxSmallBatch run on the CUDA cores when their activations
 // fit the small-batch kernel's shared memory.  Larger batches are a dense
@@ -828,13 +803,12 @@ static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream
   }
 }
 
-cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* scales,
-                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
-                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream) {
+cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
+                        int bits, int64_t N, int64_t K, float* y, void* workspace,
+                        int32_t* dev_status, int num_sms, cudaStream_t stream) {
   GemvArgs a;
   a.x = static_cast<const uint16_t*>(x);
   a.packed = static_cast<const uint8_t*>(packed);
-  a.scales = static_cast<const uint16_t*>(scales);
   a.codebook = static_cast<const uint16_t*>(codebook);
   a.y = y;
   a.xch = static_cast<unsigned long long*>(workspace);
@@ -848,7 +822,7 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   const bool small = bits == 4 ? small_fits<4>(M, K) : small_fits<3>(M, K);
   if (!small)
-    return launch_gemm(x, M, packed, scales, codebook, bits, N, K, y, workspace, dev_status,
+    return launch_gemm(x, M, packed, codebook, bits, N, K, y, workspace, dev_status,
                        num_sms, stream);
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
                    : launch_bits<3>(a, int(M), num_sms, stream);

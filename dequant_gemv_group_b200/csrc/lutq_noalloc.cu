@@ -22,9 +22,9 @@
 #include "lutq_common.cuh"
 
 namespace lutq {
-cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* scales,
-                        const void* codebook, int bits, int64_t N, int64_t K, float* y,
-                        void* workspace, int32_t* dev_status, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
+                        int bits, int64_t N, int64_t K, float* y, void* workspace,
+                        int32_t* dev_status, int num_sms, cudaStream_t stream);
 int64_t gemv_workspace_bytes(int64_t M, int64_t N);
 }  // namespace lutq
 
@@ -44,17 +44,16 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 
 extern "C" lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const void* packed,
-                                         const void* scales_bf16, const void* codebook_bf16,
-                                         int bits, int64_t N, int64_t K, float* y,
-                                         int32_t* dev_status, void* stream) {
-  if (!x_bf16 || !packed || !scales_bf16 || !codebook_bf16 || !y) return LUTQ_ERR_INVALID_ARG;
+                                         const void* codebook_bf16, int bits, int64_t N,
+                                         int64_t K, float* y, int32_t* dev_status,
+                                         void* stream) {
+  if (!x_bf16 || !packed || !codebook_bf16 || !y) return LUTQ_ERR_INVALID_ARG;
   if (bits != 3 && bits != 4) return LUTQ_ERR_BITS;
   if (N < lutq::kStrip || K < lutq::kGroup || N % lutq::kStrip != 0 || K % lutq::kGroup != 0 ||
       N > (int64_t(1) << 31) || K > (int64_t(1) << 31))
     return LUTQ_ERR_SHAPE;
   if (M < 1 || M > 16) return LUTQ_ERR_SHAPE;
-  if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(scales_bf16) ||
-      !aligned16(codebook_bf16) || !aligned16(y))
+  if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(codebook_bf16) || !aligned16(y))
     return LUTQ_ERR_ALIGN;
   // The fixed array must hold this problem's scratch; nothing is launched if not.
   const int64_t need = lutq::gemv_workspace_bytes(M, N);
@@ -80,7 +79,7 @@ extern "C" lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const vo
   if (cudaMemsetAsync(g_scratch_addr[dev], 0, size_t(need), s) != cudaSuccess)
     return LUTQ_ERR_CUDA;
   const cudaError_t err =
-      lutq::launch_gemv(x_bf16, M, packed, scales_bf16, codebook_bf16, bits, N, K, y,
-                        g_scratch_addr[dev], dev_status, g_scratch_sms[dev], s);
+      lutq::launch_gemv(x_bf16, M, packed, codebook_bf16, bits, N, K, y, g_scratch_addr[dev],
+                        dev_status, g_scratch_sms[dev], s);
   return err == cudaSuccess ? LUTQ_OK : LUTQ_ERR_CUDA;
 }

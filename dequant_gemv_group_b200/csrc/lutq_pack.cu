@@ -1,11 +1,15 @@
-// Offline restructuring of the codes into layout V1 (the FLUTE abstract,
-// "Daily Papers" listing: repack the quantized matrix offline so that the
-// product kernel needs few bit operations to unpack, including 3-bit widths).
+// Offline restructuring of the codes and scales into layout V2 (the FLUTE
+// abstract, "Daily Papers" listing: repack the quantized matrix offline so
+// that the product kernel needs few bit operations to unpack, including 3-bit
+// widths).
 //
 // One thread writes one 16-byte output word; threads are numbered in output
-// order, so a warp writes 512 contiguous bytes.  Word id -> (tile, w, r):
-// r = id % 32, w = (id / 32) % words_per_row, tile = id / (32 * words_per_row),
-// tile = strip * G + g.  Codes >= 2^bits are reported and masked.
+// order, so a warp writes 512 contiguous bytes.  The U * 32 * words_per_row
+// code words come first: word id -> (tile, w, r) with r = id % 32,
+// w = (id / 32) % words_per_row, tile = id / (32 * words_per_row) =
+// strip * G + g.  Then 4 words of scales per tile: word j of tile t holds
+// slots 8 j .. 8 j + 7, slot 4 rq + i being row rq + 8 i.  Codes >= 2^bits
+// are reported and masked.
 #include "lutq_common.cuh"
 
 namespace lutq {
@@ -22,18 +26,36 @@ __device__ __forceinline__ void load_codes(const uint8_t* p, uint8_t* out, int n
 
 template <int BITS>
 __global__ void __launch_bounds__(256)
-pack_kernel(const uint8_t* __restrict__ codes, int64_t N, int64_t K, uint4* __restrict__ packed,
-            int32_t* dev_status) {
+pack_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t N,
+            int64_t K, uint4* __restrict__ packed, int32_t* dev_status) {
   constexpr int WPR = words_per_row(BITS);
+  constexpr int CW = WPR * kStrip;               // code words of a tile
+  constexpr int SW = kScaleBytes / 16;           // scale words of a tile
   constexpr uint32_t kMask = (1u << BITS) - 1u;
   const int64_t G = K / kGroup;
-  const int64_t words = (N / kStrip) * G * WPR * kStrip;
+  const int64_t U = (N / kStrip) * G;
+  const int64_t words = U * (CW + SW);
   bool bad = false;
   for (int64_t id = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; id < words;
        id += int64_t(gridDim.x) * blockDim.x) {
+    if (id >= U * CW) {
+      // scale word: slots 8 j .. 8 j + 7 of its tile
+      const int64_t tile = (id - U * CW) / SW;
+      const int slot0 = 8 * int((id - U * CW) % SW);
+      const int64_t strip = tile / G, g = tile % G;
+      uint32_t h[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int slot = slot0 + t, r = (slot >> 2) + 8 * (slot & 3);
+        h[t] = scales[(strip * kStrip + r) * G + g];
+      }
+      packed[id] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
+                              h[6] | (h[7] << 16));
+      continue;
+    }
     const int r = int(id % kStrip);
     const int w = int((id / kStrip) % WPR);
-    const int64_t tile = id / (kStrip * WPR);
+    const int64_t tile = id / CW;
     const int64_t strip = tile / G, g = tile % G;
     const uint8_t* row = codes + (strip * kStrip + r) * K + g * kGroup;
     uint8_t out[16];
@@ -99,18 +121,20 @@ pack_kernel(const uint8_t* __restrict__ codes, int64_t N, int64_t K, uint4* __re
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) report(dev_status, LUTQ_ERR_CODE_RANGE);
 }
 
-cudaError_t launch_pack(const uint8_t* codes, int64_t N, int64_t K, int bits, void* packed,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream) {
-  const int64_t words = (N / kStrip) * (K / kGroup) * words_per_row(bits) * kStrip;
+cudaError_t launch_pack(const uint8_t* codes, const void* scales, int64_t N, int64_t K,
+                        int bits, void* packed, int32_t* dev_status, int num_sms,
+                        cudaStream_t stream) {
+  const int64_t words = (N / kStrip) * (K / kGroup) * ((tile_bytes(bits) + kScaleBytes) / 16);
   int64_t blocks = (words + 255) / 256;
   const int64_t cap = int64_t(num_sms) * 8;
   if (blocks > cap) blocks = cap;
+  const uint16_t* sc = static_cast<const uint16_t*>(scales);
   if (bits == 4)
-    pack_kernel<4><<<unsigned(blocks), 256, 0, stream>>>(codes, N, K, static_cast<uint4*>(packed),
-                                                        dev_status);
+    pack_kernel<4><<<unsigned(blocks), 256, 0, stream>>>(codes, sc, N, K,
+                                                        static_cast<uint4*>(packed), dev_status);
   else
-    pack_kernel<3><<<unsigned(blocks), 256, 0, stream>>>(codes, N, K, static_cast<uint4*>(packed),
-                                                        dev_status);
+    pack_kernel<3><<<unsigned(blocks), 256, 0, stream>>>(codes, sc, N, K,
+                                                        static_cast<uint4*>(packed), dev_status);
   return cudaGetLastError();
 }
 

@@ -12,6 +12,7 @@
  * Notation: W[N,K] bf16 weights (row n = output feature, K = reduction),
  * G = K/128 groups per row, codebook c[0 .. 2^bits - 1] (bf16), codes
  * q[N,K] (uint8), scales s[N,G] (bf16), x[M,K] bf16 activations, y[M,N] fp32.
+ * lutq_pack merges q and s into one packed matrix that the products read.
  * The dequantized weight is s[n, k/128] * c[q[n,k]].
  *
  * Conventions shared by every call:
@@ -64,12 +65,14 @@ typedef enum {
 const char* lutq_status_string(int status);
 
 /* Version of the packed layout produced by lutq_pack and read by lutq_gemv /
- * lutq_gemm.  Returns 1 for layout V1 (strips of 32 rows, 16-byte words
- * interleaved across the rows of a strip; see lutq_pack). */
+ * lutq_gemm.  Returns 2 for layout V2 (strips of 32 rows, 16-byte words
+ * interleaved across the rows of a strip, then the scales in blocks of 32;
+ * see lutq_pack). */
 int lutq_layout_version(void);
 
-/* Size in bytes of the packed codes of an N x K matrix: N*K/2 for 4 bits,
- * 3*N*K/8 for 3 bits.  Returns -1 for an invalid shape or bit width. */
+/* Size in bytes of the packed matrix (codes and scales) of an N x K matrix:
+ * N*K/2 + N*K/64 for 4 bits, 3*N*K/8 + N*K/64 for 3 bits.  Returns -1 for
+ * an invalid shape or bit width. */
 int64_t lutq_packed_bytes(int64_t N, int64_t K, int bits);
 
 /*
@@ -116,17 +119,22 @@ lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K,
                           int32_t* dev_status, void* stream);
 
 /*
- * lutq_pack - offline restructuring of the codes into layout V1.
+ * lutq_pack - offline restructuring of the codes and scales into layout V2.
  *
  * Source: the FLUTE abstract ("offline restructuring of the quantized weight
  * matrix to minimize bit manipulations associated with unpacking"; 3-bit,
  * non-evenly-divisible widths).
  *
- * Layout V1.  Rows form strips of 32; G = K/128.  The tile of (strip s,
- * group g) starts at byte (s*G + g)*T, T = 2048 (4 bit) or 1536 (3 bit).  A
- * tile is made of 16-byte words; word w of row r (0..31 within the strip) is at
- * byte (32*w + r)*16 of the tile, so one word index over a strip is 512
- * contiguous bytes (one coalesced 16-byte load per lane of a warp).
+ * Layout V2.  Rows form strips of 32; G = K/128; the unit t = s*G + g is
+ * (strip s, group g), U = (N/32)*G units.  The codes of unit t take C bytes
+ * at byte t*C, C = 2048 (4 bit) or 1536 (3 bit); its 32 scales take the 64
+ * bytes at U*C + t*64.  The codes are 16-byte words; word w of row r (0..31
+ * within the strip) is at byte (32*w + r)*16 of the unit's codes, so one word
+ * index over a strip is 512 contiguous bytes (one coalesced 16-byte load per
+ * lane of a warp).  The scale s[32s + r, g] (bf16 bits, little-endian) is at
+ * byte 2*(4*(r % 8) + r / 8) of the unit's 64: the four rows r0, r0+8,
+ * r0+16, r0+24 that one lane of the product kernel handles have their
+ * scales in 8 consecutive bytes.
  *  4 bit: words 0..3 hold k = 128g + 32w + 0..31; byte i holds the codes
  *         (k0+2i, k0+2i+1), the even one in the low nibble, so every byte is
  *         directly an index into a 256-entry table of code pairs.
@@ -141,11 +149,12 @@ lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K,
  *         yields four pair indices at once.
  *
  * codes  device, uint8 [N,K] (values < 2^bits).
+ * scales device, bf16 [N,K/128] row-major (as lutq_quantize writes them).
  * packed device, lutq_packed_bytes(N,K,bits) bytes, written.
  * dev_status device int32 or NULL: LUTQ_ERR_CODE_RANGE if a code >= 2^bits.
  */
-lutq_status lutq_pack(const uint8_t* codes, int64_t N, int64_t K, int bits,
-                      void* packed, int32_t* dev_status, void* stream);
+lutq_status lutq_pack(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
+                      int bits, void* packed, int32_t* dev_status, void* stream);
 
 /*
  * lutq_workspace_bytes - device scratch size needed by lutq_gemv / lutq_gemm
@@ -174,15 +183,14 @@ int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
  * depend on timing.
  * The CUDA-core kernel is launched as a programmatic dependent of the work
  * before it on `stream`: its set-up overlaps the end of that work, and when
- * its plan leaves multiprocessors free and the matrix (packed bytes and
- * scales) is at most 64 MiB, extra thread blocks on those multiprocessors
+ * its plan leaves multiprocessors free and the packed matrix is at most
+ * 64 MiB, extra thread blocks on those multiprocessors
  * bring the matrix into L2 meanwhile.  Nothing is read into the kernel
  * before the preceding work is complete, so the caller need not order
  * anything.
  *
  * x        device bf16 [M,K] row-major.
- * packed   device, layout V1 (lutq_pack).
- * scales   device bf16 [N,K/128] row-major.
+ * packed   device, layout V2 (lutq_pack): the codes and the scales s.
  * codebook device bf16 [1 << bits].
  * y        device fp32 [M,N] row-major, written (no accumulation into y).
  * workspace device, at least lutq_workspace_bytes(M,N,K,bits) bytes, zero-
@@ -194,8 +202,7 @@ int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
  * Returns LUTQ_ERR_SHAPE if M is outside 1..16.
  */
 lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
-                      const void* scales_bf16, const void* codebook_bf16,
-                      int bits, int64_t N, int64_t K, float* y,
+                      const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
                       void* workspace, int64_t workspace_bytes,
                       int32_t* dev_status, void* stream);
 
@@ -222,8 +229,8 @@ lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
  *    (8 * M * N bytes, rounded up to 256) exceeds 4 MiB.
  */
 lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const void* packed,
-                              const void* scales_bf16, const void* codebook_bf16,
-                              int bits, int64_t N, int64_t K, float* y,
+                              const void* codebook_bf16, int bits, int64_t N, int64_t K,
+                              float* y,
                               int32_t* dev_status, void* stream);
 
 /*
@@ -266,8 +273,7 @@ lutq_status lutq_selftest_wait_timeout(int32_t* dev_status, int64_t limit_ns, vo
  * LUTQ_ERR_TIMEOUT if a pipeline wait inside the kernel exceeds its bound.
  */
 lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
-                      const void* scales_bf16, const void* codebook_bf16,
-                      int bits, int64_t N, int64_t K, float* y,
+                      const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
                       void* workspace, int64_t workspace_bytes,
                       int32_t* dev_status, void* stream);
 

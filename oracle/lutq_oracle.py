@@ -45,8 +45,8 @@ import numpy as np
 import scipy.special
 
 GROUP = 128          # weights per quantization group along K
-STRIP = 32           # rows per packing strip (layout V1)
-LAYOUT_VERSION = 1
+STRIP = 32           # rows per packing strip (layout V2)
+LAYOUT_VERSION = 2
 
 CODEBOOK_KINDS = ("nf4", "logb", "lloyd_max3", "uniform4")
 
@@ -229,14 +229,17 @@ def quantize(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
 
 
 # --------------------------------------------------------------------------
-# Packing, layout V1 (the offline restructuring of the FLUTE abstract)
+# Packing, layout V2 (the offline restructuring of the FLUTE abstract)
 # --------------------------------------------------------------------------
 #
-# Rows come in strips of 32; groups are 128 codes along K.  The tile of
-# (strip s, group g) starts at byte (s * G + g) * T with T = 2048 (4-bit) or
-# 1536 (3-bit).  A tile is a sequence of 16-byte words; word w of row r (r in
-# 0..31 within the strip) sits at byte (32 * w + r) * 16 of the tile, so one
-# word index over a strip is 512 contiguous bytes.
+# Rows come in strips of 32; groups are 128 codes along K.  Unit t = s * G + g
+# is (strip s, group g); there are U = (N / 32) * G units.  The codes of unit
+# t take C bytes at byte t * C, C = 2048 (4-bit) or 1536 (3-bit); its 32
+# scales take the 64 bytes at U * C + t * 64.  The codes are a sequence of
+# 16-byte words; word w of row r (r in 0..31 within the strip) sits at byte
+# (32 * w + r) * 16 of the unit's codes, so one word index over a strip is 512
+# contiguous bytes.  The scale of row r (bf16 bits, little-endian) sits at
+# byte 2 * (4 * (r % 8) + r // 8) of the unit's 64.
 #
 # 4-bit: words w = 0..3 cover k = 128g + 32w + (0..31).  Byte i of the word
 #   holds the pair of codes (k0 + 2i, k0 + 2i + 1): even code in the low nibble.
@@ -253,12 +256,20 @@ def quantize(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
 #     bits 5:4 = hi2(pair 8j + b     of lo word 0)
 #     bits 7:6 = hi2(pair 8j + b     of lo word 1)
 
-def packed_bytes(n: int, k: int, bits: int) -> int:
+SCALE_BLOCK = 64     # bytes of one unit's scales
+
+
+def code_bytes(bits: int) -> int:
+    """Bytes of codes of one unit."""
     if bits == 4:
-        return n * k // 2
+        return 2048
     if bits == 3:
-        return 3 * n * k // 8
+        return 1536
     raise ValueError("bits must be 3 or 4")
+
+
+def packed_bytes(n: int, k: int, bits: int) -> int:
+    return (n // STRIP) * (k // GROUP) * (code_bytes(bits) + SCALE_BLOCK)
 
 
 def _check_shape(n: int, k: int) -> None:
@@ -266,11 +277,26 @@ def _check_shape(n: int, k: int) -> None:
         raise ValueError("N must be a multiple of 32 and K of 128")
 
 
-def pack(codes, bits: int) -> np.ndarray:
-    """codes uint8[N, K] -> packed uint8[packed_bytes(N, K, bits)] (layout V1)."""
+def pack(codes, scale_bits, bits: int) -> np.ndarray:
+    """codes uint8[N, K] and scale_bits uint16[N, K/128] (bf16 bits) ->
+    packed uint8[packed_bytes(N, K, bits)] (layout V2)."""
     q = np.asarray(codes, dtype=np.uint8)
     n, k = q.shape
     _check_shape(n, k)
+    sb = np.asarray(scale_bits, dtype=np.uint16)
+    if sb.shape != (n, k // GROUP):
+        raise ValueError("scales shape mismatch")
+    code_tiles = _pack_codes(q, bits)                       # [s, g, C]
+    ns, g = n // STRIP, k // GROUP
+    # row r = 8 i + rq of strip s -> scale position 4 rq + i
+    sc = sb.reshape(ns, 4, 8, g).transpose(0, 3, 2, 1)      # [s, g, rq, i]
+    sc_bytes = np.ascontiguousarray(sc).astype("<u2").view(np.uint8).reshape(-1)
+    return np.concatenate([code_tiles.reshape(-1), sc_bytes])
+
+
+def _pack_codes(q, bits: int) -> np.ndarray:
+    """The code bytes of every tile, [strips, groups, code_bytes(bits)]."""
+    n, k = q.shape
     if np.any(q >= (1 << bits)):
         raise ValueError("code out of range")
     ns, g = n // STRIP, k // GROUP
@@ -279,7 +305,7 @@ def pack(codes, bits: int) -> np.ndarray:
         t = q.reshape(ns, STRIP, g, 4, 16, 2)
         byte = t[..., 0] | (t[..., 1] << 4)                 # [s, r, g, w, i]
         tiles = byte.transpose(0, 2, 3, 1, 4)               # [s, g, w, r, i]
-        return np.ascontiguousarray(tiles).reshape(-1)
+        return np.ascontiguousarray(tiles).reshape(ns, g, -1)
     if bits == 3:
         # k = 128 g + 64 w + 16 j + 8 h + 2 b + e  (h: low/high nibble half)
         t = q.reshape(ns, STRIP, g, 2, 4, 2, 4, 2)
@@ -295,23 +321,29 @@ def pack(codes, bits: int) -> np.ndarray:
         hi_words = hi_byte.reshape(ns, STRIP, g, 1, 16)
         words = np.concatenate([lo_words, hi_words], axis=3)  # [s, r, g, 3, 16]
         tiles = words.transpose(0, 2, 3, 1, 4)              # [s, g, w, r, 16]
-        return np.ascontiguousarray(tiles).reshape(-1).astype(np.uint8)
+        return np.ascontiguousarray(tiles).reshape(ns, g, -1).astype(np.uint8)
     raise ValueError("bits must be 3 or 4")
 
 
-def unpack(packed, n: int, k: int, bits: int) -> np.ndarray:
-    """Inverse of :func:`pack`, written byte by byte from the layout text."""
+def unpack(packed, n: int, k: int, bits: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Inverse of :func:`pack`, written byte by byte from the layout text:
+    (codes uint8[N, K], scale_bits uint16[N, K/128])."""
     p = np.asarray(packed, dtype=np.uint8)
     _check_shape(n, k)
     if p.size != packed_bytes(n, k, bits):
         raise ValueError("packed size mismatch")
     g = k // GROUP
     q = np.zeros((n, k), dtype=np.uint8)
-    tile_bytes = 2048 if bits == 4 else 1536
+    sb = np.zeros((n, g), dtype=np.uint16)
+    cb = code_bytes(bits)
+    units = (n // STRIP) * g
     for row in range(n):
         s, r = divmod(row, STRIP)
         for gi in range(g):
-            base = (s * g + gi) * tile_bytes
+            t = s * g + gi
+            base = t * cb
+            at = units * cb + t * SCALE_BLOCK + 2 * (4 * (r % 8) + r // 8)
+            sb[row, gi] = int(p[at]) | (int(p[at + 1]) << 8)
             if bits == 4:
                 for w in range(4):
                     word = p[base + (32 * w + r) * 16: base + (32 * w + r) * 16 + 16]
@@ -335,7 +367,7 @@ def unpack(packed, n: int, k: int, bits: int) -> np.ndarray:
                                 kk = GROUP * gi + 64 * w + 2 * pair
                                 q[row, kk] = (l2 & 3) | ((h2 & 1) << 2)
                                 q[row, kk + 1] = ((l2 >> 2) & 3) | (((h2 >> 1) & 1) << 2)
-    return q
+    return q, sb
 
 
 # --------------------------------------------------------------------------

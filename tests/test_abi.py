@@ -36,7 +36,7 @@ def test_library_exports_every_declared_function(lq):
 
 
 def test_layout_version_and_sizes(lq):
-    assert lq.lutq_layout_version() == O.LAYOUT_VERSION == 1
+    assert lq.lutq_layout_version() == O.LAYOUT_VERSION == 2
     for n, k, bits in [(4096, 14336, 4), (4096, 4096, 3), (32, 128, 4), (28672, 8192, 3)]:
         assert lq.lutq_packed_bytes(n, k, bits) == O.packed_bytes(n, k, bits)
     assert lq.lutq_packed_bytes(33, 128, 4) == -1
@@ -84,24 +84,28 @@ def test_quantize_argument_errors(lq):
 
 def test_pack_argument_errors(lq):
     f = lq.lib.lutq_pack
-    assert f(None, 32, 128, 4, A, None, None) == 1
-    assert f(A, 32, 128, 2, A, None, None) == 3
-    assert f(A, 64, 64, 4, A, None, None) == 2
-    assert f(A, 32, 128, 4, A + 8, None, None) == 4
+    assert f(None, A, 32, 128, 4, A, None, None) == 1
+    assert f(A, None, 32, 128, 4, A, None, None) == 1             # null scales
+    assert f(A, A, 32, 128, 2, A, None, None) == 3
+    assert f(A, A, 64, 64, 4, A, None, None) == 2
+    assert f(A, A, 32, 128, 4, A + 8, None, None) == 4
+    assert f(A, A + 2, 32, 128, 4, A, None, None) == 4            # misaligned scales
 
 
 @pytest.mark.parametrize("name", ["lutq_gemv", "lutq_gemm"])
 def test_product_argument_errors(lq, name):
     f = getattr(lq.lib, name)
     ws = lq.lutq_workspace_bytes(1, 64, 256, 4)
-    ok = dict(x=A, m=1, p=A, s=A, c=A, bits=4, n=64, k=256, y=A, ws=A, wsb=ws)
+    ok = dict(x=A, m=1, p=A, c=A, bits=4, n=64, k=256, y=A, ws=A, wsb=ws)
 
     def call(**kw):
         a = dict(ok, **kw)
-        return f(a["x"], a["m"], a["p"], a["s"], a["c"], a["bits"], a["n"], a["k"], a["y"],
+        return f(a["x"], a["m"], a["p"], a["c"], a["bits"], a["n"], a["k"], a["y"],
                  a["ws"], a["wsb"], None, None)
 
     assert call(x=None) == 1
+    assert call(p=None) == 1
+    assert call(c=A + 8) == 4
     assert call(bits=2) == 3
     assert call(n=48) == 2
     assert call(k=200) == 2

@@ -30,7 +30,7 @@ def _prep(lq, w, kind, bits):
     cb = lq.lutq_codebook(kind, bits).cuda()
     st = lq.new_status()
     codes, scales = lq.lutq_quantize(w.cuda(), cb, bits, status=st)
-    packed = lq.lutq_pack(codes, bits, status=st)
+    packed = lq.lutq_pack(codes, scales, bits, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     return cb, codes, scales, packed
@@ -41,7 +41,7 @@ def _gemm(lq, x, packed, scales, cb, bits, n, k, ws=None):
     if ws is None:
         ws = lq.new_workspace(m, n, k, bits)
     st = lq.new_status()
-    y = lq.lutq_gemm(x.cuda(), packed, scales, cb, bits, n, k, workspace=ws, status=st)
+    y = lq.lutq_gemm(x.cuda(), packed, cb, bits, n, k, workspace=ws, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0, lq.lutq_status_string(int(st.item()))
     return y.cpu().numpy(), ws
@@ -94,7 +94,7 @@ def test_gemm_deterministic_and_agrees_with_gemv(lq):
     y2, _ = _gemm(lq, x, packed, scales, cb, 4, n, k, ws=ws)
     np.testing.assert_array_equal(y1, y2)
     st = lq.new_status()
-    yv = lq.lutq_gemv(x.cuda(), packed, scales, cb, 4, n, k, workspace=ws, status=st)
+    yv = lq.lutq_gemv(x.cuda(), packed, cb, 4, n, k, workspace=ws, status=st)
     torch.cuda.synchronize()
     assert O.rel_error_gate(y1, yv.cpu().numpy().astype(np.float64)) <= TOL
 

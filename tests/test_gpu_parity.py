@@ -45,7 +45,7 @@ def _quantize_pack(lq, w_cpu, kind, bits):
     cb, levels = _cb(lq, kind, bits)
     st = lq.new_status()
     codes, scales = lq.lutq_quantize(w_cpu.cuda(), cb, bits, status=st)
-    packed = lq.lutq_pack(codes, bits, status=st)
+    packed = lq.lutq_pack(codes, scales, bits, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     return cb, levels, codes, scales, packed
@@ -56,7 +56,7 @@ def _gemv(lq, x_cpu, packed, scales, cb, bits, n, k, ws=None):
     if ws is None:
         ws = lq.new_workspace(m, n, k, bits)
     st = lq.new_status()
-    y = lq.lutq_gemv(x_cpu.cuda(), packed, scales, cb, bits, n, k, workspace=ws, status=st)
+    y = lq.lutq_gemv(x_cpu.cuda(), packed, cb, bits, n, k, workspace=ws, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     return y.cpu().numpy(), ws
@@ -73,7 +73,7 @@ def test_quantize_and_pack_bit_exact(lq, kind, bits, n, k):
     ref_codes, ref_sb = O.quantize(_f32(w), levels, bits)
     np.testing.assert_array_equal(codes.cpu().numpy(), ref_codes)
     np.testing.assert_array_equal(_bits16(scales), ref_sb)
-    np.testing.assert_array_equal(packed.cpu().numpy(), O.pack(ref_codes, bits))
+    np.testing.assert_array_equal(packed.cpu().numpy(), O.pack(ref_codes, ref_sb, bits))
 
 
 def test_quantize_edge_cases(lq):
@@ -117,7 +117,8 @@ def test_pack_reports_code_range(lq):
     codes = torch.zeros((32, 128), dtype=torch.uint8)
     codes[5, 17] = 9
     st = lq.new_status()
-    lq.lutq_pack(codes.cuda(), 3, status=st)
+    scales = torch.ones((32, 1), dtype=torch.bfloat16, device="cuda")
+    lq.lutq_pack(codes.cuda(), scales, 3, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 6
 
@@ -188,13 +189,17 @@ def _full_size_case(lq, lay, kind, bits, batches):
     ref_codes, ref_sb = O.quantize(w_rows, levels, bits)
     np.testing.assert_array_equal(codes[rows].cpu().numpy(), ref_codes)
     np.testing.assert_array_equal(_bits16(scales[rows]), ref_sb)
-    # packed strips: tiles (s, 0..G-1) are contiguous
+    # packed strips: the codes of units (s, 0..G-1) are contiguous, and so
+    # are their scale blocks
     tb = 2048 if bits == 4 else 1536
     g = k // 128
+    units = (n // 32) * g
     pk = packed.cpu().numpy()
     for i, s in enumerate(strips):
-        want = O.pack(ref_codes[32 * i: 32 * i + 32], bits)
-        np.testing.assert_array_equal(pk[s * g * tb:(s + 1) * g * tb], want)
+        want = O.pack(ref_codes[32 * i: 32 * i + 32], ref_sb[32 * i: 32 * i + 32], bits)
+        np.testing.assert_array_equal(pk[s * g * tb:(s + 1) * g * tb], want[:g * tb])
+        sc0 = units * tb + s * g * 64
+        np.testing.assert_array_equal(pk[sc0:sc0 + g * 64], want[g * tb:])
     del w
     ws = lq.new_workspace(max(batches), n, k, bits)
     for m in batches:

@@ -48,9 +48,9 @@ def test_context_usable_after_timeout(lq):
     _, levels = O.codebook("nf4", bits)
     st2 = lq.new_status()
     codes, scales = lq.lutq_quantize(w.cuda(), cb.cuda(), bits, status=st2)
-    packed = lq.lutq_pack(codes, bits, status=st2)
+    packed = lq.lutq_pack(codes, scales, bits, status=st2)
     x = workloads.activations(1, k, seed=4)
-    y = lq.lutq_gemv(x.cuda(), packed, scales, cb.cuda(), bits, n, k,
+    y = lq.lutq_gemv(x.cuda(), packed, cb.cuda(), bits, n, k,
                      workspace=lq.new_workspace(1, n, k, bits), status=st2)
     torch.cuda.synchronize()
     assert int(st.item()) == LUTQ_ERR_TIMEOUT

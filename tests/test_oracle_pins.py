@@ -295,27 +295,35 @@ def test_quantize_rejects_nonfinite():
 
 # ---------------------------------------------------------------- packing
 
+def _zero_scales(n, k):
+    return np.zeros((n, k // 128), np.uint16)
+
+
 def test_packed_size_formula():
-    assert O.packed_bytes(4096, 14336, 4) == 4096 * 14336 // 2
-    assert O.packed_bytes(4096, 4096, 3) == 3 * 4096 * 4096 // 8
+    # codes (4 or 3 bits per weight) plus one 16-bit scale per 128 weights
+    assert O.packed_bytes(4096, 14336, 4) == 4096 * 14336 // 2 + 4096 * 14336 // 64
+    assert O.packed_bytes(4096, 4096, 3) == 3 * 4096 * 4096 // 8 + 4096 * 4096 // 64
     q = np.zeros((64, 256), np.uint8)
-    assert O.pack(q, 4).size == 64 * 256 // 2
-    assert O.pack(q, 3).size == 3 * 64 * 256 // 8
+    assert O.pack(q, _zero_scales(64, 256), 4).size == 64 * 256 // 2 + 64 * 256 // 64
+    assert O.pack(q, _zero_scales(64, 256), 3).size == 3 * 64 * 256 // 8 + 64 * 256 // 64
 
 
 @pytest.mark.parametrize("bits", [3, 4])
 def test_pack_unpack_roundtrip(bits):
     rng = np.random.default_rng(bits)
     q = rng.integers(0, 1 << bits, size=(64, 384), dtype=np.uint8)
-    np.testing.assert_array_equal(O.unpack(O.pack(q, bits), 64, 384, bits), q)
+    sb = rng.integers(0, 1 << 16, size=(64, 3), dtype=np.uint16)
+    q2, sb2 = O.unpack(O.pack(q, sb, bits), 64, 384, bits)
+    np.testing.assert_array_equal(q2, q)
+    np.testing.assert_array_equal(sb2, sb)
 
 
 def test_pack_w4_hand_derived_bytes():
     n, k = 64, 256
     nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
     q = ((nn + kk + 5 * (kk // 32)) % 16).astype(np.uint8)
-    p = O.pack(q, 4)
-    with open(os.path.join(GOLDEN, "pack_v1_w4_pattern.txt")) as f:
+    p = O.pack(q, _zero_scales(n, k), 4)
+    with open(os.path.join(GOLDEN, "pack_v2_w4_pattern.txt")) as f:
         for line in f:
             if line.startswith("#") or not line.strip():
                 continue
@@ -325,8 +333,28 @@ def test_pack_w4_hand_derived_bytes():
             assert bytes(p[off:off + 16]) == want, off
 
 
+def test_pack_scales_hand_derived_bytes():
+    n, k = 64, 256
+    nn, gg = np.meshgrid(np.arange(n), np.arange(k // 128), indexing="ij")
+    sb = (0x3C00 + 4 * nn + gg).astype(np.uint16)
+    p = O.pack(np.zeros((n, k), np.uint8), sb, 4)
+    seen = 0
+    with open(os.path.join(GOLDEN, "pack_v2_scales.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            parts = line.split()
+            off = int(parts[0])
+            assert bytes(p[off:off + 2]) == bytes(int(b, 16) for b in parts[1:]), off
+            seen += 1
+    assert seen == 5
+    # every code byte is zero; the scale blocks hold all 128 scales once
+    assert not p[:8192].any()
+    assert sorted(p[8192:].copy().view("<u2").tolist()) == sorted(sb.reshape(-1).tolist())
+
+
 def test_pack_w3_hand_derived_probes():
-    with open(os.path.join(GOLDEN, "pack_v1_w3_probes.txt")) as f:
+    with open(os.path.join(GOLDEN, "pack_v2_w3_probes.txt")) as f:
         for line in f:
             if line.startswith("#") or not line.strip():
                 continue
@@ -334,7 +362,7 @@ def test_pack_w3_hand_derived_probes():
             _, row, kk, qv = left.split()
             q = np.zeros((32, 128), np.uint8)
             q[int(row), int(kk)] = int(qv)
-            p = O.pack(q, 3)
+            p = O.pack(q, _zero_scales(32, 128), 3)
             vals = right.split()
             want = {int(vals[i]): int(vals[i + 1], 16) for i in range(0, len(vals), 2)}
             nz = {int(i): int(p[i]) for i in np.nonzero(p)[0]}

@@ -36,18 +36,17 @@ def test_noalloc_matches_workspace_gemv_twice(lq, n, k, bits, kind, m):
     w = workloads.normal_weights(n, k, 0.02, seed=21, outlier_frac=1e-3).cuda()
     cb = lq.lutq_codebook(kind, bits).cuda()
     codes, scales = lq.lutq_quantize(w, cb, bits)
-    packed = lq.lutq_pack(codes, bits)
+    packed = lq.lutq_pack(codes, scales, bits)
     x = workloads.activations(m, k, seed=22).cuda()
     ws = lq.new_workspace(m, n, k, bits)
-    y_ref = lq.lutq_gemv(x, packed, scales, cb, bits, n, k, workspace=ws)
+    y_ref = lq.lutq_gemv(x, packed, cb, bits, n, k, workspace=ws)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream().cuda_stream
     for _ in range(2):
         y = torch.full((m, n), float("nan"), dtype=torch.float32, device="cuda")
         st = lq.new_status()
-        rc = lq.lib.lutq_gemv_noalloc(x.data_ptr(), m, packed.data_ptr(), scales.data_ptr(),
-                                      cb.data_ptr(), bits, n, k, y.data_ptr(), st.data_ptr(),
-                                      stream)
+        rc = lq.lib.lutq_gemv_noalloc(x.data_ptr(), m, packed.data_ptr(), cb.data_ptr(), bits,
+                                      n, k, y.data_ptr(), st.data_ptr(), stream)
         torch.cuda.synchronize()
         assert rc == 0, lq.lutq_status_string(rc)
         assert int(st.item()) == 0
@@ -59,5 +58,5 @@ def test_noalloc_rejects_problems_beyond_its_array(lq):
     # size check comes before any device work, so aligned placeholder
     # addresses are never touched.
     a = 1 << 20
-    rc = lq.lib.lutq_gemv_noalloc(a, 1, a, a, a, 4, 1 << 26, 128, a, None, None)
+    rc = lq.lib.lutq_gemv_noalloc(a, 1, a, a, 4, 1 << 26, 128, a, None, None)
     assert rc == 9
