@@ -419,13 +419,10 @@ __device__ __forceinline__ void unit_partial(float (&su)[4][M], const uint4 (&wd
   }
 }
 
-// Prefetch depth NB: tiles in registers, the one being consumed and the next
-// (a third buffer measured 2% slower on the 4096 x 14336 layer once the
-// weights come from L2).
-template <int BITS, int M>
-struct SmallCfg {
-  static constexpr int NB = 2;
-};
+// Prefetch depth NB: tiles in registers ahead of the one being consumed.
+// Two when prefetching blocks have brought the weights into L2 (a third
+// buffer measured 2% slower on the 4096 x 14336 layer); three for a single
+// batch row whose weights come from HBM (4% faster on 8192 x 28672, 3 bit).
 
 // base + i * scale as one wide multiply-add (i, scale 32-bit).
 template <typename T>
@@ -450,9 +447,8 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-template <int BITS, int M>
+template <int BITS, int M, int NB>
 __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a) {
-  constexpr int NB = SmallCfg<BITS, M>::NB;
   constexpr int TB = tile_bytes(BITS);
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ WarpTable<kM1Warps> wt;
@@ -757,11 +753,14 @@ static int64_t small_smem(int64_t K, int M) {
 
 template <int BITS, int M>
 static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
-  static SmemGrant grant;
+  static SmemGrant grant2, grant3;
   const int smem = int(small_smem(a.K, M));
-  cudaError_t err = grant_smem(gemv_small_kernel<BITS, M>, grant, smem);
-  if (err != cudaSuccess) return err;
   apply_plan(a, num_sms, BITS);
+  constexpr int kDeep = M == 1 ? 3 : 2;
+  const bool deep = M == 1 && a.pf_ctas == 0;
+  auto kernel = deep ? gemv_small_kernel<BITS, M, kDeep> : gemv_small_kernel<BITS, M, 2>;
+  cudaError_t err = grant_smem(kernel, deep ? grant3 : grant2, smem);
+  if (err != cudaSuccess) return err;
   // programmatic dependent launch: the prefetching blocks and the work
   // blocks' set-up may overlap the end of the preceding kernel on the stream
   cudaLaunchConfig_t cfg = {};
@@ -774,7 +773,7 @@ static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_small_kernel<BITS, M>, a);
+  return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
