@@ -64,6 +64,7 @@ struct GemmCfg {
   static_assert(DCOL + DS * NT <= kTmemCols, "tensor memory columns");
 };
 constexpr int kMaxPromoteGroups = 2;
+constexpr int kScaleRingBytes = 4 * kMaxPromoteGroups * 4 * 32 * 4;  // [warp][SD][lane] u32
 
 struct GemmArgs {
   const uint8_t* packed;
@@ -343,19 +344,30 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     const int sw = warp & 3, pg = (warp - DW) >> 2;
     UnitPos cur;
     cur.init(u0, per_bt, a.G);
-    // The group scales of the next SD units are loaded ahead.
+    // The group scales of the next SD units travel ahead of use through a
+    // ring in shared memory (one 4-byte asynchronous copy per lane and unit,
+    // one copy group per unit): waiting for unit i's group never waits for a
+    // later unit's load.  Holding the ring in registers and shifting it made
+    // every unit wait for the load issued one unit before (a global-load
+    // latency per unit).
     constexpr int SD = 4;
-    uint32_t sq[SD];
     UnitPos pf = cur;
-    auto scale_of = [&](const UnitPos& p) -> uint32_t {
+    const uint32_t ring = bar_sa + 512u + uint32_t((warp - DW) * SD * 32 * 4);
+    const uint32_t half = uint32_t(scale_slot(lane) >> 1) & 1u;  // which bf16 of the word
+    auto issue_scale = [&](const UnitPos& p, int slot, bool live) {
       const int64_t r0 = p.tau * kTileRows + sw * 32;
-      if (r0 >= a.N) return 0u;
-      const uint8_t* b = a.scales + ((r0 / kStrip) * a.G + p.g) * kScaleBytes + scale_slot(lane);
-      return uint32_t(__ldg(reinterpret_cast<const uint16_t*>(b)));
+      if (live && r0 < a.N) {
+        const uint8_t* b =
+            a.scales + ((r0 / kStrip) * a.G + p.g) * kScaleBytes + (scale_slot(lane) & ~3);
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
+                     ::"r"(ring + uint32_t((slot * 32 + lane) * 4)), "l"(b)
+                     : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
     };
 #pragma unroll
     for (int d = 0; d < SD; ++d) {
-      sq[d] = d < n ? scale_of(pf) : 0u;
+      issue_scale(pf, d, d < n);
       pf.next(a.G, a.ntiles);
     }
     float acc[NC];
@@ -364,10 +376,10 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     for (int i = 0; i < n; ++i) {
       const int64_t row = cur.tau * kTileRows + sw * 32 + lane;
       const bool valid = cur.tau * kTileRows + sw * 32 < a.N;
-      const float s = __uint_as_float(sq[0] << 16);
-#pragma unroll
-      for (int d = 0; d < SD - 1; ++d) sq[d] = sq[d + 1];
-      sq[SD - 1] = (i + SD < n) ? scale_of(pf) : 0u;
+      asm volatile("cp.async.wait_group %0;" ::"n"(SD - 1) : "memory");
+      const uint32_t sw2 = lds32(ring + uint32_t(((i % SD) * 32 + lane) * 4));
+      const float s = half ? bf16_hi_to_f32(sw2) : bf16_lo_to_f32(sw2);
+      issue_scale(pf, i % SD, i + SD < n);
       pf.next(a.G, a.ntiles);
       const int ds = i % DS;
       const bool ok = mbar_wait(bar(B_DF + ds), uint32_t(i / DS) & 1u, abort_flag, kWaitLimitNs);
@@ -396,6 +408,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
       }
       cur.next(a.G, a.ntiles);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == W_XLOAD) {
     if (lane == 0) {
       int issued = 0;
@@ -519,7 +532,9 @@ static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
                              cudaStream_t stream) {
   using Cfg = GemmCfg<NT>;
   static int granted[64] = {0};
-  const int smem = 1024 + kLutBytes + Cfg::XS * Cfg::XSTAGE + 512;
+  // alignment slack, table, activation stages, barriers and flags (512),
+  // the promotion warps' scale rings
+  const int smem = 1024 + kLutBytes + Cfg::XS * Cfg::XSTAGE + 512 + kScaleRingBytes;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
