@@ -404,6 +404,64 @@ def gemv(x, codes, scale_bits, levels_f32) -> np.ndarray:
     return np.sum(partial * s.T[:, None, :], axis=0)
 
 
+# --------------------------------------------------------------------------
+# Randomized Hadamard rotation ("TurboQuant: A first-principles walkthrough":
+# before quantizing, a randomized Hadamard transform can stand in for a
+# uniform random rotation)
+# --------------------------------------------------------------------------
+#
+# Readings (the page gives no construction): the rotation acts on each group
+# of 128 consecutive k; it is R = H diag(s) with H the Sylvester Hadamard
+# matrix of order 128 (entries +-1, H H^T = 128 I) and s a vector of 128
+# random signs that the caller draws and passes in.  The weights are rotated
+# offline without normalisation, w_g -> H diag(s) w_g (exact integer
+# combinations of the bf16 weights, rounded once to bf16), and the
+# activations online with the 1/128 that makes the pair orthogonal,
+# x_g -> H diag(s) x_g / 128 (rounded once to bf16).  Then
+# sum_g (R w_g) . (R x_g) / 128 = sum_g w_g . x_g.
+
+def hadamard(n: int = GROUP) -> np.ndarray:
+    """Sylvester Hadamard matrix of order n (a power of two), by the doubling
+    recursion H_2m = [[H_m, H_m], [H_m, -H_m]]."""
+    if n < 1 or n & (n - 1):
+        raise ValueError("order must be a power of two")
+    h = np.ones((1, 1), dtype=np.float64)
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def _check_signs(signs) -> np.ndarray:
+    s = np.asarray(signs, dtype=np.float64).reshape(-1)
+    if s.size != GROUP or not np.all(np.abs(s) == 1.0):
+        raise ValueError("signs must be 128 values of +1 or -1")
+    return s
+
+
+def rht_weights(w, signs) -> np.ndarray:
+    """W[N, K] -> each row's groups w_g replaced by H diag(s) w_g, computed in
+    fp64 and rounded once to bf16 (returned as fp64 values)."""
+    s = _check_signs(signs)
+    wf = np.asarray(w, dtype=np.float64)
+    n, k = wf.shape
+    _check_shape(STRIP, k)
+    h = hadamard(GROUP)
+    rot = np.matmul(wf.reshape(n, k // GROUP, GROUP) * s, h.T)   # row vectors: (H v)^T = v^T H^T
+    return bf16_round(rot.reshape(n, k))
+
+
+def rht_activations(x, signs) -> np.ndarray:
+    """x[M, K] -> each row's groups x_g replaced by H diag(s) x_g / 128, fp64,
+    rounded once to bf16 (returned as fp64 values)."""
+    s = _check_signs(signs)
+    xf = np.asarray(x, dtype=np.float64)
+    m, k = xf.shape
+    _check_shape(STRIP, k)
+    h = hadamard(GROUP)
+    rot = np.matmul(xf.reshape(m, k // GROUP, GROUP) * s, h.T) / GROUP
+    return bf16_round(rot.reshape(m, k))
+
+
 def gemv_rows(x, w_rows, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Quantize a subset of rows and return (codes, scale bits, y[:, rows]).
 

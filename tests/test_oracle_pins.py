@@ -15,6 +15,7 @@ import pytest
 import scipy.integrate
 import torch
 
+import workloads
 from oracle import lutq_oracle as O
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -447,3 +448,78 @@ def test_rel_error_gate():
     y = r.copy()
     y[0, 2] = 1e-3          # floor = 1e-2 * rms(r) = 1e-2 * sqrt(21/4)
     assert abs(O.rel_error_gate(y, r) - 1e-3 / (1e-2 * math.sqrt(21 / 4))) < 1e-12
+
+
+# ---------------------------------------------------------------- Hadamard rotation
+
+def _parity_sign(i, j):
+    return -1.0 if bin(i & j).count("1") % 2 else 1.0
+
+
+def test_hadamard_closed_form_and_library():
+    import scipy.linalg
+    h = O.hadamard(128)
+    want = np.array([[_parity_sign(i, j) for j in range(128)] for i in range(128)])
+    np.testing.assert_array_equal(h, want)                          # (-1)^popcount(i & j)
+    np.testing.assert_array_equal(h, scipy.linalg.hadamard(128))    # library construction
+    np.testing.assert_array_equal(h @ h.T, 128.0 * np.eye(128))
+
+
+def test_rht_of_unit_vectors_is_a_signed_hadamard_column():
+    signs = workloads.rht_signs(5).numpy().astype(np.float64)
+    w = np.zeros((3, 256))
+    cases = [(0, 7, 1.0), (1, 228, 1.0), (2, 255, -2.0)]
+    for row, k, val in cases:
+        w[row, k] = val
+    r = O.rht_weights(w, signs)
+    x = O.rht_activations(w, signs)
+    for row, k, val in cases:
+        g, j = divmod(k, 128)
+        col = np.array([_parity_sign(i, j) for i in range(128)]) * signs[j] * val
+        np.testing.assert_array_equal(r[row, 128 * g:128 * g + 128], col)
+        np.testing.assert_array_equal(x[row, 128 * g:128 * g + 128], col / 128.0)
+        rest = np.delete(r[row], np.arange(128 * g, 128 * g + 128))
+        assert not rest.any()
+
+
+def test_rht_pair_preserves_inner_products_exactly():
+    # small-integer data: every rotated weight is an integer in [-128, 128] and
+    # every rotated activation that over 128, all exact in bf16
+    rng = np.random.default_rng(3)
+    w = rng.integers(-1, 2, size=(5, 384)).astype(np.float64)
+    x = rng.integers(-1, 2, size=(2, 384)).astype(np.float64)
+    signs = workloads.rht_signs(9).numpy()
+    rw, rx = O.rht_weights(w, signs), O.rht_activations(x, signs)
+    np.testing.assert_array_equal(rx @ rw.T, x @ w.T)
+
+
+def test_rht_twice_with_plus_signs_scales_by_128():
+    rng = np.random.default_rng(4)
+    w = rng.integers(-1, 2, size=(4, 256)).astype(np.float64)
+    ones = np.ones(128)
+    np.testing.assert_array_equal(O.rht_weights(O.rht_weights(w, ones), ones), 128.0 * w)
+
+
+def test_rht_rejects_bad_signs():
+    w = np.zeros((1, 128))
+    with pytest.raises(ValueError):
+        O.rht_weights(w, np.zeros(128))
+    with pytest.raises(ValueError):
+        O.rht_activations(w, np.ones(64))
+
+
+def test_rht_lowers_quantization_error_with_outliers():
+    # the reason for the rotation: spreading a group's outliers over all 128
+    # coordinates before round-to-nearest lowers the product's error
+    w = workloads.normal_weights(64, 1024, 0.02, seed=12, outlier_frac=1e-2).float().numpy()
+    x = workloads.activations(4, 1024, seed=13).float().numpy()
+    signs = workloads.rht_signs(14).numpy()
+    lv = _levels("nf4", 4)
+    exact = x.astype(np.float64) @ w.astype(np.float64).T
+    codes, sb = O.quantize(w, lv, 4)
+    err_plain = np.linalg.norm(O.gemv(x, codes, sb, lv) - exact)
+    wr = O.rht_weights(w, signs).astype(np.float32)
+    xr = O.rht_activations(x, signs).astype(np.float32)
+    codes_r, sb_r = O.quantize(wr, lv, 4)
+    err_rht = np.linalg.norm(O.gemv(xr, codes_r, sb_r, lv) - exact)
+    assert err_rht < 0.9 * err_plain

@@ -92,6 +92,12 @@ def activations(m: int, k: int, seed: int) -> torch.Tensor:
     return torch.randn((m, k), generator=gen, dtype=torch.float32).to(torch.bfloat16)
 
 
+def rht_signs(seed: int) -> torch.Tensor:
+    """128 random signs (+1 / -1, int8) for the randomized Hadamard rotation."""
+    gen = torch.Generator().manual_seed(seed)
+    return (torch.randint(0, 2, (128,), generator=gen) * 2 - 1).to(torch.int8)
+
+
 @dataclasses.dataclass(frozen=True)
 class Layer:
     """One weight matrix of a workload: W[n, k] and how it is drawn."""
