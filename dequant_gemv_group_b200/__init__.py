@@ -14,10 +14,13 @@ from ._binding import (  # noqa: F401
     lutq_gemv,
     lutq_gemv_noalloc,
     lutq_gemv_plan,
+    lutq_gemv_rht,
     lutq_layout_version,
     lutq_pack,
     lutq_packed_bytes,
     lutq_quantize,
+    lutq_rht_activations,
+    lutq_rht_weights,
     lutq_selftest_wait_timeout,
     lutq_status_string,
     lutq_workspace_bytes,

@@ -44,6 +44,10 @@ _SIGS = {
     "lutq_gemv_noalloc": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
     "lutq_gemv_plan": (_i32, [_i64, _i64, _i32, _vp]),
     "lutq_selftest_wait_timeout": (_i32, [_vp, _i64, _vp]),
+    "lutq_rht_weights": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "lutq_rht_activations": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "lutq_gemv_rht": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
+                             _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -189,3 +193,38 @@ def lutq_gemm(x, packed, codebook, bits, n, k, y=None, workspace=None, status=No
     """y[M, N] (fp32) on the tensor cores; see lutq_gemm in include/lutq.h."""
     return _product(lib.lutq_gemm, "lutq_gemm", x, packed, codebook, bits, n, k, y, workspace,
                     status)
+
+
+def _rht(fn, where, t: torch.Tensor, signs: torch.Tensor) -> torch.Tensor:
+    _need(t, torch.bfloat16, where)
+    _need(signs, torch.int8, "signs")
+    if signs.numel() != 128:
+        raise LutqError(1, where + ": 128 signs")
+    rows, k = t.shape
+    out = torch.empty_like(t)
+    _check(fn(t.data_ptr(), rows, k, signs.data_ptr(), out.data_ptr(), _stream()), where)
+    return out
+
+
+def lutq_rht_weights(w: torch.Tensor, signs: torch.Tensor) -> torch.Tensor:
+    """W bf16 [N, K] -> each 128-group rotated by H diag(s) (see include/lutq.h)."""
+    return _rht(lib.lutq_rht_weights, "lutq_rht_weights", w, signs)
+
+
+def lutq_rht_activations(x: torch.Tensor, signs: torch.Tensor) -> torch.Tensor:
+    """x bf16 [M, K] -> each 128-group rotated by H diag(s) / 128."""
+    return _rht(lib.lutq_rht_activations, "lutq_rht_activations", x, signs)
+
+
+def lutq_gemv_rht(x, packed, codebook, signs, bits, n, k, y=None, workspace=None, status=None):
+    """lutq_gemv on rotated weights, rotating x inside the kernel (M = 1..4)."""
+    _need(x, torch.bfloat16, "x")
+    _need(signs, torch.int8, "signs")
+    m = x.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    _check(lib.lutq_gemv_rht(x.data_ptr(), m, packed.data_ptr(), codebook.data_ptr(),
+                             signs.data_ptr(), bits, n, k, y.data_ptr(), ws_ptr, ws_bytes,
+                             _ptr(status), _stream()), "lutq_gemv_rht")
+    return y

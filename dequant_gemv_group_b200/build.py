@@ -24,7 +24,7 @@ PER_FILE = {
     "lutq_quantize.cu": ["-fmad=false", "-ftz=false", "-prec-div=true", "-prec-sqrt=true"],
 }
 SOURCES = ["lutq_api.cu", "lutq_quantize.cu", "lutq_pack.cu", "lutq_gemv.cu", "lutq_gemm.cu",
-           "lutq_noalloc.cu", "lutq_selftest.cu"]
+           "lutq_noalloc.cu", "lutq_selftest.cu", "lutq_rht.cu"]
 HOST_SOURCES = ["lutq_codebook.cpp"]
 
 

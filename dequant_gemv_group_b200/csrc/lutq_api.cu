@@ -20,6 +20,13 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const void* codebook,
+                            const int8_t* signs, int bits, int64_t N, int64_t K, float* y,
+                            void* workspace, int32_t* dev_status, int num_sms,
+                            cudaStream_t stream);
+bool gemv_small_path(int64_t M, int64_t K, int bits);
+cudaError_t launch_rht(const void* in, int64_t rows, int64_t K, const int8_t* signs,
+                       bool activations, void* out, int num_sms, cudaStream_t stream);
 int64_t gemv_workspace_bytes(int64_t M, int64_t N);
 void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out);
 int64_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
@@ -177,6 +184,52 @@ lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_gemm(x_bf16, M, packed, codebook_bf16, bits, N, K, y, workspace,
                                      dev_status, sms, static_cast<cudaStream_t>(stream)));
+}
+
+static lutq_status rht(const void* in, int64_t rows, int64_t K, const int8_t* signs, void* out,
+                       bool activations, void* stream) {
+  if (!in || !signs || !out) return LUTQ_ERR_INVALID_ARG;
+  if (rows < 1 || K < lutq::kGroup || K % lutq::kGroup != 0 || rows > (int64_t(1) << 31) ||
+      K > (int64_t(1) << 31))
+    return LUTQ_ERR_SHAPE;
+  if (!aligned16(in) || !aligned16(signs) || !aligned16(out)) return LUTQ_ERR_ALIGN;
+  const char* a = static_cast<const char*>(in);
+  const char* b = static_cast<const char*>(out);
+  const int64_t bytes = rows * K * 2;
+  if (a < b + bytes && b < a + bytes) return LUTQ_ERR_INVALID_ARG;  // overlap
+  int sms = 0;
+  lutq_status st;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_rht(in, rows, K, signs, activations, out, sms,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_rht_weights(const void* W_bf16, int64_t N, int64_t K, const int8_t* signs,
+                             void* W_rot_bf16, void* stream) {
+  return rht(W_bf16, N, K, signs, W_rot_bf16, false, stream);
+}
+
+lutq_status lutq_rht_activations(const void* x_bf16, int64_t M, int64_t K, const int8_t* signs,
+                                 void* x_rot_bf16, void* stream) {
+  return rht(x_bf16, M, K, signs, x_rot_bf16, true, stream);
+}
+
+lutq_status lutq_gemv_rht(const void* x_bf16, int64_t M, const void* packed,
+                          const void* codebook_bf16, const int8_t* signs, int bits, int64_t N,
+                          int64_t K, float* y, void* workspace, int64_t workspace_bytes,
+                          int32_t* dev_status, void* stream) {
+  if (!signs) return LUTQ_ERR_INVALID_ARG;
+  lutq_status st = check_product_args(x_bf16, M, 16, packed, codebook_bf16, bits, N, K, y,
+                                      workspace, workspace_bytes,
+                                      lutq_workspace_bytes(M, N, K, bits));
+  if (st != LUTQ_OK) return st;
+  if (!aligned16(signs)) return LUTQ_ERR_ALIGN;
+  if (!lutq::gemv_small_path(M, K, bits)) return LUTQ_ERR_SHAPE;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_gemv_rht(x_bf16, M, packed, codebook_bf16, signs, bits, N, K, y,
+                                         workspace, dev_status, sms,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -43,10 +43,13 @@
 // loads the activations into shared memory and builds the lookup table,
 // and each warp keeps NB tiles (codes and scales) in flight in registers,
 // loaded under one predicate so that the loop has no branch per load.
+#include <cuda_bf16.h>
+
 #include <algorithm>
 
 #include "lutq_common.cuh"
 #include "lutq_lut.cuh"
+#include "lutq_rht.cuh"
 #include "lutq_sm100.cuh"
 
 namespace lutq {
@@ -65,6 +68,7 @@ struct GemvArgs {
   float* y;                 // fp32 [M, N]
   unsigned long long* xch;  // [M][N] exchange slots of strips split between two CTAs (zero between calls)
   int32_t* status;          // caller's device status word or null
+  const int8_t* signs;      // randomized Hadamard rotation of x first (null: none)
   int64_t N, K, G, U;       // U = number of units
   int C;                    // CTAs
   // work plan (choose_plan): kind 0 = ranges of the unit sequence, strip-
@@ -564,6 +568,43 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
   build_lut_shfl<BITS>(smem + (kLutAt - sbase), cbv);
 #pragma unroll
   for (int t = 1; t < NB; ++t) fetch(buf[t], sbuf[t]);
+  if (a.signs != nullptr) {
+    // Rotate every 128-long group of the activations in place, eight lanes
+    // per group: x_g <- H diag(s) x_g / 128, fp32 butterflies (as
+    // lutq_rht_activations), rounded once to bf16 (group t = m G + g of
+    // batch row m sits at 256 t).
+    const uint4 signs16 = reinterpret_cast<const uint4*>(a.signs)[lane & 7];
+    __syncthreads();  // the block's activation stores
+    uint8_t* xs = smem + (kXAt - sbase);
+    const uint32_t groups = uint32_t(M) * G;
+    for (uint32_t t0 = 4u * uint32_t(wl); t0 < groups; t0 += 4u * kM1Warps) {
+      const uint32_t t = t0 + uint32_t(lane >> 3);
+      uint4* p = reinterpret_cast<uint4*>(xs + t * kXGroupBytes + 32u * uint32_t(lane & 7));
+      uint4 r0 = make_uint4(0, 0, 0, 0), r1 = r0;
+      if (t < groups) {
+        r0 = p[0];
+        r1 = p[1];
+      }
+      const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = bf16_lo_to_f32(w[i]);
+        v[2 * i + 1] = bf16_hi_to_f32(w[i]);
+      }
+      rht128_octet(v, signs16);
+      uint32_t h[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        h[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i] * (1.0f / kGroup))) |
+               (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1] * (1.0f / kGroup))))
+                << 16);
+      if (t < groups) {
+        p[0] = make_uint4(h[0], h[1], h[2], h[3]);
+        p[1] = make_uint4(h[4], h[5], h[6], h[7]);
+      }
+    }
+  }
   __syncthreads();  // table, activations
 
   const uint32_t lane_e = uint32_t(lane) * 4u, lane_o = 128u + uint32_t(lane) * 4u;
@@ -812,6 +853,7 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   a.y = y;
   a.xch = static_cast<unsigned long long*>(workspace);
   a.status = dev_status;
+  a.signs = nullptr;
   a.N = N;
   a.K = K;
   a.G = K / kGroup;
@@ -823,6 +865,36 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   if (!small)
     return launch_gemm(x, M, packed, codebook, bits, N, K, y, workspace, dev_status,
                        num_sms, stream);
+  return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
+                   : launch_bits<3>(a, int(M), num_sms, stream);
+}
+
+// Whether lutq_gemv runs an M x K product on the CUDA-core kernel.
+bool gemv_small_path(int64_t M, int64_t K, int bits) {
+  return bits == 4 ? small_fits<4>(M, K) : small_fits<3>(M, K);
+}
+
+// lutq_gemv with the activations rotated in the kernel's prologue; only for
+// the CUDA-core kernel (the caller checks gemv_small_path).
+cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const void* codebook,
+                            const int8_t* signs, int bits, int64_t N, int64_t K, float* y,
+                            void* workspace, int32_t* dev_status, int num_sms,
+                            cudaStream_t stream) {
+  if (!gemv_small_path(M, K, bits)) return cudaErrorInvalidValue;
+  GemvArgs a;
+  a.x = static_cast<const uint16_t*>(x);
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.codebook = static_cast<const uint16_t*>(codebook);
+  a.y = y;
+  a.xch = static_cast<unsigned long long*>(workspace);
+  a.status = dev_status;
+  a.signs = signs;
+  a.N = N;
+  a.K = K;
+  a.G = K / kGroup;
+  a.U = (N / kStrip) * a.G;
+  a.C = 0;
+  if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
                    : launch_bits<3>(a, int(M), num_sms, stream);
 }

@@ -267,6 +267,47 @@ lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan);
 lutq_status lutq_selftest_wait_timeout(int32_t* dev_status, int64_t limit_ns, void* stream);
 
 /*
+ * lutq_rht_weights / lutq_rht_activations - randomized Hadamard rotation of
+ * every 128-long group of each row.
+ *
+ * Source: "TurboQuant: A first-principles walkthrough" (a randomized Hadamard
+ * transform can replace a uniform random rotation before quantizing).  With H
+ * the Sylvester Hadamard matrix of order 128 (H[i][j] = (-1)^popcount(i & j),
+ * H H^T = 128 I) and s the caller's 128 random signs:
+ *   weights:     g -> H diag(s) g          (offline, before lutq_quantize)
+ *   activations: g -> H diag(s) g / 128    (before the product)
+ * so that sum_g (H diag(s) w_g) . (H diag(s) x_g / 128) = w . x.  Sums are
+ * taken in fp64 and rounded once to bf16 (exact before the rounding for bf16
+ * inputs whose exponents span fewer than 38 binades).
+ *
+ * in       device bf16 [rows, K] row-major (rows = N or M >= 1, K % 128 == 0).
+ * signs    device int8 [128]; a negative value means -1, any other +1.
+ * out      device bf16 [rows, K], written; may not overlap `in`.
+ * Pointers 16-byte aligned.  Asynchronous on `stream`.
+ */
+lutq_status lutq_rht_weights(const void* W_bf16, int64_t N, int64_t K, const int8_t* signs,
+                             void* W_rot_bf16, void* stream);
+lutq_status lutq_rht_activations(const void* x_bf16, int64_t M, int64_t K, const int8_t* signs,
+                                 void* x_rot_bf16, void* stream);
+
+/*
+ * lutq_gemv_rht - lutq_gemv on rotated weights, rotating the activations
+ * inside the kernel: y = x_rot . dequant(packed)^T with x_rot the
+ * lutq_rht_activations rotation of x (computed on the activations in shared
+ * memory, in the kernel's prologue, with the same arithmetic, so the result
+ * equals lutq_gemv on lutq_rht_activations(x) bit for bit).  `packed` holds
+ * the quantized rotated weights (lutq_rht_weights -> lutq_quantize ->
+ * lutq_pack).  Only for products that run on the CUDA-core kernel (M = 1..4
+ * and M * (K + 2048) <= 80896); otherwise returns LUTQ_ERR_SHAPE and the
+ * caller rotates with lutq_rht_activations and calls lutq_gemm.  Other
+ * arguments as lutq_gemv; signs as lutq_rht_activations.
+ */
+lutq_status lutq_gemv_rht(const void* x_bf16, int64_t M, const void* packed,
+                          const void* codebook_bf16, const int8_t* signs, int bits, int64_t N,
+                          int64_t K, float* y, void* workspace, int64_t workspace_bytes,
+                          int32_t* dev_status, void* stream);
+
+/*
  * lutq_gemm - the same product on the tensor cores (tcgen05), for batches
  * where the problem is a dense contraction (tuned for M >= 32; any M >= 1 is
  * accepted).  Arguments and numerics as lutq_gemv.  dev_status receives

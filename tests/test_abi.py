@@ -116,3 +116,29 @@ def test_product_argument_errors(lq, name):
     if ws > 0:
         assert call(ws=None) == 9
         assert call(wsb=ws - 1) == 9
+
+
+def test_rht_argument_errors(lq):
+    for f in (lq.lib.lutq_rht_weights, lq.lib.lutq_rht_activations):
+        assert f(None, 32, 128, A, A + 4096, None) == 1              # null input
+        assert f(A, 32, 128, None, A + 4096, None) == 1              # null signs
+        assert f(A, 0, 128, A, A + 4096, None) == 2                  # no rows
+        assert f(A, 32, 200, A, A + 4096 * 4, None) == 2             # K % 128
+        assert f(A + 2, 32, 128, A, A + 1 << 16, None) == 4          # misaligned
+        assert f(A, 32, 128, A, A + 2048, None) == 1                 # in and out overlap
+
+
+def test_gemv_rht_argument_errors(lq):
+    f = lq.lib.lutq_gemv_rht
+    ws = lq.lutq_workspace_bytes(1, 64, 256, 4)
+
+    def call(**kw):
+        a = dict(dict(x=A, m=1, p=A, c=A, s=A, bits=4, n=64, k=256, y=A, ws=A, wsb=ws), **kw)
+        return f(a["x"], a["m"], a["p"], a["c"], a["s"], a["bits"], a["n"], a["k"], a["y"],
+                 a["ws"], a["wsb"], None, None)
+
+    assert call(s=None) == 1
+    assert call(s=A + 4) == 4
+    assert call(m=5) == 2                  # beyond the CUDA-core kernel: rotate and use lutq_gemm
+    assert call(m=1, k=128 * 700) == 2     # activations too long for its shared memory
+    assert call(bits=5) == 3
