@@ -300,6 +300,43 @@ def side_measurements(lq, dev, args):
     assert int(st.item()) == 0
     q_bytes = n * k * 2 + n * k + n * (k // 128) * 2
     p_bytes = n * k + (n * k * bits) // 8 + 2 * n * (k // 128) * 2
+    # randomized Hadamard rotation fused into the GEMV, batch 1, on the same
+    # layer: throughput (graph-replayed, weights rotating over copies larger
+    # than L2) and the product's error against the unquantized one with and
+    # without the rotation
+    signs = workloads.rht_signs(1).to(dev)
+    x1 = workloads.activations(1, k, seed=1).to(dev)
+    y1 = torch.empty((1, n), dtype=torch.float32, device=dev)
+    ws1 = lq.new_workspace(1, n, k, bits, dev)
+    packed_plain = lq.lutq_pack(codes, scales, bits, status=st)
+    wr = lq.lutq_rht_weights(w, signs)
+    codes_r, scales_r = lq.lutq_quantize(wr, cb, bits, status=st)
+    packed_r = lq.lutq_pack(codes_r, scales_r, bits, status=st)
+    del wr, codes_r, scales_r
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(2, int(np.ceil(3 * l2 / packed_r.numel())) + 1)
+    packs_r = [packed_r] + [packed_r.clone() for _ in range(copies - 1)]
+    call_r = lambda i: lq.lutq_gemv_rht(x1, packs_r[i % copies], cb, signs, bits, n, k, y=y1,
+                                        workspace=ws1, status=st)
+    for i in range(4):
+        call_r(i)
+    g_r = capture(call_r, 128)
+    g_r.replay()
+    t_r = time_events(lambda i: g_r.replay(), 8) / 128
+    del g_r
+    exact = (x1.double() @ w.double().t()).cpu().numpy()
+    y_plain = lq.lutq_gemv(x1, packed_plain, cb, bits, n, k, workspace=ws1, status=st)
+    y_rot = lq.lutq_gemv_rht(x1, packed_r, cb, signs, bits, n, k, workspace=ws1, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    err_plain = float(np.linalg.norm(y_plain.double().cpu().numpy() - exact) / np.linalg.norm(exact))
+    err_rot = float(np.linalg.norm(y_rot.double().cpu().numpy() - exact) / np.linalg.norm(exact))
+    out["rht"] = {"workload": f"{args.workload}/{args.layer} W[{n},{k}] {args.codebook} W{bits} "
+                              "batch1, activations rotated in the GEMV prologue",
+                  "value": algorithmic_bytes(1, n, k, bits) / t_r / 1e9, "unit": "GB/s",
+                  "us": t_r * 1e6, "kernel": "lutq::gemv_small_kernel (rotating)",
+                  "rel_error_vs_unquantized": {"plain": err_plain, "rotated": err_rot}}
+    del packs_r, packed_r, packed_plain
     out["offline"] = {"quantize_gbs": q_bytes / tq / 1e9, "quantize_us": tq * 1e6,
                       "pack_gbs": p_bytes / tp / 1e9, "pack_us": tp * 1e6,
                       "note": "W bf16 -> codes u8 + scales; codes + scales -> layout V2 (L2-warm)"}
