@@ -462,6 +462,68 @@ def rht_activations(x, signs) -> np.ndarray:
     return bf16_round(rot.reshape(m, k))
 
 
+# --------------------------------------------------------------------------
+# Codebook fitted to a layer (Lloyd-Max on the layer's own normalised
+# weights: "TurboQuant: A first-principles walkthrough" names the Lloyd-Max
+# algorithm; the FLUTE abstract speaks of extending NormalFloat)
+# --------------------------------------------------------------------------
+#
+# Readings (the pages give no procedure): the data are the normalised weights
+# v = fp32(w) / fp32(s) of the quantizer (s = the group's absolute maximum);
+# they are counted in HIST_BINS equal bins over [-1, 1], bin
+# b = floor(fp32(v + 1) * HIST_BINS / 2) (clamped to the last bin), whose
+# centre is c_b = (2 b + 1 - HIST_BINS) / HIST_BINS; Lloyd-Max then alternates
+# (1) each bin to its nearest level (fp64 distance, ties to the lowest level)
+# and (2) each level to the count-weighted mean of its bins' centres, an exact
+# integer ratio (a level whose cell is empty stays), from a starting codebook
+# until the assignment no longer changes or max_iter passes; the levels are
+# rounded once to bf16.
+
+HIST_BINS = 16384
+
+
+def fit_histogram(w) -> np.ndarray:
+    """Counts (int64[HIST_BINS]) of W's normalised weights v = w / s."""
+    w = np.asarray(w, dtype=np.float32)
+    n, k = w.shape
+    if k % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    if not np.all(np.isfinite(w)):
+        raise ValueError("non-finite weight")
+    wg = w.reshape(n, k // GROUP, GROUP)
+    s = np.broadcast_to(np.max(np.abs(wg), axis=2)[:, :, None], wg.shape)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s > 0, wg / s, np.float32(0.0)).astype(np.float32)
+    b = np.floor((v + np.float32(1.0)).astype(np.float32) * np.float32(HIST_BINS // 2))
+    b = np.minimum(b.astype(np.int64), HIST_BINS - 1)
+    return np.bincount(b.reshape(-1), minlength=HIST_BINS).astype(np.int64)
+
+
+def fit_codebook(hist, init_levels, max_iter: int = 100) -> np.ndarray:
+    """Lloyd-Max on a fit_histogram histogram from init_levels (ascending);
+    returns the levels rounded to bf16 (fp64 values)."""
+    counts = np.asarray(hist, dtype=np.int64).reshape(-1)
+    if counts.size != HIST_BINS:
+        raise ValueError("histogram size")
+    levels = np.asarray(init_levels, dtype=np.float64).copy()
+    ints = 2 * np.arange(HIST_BINS, dtype=np.int64) + 1 - HIST_BINS   # centre * HIST_BINS
+    centres = ints / float(HIST_BINS)                                  # exact in fp64
+    assign = None
+    for _ in range(max_iter):
+        # nearest level in fp64; argmin keeps the first (lowest) of equal distances
+        new_assign = np.argmin(np.abs(centres[:, None] - levels[None, :]), axis=1)
+        if assign is not None and np.array_equal(new_assign, assign):
+            break
+        assign = new_assign
+        for i in range(levels.size):
+            cell = assign == i
+            den = int(np.sum(counts[cell]))
+            if den:
+                num = int(np.sum(counts[cell] * ints[cell]))   # exact: |num| < 2^59
+                levels[i] = float(num) / float(den * HIST_BINS)
+    return bf16_round(levels)
+
+
 def gemv_rows(x, w_rows, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Quantize a subset of rows and return (codes, scale bits, y[:, rows]).
 

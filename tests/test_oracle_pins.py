@@ -523,3 +523,47 @@ def test_rht_lowers_quantization_error_with_outliers():
     codes_r, sb_r = O.quantize(wr, lv, 4)
     err_rht = np.linalg.norm(O.gemv(xr, codes_r, sb_r, lv) - exact)
     assert err_rht < 0.9 * err_plain
+
+
+# ---------------------------------------------------------------- codebook fitted to a layer
+
+def test_fit_histogram_hand_values():
+    w = np.zeros((1, 256), np.float32)
+    w[0, :4] = [2.0, -2.0, 1.0, -0.5]       # group 0: s = 2 -> v = 1, -1, 0.5, -0.25, then 124 zeros
+    h = O.fit_histogram(w)                   # group 1 is all zero (s = 0): 128 zeros
+    want = np.zeros(O.HIST_BINS, np.int64)
+    want[O.HIST_BINS - 1] += 1               # v = 1: (1 + 1) * 8192 = 16384, clamped
+    want[0] += 1                             # v = -1
+    want[12288] += 1                         # v = 0.5: 1.5 * 8192
+    want[6144] += 1                          # v = -0.25: 0.75 * 8192
+    want[8192] += 124 + 128                  # v = 0
+    np.testing.assert_array_equal(h, want)
+
+
+def test_fit_two_clusters_lands_on_their_centres():
+    h = np.zeros(O.HIST_BINS, np.int64)
+    h[1000] = 10
+    h[15000] = 30
+    got = O.fit_codebook(h, np.array([-0.5, 0.5]))
+    centres = (2 * np.array([1000, 15000]) + 1 - O.HIST_BINS) / O.HIST_BINS
+    np.testing.assert_array_equal(got, O.bf16_round(centres))
+    # a level whose cell stays empty keeps its starting value
+    got3 = O.fit_codebook(h, np.array([-0.5, 0.25, 0.5]))
+    assert got3[0] == O.bf16_round(np.array([centres[0]]))[0] and got3[1] == 0.25
+
+
+def _hist_distortion(h, levels):
+    c = (2 * np.arange(O.HIST_BINS) + 1 - O.HIST_BINS) / O.HIST_BINS
+    d = np.min(np.abs(c[:, None] - np.asarray(levels)[None, :]), axis=1)
+    return float(np.sum(h * d * d))
+
+
+def test_fit_lowers_the_layers_distortion():
+    w = workloads.student_t_weights(256, 1024, 5, 0.02, seed=21, outlier_frac=1e-3).float().numpy()
+    h = O.fit_histogram(w)
+    assert h.sum() == w.size
+    for kind, bits in (("nf4", 4), ("lloyd_max3", 3)):
+        _, init = O.codebook(kind, bits)
+        fitted = O.fit_codebook(h, init)
+        assert np.all(np.diff(fitted) > 0)
+        assert _hist_distortion(h, fitted) < 0.97 * _hist_distortion(h, init)
