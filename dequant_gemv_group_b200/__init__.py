@@ -10,6 +10,8 @@ from ._binding import (  # noqa: F401
     LutqError,
     lib,
     lutq_codebook,
+    lutq_fit_codebook,
+    lutq_fit_histogram,
     lutq_gemm,
     lutq_gemv,
     lutq_gemv_noalloc,

@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "liblutq.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python -m dequant_gemv_group_b200.build`")
+    raise ImportError(f"{LIB_PATH} is not built; run `python dequant_gemv_group_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -44,6 +44,8 @@ _SIGS = {
     "lutq_gemv_noalloc": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
     "lutq_gemv_plan": (_i32, [_i64, _i64, _i32, _vp]),
     "lutq_selftest_wait_timeout": (_i32, [_vp, _i64, _vp]),
+    "lutq_fit_histogram": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "lutq_fit_codebook": (_i32, [_vp, _i32, _vp, _i32, _vp]),
     "lutq_rht_weights": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "lutq_rht_activations": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "lutq_gemv_rht": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
@@ -228,3 +230,33 @@ def lutq_gemv_rht(x, packed, codebook, signs, bits, n, k, y=None, workspace=None
                              signs.data_ptr(), bits, n, k, y.data_ptr(), ws_ptr, ws_bytes,
                              _ptr(status), _stream()), "lutq_gemv_rht")
     return y
+
+
+HIST_BINS = 16384
+
+
+def lutq_fit_histogram(w: torch.Tensor, hist: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Add W's normalised-weight counts to hist (int64 [16384] on W's device,
+    zeros if None) and return it."""
+    _need(w, torch.bfloat16, "W")
+    n, k = w.shape
+    if hist is None:
+        hist = torch.zeros(HIST_BINS, dtype=torch.int64, device=w.device)
+    _need(hist, torch.int64, "hist")
+    _check(lib.lutq_fit_histogram(w.data_ptr(), n, k, hist.data_ptr(), _ptr(status), _stream()),
+           "lutq_fit_histogram")
+    return hist
+
+
+def lutq_fit_codebook(hist, bits: int, init: torch.Tensor, max_iter: int = 100) -> torch.Tensor:
+    """Lloyd-Max from init (bf16, CPU) on a histogram (CPU, from
+    lutq_fit_histogram); returns the fitted codebook (bf16, CPU)."""
+    h = torch.as_tensor(hist).to(device="cpu", dtype=torch.int64).contiguous()
+    if h.numel() != HIST_BINS:
+        raise LutqError(1, "lutq_fit_codebook: histogram size")
+    init_c = init.to(device="cpu", dtype=torch.bfloat16).contiguous()
+    out = torch.empty(1 << bits, dtype=torch.bfloat16)
+    _check(lib.lutq_fit_codebook(h.data_ptr(), bits, init_c.data_ptr(), max_iter, out.data_ptr()),
+           "lutq_fit_codebook")
+    return out

@@ -1,6 +1,7 @@
 """Build liblutq.so (the CUDA kernels and the C ABI) in-tree for sm_100a.
 
-Run as ``python -m dequant_gemv_group_b200.build`` or call :func:`build`.
+Run as ``python dequant_gemv_group_b200/build.py`` (the package itself needs the
+library to import) or call :func:`build`.
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ PER_FILE = {
     "lutq_quantize.cu": ["-fmad=false", "-ftz=false", "-prec-div=true", "-prec-sqrt=true"],
 }
 SOURCES = ["lutq_api.cu", "lutq_quantize.cu", "lutq_pack.cu", "lutq_gemv.cu", "lutq_gemm.cu",
-           "lutq_noalloc.cu", "lutq_selftest.cu", "lutq_rht.cu"]
+           "lutq_noalloc.cu", "lutq_selftest.cu", "lutq_rht.cu", "lutq_fit.cu"]
 HOST_SOURCES = ["lutq_codebook.cpp"]
 
 

@@ -27,6 +27,8 @@ cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const 
 bool gemv_small_path(int64_t M, int64_t K, int bits);
 cudaError_t launch_rht(const void* in, int64_t rows, int64_t K, const int8_t* signs,
                        bool activations, void* out, int num_sms, cudaStream_t stream);
+cudaError_t launch_fit_histogram(const void* W, int64_t N, int64_t K, uint64_t* hist,
+                                 int32_t* dev_status, int num_sms, cudaStream_t stream);
 int64_t gemv_workspace_bytes(int64_t M, int64_t N);
 void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out);
 int64_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
@@ -202,6 +204,20 @@ static lutq_status rht(const void* in, int64_t rows, int64_t K, const int8_t* si
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_rht(in, rows, K, signs, activations, out, sms,
                                     static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_fit_histogram(const void* W_bf16, int64_t N, int64_t K, uint64_t* hist,
+                               int32_t* dev_status, void* stream) {
+  if (!W_bf16 || !hist) return LUTQ_ERR_INVALID_ARG;
+  if (N < 1 || K < lutq::kGroup || K % lutq::kGroup != 0 || N > (int64_t(1) << 31) ||
+      K > (int64_t(1) << 31))
+    return LUTQ_ERR_SHAPE;
+  if (!aligned16(W_bf16) || !aligned16(hist)) return LUTQ_ERR_ALIGN;
+  int sms = 0;
+  lutq_status st;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_fit_histogram(W_bf16, N, K, hist, dev_status, sms,
+                                              static_cast<cudaStream_t>(stream)));
 }
 
 lutq_status lutq_rht_weights(const void* W_bf16, int64_t N, int64_t K, const int8_t* signs,

@@ -133,3 +133,62 @@ extern "C" lutq_status lutq_codebook(int kind, int bits, uint16_t* out_bf16) {
   for (size_t i = 0; i < lv.size(); ++i) out_bf16[i] = to_bf16_rne(lv[i]);
   return LUTQ_OK;
 }
+
+// Lloyd-Max on a histogram of normalised weights (kHistBins bins over
+// [-1, 1], centre of bin b = (2 b + 1 - kHistBins) / kHistBins): alternately
+// give every bin to its nearest level (fp64 distance, ties to the lower
+// level) and move every level to the count-weighted mean of its bins' centres
+// (an exact integer ratio: |numerator| < 2^59 for fewer than 2^31 weights; a
+// level whose cell is empty stays), until the assignment repeats or max_iter
+// passes; the levels are rounded once to bf16.  The method is the Lloyd-Max
+// algorithm ("TurboQuant: A first-principles walkthrough") applied to the
+// layer's own weights.
+extern "C" lutq_status lutq_fit_codebook(const uint64_t* hist, int bits, const uint16_t* init_bf16,
+                                         int max_iter, uint16_t* out_bf16) {
+  constexpr int kHistBins = 16384;
+  if (hist == nullptr || init_bf16 == nullptr || out_bf16 == nullptr || max_iter < 0)
+    return LUTQ_ERR_INVALID_ARG;
+  if (bits != 3 && bits != 4) return LUTQ_ERR_BITS;
+  uint64_t total = 0;
+  for (int b = 0; b < kHistBins; ++b) {
+    total += hist[b];
+    if (hist[b] >= (uint64_t(1) << 31) || total >= (uint64_t(1) << 31)) return LUTQ_ERR_INVALID_ARG;
+  }
+  const int n = 1 << bits;
+  std::vector<double> levels(n);
+  for (int i = 0; i < n; ++i) {
+    const uint32_t u = uint32_t(init_bf16[i]) << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    if (!std::isfinite(f)) return LUTQ_ERR_INVALID_ARG;
+    levels[i] = f;
+  }
+  std::vector<int> assign(kHistBins, -1), next(kHistBins);
+  for (int it = 0; it < max_iter; ++it) {
+    for (int b = 0; b < kHistBins; ++b) {
+      const double c = double(2 * b + 1 - kHistBins) / double(kHistBins);
+      int best = 0;
+      double best_d = std::fabs(c - levels[0]);
+      for (int i = 1; i < n; ++i) {
+        const double d = std::fabs(c - levels[i]);
+        if (d < best_d) {
+          best = i;
+          best_d = d;
+        }
+      }
+      next[b] = best;
+    }
+    if (it > 0 && next == assign) break;
+    assign.swap(next);
+    std::vector<int64_t> num(n, 0), den(n, 0);
+    for (int b = 0; b < kHistBins; ++b) {
+      if (hist[b] == 0) continue;
+      num[assign[b]] += int64_t(hist[b]) * int64_t(2 * b + 1 - kHistBins);
+      den[assign[b]] += int64_t(hist[b]);
+    }
+    for (int i = 0; i < n; ++i)
+      if (den[i] != 0) levels[i] = double(num[i]) / double(den[i] * kHistBins);
+  }
+  for (int i = 0; i < n; ++i) out_bf16[i] = to_bf16_rne(levels[i]);
+  return LUTQ_OK;
+}

@@ -267,6 +267,36 @@ lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan);
 lutq_status lutq_selftest_wait_timeout(int32_t* dev_status, int64_t limit_ns, void* stream);
 
 /*
+ * lutq_fit_histogram / lutq_fit_codebook - a codebook fitted to a layer.
+ *
+ * Source: "TurboQuant: A first-principles walkthrough" (the Lloyd-Max
+ * algorithm) applied to the layer's own normalised weights, the family of the
+ * FLUTE abstract's extension of NormalFloat.  Readings: the data are the
+ * values v = fp32(w) / fp32(s) that lutq_quantize compares with the levels
+ * (s = the group's absolute maximum, v = 0 for an all-zero group), counted in
+ * 16384 bins over [-1, 1]: bin b = floor(fp32(v + 1) * 8192), clamped to
+ * 16383, centre c_b = (2b + 1 - 16384) / 16384.  Lloyd-Max from a starting
+ * codebook: each bin to its nearest level (fp64 distance, ties to the lower
+ * level), each level to the count-weighted mean of its bins' centres (an
+ * exact integer ratio; a level with no bins stays), until the assignment
+ * repeats or max_iter passes; the levels are rounded once to bf16.
+ *
+ * lutq_fit_histogram (device): W bf16 [N,K] row-major (K % 128 == 0, N >= 1);
+ *   hist device uint64 [16384], ADDED to (zero it first; several matrices
+ *   may share one histogram); dev_status: LUTQ_ERR_NONFINITE for a NaN or
+ *   infinite weight.  Asynchronous on `stream`; pointers 16-byte aligned.
+ * lutq_fit_codebook (HOST, no GPU use): hist host uint64 [16384] (fewer than
+ *   2^31 weights in all); init host bf16 [1 << bits] ascending (e.g. from
+ *   lutq_codebook); out host bf16 [1 << bits], written (ascending).
+ *   Returns LUTQ_ERR_BITS for bits other than 3 or 4, LUTQ_ERR_INVALID_ARG
+ *   for NULL pointers, max_iter < 0, a non-finite start or too many counts.
+ */
+lutq_status lutq_fit_histogram(const void* W_bf16, int64_t N, int64_t K, uint64_t* hist,
+                               int32_t* dev_status, void* stream);
+lutq_status lutq_fit_codebook(const uint64_t* hist, int bits, const uint16_t* init_bf16,
+                              int max_iter, uint16_t* out_bf16);
+
+/*
  * lutq_rht_weights / lutq_rht_activations - randomized Hadamard rotation of
  * every 128-long group of each row.
  *
