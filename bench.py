@@ -337,6 +337,27 @@ def side_measurements(lq, dev, args):
                   "us": t_r * 1e6, "kernel": "lutq::gemv_small_kernel (rotating)",
                   "rel_error_vs_unquantized": {"plain": err_plain, "rotated": err_rot}}
     del packs_r, packed_r, packed_plain
+    # codebook fitted to the same layer: the histogram pass (GB/s of weights
+    # read) and the product's error against the unquantized one, starting
+    # codebook against fitted
+    hist = torch.zeros(lq.HIST_BINS, dtype=torch.int64, device=dev)
+    lq.lutq_fit_histogram(w, hist=hist, status=st)
+    th = time_events(lambda i: lq.lutq_fit_histogram(w, hist=hist, status=st), 5)
+    hist.zero_()
+    lq.lutq_fit_histogram(w, hist=hist, status=st)
+    fitted = lq.lutq_fit_codebook(hist.cpu(), bits, cb.cpu()).to(dev)
+    codes_f, scales_f = lq.lutq_quantize(w, fitted, bits, status=st)
+    y_fit = lq.lutq_gemv(x1, lq.lutq_pack(codes_f, scales_f, bits, status=st), fitted, bits, n, k,
+                         workspace=ws1, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    err_fit = float(np.linalg.norm(y_fit.double().cpu().numpy() - exact) / np.linalg.norm(exact))
+    out["fitted_codebook"] = {"histogram_gbs": n * k * 2 / th / 1e9, "histogram_us": th * 1e6,
+                              "rel_error_vs_unquantized": {args.codebook: err_plain,
+                                                           "fitted": err_fit},
+                              "note": "Lloyd-Max on the layer's normalised weights from "
+                                      f"{args.codebook}; same GEMV"}
+    del codes_f, scales_f
     out["offline"] = {"quantize_gbs": q_bytes / tq / 1e9, "quantize_us": tq * 1e6,
                       "pack_gbs": p_bytes / tp / 1e9, "pack_us": tp * 1e6,
                       "note": "W bf16 -> codes u8 + scales; codes + scales -> layout V2 (L2-warm)"}

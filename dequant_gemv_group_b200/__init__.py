@@ -6,6 +6,7 @@ The work is done by ``liblutq.so`` (CUDA kernels behind a C ABI, declared in
 """
 from ._binding import (  # noqa: F401
     CODEBOOK_KINDS,
+    HIST_BINS,
     LIB_PATH,
     LutqError,
     lib,

@@ -48,7 +48,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kTmemCols = 512;
 template <int NT>
 struct GemmCfg {
-  static constexpr int XS = NT >= 128 ? 3 : 4;     // activation stages (shared memory)
+  // activation stages (shared memory); two at N_tile = 128 leave 32 KB more
+  // to L1 (measured 2% faster at batch 128 than three; four: 25% slower)
+  static constexpr int XS = NT >= 128 ? 2 : 4;
   static constexpr int XSTAGE = 2 * NT * 128;       // two boxes of NT rows x 128 bytes
   static constexpr int AS = 4;                      // A stages in tensor memory (64 columns each)
   static constexpr int DS = NT >= 128 ? 2 : (NT >= 64 ? 3 : 4);  // partial stages (NT columns)
