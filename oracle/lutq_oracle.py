@@ -33,6 +33,9 @@ silent the build's readings are used and stated at each function:
   minimising the fp32 value |v - c_i|; an all-zero group uses v = 0;
 * the product is y[m, n] = sum_g s[n, g] * sum_{k in g} x[m, k] * c[q[n, k]]
   accumulated in fp64 (every product is exact in fp64).
+* per-group types (BitMoD abstract): up to 4 (4-bit) or 2 (3-bit) codebooks;
+  a group takes the type of smallest squared RTN error, summed in fp64 in k
+  order, lowest index on ties.
 
 Parity of every function here is pinned in ``tests/test_oracle_pins.py``.
 """
@@ -522,6 +525,160 @@ def fit_codebook(hist, init_levels, max_iter: int = 100) -> np.ndarray:
                 num = int(np.sum(counts[cell] * ints[cell]))   # exact: |num| < 2^59
                 levels[i] = float(num) / float(den * HIST_BINS)
     return bf16_round(levels)
+
+
+# --------------------------------------------------------------------------
+# Per-group data types (BitMoD abstract: each group of 128 weights may be
+# quantized with its own numerical data type)
+# --------------------------------------------------------------------------
+#
+# Readings (the abstract names the idea, not the types or the rule): a layer
+# has T codebooks ("types"), T <= 4 for 4-bit codes and T <= 2 for 3-bit
+# codes.  Every group keeps the absolute-maximum scale s; for each type t the
+# codes q_t are the RTN codes of quantize() on that type's levels, and the
+# group's error is
+#     E_t = sum over k = 0, 1, ..., 127 in this order of d_k * d_k,
+#     d_k = fp32(v_k - c_t[q_t[k]])   (the RTN distance, signed),
+# each product exact in fp64 and each addition rounded in fp64.  The group
+# takes the lowest t of smallest E_t (strictly smaller replaces), and its
+# codes are that type's.  Packing appends, after the scale blocks, 8 bytes per
+# unit t = strip * G + g: byte rq (0..7) holds the types of rows rq + 8 i,
+# i = 0..3, in bits 2i + 1 : 2i.
+
+MAX_TYPES = {4: 4, 3: 2}
+TYPE_BLOCK = 8       # bytes of one unit's group types
+
+
+def _normalised(w) -> Tuple[np.ndarray, np.ndarray]:
+    """Per group of 128: v = fp32(w) / fp32(s) with s the absolute maximum
+    (v = 0 when s == 0), as quantize() computes them; (v[N, G, 128], s[N, G])."""
+    w = np.asarray(w, dtype=np.float32)
+    n, k = w.shape
+    if k % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    if not np.all(np.isfinite(w)):
+        raise ValueError("non-finite weight")
+    wg = w.reshape(n, k // GROUP, GROUP)
+    s = np.max(np.abs(wg), axis=2)
+    s_b = np.broadcast_to(s[:, :, None], wg.shape)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s_b > 0, wg / s_b, np.float32(0.0)).astype(np.float32)
+    return v, s
+
+
+def type_errors(w, type_levels, bits: int) -> np.ndarray:
+    """E[t, n, g] (fp64): each type's squared RTN error over the group, summed
+    over k in increasing order."""
+    levels = [np.asarray(l, dtype=np.float32) for l in type_levels]
+    v, _ = _normalised(w)
+    n, g, _ = v.shape
+    errs = np.zeros((len(levels), n, g), dtype=np.float64)
+    for t, lv in enumerate(levels):
+        codes, _ = quantize(w, lv, bits)
+        c = lv[codes.reshape(n, g, GROUP)]                   # float32 levels
+        d = (v - c).astype(np.float32).astype(np.float64)    # the fp32 difference
+        for kk in range(GROUP):                              # k = 0, 1, ..., 127
+            errs[t] = errs[t] + d[:, :, kk] * d[:, :, kk]
+    return errs
+
+
+def quantize_typed(w, type_levels, bits: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """(codes uint8[N, K], scale bits uint16[N, G], types uint8[N, G]): every
+    group quantized with the type of smallest error (lowest index on ties)."""
+    if bits not in MAX_TYPES:
+        raise ValueError("bits must be 3 or 4")
+    if not 1 <= len(type_levels) <= MAX_TYPES[bits]:
+        raise ValueError("number of types")
+    errs = type_errors(w, type_levels, bits)
+    n, g = errs.shape[1:]
+    best = np.zeros((n, g), dtype=np.uint8)
+    best_e = errs[0].copy()
+    for t in range(1, len(type_levels)):
+        take = errs[t] < best_e
+        best[take] = t
+        best_e[take] = errs[t][take]
+    codes = np.zeros((n, g * GROUP), dtype=np.uint8)
+    sb = None
+    for t, lv in enumerate(type_levels):
+        q_t, sb = quantize(w, lv, bits)
+        pick = np.repeat(best == t, GROUP, axis=1)
+        codes[pick] = q_t[pick]
+    return codes, sb, best
+
+
+def packed_bytes_typed(n: int, k: int, bits: int) -> int:
+    return packed_bytes(n, k, bits) + (n // STRIP) * (k // GROUP) * TYPE_BLOCK
+
+
+def pack_typed(codes, scale_bits, types, bits: int) -> np.ndarray:
+    """pack() followed by the type blocks (8 bytes per unit)."""
+    q = np.asarray(codes, dtype=np.uint8)
+    n, k = q.shape
+    ty = np.asarray(types, dtype=np.uint8)
+    g = k // GROUP
+    if ty.shape != (n, g):
+        raise ValueError("types shape mismatch")
+    if np.any(ty >= MAX_TYPES[bits]):
+        raise ValueError("type out of range")
+    body = pack(q, scale_bits, bits)
+    # row r = 8 i + rq of strip s -> bits 2i+1:2i of byte rq of unit (s, g)
+    t4 = ty.reshape(n // STRIP, 4, 8, g).astype(np.uint32)      # [s, i, rq, g]
+    byte = np.zeros((n // STRIP, 8, g), dtype=np.uint32)
+    for i in range(4):
+        byte |= t4[:, i] << (2 * i)
+    blocks = byte.transpose(0, 2, 1).astype(np.uint8)             # [s, g, rq]
+    return np.concatenate([body, np.ascontiguousarray(blocks).reshape(-1)])
+
+
+def unpack_typed(packed, n: int, k: int, bits: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Inverse of pack_typed, the type bytes read one by one."""
+    p = np.asarray(packed, dtype=np.uint8)
+    if p.size != packed_bytes_typed(n, k, bits):
+        raise ValueError("packed size mismatch")
+    body = packed_bytes(n, k, bits)
+    q, sb = unpack(p[:body], n, k, bits)
+    g = k // GROUP
+    ty = np.zeros((n, g), dtype=np.uint8)
+    for row in range(n):
+        s, r = divmod(row, STRIP)
+        for gi in range(g):
+            byte = int(p[body + (s * g + gi) * TYPE_BLOCK + r % 8])
+            ty[row, gi] = (byte >> (2 * (r // 8))) & 3
+    return q, sb, ty
+
+
+def typed_levels(types, type_levels) -> np.ndarray:
+    """c[n, g, i]: the levels (fp64) of each group's type."""
+    table = np.stack([np.asarray(l, dtype=np.float64) for l in type_levels])
+    return table[np.asarray(types)]
+
+
+def dequant_typed(codes, scale_bits, types, type_levels) -> np.ndarray:
+    """W_hat[n, k] = s[n, g] * c_{type[n, g]}[q[n, k]] in fp64 (exact)."""
+    q = np.asarray(codes)
+    n, k = q.shape
+    c = typed_levels(types, type_levels)                          # [N, G, L]
+    qg = q.reshape(n, k // GROUP, GROUP)
+    vals = np.take_along_axis(c, qg.astype(np.int64), axis=2)     # [N, G, 128]
+    s = bf16_bits_to_f32(scale_bits).astype(np.float64)
+    return (vals * s[:, :, None]).reshape(n, k)
+
+
+def gemv_typed(x, codes, scale_bits, types, type_levels) -> np.ndarray:
+    """y[m, n] = sum_g s[n, g] * sum_{k in g} x[m, k] * c_{type[n, g]}[q[n, k]]
+    in fp64: the per-group partial sum with the group's own levels, rescaled
+    once per group."""
+    xf = np.asarray(x, dtype=np.float64)
+    q = np.asarray(codes)
+    n, k = q.shape
+    m = xf.shape[0]
+    g = k // GROUP
+    c = typed_levels(types, type_levels)
+    cq = np.take_along_axis(c, q.reshape(n, g, GROUP).astype(np.int64), axis=2)  # [N, G, 128]
+    xg = xf.reshape(m, g, GROUP)
+    partial = np.einsum("mgk,ngk->gmn", xg, cq)                   # [G, M, N]
+    s = bf16_bits_to_f32(scale_bits).astype(np.float64)
+    return np.sum(partial * s.T[:, None, :], axis=0)
 
 
 def gemv_rows(x, w_rows, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
