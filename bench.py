@@ -358,6 +358,42 @@ def side_measurements(lq, dev, args):
                               "note": "Lloyd-Max on the layer's normalised weights from "
                                       f"{args.codebook}; same GEMV"}
     del codes_f, scales_f
+    # per-group data types on the same layer: the codebooks of the run, then
+    # (4-bit) log-b and uniform, and the fitted one; each group takes the type
+    # of smallest error.  Throughput of the typed GEMV at batch 1 (graph
+    # replay, weights rotating over copies larger than L2), the typed
+    # quantizer's time, and the product's error against the unquantized one
+    tables = [cb] + ([lq.lutq_codebook("logb", 4).to(dev), lq.lutq_codebook("uniform4", 4).to(dev)]
+                     if bits == 4 else []) + [fitted]
+    tables = tables[:lq.lutq_max_types(bits)]
+    cbs = torch.stack(tables).contiguous()
+    codes_t, scales_t, types_t = lq.lutq_quantize_typed(w, cbs, bits, status=st)
+    tt = time_events(lambda i: lq.lutq_quantize_typed(w, cbs, bits, status=st), 1)
+    packed_t = lq.lutq_pack_typed(codes_t, scales_t, types_t, bits, status=st)
+    counts = torch.bincount(types_t.reshape(-1).long(), minlength=len(tables)).cpu().tolist()
+    del codes_t, scales_t, types_t
+    copies = max(2, int(np.ceil(3 * l2 / packed_t.numel())) + 1)
+    packs_t = [packed_t] + [packed_t.clone() for _ in range(copies - 1)]
+    call_t = lambda i: lq.lutq_gemv_typed(x1, packs_t[i % copies], cbs, bits, n, k, y=y1,
+                                          workspace=ws1, status=st)
+    for i in range(4):
+        call_t(i)
+    g_t = capture(call_t, 128)
+    g_t.replay()
+    t_t = time_events(lambda i: g_t.replay(), 8) / 128
+    del g_t
+    y_typed = lq.lutq_gemv_typed(x1, packed_t, cbs, bits, n, k, workspace=ws1, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    err_typed = float(np.linalg.norm(y_typed.double().cpu().numpy() - exact) / np.linalg.norm(exact))
+    typed_bytes = algorithmic_bytes(1, n, k, bits) + (n // 32) * (k // 128) * 8
+    out["typed"] = {"workload": f"{args.workload}/{args.layer} W[{n},{k}] W{bits} batch1, "
+                                f"{len(tables)} codebooks chosen per group of 128",
+                    "value": typed_bytes / t_t / 1e9, "unit": "GB/s", "us": t_t * 1e6,
+                    "kernel": "lutq::gemv_small_kernel (typed)",
+                    "quantize_typed_us": tt * 1e6, "groups_per_type": counts,
+                    "rel_error_vs_unquantized": {args.codebook: err_plain, "typed": err_typed}}
+    del packs_t, packed_t
     out["offline"] = {"quantize_gbs": q_bytes / tq / 1e9, "quantize_us": tq * 1e6,
                       "pack_gbs": p_bytes / tp / 1e9, "pack_us": tp * 1e6,
                       "note": "W bf16 -> codes u8 + scales; codes + scales -> layout V2 (L2-warm)"}

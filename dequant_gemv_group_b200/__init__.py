@@ -18,10 +18,15 @@ from ._binding import (  # noqa: F401
     lutq_gemv_noalloc,
     lutq_gemv_plan,
     lutq_gemv_rht,
+    lutq_gemv_typed,
     lutq_layout_version,
+    lutq_max_types,
     lutq_pack,
+    lutq_pack_typed,
     lutq_packed_bytes,
+    lutq_packed_bytes_typed,
     lutq_quantize,
+    lutq_quantize_typed,
     lutq_rht_activations,
     lutq_rht_weights,
     lutq_selftest_wait_timeout,

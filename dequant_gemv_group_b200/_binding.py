@@ -50,6 +50,12 @@ _SIGS = {
     "lutq_rht_activations": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "lutq_gemv_rht": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
                              _vp]),
+    "lutq_max_types": (_i32, [_i32]),
+    "lutq_packed_bytes_typed": (_i64, [_i64, _i64, _i32]),
+    "lutq_quantize_typed": (_i32, [_vp, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "lutq_pack_typed": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "lutq_gemv_typed": (_i32, [_vp, _i64, _vp, _vp, _i32, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
+                               _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -229,6 +235,68 @@ def lutq_gemv_rht(x, packed, codebook, signs, bits, n, k, y=None, workspace=None
     _check(lib.lutq_gemv_rht(x.data_ptr(), m, packed.data_ptr(), codebook.data_ptr(),
                              signs.data_ptr(), bits, n, k, y.data_ptr(), ws_ptr, ws_bytes,
                              _ptr(status), _stream()), "lutq_gemv_rht")
+    return y
+
+
+def lutq_max_types(bits: int) -> int:
+    return int(lib.lutq_max_types(bits))
+
+
+def lutq_packed_bytes_typed(n: int, k: int, bits: int) -> int:
+    return int(lib.lutq_packed_bytes_typed(n, k, bits))
+
+
+def lutq_quantize_typed(w: torch.Tensor, codebooks: torch.Tensor, bits: int,
+                        status: Optional[torch.Tensor] = None
+                        ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """W bf16 [N, K] and codebooks bf16 [T, 2^bits] -> (codes uint8 [N, K],
+    scales bf16 [N, K/128], group types uint8 [N, K/128]); see
+    lutq_quantize_typed in include/lutq.h."""
+    _need(w, torch.bfloat16, "W")
+    _need(codebooks, torch.bfloat16, "codebooks")
+    if codebooks.dim() != 2 or codebooks.shape[1] != (1 << bits):
+        raise LutqError(3, "lutq_quantize_typed: codebooks must be [T, 2^bits]")
+    n, k = w.shape
+    g = max(k // 128, 1)
+    codes = torch.empty((n, k), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((n, g), dtype=torch.bfloat16, device=w.device)
+    types = torch.empty((n, g), dtype=torch.uint8, device=w.device)
+    _check(lib.lutq_quantize_typed(w.data_ptr(), n, k, codebooks.data_ptr(), codebooks.shape[0],
+                                   bits, codes.data_ptr(), scales.data_ptr(), types.data_ptr(),
+                                   _ptr(status), _stream()), "lutq_quantize_typed")
+    return codes, scales, types
+
+
+def lutq_pack_typed(codes: torch.Tensor, scales: torch.Tensor, types: torch.Tensor, bits: int,
+                    status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """codes, scales and group types -> the packed matrix with type blocks."""
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.bfloat16, "scales")
+    _need(types, torch.uint8, "types")
+    n, k = codes.shape
+    if tuple(scales.shape) != (n, k // 128) or tuple(types.shape) != (n, k // 128):
+        raise LutqError(2, "lutq_pack_typed: scales / types shape")
+    nb = lutq_packed_bytes_typed(n, k, bits)
+    if nb < 0:
+        raise LutqError(2, "lutq_packed_bytes_typed")
+    packed = torch.empty(nb, dtype=torch.uint8, device=codes.device)
+    _check(lib.lutq_pack_typed(codes.data_ptr(), scales.data_ptr(), types.data_ptr(), n, k, bits,
+                               packed.data_ptr(), _ptr(status), _stream()), "lutq_pack_typed")
+    return packed
+
+
+def lutq_gemv_typed(x, packed, codebooks, bits, n, k, y=None, workspace=None, status=None):
+    """y[M, N] (fp32) with per-group types, codebooks bf16 [T, 2^bits]
+    (M = 1..4; see lutq_gemv_typed in include/lutq.h)."""
+    _need(x, torch.bfloat16, "x")
+    _need(codebooks, torch.bfloat16, "codebooks")
+    m = x.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    _check(lib.lutq_gemv_typed(x.data_ptr(), m, packed.data_ptr(), codebooks.data_ptr(),
+                               codebooks.shape[0], bits, n, k, y.data_ptr(), ws_ptr, ws_bytes,
+                               _ptr(status), _stream()), "lutq_gemv_typed")
     return y
 
 

@@ -25,6 +25,17 @@ cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const 
                             void* workspace, int32_t* dev_status, int num_sms,
                             cudaStream_t stream);
 bool gemv_small_path(int64_t M, int64_t K, int bits);
+bool gemv_typed_path(int64_t M, int64_t K);
+cudaError_t launch_quantize_typed(const void* W, int64_t N, int64_t K, const void* codebooks,
+                                  int types, int bits, uint8_t* codes, void* scales,
+                                  uint8_t* group_types, int32_t* dev_status, int num_sms,
+                                  cudaStream_t stream);
+cudaError_t launch_pack_types(const uint8_t* types, int64_t N, int64_t K, int bits, void* packed,
+                              int32_t* dev_status, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemv_typed(const void* x, int64_t M, const void* packed, const void* codebooks,
+                              int types, int bits, int64_t N, int64_t K, float* y,
+                              void* workspace, int32_t* dev_status, int num_sms,
+                              cudaStream_t stream);
 cudaError_t launch_rht(const void* in, int64_t rows, int64_t K, const int8_t* signs,
                        bool activations, void* out, int num_sms, cudaStream_t stream);
 cudaError_t launch_fit_histogram(const void* W, int64_t N, int64_t K, uint64_t* hist,
@@ -246,6 +257,64 @@ lutq_status lutq_gemv_rht(const void* x_bf16, int64_t M, const void* packed,
   return from_cuda(lutq::launch_gemv_rht(x_bf16, M, packed, codebook_bf16, signs, bits, N, K, y,
                                          workspace, dev_status, sms,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+int lutq_max_types(int bits) { return check_bits(bits) == LUTQ_OK ? lutq::max_types(bits) : -1; }
+
+int64_t lutq_packed_bytes_typed(int64_t N, int64_t K, int bits) {
+  const int64_t body = lutq_packed_bytes(N, K, bits);
+  if (body < 0) return -1;
+  return body + (N / lutq::kStrip) * (K / lutq::kGroup) * lutq::kTypeBytes;
+}
+
+lutq_status lutq_quantize_typed(const void* W_bf16, int64_t N, int64_t K,
+                                const void* codebooks_bf16, int types, int bits, uint8_t* codes,
+                                void* scales_bf16, uint8_t* group_types, int32_t* dev_status,
+                                void* stream) {
+  if (!W_bf16 || !codebooks_bf16 || !codes || !scales_bf16 || !group_types)
+    return LUTQ_ERR_INVALID_ARG;
+  lutq_status st = check_bits(bits);
+  if (st != LUTQ_OK) return st;
+  if (types < 1 || types > lutq::max_types(bits)) return LUTQ_ERR_INVALID_ARG;
+  if ((st = check_shape(N, K)) != LUTQ_OK) return st;
+  if (!aligned16(W_bf16) || !aligned16(codebooks_bf16) || !aligned16(codes) ||
+      !aligned16(scales_bf16) || !aligned16(group_types))
+    return LUTQ_ERR_ALIGN;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_quantize_typed(W_bf16, N, K, codebooks_bf16, types, bits, codes,
+                                               scales_bf16, group_types, dev_status, sms,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_pack_typed(const uint8_t* codes, const void* scales_bf16,
+                            const uint8_t* group_types, int64_t N, int64_t K, int bits,
+                            void* packed, int32_t* dev_status, void* stream) {
+  if (!group_types) return LUTQ_ERR_INVALID_ARG;
+  if (!aligned16(group_types)) return LUTQ_ERR_ALIGN;
+  lutq_status st = lutq_pack(codes, scales_bf16, N, K, bits, packed, dev_status, stream);
+  if (st != LUTQ_OK) return st;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_pack_types(group_types, N, K, bits, packed, dev_status, sms,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_gemv_typed(const void* x_bf16, int64_t M, const void* packed,
+                            const void* codebooks_bf16, int types, int bits, int64_t N, int64_t K,
+                            float* y, void* workspace, int64_t workspace_bytes,
+                            int32_t* dev_status, void* stream) {
+  lutq_status st = check_product_args(x_bf16, M, 16, packed, codebooks_bf16, bits, N, K, y,
+                                      workspace, workspace_bytes,
+                                      lutq_workspace_bytes(M, N, K, bits));
+  if (st != LUTQ_OK) return st;
+  if (types < 1 || types > lutq::max_types(bits)) return LUTQ_ERR_INVALID_ARG;
+  if (!lutq::gemv_typed_path(M, K)) return LUTQ_ERR_SHAPE;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_gemv_typed(x_bf16, M, packed, codebooks_bf16, types, bits, N, K,
+                                           y, workspace, dev_status, sms,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

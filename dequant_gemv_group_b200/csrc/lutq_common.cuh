@@ -20,6 +20,12 @@ __host__ __device__ constexpr int tile_bytes(int bits) { return bits == 4 ? 2048
 __host__ __device__ constexpr int scale_slot(int r) { return 2 * (4 * (r & 7) + (r >> 3)); }
 __host__ __device__ constexpr int words_per_row(int bits) { return bits == 4 ? 4 : 3; }
 
+// Per-group data types: up to 4 codebooks with 4-bit codes, 2 with 3-bit
+// codes (the kernels' tables must fit shared memory); a matrix packed with
+// types carries 8 type bytes per unit after the scale blocks.
+constexpr int kTypeBytes = 8;
+__host__ __device__ constexpr int max_types(int bits) { return bits == 4 ? 4 : 2; }
+
 // Record a device-side error: the first non-zero code wins.
 __device__ __forceinline__ void report(int32_t* dev_status, int code) {
   if (dev_status != nullptr) atomicCAS(dev_status, 0, code);

@@ -69,6 +69,8 @@ struct GemvArgs {
   unsigned long long* xch;  // [M][N] exchange slots of strips split between two CTAs (zero between calls)
   int32_t* status;          // caller's device status word or null
   const int8_t* signs;      // randomized Hadamard rotation of x first (null: none)
+  int types;                // per-group data types: codebook holds `types` tables
+                            // and the packed matrix its type blocks (0: untyped)
   int64_t N, K, G, U;       // U = number of units
   int C;                    // CTAs
   // work plan (choose_plan): kind 0 = ranges of the unit sequence, strip-
@@ -248,15 +250,21 @@ __device__ void cta_finish(const GemvArgs& a, const Span& p, const float* all_sl
 // formed as (row << 8 | column); kLutAt goes into the load's offset.
 constexpr uint32_t kSbaseMax = 4096;
 constexpr uint32_t kLutAt = kSbaseMax;
-constexpr uint32_t kXAt = kLutAt + 0x10000;
 constexpr uint32_t kXChunkBytes = 64;
 constexpr uint32_t kXGroupBytes = 4 * kXChunkBytes;
 
-__host__ __device__ constexpr uint32_t slots_at(uint32_t K, int M) {
-  return kXAt + uint32_t(M) * K * 2u;  // K * 2 is a multiple of 256
+// With per-group data types the table region is 128 KB: table t of 4-bit
+// codes in row half t & 1 of the 64 KB at (t >> 1) << 16, table t of 3-bit
+// codes (both halves) in the 64 KB at t << 16.  The address bits 23:16 come
+// from bits 15:8 of the lane's column word.
+__host__ __device__ constexpr uint32_t x_at(bool typed) {
+  return kLutAt + (typed ? 0x20000u : 0x10000u);
 }
-__host__ __device__ constexpr uint32_t small_end(uint32_t K, int M) {
-  return slots_at(K, M) + uint32_t(kM1Warps * 2 * M * kStrip * 4);
+__host__ __device__ constexpr uint32_t slots_at(uint32_t K, int M, bool typed) {
+  return x_at(typed) + uint32_t(M) * K * 2u;  // K * 2 is a multiple of 256
+}
+__host__ __device__ constexpr uint32_t small_end(uint32_t K, int M, bool typed) {
+  return slots_at(K, M, typed) + uint32_t(kM1Warps * 2 * M * kStrip * 4);
 }
 
 // The table entry (a bf16x2 pair of levels) at table address t.
@@ -295,15 +303,16 @@ __device__ __forceinline__ void pair_first(float& acc, uint32_t lv, uint32_t xw)
 // read).
 template <bool FIRST, int M>
 __device__ __forceinline__ void quad4(float (&su)[4][M], const uint32_t (&idx)[4],
-                                      uint32_t lane_col, const uint32_t (&xq)[M][4]) {
+                                      const uint32_t (&lc)[4], const uint32_t (&xq)[M][4]) {
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     uint32_t lv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      // row = byte b of the index word (bits 15:8), column = the lane's
-      // (bits 7:0; lane_col < 256, so bits 31:16 are zero)
-      lv[i] = lut_ld(__byte_perm(idx[i], lane_col, 0x6504u | (uint32_t(b) << 4)));
+      // row = byte b of the index word (bits 15:8), column = byte 0 of row
+      // i's column word (bits 7:0), table = its byte 1 (bits 23:16; byte 2
+      // is zero)
+      lv[i] = lut_ld(__byte_perm(idx[i], lc[i], 0x6504u | (uint32_t(b) << 4)));
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -380,11 +389,20 @@ __device__ __forceinline__ void fetch_unit(uint4 (&wd)[4], uint32_t (&sv)[2], co
   }
 }
 
+// The lane's type byte of one unit (per-group data types), loaded only if
+// live > 0.
+__device__ __forceinline__ void fetch_type_byte(uint32_t& ty, const uint8_t* p, int live) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.gt.s32 p, %2, 0;\n\t@p ld.global.nc.u8 %0, [%1];\n\t}"
+      : "+r"(ty) : "l"(p), "r"(live));
+}
+
 // Row sums of one unit for the lane's four rows and the M batch rows; xa is
 // the address of the lane's 32 activations of the group for batch row 0.
 template <int BITS, int M>
 __device__ __forceinline__ void unit_partial(float (&su)[4][M], const uint4 (&wd)[4],
-                                             uint32_t lane_e, uint32_t lane_o, uint32_t hi_shift,
+                                             const uint32_t (&lce)[4], const uint32_t (&lco)[4],
+                                             uint32_t hi_shift,
                                              uint32_t xa, uint32_t xstride) {
   uint32_t xq[M][4];
   if (BITS == 4) {
@@ -396,9 +414,9 @@ __device__ __forceinline__ void unit_partial(float (&su)[4][M], const uint4 (&wd
                                j == 0 ? wd[2].x : j == 1 ? wd[2].y : j == 2 ? wd[2].z : wd[2].w,
                                j == 0 ? wd[3].x : j == 1 ? wd[3].y : j == 2 ? wd[3].z : wd[3].w};
       if (j == 0)
-        quad4<true, M>(su, idx, lane_e, xq);
+        quad4<true, M>(su, idx, lce, xq);
       else
-        quad4<false, M>(su, idx, lane_e, xq);
+        quad4<false, M>(su, idx, lce, xq);
     }
   } else {
     // lo u32 j goes with hi u32 j; lo word 1 reads its hi fields two bits up
@@ -414,11 +432,11 @@ __device__ __forceinline__ void unit_partial(float (&su)[4][M], const uint4 (&wd
       }
       load_xq<M>(xq, xa + 32u * j, xstride);
       if (j == 0)
-        quad4<true, M>(su, e, lane_e, xq);
+        quad4<true, M>(su, e, lce, xq);
       else
-        quad4<false, M>(su, e, lane_e, xq);
+        quad4<false, M>(su, e, lce, xq);
       load_xq<M>(xq, xa + 32u * j + 16u, xstride);
-      quad4<false, M>(su, o, lane_o, xq);
+      quad4<false, M>(su, o, lco, xq);
     }
   }
 }
@@ -442,18 +460,20 @@ __device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
-__device__ __forceinline__ uint32_t ld_cg_u16(const uint16_t* p) {
+__device__ __forceinline__ uint32_t ld_cg_u32(const uint16_t* p) {
   uint32_t r;
-  asm volatile("ld.global.cg.u16 %0, [%1];" : "=r"(r) : "l"(p));
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(r) : "l"(p));
   return r;
 }
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-template <int BITS, int M, int NB>
+template <int BITS, int M, int NB, bool TYPED>
 __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a) {
   constexpr int TB = tile_bytes(BITS);
+  constexpr int UB = TB + kScaleBytes + (TYPED ? kTypeBytes : 0);  // packed bytes per unit
+  constexpr uint32_t kXAt = x_at(TYPED);
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ WarpTable<kM1Warps> wt;
   const uint32_t sbase = sm_addr(smem);
@@ -466,7 +486,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
   // prefetch reads nothing into the kernel, so it needs no wait for the
   // preceding kernel).
   if (blockIdx.x < a.pf_ctas) {
-    const uint32_t lines = uint32_t((uint64_t(a.U) * (TB + kScaleBytes) + 127u) / 128u);
+    const uint32_t lines = uint32_t((uint64_t(a.U) * UB + 127u) / 128u);
     for (uint32_t j = blockIdx.x * blockDim.x + threadIdx.x; j < lines;
          j += a.pf_ctas * blockDim.x)
       prefetch_l2(a.packed + uint64_t(j) * 128u);
@@ -492,6 +512,8 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
   const uint8_t* const pk = a.packed + lane_off;
   // the scales of the lane's rows rq + 8 i, i = 0..3: 8 bytes of each unit's 64
   const uint8_t* const psc = a.packed + uint64_t(a.U) * TB + scale_slot(rq);
+  // per-group types: byte rq of each unit's 8 (rows rq + 8 i in bits 2i+1:2i)
+  const uint8_t* const pty = a.packed + uint64_t(a.U) * (TB + kScaleBytes) + rq;
 
   // Before the preceding kernel on the stream is complete (this kernel is
   // its programmatic dependent) nothing is read.  Without prefetching CTAs,
@@ -506,6 +528,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 #pragma unroll
         for (int i = 0; i < 4; ++i) prefetch_l2(p + 128 * i);
         if (lane == 0) prefetch_l2(wide_addr(psc, t, uint32_t(kScaleBytes)));
+        if (TYPED && lane == 0) prefetch_l2(wide_addr(pty, t, uint32_t(kTypeBytes)));
       }
       ++t;
       if (--l == 0) {
@@ -524,9 +547,10 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
     return;
   }
 
-  auto fetch = [&](uint4 (&wd)[4], uint32_t (&sv)[2]) {
+  auto fetch = [&](uint4 (&wd)[4], uint32_t (&sv)[2], uint32_t& ty) {
     fetch_unit<BITS>(wd, sv, wide_addr(pk, ft, TB), hi_delta,
                      wide_addr(psc, ft, uint32_t(kScaleBytes)), fn);
+    if (TYPED) fetch_type_byte(ty, wide_addr(pty, ft, uint32_t(kTypeBytes)), fn);
     --fn;
     ++ft;
     if (--fleft == 0) {  // on to the window's first group of the next strip
@@ -541,7 +565,10 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
   // and the first tile; the other NB - 1 tiles once the activations are in.
   uint4 buf[NB][4];
   uint32_t sbuf[NB][2];
-  uint32_t cbv;
+  uint32_t tbuf[NB];
+#pragma unroll
+  for (int t = 0; t < NB; ++t) tbuf[t] = 0;
+  uint32_t cbw = 0;  // bytes 4 lane .. 4 lane + 3 of the codebook array
   {
     constexpr uint32_t kStep = kM1Warps * 32 * 16;
     const uint32_t xbytes = uint32_t(M) * K * 2u;
@@ -552,8 +579,9 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 #pragma unroll
     for (int j = 0; j < 4; ++j)
       if (o + j * kStep < xbytes) v[j] = ld_cg_v4(xg + o + j * kStep);
-    cbv = ld_cg_u16(a.codebook + (lane & ((1 << BITS) - 1)));
-    fetch(buf[0], sbuf[0]);
+    // all tables in one warp-wide load (at most 128 bytes)
+    if (lane < ((TYPED ? a.types : 1) << (BITS - 1))) cbw = ld_cg_u32(a.codebook + 2 * lane);
+    fetch(buf[0], sbuf[0], tbuf[0]);
     for (;;) {
 #pragma unroll
       for (int j = 0; j < 4; ++j)
@@ -565,9 +593,12 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
         if (o + j * kStep < xbytes) v[j] = ld_cg_v4(xg + o + j * kStep);
     }
   }
-  build_lut_shfl<BITS>(smem + (kLutAt - sbase), cbv);
+  if (TYPED)
+    build_luts_typed<BITS>(smem + (kLutAt - sbase), cbw, a.types);
+  else
+    build_lut_shfl<BITS>(smem + (kLutAt - sbase), cbw);
 #pragma unroll
-  for (int t = 1; t < NB; ++t) fetch(buf[t], sbuf[t]);
+  for (int t = 1; t < NB; ++t) fetch(buf[t], sbuf[t], tbuf[t]);
   if (a.signs != nullptr) {
     // Rotate every 128-long group of the activations in place, eight lanes
     // per group: x_g <- H diag(s) x_g / 128, fp32 butterflies (as
@@ -609,7 +640,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 
   const uint32_t lane_e = uint32_t(lane) * 4u, lane_o = 128u + uint32_t(lane) * 4u;
   const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
-  float* const slots = reinterpret_cast<float*>(smem + (slots_at(K, M) - sbase));
+  float* const slots = reinterpret_cast<float*>(smem + (slots_at(K, M, TYPED) - sbase));
   float* const my_slots = slots + wl * 2 * M * kStrip;
   int rows[4];
 #pragma unroll
@@ -631,9 +662,21 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 #pragma unroll
       for (int m = 0; m < M; ++m) acc[i][m] = 0.0f;
     // Consume the unit held in (wd, sv); true once the range is done.
-    auto step = [&](const uint4 (&wd)[4], const uint32_t (&sv)[2]) -> bool {
+    auto step = [&](const uint4 (&wd)[4], const uint32_t (&sv)[2], uint32_t ty) -> bool {
+      // each row's column words: the lane's column, and with per-group types
+      // the row's table (4-bit: type bit 0 -> address bit 7, bit 1 -> bit 16;
+      // 3-bit: type bit 0 -> bit 16)
+      uint32_t lce[4], lco[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t sel = 0;
+        if (TYPED)
+          sel = BITS == 4 ? ((ty << 7) >> (2 * i)) & 0x180u : ((ty << 8) >> (2 * i)) & 0x100u;
+        lce[i] = lane_e | sel;
+        lco[i] = lane_o | sel;
+      }
       float su[4][M];
-      unit_partial<BITS, M>(su, wd, lane_e, lane_o, hi_shift, xa, xstride);
+      unit_partial<BITS, M>(su, wd, lce, lco, hi_shift, xa, xstride);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float s = (i & 1) ? bf16_hi_to_f32(sv[i >> 1]) : bf16_lo_to_f32(sv[i >> 1]);
@@ -666,8 +709,8 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
     for (;;) {
 #pragma unroll
       for (int t = 0; t < NB; ++t) {
-        if (step(buf[t], sbuf[t])) goto range_done;
-        fetch(buf[t], sbuf[t]);
+        if (step(buf[t], sbuf[t], tbuf[t])) goto range_done;
+        fetch(buf[t], sbuf[t], tbuf[t]);
       }
     }
   range_done:;
@@ -776,6 +819,7 @@ void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out) {
 constexpr int64_t kPrefetchBytes = int64_t(64) << 20;
 
 static void apply_plan(GemvArgs& a, int num_sms, int bits) {
+  const int64_t unit_bytes = tile_bytes(bits) + kScaleBytes + (a.types > 0 ? kTypeBytes : 0);
   const Plan pl = choose_plan(a.N / kStrip, a.G, num_sms);
   a.C = pl.C;
   a.kind = pl.kind;
@@ -783,23 +827,24 @@ static void apply_plan(GemvArgs& a, int num_sms, int bits) {
   a.Cm = pl.Cm;
   a.T = pl.T;
   a.nh = pl.nh;
-  const int64_t bytes = a.U * (tile_bytes(bits) + kScaleBytes);
+  const int64_t bytes = a.U * unit_bytes;
   a.pf_ctas = pl.C < num_sms && bytes <= kPrefetchBytes ? uint32_t(num_sms - pl.C) : 0u;
 }
 
 
-static int64_t small_smem(int64_t K, int M) {
-  return K < (int64_t(1) << 20) ? int64_t(small_end(uint32_t(K), M)) : int64_t(1) << 30;
+static int64_t small_smem(int64_t K, int M, bool typed) {
+  return K < (int64_t(1) << 20) ? int64_t(small_end(uint32_t(K), M, typed)) : int64_t(1) << 30;
 }
 
-template <int BITS, int M>
+template <int BITS, int M, bool TYPED>
 static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
   static SmemGrant grant2, grant3;
-  const int smem = int(small_smem(a.K, M));
+  const int smem = int(small_smem(a.K, M, TYPED));
   apply_plan(a, num_sms, BITS);
-  constexpr int kDeep = M == 1 ? 3 : 2;
-  const bool deep = M == 1 && a.pf_ctas == 0;
-  auto kernel = deep ? gemv_small_kernel<BITS, M, kDeep> : gemv_small_kernel<BITS, M, 2>;
+  constexpr int kDeep = M == 1 && !TYPED ? 3 : 2;
+  const bool deep = M == 1 && !TYPED && a.pf_ctas == 0;
+  auto kernel = deep ? gemv_small_kernel<BITS, M, kDeep, TYPED>
+                     : gemv_small_kernel<BITS, M, 2, TYPED>;
   cudaError_t err = grant_smem(kernel, deep ? grant3 : grant2, smem);
   if (err != cudaSuccess) return err;
   // programmatic dependent launch: the prefetching blocks and the work
@@ -828,18 +873,18 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
 // so they, and over-long rows, take the tcgen05 kernel of lutq_gemm.
 constexpr int kMaxSmallBatch = 4;
 
-template <int BITS>
-static bool small_fits(int64_t M, int64_t K) {
-  return M >= 1 && M <= kMaxSmallBatch && small_smem(K, int(M)) <= kMaxSmemPerBlock - 1024;
+static bool small_fits(int64_t M, int64_t K, bool typed = false) {
+  return M >= 1 && M <= kMaxSmallBatch &&
+         small_smem(K, int(M), typed) <= kMaxSmemPerBlock - 1024;
 }
 
-template <int BITS>
+template <int BITS, bool TYPED = false>
 static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream_t s) {
   switch (M) {
-    case 1: return launch_small<BITS, 1>(a, num_sms, s);
-    case 2: return launch_small<BITS, 2>(a, num_sms, s);
-    case 3: return launch_small<BITS, 3>(a, num_sms, s);
-    default: return launch_small<BITS, 4>(a, num_sms, s);
+    case 1: return launch_small<BITS, 1, TYPED>(a, num_sms, s);
+    case 2: return launch_small<BITS, 2, TYPED>(a, num_sms, s);
+    case 3: return launch_small<BITS, 3, TYPED>(a, num_sms, s);
+    default: return launch_small<BITS, 4, TYPED>(a, num_sms, s);
   }
 }
 
@@ -854,6 +899,7 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   a.xch = static_cast<unsigned long long*>(workspace);
   a.status = dev_status;
   a.signs = nullptr;
+  a.types = 0;
   a.N = N;
   a.K = K;
   a.G = K / kGroup;
@@ -861,8 +907,7 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   a.C = 0;
   // unit indices and range arithmetic are 32-bit (U * CTAs < 2^32)
   if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
-  const bool small = bits == 4 ? small_fits<4>(M, K) : small_fits<3>(M, K);
-  if (!small)
+  if (!small_fits(M, K))
     return launch_gemm(x, M, packed, codebook, bits, N, K, y, workspace, dev_status,
                        num_sms, stream);
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
@@ -871,8 +916,13 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
 
 // Whether lutq_gemv runs an M x K product on the CUDA-core kernel.
 bool gemv_small_path(int64_t M, int64_t K, int bits) {
-  return bits == 4 ? small_fits<4>(M, K) : small_fits<3>(M, K);
+  (void)bits;
+  return small_fits(M, K);
 }
+
+// Whether lutq_gemv_typed can run an M x K product (the CUDA-core kernel with
+// the 128 KB table region).
+bool gemv_typed_path(int64_t M, int64_t K) { return small_fits(M, K, true); }
 
 // lutq_gemv with the activations rotated in the kernel's prologue; only for
 // the CUDA-core kernel (the caller checks gemv_small_path).
@@ -889,6 +939,7 @@ cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const 
   a.xch = static_cast<unsigned long long*>(workspace);
   a.status = dev_status;
   a.signs = signs;
+  a.types = 0;
   a.N = N;
   a.K = K;
   a.G = K / kGroup;
@@ -897,6 +948,34 @@ cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const 
   if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
                    : launch_bits<3>(a, int(M), num_sms, stream);
+}
+
+// lutq_gemv with per-group data types: `codebooks` holds `types` tables of
+// 2^bits levels and `packed` the type blocks; only for the CUDA-core kernel
+// (the caller checks gemv_typed_path).
+cudaError_t launch_gemv_typed(const void* x, int64_t M, const void* packed, const void* codebooks,
+                              int types, int bits, int64_t N, int64_t K, float* y,
+                              void* workspace, int32_t* dev_status, int num_sms,
+                              cudaStream_t stream) {
+  if (!gemv_typed_path(M, K) || types < 1 || types > max_types(bits))
+    return cudaErrorInvalidValue;
+  GemvArgs a;
+  a.x = static_cast<const uint16_t*>(x);
+  a.packed = static_cast<const uint8_t*>(packed);
+  a.codebook = static_cast<const uint16_t*>(codebooks);
+  a.y = y;
+  a.xch = static_cast<unsigned long long*>(workspace);
+  a.status = dev_status;
+  a.signs = nullptr;
+  a.types = types;
+  a.N = N;
+  a.K = K;
+  a.G = K / kGroup;
+  a.U = (N / kStrip) * a.G;
+  a.C = 0;
+  if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
+  return bits == 4 ? launch_bits<4, true>(a, int(M), num_sms, stream)
+                   : launch_bits<3, true>(a, int(M), num_sms, stream);
 }
 
 }  // namespace lutq

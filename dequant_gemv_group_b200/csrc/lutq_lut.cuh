@@ -35,34 +35,67 @@ __device__ __forceinline__ uint32_t lut_entry(const uint16_t* cb, int e, int hal
   return uint32_t(cb[qe]) | (uint32_t(cb[qo]) << 16);
 }
 
-// Fill the lane-duplicated table from a codebook held in registers: lane t of
-// every warp passes cbv = codebook[t mod 2^BITS], and each pair value is
-// assembled with two shuffles, so no shared staging or barrier comes before
-// the build (callers synchronize after it).  Thread i writes the 16-byte
-// chunks i, i + blockDim.x, ...; blockDim.x is a multiple of 32, so all lanes
-// of a warp take the same number of turns, as the shuffles require.
+// Fill the lane-duplicated table from codebooks held in registers: lane l of
+// every warp passes cbw = bytes 4l .. 4l+3 of the flattened codebook array
+// [types][2^BITS] (bf16 levels 2l and 2l+1, one warp-wide load for all
+// tables), and each pair value is assembled with two shuffles, so no shared
+// staging or barrier comes before the build (callers synchronize after it).
+// Thread i builds the value of half-row i (4-bit: row i; 3-bit: row i / 2,
+// half i % 2), then i + blockDim.x, ..., and stores it to the half-row's
+// eight 16-byte chunks, starting at chunk i mod 8 so that each eight
+// consecutive lanes cover all 32 banks.  blockDim.x is a multiple of 32, so
+// all lanes of a warp take the same number of turns, as the shuffles
+// require.
+//
+// w4_half (4-bit only): which half of each row the table goes to (0 = E, 1 =
+// O); a second 4-bit table can live in the half that 4-bit codes leave free.
 template <int BITS>
-__device__ __forceinline__ void build_lut_shfl(uint8_t* lut, uint32_t cbv) {
+__device__ __forceinline__ uint32_t level_of(uint32_t cbw, int t, uint32_t q) {
+  const uint32_t w = __shfl_sync(0xffffffffu, cbw, int((uint32_t(t) << (BITS - 1)) + (q >> 1)));
+  return (q & 1) ? (w >> 16) : (w & 0xffffu);
+}
+
+template <int BITS>
+__device__ __forceinline__ void lut_half_row(uint8_t* lut, uint32_t cbw, int t, int i,
+                                             int w4_half) {
   constexpr int HALVES = BITS == 4 ? 1 : 2;
-  constexpr int CHUNKS = 256 * HALVES * 8;  // 8 chunks of 16 bytes per half row
-  static_assert(CHUNKS % 32 == 0, "whole warps");
-  for (int c = threadIdx.x; c < CHUNKS; c += blockDim.x) {
-    const int e = c / (HALVES * 8), h = (c / 8) % HALVES;
-    uint32_t qe, qo;
-    if (BITS == 4) {
-      qe = e & 15;
-      qo = e >> 4;
-    } else if (h == 0) {
-      qe = (e & 3) | (((e >> 4) & 1) << 2);
-      qo = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
-    } else {
-      qe = ((e >> 4) & 3) | ((e & 1) << 2);
-      qo = ((e >> 6) & 3) | (((e >> 1) & 1) << 2);
-    }
-    const uint32_t ve = __shfl_sync(0xffffffffu, cbv, int(qe));
-    const uint32_t vo = __shfl_sync(0xffffffffu, cbv, int(qo));
-    const uint32_t v = (ve & 0xffffu) | (vo << 16);
-    reinterpret_cast<uint4*>(lut)[e * 16 + h * 8 + (c & 7)] = make_uint4(v, v, v, v);
+  const int e = i / HALVES, h = i % HALVES;
+  uint32_t qe, qo;
+  if (BITS == 4) {
+    qe = e & 15;
+    qo = e >> 4;
+  } else if (h == 0) {
+    qe = (e & 3) | (((e >> 4) & 1) << 2);
+    qo = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
+  } else {
+    qe = ((e >> 4) & 3) | ((e & 1) << 2);
+    qo = ((e >> 6) & 3) | (((e >> 1) & 1) << 2);
+  }
+  const uint32_t v = level_of<BITS>(cbw, t, qe) | (level_of<BITS>(cbw, t, qo) << 16);
+  const uint4 v4 = make_uint4(v, v, v, v);
+  uint4* half_row = reinterpret_cast<uint4*>(lut) + e * 16 + (h + w4_half) * 8;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) half_row[(j + i) & 7] = v4;
+}
+
+template <int BITS>
+__device__ __forceinline__ void build_lut_shfl(uint8_t* lut, uint32_t cbw) {
+  constexpr int VALUES = 256 * (BITS == 4 ? 1 : 2);
+  static_assert(VALUES % 32 == 0, "whole warps");
+  for (int i = threadIdx.x; i < VALUES; i += blockDim.x) lut_half_row<BITS>(lut, cbw, 0, i, 0);
+}
+
+// The tables of per-group data types, all threads sharing the work: table t
+// of 4-bit codes in row half t & 1 of the 64 KB at (t >> 1) << 16, table t of
+// 3-bit codes in the 64 KB at t << 16.  A warp's lanes always work on the
+// same table (its value count is a multiple of 32).
+template <int BITS>
+__device__ __forceinline__ void build_luts_typed(uint8_t* lut, uint32_t cbw, int types) {
+  constexpr int VALUES = 256 * (BITS == 4 ? 1 : 2);
+  for (int i = threadIdx.x; i < types * VALUES; i += blockDim.x) {
+    const int t = i / VALUES;
+    lut_half_row<BITS>(lut + ((BITS == 4 ? t >> 1 : t) << 16), cbw, t, i % VALUES,
+                       BITS == 4 ? (t & 1) : 0);
   }
 }
 

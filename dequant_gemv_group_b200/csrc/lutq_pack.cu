@@ -138,4 +138,43 @@ cudaError_t launch_pack(const uint8_t* codes, const void* scales, int64_t N, int
   return cudaGetLastError();
 }
 
+// The type blocks of a matrix with per-group data types (BitMoD abstract,
+// same listing): after the U scale blocks, 8 bytes per unit t = s * G + g;
+// byte rq holds the types of rows rq + 8 i (i = 0..3) of strip s, group g, in
+// bits 2i+1:2i.  One thread per byte.  A type >= max_types is reported
+// (LUTQ_ERR_CODE_RANGE) and stored modulo 4.
+__global__ void __launch_bounds__(256)
+pack_types_kernel(const uint8_t* __restrict__ types, int64_t G, int64_t bytes, int max_types,
+                  uint8_t* __restrict__ out, int32_t* dev_status) {
+  bool bad = false;
+  for (int64_t id = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; id < bytes;
+       id += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t t = id >> 3, rq = id & 7;
+    const int64_t s = t / G, g = t % G;
+    uint32_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t ty = types[(s * kStrip + rq + 8 * i) * G + g];
+      bad |= ty >= uint32_t(max_types);
+      v |= (ty & 3u) << (2 * i);
+    }
+    out[id] = uint8_t(v);
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) report(dev_status, LUTQ_ERR_CODE_RANGE);
+}
+
+cudaError_t launch_pack_types(const uint8_t* types, int64_t N, int64_t K, int bits, void* packed,
+                              int32_t* dev_status, int num_sms, cudaStream_t stream) {
+  const int64_t U = (N / kStrip) * (K / kGroup);
+  const int64_t bytes = U * kTypeBytes;
+  int64_t blocks = (bytes + 255) / 256;
+  const int64_t cap = int64_t(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  uint8_t* out = static_cast<uint8_t*>(packed) + U * (tile_bytes(bits) + kScaleBytes);
+  pack_types_kernel<<<unsigned(blocks), 256, 0, stream>>>(types, K / kGroup, bytes,
+                                                          max_types(bits), out, dev_status);
+  return cudaGetLastError();
+}
+
 }  // namespace lutq

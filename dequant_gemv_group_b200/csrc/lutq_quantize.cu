@@ -60,6 +60,129 @@ quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
   if (__any_sync(0xffffffffu, bad) && lane == 0) report(dev_status, LUTQ_ERR_NONFINITE);
 }
 
+// Per-group data types (BitMoD abstract, same listing: each group of 128
+// weights may be quantized with its own data type).  One thread per (row,
+// group): the absolute maximum, then for every type t the RTN codes and the
+// squared error E_t = sum over k = 0..127, in that order, of d * d in fp64,
+// d = fp32(v - c_t[q]) the RTN distance (each product exact, each addition
+// rounded once); the group takes the lowest t of smallest E_t and is written
+// with that type's codes.  codebooks: [types][2^BITS] bf16.
+template <int BITS>
+__global__ void __launch_bounds__(256)
+quantize_typed_kernel(const uint4* __restrict__ W, int64_t units,
+                      const uint16_t* __restrict__ codebooks, int types,
+                      uint2* __restrict__ codes, uint16_t* __restrict__ scales,
+                      uint8_t* __restrict__ group_types, int32_t* dev_status) {
+  constexpr int L = 1 << BITS;
+  constexpr int kMaxTypes = 4;
+  __shared__ float levels[kMaxTypes][L];
+  for (int i = threadIdx.x; i < types * L; i += blockDim.x)
+    levels[i / L][i % L] = __uint_as_float(uint32_t(codebooks[i]) << 16);
+  __syncthreads();
+
+  // the lowest index of smallest fp32 distance |v - c_i| (as quantize_kernel)
+  auto nearest = [&](float v, int t) -> uint32_t {
+    float best = INFINITY;
+    uint32_t bi = 0;
+#pragma unroll
+    for (int c = 0; c < L; ++c) {
+      const float d = fabsf(__fsub_rn(v, levels[t][c]));
+      if (d < best) {
+        best = d;
+        bi = c;
+      }
+    }
+    return bi;
+  };
+  auto values = [](const uint4& r, float (&w)[8]) {
+    const uint32_t x[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      w[2 * i] = bf16_lo_to_f32(x[i]);
+      w[2 * i + 1] = bf16_hi_to_f32(x[i]);
+    }
+  };
+
+  bool bad = false;
+  for (int64_t u = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u < units;
+       u += int64_t(gridDim.x) * blockDim.x) {
+    const uint4* src = W + u * (kGroup / 8);
+    float amax = 0.0f;
+    for (int j = 0; j < kGroup / 8; ++j) {
+      float w[8];
+      values(src[j], w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (!isfinite(w[i])) bad = true;
+        amax = fmaxf(amax, fabsf(w[i]));
+      }
+    }
+    double err[kMaxTypes] = {0.0, 0.0, 0.0, 0.0};
+    for (int j = 0; j < kGroup / 8; ++j) {
+      float w[8];
+      values(src[j], w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float v = amax > 0.0f ? __fdiv_rn(w[i], amax) : 0.0f;
+#pragma unroll
+        for (int t = 0; t < kMaxTypes; ++t) {
+          if (t >= types) break;
+          const double d = double(__fsub_rn(v, levels[t][nearest(v, t)]));
+          err[t] = __dadd_rn(err[t], __dmul_rn(d, d));
+        }
+      }
+    }
+    int pick = 0;
+    double best = err[0];
+#pragma unroll
+    for (int t = 1; t < kMaxTypes; ++t)
+      if (t < types && err[t] < best) {
+        best = err[t];
+        pick = t;
+      }
+    for (int j = 0; j < kGroup / 8; ++j) {
+      float w[8];
+      values(src[j], w);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float v = amax > 0.0f ? __fdiv_rn(w[i], amax) : 0.0f;
+        const uint32_t q = nearest(v, pick);
+        if (i < 4)
+          lo |= q << (8 * i);
+        else
+          hi |= q << (8 * (i - 4));
+      }
+      codes[u * (kGroup / 8) + j] = make_uint2(lo, hi);
+    }
+    scales[u] = uint16_t(__float_as_uint(amax) >> 16);
+    group_types[u] = uint8_t(pick);
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) report(dev_status, LUTQ_ERR_NONFINITE);
+}
+
+cudaError_t launch_quantize_typed(const void* W, int64_t N, int64_t K, const void* codebooks,
+                                  int types, int bits, uint8_t* codes, void* scales,
+                                  uint8_t* group_types, int32_t* dev_status, int num_sms,
+                                  cudaStream_t stream) {
+  const int64_t units = N * (K / kGroup);
+  int64_t blocks = (units + 255) / 256;
+  const int64_t cap = int64_t(num_sms) * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const uint4* w = static_cast<const uint4*>(W);
+  const uint16_t* cb = static_cast<const uint16_t*>(codebooks);
+  uint2* c = reinterpret_cast<uint2*>(codes);
+  uint16_t* s = static_cast<uint16_t*>(scales);
+  if (bits == 4)
+    quantize_typed_kernel<4><<<unsigned(blocks), 256, 0, stream>>>(w, units, cb, types, c, s,
+                                                                    group_types, dev_status);
+  else
+    quantize_typed_kernel<3><<<unsigned(blocks), 256, 0, stream>>>(w, units, cb, types, c, s,
+                                                                    group_types, dev_status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* codebook, int bits,
                             uint8_t* codes, void* scales, int32_t* dev_status, int num_sms,
                             cudaStream_t stream) {

@@ -348,6 +348,57 @@ lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
                       void* workspace, int64_t workspace_bytes,
                       int32_t* dev_status, void* stream);
 
+/*
+ * Per-group data types.
+ *
+ * Source: BitMoD abstract ("Daily Papers" listing, query "group-128"): each
+ * group of 128 weights may be quantized with its own numerical data type.
+ * Reading (the abstract gives neither the types nor the rule): a layer has T
+ * codebooks ("types"), T <= 4 with 4-bit codes and T <= 2 with 3-bit codes
+ * (lutq_max_types); every group keeps its absolute-maximum scale, and takes
+ * the type whose RTN codes give the smallest squared error
+ *   E_t = sum over k = 0, 1, ..., 127 in this order of d_k * d_k,
+ *   d_k = fp32(v_k - c_t[q_t[k]]),  v_k = fp32(w_k) / fp32(s),
+ * each product exact in fp64 and each addition rounded in fp64; ties go to
+ * the lowest type index.  The codes are that type's RTN codes.
+ *
+ * Packed layout with types: layout V2 (lutq_pack) followed by 8 bytes per
+ * unit u = strip * (K / 128) + group at byte U * (C + 64) + 8 u (U units, C
+ * code bytes per unit); byte rq (0..7) holds the types of rows rq + 8 i
+ * (i = 0..3) of the strip in bits 2i+1:2i.  lutq_packed_bytes_typed gives
+ * the size, U * (C + 72).
+ *
+ * codebooks_bf16  device bf16 [types][2^bits] (type t's levels at t * 2^bits).
+ * group_types     device uint8 [N, K/128] row-major.
+ *
+ * lutq_quantize_typed: as lutq_quantize, and writes group_types.  Returns
+ *   LUTQ_ERR_INVALID_ARG for types outside 1..lutq_max_types(bits).
+ * lutq_pack_typed: as lutq_pack into a buffer of lutq_packed_bytes_typed
+ *   bytes, then the type blocks; dev_status: LUTQ_ERR_CODE_RANGE for a code
+ *   >= 2^bits or a type >= lutq_max_types(bits) (stored modulo 4).
+ * lutq_gemv_typed: y[m, n] = sum_g s[n, g] * sum_{k in g} x[m, k] *
+ *   c_{type[n, g]}[q[n, k]], numerics as lutq_gemv.  Runs on the CUDA-core
+ *   kernel only, whose shared memory then holds a 128 KB table region:
+ *   M = 1..4 with M * (K + 2048) <= 48128, else LUTQ_ERR_SHAPE.  `types` must
+ *   be the count the matrix was quantized with: a stored type >= types reads
+ *   a table that is not filled (unspecified values, no out-of-bounds access).
+ *   Other arguments, workspace and errors as lutq_gemv.
+ * All three are asynchronous on `stream`; pointers 16-byte aligned.
+ */
+int lutq_max_types(int bits);
+int64_t lutq_packed_bytes_typed(int64_t N, int64_t K, int bits);
+lutq_status lutq_quantize_typed(const void* W_bf16, int64_t N, int64_t K,
+                                const void* codebooks_bf16, int types, int bits, uint8_t* codes,
+                                void* scales_bf16, uint8_t* group_types, int32_t* dev_status,
+                                void* stream);
+lutq_status lutq_pack_typed(const uint8_t* codes, const void* scales_bf16,
+                            const uint8_t* group_types, int64_t N, int64_t K, int bits,
+                            void* packed, int32_t* dev_status, void* stream);
+lutq_status lutq_gemv_typed(const void* x_bf16, int64_t M, const void* packed,
+                            const void* codebooks_bf16, int types, int bits, int64_t N, int64_t K,
+                            float* y, void* workspace, int64_t workspace_bytes,
+                            int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

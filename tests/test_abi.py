@@ -142,3 +142,43 @@ def test_gemv_rht_argument_errors(lq):
     assert call(m=5) == 2                  # beyond the CUDA-core kernel: rotate and use lutq_gemm
     assert call(m=1, k=128 * 700) == 2     # activations too long for its shared memory
     assert call(bits=5) == 3
+
+
+def test_typed_sizes_and_limits(lq):
+    assert lq.lutq_max_types(4) == O.MAX_TYPES[4] == 4
+    assert lq.lutq_max_types(3) == O.MAX_TYPES[3] == 2
+    assert lq.lutq_max_types(5) == -1
+    for n, k, bits in [(4096, 14336, 4), (4096, 4096, 3), (32, 128, 4)]:
+        assert lq.lutq_packed_bytes_typed(n, k, bits) == O.packed_bytes_typed(n, k, bits)
+    assert lq.lutq_packed_bytes_typed(33, 128, 4) == -1
+
+
+def test_typed_argument_errors(lq):
+    q = lq.lib.lutq_quantize_typed
+    assert q(A, 32, 128, A, 2, 4, A, A, None, None, None) == 1     # null types output
+    assert q(A, 32, 128, A, 0, 4, A, A, A, None, None) == 1        # no type
+    assert q(A, 32, 128, A, 5, 4, A, A, A, None, None) == 1        # 5 types of 4-bit codes
+    assert q(A, 32, 128, A, 3, 3, A, A, A, None, None) == 1        # 3 types of 3-bit codes
+    assert q(A, 32, 128, A, 2, 5, A, A, A, None, None) == 3        # bits
+    assert q(A, 33, 128, A, 2, 4, A, A, A, None, None) == 2        # N % 32
+    assert q(A, 32, 128, A, 2, 4, A, A, A + 4, None, None) == 4    # misaligned types
+    p = lq.lib.lutq_pack_typed
+    assert p(A, A, None, 32, 128, 4, A, None, None) == 1
+    assert p(A, A, A + 2, 32, 128, 4, A, None, None) == 4
+    assert p(A, A, A, 32, 100, 4, A, None, None) == 2
+    g = lq.lib.lutq_gemv_typed
+    ws = lq.lutq_workspace_bytes(1, 64, 256, 4)
+
+    def call(**kw):
+        a = dict(dict(x=A, m=1, p=A, c=A, t=2, bits=4, n=64, k=256, y=A, ws=A, wsb=ws), **kw)
+        return g(a["x"], a["m"], a["p"], a["c"], a["t"], a["bits"], a["n"], a["k"], a["y"],
+                 a["ws"], a["wsb"], None, None)
+
+    assert call(t=0) == 1
+    assert call(t=5) == 1
+    assert call(bits=3, t=3) == 1
+    assert call(m=5) == 2                      # only the CUDA-core kernel
+    assert call(m=1, k=128 * 361) == 2         # 1 * (46208 + 2048) > 48128
+    assert call(m=2, k=128 * 180) == 2         # 2 * (23040 + 2048) > 48128
+    assert call(c=A + 8) == 4
+    assert call(x=None) == 1

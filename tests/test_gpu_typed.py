@@ -1,0 +1,170 @@
+"""Per-group data types on the GPU against the oracle (through the C ABI):
+codes, scales, group types and packed bytes bit for bit; the typed product
+within the 2e-3 gate of the oracle's typed product, bit for bit on one-hot
+activations, and bit for bit equal to lutq_gemv when every group has the
+same single type."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import lutq_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+KINDS4 = ("nf4", "logb", "uniform4")
+
+
+@pytest.fixture(scope="module")
+def lq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import dequant_gemv_group_b200 as m
+    return m
+
+
+def _f32(t):
+    return t.float().cpu().numpy()
+
+
+def _bits16(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _tables(lq, bits, t):
+    """Device codebooks [t, 2^bits] and the oracle's level lists."""
+    if bits == 4:
+        kinds = (KINDS4 + ("nf4",))[:t]
+        cbs = [lq.lutq_codebook(k, 4) for k in kinds]
+        levels = [O.codebook(k, 4)[1] for k in kinds]
+        if t == 4:
+            # a fourth type: NF4 levels shrunk by 0.75 except the two ends
+            lv = O.bf16_round(levels[0].astype(np.float64) * 0.75).astype(np.float32)
+            lv[0], lv[-1] = -1.0, 1.0
+            levels[3] = lv
+            cbs[3] = torch.from_numpy(O.bf16_bits(lv).view(np.int16)).view(torch.bfloat16)
+    else:
+        lm = O.codebook("lloyd_max3", 3)[1]
+        levels = [lm]
+        if t == 2:
+            lv = O.bf16_round(lm.astype(np.float64) * 0.9).astype(np.float32)
+            lv[0], lv[-1] = -1.0, 1.0
+            levels.append(lv)
+        cbs = [torch.from_numpy(O.bf16_bits(l).view(np.int16)).view(torch.bfloat16) for l in levels]
+    return torch.stack(cbs).contiguous().cuda(), levels
+
+
+def _typed_layer(lq, w_cpu, bits, t):
+    cbs, levels = _tables(lq, bits, t)
+    st = lq.new_status()
+    codes, scales, types = lq.lutq_quantize_typed(w_cpu.cuda(), cbs, bits, status=st)
+    packed = lq.lutq_pack_typed(codes, scales, types, bits, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return cbs, levels, codes, scales, types, packed
+
+
+CASES = [(4, 1), (4, 2), (4, 3), (4, 4), (3, 1), (3, 2)]
+
+
+@pytest.mark.parametrize("bits,t", CASES)
+@pytest.mark.parametrize("n,k", [(96, 1152), (1024, 4096)])
+def test_quantize_and_pack_typed_bit_exact(lq, bits, t, n, k):
+    w = workloads.normal_weights(n, k, 0.02, seed=n + t, outlier_frac=1e-2)
+    w[5, 128:256] = 0.0                               # an all-zero group
+    w[7, :128] = w[7, :128] * 2.0 ** -120             # subnormal-scaled group
+    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    rc, rs, rt = O.quantize_typed(_f32(w), levels, bits)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+    np.testing.assert_array_equal(_bits16(scales), rs)
+    np.testing.assert_array_equal(types.cpu().numpy(), rt)
+    if t > 1:
+        assert len(np.unique(rt)) > 1                 # the case exercises the choice
+    np.testing.assert_array_equal(packed.cpu().numpy(), O.pack_typed(rc, rs, rt, bits))
+
+
+@pytest.mark.parametrize("bits,t", CASES)
+@pytest.mark.parametrize("m", [1, 2, 3, 4])
+@pytest.mark.parametrize("n,k", [(96, 1152), (1024, 4096), (320, 4224)])
+def test_gemv_typed_matches_oracle(lq, bits, t, m, n, k):
+    w = workloads.normal_weights(n, k, 0.02, seed=3 * n + t, outlier_frac=1e-2)
+    x = workloads.activations(m, k, seed=m + 7)
+    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    st = lq.new_status()
+    y = lq.lutq_gemv_typed(x.cuda(), packed, cbs, bits, n, k,
+                           workspace=lq.new_workspace(m, n, k, bits), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
+                         levels)
+    assert O.rel_error_gate(y.cpu().numpy(), y_ref) <= TOL
+
+
+@pytest.mark.parametrize("bits,t", [(4, 4), (3, 2)])
+def test_gemv_typed_one_hot_is_the_dequantized_weight(lq, bits, t):
+    n, k = 256, 1024
+    w = workloads.normal_weights(n, k, 0.02, seed=41, outlier_frac=1e-2)
+    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    wh = O.dequant_typed(codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(), levels)
+    ws = lq.new_workspace(1, n, k, bits)
+    for kk in (0, 129, 1023):
+        e = torch.zeros((1, k), dtype=torch.bfloat16)
+        e[0, kk] = 1.0
+        y = lq.lutq_gemv_typed(e.cuda(), packed, cbs, bits, n, k, workspace=ws)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(y.cpu().numpy()[0].astype(np.float64), wh[:, kk])
+
+
+@pytest.mark.parametrize("bits,kind", [(4, "nf4"), (3, "lloyd_max3")])
+@pytest.mark.parametrize("m", [1, 3])
+def test_single_type_equals_lutq_gemv_bitwise(lq, bits, kind, m):
+    n, k = 1024, 4096
+    w = workloads.normal_weights(n, k, 0.02, seed=43, outlier_frac=1e-3)
+    x = workloads.activations(m, k, seed=44).cuda()
+    cb = lq.lutq_codebook(kind, bits).cuda()
+    codes, scales, types = lq.lutq_quantize_typed(w.cuda(), cb[None].contiguous(), bits)
+    c0, s0 = lq.lutq_quantize(w.cuda(), cb, bits)
+    torch.cuda.synchronize()
+    assert torch.equal(codes, c0) and torch.equal(scales, s0) and not types.any()
+    ws = lq.new_workspace(m, n, k, bits)
+    y_t = lq.lutq_gemv_typed(x, lq.lutq_pack_typed(codes, scales, types, bits),
+                             cb[None].contiguous(), bits, n, k, workspace=ws)
+    y_u = lq.lutq_gemv(x, lq.lutq_pack(c0, s0, bits), cb, bits, n, k, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y_t, y_u)
+
+
+def test_pack_typed_reports_out_of_range_types(lq):
+    n, k = 64, 256
+    codes = torch.zeros((n, k), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((n, 2), dtype=torch.bfloat16, device="cuda")
+    types = torch.zeros((n, 2), dtype=torch.uint8, device="cuda")
+    types[9, 1] = 2                                   # 3-bit codes allow types 0 and 1
+    st = lq.new_status()
+    lq.lutq_pack_typed(codes, scales, types, 3, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 6                        # LUTQ_ERR_CODE_RANGE
+    st.zero_()
+    lq.lutq_pack_typed(codes, scales, types, 4, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+
+
+def test_gemv_typed_full_size_layer(lq):
+    lay = workloads.layer("llama3_8b_w4_nf4", "down")
+    n, k = lay.n, lay.k
+    w = lay.weights(seed=0)
+    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, 4, 4)
+    x = workloads.activations(1, k, seed=1)
+    y = lq.lutq_gemv_typed(x.cuda(), packed, cbs, 4, n, k, workspace=lq.new_workspace(1, n, k, 4))
+    torch.cuda.synchronize()
+    strips = [0, 63, 127]
+    rows = np.concatenate([np.arange(32 * s, 32 * s + 32) for s in strips])
+    rc, rs, rt = O.quantize_typed(_f32(w[rows]), levels, 4)
+    np.testing.assert_array_equal(codes[rows].cpu().numpy(), rc)
+    np.testing.assert_array_equal(types[rows].cpu().numpy(), rt)
+    y_ref = O.gemv_typed(_f32(x), rc, rs, rt, levels)
+    assert O.rel_error_gate(y.cpu().numpy()[:, rows], y_ref) <= TOL
+    # every type is used on this layer
+    assert set(np.unique(types.cpu().numpy()).tolist()) == {0, 1, 2, 3}
