@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     lutq_fit_codebook,
     lutq_fit_histogram,
     lutq_gemm,
+    lutq_gemm_typed,
     lutq_gemv,
     lutq_gemv_noalloc,
     lutq_gemv_plan,

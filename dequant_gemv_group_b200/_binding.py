@@ -56,6 +56,8 @@ _SIGS = {
     "lutq_pack_typed": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "lutq_gemv_typed": (_i32, [_vp, _i64, _vp, _vp, _i32, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
                                _vp]),
+    "lutq_gemm_typed": (_i32, [_vp, _i64, _vp, _vp, _i32, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
+                               _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -285,19 +287,29 @@ def lutq_pack_typed(codes: torch.Tensor, scales: torch.Tensor, types: torch.Tens
     return packed
 
 
-def lutq_gemv_typed(x, packed, codebooks, bits, n, k, y=None, workspace=None, status=None):
-    """y[M, N] (fp32) with per-group types, codebooks bf16 [T, 2^bits]
-    (M = 1..4; see lutq_gemv_typed in include/lutq.h)."""
+def _typed_product(fn, where, x, packed, codebooks, bits, n, k, y, workspace, status):
     _need(x, torch.bfloat16, "x")
     _need(codebooks, torch.bfloat16, "codebooks")
     m = x.shape[0]
     if y is None:
         y = torch.empty((m, n), dtype=torch.float32, device=x.device)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
-    _check(lib.lutq_gemv_typed(x.data_ptr(), m, packed.data_ptr(), codebooks.data_ptr(),
-                               codebooks.shape[0], bits, n, k, y.data_ptr(), ws_ptr, ws_bytes,
-                               _ptr(status), _stream()), "lutq_gemv_typed")
+    _check(fn(x.data_ptr(), m, packed.data_ptr(), codebooks.data_ptr(), codebooks.shape[0], bits,
+              n, k, y.data_ptr(), ws_ptr, ws_bytes, _ptr(status), _stream()), where)
     return y
+
+
+def lutq_gemv_typed(x, packed, codebooks, bits, n, k, y=None, workspace=None, status=None):
+    """y[M, N] (fp32) with per-group types, codebooks bf16 [T, 2^bits]
+    (M = 1..16; see lutq_gemv_typed in include/lutq.h)."""
+    return _typed_product(lib.lutq_gemv_typed, "lutq_gemv_typed", x, packed, codebooks, bits,
+                          n, k, y, workspace, status)
+
+
+def lutq_gemm_typed(x, packed, codebooks, bits, n, k, y=None, workspace=None, status=None):
+    """The typed product on the tensor cores (any M >= 1)."""
+    return _typed_product(lib.lutq_gemm_typed, "lutq_gemm_typed", x, packed, codebooks, bits,
+                          n, k, y, workspace, status)
 
 
 HIST_BINS = 16384

@@ -19,13 +19,13 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
                         int32_t* dev_status, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream);
+                        int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0);
 cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const void* codebook,
                             const int8_t* signs, int bits, int64_t N, int64_t K, float* y,
                             void* workspace, int32_t* dev_status, int num_sms,
                             cudaStream_t stream);
 bool gemv_small_path(int64_t M, int64_t K, int bits);
-bool gemv_typed_path(int64_t M, int64_t K);
+bool gemv_typed_path(int64_t M, int64_t K, int bits, int types);
 cudaError_t launch_quantize_typed(const void* W, int64_t N, int64_t K, const void* codebooks,
                                   int types, int bits, uint8_t* codes, void* scales,
                                   uint8_t* group_types, int32_t* dev_status, int num_sms,
@@ -309,12 +309,26 @@ lutq_status lutq_gemv_typed(const void* x_bf16, int64_t M, const void* packed,
                                       lutq_workspace_bytes(M, N, K, bits));
   if (st != LUTQ_OK) return st;
   if (types < 1 || types > lutq::max_types(bits)) return LUTQ_ERR_INVALID_ARG;
-  if (!lutq::gemv_typed_path(M, K)) return LUTQ_ERR_SHAPE;
   int sms = 0;
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_gemv_typed(x_bf16, M, packed, codebooks_bf16, types, bits, N, K,
                                            y, workspace, dev_status, sms,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_gemm_typed(const void* x_bf16, int64_t M, const void* packed,
+                            const void* codebooks_bf16, int types, int bits, int64_t N, int64_t K,
+                            float* y, void* workspace, int64_t workspace_bytes,
+                            int32_t* dev_status, void* stream) {
+  lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, codebooks_bf16, bits,
+                                      N, K, y, workspace, workspace_bytes,
+                                      lutq_workspace_bytes(M, N, K, bits));
+  if (st != LUTQ_OK) return st;
+  if (types < 1 || types > lutq::max_types(bits)) return LUTQ_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_gemm(x_bf16, M, packed, codebooks_bf16, bits, N, K, y, workspace,
+                                     dev_status, sms, static_cast<cudaStream_t>(stream), types));
 }
 
 }  // extern "C"

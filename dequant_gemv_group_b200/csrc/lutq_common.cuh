@@ -26,6 +26,16 @@ __host__ __device__ constexpr int words_per_row(int bits) { return bits == 4 ? 4
 constexpr int kTypeBytes = 8;
 __host__ __device__ constexpr int max_types(int bits) { return bits == 4 ? 4 : 2; }
 
+// Bytes of the lookup-table region in shared memory: one 64 KB region of 256
+// rows of 256 bytes (4-bit codes use the first half of each row, 3-bit codes
+// both halves).  With per-group data types table t of 4-bit codes takes row
+// half t & 1 of the region (t >> 1), table t of 3-bit codes region t; so one
+// region holds up to two 4-bit tables or one 3-bit table, otherwise two
+// regions are needed.  types = 0 means a single codebook.
+__host__ __device__ constexpr int table_region_bytes(int bits, int types) {
+  return types <= (bits == 4 ? 2 : 1) ? 0x10000 : 0x20000;
+}
+
 // Record a device-side error: the first non-zero code wins.
 __device__ __forceinline__ void report(int32_t* dev_status, int code) {
   if (dev_status != nullptr) atomicCAS(dev_status, 0, code);

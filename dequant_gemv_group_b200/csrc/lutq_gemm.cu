@@ -71,7 +71,10 @@ constexpr int kScaleRingBytes = 4 * kMaxPromoteGroups * 4 * 32 * 4;  // [warp][S
 struct GemmArgs {
   const uint8_t* packed;
   const uint8_t* scales;    // the packed matrix's scale blocks (layout V2)
-  const uint16_t* codebook;
+  const uint8_t* types;     // per-group data types: the type blocks (else unused)
+  const uint16_t* codebook; // [types][2^BITS] with per-group types
+  int ntypes;               // tables in `codebook` (1 without per-group types)
+  int lut_bytes;            // the table region (table_region_bytes)
   float* y;
   float* part;        // [kGemmMaxCtas][2][4][NT][32]: (CTA, slot, strip, column, row)
   int* counters;      // [BT * NTILES * 4 * kMaxPromoteGroups]
@@ -207,7 +210,7 @@ __device__ __forceinline__ void tmem_st_cols32(uint32_t taddr, const uint32_t (&
       : "memory");
 }
 
-template <int BITS, int NT>
+template <int BITS, int NT, bool TYPED>
 __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, GemmArgs a) {
   using Cfg = GemmCfg<NT>;
@@ -223,7 +226,12 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   uint8_t* base = smem_raw + (base_sa - raw_sa);
   uint8_t* lut = base;
   const uint32_t lut_sa = base_sa;
-  const uint32_t xst_sa = base_sa + kLutBytes;
+  // the table region: 64 KB, or 128 KB for per-group data types that need
+  // it (table t of 4-bit codes in row half t & 1 of the 64 KB at (t >> 1)
+  // << 16, table t of 3-bit codes in the 64 KB at t << 16, as in the
+  // CUDA-core kernel)
+  const int LUTB = TYPED ? a.lut_bytes : kLutBytes;
+  const uint32_t xst_sa = base_sa + uint32_t(LUTB);
   const uint32_t bar_sa = xst_sa + XS * Cfg::XSTAGE;
   // barrier ids
   constexpr int B_XF = 0, B_XE = XS, B_AF = 2 * XS, B_AE = B_AF + AS, B_DF = B_AE + AS,
@@ -251,15 +259,21 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (threadIdx.x < (1 << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
+  if (threadIdx.x < (a.ntypes << BITS)) cbs[threadIdx.x] = a.codebook[threadIdx.x];
   if (warp == W_MMA) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < kLutBytes / 16; c += blockDim.x) {
-    const uint32_t v = lut_entry<BITS>(cbs, c >> 4, (c >> 3) & 1);
-    reinterpret_cast<uint4*>(lut)[c] = make_uint4(v, v, v, v);
+  for (int c = threadIdx.x; c < LUTB / 16; c += blockDim.x) {
+    // 16-byte chunk c: row e = (c >> 4) & 255, half (c >> 3) & 1 of the
+    // 64 KB region c >> 12; without types one table (4-bit codes: both halves)
+    const int half = (c >> 3) & 1, region = c >> 12;
+    const int t = TYPED ? (BITS == 4 ? 2 * region + half : region) : 0;
+    if (t < a.ntypes) {
+      const uint32_t v = lut_entry<BITS>(cbs + (t << BITS), (c >> 4) & 255, half);
+      reinterpret_cast<uint4*>(lut)[c] = make_uint4(v, v, v, v);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -286,34 +300,57 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     UnitPos fp;  // the next unit to fetch
     fp.init(u0, per_bt, a.G);
     int fetched = 0;
-    auto fetch = [&](uint4 (&wd)[NWL]) {
+    // per-group types: the lane's row is lane (rq = lane & 7, i = lane >> 3)
+    // of its strip; its type is bits 2i+1:2i of byte rq of the unit's block
+    auto fetch = [&](uint4 (&wd)[NWL], uint32_t& ty) {
       if (fetched < n && fp.tau * kTileRows + sw * 32 < a.N) {
-        const uint8_t* t = a.packed + ((fp.tau * 4 + sw) * a.G + fp.g) * TB + lane * 16;
+        const int64_t tile = (fp.tau * 4 + sw) * a.G + fp.g;
+        const uint8_t* t = a.packed + tile * TB + lane * 16;
 #pragma unroll
         for (int j = 0; j < NWL; ++j) wd[j] = ld_stream_v4(t + word_of(j) * 512);
+        if (TYPED)  // issued here, with the unit's words (a plain load may sink to its use)
+          asm volatile("ld.global.nc.u8 %0, [%1];"
+                       : "=r"(ty) : "l"(a.types + tile * kTypeBytes + (lane & 7)));
       }
       ++fetched;
       fp.next(a.G, a.ntiles);
     };
     uint4 ring[NB][NWL];
+    uint32_t tyring[NB];
 #pragma unroll
-    for (int t = 0; t < NB; ++t) fetch(ring[t]);
+    for (int t = 0; t < NB; ++t) {
+      tyring[t] = 0;
+      fetch(ring[t], tyring[t]);
+    }
     UnitPos pos;
     pos.init(u0, per_bt, a.G);
     bool ok = true;
     // decode unit i from wd, refill wd with unit i + NB, hand the tile to the MMA
-    auto step = [&](uint4 (&wd)[NWL], int i) {
+    auto step = [&](uint4 (&wd)[NWL], uint32_t& ty, int i) {
       const bool valid = pos.tau * kTileRows + sw * 32 < a.N;
       uint32_t av[Cfg::KC];
       if (valid) {
+        // the row's table: 4-bit, type bit 0 -> address bit 7 (row half),
+        // bit 1 -> bit 16; 3-bit, type bit 0 -> bit 16 (through byte 1 of
+        // the column word)
+        // (masked to the table region, so that a type >= ntypes reads an
+        // unfilled table inside it, never the activation stages)
+        uint32_t sel = 0;
+        if (TYPED) {
+          const uint32_t f = (ty >> (2 * (lane >> 3))) & 3u;
+          sel = (BITS == 4 ? ((f & 1u) << 7) | ((f >> 1) << 8) : (f & 1u) << 8) &
+                ((BITS == 4 ? 0x080u : 0u) | (LUTB > kLutBytes ? 0x100u : 0u));
+        }
         if (DW == 8)
           decode_group_half<BITS>(reinterpret_cast<uint32_t(&)[32]>(av),
-                                  reinterpret_cast<const uint4(&)[2]>(wd), kh, lut_sa, off_e, off_o);
+                                  reinterpret_cast<const uint4(&)[2]>(wd), kh, lut_sa,
+                                  off_e | sel, off_o | sel);
         else
           decode_group_row<BITS>(reinterpret_cast<uint32_t(&)[64]>(av),
-                                 reinterpret_cast<const uint4(&)[4]>(wd), lut_sa, off_e, off_o);
+                                 reinterpret_cast<const uint4(&)[4]>(wd), lut_sa, off_e | sel,
+                                 off_o | sel);
       }
-      fetch(wd);
+      fetch(wd, ty);
       const int as = i % AS;
       ok = mbar_wait(bar(B_AE + as), (uint32_t(i / AS) & 1u) ^ 1u, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -338,7 +375,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
 #pragma unroll
       for (int t = 0; t < NB; ++t) {
         if (i + t >= n || !ok) break;
-        step(ring[t], i + t);
+        step(ring[t], tyring[t], i + t);
       }
     }
   } else if (warp < W_XLOAD) {
@@ -529,32 +566,45 @@ static cudaError_t make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BITS, int NT>
+template <int BITS, int NT, bool TYPED>
 static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
                              cudaStream_t stream) {
   using Cfg = GemmCfg<NT>;
   static int granted[64] = {0};
   // alignment slack, table, activation stages, barriers and flags (512),
   // the promotion warps' scale rings
-  const int smem = 1024 + kLutBytes + Cfg::XS * Cfg::XSTAGE + 512 + kScaleRingBytes;
+  const int smem = 1024 + a.lut_bytes + Cfg::XS * Cfg::XSTAGE + 512 + kScaleRingBytes;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (granted[dev] < smem) {
-    err = cudaFuncSetAttribute(gemm_kernel<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               smem);
+    err = cudaFuncSetAttribute(gemm_kernel<BITS, NT, TYPED>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     granted[dev] = smem;
   }
   a.C = int(std::min<int64_t>(std::min<int64_t>(num_sms, kGemmMaxCtas), a.U));
-  gemm_kernel<BITS, NT><<<unsigned(a.C), Cfg::THREADS, smem, stream>>>(map, a);
+  gemm_kernel<BITS, NT, TYPED><<<unsigned(a.C), Cfg::THREADS, smem, stream>>>(map, a);
   return cudaGetLastError();
 }
 
+template <int BITS, bool TYPED>
+static cudaError_t launch_nts(int nt, const CUtensorMap& map, const GemmArgs& a, int num_sms,
+                              cudaStream_t stream) {
+  switch (nt) {
+    case 16: return launch_nt<BITS, 16, TYPED>(map, a, num_sms, stream);
+    case 32: return launch_nt<BITS, 32, TYPED>(map, a, num_sms, stream);
+    case 64: return launch_nt<BITS, 64, TYPED>(map, a, num_sms, stream);
+    default: return launch_nt<BITS, 128, TYPED>(map, a, num_sms, stream);
+  }
+}
+
+// types = 0: one codebook; 1..max_types(bits): per-group data types (the
+// packed matrix carries its type blocks and `codebook` holds `types` tables).
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream) {
+                        int32_t* dev_status, int num_sms, cudaStream_t stream, int types) {
   const int nt = gemm_nt(M);
   CUtensorMap map;
   std::memset(&map, 0, sizeof(map));
@@ -563,7 +613,10 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
   GemmArgs a;
   a.packed = static_cast<const uint8_t*>(packed);
   a.scales = a.packed + (N / kStrip) * (K / kGroup) * tile_bytes(bits);
+  a.types = a.scales + (N / kStrip) * (K / kGroup) * kScaleBytes;
   a.codebook = static_cast<const uint16_t*>(codebook);
+  a.ntypes = types > 0 ? types : 1;
+  a.lut_bytes = table_region_bytes(bits, types);
   a.y = y;
   a.dev_status = dev_status;
   a.N = N;
@@ -578,20 +631,11 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
   a.counters = static_cast<int*>(workspace);
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + counters);
   a.C = 0;
-  if (bits == 4) {
-    switch (nt) {
-      case 16: return launch_nt<4, 16>(map, a, num_sms, stream);
-      case 32: return launch_nt<4, 32>(map, a, num_sms, stream);
-      case 64: return launch_nt<4, 64>(map, a, num_sms, stream);
-      default: return launch_nt<4, 128>(map, a, num_sms, stream);
-    }
-  }
-  switch (nt) {
-    case 16: return launch_nt<3, 16>(map, a, num_sms, stream);
-    case 32: return launch_nt<3, 32>(map, a, num_sms, stream);
-    case 64: return launch_nt<3, 64>(map, a, num_sms, stream);
-    default: return launch_nt<3, 128>(map, a, num_sms, stream);
-  }
+  if (types > 0)
+    return bits == 4 ? launch_nts<4, true>(nt, map, a, num_sms, stream)
+                     : launch_nts<3, true>(nt, map, a, num_sms, stream);
+  return bits == 4 ? launch_nts<4, false>(nt, map, a, num_sms, stream)
+                   : launch_nts<3, false>(nt, map, a, num_sms, stream);
 }
 
 }  // namespace lutq

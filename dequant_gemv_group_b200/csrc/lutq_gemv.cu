@@ -240,31 +240,31 @@ __device__ void cta_finish(const GemvArgs& a, const Span& p, const float* all_sl
 // Shared-window layout of the small-batch kernel, in addresses of the CTA's
 // shared window (the block's own static shared memory and the system's
 // reserved bytes lie below kSbaseMax, where dynamic shared memory begins):
-//   [kLutAt, kXAt)                 the lookup table, 256 rows of 256 bytes
-//   [kXAt, slots_at(K, M))         activations, bf16 in order, batch row by
+//   [kLutAt, xat)                  the lookup tables: 64 KB (256 rows of 256
+//                                  bytes) or, for per-group data types that
+//                                  need it, 128 KB (table_region_bytes)
+//   [xat, slots_at(K, M, L))       activations, bf16 in order, batch row by
 //                                  batch row: a group's four chunks of 32
 //                                  values (64 bytes each) are contiguous
-//   [slots_at(K, M), small_end)    warp slots, [NW][2][M][32] fp32
-// The dynamic size small_end(K, M) therefore covers the window up to the end
-// of the slots whatever the exact start (<= kSbaseMax).  A table address is
-// formed as (row << 8 | column); kLutAt goes into the load's offset.
+//   [slots_at(K, M, L), small_end) warp slots, [NW][2][M][32] fp32
+// with xat = kLutAt + L, L the table bytes.  The dynamic size small_end
+// therefore covers the window up to the end of the slots whatever the exact
+// start (<= kSbaseMax).  A table address is formed as (table << 16 | row << 8
+// | column); kLutAt goes into the load's offset.
 constexpr uint32_t kSbaseMax = 4096;
 constexpr uint32_t kLutAt = kSbaseMax;
 constexpr uint32_t kXChunkBytes = 64;
 constexpr uint32_t kXGroupBytes = 4 * kXChunkBytes;
 
-// With per-group data types the table region is 128 KB: table t of 4-bit
-// codes in row half t & 1 of the 64 KB at (t >> 1) << 16, table t of 3-bit
-// codes (both halves) in the 64 KB at t << 16.  The address bits 23:16 come
-// from bits 15:8 of the lane's column word.
-__host__ __device__ constexpr uint32_t x_at(bool typed) {
-  return kLutAt + (typed ? 0x20000u : 0x10000u);
+// With per-group data types, table t of 4-bit codes sits in row half t & 1
+// of the 64 KB at (t >> 1) << 16, table t of 3-bit codes (both halves) in the
+// 64 KB at t << 16; the address bits 23:16 come from bits 15:8 of the lane's
+// column word.
+__host__ __device__ constexpr uint32_t slots_at(uint32_t K, int M, uint32_t lut_bytes) {
+  return kLutAt + lut_bytes + uint32_t(M) * K * 2u;  // K * 2 is a multiple of 256
 }
-__host__ __device__ constexpr uint32_t slots_at(uint32_t K, int M, bool typed) {
-  return x_at(typed) + uint32_t(M) * K * 2u;  // K * 2 is a multiple of 256
-}
-__host__ __device__ constexpr uint32_t small_end(uint32_t K, int M, bool typed) {
-  return slots_at(K, M, typed) + uint32_t(kM1Warps * 2 * M * kStrip * 4);
+__host__ __device__ constexpr uint32_t small_end(uint32_t K, int M, uint32_t lut_bytes) {
+  return slots_at(K, M, lut_bytes) + uint32_t(kM1Warps * 2 * M * kStrip * 4);
 }
 
 // The table entry (a bf16x2 pair of levels) at table address t.
@@ -469,11 +469,19 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-template <int BITS, int M, int NB, bool TYPED>
+// TREG: 0 without per-group data types; 1 or 2 with them, the table region
+// being TREG x 64 KB (table_region_bytes).
+template <int BITS, int M, int NB, int TREG>
 __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a) {
+  constexpr bool TYPED = TREG > 0;
   constexpr int TB = tile_bytes(BITS);
   constexpr int UB = TB + kScaleBytes + (TYPED ? kTypeBytes : 0);  // packed bytes per unit
-  constexpr uint32_t kXAt = x_at(TYPED);
+  constexpr uint32_t kLutRegion = TREG == 2 ? 0x20000u : 0x10000u;
+  constexpr uint32_t kXAt = kLutAt + kLutRegion;
+  // Table-select bits a lookup may use: with one 64 KB region only the row
+  // half (4-bit codes), so every address stays inside the tables whatever
+  // type a group stores (a type >= types reads an unfilled table).
+  constexpr uint32_t sel_mask = (BITS == 4 ? 0x080u : 0u) | (TREG == 2 ? 0x100u : 0u);
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ WarpTable<kM1Warps> wt;
   const uint32_t sbase = sm_addr(smem);
@@ -640,7 +648,8 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 
   const uint32_t lane_e = uint32_t(lane) * 4u, lane_o = 128u + uint32_t(lane) * 4u;
   const uint32_t hi_shift = BITS == 3 ? 2u * uint32_t(q >> 1) : 0u;
-  float* const slots = reinterpret_cast<float*>(smem + (slots_at(K, M, TYPED) - sbase));
+  float* const slots = reinterpret_cast<float*>(
+      smem + (slots_at(K, M, kLutRegion) - sbase));
   float* const my_slots = slots + wl * 2 * M * kStrip;
   int rows[4];
 #pragma unroll
@@ -671,7 +680,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
       for (int i = 0; i < 4; ++i) {
         uint32_t sel = 0;
         if (TYPED)
-          sel = BITS == 4 ? ((ty << 7) >> (2 * i)) & 0x180u : ((ty << 8) >> (2 * i)) & 0x100u;
+          sel = (BITS == 4 ? (ty << 7) >> (2 * i) : (ty << 8) >> (2 * i)) & sel_mask;
         lce[i] = lane_e | sel;
         lco[i] = lane_o | sel;
       }
@@ -832,19 +841,21 @@ static void apply_plan(GemvArgs& a, int num_sms, int bits) {
 }
 
 
-static int64_t small_smem(int64_t K, int M, bool typed) {
-  return K < (int64_t(1) << 20) ? int64_t(small_end(uint32_t(K), M, typed)) : int64_t(1) << 30;
+static int64_t small_smem(int64_t K, int M, int lut_bytes) {
+  return K < (int64_t(1) << 20) ? int64_t(small_end(uint32_t(K), M, uint32_t(lut_bytes)))
+                                : int64_t(1) << 30;
 }
 
-template <int BITS, int M, bool TYPED>
+template <int BITS, int M, int TREG>
 static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
+  constexpr bool TYPED = TREG > 0;
   static SmemGrant grant2, grant3;
-  const int smem = int(small_smem(a.K, M, TYPED));
+  const int smem = int(small_smem(a.K, M, TREG == 2 ? 0x20000 : 0x10000));
   apply_plan(a, num_sms, BITS);
   constexpr int kDeep = M == 1 && !TYPED ? 3 : 2;
   const bool deep = M == 1 && !TYPED && a.pf_ctas == 0;
-  auto kernel = deep ? gemv_small_kernel<BITS, M, kDeep, TYPED>
-                     : gemv_small_kernel<BITS, M, 2, TYPED>;
+  auto kernel = deep ? gemv_small_kernel<BITS, M, kDeep, TREG>
+                     : gemv_small_kernel<BITS, M, 2, TREG>;
   cudaError_t err = grant_smem(kernel, deep ? grant3 : grant2, smem);
   if (err != cudaSuccess) return err;
   // programmatic dependent launch: the prefetching blocks and the work
@@ -864,7 +875,7 @@ static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
 
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream);
+                        int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0);
 
 // Batches up to kMaxSmallBatch run on the CUDA cores when their activations
 // fit the small-batch kernel's shared memory.  Larger batches are a dense
@@ -873,18 +884,18 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
 // so they, and over-long rows, take the tcgen05 kernel of lutq_gemm.
 constexpr int kMaxSmallBatch = 4;
 
-static bool small_fits(int64_t M, int64_t K, bool typed = false) {
+static bool small_fits(int64_t M, int64_t K, int lut_bytes = 0x10000) {
   return M >= 1 && M <= kMaxSmallBatch &&
-         small_smem(K, int(M), typed) <= kMaxSmemPerBlock - 1024;
+         small_smem(K, int(M), lut_bytes) <= kMaxSmemPerBlock - 1024;
 }
 
-template <int BITS, bool TYPED = false>
+template <int BITS, int TREG = 0>
 static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream_t s) {
   switch (M) {
-    case 1: return launch_small<BITS, 1, TYPED>(a, num_sms, s);
-    case 2: return launch_small<BITS, 2, TYPED>(a, num_sms, s);
-    case 3: return launch_small<BITS, 3, TYPED>(a, num_sms, s);
-    default: return launch_small<BITS, 4, TYPED>(a, num_sms, s);
+    case 1: return launch_small<BITS, 1, TREG>(a, num_sms, s);
+    case 2: return launch_small<BITS, 2, TREG>(a, num_sms, s);
+    case 3: return launch_small<BITS, 3, TREG>(a, num_sms, s);
+    default: return launch_small<BITS, 4, TREG>(a, num_sms, s);
   }
 }
 
@@ -920,9 +931,11 @@ bool gemv_small_path(int64_t M, int64_t K, int bits) {
   return small_fits(M, K);
 }
 
-// Whether lutq_gemv_typed can run an M x K product (the CUDA-core kernel with
-// the 128 KB table region).
-bool gemv_typed_path(int64_t M, int64_t K) { return small_fits(M, K, true); }
+// Whether lutq_gemv_typed runs an M x K product on the CUDA-core kernel (with
+// the table region that `types` tables need).
+bool gemv_typed_path(int64_t M, int64_t K, int bits, int types) {
+  return small_fits(M, K, table_region_bytes(bits, types));
+}
 
 // lutq_gemv with the activations rotated in the kernel's prologue; only for
 // the CUDA-core kernel (the caller checks gemv_small_path).
@@ -951,14 +964,16 @@ cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const 
 }
 
 // lutq_gemv with per-group data types: `codebooks` holds `types` tables of
-// 2^bits levels and `packed` the type blocks; only for the CUDA-core kernel
-// (the caller checks gemv_typed_path).
+// 2^bits levels and `packed` the type blocks.  The CUDA-core kernel (with its
+// 128 KB table region) where it fits, the tensor-core kernel otherwise.
 cudaError_t launch_gemv_typed(const void* x, int64_t M, const void* packed, const void* codebooks,
                               int types, int bits, int64_t N, int64_t K, float* y,
                               void* workspace, int32_t* dev_status, int num_sms,
                               cudaStream_t stream) {
-  if (!gemv_typed_path(M, K) || types < 1 || types > max_types(bits))
-    return cudaErrorInvalidValue;
+  if (types < 1 || types > max_types(bits)) return cudaErrorInvalidValue;
+  if (!gemv_typed_path(M, K, bits, types))
+    return launch_gemm(x, M, packed, codebooks, bits, N, K, y, workspace, dev_status, num_sms,
+                       stream, types);
   GemvArgs a;
   a.x = static_cast<const uint16_t*>(x);
   a.packed = static_cast<const uint8_t*>(packed);
@@ -974,8 +989,11 @@ cudaError_t launch_gemv_typed(const void* x, int64_t M, const void* packed, cons
   a.U = (N / kStrip) * a.G;
   a.C = 0;
   if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
-  return bits == 4 ? launch_bits<4, true>(a, int(M), num_sms, stream)
-                   : launch_bits<3, true>(a, int(M), num_sms, stream);
+  if (table_region_bytes(bits, types) > 0x10000)
+    return bits == 4 ? launch_bits<4, 2>(a, int(M), num_sms, stream)
+                     : launch_bits<3, 2>(a, int(M), num_sms, stream);
+  return bits == 4 ? launch_bits<4, 1>(a, int(M), num_sms, stream)
+                   : launch_bits<3, 1>(a, int(M), num_sms, stream);
 }
 
 }  // namespace lutq

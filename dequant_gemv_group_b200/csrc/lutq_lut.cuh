@@ -99,9 +99,11 @@ __device__ __forceinline__ void build_luts_typed(uint8_t* lut, uint32_t cbw, int
   }
 }
 
-// (byte `byte` of word) << 8 | lane_off, with lane_off < 256.
+// (byte 1 of lane_off) << 16 | (byte `byte` of word) << 8 | (byte 0 of
+// lane_off), with lane_off < 65536: byte 1 of lane_off selects a 64 KB table
+// (per-group data types), and is zero otherwise.
 __device__ __forceinline__ uint32_t lut_addr(uint32_t word, uint32_t lane_off, int byte) {
-  return __byte_perm(word, lane_off, 0x5504u | (uint32_t(byte) << 4));
+  return __byte_perm(word, lane_off, 0x6504u | (uint32_t(byte) << 4));
 }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t smem_addr) {

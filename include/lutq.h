@@ -377,13 +377,17 @@ lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
  *   bytes, then the type blocks; dev_status: LUTQ_ERR_CODE_RANGE for a code
  *   >= 2^bits or a type >= lutq_max_types(bits) (stored modulo 4).
  * lutq_gemv_typed: y[m, n] = sum_g s[n, g] * sum_{k in g} x[m, k] *
- *   c_{type[n, g]}[q[n, k]], numerics as lutq_gemv.  Runs on the CUDA-core
- *   kernel only, whose shared memory then holds a 128 KB table region:
- *   M = 1..4 with M * (K + 2048) <= 48128, else LUTQ_ERR_SHAPE.  `types` must
- *   be the count the matrix was quantized with: a stored type >= types reads
- *   a table that is not filled (unspecified values, no out-of-bounds access).
- *   Other arguments, workspace and errors as lutq_gemv.
- * All three are asynchronous on `stream`; pointers 16-byte aligned.
+ *   c_{type[n, g]}[q[n, k]], numerics as lutq_gemv, M = 1..16.  The tables
+ *   take 64 KB of shared memory for up to two 4-bit types or one 3-bit type,
+ *   128 KB otherwise; the CUDA-core kernel runs M = 1..4 with
+ *   M * (K + 2048) <= 80896 (64 KB of tables) or <= 48128 (128 KB), other
+ *   products go to the tensor-core kernel (as lutq_gemm_typed).  `types` must be the count the
+ *   matrix was quantized with: a stored type >= types reads a table that is
+ *   not filled (unspecified values, no out-of-bounds access).  Other
+ *   arguments, workspace and errors as lutq_gemv.
+ * lutq_gemm_typed: the same product on the tensor cores (any M >= 1), as
+ *   lutq_gemm.
+ * All are asynchronous on `stream`; pointers 16-byte aligned.
  */
 int lutq_max_types(int bits);
 int64_t lutq_packed_bytes_typed(int64_t N, int64_t K, int bits);
@@ -395,6 +399,10 @@ lutq_status lutq_pack_typed(const uint8_t* codes, const void* scales_bf16,
                             const uint8_t* group_types, int64_t N, int64_t K, int bits,
                             void* packed, int32_t* dev_status, void* stream);
 lutq_status lutq_gemv_typed(const void* x_bf16, int64_t M, const void* packed,
+                            const void* codebooks_bf16, int types, int bits, int64_t N, int64_t K,
+                            float* y, void* workspace, int64_t workspace_bytes,
+                            int32_t* dev_status, void* stream);
+lutq_status lutq_gemm_typed(const void* x_bf16, int64_t M, const void* packed,
                             const void* codebooks_bf16, int types, int bits, int64_t N, int64_t K,
                             float* y, void* workspace, int64_t workspace_bytes,
                             int32_t* dev_status, void* stream);

@@ -177,8 +177,11 @@ def test_typed_argument_errors(lq):
     assert call(t=0) == 1
     assert call(t=5) == 1
     assert call(bits=3, t=3) == 1
-    assert call(m=5) == 2                      # only the CUDA-core kernel
-    assert call(m=1, k=128 * 361) == 2         # 1 * (46208 + 2048) > 48128
-    assert call(m=2, k=128 * 180) == 2         # 2 * (23040 + 2048) > 48128
+    assert call(m=17) == 2                     # lutq_gemv's batch range
+    assert call(m=0) == 2
     assert call(c=A + 8) == 4
     assert call(x=None) == 1
+    gg = lq.lib.lutq_gemm_typed
+    assert gg(A, 1, A, A, 0, 4, 64, 256, A, A, ws, None, None) == 1
+    assert gg(A, 1, A, A, 3, 3, 64, 256, A, A, ws, None, None) == 1
+    assert gg(A, 1, A, A, 2, 4, 64, 200, A, A, ws, None, None) == 2

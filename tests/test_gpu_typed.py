@@ -168,3 +168,113 @@ def test_gemv_typed_full_size_layer(lq):
     assert O.rel_error_gate(y.cpu().numpy()[:, rows], y_ref) <= TOL
     # every type is used on this layer
     assert set(np.unique(types.cpu().numpy()).tolist()) == {0, 1, 2, 3}
+
+
+@pytest.mark.parametrize("bits,t", [(4, 4), (4, 2), (3, 2)])
+@pytest.mark.parametrize("m", [5, 16, 32, 64, 128])
+@pytest.mark.parametrize("n,k", [(256, 1024), (320, 4224)])
+def test_typed_tensor_core_path_matches_oracle(lq, bits, t, m, n, k):
+    # batches beyond the CUDA-core kernel: lutq_gemv_typed (M <= 16) and
+    # lutq_gemm_typed both run the tcgen05 kernel with the 128 KB table region
+    w = workloads.normal_weights(n, k, 0.02, seed=5 * n + t, outlier_frac=1e-2)
+    x = workloads.activations(m, k, seed=m + 11)
+    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
+                         levels)
+    ws = lq.new_workspace(m, n, k, bits)
+    st = lq.new_status()
+    fns = [lq.lutq_gemm_typed] + ([lq.lutq_gemv_typed] if m <= 16 else [])
+    for fn in fns:
+        y = fn(x.cuda(), packed, cbs, bits, n, k, workspace=ws, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert O.rel_error_gate(y.cpu().numpy(), y_ref) <= TOL, fn.__name__
+
+
+def test_typed_long_rows_take_the_tensor_core_path(lq):
+    # M = 1 with K beyond the CUDA-core kernel's shared memory (K + 2048 > 48128)
+    n, k, bits, t = 64, 128 * 380, 4, 4
+    w = workloads.normal_weights(n, k, 0.02, seed=61, outlier_frac=1e-2)
+    x = workloads.activations(1, k, seed=62)
+    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    st = lq.new_status()
+    y = lq.lutq_gemv_typed(x.cuda(), packed, cbs, bits, n, k,
+                           workspace=lq.new_workspace(1, n, k, bits), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
+                         levels)
+    assert O.rel_error_gate(y.cpu().numpy(), y_ref) <= TOL
+
+
+@pytest.mark.parametrize("bits,t", [(4, 4), (3, 2)])
+def test_typed_gemm_one_hot_is_the_dequantized_weight(lq, bits, t):
+    n, k, m = 256, 1024, 32
+    w = workloads.normal_weights(n, k, 0.02, seed=71, outlier_frac=1e-2)
+    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    wh = O.dequant_typed(codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(), levels)
+    x = torch.zeros((m, k), dtype=torch.bfloat16)
+    cols = (np.arange(m) * 37) % k
+    x[np.arange(m), cols] = 1.0
+    y = lq.lutq_gemm_typed(x.cuda(), packed, cbs, bits, n, k,
+                           workspace=lq.new_workspace(m, n, k, bits))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(y.cpu().numpy().astype(np.float64), wh[:, cols].T)
+
+
+def test_typed_gemm_single_type_equals_lutq_gemm_bitwise(lq):
+    n, k, m, bits = 512, 2048, 64, 4
+    w = workloads.normal_weights(n, k, 0.02, seed=73, outlier_frac=1e-3)
+    x = workloads.activations(m, k, seed=74).cuda()
+    cb = lq.lutq_codebook("nf4", bits).cuda()
+    codes, scales, types = lq.lutq_quantize_typed(w.cuda(), cb[None].contiguous(), bits)
+    ws = lq.new_workspace(m, n, k, bits)
+    y_t = lq.lutq_gemm_typed(x, lq.lutq_pack_typed(codes, scales, types, bits),
+                             cb[None].contiguous(), bits, n, k, workspace=ws)
+    y_u = lq.lutq_gemm(x, lq.lutq_pack(codes, scales, bits), cb, bits, n, k, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y_t, y_u)
+
+
+@pytest.mark.parametrize("t", [2, 4])
+def test_typed_route_by_table_region(lq, t):
+    # M = 4, K = 14336: 4 * (K + 2048) = 65536 fits the CUDA-core kernel with
+    # 64 KB of tables (two 4-bit types) but not with 128 KB (four), which
+    # then runs on the tensor cores; both within the gate
+    n, k, m, bits = 256, 14336, 4, 4
+    w = workloads.normal_weights(n, k, 0.02, seed=81 + t, outlier_frac=1e-2)
+    x = workloads.activations(m, k, seed=82)
+    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    st = lq.new_status()
+    y = lq.lutq_gemv_typed(x.cuda(), packed, cbs, bits, n, k,
+                           workspace=lq.new_workspace(m, n, k, bits), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
+                         levels)
+    assert O.rel_error_gate(y.cpu().numpy(), y_ref) <= TOL
+
+
+@pytest.mark.parametrize("bits,t_data,t_call,m", [(4, 4, 1, 1), (4, 4, 2, 2), (4, 4, 2, 32),
+                                                  (3, 2, 1, 1), (3, 2, 1, 32)])
+def test_types_beyond_the_count_stay_inside_the_tables(lq, bits, t_data, t_call, m):
+    # a matrix quantized with more types than the call passes: the lookups of
+    # the extra types are masked to the smaller table region (values
+    # unspecified, every access in bounds); the call and the device stay sound
+    n, k = 256, 2048
+    w = workloads.normal_weights(n, k, 0.02, seed=91, outlier_frac=1e-2)
+    x = workloads.activations(m, k, seed=92).cuda()
+    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t_data)
+    assert int(types.max().item()) >= t_call
+    fn = lq.lutq_gemv_typed if m <= 16 else lq.lutq_gemm_typed
+    st = lq.new_status()
+    fn(x, packed, cbs[:t_call].contiguous(), bits, n, k,
+       workspace=lq.new_workspace(m, n, k, bits), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    # the correct call afterwards is still exact
+    y = fn(x, packed, cbs, bits, n, k, workspace=lq.new_workspace(m, n, k, bits))
+    torch.cuda.synchronize()
+    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
+                         levels)
+    assert O.rel_error_gate(y.cpu().numpy(), y_ref) <= TOL
