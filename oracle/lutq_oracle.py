@@ -231,6 +231,38 @@ def quantize(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
     return best_i.reshape(n, k), scale_bits
 
 
+def quantize_rowscale(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
+    """RTN with one scale per row (Tetra abstract, aiqbench news item: one
+    scale per matrix row; here the row's absolute maximum, not retrained).
+
+    s[n] = max_k |W[n, k]|; v = fp32(W) / fp32(s[n]) (0 when s == 0); q as in
+    quantize().  The scale is returned in every group's slot, scale bits
+    uint16[N, K/128], so packing and the product are those of quantize().
+    """
+    w = np.asarray(w, dtype=np.float32)
+    n, k = w.shape
+    if k % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    if not np.all(np.isfinite(w)):
+        raise ValueError("non-finite weight")
+    levels = np.asarray(levels_f32, dtype=np.float32)
+    if levels.shape != (1 << bits,):
+        raise ValueError("codebook size must be 2^bits")
+    s = np.max(np.abs(w), axis=1)                            # float32, exact
+    s_b = np.broadcast_to(s[:, None], w.shape)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s_b > 0, w / s_b, np.float32(0.0)).astype(np.float32)
+    best_d = np.full(v.shape, np.inf, dtype=np.float32)
+    best_i = np.zeros(v.shape, dtype=np.uint8)
+    for i in range(levels.size):
+        d = np.abs(v - levels[i])
+        take = d < best_d
+        best_i[take] = i
+        best_d[take] = d[take]
+    sb_row = (s.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    return best_i, np.repeat(sb_row[:, None], k // GROUP, axis=1)
+
+
 # --------------------------------------------------------------------------
 # Packing, layout V2 (the offline restructuring of the FLUTE abstract)
 # --------------------------------------------------------------------------

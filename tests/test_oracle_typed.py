@@ -225,3 +225,46 @@ def test_gemv_typed_exact_sum_and_one_hot():
         same = np.full_like(ty, t)
         np.testing.assert_allclose(O.gemv_typed(x, codes, sb, same, tables),
                                    O.gemv(x, codes, sb, tables[t]), rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- per-row scale
+# (Tetra abstract, aiqbench news item: one scale per matrix row)
+
+@pytest.mark.parametrize("bits,kind", [(4, "nf4"), (3, "lloyd_max3")])
+def test_rowscale_single_group_is_plain_rtn(bits, kind):
+    # K = 128: the row is one group, so the two rules coincide
+    w = _weights(64, 128, seed=21)
+    lv = _levels(kind, bits)
+    np.testing.assert_array_equal(O.quantize_rowscale(w, lv, bits)[0], O.quantize(w, lv, bits)[0])
+    np.testing.assert_array_equal(O.quantize_rowscale(w, lv, bits)[1], O.quantize(w, lv, bits)[1])
+
+
+def test_rowscale_equals_group_rtn_when_every_group_holds_the_row_max():
+    w = _weights(32, 512, seed=22)
+    m = np.max(np.abs(w), axis=1)
+    for g in range(4):
+        w[:, 128 * g + 7] = m                       # every group reaches the row maximum
+    lv = _levels("nf4")
+    c1, s1 = O.quantize_rowscale(w, lv, 4)
+    c0, s0 = O.quantize(w, lv, 4)
+    np.testing.assert_array_equal(c1, c0)
+    np.testing.assert_array_equal(s1, s0)
+
+
+def test_rowscale_scale_is_the_row_max_and_codes_by_brute_force():
+    w = _weights(16, 384, seed=23)
+    lv = _levels("logb")
+    codes, sb = O.quantize_rowscale(w, lv, 4)
+    s = O.bf16_bits_to_f32(sb)
+    assert np.all(s == np.max(np.abs(w), axis=1)[:, None])
+    # brute force in fp64 on the exact quotient: agrees except at near-ties
+    v = w.astype(np.float64) / np.max(np.abs(w), axis=1, keepdims=True).astype(np.float64)
+    d = np.abs(v[..., None] - lv.astype(np.float64))
+    ref = np.argmin(d, axis=-1)
+    srt = np.sort(d, axis=-1)
+    tie = (srt[..., 1] - srt[..., 0]) < 1e-6
+    assert np.all((codes == ref) | tie)
+    assert np.mean(tie) < 1e-3
+    # the row maximum maps to a +-1 level
+    arg = np.argmax(np.abs(w), axis=1)
+    assert np.all(np.abs(lv[codes[np.arange(16), arg]]) == 1.0)
