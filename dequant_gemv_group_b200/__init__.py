@@ -14,9 +14,11 @@ from ._binding import (  # noqa: F401
     lutq_fit_codebook,
     lutq_fit_histogram,
     lutq_gemm,
+    lutq_gemm_out_bf16,
     lutq_gemm_typed,
     lutq_gemv,
     lutq_gemv_noalloc,
+    lutq_gemv_out_bf16,
     lutq_gemv_plan,
     lutq_gemv_rht,
     lutq_gemv_typed,
@@ -27,6 +29,7 @@ from ._binding import (  # noqa: F401
     lutq_packed_bytes,
     lutq_packed_bytes_typed,
     lutq_quantize,
+    lutq_quantize_rowscale,
     lutq_quantize_typed,
     lutq_rht_activations,
     lutq_rht_weights,

@@ -37,10 +37,15 @@ _SIGS = {
     "lutq_packed_bytes": (_i64, [_i64, _i64, _i32]),
     "lutq_codebook": (_i32, [_i32, _i32, _vp]),
     "lutq_quantize": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "lutq_quantize_rowscale": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
     "lutq_pack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "lutq_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32]),
     "lutq_gemv": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "lutq_gemm": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
+    "lutq_gemv_out_bf16": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
+                                  _vp]),
+    "lutq_gemm_out_bf16": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
+                                  _vp]),
     "lutq_gemv_noalloc": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp]),
     "lutq_gemv_plan": (_i32, [_i64, _i64, _i32, _vp]),
     "lutq_selftest_wait_timeout": (_i32, [_vp, _i64, _vp]),
@@ -151,6 +156,21 @@ def lutq_quantize(w: torch.Tensor, codebook: torch.Tensor, bits: int,
     return codes, scales
 
 
+def lutq_quantize_rowscale(w: torch.Tensor, codebook: torch.Tensor, bits: int,
+                           status: Optional[torch.Tensor] = None
+                           ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """lutq_quantize with one scale per row (in every group's slot)."""
+    _need(w, torch.bfloat16, "W")
+    _need(codebook, torch.bfloat16, "codebook")
+    n, k = w.shape
+    codes = torch.empty((n, k), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((n, max(k // 128, 1)), dtype=torch.bfloat16, device=w.device)
+    _check(lib.lutq_quantize_rowscale(w.data_ptr(), n, k, codebook.data_ptr(), bits,
+                                      codes.data_ptr(), scales.data_ptr(), _ptr(status),
+                                      _stream()), "lutq_quantize_rowscale")
+    return codes, scales
+
+
 def lutq_pack(codes: torch.Tensor, scales: torch.Tensor, bits: int,
               status: Optional[torch.Tensor] = None) -> torch.Tensor:
     """codes uint8 [N, K] and scales bf16 [N, K/128] -> the packed matrix
@@ -169,11 +189,12 @@ def lutq_pack(codes: torch.Tensor, scales: torch.Tensor, bits: int,
     return packed
 
 
-def _product(fn, where, x, packed, codebook, bits, n, k, y, workspace, status):
+def _product(fn, where, x, packed, codebook, bits, n, k, y, workspace, status,
+             y_dtype=torch.float32):
     _need(x, torch.bfloat16, "x")
     m = x.shape[0]
     if y is None:
-        y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+        y = torch.empty((m, n), dtype=y_dtype, device=x.device)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
     _check(fn(x.data_ptr(), m, packed.data_ptr(), codebook.data_ptr(), bits, n, k, y.data_ptr(),
               ws_ptr, ws_bytes, _ptr(status), _stream()), where)
@@ -184,6 +205,18 @@ def lutq_gemv(x, packed, codebook, bits, n, k, y=None, workspace=None, status=No
     """y[M, N] (fp32) for M = 1..16; see lutq_gemv in include/lutq.h."""
     return _product(lib.lutq_gemv, "lutq_gemv", x, packed, codebook, bits, n, k, y, workspace,
                     status)
+
+
+def lutq_gemv_out_bf16(x, packed, codebook, bits, n, k, y=None, workspace=None, status=None):
+    """lutq_gemv writing y as bf16 (the fp32 sums rounded once)."""
+    return _product(lib.lutq_gemv_out_bf16, "lutq_gemv_out_bf16", x, packed, codebook, bits, n,
+                    k, y, workspace, status, torch.bfloat16)
+
+
+def lutq_gemm_out_bf16(x, packed, codebook, bits, n, k, y=None, workspace=None, status=None):
+    """lutq_gemm writing y as bf16 (the fp32 sums rounded once)."""
+    return _product(lib.lutq_gemm_out_bf16, "lutq_gemm_out_bf16", x, packed, codebook, bits, n,
+                    k, y, workspace, status, torch.bfloat16)
 
 
 def lutq_gemv_noalloc(x, packed, codebook, bits, n, k, y=None, status=None):

@@ -10,16 +10,18 @@
 namespace lutq {
 cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* codebook, int bits,
                             uint8_t* codes, void* scales, int32_t* dev_status, int num_sms,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool row_scale = false);
 cudaError_t launch_pack(const uint8_t* codes, const void* scales, int64_t N, int64_t K,
                         int bits, void* packed, int32_t* dev_status, int num_sms,
                         cudaStream_t stream);
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream);
+                        int32_t* dev_status, int num_sms, cudaStream_t stream,
+                        bool y_bf16 = false);
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0);
+                        int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0,
+                        bool y_bf16 = false);
 cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const void* codebook,
                             const int8_t* signs, int bits, int64_t N, int64_t K, float* y,
                             void* workspace, int32_t* dev_status, int num_sms,
@@ -124,9 +126,9 @@ int64_t lutq_packed_bytes(int64_t N, int64_t K, int bits) {
   return (N / lutq::kStrip) * (K / lutq::kGroup) * (lutq::tile_bytes(bits) + lutq::kScaleBytes);
 }
 
-lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K, const void* codebook_bf16,
-                          int bits, uint8_t* codes, void* scales_bf16, int32_t* dev_status,
-                          void* stream) {
+static lutq_status quantize(const void* W_bf16, int64_t N, int64_t K, const void* codebook_bf16,
+                            int bits, uint8_t* codes, void* scales_bf16, int32_t* dev_status,
+                            void* stream, bool row_scale) {
   if (!W_bf16 || !codebook_bf16 || !codes || !scales_bf16) return LUTQ_ERR_INVALID_ARG;
   lutq_status st = check_bits(bits);
   if (st != LUTQ_OK) return st;
@@ -137,7 +139,22 @@ lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K, const void* 
   int sms = 0;
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16,
-                                         dev_status, sms, static_cast<cudaStream_t>(stream)));
+                                         dev_status, sms, static_cast<cudaStream_t>(stream),
+                                         row_scale));
+}
+
+lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K, const void* codebook_bf16,
+                          int bits, uint8_t* codes, void* scales_bf16, int32_t* dev_status,
+                          void* stream) {
+  return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream,
+                  false);
+}
+
+lutq_status lutq_quantize_rowscale(const void* W_bf16, int64_t N, int64_t K,
+                                   const void* codebook_bf16, int bits, uint8_t* codes,
+                                   void* scales_bf16, int32_t* dev_status, void* stream) {
+  return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream,
+                  true);
 }
 
 lutq_status lutq_pack(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
@@ -183,6 +200,36 @@ lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_gemv(x_bf16, M, packed, codebook_bf16, bits, N, K, y, workspace,
                                      dev_status, sms, static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_gemv_out_bf16(const void* x_bf16, int64_t M, const void* packed,
+                               const void* codebook_bf16, int bits, int64_t N, int64_t K,
+                               void* y_bf16, void* workspace, int64_t workspace_bytes,
+                               int32_t* dev_status, void* stream) {
+  lutq_status st = check_product_args(x_bf16, M, 16, packed, codebook_bf16, bits, N, K,
+                                      static_cast<const float*>(y_bf16), workspace,
+                                      workspace_bytes, lutq_workspace_bytes(M, N, K, bits));
+  if (st != LUTQ_OK) return st;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_gemv(x_bf16, M, packed, codebook_bf16, bits, N, K,
+                                     static_cast<float*>(y_bf16), workspace, dev_status, sms,
+                                     static_cast<cudaStream_t>(stream), true));
+}
+
+lutq_status lutq_gemm_out_bf16(const void* x_bf16, int64_t M, const void* packed,
+                               const void* codebook_bf16, int bits, int64_t N, int64_t K,
+                               void* y_bf16, void* workspace, int64_t workspace_bytes,
+                               int32_t* dev_status, void* stream) {
+  lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, codebook_bf16, bits,
+                                      N, K, static_cast<const float*>(y_bf16), workspace,
+                                      workspace_bytes, lutq_workspace_bytes(M, N, K, bits));
+  if (st != LUTQ_OK) return st;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_gemm(x_bf16, M, packed, codebook_bf16, bits, N, K,
+                                     static_cast<float*>(y_bf16), workspace, dev_status, sms,
+                                     static_cast<cudaStream_t>(stream), 0, true));
 }
 
 lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,

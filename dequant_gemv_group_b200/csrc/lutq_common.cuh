@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "lutq.h"
@@ -39,6 +40,16 @@ __host__ __device__ constexpr int table_region_bytes(int bits, int types) {
 // Record a device-side error: the first non-zero code wins.
 __device__ __forceinline__ void report(int32_t* dev_status, int code) {
   if (dev_status != nullptr) atomicCAS(dev_status, 0, code);
+}
+
+// Store output value i: fp32, or (y_bf16) the fp32 value rounded once to
+// bf16 (round to nearest even; the bf16 output variant of the products).
+__device__ __forceinline__ void store_y(float* y, int y_bf16, int64_t i, float v) {
+  if (y_bf16) {
+    reinterpret_cast<uint16_t*>(y)[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  } else {
+    y[i] = v;
+  }
 }
 
 __device__ __forceinline__ float bf16_lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }

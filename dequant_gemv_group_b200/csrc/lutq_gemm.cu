@@ -75,6 +75,7 @@ struct GemmArgs {
   const uint16_t* codebook; // [types][2^BITS] with per-group types
   int ntypes;               // tables in `codebook` (1 without per-group types)
   int lut_bytes;            // the table region (table_region_bytes)
+  int y_bf16;               // y is bf16 (the fp32 sums rounded once) instead of fp32
   float* y;
   float* part;        // [kGemmMaxCtas][2][4][NT][32]: (CTA, slot, strip, column, row)
   int* counters;      // [BT * NTILES * 4 * kMaxPromoteGroups]
@@ -143,11 +144,11 @@ __device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t s
   const uint32_t U = uint32_t(a.U), C = uint32_t(a.C);
   const uint32_t c_lo = g_unit_owner(uint32_t(seg_begin), U, C);
   const uint32_t c_hi = g_unit_owner(uint32_t(seg_end - 1), U, C);
-  float* ycol = a.y + (bt * kTileRows + c0) * a.N + row;
+  const int64_t ycol = (bt * kTileRows + c0) * a.N + row;
   if (c_lo == c_hi) {
 #pragma unroll
     for (int j = 0; j < NC; ++j)
-      if (c0 + j < mt) ycol[int64_t(j) * a.N] = acc[j];
+      if (c0 + j < mt) store_y(a.y, a.y_bf16, ycol + int64_t(j) * a.N, acc[j]);
     return;
   }
   const int64_t cta = blockIdx.x;
@@ -172,7 +173,7 @@ __device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t s
   }
 #pragma unroll
   for (int j = 0; j < NC; ++j)
-    if (c0 + j < mt) ycol[int64_t(j) * a.N] = acc[j];
+    if (c0 + j < mt) store_y(a.y, a.y_bf16, ycol + int64_t(j) * a.N, acc[j]);
   if (lane == 0) *counter = 0;
 }
 
@@ -604,7 +605,8 @@ static cudaError_t launch_nts(int nt, const CUtensorMap& map, const GemmArgs& a,
 // packed matrix carries its type blocks and `codebook` holds `types` tables).
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream, int types) {
+                        int32_t* dev_status, int num_sms, cudaStream_t stream, int types,
+                        bool y_bf16) {
   const int nt = gemm_nt(M);
   CUtensorMap map;
   std::memset(&map, 0, sizeof(map));
@@ -617,6 +619,7 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
   a.codebook = static_cast<const uint16_t*>(codebook);
   a.ntypes = types > 0 ? types : 1;
   a.lut_bytes = table_region_bytes(bits, types);
+  a.y_bf16 = y_bf16 ? 1 : 0;
   a.y = y;
   a.dev_status = dev_status;
   a.N = N;

@@ -69,6 +69,7 @@ struct GemvArgs {
   unsigned long long* xch;  // [M][N] exchange slots of strips split between two CTAs (zero between calls)
   int32_t* status;          // caller's device status word or null
   const int8_t* signs;      // randomized Hadamard rotation of x first (null: none)
+  int y_bf16;               // y is bf16 (the fp32 sums rounded once) instead of fp32
   int types;                // per-group data types: codebook holds `types` tables
                             // and the packed matrix its type blocks (0: untyped)
   int64_t N, K, G, U;       // U = number of units
@@ -164,7 +165,8 @@ __device__ __forceinline__ void deposit_strip(const GemvArgs& a, const Span& p, 
 #pragma unroll
     for (int i = 0; i < R; ++i)
 #pragma unroll
-      for (int m = 0; m < M; ++m) a.y[m * a.N + int64_t(strip) * kStrip + rows[i]] = vals[i][m];
+      for (int m = 0; m < M; ++m)
+        store_y(a.y, a.y_bf16, m * a.N + int64_t(strip) * kStrip + rows[i], vals[i][m]);
     return;
   }
   const int sl = (strip == first_strip) ? 0 : 1;
@@ -179,11 +181,12 @@ __device__ __forceinline__ void deposit_strip(const GemvArgs& a, const Span& p, 
 // takes it, writes the sum and clears the slot for the next call.  Both
 // orders give the same fp32 sum (addition of two values commutes), so the
 // result does not depend on timing.
-__device__ __forceinline__ void exchange_half(unsigned long long* slot, float v, float* y) {
+__device__ __forceinline__ void exchange_half(unsigned long long* slot, float v,
+                                              const GemvArgs& a, int64_t yi) {
   const unsigned long long mine = (1ull << 32) | __float_as_uint(v);
   const unsigned long long other = atomicExch(slot, mine);
   if (other != 0ull) {
-    *y = v + __uint_as_float(uint32_t(other));
+    store_y(a.y, a.y_bf16, yi, v + __uint_as_float(uint32_t(other)));
     *slot = 0ull;
   }
 }
@@ -220,15 +223,15 @@ __device__ void cta_finish(const GemvArgs& a, const Span& p, const float* all_sl
       for (int m = 0; m < M; ++m) sum[m] += some ? src[m * kStrip + lane] : 0.0f;
     }
     if (full && whole) continue;  // written by its warp
-    float* yrow = a.y + int64_t(strip) * kStrip + lane;
+    const int64_t yrow = int64_t(strip) * kStrip + lane;
     if (full && lo >= p.v0 && hi <= p.v1) {
 #pragma unroll
-      for (int m = 0; m < M; ++m) yrow[m * a.N] = sum[m];
+      for (int m = 0; m < M; ++m) store_y(a.y, a.y_bf16, yrow + m * a.N, sum[m]);
       continue;
     }
-    unsigned long long* xrow = a.xch + int64_t(strip) * kStrip + lane;
+    unsigned long long* xrow = a.xch + yrow;
 #pragma unroll
-    for (int m = 0; m < M; ++m) exchange_half(xrow + m * a.N, sum[m], yrow + m * a.N);
+    for (int m = 0; m < M; ++m) exchange_half(xrow + m * a.N, sum[m], a, yrow + m * a.N);
   }
 }
 
@@ -875,7 +878,8 @@ static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
 
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0);
+                        int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0,
+                        bool y_bf16 = false);
 
 // Batches up to kMaxSmallBatch run on the CUDA cores when their activations
 // fit the small-batch kernel's shared memory.  Larger batches are a dense
@@ -901,8 +905,9 @@ static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream
 
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream) {
+                        int32_t* dev_status, int num_sms, cudaStream_t stream, bool y_bf16) {
   GemvArgs a;
+  a.y_bf16 = y_bf16 ? 1 : 0;
   a.x = static_cast<const uint16_t*>(x);
   a.packed = static_cast<const uint8_t*>(packed);
   a.codebook = static_cast<const uint16_t*>(codebook);
@@ -920,7 +925,7 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   if (!small_fits(M, K))
     return launch_gemm(x, M, packed, codebook, bits, N, K, y, workspace, dev_status,
-                       num_sms, stream);
+                       num_sms, stream, 0, y_bf16);
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
                    : launch_bits<3>(a, int(M), num_sms, stream);
 }
@@ -952,6 +957,7 @@ cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const 
   a.xch = static_cast<unsigned long long*>(workspace);
   a.status = dev_status;
   a.signs = signs;
+  a.y_bf16 = 0;
   a.types = 0;
   a.N = N;
   a.K = K;
@@ -982,6 +988,7 @@ cudaError_t launch_gemv_typed(const void* x, int64_t M, const void* packed, cons
   a.xch = static_cast<unsigned long long*>(workspace);
   a.status = dev_status;
   a.signs = nullptr;
+  a.y_bf16 = 0;
   a.types = types;
   a.N = N;
   a.K = K;

@@ -24,7 +24,8 @@
 namespace lutq {
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream);
+                        int32_t* dev_status, int num_sms, cudaStream_t stream,
+                        bool y_bf16 = false);
 int64_t gemv_workspace_bytes(int64_t M, int64_t N);
 }  // namespace lutq
 

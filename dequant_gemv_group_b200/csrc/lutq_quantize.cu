@@ -12,7 +12,11 @@
 
 namespace lutq {
 
-template <int BITS>
+// ROW: one scale per row (Tetra abstract, aiqbench news item: one scale per
+// matrix row; here the row's absolute maximum): row_amax_kernel has left the
+// row's maximum in the row's first scale slot, every group divides by it and
+// the other slots receive a copy.
+template <int BITS, bool ROW>
 __global__ void __launch_bounds__(256)
 quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
                 const uint16_t* __restrict__ codebook, uint32_t* __restrict__ codes,
@@ -40,6 +44,8 @@ quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const int64_t g = u % groups;
+    if (ROW) amax = __uint_as_float(uint32_t(scales[u - g]) << 16);
 
     uint32_t packed4 = 0;
 #pragma unroll
@@ -55,9 +61,34 @@ quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
       packed4 |= bi << (8 * i);
     }
     codes[u * 32 + lane] = packed4;
-    if (lane == 0) scales[u] = uint16_t(__float_as_uint(amax) >> 16);
+    if (lane == 0 && (!ROW || g != 0)) scales[u] = uint16_t(__float_as_uint(amax) >> 16);
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) report(dev_status, LUTQ_ERR_NONFINITE);
+}
+
+// The absolute maximum of each row (one warp per row, 16-byte loads), as
+// bf16 bits (exact: the maximum of bf16 magnitudes) into the row's first
+// scale slot.
+__global__ void __launch_bounds__(256)
+row_amax_kernel(const uint4* __restrict__ W, int64_t n_rows, int64_t K, int64_t groups,
+                uint16_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows;
+       r += warps) {
+    const uint4* row = W + r * (K / 8);
+    float amax = 0.0f;
+    for (int64_t j = lane; j < K / 8; j += 32) {
+      const uint4 v = row[j];
+      const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_f32(x[i])), fabsf(bf16_hi_to_f32(x[i]))));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) scales[r * groups] = uint16_t(__float_as_uint(amax) >> 16);
+  }
 }
 
 // Per-group data types (BitMoD abstract, same listing: each group of 128
@@ -185,19 +216,33 @@ cudaError_t launch_quantize_typed(const void* W, int64_t N, int64_t K, const voi
 
 cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* codebook, int bits,
                             uint8_t* codes, void* scales, int32_t* dev_status, int num_sms,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, bool row_scale) {
   const int64_t units = N * (K / kGroup);
   int64_t blocks = (units + 7) / 8;
   const int64_t cap = int64_t(num_sms) * 8;
   if (blocks > cap) blocks = cap;
-  if (bits == 4)
-    quantize_kernel<4><<<unsigned(blocks), 256, 0, stream>>>(
-        static_cast<const uint2*>(W), N, K / kGroup, static_cast<const uint16_t*>(codebook),
-        reinterpret_cast<uint32_t*>(codes), static_cast<uint16_t*>(scales), dev_status);
-  else
-    quantize_kernel<3><<<unsigned(blocks), 256, 0, stream>>>(
-        static_cast<const uint2*>(W), N, K / kGroup, static_cast<const uint16_t*>(codebook),
-        reinterpret_cast<uint32_t*>(codes), static_cast<uint16_t*>(scales), dev_status);
+  const uint2* w = static_cast<const uint2*>(W);
+  const uint16_t* cb = static_cast<const uint16_t*>(codebook);
+  uint32_t* c = reinterpret_cast<uint32_t*>(codes);
+  uint16_t* s = static_cast<uint16_t*>(scales);
+  if (row_scale) {
+    int64_t rb = (N + 7) / 8;
+    if (rb > int64_t(num_sms) * 8) rb = int64_t(num_sms) * 8;
+    row_amax_kernel<<<unsigned(rb), 256, 0, stream>>>(static_cast<const uint4*>(W), N, K,
+                                                      K / kGroup, s);
+    if (bits == 4)
+      quantize_kernel<4, true><<<unsigned(blocks), 256, 0, stream>>>(w, N, K / kGroup, cb, c, s,
+                                                                     dev_status);
+    else
+      quantize_kernel<3, true><<<unsigned(blocks), 256, 0, stream>>>(w, N, K / kGroup, cb, c, s,
+                                                                     dev_status);
+  } else if (bits == 4) {
+    quantize_kernel<4, false><<<unsigned(blocks), 256, 0, stream>>>(w, N, K / kGroup, cb, c, s,
+                                                                    dev_status);
+  } else {
+    quantize_kernel<3, false><<<unsigned(blocks), 256, 0, stream>>>(w, N, K / kGroup, cb, c, s,
+                                                                    dev_status);
+  }
   return cudaGetLastError();
 }
 

@@ -119,6 +119,22 @@ lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K,
                           int32_t* dev_status, void* stream);
 
 /*
+ * lutq_quantize_rowscale - lutq_quantize with one scale per row.
+ *
+ * Source: the Tetra abstract (aiqbench news item) keeps one scale per matrix
+ * row; here, without retraining, the row's absolute maximum:
+ *   s[n]   = max_k |W[n,k]|                    (exact in bf16)
+ *   v      = float(W[n,k]) / float(s[n])       (IEEE fp32 divide; 0 if s == 0)
+ *   q[n,k] = lowest i minimising the fp32 value |v - c_i|.
+ * s[n] is written to every group's slot of `scales` (bf16 [N,K/128]), so
+ * lutq_pack and the products take the result unchanged.  Arguments, errors
+ * and asynchrony as lutq_quantize.
+ */
+lutq_status lutq_quantize_rowscale(const void* W_bf16, int64_t N, int64_t K,
+                                   const void* codebook_bf16, int bits, uint8_t* codes,
+                                   void* scales_bf16, int32_t* dev_status, void* stream);
+
+/*
  * lutq_pack - offline restructuring of the codes and scales into layout V2.
  *
  * Source: the FLUTE abstract ("offline restructuring of the quantized weight
@@ -336,6 +352,22 @@ lutq_status lutq_gemv_rht(const void* x_bf16, int64_t M, const void* packed,
                           const void* codebook_bf16, const int8_t* signs, int bits, int64_t N,
                           int64_t K, float* y, void* workspace, int64_t workspace_bytes,
                           int32_t* dev_status, void* stream);
+
+/*
+ * lutq_gemv_out_bf16 / lutq_gemm_out_bf16 - lutq_gemv / lutq_gemm writing y as
+ * bf16: each fp32 sum that the fp32 calls write is rounded once to bf16
+ * (round to nearest even), so y_bf16 equals the fp32 result rounded, bit for
+ * bit.  y_bf16: device bf16 [M, N] row-major, 16-byte aligned.  Other
+ * arguments, workspace and errors as lutq_gemv / lutq_gemm.
+ */
+lutq_status lutq_gemv_out_bf16(const void* x_bf16, int64_t M, const void* packed,
+                               const void* codebook_bf16, int bits, int64_t N, int64_t K,
+                               void* y_bf16, void* workspace, int64_t workspace_bytes,
+                               int32_t* dev_status, void* stream);
+lutq_status lutq_gemm_out_bf16(const void* x_bf16, int64_t M, const void* packed,
+                               const void* codebook_bf16, int bits, int64_t N, int64_t K,
+                               void* y_bf16, void* workspace, int64_t workspace_bytes,
+                               int32_t* dev_status, void* stream);
 
 /*
  * lutq_gemm - the same product on the tensor cores (tcgen05), for batches

@@ -72,8 +72,9 @@ def test_codebook_bits_mismatch(lq):
 A = 1 << 20
 
 
-def test_quantize_argument_errors(lq):
-    f = lq.lib.lutq_quantize
+@pytest.mark.parametrize("name", ["lutq_quantize", "lutq_quantize_rowscale"])
+def test_quantize_argument_errors(lq, name):
+    f = getattr(lq.lib, name)
     assert f(None, 32, 128, A, 4, A, A, None, None) == 1          # null W
     assert f(A, 32, 128, A, 5, A, A, None, None) == 3             # bits
     assert f(A, 33, 128, A, 4, A, A, None, None) == 2             # N % 32
