@@ -263,6 +263,34 @@ def quantize_rowscale(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]
     return best_i, np.repeat(sb_row[:, None], k // GROUP, axis=1)
 
 
+def quantize_tensorscale(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
+    """RTN with one scale for the whole matrix (tensor-wise granularity, the
+    comparison baseline of the Log_bQuant abstract): s = max |W| over all
+    entries, v = fp32(W) / fp32(s), q as in quantize(); s in every slot."""
+    w = np.asarray(w, dtype=np.float32)
+    n, k = w.shape
+    if k % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    codes, sb = quantize_rowscale(np.concatenate([w.reshape(1, -1)]), levels_f32, bits)
+    return codes.reshape(n, k), np.full((n, k // GROUP), sb[0, 0], dtype=np.uint16)
+
+
+def asym_linear_levels(w_min: float, w_max: float, bits: int) -> np.ndarray:
+    """Asymmetric linear codebook (Log_bQuant abstract: asymmetric linear
+    quantization, the uniform baseline it compares with).  Reading: the 2^bits
+    evenly spaced values from w_min to w_max, divided by S = max(|w_min|,
+    |w_max|) so that they lie in [-1, 1] (the matrix's scale S then comes from
+    quantize_tensorscale); computed in fp64, rounded once to bf16."""
+    if not (w_min <= w_max) or not np.isfinite(w_min) or not np.isfinite(w_max):
+        raise ValueError("need finite w_min <= w_max")
+    s = max(abs(w_min), abs(w_max))
+    n = 1 << bits
+    if s == 0:
+        return np.zeros(n)
+    i = np.arange(n, dtype=np.float64)
+    return bf16_round((w_min + i * (w_max - w_min) / (n - 1)) / s)
+
+
 # --------------------------------------------------------------------------
 # Packing, layout V2 (the offline restructuring of the FLUTE abstract)
 # --------------------------------------------------------------------------

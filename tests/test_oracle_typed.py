@@ -268,3 +268,45 @@ def test_rowscale_scale_is_the_row_max_and_codes_by_brute_force():
     # the row maximum maps to a +-1 level
     arg = np.argmax(np.abs(w), axis=1)
     assert np.all(np.abs(lv[codes[np.arange(16), arg]]) == 1.0)
+
+
+# ------------------------------------------- tensor-wise asymmetric linear
+# (Log_bQuant abstract: the asymmetric linear, tensor-wise baseline)
+
+def test_tensorscale_is_rowscale_of_the_flattened_matrix_and_the_global_max():
+    w = _weights(32, 256, seed=31)
+    lv = _levels("uniform4")
+    codes, sb = O.quantize_tensorscale(w, lv, 4)
+    s = O.bf16_bits_to_f32(sb)
+    assert np.all(s == np.max(np.abs(w)))
+    c1, _ = O.quantize_rowscale(w.reshape(1, -1), lv, 4)
+    np.testing.assert_array_equal(codes, c1.reshape(32, 256))
+    # a single-row matrix: tensor scale = row scale
+    np.testing.assert_array_equal(O.quantize_tensorscale(w[:1], lv, 4)[0],
+                                  O.quantize_rowscale(w[:1], lv, 4)[0])
+
+
+def test_asym_linear_levels_closed_form():
+    lv = O.asym_linear_levels(-0.5, 1.0, 4)
+    # (w_min + i (w_max - w_min) / 15) / 1.0 = -0.5 + 0.1 i, each rounded to bf16
+    want = O.bf16_round(np.array([-0.5 + 0.1 * i for i in range(16)]))
+    np.testing.assert_array_equal(lv, want)
+    assert lv[0] == -0.5 and lv[-1] == 1.0
+    assert np.all(np.diff(lv) > 0)
+    lv3 = O.asym_linear_levels(-2.0, 0.5, 3)            # S = 2: from -1 to 0.25
+    assert lv3[0] == -1.0 and lv3[-1] == 0.25 and lv3.size == 8
+    np.testing.assert_array_equal(O.asym_linear_levels(0.0, 0.0, 4), np.zeros(16))
+    with pytest.raises(ValueError):
+        O.asym_linear_levels(1.0, -1.0, 4)
+
+
+def test_asym_linear_grid_points_quantize_exactly():
+    # weights on the (bf16) grid times S quantize to themselves
+    lv = O.asym_linear_levels(-0.25, 1.0, 4).astype(np.float32)
+    rng = np.random.default_rng(33)
+    idx = rng.integers(0, 16, size=(32, 256))
+    idx[0, 0] = 15                                       # the maximum, +1 * S
+    w = (lv[idx] * np.float32(0.5)).astype(np.float32)  # S = 0.5, exact
+    codes, sb = O.quantize_tensorscale(w, lv, 4)
+    np.testing.assert_array_equal(codes, idx)
+    np.testing.assert_array_equal(O.dequant(codes, sb, lv), w)
