@@ -394,6 +394,28 @@ def side_measurements(lq, dev, args):
                     "quantize_typed_us": tt * 1e6, "groups_per_type": counts,
                     "rel_error_vs_unquantized": {args.codebook: err_plain, "typed": err_typed}}
     del packs_t, packed_t
+    # the baselines of the pages' quantizers, same layer, same GEMV: one scale
+    # per row, and the tensor-wise asymmetric linear quantizer (levels evenly
+    # spaced from min W to max W, one scale for the matrix)
+    errs = {}
+    codes_b, scales_b = lq.lutq_quantize_rowscale(w, cb, bits, status=st)
+    y_b = lq.lutq_gemv(x1, lq.lutq_pack(codes_b, scales_b, bits, status=st), cb, bits, n, k,
+                       workspace=ws1, status=st)
+    errs[f"{args.codebook}_row_scale"] = y_b
+    wmin, wmax = float(w.float().min()), float(w.float().max())
+    cb_a = lq.lutq_codebook_asym_linear(wmin, wmax, bits).to(dev)
+    codes_b, scales_b = lq.lutq_quantize_tensorscale(w, cb_a, bits, status=st)
+    y_b = lq.lutq_gemv(x1, lq.lutq_pack(codes_b, scales_b, bits, status=st), cb_a, bits, n, k,
+                       workspace=ws1, status=st)
+    errs["asym_linear_tensor_scale"] = y_b
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    out["baselines"] = {"rel_error_vs_unquantized": dict(
+        {f"{args.codebook}_group128": err_plain},
+        **{key: float(np.linalg.norm(v.double().cpu().numpy() - exact) / np.linalg.norm(exact))
+           for key, v in errs.items()}),
+        "note": "same layer and GEMV; scales per group of 128, per row, or one per matrix"}
+    del codes_b, scales_b, errs
     out["offline"] = {"quantize_gbs": q_bytes / tq / 1e9, "quantize_us": tq * 1e6,
                       "pack_gbs": p_bytes / tp / 1e9, "pack_us": tp * 1e6,
                       "note": "W bf16 -> codes u8 + scales; codes + scales -> layout V2 (L2-warm)"}

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     LutqError,
     lib,
     lutq_codebook,
+    lutq_codebook_asym_linear,
     lutq_fit_codebook,
     lutq_fit_histogram,
     lutq_gemm,
@@ -30,6 +31,7 @@ from ._binding import (  # noqa: F401
     lutq_packed_bytes_typed,
     lutq_quantize,
     lutq_quantize_rowscale,
+    lutq_quantize_tensorscale,
     lutq_quantize_typed,
     lutq_rht_activations,
     lutq_rht_weights,

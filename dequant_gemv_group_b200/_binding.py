@@ -38,6 +38,8 @@ _SIGS = {
     "lutq_codebook": (_i32, [_i32, _i32, _vp]),
     "lutq_quantize": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
     "lutq_quantize_rowscale": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "lutq_quantize_tensorscale": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "lutq_codebook_asym_linear": (_i32, [ctypes.c_double, ctypes.c_double, _i32, _vp]),
     "lutq_pack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "lutq_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32]),
     "lutq_gemv": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
@@ -156,19 +158,39 @@ def lutq_quantize(w: torch.Tensor, codebook: torch.Tensor, bits: int,
     return codes, scales
 
 
-def lutq_quantize_rowscale(w: torch.Tensor, codebook: torch.Tensor, bits: int,
-                           status: Optional[torch.Tensor] = None
-                           ) -> Tuple[torch.Tensor, torch.Tensor]:
-    """lutq_quantize with one scale per row (in every group's slot)."""
+def _quantize_scoped(fn, where, w, codebook, bits, status):
     _need(w, torch.bfloat16, "W")
     _need(codebook, torch.bfloat16, "codebook")
     n, k = w.shape
     codes = torch.empty((n, k), dtype=torch.uint8, device=w.device)
     scales = torch.empty((n, max(k // 128, 1)), dtype=torch.bfloat16, device=w.device)
-    _check(lib.lutq_quantize_rowscale(w.data_ptr(), n, k, codebook.data_ptr(), bits,
-                                      codes.data_ptr(), scales.data_ptr(), _ptr(status),
-                                      _stream()), "lutq_quantize_rowscale")
+    _check(fn(w.data_ptr(), n, k, codebook.data_ptr(), bits, codes.data_ptr(), scales.data_ptr(),
+              _ptr(status), _stream()), where)
     return codes, scales
+
+
+def lutq_quantize_rowscale(w: torch.Tensor, codebook: torch.Tensor, bits: int,
+                           status: Optional[torch.Tensor] = None
+                           ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """lutq_quantize with one scale per row (in every group's slot)."""
+    return _quantize_scoped(lib.lutq_quantize_rowscale, "lutq_quantize_rowscale", w, codebook,
+                            bits, status)
+
+
+def lutq_quantize_tensorscale(w: torch.Tensor, codebook: torch.Tensor, bits: int,
+                              status: Optional[torch.Tensor] = None
+                              ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """lutq_quantize with one scale for the matrix (in every slot)."""
+    return _quantize_scoped(lib.lutq_quantize_tensorscale, "lutq_quantize_tensorscale", w,
+                            codebook, bits, status)
+
+
+def lutq_codebook_asym_linear(w_min: float, w_max: float, bits: int) -> torch.Tensor:
+    """The asymmetric linear codebook from w_min to w_max (bf16, host)."""
+    out = torch.empty(1 << bits, dtype=torch.int16)
+    _check(lib.lutq_codebook_asym_linear(float(w_min), float(w_max), bits, out.data_ptr()),
+           "lutq_codebook_asym_linear")
+    return out.view(torch.bfloat16)
 
 
 def lutq_pack(codes: torch.Tensor, scales: torch.Tensor, bits: int,

@@ -10,7 +10,7 @@
 namespace lutq {
 cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* codebook, int bits,
                             uint8_t* codes, void* scales, int32_t* dev_status, int num_sms,
-                            cudaStream_t stream, bool row_scale = false);
+                            cudaStream_t stream, int scope = 0);
 cudaError_t launch_pack(const uint8_t* codes, const void* scales, int64_t N, int64_t K,
                         int bits, void* packed, int32_t* dev_status, int num_sms,
                         cudaStream_t stream);
@@ -128,7 +128,7 @@ int64_t lutq_packed_bytes(int64_t N, int64_t K, int bits) {
 
 static lutq_status quantize(const void* W_bf16, int64_t N, int64_t K, const void* codebook_bf16,
                             int bits, uint8_t* codes, void* scales_bf16, int32_t* dev_status,
-                            void* stream, bool row_scale) {
+                            void* stream, int scope) {
   if (!W_bf16 || !codebook_bf16 || !codes || !scales_bf16) return LUTQ_ERR_INVALID_ARG;
   lutq_status st = check_bits(bits);
   if (st != LUTQ_OK) return st;
@@ -140,21 +140,25 @@ static lutq_status quantize(const void* W_bf16, int64_t N, int64_t K, const void
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16,
                                          dev_status, sms, static_cast<cudaStream_t>(stream),
-                                         row_scale));
+                                         scope));
 }
 
 lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K, const void* codebook_bf16,
                           int bits, uint8_t* codes, void* scales_bf16, int32_t* dev_status,
                           void* stream) {
-  return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream,
-                  false);
+  return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 0);
 }
 
 lutq_status lutq_quantize_rowscale(const void* W_bf16, int64_t N, int64_t K,
                                    const void* codebook_bf16, int bits, uint8_t* codes,
                                    void* scales_bf16, int32_t* dev_status, void* stream) {
-  return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream,
-                  true);
+  return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 1);
+}
+
+lutq_status lutq_quantize_tensorscale(const void* W_bf16, int64_t N, int64_t K,
+                                      const void* codebook_bf16, int bits, uint8_t* codes,
+                                      void* scales_bf16, int32_t* dev_status, void* stream) {
+  return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 2);
 }
 
 lutq_status lutq_pack(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,

@@ -134,6 +134,25 @@ extern "C" lutq_status lutq_codebook(int kind, int bits, uint16_t* out_bf16) {
   return LUTQ_OK;
 }
 
+// Asymmetric linear codebook (Log_bQuant abstract: the asymmetric linear
+// quantization it compares with): the 2^bits evenly spaced values from w_min
+// to w_max, divided by S = max(|w_min|, |w_max|) (the matrix's scale, as
+// lutq_quantize_tensorscale writes it), fp64, rounded once to bf16.
+extern "C" lutq_status lutq_codebook_asym_linear(double w_min, double w_max, int bits,
+                                                 uint16_t* out_bf16) {
+  if (out_bf16 == nullptr) return LUTQ_ERR_INVALID_ARG;
+  if (bits != 3 && bits != 4) return LUTQ_ERR_BITS;
+  if (!std::isfinite(w_min) || !std::isfinite(w_max) || !(w_min <= w_max))
+    return LUTQ_ERR_INVALID_ARG;
+  const int n = 1 << bits;
+  const double s = std::max(std::fabs(w_min), std::fabs(w_max));
+  for (int i = 0; i < n; ++i) {
+    const double v = s == 0.0 ? 0.0 : (w_min + i * (w_max - w_min) / (n - 1)) / s;
+    out_bf16[i] = to_bf16_rne(v);
+  }
+  return LUTQ_OK;
+}
+
 // Lloyd-Max on a histogram of normalised weights (kHistBins bins over
 // [-1, 1], centre of bin b = (2 b + 1 - kHistBins) / kHistBins): alternately
 // give every bin to its nearest level (fp64 distance, ties to the lower

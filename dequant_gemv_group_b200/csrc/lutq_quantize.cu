@@ -12,11 +12,14 @@
 
 namespace lutq {
 
-// ROW: one scale per row (Tetra abstract, aiqbench news item: one scale per
-// matrix row; here the row's absolute maximum): row_amax_kernel has left the
-// row's maximum in the row's first scale slot, every group divides by it and
-// the other slots receive a copy.
-template <int BITS, bool ROW>
+// SCOPE of the scale: 0, the group's absolute maximum; 1, one scale per row
+// (Tetra abstract, aiqbench news item: one scale per matrix row; here the
+// row's absolute maximum), which row_amax_kernel has left in the row's first
+// scale slot; 2, one scale for the matrix (the tensor-wise granularity of the
+// Log_bQuant abstract's baseline), left in the first slot of row 0 by
+// tensor_amax_kernel.  Every group divides by that scale and the other slots
+// receive a copy.
+template <int BITS, int SCOPE>
 __global__ void __launch_bounds__(256)
 quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
                 const uint16_t* __restrict__ codebook, uint32_t* __restrict__ codes,
@@ -45,7 +48,8 @@ quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     const int64_t g = u % groups;
-    if (ROW) amax = __uint_as_float(uint32_t(scales[u - g]) << 16);
+    if (SCOPE == 1) amax = __uint_as_float(uint32_t(scales[u - g]) << 16);
+    if (SCOPE == 2) amax = __uint_as_float(uint32_t(scales[0]) << 16);
 
     uint32_t packed4 = 0;
 #pragma unroll
@@ -61,7 +65,8 @@ quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
       packed4 |= bi << (8 * i);
     }
     codes[u * 32 + lane] = packed4;
-    if (lane == 0 && (!ROW || g != 0)) scales[u] = uint16_t(__float_as_uint(amax) >> 16);
+    const bool source = (SCOPE == 1 && g == 0) || (SCOPE == 2 && u == 0);
+    if (lane == 0 && !source) scales[u] = uint16_t(__float_as_uint(amax) >> 16);
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) report(dev_status, LUTQ_ERR_NONFINITE);
 }
@@ -214,9 +219,23 @@ cudaError_t launch_quantize_typed(const void* W, int64_t N, int64_t K, const voi
   return cudaGetLastError();
 }
 
+// The maximum of the rows' maxima (left by row_amax_kernel in each row's
+// first slot) into the first slot of row 0: one block.
+__global__ void __launch_bounds__(1024)
+tensor_amax_kernel(int64_t n_rows, int64_t groups, uint16_t* __restrict__ scales) {
+  __shared__ uint32_t best;
+  if (threadIdx.x == 0) best = 0;
+  __syncthreads();
+  uint32_t m = 0;  // bf16 bits of non-negative values order as integers
+  for (int64_t r = threadIdx.x; r < n_rows; r += blockDim.x) m = max(m, uint32_t(scales[r * groups]));
+  atomicMax(&best, m);
+  __syncthreads();
+  if (threadIdx.x == 0) scales[0] = uint16_t(best);
+}
+
 cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* codebook, int bits,
                             uint8_t* codes, void* scales, int32_t* dev_status, int num_sms,
-                            cudaStream_t stream, bool row_scale) {
+                            cudaStream_t stream, int scope) {
   const int64_t units = N * (K / kGroup);
   int64_t blocks = (units + 7) / 8;
   const int64_t cap = int64_t(num_sms) * 8;
@@ -225,23 +244,21 @@ cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* cod
   const uint16_t* cb = static_cast<const uint16_t*>(codebook);
   uint32_t* c = reinterpret_cast<uint32_t*>(codes);
   uint16_t* s = static_cast<uint16_t*>(scales);
-  if (row_scale) {
+  if (scope > 0) {
     int64_t rb = (N + 7) / 8;
     if (rb > int64_t(num_sms) * 8) rb = int64_t(num_sms) * 8;
     row_amax_kernel<<<unsigned(rb), 256, 0, stream>>>(static_cast<const uint4*>(W), N, K,
                                                       K / kGroup, s);
-    if (bits == 4)
-      quantize_kernel<4, true><<<unsigned(blocks), 256, 0, stream>>>(w, N, K / kGroup, cb, c, s,
-                                                                     dev_status);
-    else
-      quantize_kernel<3, true><<<unsigned(blocks), 256, 0, stream>>>(w, N, K / kGroup, cb, c, s,
-                                                                     dev_status);
-  } else if (bits == 4) {
-    quantize_kernel<4, false><<<unsigned(blocks), 256, 0, stream>>>(w, N, K / kGroup, cb, c, s,
-                                                                    dev_status);
-  } else {
-    quantize_kernel<3, false><<<unsigned(blocks), 256, 0, stream>>>(w, N, K / kGroup, cb, c, s,
-                                                                    dev_status);
+  }
+  if (scope == 2) tensor_amax_kernel<<<1, 1024, 0, stream>>>(N, K / kGroup, s);
+  const int64_t G = K / kGroup;
+  switch (scope * 2 + (bits == 4 ? 1 : 0)) {
+    case 0: quantize_kernel<3, 0><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    case 1: quantize_kernel<4, 0><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    case 2: quantize_kernel<3, 1><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    case 3: quantize_kernel<4, 1><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    case 4: quantize_kernel<3, 2><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    default: quantize_kernel<4, 2><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
   }
   return cudaGetLastError();
 }

@@ -135,6 +135,31 @@ lutq_status lutq_quantize_rowscale(const void* W_bf16, int64_t N, int64_t K,
                                    void* scales_bf16, int32_t* dev_status, void* stream);
 
 /*
+ * lutq_quantize_tensorscale - lutq_quantize with one scale for the matrix.
+ *
+ * Source: the Log_bQuant abstract (catalyzex author page) compares with
+ * asymmetric linear quantization at tensor-wise granularity.  s = max |W|
+ * over all of W (exact in bf16), v = float(W[n,k]) / float(s), q as in
+ * lutq_quantize; s is written to every slot of `scales`.  With the codebook
+ * of lutq_codebook_asym_linear(min W, max W) this is that baseline: levels
+ * evenly spaced from min W to max W.  Arguments, errors and asynchrony as
+ * lutq_quantize.
+ */
+lutq_status lutq_quantize_tensorscale(const void* W_bf16, int64_t N, int64_t K,
+                                      const void* codebook_bf16, int bits, uint8_t* codes,
+                                      void* scales_bf16, int32_t* dev_status, void* stream);
+
+/*
+ * lutq_codebook_asym_linear - the asymmetric linear codebook: the 2^bits
+ * evenly spaced values from w_min to w_max divided by max(|w_min|, |w_max|),
+ * computed in fp64 and rounded once to bf16 (all zero if both are zero).
+ * out_bf16: host, 2^bits uint16 bf16 bit patterns, written.  Returns
+ * LUTQ_ERR_BITS for bits other than 3 or 4, LUTQ_ERR_INVALID_ARG for a NULL
+ * output, non-finite bounds or w_min > w_max.  No GPU use.
+ */
+lutq_status lutq_codebook_asym_linear(double w_min, double w_max, int bits, uint16_t* out_bf16);
+
+/*
  * lutq_pack - offline restructuring of the codes and scales into layout V2.
  *
  * Source: the FLUTE abstract ("offline restructuring of the quantized weight

@@ -7,6 +7,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 from oracle import lutq_oracle as O
 
@@ -72,7 +73,8 @@ def test_codebook_bits_mismatch(lq):
 A = 1 << 20
 
 
-@pytest.mark.parametrize("name", ["lutq_quantize", "lutq_quantize_rowscale"])
+@pytest.mark.parametrize("name", ["lutq_quantize", "lutq_quantize_rowscale",
+                                  "lutq_quantize_tensorscale"])
 def test_quantize_argument_errors(lq, name):
     f = getattr(lq.lib, name)
     assert f(None, 32, 128, A, 4, A, A, None, None) == 1          # null W
@@ -186,3 +188,16 @@ def test_typed_argument_errors(lq):
     assert gg(A, 1, A, A, 0, 4, 64, 256, A, A, ws, None, None) == 1
     assert gg(A, 1, A, A, 3, 3, 64, 256, A, A, ws, None, None) == 1
     assert gg(A, 1, A, A, 2, 4, 64, 200, A, A, ws, None, None) == 2
+
+
+def test_asym_linear_codebook_bit_exact_vs_oracle(lq):
+    for lo, hi, bits in [(-0.5, 1.0, 4), (-2.0, 0.5, 3), (-0.031, 0.027, 4), (0.0, 0.0, 4),
+                         (0.125, 0.5, 4)]:
+        got = lq.lutq_codebook_asym_linear(lo, hi, bits).view(torch.int16).numpy().view(np.uint16)
+        np.testing.assert_array_equal(got, O.bf16_bits(O.asym_linear_levels(lo, hi, bits)))
+    f = lq.lib.lutq_codebook_asym_linear
+    buf = (ctypes.c_uint16 * 16)()
+    assert f(1.0, -1.0, 4, buf) == 1
+    assert f(-1.0, 1.0, 5, buf) == 3
+    assert f(float("nan"), 1.0, 4, buf) == 1
+    assert f(-1.0, 1.0, 4, None) == 1

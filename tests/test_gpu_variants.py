@@ -88,3 +88,28 @@ def test_bf16_output_is_the_fp32_output_rounded(lq, n, k, m, kind, bits):
             rows = np.arange(min(n, 256))
             y_ref = O.gemv(_f32(x), codes[rows].cpu().numpy(), _bits16(scales[rows]), levels)
         assert O.rel_error_gate(_f32(y16)[:, :y_ref.shape[1]], y_ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("bits", [4, 3])
+@pytest.mark.parametrize("n,k", [(96, 1152), (1024, 4096), (4096, 256)])
+def test_tensorscale_asym_linear_bit_exact_and_product(lq, bits, n, k):
+    # the tensor-wise asymmetric linear baseline: levels evenly spaced from
+    # min W to max W over one scale for the matrix
+    w = workloads.normal_weights(n, k, 0.02, seed=3 * n + bits, outlier_frac=1e-3)
+    lo, hi = float(w.float().min()), float(w.float().max())
+    cb = lq.lutq_codebook_asym_linear(lo, hi, bits)
+    levels = O.asym_linear_levels(lo, hi, bits).astype(np.float32)
+    np.testing.assert_array_equal(_bits16(cb), O.bf16_bits(levels))
+    st = lq.new_status()
+    codes, scales = lq.lutq_quantize_tensorscale(w.cuda(), cb.cuda(), bits, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rc, rs = O.quantize_tensorscale(_f32(w), levels, bits)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+    np.testing.assert_array_equal(_bits16(scales), rs)
+    x = workloads.activations(1, k, seed=9)
+    y = lq.lutq_gemv(x.cuda(), lq.lutq_pack(codes, scales, bits), cb.cuda(), bits, n, k,
+                     workspace=lq.new_workspace(1, n, k, bits), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert O.rel_error_gate(y.cpu().numpy(), O.gemv(_f32(x), rc, rs, levels)) <= TOL
