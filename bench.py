@@ -152,11 +152,20 @@ def barrier(world):
 
 
 def max_over_ranks(world, value):
+    """The largest of the ranks' values (a time: the job takes as long as its
+    slowest rank).  NCCL reduces on the device, other backends on the host."""
     if world == 1:
         return value
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_rate(bytes_per_step, steps, max_seconds, world):
+    """Whole-job GB/s: the bytes all ranks processed (each rank runs the same
+    steps on its own replica) over the slowest rank's time."""
+    return bytes_per_step * steps * world / max_seconds / 1e9
 
 
 # ---------------------------------------------------------------------- oracle arm
@@ -488,8 +497,8 @@ def run_lutq(args, world, rank, local):
 
     nbytes = algorithmic_bytes(m, n, k, bits)
     per_step_s = ms / 1e3 / args.steps
-    gbs_rank = nbytes / per_step_s / 1e9
-    value = gbs_rank * world
+    gbs_rank = nbytes / per_step_s / 1e9          # one GPU (the slowest rank)
+    value = aggregate_rate(nbytes, args.steps, ms / 1e3, world)
 
     # plain stream launches (no graph), for context
     torch.cuda.synchronize()
@@ -520,7 +529,7 @@ def run_lutq(args, world, rank, local):
         y_host.copy_(y, non_blocking=True)
         torch.cuda.synchronize()
     e2e_s = max_over_ranks(world, time.perf_counter() - t0)
-    e2e_gbs = nbytes * e2e_steps / e2e_s / 1e9 * world
+    e2e_gbs = aggregate_rate(nbytes, e2e_steps, e2e_s, world)
 
     extra = side_measurements(lq, dev, args) if not args.no_side else {}
 
