@@ -263,6 +263,19 @@ def quantize_rowscale(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]
     return best_i, np.repeat(sb_row[:, None], k // GROUP, axis=1)
 
 
+def quantize_group256(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
+    """RTN with one scale per group of 256 along K (the group-size variant):
+    s = max |W| over the 256 weights, v = fp32(W) / fp32(s), q as in
+    quantize(); each 256-group's scale fills the slots of its two 128-groups,
+    so packing and the product are those of quantize().  K % 256 == 0."""
+    w = np.asarray(w, dtype=np.float32)
+    n, k = w.shape
+    if k % 256:
+        raise ValueError("K must be a multiple of 256")
+    codes, sb = quantize_rowscale(w.reshape(n * (k // 256), 256), levels_f32, bits)
+    return codes.reshape(n, k), np.repeat(sb[:, 0].reshape(n, k // 256), 2, axis=1)
+
+
 def quantize_tensorscale(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
     """RTN with one scale for the whole matrix (tensor-wise granularity, the
     comparison baseline of the Log_bQuant abstract): s = max |W| over all

@@ -310,3 +310,35 @@ def test_asym_linear_grid_points_quantize_exactly():
     codes, sb = O.quantize_tensorscale(w, lv, 4)
     np.testing.assert_array_equal(codes, idx)
     np.testing.assert_array_equal(O.dequant(codes, sb, lv), w)
+
+
+# ------------------------------------------------------------ group of 256
+
+def test_group256_scale_is_the_256_max_and_codes_by_brute_force():
+    w = _weights(16, 768, seed=41)
+    lv = _levels("nf4")
+    codes, sb = O.quantize_group256(w, lv, 4)
+    s = O.bf16_bits_to_f32(sb)
+    m256 = np.max(np.abs(w.reshape(16, 3, 256)), axis=2)
+    np.testing.assert_array_equal(s, np.repeat(m256, 2, axis=1))
+    v = w.astype(np.float64) / np.repeat(m256, 256, axis=1).astype(np.float64)
+    d = np.abs(v[..., None] - lv.astype(np.float64))
+    ref = np.argmin(d, axis=-1)
+    srt = np.sort(d, axis=-1)
+    tie = (srt[..., 1] - srt[..., 0]) < 1e-6
+    assert np.all((codes == ref) | tie)
+
+
+def test_group256_equals_group128_when_both_halves_share_the_max():
+    w = _weights(32, 512, seed=42)
+    m = np.max(np.abs(w.reshape(32, 2, 256)), axis=2)
+    for j in range(2):
+        w[:, 256 * j + 5] = m[:, j]
+        w[:, 256 * j + 133] = -m[:, j]            # both 128-halves reach the 256 maximum
+    lv = _levels("logb")
+    c2, s2 = O.quantize_group256(w, lv, 4)
+    c1, s1 = O.quantize(w, lv, 4)
+    np.testing.assert_array_equal(c2, c1)
+    np.testing.assert_array_equal(s2, s1)
+    with pytest.raises(ValueError):
+        O.quantize_group256(w[:, :384], lv, 4)
