@@ -30,6 +30,7 @@ from ._binding import (  # noqa: F401
     lutq_packed_bytes,
     lutq_packed_bytes_typed,
     lutq_quantize,
+    lutq_quantize_group256,
     lutq_quantize_rowscale,
     lutq_quantize_tensorscale,
     lutq_quantize_typed,

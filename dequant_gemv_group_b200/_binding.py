@@ -39,6 +39,7 @@ _SIGS = {
     "lutq_quantize": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
     "lutq_quantize_rowscale": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
     "lutq_quantize_tensorscale": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "lutq_quantize_group256": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
     "lutq_codebook_asym_linear": (_i32, [ctypes.c_double, ctypes.c_double, _i32, _vp]),
     "lutq_pack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "lutq_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32]),
@@ -174,6 +175,14 @@ def lutq_quantize_rowscale(w: torch.Tensor, codebook: torch.Tensor, bits: int,
                            ) -> Tuple[torch.Tensor, torch.Tensor]:
     """lutq_quantize with one scale per row (in every group's slot)."""
     return _quantize_scoped(lib.lutq_quantize_rowscale, "lutq_quantize_rowscale", w, codebook,
+                            bits, status)
+
+
+def lutq_quantize_group256(w: torch.Tensor, codebook: torch.Tensor, bits: int,
+                           status: Optional[torch.Tensor] = None
+                           ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """lutq_quantize with one scale per group of 256 (in both 128-group slots)."""
+    return _quantize_scoped(lib.lutq_quantize_group256, "lutq_quantize_group256", w, codebook,
                             bits, status)
 
 

@@ -133,6 +133,7 @@ static lutq_status quantize(const void* W_bf16, int64_t N, int64_t K, const void
   lutq_status st = check_bits(bits);
   if (st != LUTQ_OK) return st;
   if ((st = check_shape(N, K)) != LUTQ_OK) return st;
+  if (scope == 3 && K % 256 != 0) return LUTQ_ERR_SHAPE;  // groups of 256
   if (!aligned16(W_bf16) || !aligned16(codebook_bf16) || !aligned16(codes) ||
       !aligned16(scales_bf16))
     return LUTQ_ERR_ALIGN;
@@ -153,6 +154,12 @@ lutq_status lutq_quantize_rowscale(const void* W_bf16, int64_t N, int64_t K,
                                    const void* codebook_bf16, int bits, uint8_t* codes,
                                    void* scales_bf16, int32_t* dev_status, void* stream) {
   return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 1);
+}
+
+lutq_status lutq_quantize_group256(const void* W_bf16, int64_t N, int64_t K,
+                                   const void* codebook_bf16, int bits, uint8_t* codes,
+                                   void* scales_bf16, int32_t* dev_status, void* stream) {
+  return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 3);
 }
 
 lutq_status lutq_quantize_tensorscale(const void* W_bf16, int64_t N, int64_t K,

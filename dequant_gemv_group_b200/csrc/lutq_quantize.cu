@@ -17,8 +17,9 @@ namespace lutq {
 // row's absolute maximum), which row_amax_kernel has left in the row's first
 // scale slot; 2, one scale for the matrix (the tensor-wise granularity of the
 // Log_bQuant abstract's baseline), left in the first slot of row 0 by
-// tensor_amax_kernel.  Every group divides by that scale and the other slots
-// receive a copy.
+// tensor_amax_kernel; 3, one scale per group of 256 along K (the group-size
+// variant), left in the even 128-group's slot by pair_amax_kernel.  Every
+// group divides by that scale and the other slots receive a copy.
 template <int BITS, int SCOPE>
 __global__ void __launch_bounds__(256)
 quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
@@ -50,6 +51,7 @@ quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
     const int64_t g = u % groups;
     if (SCOPE == 1) amax = __uint_as_float(uint32_t(scales[u - g]) << 16);
     if (SCOPE == 2) amax = __uint_as_float(uint32_t(scales[0]) << 16);
+    if (SCOPE == 3) amax = __uint_as_float(uint32_t(scales[u - (g & 1)]) << 16);
 
     uint32_t packed4 = 0;
 #pragma unroll
@@ -65,7 +67,8 @@ quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
       packed4 |= bi << (8 * i);
     }
     codes[u * 32 + lane] = packed4;
-    const bool source = (SCOPE == 1 && g == 0) || (SCOPE == 2 && u == 0);
+    const bool source =
+        (SCOPE == 1 && g == 0) || (SCOPE == 2 && u == 0) || (SCOPE == 3 && (g & 1) == 0);
     if (lane == 0 && !source) scales[u] = uint16_t(__float_as_uint(amax) >> 16);
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) report(dev_status, LUTQ_ERR_NONFINITE);
@@ -219,6 +222,31 @@ cudaError_t launch_quantize_typed(const void* W, int64_t N, int64_t K, const voi
   return cudaGetLastError();
 }
 
+// The absolute maximum of each group of 256 along K (one warp per group, one
+// 16-byte load per lane) as bf16 bits into the slot of its even 128-group.
+// groups (of 128) is even.
+__global__ void __launch_bounds__(256)
+pair_amax_kernel(const uint4* __restrict__ W, int64_t n_rows, int64_t K, int64_t groups,
+                 uint16_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int64_t pairs = groups / 2;
+  const int64_t tasks = n_rows * pairs;
+  const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < tasks;
+       t += warps) {
+    const int64_t row = t / pairs, j = t - row * pairs;
+    const uint4 v = W[row * (K / 8) + j * 32 + lane];
+    const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_f32(x[i])), fabsf(bf16_hi_to_f32(x[i]))));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) scales[row * groups + 2 * j] = uint16_t(__float_as_uint(amax) >> 16);
+  }
+}
+
 // The maximum of the rows' maxima (left by row_amax_kernel in each row's
 // first slot) into the first slot of row 0: one block.
 __global__ void __launch_bounds__(1024)
@@ -244,7 +272,13 @@ cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* cod
   const uint16_t* cb = static_cast<const uint16_t*>(codebook);
   uint32_t* c = reinterpret_cast<uint32_t*>(codes);
   uint16_t* s = static_cast<uint16_t*>(scales);
-  if (scope > 0) {
+  if (scope == 3) {
+    int64_t pb = (N * (K / 256) + 7) / 8;
+    if (pb > int64_t(num_sms) * 16) pb = int64_t(num_sms) * 16;
+    pair_amax_kernel<<<unsigned(pb), 256, 0, stream>>>(static_cast<const uint4*>(W), N, K,
+                                                       K / kGroup, s);
+  }
+  if (scope == 1 || scope == 2) {
     int64_t rb = (N + 7) / 8;
     if (rb > int64_t(num_sms) * 8) rb = int64_t(num_sms) * 8;
     row_amax_kernel<<<unsigned(rb), 256, 0, stream>>>(static_cast<const uint4*>(W), N, K,
@@ -258,7 +292,9 @@ cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* cod
     case 2: quantize_kernel<3, 1><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
     case 3: quantize_kernel<4, 1><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
     case 4: quantize_kernel<3, 2><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
-    default: quantize_kernel<4, 2><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    case 5: quantize_kernel<4, 2><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    case 6: quantize_kernel<3, 3><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    default: quantize_kernel<4, 3><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
   }
   return cudaGetLastError();
 }

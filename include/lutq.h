@@ -135,6 +135,18 @@ lutq_status lutq_quantize_rowscale(const void* W_bf16, int64_t N, int64_t K,
                                    void* scales_bf16, int32_t* dev_status, void* stream);
 
 /*
+ * lutq_quantize_group256 - lutq_quantize with one scale per group of 256
+ * consecutive weights along K (the group-size variant of the FLUTE
+ * abstract's group quantization): s = max |W| over the 256, v and q as in
+ * lutq_quantize.  The scale fills the slots of both 128-groups of `scales`
+ * (bf16 [N,K/128]), so lutq_pack and the products take the result unchanged.
+ * Returns LUTQ_ERR_SHAPE unless K % 256 == 0; otherwise as lutq_quantize.
+ */
+lutq_status lutq_quantize_group256(const void* W_bf16, int64_t N, int64_t K,
+                                   const void* codebook_bf16, int bits, uint8_t* codes,
+                                   void* scales_bf16, int32_t* dev_status, void* stream);
+
+/*
  * lutq_quantize_tensorscale - lutq_quantize with one scale for the matrix.
  *
  * Source: the Log_bQuant abstract (catalyzex author page) compares with

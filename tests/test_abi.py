@@ -74,7 +74,7 @@ A = 1 << 20
 
 
 @pytest.mark.parametrize("name", ["lutq_quantize", "lutq_quantize_rowscale",
-                                  "lutq_quantize_tensorscale"])
+                                  "lutq_quantize_tensorscale", "lutq_quantize_group256"])
 def test_quantize_argument_errors(lq, name):
     f = getattr(lq.lib, name)
     assert f(None, 32, 128, A, 4, A, A, None, None) == 1          # null W
@@ -82,7 +82,7 @@ def test_quantize_argument_errors(lq, name):
     assert f(A, 33, 128, A, 4, A, A, None, None) == 2             # N % 32
     assert f(A, 32, 130, A, 4, A, A, None, None) == 2             # K % 128
     assert f(A, 0, 128, A, 4, A, A, None, None) == 2              # empty
-    assert f(A + 2, 32, 128, A, 4, A, A, None, None) == 4         # misaligned
+    assert f(A + 2, 32, 256, A, 4, A, A, None, None) == 4         # misaligned
 
 
 def test_pack_argument_errors(lq):
@@ -201,3 +201,9 @@ def test_asym_linear_codebook_bit_exact_vs_oracle(lq):
     assert f(-1.0, 1.0, 5, buf) == 3
     assert f(float("nan"), 1.0, 4, buf) == 1
     assert f(-1.0, 1.0, 4, None) == 1
+
+
+def test_group256_needs_k_multiple_of_256(lq):
+    f = lq.lib.lutq_quantize_group256
+    assert f(A, 32, 384, A, 4, A, A, None, None) == 2
+    assert f(A, 32, 128, A, 4, A, A, None, None) == 2

@@ -113,3 +113,25 @@ def test_tensorscale_asym_linear_bit_exact_and_product(lq, bits, n, k):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert O.rel_error_gate(y.cpu().numpy(), O.gemv(_f32(x), rc, rs, levels)) <= TOL
+
+
+@pytest.mark.parametrize("kind,bits", [("nf4", 4), ("lloyd_max3", 3)])
+@pytest.mark.parametrize("n,k", [(32, 256), (96, 1280), (1024, 4096)])
+def test_group256_quantize_bit_exact_and_product(lq, kind, bits, n, k):
+    w = workloads.normal_weights(n, k, 0.02, seed=7 * n + bits, outlier_frac=1e-2)
+    w[5, 256:512] = 0.0                               # an all-zero 256-group
+    cb = lq.lutq_codebook(kind, bits).cuda()
+    _, levels = O.codebook(kind, bits)
+    st = lq.new_status()
+    codes, scales = lq.lutq_quantize_group256(w.cuda(), cb, bits, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rc, rs = O.quantize_group256(_f32(w), levels, bits)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+    np.testing.assert_array_equal(_bits16(scales), rs)
+    x = workloads.activations(3, k, seed=13)
+    y = lq.lutq_gemv(x.cuda(), lq.lutq_pack(codes, scales, bits, status=st), cb, bits, n, k,
+                     workspace=lq.new_workspace(3, n, k, bits), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert O.rel_error_gate(y.cpu().numpy(), O.gemv(_f32(x), rc, rs, levels)) <= TOL
