@@ -276,6 +276,68 @@ def quantize_group256(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]
     return codes.reshape(n, k), np.repeat(sb[:, 0].reshape(n, k // 256), 2, axis=1)
 
 
+def quantize_group64(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
+    """RTN with one scale per group of 64 along K (the finer group-size
+    variant): s = max |W| over the 64, v and q as in quantize().  Returns
+    (codes uint8[N, K], scale bits uint16[N, K/64])."""
+    w = np.asarray(w, dtype=np.float32)
+    n, k = w.shape
+    if k % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    if not np.all(np.isfinite(w)):
+        raise ValueError("non-finite weight")
+    levels = np.asarray(levels_f32, dtype=np.float32)
+    if levels.shape != (1 << bits,):
+        raise ValueError("codebook size must be 2^bits")
+    wg = w.reshape(n, k // 64, 64)
+    s = np.max(np.abs(wg), axis=2)
+    s_b = np.broadcast_to(s[:, :, None], wg.shape)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s_b > 0, wg / s_b, np.float32(0.0)).astype(np.float32)
+    best_d = np.full(v.shape, np.inf, dtype=np.float32)
+    best_i = np.zeros(v.shape, dtype=np.uint8)
+    for i in range(levels.size):
+        d = np.abs(v - levels[i])
+        take = d < best_d
+        best_i[take] = i
+        best_d[take] = d[take]
+    return best_i.reshape(n, k), (s.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def pack_group64(codes, scale_bits, bits: int) -> np.ndarray:
+    """Layout V2 with 128-byte scale blocks: the codes as pack(); then for
+    unit t = s * G + g the 128 bytes at U * C + 128 t, the first 64 holding
+    the scales of the 64-group k in [128 g, 128 g + 64) and the second 64 those
+    of [128 g + 64, 128 g + 128), each half in the row order of pack()'s
+    64-byte block (row r at byte 2 * (4 * (r % 8) + r // 8))."""
+    q = np.asarray(codes, dtype=np.uint8)
+    n, k = q.shape
+    _check_shape(n, k)
+    sb = np.asarray(scale_bits, dtype=np.uint16)
+    if sb.shape != (n, k // 64):
+        raise ValueError("scales shape mismatch")
+    code_tiles = _pack_codes(q, bits)
+    ns, g = n // STRIP, k // GROUP
+    sc = sb.reshape(ns, 4, 8, g, 2).transpose(0, 3, 4, 2, 1)    # [s, g, half, rq, i]
+    sc_bytes = np.ascontiguousarray(sc).astype("<u2").view(np.uint8).reshape(-1)
+    return np.concatenate([code_tiles.reshape(-1), sc_bytes])
+
+
+def gemv_group64(x, codes, scale_bits, levels_f32) -> np.ndarray:
+    """y[m, n] = sum_h s[n, h] * sum_{k in h} x[m, k] * c[q[n, k]] over the
+    64-groups h, in fp64."""
+    xf = np.asarray(x, dtype=np.float64)
+    q = np.asarray(codes)
+    n, k = q.shape
+    m = xf.shape[0]
+    h = k // 64
+    c = np.asarray(levels_f32, dtype=np.float64)
+    cq = c[q].reshape(n, h, 64)
+    s = bf16_bits_to_f32(scale_bits).astype(np.float64)
+    partial = np.einsum("mhk,nhk->hmn", xf.reshape(m, h, 64), cq)
+    return np.sum(partial * s.T[:, None, :], axis=0)
+
+
 def quantize_tensorscale(w, levels_f32, bits: int) -> Tuple[np.ndarray, np.ndarray]:
     """RTN with one scale for the whole matrix (tensor-wise granularity, the
     comparison baseline of the Log_bQuant abstract): s = max |W| over all

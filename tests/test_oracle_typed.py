@@ -342,3 +342,52 @@ def test_group256_equals_group128_when_both_halves_share_the_max():
     np.testing.assert_array_equal(s2, s1)
     with pytest.raises(ValueError):
         O.quantize_group256(w[:, :384], lv, 4)
+
+
+# ------------------------------------------------------------- group of 64
+
+def test_group64_scales_codes_and_product():
+    w = _weights(32, 256, seed=51)
+    lv = _levels("nf4")
+    codes, sb = O.quantize_group64(w, lv, 4)
+    s = O.bf16_bits_to_f32(sb)
+    np.testing.assert_array_equal(s, np.max(np.abs(w.reshape(32, 4, 64)), axis=2))
+    v = w.astype(np.float64) / np.repeat(s, 64, axis=1).astype(np.float64)
+    d = np.abs(v[..., None] - lv.astype(np.float64))
+    srt = np.sort(d, axis=-1)
+    tie = (srt[..., 1] - srt[..., 0]) < 1e-6
+    assert np.all((codes == np.argmin(d, axis=-1)) | tie)
+    # the product: the library matmul of the dequantized matrix
+    x = O.bf16_round(np.random.default_rng(52).standard_normal((2, 256))).astype(np.float32)
+    wh = lv.astype(np.float64)[codes] * np.repeat(s, 64, axis=1)
+    np.testing.assert_allclose(O.gemv_group64(x, codes, sb, lv), x.astype(np.float64) @ wh.T,
+                               rtol=1e-12, atol=1e-12)
+    # groups of 64 whose two halves share the 128 maximum give the 128 result
+    w2 = w.copy()
+    m = np.max(np.abs(w2.reshape(32, 2, 128)), axis=2)
+    for g in range(2):
+        w2[:, 128 * g + 3] = m[:, g]
+        w2[:, 128 * g + 70] = m[:, g]
+    c64, s64 = O.quantize_group64(w2, lv, 4)
+    c128, s128 = O.quantize(w2, lv, 4)
+    np.testing.assert_array_equal(c64, c128)
+    np.testing.assert_array_equal(s64[:, ::2], s128)
+
+
+def test_pack_group64_hand_derived_scale_bytes():
+    n, k = 64, 256
+    nn, hh = np.meshgrid(np.arange(n), np.arange(4), indexing="ij")
+    sb = (0x3C00 + 8 * nn + hh).astype(np.uint16)
+    p = O.pack_group64(np.zeros((n, k), np.uint8), sb, 4)
+    assert p.size == 8192 + 4 * 128
+    seen = 0
+    with open(os.path.join(GOLDEN, "pack_v2_scales_group64.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            parts = line.split()
+            off = int(parts[0])
+            assert bytes(p[off:off + 2]) == bytes(int(b, 16) for b in parts[1:]), off
+            seen += 1
+    assert seen == 5
+    assert sorted(p[8192:].copy().view("<u2").tolist()) == sorted(sb.reshape(-1).tolist())
