@@ -35,7 +35,12 @@ silent the build's readings are used and stated at each function:
   accumulated in fp64 (every product is exact in fp64).
 * per-group types (BitMoD abstract): up to 4 (4-bit) or 2 (3-bit) codebooks;
   a group takes the type of smallest squared RTN error, summed in fp64 in k
-  order, lowest index on ties.
+  order, lowest index on ties;
+* scale variants: one scale per row (Tetra abstract: the row's absolute
+  maximum, not retrained), one per matrix with an asymmetric linear codebook
+  from min W to max W (the Log_bQuant abstract's baseline), one per 256 or
+  per 64 weights along K; the first three fill every 128-group's slot, so
+  pack() and gemv() serve them unchanged.
 
 Parity of every function here is pinned in ``tests/test_oracle_pins.py``.
 """
