@@ -93,46 +93,82 @@ def ncu_traffic(kernel_key, files):
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clocks and clock-event reasons of one GPU, read through NVML by a
+    thread every 0.5 ms from start() to stop(), plus explicit reads at the
+    edges of the timed region (mark()), so that even a timed region shorter
+    than the polling interval has samples taken while the GPU was busy."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.tmp = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+    def __init__(self, device):
+        import threading
+        self.samples, self.marks, self.reasons = [], [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.handle = None
+        try:
+            import pynvml
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            uuid = str(getattr(torch.cuda.get_device_properties(device), "uuid", ""))
+            try:
+                self.handle = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(int(device))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle,
+                                                                  pynvml.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: report why
+            self.error = f"nvml unavailable: {e}"
+
+    def _read(self):
+        nv = self.nv
+        mhz = float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        for name, const in self.REASONS:
+            if bits & getattr(nv, const, 0):
+                self.reasons.add(name)
+        return mhz
+
+    def _poll(self):
+        import time as _t
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._read())
+            except Exception:
+                pass
+            _t.sleep(0.0005)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.tmp, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+        import threading
+        if self.handle is None:
+            return
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
+
+    def mark(self):
+        if self.handle is not None:
+            try:
+                self.marks.append(self._read())
+            except Exception:
+                pass
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        self.proc.wait()
-        self.tmp.flush()
-        rows = [ln.split(",") for ln in open(self.tmp.name).read().splitlines() if ln.strip()]
-        os.unlink(self.tmp.name)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
-            except (ValueError, IndexError):
-                continue
-            for name, v in zip(names, r[5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": float(np.median(sm)) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [getattr(self, "error", "")],
+                    "samples": 0}
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        allv = self.samples + self.marks
+        busy = [v for v in allv if self.max_mhz and v >= 0.5 * self.max_mhz] or allv
+        return {"sm_mhz": float(np.median(busy)) if busy else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(allv),
+                "edge_mhz": self.marks, "source": "nvml, 0.5 ms polling + reads at the "
+                                                  "timed region's edges"}
 
 
 def dist_setup(args):
@@ -180,12 +216,33 @@ def oracle_sample(lay, kind, bits, m, rows):
 
 
 def oracle_threads():
+    """Threads the oracle's BLAS pool uses (all the cores this process may run on)."""
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
         return max(n) if n else 1
     except Exception:
         return 1
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def limited_threads(n):
+    """A context in which the oracle's BLAS pool uses n threads."""
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=n, user_api="blas")
+    except Exception:
+        import contextlib
+        return contextlib.nullcontext()
 
 
 def time_oracle(lay, kind, bits, m, rows, seconds=None, calls=None):
@@ -222,7 +279,7 @@ def run_reference(args, world, rank):
     el = time.perf_counter() - t0
     gbs = algorithmic_bytes(m, rows, lay.k, args.bits) * args.steps / el / 1e9
     sample = f"{rows} of {lay.n} rows of the layer per step (oracle-quantized), fp64 numpy"
-    cores = oracle_threads()
+    cores = oracle_threads()  # the BLAS pool spans the process's cores
     line = {
         "impl": "reference", "metric": "dequant-fused GEMV HBM GB/s", "value": gbs,
         "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -230,7 +287,8 @@ def run_reference(args, world, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(args, lay),
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu": cpu_model(),
+                         "affinity_cores": len(os.sched_getaffinity(0))},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -246,10 +304,21 @@ def workload_config(args, lay):
 # ---------------------------------------------------------------------- lutq arm
 
 def capture(fn, count):
+    """A CUDA graph of fn(0) .. fn(count - 1), uploaded to the device, so that
+    its first replay does not also pay for moving the graph there."""
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(count):
             fn(i)
+    try:
+        from cuda.bindings import driver as cu
+        err, = cu.cuGraphUpload(cu.CUgraphExec(g.raw_cuda_graph_exec()),
+                                cu.CUstream(torch.cuda.current_stream().cuda_stream))
+        if err != cu.CUresult.CUDA_SUCCESS:
+            raise RuntimeError(str(err))
+        torch.cuda.synchronize()
+    except Exception as e:  # the graph still replays; its first replay uploads it
+        print(f"bench: graph upload skipped ({e})", file=sys.stderr)
     return g
 
 
@@ -472,7 +541,7 @@ def run_lutq(args, world, rank, local):
     w_graph = capture(step, args.warmup) if 0 < args.warmup <= 4096 else None
 
     stream = torch.cuda.current_stream()
-    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
     sampler.start()
     if w_graph is not None:
         w_graph.replay()
@@ -481,6 +550,7 @@ def run_lutq(args, world, rank, local):
             step(i)
     barrier(world)
     torch.cuda.synchronize()
+    sampler.mark()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for _ in range(args.steps // chunk):
@@ -488,12 +558,36 @@ def run_lutq(args, world, rank, local):
     if g_rem is not None:
         g_rem.replay()
     ev1.record(stream)
+    sampler.mark()
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop()
     ms = ev0.elapsed_time(ev1)
     ms = max_over_ranks(world, ms)
     assert int(st.item()) == 0
+    if clocks.get("sm_mhz"):
+        clocks["sm_cycles_per_step"] = ms / args.steps * 1e-3 * clocks["sm_mhz"] * 1e6
+
+    # context for the timed number: one call on an idle GPU (nothing to
+    # overlap its start with), and the per-call time of long graph replays
+    # (steady state: every call's start overlaps the previous call's end)
+    iso = []
+    for i in range(20):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        iso.append(e0.elapsed_time(e1) * 1e3)
+    reps = max(1, min(16, 4096 // chunk))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g_chunk.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    steady_us = e0.elapsed_time(e1) * 1e3 / (reps * chunk)
 
     nbytes = algorithmic_bytes(m, n, k, bits)
     per_step_s = ms / 1e3 / args.steps
@@ -540,10 +634,14 @@ def run_lutq(args, world, rank, local):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(args, lay), parallelism=f"replicas{world}",
-                       launch="cuda_graph",
-                       l2=f"weights rotate over {copies} copies "
-                          f"({copies * per_copy / 1e6:.0f} MB > 3x L2 {l2 / 1e6:.0f} MB)"),
+        "config": workload_config(args, lay),
+        "timing": {"parallelism": f"replicas{world}", "launch": "cuda_graph",
+                   "l2": f"weights rotate over {copies} copies "
+                         f"({copies * per_copy / 1e6:.0f} MB > 3x L2 {l2 / 1e6:.0f} MB); "
+                         "graphs uploaded to the device before the timed region",
+                   "isolated_call_us": float(np.median(iso)),
+                   "steady_state_us": steady_us,
+                   "steady_state_gbs": nbytes / steady_us / 1e3},
         "roofline": {"bound": "hbm", "achieved": gbs_rank, "peak": hbm_peak, "unit": "GB/s",
                      "frac": gbs_rank / hbm_peak, "peak_source": peak_kind,
                      "bytes_per_launch": nbytes, "traffic": ncu_traffic(kernel_key,
@@ -560,11 +658,17 @@ def run_lutq(args, world, rank, local):
     line.update(extra)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         rows = 512
-        gbs_cpu, per_call, calls = time_oracle(lay, args.codebook, bits, m, rows, seconds=10.0)
+        with limited_threads(1):
+            gbs_1, per_call_1, calls_1 = time_oracle(lay, args.codebook, bits, m, rows,
+                                                     seconds=8.0)
+        gbs_cpu, per_call, calls = time_oracle(lay, args.codebook, bits, m, rows, seconds=8.0)
         line["cpu_baseline"] = {
             "value": gbs_cpu, "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
             "sample": f"{rows} of {n} rows (oracle-quantized), {calls} calls of the oracle "
-                      f"product, {per_call * 1e3:.1f} ms each"}
+                      f"product, {per_call * 1e3:.1f} ms each",
+            "single_thread": {"value": gbs_1, "unit": "GB/s", "calls": calls_1,
+                              "ms_per_call": per_call_1 * 1e3},
+            "cpu": cpu_model(), "affinity_cores": len(os.sched_getaffinity(0))}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -43,6 +43,7 @@ _SIGS = {
     "lutq_codebook_asym_linear": (_i32, [ctypes.c_double, ctypes.c_double, _i32, _vp]),
     "lutq_pack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "lutq_workspace_bytes": (_i64, [_i64, _i64, _i64, _i32]),
+    "lutq_workspace_zero_bytes": (_i64, [_i64, _i64, _i64, _i32]),
     "lutq_gemv": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "lutq_gemm": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp]),
     "lutq_gemv_out_bf16": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
@@ -106,6 +107,10 @@ def lutq_packed_bytes(n: int, k: int, bits: int) -> int:
 
 def lutq_workspace_bytes(m: int, n: int, k: int, bits: int) -> int:
     return lib.lutq_workspace_bytes(m, n, k, bits)
+
+
+def lutq_workspace_zero_bytes(m: int, n: int, k: int, bits: int) -> int:
+    return lib.lutq_workspace_zero_bytes(m, n, k, bits)
 
 
 def lutq_gemv_plan(n: int, k: int, num_sms: int) -> dict:

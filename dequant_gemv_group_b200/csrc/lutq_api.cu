@@ -1,6 +1,7 @@
 // C ABI of liblutq: argument checks and kernel launches.  Every argument error
 // is returned before anything is launched; device-side conditions go to the
 // caller's dev_status word.
+#include <algorithm>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -17,11 +18,11 @@ cudaError_t launch_pack(const uint8_t* codes, const void* scales, int64_t N, int
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream,
-                        bool y_bf16 = false);
+                        bool y_bf16 = false, int64_t zero_bytes = -1);
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0,
-                        bool y_bf16 = false);
+                        bool y_bf16 = false, int64_t zero_bytes = -1);
 cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const void* codebook,
                             const int8_t* signs, int bits, int64_t N, int64_t K, float* y,
                             void* workspace, int32_t* dev_status, int num_sms,
@@ -44,7 +45,19 @@ cudaError_t launch_fit_histogram(const void* W, int64_t N, int64_t K, uint64_t* 
                                  int32_t* dev_status, int num_sms, cudaStream_t stream);
 int64_t gemv_workspace_bytes(int64_t M, int64_t N);
 void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out);
-int64_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int64_t gemm_counter_bytes(int64_t M, int64_t N);
+int64_t gemm_scratch_bytes(int64_t M);
+
+// The zero region of the workspace: the larger of the CUDA-core GEMV's
+// exchange slots (M <= 4) and the tensor-core kernel's tile counters.  It
+// does not depend on M up to M = 128 * 128 (the tensor-core kernel's
+// counters grow with the number of 128-row batch tiles), so one workspace
+// serves calls of any batch size up to the one it was sized for.
+int64_t workspace_zero_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)K;
+  const int64_t z = std::max(gemm_counter_bytes(M, N), gemv_workspace_bytes(4, N));
+  return (z + 255) / 256 * 256;
+}
 }  // namespace lutq
 
 namespace {
@@ -191,12 +204,12 @@ lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan) {
 
 int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
   if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK || M < 1) return -1;
-  if (M <= 16) {
-    const int64_t a = lutq::gemv_workspace_bytes(M, N);
-    const int64_t b = lutq::gemm_workspace_bytes(M, N, K);
-    return a > b ? a : b;
-  }
-  return lutq::gemm_workspace_bytes(M, N, K);
+  return lutq::workspace_zero_bytes(M, N, K) + lutq::gemm_scratch_bytes(M);
+}
+
+int64_t lutq_workspace_zero_bytes(int64_t M, int64_t N, int64_t K, int bits) {
+  if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK || M < 1) return -1;
+  return lutq::workspace_zero_bytes(M, N, K);
 }
 
 lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,

@@ -37,6 +37,14 @@ __host__ __device__ constexpr int table_region_bytes(int bits, int types) {
   return types <= (bits == 4 ? 2 : 1) ? 0x10000 : 0x20000;
 }
 
+// Workspace layout of the products (host): every kernel keeps the data that
+// must be zero between calls (exchange slots, arrival counters) at the front,
+// in [0, workspace_zero_bytes), and leaves them zero; scratch that a call
+// may leave as it likes (partial sums) starts at workspace_zero_bytes.  The
+// zero region covers every kernel the problem may take, so one workspace
+// serves lutq_gemv and lutq_gemm calls of the same problem in any order.
+int64_t workspace_zero_bytes(int64_t M, int64_t N, int64_t K);
+
 // Record a device-side error: the first non-zero code wins.
 __device__ __forceinline__ void report(int32_t* dev_status, int code) {
   if (dev_status != nullptr) atomicCAS(dev_status, 0, code);

@@ -341,6 +341,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
           const uint32_t f = (ty >> (2 * (lane >> 3))) & 3u;
           sel = (BITS == 4 ? ((f & 1u) << 7) | ((f >> 1) << 8) : (f & 1u) << 8) &
                 ((BITS == 4 ? 0x080u : 0u) | (LUTB > kLutBytes ? 0x100u : 0u));
+          // a stored type without a table in this call is reported
+          if (f >= uint32_t(a.ntypes)) report(a.dev_status, LUTQ_ERR_CODE_RANGE);
         }
         if (DW == 8)
           decode_group_half<BITS>(reinterpret_cast<uint32_t(&)[32]>(av),
@@ -525,13 +527,17 @@ static int gemm_nt(int64_t M) {
   return 128;
 }
 
-int64_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  (void)K;
-  const int nt = gemm_nt(M);
+// Arrival counters (zero between calls) and split partial sums (scratch).
+int64_t gemm_counter_bytes(int64_t M, int64_t N) {
   const int64_t bt = (M + kTileRows - 1) / kTileRows;
   const int64_t ntiles = (N + kTileRows - 1) / kTileRows;
-  const int64_t counters = (bt * ntiles * 4 * kMaxPromoteGroups * 4 + 255) / 256 * 256;
-  return counters + int64_t(kGemmMaxCtas) * 2 * 4 * nt * 32 * 4;
+  return (bt * ntiles * 4 * kMaxPromoteGroups * 4 + 255) / 256 * 256;
+}
+int64_t gemm_scratch_bytes(int64_t M) {
+  return int64_t(kGemmMaxCtas) * 2 * 4 * gemm_nt(M) * 32 * 4;
+}
+int64_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return workspace_zero_bytes(M, N, K) + gemm_scratch_bytes(M);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -606,7 +612,7 @@ static cudaError_t launch_nts(int nt, const CUtensorMap& map, const GemmArgs& a,
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream, int types,
-                        bool y_bf16) {
+                        bool y_bf16, int64_t zero_bytes) {
   const int nt = gemm_nt(M);
   CUtensorMap map;
   std::memset(&map, 0, sizeof(map));
@@ -630,9 +636,10 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
   a.U = bt * a.ntiles * a.G;
   // unit indices and range arithmetic are 32-bit (U * CTAs < 2^32)
   if (a.U * kGemmMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
-  const int64_t counters = (bt * a.ntiles * 4 * kMaxPromoteGroups * 4 + 255) / 256 * 256;
+  // counters at the front of the workspace, partial sums after its zero region
+  if (zero_bytes < 0) zero_bytes = workspace_zero_bytes(M, N, K);
   a.counters = static_cast<int*>(workspace);
-  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + counters);
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + zero_bytes);
   a.C = 0;
   if (types > 0)
     return bits == 4 ? launch_nts<4, true>(nt, map, a, num_sms, stream)

@@ -687,6 +687,14 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
         lce[i] = lane_e | sel;
         lco[i] = lane_o | sel;
       }
+      if (TYPED) {
+        // a group whose stored type has no table in this call is reported
+        // (its lookups stay inside the allocated tables)
+        const uint32_t T = uint32_t(a.types);
+        if ((ty & 3u) >= T || ((ty >> 2) & 3u) >= T || ((ty >> 4) & 3u) >= T ||
+            ((ty >> 6) & 3u) >= T)
+          report(a.status, LUTQ_ERR_CODE_RANGE);
+      }
       float su[4][M];
       unit_partial<BITS, M>(su, wd, lce, lco, hi_shift, xa, xstride);
 #pragma unroll
@@ -879,7 +887,7 @@ static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0,
-                        bool y_bf16 = false);
+                        bool y_bf16 = false, int64_t zero_bytes = -1);
 
 // Batches up to kMaxSmallBatch run on the CUDA cores when their activations
 // fit the small-batch kernel's shared memory.  Larger batches are a dense
@@ -905,7 +913,8 @@ static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream
 
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
-                        int32_t* dev_status, int num_sms, cudaStream_t stream, bool y_bf16) {
+                        int32_t* dev_status, int num_sms, cudaStream_t stream, bool y_bf16,
+                        int64_t zero_bytes) {
   GemvArgs a;
   a.y_bf16 = y_bf16 ? 1 : 0;
   a.x = static_cast<const uint16_t*>(x);
@@ -925,7 +934,7 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   if (!small_fits(M, K))
     return launch_gemm(x, M, packed, codebook, bits, N, K, y, workspace, dev_status,
-                       num_sms, stream, 0, y_bf16);
+                       num_sms, stream, 0, y_bf16, zero_bytes);
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
                    : launch_bits<3>(a, int(M), num_sms, stream);
 }

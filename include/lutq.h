@@ -211,12 +211,23 @@ lutq_status lutq_pack(const uint8_t* codes, const void* scales_bf16, int64_t N, 
 
 /*
  * lutq_workspace_bytes - device scratch size needed by lutq_gemv / lutq_gemm
- * for this problem (lutq_gemv: one 8-byte exchange slot per output value,
- * where the two halves of a row split between two thread blocks meet;
- * lutq_gemm: split-K partial sums and per-tile arrival counters).
+ * for this problem, whichever kernel runs it: one 8-byte exchange slot per
+ * output value of up to 4 batch rows, where the two halves of a row split
+ * between two thread blocks meet (the CUDA-core GEMV), per-tile arrival
+ * counters and split-K partial sums (the tensor-core kernel).
  * Returns -1 for an invalid argument.  The value does not depend on the device.
  */
 int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
+
+/*
+ * lutq_workspace_zero_bytes - the front part of that workspace which every
+ * lutq_gemv / lutq_gemm call of this problem finds zero at its start and
+ * leaves zero at its end (exchange slots and arrival counters of whichever
+ * kernel runs it); the rest is scratch whose contents do not matter.  A
+ * workspace therefore needs clearing (e.g. cudaMemset of these bytes) only
+ * before its first use.  Returns -1 for an invalid argument.
+ */
+int64_t lutq_workspace_zero_bytes(int64_t M, int64_t N, int64_t K, int bits);
 
 /*
  * lutq_gemv - fused dequantize-and-multiply for small batches, M = 1..16.

@@ -136,7 +136,9 @@ def test_gemv_rht_argument_errors(lq):
     ws = lq.lutq_workspace_bytes(1, 64, 256, 4)
 
     def call(**kw):
-        a = dict(dict(x=A, m=1, p=A, c=A, s=A, bits=4, n=64, k=256, y=A, ws=A, wsb=ws), **kw)
+        a = dict(dict(x=A, m=1, p=A, c=A, s=A, bits=4, n=64, k=256, y=A, ws=A, wsb=None), **kw)
+        if a["wsb"] is None:  # a workspace of the problem's own size
+            a["wsb"] = max(ws, lq.lutq_workspace_bytes(a["m"], a["n"], a["k"], 4))
         return f(a["x"], a["m"], a["p"], a["c"], a["s"], a["bits"], a["n"], a["k"], a["y"],
                  a["ws"], a["wsb"], None, None)
 

@@ -249,6 +249,8 @@ def test_gemv_split_strips(lq, kind, bits, n, k, want_kind, want_align):
     ref_codes, ref_sb = O.quantize(_f32(w[rows]), levels, bits)
     np.testing.assert_array_equal(codes[rows].cpu().numpy(), ref_codes)
     ws = lq.new_workspace(3, n, k, bits)
+    zero = lq.lutq_workspace_zero_bytes(3, n, k, bits)
+    assert zero >= 8 * 3 * n                          # the exchange slots
     for m in (1, 3):
         x = workloads.activations(m, k, seed=31 + m)
         y, _ = _gemv(lq, x, packed, scales, cb, bits, n, k, ws=ws)
@@ -256,7 +258,7 @@ def test_gemv_split_strips(lq, kind, bits, n, k, want_kind, want_align):
         assert O.rel_error_gate(y[:, rows], y_ref) <= TOL, (n, k, m)
         # the exchange slots are clear again (this shape runs on the CUDA
         # cores), and a second call gives the same bits
-        assert int(ws.count_nonzero().item()) == 0
+        assert int(ws[:zero].count_nonzero().item()) == 0
         y2, _ = _gemv(lq, x, packed, scales, cb, bits, n, k, ws=ws)
         np.testing.assert_array_equal(y, y2)
 

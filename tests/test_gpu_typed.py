@@ -55,14 +55,37 @@ def _tables(lq, bits, t):
     return torch.stack(cbs).contiguous().cuda(), levels
 
 
-def _typed_layer(lq, w_cpu, bits, t):
+_ORACLE_CACHE = {}
+
+
+def _oracle_typed(w_cpu, levels, bits, key):
+    """The oracle's codes, scale bits and group types of w; cached under `key`
+    (a case whose weights depend only on the key) when one is given."""
+    if key is None:
+        return O.quantize_typed(_f32(w_cpu), levels, bits)
+    if key not in _ORACLE_CACHE:
+        _ORACLE_CACHE.clear()
+        _ORACLE_CACHE[key] = O.quantize_typed(_f32(w_cpu), levels, bits)
+    return _ORACLE_CACHE[key]
+
+
+def _typed_layer(lq, w_cpu, bits, t, key=None):
+    """Quantize and pack w on the GPU with t types, and check the codes,
+    scales and types against the oracle's, so that every product check below
+    can take the oracle's own quantization as its reference.  Returns the
+    device tables, the oracle's level lists, the GPU's packed matrix and the
+    oracle's (codes, scale bits, types)."""
     cbs, levels = _tables(lq, bits, t)
     st = lq.new_status()
     codes, scales, types = lq.lutq_quantize_typed(w_cpu.cuda(), cbs, bits, status=st)
     packed = lq.lutq_pack_typed(codes, scales, types, bits, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    return cbs, levels, codes, scales, types, packed
+    ref = _oracle_typed(w_cpu, levels, bits, key)
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref[0])
+    np.testing.assert_array_equal(_bits16(scales), ref[1])
+    np.testing.assert_array_equal(types.cpu().numpy(), ref[2])
+    return cbs, levels, codes, scales, types, packed, ref
 
 
 CASES = [(4, 1), (4, 2), (4, 3), (4, 4), (3, 1), (3, 2)]
@@ -74,11 +97,7 @@ def test_quantize_and_pack_typed_bit_exact(lq, bits, t, n, k):
     w = workloads.normal_weights(n, k, 0.02, seed=n + t, outlier_frac=1e-2)
     w[5, 128:256] = 0.0                               # an all-zero group
     w[7, :128] = w[7, :128] * 2.0 ** -120             # subnormal-scaled group
-    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
-    rc, rs, rt = O.quantize_typed(_f32(w), levels, bits)
-    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
-    np.testing.assert_array_equal(_bits16(scales), rs)
-    np.testing.assert_array_equal(types.cpu().numpy(), rt)
+    cbs, levels, codes, scales, types, packed, (rc, rs, rt) = _typed_layer(lq, w, bits, t)
     if t > 1:
         assert len(np.unique(rt)) > 1                 # the case exercises the choice
     np.testing.assert_array_equal(packed.cpu().numpy(), O.pack_typed(rc, rs, rt, bits))
@@ -90,14 +109,14 @@ def test_quantize_and_pack_typed_bit_exact(lq, bits, t, n, k):
 def test_gemv_typed_matches_oracle(lq, bits, t, m, n, k):
     w = workloads.normal_weights(n, k, 0.02, seed=3 * n + t, outlier_frac=1e-2)
     x = workloads.activations(m, k, seed=m + 7)
-    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    cbs, levels, codes, scales, types, packed, (rc, rs, rt) = _typed_layer(
+        lq, w, bits, t, key=("gemv", bits, t, n, k))
     st = lq.new_status()
     y = lq.lutq_gemv_typed(x.cuda(), packed, cbs, bits, n, k,
                            workspace=lq.new_workspace(m, n, k, bits), status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
-                         levels)
+    y_ref = O.gemv_typed(_f32(x), rc, rs, rt, levels)
     assert O.rel_error_gate(y.cpu().numpy(), y_ref) <= TOL
 
 
@@ -105,8 +124,8 @@ def test_gemv_typed_matches_oracle(lq, bits, t, m, n, k):
 def test_gemv_typed_one_hot_is_the_dequantized_weight(lq, bits, t):
     n, k = 256, 1024
     w = workloads.normal_weights(n, k, 0.02, seed=41, outlier_frac=1e-2)
-    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
-    wh = O.dequant_typed(codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(), levels)
+    cbs, levels, codes, scales, types, packed, (rc, rs, rt) = _typed_layer(lq, w, bits, t)
+    wh = O.dequant_typed(rc, rs, rt, levels)
     ws = lq.new_workspace(1, n, k, bits)
     for kk in (0, 129, 1023):
         e = torch.zeros((1, k), dtype=torch.bfloat16)
@@ -155,7 +174,12 @@ def test_gemv_typed_full_size_layer(lq):
     lay = workloads.layer("llama3_8b_w4_nf4", "down")
     n, k = lay.n, lay.k
     w = lay.weights(seed=0)
-    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, 4, 4)
+    cbs, levels = _tables(lq, 4, 4)
+    st = lq.new_status()
+    codes, scales, types = lq.lutq_quantize_typed(w.cuda(), cbs, 4, status=st)
+    packed = lq.lutq_pack_typed(codes, scales, types, 4, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
     x = workloads.activations(1, k, seed=1)
     y = lq.lutq_gemv_typed(x.cuda(), packed, cbs, 4, n, k, workspace=lq.new_workspace(1, n, k, 4))
     torch.cuda.synchronize()
@@ -163,6 +187,7 @@ def test_gemv_typed_full_size_layer(lq):
     rows = np.concatenate([np.arange(32 * s, 32 * s + 32) for s in strips])
     rc, rs, rt = O.quantize_typed(_f32(w[rows]), levels, 4)
     np.testing.assert_array_equal(codes[rows].cpu().numpy(), rc)
+    np.testing.assert_array_equal(_bits16(scales[rows]), rs)
     np.testing.assert_array_equal(types[rows].cpu().numpy(), rt)
     y_ref = O.gemv_typed(_f32(x), rc, rs, rt, levels)
     assert O.rel_error_gate(y.cpu().numpy()[:, rows], y_ref) <= TOL
@@ -178,9 +203,9 @@ def test_typed_tensor_core_path_matches_oracle(lq, bits, t, m, n, k):
     # lutq_gemm_typed both run the tcgen05 kernel with the 128 KB table region
     w = workloads.normal_weights(n, k, 0.02, seed=5 * n + t, outlier_frac=1e-2)
     x = workloads.activations(m, k, seed=m + 11)
-    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
-    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
-                         levels)
+    cbs, levels, codes, scales, types, packed, (rc, rs, rt) = _typed_layer(
+        lq, w, bits, t, key=("tc", bits, t, n, k))
+    y_ref = O.gemv_typed(_f32(x), rc, rs, rt, levels)
     ws = lq.new_workspace(m, n, k, bits)
     st = lq.new_status()
     fns = [lq.lutq_gemm_typed] + ([lq.lutq_gemv_typed] if m <= 16 else [])
@@ -196,14 +221,13 @@ def test_typed_long_rows_take_the_tensor_core_path(lq):
     n, k, bits, t = 64, 128 * 380, 4, 4
     w = workloads.normal_weights(n, k, 0.02, seed=61, outlier_frac=1e-2)
     x = workloads.activations(1, k, seed=62)
-    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    cbs, levels, codes, scales, types, packed, (rc, rs, rt) = _typed_layer(lq, w, bits, t)
     st = lq.new_status()
     y = lq.lutq_gemv_typed(x.cuda(), packed, cbs, bits, n, k,
                            workspace=lq.new_workspace(1, n, k, bits), status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
-                         levels)
+    y_ref = O.gemv_typed(_f32(x), rc, rs, rt, levels)
     assert O.rel_error_gate(y.cpu().numpy(), y_ref) <= TOL
 
 
@@ -211,8 +235,8 @@ def test_typed_long_rows_take_the_tensor_core_path(lq):
 def test_typed_gemm_one_hot_is_the_dequantized_weight(lq, bits, t):
     n, k, m = 256, 1024, 32
     w = workloads.normal_weights(n, k, 0.02, seed=71, outlier_frac=1e-2)
-    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
-    wh = O.dequant_typed(codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(), levels)
+    cbs, levels, codes, scales, types, packed, (rc, rs, rt) = _typed_layer(lq, w, bits, t)
+    wh = O.dequant_typed(rc, rs, rt, levels)
     x = torch.zeros((m, k), dtype=torch.bfloat16)
     cols = (np.arange(m) * 37) % k
     x[np.arange(m), cols] = 1.0
@@ -244,14 +268,13 @@ def test_typed_route_by_table_region(lq, t):
     n, k, m, bits = 256, 14336, 4, 4
     w = workloads.normal_weights(n, k, 0.02, seed=81 + t, outlier_frac=1e-2)
     x = workloads.activations(m, k, seed=82)
-    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t)
+    cbs, levels, codes, scales, types, packed, (rc, rs, rt) = _typed_layer(lq, w, bits, t)
     st = lq.new_status()
     y = lq.lutq_gemv_typed(x.cuda(), packed, cbs, bits, n, k,
                            workspace=lq.new_workspace(m, n, k, bits), status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
-                         levels)
+    y_ref = O.gemv_typed(_f32(x), rc, rs, rt, levels)
     assert O.rel_error_gate(y.cpu().numpy(), y_ref) <= TOL
 
 
@@ -260,21 +283,21 @@ def test_typed_route_by_table_region(lq, t):
 def test_types_beyond_the_count_stay_inside_the_tables(lq, bits, t_data, t_call, m):
     # a matrix quantized with more types than the call passes: the lookups of
     # the extra types are masked to the smaller table region (values
-    # unspecified, every access in bounds); the call and the device stay sound
+    # unspecified, every access in bounds), the call reports
+    # LUTQ_ERR_CODE_RANGE, and the call and the device stay sound
     n, k = 256, 2048
     w = workloads.normal_weights(n, k, 0.02, seed=91, outlier_frac=1e-2)
     x = workloads.activations(m, k, seed=92).cuda()
-    cbs, levels, codes, scales, types, packed = _typed_layer(lq, w, bits, t_data)
+    cbs, levels, codes, scales, types, packed, (rc, rs, rt) = _typed_layer(lq, w, bits, t_data)
     assert int(types.max().item()) >= t_call
     fn = lq.lutq_gemv_typed if m <= 16 else lq.lutq_gemm_typed
     st = lq.new_status()
     fn(x, packed, cbs[:t_call].contiguous(), bits, n, k,
        workspace=lq.new_workspace(m, n, k, bits), status=st)
     torch.cuda.synchronize()
-    assert int(st.item()) == 0
+    assert int(st.item()) == 6                        # LUTQ_ERR_CODE_RANGE
     # the correct call afterwards is still exact
     y = fn(x, packed, cbs, bits, n, k, workspace=lq.new_workspace(m, n, k, bits))
     torch.cuda.synchronize()
-    y_ref = O.gemv_typed(_f32(x), codes.cpu().numpy(), _bits16(scales), types.cpu().numpy(),
-                         levels)
+    y_ref = O.gemv_typed(_f32(x.cpu()), rc, rs, rt, levels)
     assert O.rel_error_gate(y.cpu().numpy(), y_ref) <= TOL

@@ -60,7 +60,13 @@ def _layer(lq, n, k, kind, bits, seed):
     _, levels = O.codebook(kind, bits)
     codes, scales = lq.lutq_quantize(w.cuda(), cb, bits)
     packed = lq.lutq_pack(codes, scales, bits)
-    return cb, levels, codes, scales, packed
+    # the oracle's own quantization of the first rows (at most 256), checked
+    # against the GPU's: the product checks below take it as their reference
+    rows = np.arange(min(n, 256))
+    rc, rs = O.quantize(_f32(w[rows]), levels, bits)
+    np.testing.assert_array_equal(codes[rows].cpu().numpy(), rc)
+    np.testing.assert_array_equal(_bits16(scales[rows]), rs)
+    return cb, levels, (rc, rs), packed
 
 
 # shapes that select each GEMV work plan (whole strips, unit ranges,
@@ -70,7 +76,7 @@ def _layer(lq, n, k, kind, bits, seed):
                                    (320, 4224, 128)])
 @pytest.mark.parametrize("kind,bits", [("nf4", 4), ("lloyd_max3", 3)])
 def test_bf16_output_is_the_fp32_output_rounded(lq, n, k, m, kind, bits):
-    cb, levels, codes, scales, packed = _layer(lq, n, k, kind, bits, seed=n + m)
+    cb, levels, (rc, rs), packed = _layer(lq, n, k, kind, bits, seed=n + m)
     x = workloads.activations(m, k, seed=m).cuda()
     ws = lq.new_workspace(m, n, k, bits)
     st = lq.new_status()
@@ -85,8 +91,7 @@ def test_bf16_output_is_the_fp32_output_rounded(lq, n, k, m, kind, bits):
         assert y16.dtype == torch.bfloat16
         assert torch.equal(y16, y32.to(torch.bfloat16)), bf16_fn.__name__
         if y_ref is None:
-            rows = np.arange(min(n, 256))
-            y_ref = O.gemv(_f32(x), codes[rows].cpu().numpy(), _bits16(scales[rows]), levels)
+            y_ref = O.gemv(_f32(x), rc, rs, levels)
         assert O.rel_error_gate(_f32(y16)[:, :y_ref.shape[1]], y_ref) <= TOL_BF16
 
 
