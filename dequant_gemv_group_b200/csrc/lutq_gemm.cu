@@ -54,7 +54,7 @@ struct GemmCfg {
   static constexpr int XSTAGE = 2 * NT * 128;       // two boxes of NT rows x 128 bytes
   static constexpr int AS = 4;                      // A stages in tensor memory (64 columns each)
   static constexpr int DS = NT >= 128 ? 2 : (NT >= 64 ? 3 : 4);  // partial stages (NT columns)
-  static constexpr int DW = NT >= 128 ? 4 : 8;      // dequant warps (8: two per lane quarter)
+  static constexpr int DW = NT >= 64 ? 4 : 8;       // dequant warps (8: two per lane quarter)
   static constexpr int NB = DW == 8 ? 4 : 2;        // units of packed words in flight per lane
   static constexpr int KC = 64 * 4 / DW;            // A columns written per dequant warp
   static constexpr int PG = NT >= 128 ? 2 : 1;      // promotion warp groups
@@ -180,7 +180,7 @@ __device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t s
 // Position (batch tile, row tile, group) of consecutive units, advanced
 // without divisions.
 struct UnitPos {
-  int64_t bt, tau, g;
+  uint32_t bt, tau, g;
   __device__ void init(uint32_t u, uint32_t per_bt, uint32_t G) {
     const uint32_t b = u / per_bt, r = u - b * per_bt, t = r / G;
     bt = b;
@@ -188,9 +188,9 @@ struct UnitPos {
     g = r - t * G;
   }
   __device__ void next(int64_t G, int64_t ntiles) {
-    if (++g == G) {
+    if (++g == uint32_t(G)) {
       g = 0;
-      if (++tau == ntiles) {
+      if (++tau == uint32_t(ntiles)) {
         tau = 0;
         ++bt;
       }
@@ -326,32 +326,37 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     UnitPos pos;
     pos.init(u0, per_bt, a.G);
     bool ok = true;
+    // the row's table: 4-bit, type bit 0 -> address bit 7 (row half), bit 1
+    // -> bit 16; 3-bit, type bit 0 -> bit 16 (through byte 1 of the column
+    // word), masked to the table region, so that a type >= ntypes reads an
+    // unfilled table inside it, never the activation stages
+    auto sel_of = [&](uint32_t ty) -> uint32_t {
+      if (!TYPED) return 0u;
+      const uint32_t f = (ty >> (2 * (lane >> 3))) & 3u;
+      return (BITS == 4 ? ((f & 1u) << 7) | ((f >> 1) << 8) : (f & 1u) << 8) &
+             ((BITS == 4 ? 0x080u : 0u) | (LUTB > kLutBytes ? 0x100u : 0u));
+    };
     // decode unit i from wd, refill wd with unit i + NB, hand the tile to the MMA
     auto step = [&](uint4 (&wd)[NWL], uint32_t& ty, int i) {
       const bool valid = pos.tau * kTileRows + sw * 32 < a.N;
-      uint32_t av[Cfg::KC];
+      uint32_t av[32];
+      const uint32_t sel = sel_of(ty);
+      // a warp that owns the whole row (DW = 4) decodes it in two halves of
+      // 32 pairs, storing each before decoding the next (32 registers of
+      // pairs live, not 64); the second half's words are kept aside so that
+      // the ring slot is refilled right after the first decode, as early as
+      // with one half
+      uint4 h1[2];
+      if (DW == 4) {
+        h1[0] = wd[BITS == 4 ? 2 : 1];
+        h1[1] = wd[BITS == 4 ? 3 : 2];
+      }
       if (valid) {
-        // the row's table: 4-bit, type bit 0 -> address bit 7 (row half),
-        // bit 1 -> bit 16; 3-bit, type bit 0 -> bit 16 (through byte 1 of
-        // the column word)
-        // (masked to the table region, so that a type >= ntypes reads an
-        // unfilled table inside it, never the activation stages)
-        uint32_t sel = 0;
-        if (TYPED) {
-          const uint32_t f = (ty >> (2 * (lane >> 3))) & 3u;
-          sel = (BITS == 4 ? ((f & 1u) << 7) | ((f >> 1) << 8) : (f & 1u) << 8) &
-                ((BITS == 4 ? 0x080u : 0u) | (LUTB > kLutBytes ? 0x100u : 0u));
-          // a stored type without a table in this call is reported
-          if (f >= uint32_t(a.ntypes)) report(a.dev_status, LUTQ_ERR_CODE_RANGE);
-        }
-        if (DW == 8)
-          decode_group_half<BITS>(reinterpret_cast<uint32_t(&)[32]>(av),
-                                  reinterpret_cast<const uint4(&)[2]>(wd), kh, lut_sa,
-                                  off_e | sel, off_o | sel);
-        else
-          decode_group_row<BITS>(reinterpret_cast<uint32_t(&)[64]>(av),
-                                 reinterpret_cast<const uint4(&)[4]>(wd), lut_sa, off_e | sel,
-                                 off_o | sel);
+        // a stored type without a table in this call is reported
+        if (TYPED && ((ty >> (2 * (lane >> 3))) & 3u) >= uint32_t(a.ntypes))
+          report(a.dev_status, LUTQ_ERR_CODE_RANGE);
+        const uint4 h0[2] = {wd[0], wd[DW == 8 ? 1 : (BITS == 4 ? 1 : 2)]};
+        decode_group_half<BITS>(av, h0, DW == 8 ? kh : 0, lut_sa, off_e | sel, off_o | sel);
       }
       fetch(wd, ty);
       const int as = i % AS;
@@ -363,10 +368,11 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
       tc_fence_after();
       if (valid) {
         const uint32_t ta = tmem + (uint32_t(sw * 32) << 16) + uint32_t(as * 64 + kh * 32);
-        if (DW == 8)
-          tmem_st_cols32(ta, reinterpret_cast<const uint32_t(&)[32]>(av));
-        else
-          tmem_st_32x32b_x64(ta, reinterpret_cast<const uint32_t(&)[64]>(av));
+        tmem_st_cols32(ta, av);
+        if (DW == 4) {
+          decode_group_half<BITS>(av, h1, 1, lut_sa, off_e | sel, off_o | sel);
+          tmem_st_cols32(ta + 32u, av);
+        }
         tmem_wait_st();
       }
       tc_fence_before();

@@ -47,7 +47,8 @@ typedef enum {
   LUTQ_ERR_BITS = 3,        /* bits is not 3 or 4 / does not match the codebook */
   LUTQ_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
   LUTQ_ERR_NONFINITE = 5,   /* device: quantize met a NaN or infinite weight */
-  LUTQ_ERR_CODE_RANGE = 6,  /* device: pack met a code >= 2^bits */
+  LUTQ_ERR_CODE_RANGE = 6,  /* device: pack met a code >= 2^bits, or a typed
+                               product a group type without a table */
   LUTQ_ERR_TIMEOUT = 7,     /* device: a bounded wait inside a kernel expired */
   LUTQ_ERR_CUDA = 8,        /* a CUDA runtime call failed */
   LUTQ_ERR_WORKSPACE = 9    /* workspace missing or smaller than required */
@@ -257,12 +258,15 @@ int64_t lutq_workspace_zero_bytes(int64_t M, int64_t N, int64_t K, int bits);
  * packed   device, layout V2 (lutq_pack): the codes and the scales s.
  * codebook device bf16 [1 << bits].
  * y        device fp32 [M,N] row-major, written (no accumulation into y).
- * workspace device, at least lutq_workspace_bytes(M,N,K,bits) bytes, zero-
- *          filled before its first use (e.g. cudaMemset); every call returns
- *          the slots and counters it relies on to zero, so the next call can
- *          use it as it is.  Calls that may run at the same time on the
- *          GPU must not share a workspace.  May be NULL only if the required
- *          size is 0.
+ * workspace device, at least lutq_workspace_bytes(M,N,K,bits) bytes, whose
+ *          first lutq_workspace_zero_bytes(M,N,K,bits) bytes are zero-filled
+ *          before its first use (e.g. cudaMemset); every call returns the
+ *          slots and counters it relies on to zero, so the next call can use
+ *          it as it is.  The zero part depends on N only (for M up to
+ *          16384), so one workspace serves lutq_gemv and lutq_gemm calls of
+ *          any batch size up to the one it was sized for, in any order.
+ *          Calls that may run at the same time on the GPU must not share a
+ *          workspace.
  * Returns LUTQ_ERR_SHAPE if M is outside 1..16.
  */
 lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
@@ -279,18 +283,24 @@ lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
  * illegal, latency-critical loops that must not call cudaMalloc (it can block
  * and synchronize the device), and plug-in hosts that give a library no
  * allocator.  The scratch that lutq_gemv takes from `workspace` lives here in
- * a fixed library-owned device array of 4 MiB, which every GPU that loads the
- * library holds until the process exits; the call allocates nothing.
- * Arguments other than the workspace, numerics and results are those of
- * lutq_gemv (M = 1..16).
- *  - The first call on a device looks up the array's device address with
- *    that device current; make that first call before any stream capture.
- *  - All calls share the array: calls that may overlap on the GPU (other
- *    streams, other threads) race and must be serialized by the caller.  Each
- *    call first clears the part of the array it uses (an asynchronous memset
- *    on `stream`), so a call never depends on what an earlier one left.
- *  - Returns LUTQ_ERR_WORKSPACE, launching nothing, if the problem's scratch
- *    (8 * M * N bytes, rounded up to 256) exceeds 4 MiB.
+ * a fixed library-owned device array of 8 MiB, which every GPU that loads the
+ * library holds until the process exits; the call allocates nothing.  The
+ * array's first 1 MiB is the zero part of the workspace, the other 7 MiB its
+ * scratch.  Arguments other than the workspace, numerics and results are
+ * those of lutq_gemv (M = 1..16).
+ *  - The first call on a device sets the array up with that device current:
+ *    it looks up the array's device address and clears the array with a
+ *    synchronous cudaMemset.  Make that first call before any stream capture.
+ *  - All calls share the array, which keeps what the last call left: calls
+ *    that may overlap on the GPU (other streams, other threads) race and must
+ *    be serialized by the caller.  Every call leaves the zero part zero and
+ *    no call writes its scratch there, so no call depends on what an earlier
+ *    one left (after a call that reported LUTQ_ERR_TIMEOUT the array's
+ *    contents, and so later results, are unspecified).
+ *  - Returns LUTQ_ERR_WORKSPACE, launching nothing, if
+ *    lutq_workspace_zero_bytes(M,N,K,bits) exceeds 1 MiB (N above 32768) or
+ *    the scratch of the tensor-core kernel the call may take (4 MiB for
+ *    M <= 16) exceeds 7 MiB.
  */
 lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const void* packed,
                               const void* codebook_bf16, int bits, int64_t N, int64_t K,
@@ -461,10 +471,11 @@ lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
  *   take 64 KB of shared memory for up to two 4-bit types or one 3-bit type,
  *   128 KB otherwise; the CUDA-core kernel runs M = 1..4 with
  *   M * (K + 2048) <= 80896 (64 KB of tables) or <= 48128 (128 KB), other
- *   products go to the tensor-core kernel (as lutq_gemm_typed).  `types` must be the count the
- *   matrix was quantized with: a stored type >= types reads a table that is
- *   not filled (unspecified values, no out-of-bounds access).  Other
- *   arguments, workspace and errors as lutq_gemv.
+ *   products go to the tensor-core kernel (as lutq_gemm_typed).  `types` must
+ *   be the count the matrix was quantized with: a group whose stored type is
+ *   >= types reads a table that is not filled (unspecified values, no
+ *   out-of-bounds access) and the call reports LUTQ_ERR_CODE_RANGE through
+ *   dev_status.  Other arguments, workspace and errors as lutq_gemv.
  * lutq_gemm_typed: the same product on the tensor cores (any M >= 1), as
  *   lutq_gemm.
  * All are asynchronous on `stream`; pointers 16-byte aligned.
