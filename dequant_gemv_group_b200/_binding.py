@@ -59,6 +59,13 @@ _SIGS = {
     "lutq_rht_activations": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "lutq_gemv_rht": (_i32, [_vp, _i64, _vp, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
                              _vp]),
+    "lutq_packed_bytes_group64": (_i64, [_i64, _i64, _i32]),
+    "lutq_quantize_group64": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "lutq_pack_group64": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "lutq_gemv_group64": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
+                                 _vp]),
+    "lutq_gemm_group64": (_i32, [_vp, _i64, _vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp,
+                                 _vp]),
     "lutq_max_types": (_i32, [_i32]),
     "lutq_packed_bytes_typed": (_i64, [_i64, _i64, _i32]),
     "lutq_quantize_typed": (_i32, [_vp, _i64, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
@@ -307,6 +314,57 @@ def lutq_gemv_rht(x, packed, codebook, signs, bits, n, k, y=None, workspace=None
                              signs.data_ptr(), bits, n, k, y.data_ptr(), ws_ptr, ws_bytes,
                              _ptr(status), _stream()), "lutq_gemv_rht")
     return y
+
+
+def lutq_packed_bytes_group64(n: int, k: int, bits: int) -> int:
+    return int(lib.lutq_packed_bytes_group64(n, k, bits))
+
+
+def lutq_quantize_group64(w: torch.Tensor, codebook: torch.Tensor, bits: int,
+                          status: Optional[torch.Tensor] = None
+                          ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """W bf16 [N, K] -> (codes uint8 [N, K], scales bf16 [N, K/64]): one
+    scale per group of 64 (see lutq_quantize_group64 in include/lutq.h)."""
+    _need(w, torch.bfloat16, "W")
+    _need(codebook, torch.bfloat16, "codebook")
+    n, k = w.shape
+    codes = torch.empty((n, k), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((n, max(k // 64, 1)), dtype=torch.bfloat16, device=w.device)
+    _check(lib.lutq_quantize_group64(w.data_ptr(), n, k, codebook.data_ptr(), bits,
+                                     codes.data_ptr(), scales.data_ptr(), _ptr(status),
+                                     _stream()), "lutq_quantize_group64")
+    return codes, scales
+
+
+def lutq_pack_group64(codes: torch.Tensor, scales: torch.Tensor, bits: int,
+                      status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """codes uint8 [N, K] and scales bf16 [N, K/64] -> the packed matrix with
+    128-byte scale blocks."""
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.bfloat16, "scales")
+    n, k = codes.shape
+    if tuple(scales.shape) != (n, k // 64):
+        raise LutqError(2, "lutq_pack_group64: scales shape")
+    nb = lutq_packed_bytes_group64(n, k, bits)
+    if nb < 0:
+        raise LutqError(2, "lutq_packed_bytes_group64")
+    packed = torch.empty(nb, dtype=torch.uint8, device=codes.device)
+    _check(lib.lutq_pack_group64(codes.data_ptr(), scales.data_ptr(), n, k, bits,
+                                 packed.data_ptr(), _ptr(status), _stream()),
+           "lutq_pack_group64")
+    return packed
+
+
+def lutq_gemv_group64(x, packed, codebook, bits, n, k, y=None, workspace=None, status=None):
+    """y[M, N] (fp32) with one scale per group of 64 (M = 1..16)."""
+    return _product(lib.lutq_gemv_group64, "lutq_gemv_group64", x, packed, codebook, bits, n, k,
+                    y, workspace, status)
+
+
+def lutq_gemm_group64(x, packed, codebook, bits, n, k, y=None, workspace=None, status=None):
+    """The group-64 product on the tensor cores (any M >= 1)."""
+    return _product(lib.lutq_gemm_group64, "lutq_gemm_group64", x, packed, codebook, bits, n, k,
+                    y, workspace, status)
 
 
 def lutq_max_types(bits: int) -> int:

@@ -14,15 +14,15 @@ cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* cod
                             cudaStream_t stream, int scope = 0);
 cudaError_t launch_pack(const uint8_t* codes, const void* scales, int64_t N, int64_t K,
                         int bits, void* packed, int32_t* dev_status, int num_sms,
-                        cudaStream_t stream);
+                        cudaStream_t stream, bool group64 = false);
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream,
-                        bool y_bf16 = false, int64_t zero_bytes = -1);
+                        bool y_bf16 = false, int64_t zero_bytes = -1, bool group64 = false);
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0,
-                        bool y_bf16 = false, int64_t zero_bytes = -1);
+                        bool y_bf16 = false, int64_t zero_bytes = -1, bool group64 = false);
 cudaError_t launch_gemv_rht(const void* x, int64_t M, const void* packed, const void* codebook,
                             const int8_t* signs, int bits, int64_t N, int64_t K, float* y,
                             void* workspace, int32_t* dev_status, int num_sms,
@@ -181,8 +181,15 @@ lutq_status lutq_quantize_tensorscale(const void* W_bf16, int64_t N, int64_t K,
   return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 2);
 }
 
-lutq_status lutq_pack(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
-                      int bits, void* packed, int32_t* dev_status, void* stream) {
+lutq_status lutq_quantize_group64(const void* W_bf16, int64_t N, int64_t K,
+                                  const void* codebook_bf16, int bits, uint8_t* codes,
+                                  void* scales_bf16, int32_t* dev_status, void* stream) {
+  return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 4);
+}
+
+static lutq_status pack(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
+                        int bits, void* packed, int32_t* dev_status, void* stream,
+                        bool group64) {
   if (!codes || !scales_bf16 || !packed) return LUTQ_ERR_INVALID_ARG;
   lutq_status st = check_bits(bits);
   if (st != LUTQ_OK) return st;
@@ -191,7 +198,24 @@ lutq_status lutq_pack(const uint8_t* codes, const void* scales_bf16, int64_t N, 
   int sms = 0;
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_pack(codes, scales_bf16, N, K, bits, packed, dev_status, sms,
-                                     static_cast<cudaStream_t>(stream)));
+                                     static_cast<cudaStream_t>(stream), group64));
+}
+
+lutq_status lutq_pack(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
+                      int bits, void* packed, int32_t* dev_status, void* stream) {
+  return pack(codes, scales_bf16, N, K, bits, packed, dev_status, stream, false);
+}
+
+int64_t lutq_packed_bytes_group64(int64_t N, int64_t K, int bits) {
+  if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK) return -1;
+  return (N / lutq::kStrip) * (K / lutq::kGroup) *
+         (lutq::tile_bytes(bits) + 2 * lutq::kScaleBytes);
+}
+
+lutq_status lutq_pack_group64(const uint8_t* codes, const void* scales_bf16, int64_t N,
+                              int64_t K, int bits, void* packed, int32_t* dev_status,
+                              void* stream) {
+  return pack(codes, scales_bf16, N, K, bits, packed, dev_status, stream, true);
 }
 
 lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan) {
@@ -268,6 +292,36 @@ lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
   if ((st = current_sms(&sms)) != LUTQ_OK) return st;
   return from_cuda(lutq::launch_gemm(x_bf16, M, packed, codebook_bf16, bits, N, K, y, workspace,
                                      dev_status, sms, static_cast<cudaStream_t>(stream)));
+}
+
+lutq_status lutq_gemv_group64(const void* x_bf16, int64_t M, const void* packed,
+                              const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
+                              void* workspace, int64_t workspace_bytes, int32_t* dev_status,
+                              void* stream) {
+  lutq_status st = check_product_args(x_bf16, M, 16, packed, codebook_bf16, bits, N, K, y,
+                                      workspace, workspace_bytes,
+                                      lutq_workspace_bytes(M, N, K, bits));
+  if (st != LUTQ_OK) return st;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_gemv(x_bf16, M, packed, codebook_bf16, bits, N, K, y, workspace,
+                                     dev_status, sms, static_cast<cudaStream_t>(stream), false,
+                                     -1, true));
+}
+
+lutq_status lutq_gemm_group64(const void* x_bf16, int64_t M, const void* packed,
+                              const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
+                              void* workspace, int64_t workspace_bytes, int32_t* dev_status,
+                              void* stream) {
+  lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, codebook_bf16, bits,
+                                      N, K, y, workspace, workspace_bytes,
+                                      lutq_workspace_bytes(M, N, K, bits));
+  if (st != LUTQ_OK) return st;
+  int sms = 0;
+  if ((st = current_sms(&sms)) != LUTQ_OK) return st;
+  return from_cuda(lutq::launch_gemm(x_bf16, M, packed, codebook_bf16, bits, N, K, y, workspace,
+                                     dev_status, sms, static_cast<cudaStream_t>(stream), 0, false,
+                                     -1, true));
 }
 
 static lutq_status rht(const void* in, int64_t rows, int64_t K, const int8_t* signs, void* out,

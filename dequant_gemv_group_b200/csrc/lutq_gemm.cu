@@ -20,6 +20,9 @@
 //              10 take alternate units) kind::f16 (A from tensor memory, B from
 //              shared memory, D fp32 in tensor memory), 8 MMAs of K = 16 per
 //              group into a fresh partial, and commits to the mbarriers.
+// With one scale per group of 64 (G64) each unit has two partials, one per
+// 64-half (MMAs 0-3 and 4-7, each into its own partial stage), and the
+// promotion warps add s[row, 2g] * first + s[row, 2g + 1] * second.
 // Products are exact (bf16 x bf16) and every group's partial is rescaled in
 // fp32, so the result matches the fp32-accumulating GEMV up to summation order.
 //
@@ -70,7 +73,8 @@ constexpr int kScaleRingBytes = 4 * kMaxPromoteGroups * 4 * 32 * 4;  // [warp][S
 
 struct GemmArgs {
   const uint8_t* packed;
-  const uint8_t* scales;    // the packed matrix's scale blocks (layout V2)
+  const uint8_t* scales;    // the packed matrix's scale blocks (layout V2; 128 bytes per
+                            // unit with one scale per group of 64)
   const uint8_t* types;     // per-group data types: the type blocks (else unused)
   const uint16_t* codebook; // [types][2^BITS] with per-group types
   int ntypes;               // tables in `codebook` (1 without per-group types)
@@ -211,10 +215,14 @@ __device__ __forceinline__ void tmem_st_cols32(uint32_t taddr, const uint32_t (&
       : "memory");
 }
 
-template <int BITS, int NT, bool TYPED>
+template <int BITS, int NT, bool TYPED, bool G64>
 __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, GemmArgs a) {
   using Cfg = GemmCfg<NT>;
+  static_assert(!(TYPED && G64), "per-group types use one scale per group of 128");
+  // partials per unit (one per scale), the scale block's bytes
+  constexpr int H = G64 ? 2 : 1;
+  constexpr int SBB = H * kScaleBytes;
   constexpr int TB = tile_bytes(BITS);
   constexpr int WPR = words_per_row(BITS);
   constexpr int XS = Cfg::XS, AS = Cfg::AS, DS = Cfg::DS, DW = Cfg::DW;
@@ -393,23 +401,27 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     UnitPos cur;
     cur.init(u0, per_bt, a.G);
     // The group scales of the next SD units travel ahead of use through a
-    // ring in shared memory (one 4-byte asynchronous copy per lane and unit,
-    // one copy group per unit): waiting for unit i's group never waits for a
+    // ring in shared memory (one 4-byte asynchronous copy per lane, unit and
+    // scale, one copy group per unit): waiting for unit i's group never waits for a
     // later unit's load.  Holding the ring in registers and shifting it made
     // every unit wait for the load issued one unit before (a global-load
     // latency per unit).
     constexpr int SD = 4;
     UnitPos pf = cur;
-    const uint32_t ring = bar_sa + 512u + uint32_t((warp - DW) * SD * 32 * 4);
+    // ring slot d: H words per lane (its scale of each 64-half with G64)
+    const uint32_t ring = bar_sa + 512u + uint32_t((warp - DW) * SD * H * 32 * 4);
     const uint32_t half = uint32_t(scale_slot(lane) >> 1) & 1u;  // which bf16 of the word
     auto issue_scale = [&](const UnitPos& p, int slot, bool live) {
       const int64_t r0 = p.tau * kTileRows + sw * 32;
       if (live && r0 < a.N) {
         const uint8_t* b =
-            a.scales + ((r0 / kStrip) * a.G + p.g) * kScaleBytes + (scale_slot(lane) & ~3);
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
-                     ::"r"(ring + uint32_t((slot * 32 + lane) * 4)), "l"(b)
-                     : "memory");
+            a.scales + ((r0 / kStrip) * a.G + p.g) * SBB + (scale_slot(lane) & ~3);
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
+                       ::"r"(ring + uint32_t(((slot * H + h) * 32 + lane) * 4)),
+                       "l"(b + h * kScaleBytes)
+                       : "memory");
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
     };
@@ -425,28 +437,37 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
       const int64_t row = cur.tau * kTileRows + sw * 32 + lane;
       const bool valid = cur.tau * kTileRows + sw * 32 < a.N;
       asm volatile("cp.async.wait_group %0;" ::"n"(SD - 1) : "memory");
-      const uint32_t sw2 = lds32(ring + uint32_t(((i % SD) * 32 + lane) * 4));
-      const float s = half ? bf16_hi_to_f32(sw2) : bf16_lo_to_f32(sw2);
+      float s[H];
+#pragma unroll
+      for (int h = 0; h < H; ++h) {
+        const uint32_t sw2 = lds32(ring + uint32_t((((i % SD) * H + h) * 32 + lane) * 4));
+        s[h] = half ? bf16_hi_to_f32(sw2) : bf16_lo_to_f32(sw2);
+      }
       issue_scale(pf, i % SD, i + SD < n);
       pf.next(a.G, a.ntiles);
-      const int ds = i % DS;
-      const bool ok = mbar_wait(bar(B_DF + ds), uint32_t(i / DS) & 1u, abort_flag, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      constexpr int CH = chunk_cols<NC>();
 #pragma unroll
-      for (int c = 0; c < NC / CH; ++c) {
-        uint32_t v[32];
-        tmem_ld_cols<NC>(tmem + (uint32_t(sw * 32) << 16) +
-                             uint32_t(Cfg::DCOL + ds * NT + pg * NC + c * CH),
-                         v);
-        tmem_wait_ld();
+      for (int h = 0; h < H; ++h) {
+        const int d = i * H + h, ds = d % DS;  // partial d of the sequence
+        const bool ok =
+            mbar_wait(bar(B_DF + ds), uint32_t(d / DS) & 1u, abort_flag, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) goto promote_done;
+        tc_fence_after();
+        constexpr int CH = chunk_cols<NC>();
 #pragma unroll
-        for (int j = 0; j < CH; ++j) acc[c * CH + j] = fmaf(s, __uint_as_float(v[j]), acc[c * CH + j]);
+        for (int c = 0; c < NC / CH; ++c) {
+          uint32_t v[32];
+          tmem_ld_cols<NC>(tmem + (uint32_t(sw * 32) << 16) +
+                               uint32_t(Cfg::DCOL + ds * NT + pg * NC + c * CH),
+                           v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < CH; ++j)
+            acc[c * CH + j] = fmaf(s[h], __uint_as_float(v[j]), acc[c * CH + j]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_DE + ds));
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_DE + ds));
       if (cur.g == a.G - 1 || i == n - 1) {
         if (valid)
           gemm_finish_strip<NT, NC>(a, acc, cur.bt * a.ntiles + cur.tau, cur.bt, row, sw, pg, u0,
@@ -456,6 +477,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
       }
       cur.next(a.G, a.ntiles);
     }
+  promote_done:
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == W_XLOAD) {
     if (lane == 0) {
@@ -488,25 +510,35 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     // faster).  Each commits its own MMAs.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, NT);
-      int issued = -1;
+      int issued = -1;  // the last partial d committed
       for (int i = warp - W_MMA; i < n; i += MW) {
-        const int xs = i % XS, as = i % AS, ds = i % DS;
+        const int xs = i % XS, as = i % AS;
         if (!mbar_wait(bar(B_XF + xs), uint32_t(i / XS) & 1u, abort_flag, kWaitLimitNs)) break;
         if (!mbar_wait(bar(B_AF + as), uint32_t(i / AS) & 1u, abort_flag, kWaitLimitNs)) break;
-        if (!mbar_wait(bar(B_DE + ds), (uint32_t(i / DS) & 1u) ^ 1u, abort_flag, kWaitLimitNs))
-          break;
-        tc_fence_after();
         const uint32_t xb = xst_sa + uint32_t(xs * Cfg::XSTAGE);
+        bool ok = true;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t b_sa = xb + uint32_t((kk >> 2) * (NT * 128) + (kk & 3) * 32);
-          mma_bf16_ts(tmem + uint32_t(Cfg::DCOL + ds * NT), tmem + uint32_t(as * 64 + 8 * kk),
-                      smem_desc_k_sw128(b_sa), idesc, kk > 0 ? 1u : 0u);
+        for (int h = 0; h < H; ++h) {
+          // partial d = i H + h: MMAs 8h/H .. 8(h+1)/H - 1 of the unit
+          const int d = i * H + h, ds = d % DS;
+          if (!mbar_wait(bar(B_DE + ds), (uint32_t(d / DS) & 1u) ^ 1u, abort_flag,
+                         kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = h * (8 / H); kk < (h + 1) * (8 / H); ++kk) {
+            const uint32_t b_sa = xb + uint32_t((kk >> 2) * (NT * 128) + (kk & 3) * 32);
+            mma_bf16_ts(tmem + uint32_t(Cfg::DCOL + ds * NT), tmem + uint32_t(as * 64 + 8 * kk),
+                        smem_desc_k_sw128(b_sa), idesc, kk > h * (8 / H) ? 1u : 0u);
+          }
+          mma_commit(bar(B_DF + ds));
+          issued = d;
         }
-        mma_commit(bar(B_DF + ds));
+        if (!ok) break;
         mma_commit(bar(B_AE + as));
         mma_commit(bar(B_XE + xs));
-        issued = i;
       }
       if (*abort_flag && issued >= 0) mbar_drain(bar(B_DF + issued % DS), uint32_t(issued / DS) & 1u);
     }
@@ -579,46 +611,49 @@ static cudaError_t make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BITS, int NT, bool TYPED>
+template <int BITS, int NT, bool TYPED, bool G64>
 static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
                              cudaStream_t stream) {
   using Cfg = GemmCfg<NT>;
   static int granted[64] = {0};
   // alignment slack, table, activation stages, barriers and flags (512),
-  // the promotion warps' scale rings
-  const int smem = 1024 + a.lut_bytes + Cfg::XS * Cfg::XSTAGE + 512 + kScaleRingBytes;
+  // the promotion warps' scale rings (two scales per lane and unit with G64)
+  const int smem =
+      1024 + a.lut_bytes + Cfg::XS * Cfg::XSTAGE + 512 + kScaleRingBytes * (G64 ? 2 : 1);
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (granted[dev] < smem) {
-    err = cudaFuncSetAttribute(gemm_kernel<BITS, NT, TYPED>,
+    err = cudaFuncSetAttribute(gemm_kernel<BITS, NT, TYPED, G64>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     granted[dev] = smem;
   }
   a.C = int(std::min<int64_t>(std::min<int64_t>(num_sms, kGemmMaxCtas), a.U));
-  gemm_kernel<BITS, NT, TYPED><<<unsigned(a.C), Cfg::THREADS, smem, stream>>>(map, a);
+  gemm_kernel<BITS, NT, TYPED, G64><<<unsigned(a.C), Cfg::THREADS, smem, stream>>>(map, a);
   return cudaGetLastError();
 }
 
-template <int BITS, bool TYPED>
+template <int BITS, bool TYPED, bool G64 = false>
 static cudaError_t launch_nts(int nt, const CUtensorMap& map, const GemmArgs& a, int num_sms,
                               cudaStream_t stream) {
   switch (nt) {
-    case 16: return launch_nt<BITS, 16, TYPED>(map, a, num_sms, stream);
-    case 32: return launch_nt<BITS, 32, TYPED>(map, a, num_sms, stream);
-    case 64: return launch_nt<BITS, 64, TYPED>(map, a, num_sms, stream);
-    default: return launch_nt<BITS, 128, TYPED>(map, a, num_sms, stream);
+    case 16: return launch_nt<BITS, 16, TYPED, G64>(map, a, num_sms, stream);
+    case 32: return launch_nt<BITS, 32, TYPED, G64>(map, a, num_sms, stream);
+    case 64: return launch_nt<BITS, 64, TYPED, G64>(map, a, num_sms, stream);
+    default: return launch_nt<BITS, 128, TYPED, G64>(map, a, num_sms, stream);
   }
 }
 
 // types = 0: one codebook; 1..max_types(bits): per-group data types (the
 // packed matrix carries its type blocks and `codebook` holds `types` tables).
+// group64: the packed matrix has 128-byte scale blocks (one scale per group
+// of 64; types must be 0).
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream, int types,
-                        bool y_bf16, int64_t zero_bytes) {
+                        bool y_bf16, int64_t zero_bytes, bool group64) {
   const int nt = gemm_nt(M);
   CUtensorMap map;
   std::memset(&map, 0, sizeof(map));
@@ -647,6 +682,11 @@ cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void
   a.counters = static_cast<int*>(workspace);
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + zero_bytes);
   a.C = 0;
+  if (group64) {
+    if (types > 0) return cudaErrorInvalidValue;
+    return bits == 4 ? launch_nts<4, false, true>(nt, map, a, num_sms, stream)
+                     : launch_nts<3, false, true>(nt, map, a, num_sms, stream);
+  }
   if (types > 0)
     return bits == 4 ? launch_nts<4, true>(nt, map, a, num_sms, stream)
                      : launch_nts<3, true>(nt, map, a, num_sms, stream);

@@ -473,12 +473,16 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 }
 
 // TREG: 0 without per-group data types; 1 or 2 with them, the table region
-// being TREG x 64 KB (table_region_bytes).
-template <int BITS, int M, int NB, int TREG>
+// being TREG x 64 KB (table_region_bytes).  SB: bytes of a unit's scale
+// block, 64 (one scale per group of 128) or 128 (one per group of 64: the
+// lane's 32 codes lie in 64-group q >> 1, whose scales are the block's
+// half q >> 1).
+template <int BITS, int M, int NB, int TREG, int SB = kScaleBytes>
 __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a) {
   constexpr bool TYPED = TREG > 0;
+  static_assert(SB == kScaleBytes || !TYPED, "per-group types use 64-byte scale blocks");
   constexpr int TB = tile_bytes(BITS);
-  constexpr int UB = TB + kScaleBytes + (TYPED ? kTypeBytes : 0);  // packed bytes per unit
+  constexpr int UB = TB + SB + (TYPED ? kTypeBytes : 0);  // packed bytes per unit
   constexpr uint32_t kLutRegion = TREG == 2 ? 0x20000u : 0x10000u;
   constexpr uint32_t kXAt = kLutAt + kLutRegion;
   // Table-select bits a lookup may use: with one 64 KB region only the row
@@ -521,8 +525,10 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
   const uint32_t lane_off = lane_tile_offset<BITS>(q, rq);
   const uint32_t hi_delta = BITS == 3 ? lane_hi_delta(q) : 0u;
   const uint8_t* const pk = a.packed + lane_off;
-  // the scales of the lane's rows rq + 8 i, i = 0..3: 8 bytes of each unit's 64
-  const uint8_t* const psc = a.packed + uint64_t(a.U) * TB + scale_slot(rq);
+  // the scales of the lane's rows rq + 8 i, i = 0..3: 8 bytes of each unit's
+  // 64 (of the half of the 128 that holds the lane's 64-group)
+  const uint8_t* const psc =
+      a.packed + uint64_t(a.U) * TB + scale_slot(rq) + (SB > kScaleBytes ? 64 * (q >> 1) : 0);
   // per-group types: byte rq of each unit's 8 (rows rq + 8 i in bits 2i+1:2i)
   const uint8_t* const pty = a.packed + uint64_t(a.U) * (TB + kScaleBytes) + rq;
 
@@ -538,7 +544,8 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
         const uint8_t* p = wide_addr(pk, t, uint32_t(TB));
 #pragma unroll
         for (int i = 0; i < 4; ++i) prefetch_l2(p + 128 * i);
-        if (lane == 0) prefetch_l2(wide_addr(psc, t, uint32_t(kScaleBytes)));
+        if (lane == 0 || (SB > kScaleBytes && lane == 16))
+          prefetch_l2(wide_addr(psc, t, uint32_t(SB)));
         if (TYPED && lane == 0) prefetch_l2(wide_addr(pty, t, uint32_t(kTypeBytes)));
       }
       ++t;
@@ -560,7 +567,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 
   auto fetch = [&](uint4 (&wd)[4], uint32_t (&sv)[2], uint32_t& ty) {
     fetch_unit<BITS>(wd, sv, wide_addr(pk, ft, TB), hi_delta,
-                     wide_addr(psc, ft, uint32_t(kScaleBytes)), fn);
+                     wide_addr(psc, ft, uint32_t(SB)), fn);
     if (TYPED) fetch_type_byte(ty, wide_addr(pty, ft, uint32_t(kTypeBytes)), fn);
     --fn;
     ++ft;
@@ -838,8 +845,8 @@ void gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* out) {
 // leaves free.
 constexpr int64_t kPrefetchBytes = int64_t(64) << 20;
 
-static void apply_plan(GemvArgs& a, int num_sms, int bits) {
-  const int64_t unit_bytes = tile_bytes(bits) + kScaleBytes + (a.types > 0 ? kTypeBytes : 0);
+static void apply_plan(GemvArgs& a, int num_sms, int bits, int sb) {
+  const int64_t unit_bytes = tile_bytes(bits) + sb + (a.types > 0 ? kTypeBytes : 0);
   const Plan pl = choose_plan(a.N / kStrip, a.G, num_sms);
   a.C = pl.C;
   a.kind = pl.kind;
@@ -857,16 +864,16 @@ static int64_t small_smem(int64_t K, int M, int lut_bytes) {
                                 : int64_t(1) << 30;
 }
 
-template <int BITS, int M, int TREG>
+template <int BITS, int M, int TREG, int SB = kScaleBytes>
 static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
   constexpr bool TYPED = TREG > 0;
   static SmemGrant grant2, grant3;
   const int smem = int(small_smem(a.K, M, TREG == 2 ? 0x20000 : 0x10000));
-  apply_plan(a, num_sms, BITS);
+  apply_plan(a, num_sms, BITS, SB);
   constexpr int kDeep = M == 1 && !TYPED ? 3 : 2;
   const bool deep = M == 1 && !TYPED && a.pf_ctas == 0;
-  auto kernel = deep ? gemv_small_kernel<BITS, M, kDeep, TREG>
-                     : gemv_small_kernel<BITS, M, 2, TREG>;
+  auto kernel = deep ? gemv_small_kernel<BITS, M, kDeep, TREG, SB>
+                     : gemv_small_kernel<BITS, M, 2, TREG, SB>;
   cudaError_t err = grant_smem(kernel, deep ? grant3 : grant2, smem);
   if (err != cudaSuccess) return err;
   // programmatic dependent launch: the prefetching blocks and the work
@@ -887,7 +894,7 @@ static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
 cudaError_t launch_gemm(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream, int types = 0,
-                        bool y_bf16 = false, int64_t zero_bytes = -1);
+                        bool y_bf16 = false, int64_t zero_bytes = -1, bool group64 = false);
 
 // Batches up to kMaxSmallBatch run on the CUDA cores when their activations
 // fit the small-batch kernel's shared memory.  Larger batches are a dense
@@ -901,20 +908,20 @@ static bool small_fits(int64_t M, int64_t K, int lut_bytes = 0x10000) {
          small_smem(K, int(M), lut_bytes) <= kMaxSmemPerBlock - 1024;
 }
 
-template <int BITS, int TREG = 0>
+template <int BITS, int TREG = 0, int SB = kScaleBytes>
 static cudaError_t launch_bits(const GemvArgs& a, int M, int num_sms, cudaStream_t s) {
   switch (M) {
-    case 1: return launch_small<BITS, 1, TREG>(a, num_sms, s);
-    case 2: return launch_small<BITS, 2, TREG>(a, num_sms, s);
-    case 3: return launch_small<BITS, 3, TREG>(a, num_sms, s);
-    default: return launch_small<BITS, 4, TREG>(a, num_sms, s);
+    case 1: return launch_small<BITS, 1, TREG, SB>(a, num_sms, s);
+    case 2: return launch_small<BITS, 2, TREG, SB>(a, num_sms, s);
+    case 3: return launch_small<BITS, 3, TREG, SB>(a, num_sms, s);
+    default: return launch_small<BITS, 4, TREG, SB>(a, num_sms, s);
   }
 }
 
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream, bool y_bf16,
-                        int64_t zero_bytes) {
+                        int64_t zero_bytes, bool group64) {
   GemvArgs a;
   a.y_bf16 = y_bf16 ? 1 : 0;
   a.x = static_cast<const uint16_t*>(x);
@@ -934,7 +941,10 @@ cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void
   if (a.U * kMaxCtas >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   if (!small_fits(M, K))
     return launch_gemm(x, M, packed, codebook, bits, N, K, y, workspace, dev_status,
-                       num_sms, stream, 0, y_bf16, zero_bytes);
+                       num_sms, stream, 0, y_bf16, zero_bytes, group64);
+  if (group64)
+    return bits == 4 ? launch_bits<4, 0, 2 * kScaleBytes>(a, int(M), num_sms, stream)
+                     : launch_bits<3, 0, 2 * kScaleBytes>(a, int(M), num_sms, stream);
   return bits == 4 ? launch_bits<4>(a, int(M), num_sms, stream)
                    : launch_bits<3>(a, int(M), num_sms, stream);
 }

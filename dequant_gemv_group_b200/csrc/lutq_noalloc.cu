@@ -32,7 +32,7 @@ namespace lutq {
 cudaError_t launch_gemv(const void* x, int64_t M, const void* packed, const void* codebook,
                         int bits, int64_t N, int64_t K, float* y, void* workspace,
                         int32_t* dev_status, int num_sms, cudaStream_t stream,
-                        bool y_bf16 = false, int64_t zero_bytes = -1);
+                        bool y_bf16 = false, int64_t zero_bytes = -1, bool group64 = false);
 int64_t gemm_scratch_bytes(int64_t M);
 }  // namespace lutq
 

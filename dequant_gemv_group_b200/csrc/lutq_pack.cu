@@ -7,9 +7,11 @@
 // order, so a warp writes 512 contiguous bytes.  The U * 32 * words_per_row
 // code words come first: word id -> (tile, w, r) with r = id % 32,
 // w = (id / 32) % words_per_row, tile = id / (32 * words_per_row) =
-// strip * G + g.  Then 4 words of scales per tile: word j of tile t holds
-// slots 8 j .. 8 j + 7, slot 4 rq + i being row rq + 8 i.  Codes >= 2^bits
-// are reported and masked.
+// strip * G + g.  Then the scale block of each tile, SB / 16 words: with one
+// scale per group of 128 (SB = 64), word j holds slots 8 j .. 8 j + 7, slot
+// 4 rq + i being row rq + 8 i; with one scale per group of 64 (SB = 128,
+// scales [N, K/64]), words 0-3 hold the first 64-group's slots in that order
+// and words 4-7 the second's.  Codes >= 2^bits are reported and masked.
 #include "lutq_common.cuh"
 
 namespace lutq {
@@ -24,13 +26,14 @@ __device__ __forceinline__ void load_codes(const uint8_t* p, uint8_t* out, int n
   }
 }
 
-template <int BITS>
+template <int BITS, int SB>
 __global__ void __launch_bounds__(256)
 pack_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t N,
             int64_t K, uint4* __restrict__ packed, int32_t* dev_status) {
   constexpr int WPR = words_per_row(BITS);
   constexpr int CW = WPR * kStrip;               // code words of a tile
-  constexpr int SW = kScaleBytes / 16;           // scale words of a tile
+  constexpr int SW = SB / 16;                    // scale words of a tile
+  constexpr int H = SB / kScaleBytes;            // scales per row and group of 128
   constexpr uint32_t kMask = (1u << BITS) - 1u;
   const int64_t G = K / kGroup;
   const int64_t U = (N / kStrip) * G;
@@ -39,15 +42,16 @@ pack_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scal
   for (int64_t id = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; id < words;
        id += int64_t(gridDim.x) * blockDim.x) {
     if (id >= U * CW) {
-      // scale word: slots 8 j .. 8 j + 7 of its tile
+      // scale word j: slots 8 (j % 4) .. 8 (j % 4) + 7 of scale half j / 4
       const int64_t tile = (id - U * CW) / SW;
-      const int slot0 = 8 * int((id - U * CW) % SW);
+      const int j = int((id - U * CW) % SW);
+      const int slot0 = 8 * (j & 3), half = j >> 2;
       const int64_t strip = tile / G, g = tile % G;
       uint32_t h[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
         const int slot = slot0 + t, r = (slot >> 2) + 8 * (slot & 3);
-        h[t] = scales[(strip * kStrip + r) * G + g];
+        h[t] = scales[(strip * kStrip + r) * (G * H) + g * H + half];
       }
       packed[id] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
                               h[6] | (h[7] << 16));
@@ -121,20 +125,24 @@ pack_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scal
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) report(dev_status, LUTQ_ERR_CODE_RANGE);
 }
 
+// group64: scales [N, K/64] into 128-byte scale blocks (else [N, K/128]
+// into 64-byte blocks).
 cudaError_t launch_pack(const uint8_t* codes, const void* scales, int64_t N, int64_t K,
                         int bits, void* packed, int32_t* dev_status, int num_sms,
-                        cudaStream_t stream) {
-  const int64_t words = (N / kStrip) * (K / kGroup) * ((tile_bytes(bits) + kScaleBytes) / 16);
+                        cudaStream_t stream, bool group64) {
+  const int sb = group64 ? 2 * kScaleBytes : kScaleBytes;
+  const int64_t words = (N / kStrip) * (K / kGroup) * ((tile_bytes(bits) + sb) / 16);
   int64_t blocks = (words + 255) / 256;
   const int64_t cap = int64_t(num_sms) * 8;
   if (blocks > cap) blocks = cap;
   const uint16_t* sc = static_cast<const uint16_t*>(scales);
-  if (bits == 4)
-    pack_kernel<4><<<unsigned(blocks), 256, 0, stream>>>(codes, sc, N, K,
-                                                        static_cast<uint4*>(packed), dev_status);
-  else
-    pack_kernel<3><<<unsigned(blocks), 256, 0, stream>>>(codes, sc, N, K,
-                                                        static_cast<uint4*>(packed), dev_status);
+  uint4* out = static_cast<uint4*>(packed);
+  switch ((bits == 4 ? 1 : 0) + (group64 ? 2 : 0)) {
+    case 0: pack_kernel<3, 64><<<unsigned(blocks), 256, 0, stream>>>(codes, sc, N, K, out, dev_status); break;
+    case 1: pack_kernel<4, 64><<<unsigned(blocks), 256, 0, stream>>>(codes, sc, N, K, out, dev_status); break;
+    case 2: pack_kernel<3, 128><<<unsigned(blocks), 256, 0, stream>>>(codes, sc, N, K, out, dev_status); break;
+    default: pack_kernel<4, 128><<<unsigned(blocks), 256, 0, stream>>>(codes, sc, N, K, out, dev_status); break;
+  }
   return cudaGetLastError();
 }
 

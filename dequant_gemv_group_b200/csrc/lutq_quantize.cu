@@ -18,8 +18,11 @@ namespace lutq {
 // scale slot; 2, one scale for the matrix (the tensor-wise granularity of the
 // Log_bQuant abstract's baseline), left in the first slot of row 0 by
 // tensor_amax_kernel; 3, one scale per group of 256 along K (the group-size
-// variant), left in the even 128-group's slot by pair_amax_kernel.  Every
-// group divides by that scale and the other slots receive a copy.
+// variant), left in the even 128-group's slot by pair_amax_kernel; 4, one
+// scale per group of 64 (the finer group-size variant): the two half-warps
+// reduce their own 64 weights and write scales [N, K/64], slot 2 u + half.
+// Every group divides by its scale; with scopes 1-3 the other slots receive a
+// copy.
 template <int BITS, int SCOPE>
 __global__ void __launch_bounds__(256)
 quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
@@ -47,7 +50,8 @@ quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
       amax = fmaxf(amax, fabsf(w[i]));
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    for (int off = SCOPE == 4 ? 8 : 16; off > 0; off >>= 1)
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     const int64_t g = u % groups;
     if (SCOPE == 1) amax = __uint_as_float(uint32_t(scales[u - g]) << 16);
     if (SCOPE == 2) amax = __uint_as_float(uint32_t(scales[0]) << 16);
@@ -69,7 +73,11 @@ quantize_kernel(const uint2* __restrict__ W, int64_t n_rows, int64_t groups,
     codes[u * 32 + lane] = packed4;
     const bool source =
         (SCOPE == 1 && g == 0) || (SCOPE == 2 && u == 0) || (SCOPE == 3 && (g & 1) == 0);
-    if (lane == 0 && !source) scales[u] = uint16_t(__float_as_uint(amax) >> 16);
+    if (SCOPE == 4) {
+      if ((lane & 15) == 0) scales[2 * u + (lane >> 4)] = uint16_t(__float_as_uint(amax) >> 16);
+    } else if (lane == 0 && !source) {
+      scales[u] = uint16_t(__float_as_uint(amax) >> 16);
+    }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) report(dev_status, LUTQ_ERR_NONFINITE);
 }
@@ -294,7 +302,9 @@ cudaError_t launch_quantize(const void* W, int64_t N, int64_t K, const void* cod
     case 4: quantize_kernel<3, 2><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
     case 5: quantize_kernel<4, 2><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
     case 6: quantize_kernel<3, 3><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
-    default: quantize_kernel<4, 3><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    case 7: quantize_kernel<4, 3><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    case 8: quantize_kernel<3, 4><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
+    default: quantize_kernel<4, 4><<<unsigned(blocks), 256, 0, stream>>>(w, N, G, cb, c, s, dev_status); break;
   }
   return cudaGetLastError();
 }

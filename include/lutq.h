@@ -439,6 +439,50 @@ lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
                       int32_t* dev_status, void* stream);
 
 /*
+ * One scale per group of 64.
+ *
+ * Source: the group-size variant of the FLUTE abstract's group quantization
+ * ("Daily Papers" listing, query "group-128"): the same RTN with a finer
+ * group of 64 consecutive weights along K.
+ *   s[n,h] = max_{k in h} |W[n,k]|  over the 64-group h (exact in bf16)
+ *   v, q   as lutq_quantize.
+ *
+ * Packed layout: layout V2's code tiles (lutq_pack), then per unit
+ * t = strip * (K/128) + g a 128-byte scale block at byte U*C + 128*t (U units,
+ * C code bytes per unit): bytes 0..63 hold the scales of the 64-group
+ * [128g, 128g + 64), bytes 64..127 those of [128g + 64, 128g + 128), each
+ * half in the row order of lutq_pack's 64-byte block (row r at byte
+ * 2*(4*(r % 8) + r / 8)).  lutq_packed_bytes_group64 gives the size,
+ * U * (C + 128).
+ *
+ * lutq_quantize_group64: arguments as lutq_quantize; scales_bf16 is
+ *   bf16 [N, K/64] row-major, written.
+ * lutq_pack_group64: codes uint8 [N,K] and scales bf16 [N, K/64] into a
+ *   buffer of lutq_packed_bytes_group64 bytes; errors as lutq_pack.
+ * lutq_gemv_group64: y[m,n] = sum_h s[n,h] * sum_{k in h} x[m,k] * c[q[n,k]],
+ *   every 64-group's partial sum rescaled once in fp32; M = 1..16, routing,
+ *   workspace (lutq_workspace_bytes), numerics and errors as lutq_gemv.
+ * lutq_gemm_group64: the same product on the tensor cores (any M >= 1), as
+ *   lutq_gemm; each unit's 8 MMAs go to two partials (one per 64-half).
+ * All are asynchronous on `stream`; pointers 16-byte aligned.
+ */
+int64_t lutq_packed_bytes_group64(int64_t N, int64_t K, int bits);
+lutq_status lutq_quantize_group64(const void* W_bf16, int64_t N, int64_t K,
+                                  const void* codebook_bf16, int bits, uint8_t* codes,
+                                  void* scales_bf16, int32_t* dev_status, void* stream);
+lutq_status lutq_pack_group64(const uint8_t* codes, const void* scales_bf16, int64_t N,
+                              int64_t K, int bits, void* packed, int32_t* dev_status,
+                              void* stream);
+lutq_status lutq_gemv_group64(const void* x_bf16, int64_t M, const void* packed,
+                              const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
+                              void* workspace, int64_t workspace_bytes, int32_t* dev_status,
+                              void* stream);
+lutq_status lutq_gemm_group64(const void* x_bf16, int64_t M, const void* packed,
+                              const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
+                              void* workspace, int64_t workspace_bytes, int32_t* dev_status,
+                              void* stream);
+
+/*
  * Per-group data types.
  *
  * Source: BitMoD abstract ("Daily Papers" listing, query "group-128"): each
