@@ -7,7 +7,9 @@ down projection W[4096, 14336], 4-bit NormalFloat, group 128, batch 1.
 
 Timing: W warm-up steps, then exactly K steps between a barrier and
 torch.cuda.synchronize() on both sides, CUDA events on the launching stream,
-max over ranks.  The K launches are replayed from CUDA graphs.  The weights
+max over ranks.  The K launches are replayed from CUDA graphs, queued behind a
+short spin kernel that ends before the start event, so the host's launch
+latency is not in the timed region.  The weights
 rotate over R device copies whose total exceeds 3x the L2 size, so no step
 finds its weights in L2.  `e2e` times the same steps through the public call
 with x copied from pinned host memory and y read back every step.
@@ -322,6 +324,16 @@ def capture(fn, count):
     return g
 
 
+def hold_stream(cycles=200_000):
+    """Keep the current stream busy for `cycles` SM clocks (about 100 us) with
+    a spin kernel, so that the launches queued after it (and the start event
+    before them) are already on the device when it ends: the event pair then
+    times the device work alone, not the host's launch latency (the
+    blocking-kernel method of NVIDIA's nvbench).  The spin runs before the
+    start event."""
+    torch.cuda._sleep(int(cycles))
+
+
 def time_events(fn, reps):
     """Average device time of fn() over reps calls (CUDA events, current stream)."""
     torch.cuda.synchronize()
@@ -472,6 +484,48 @@ def side_measurements(lq, dev, args):
                     "quantize_typed_us": tt * 1e6, "groups_per_type": counts,
                     "rel_error_vs_unquantized": {args.codebook: err_plain, "typed": err_typed}}
     del packs_t, packed_t
+    # one scale per group of 64 on the same layer: the GEMV at batch 1
+    # (graph replay, weights rotating over copies larger than L2), the
+    # tensor-core GEMM at batch 128, and the product's error against the
+    # unquantized one
+    codes_h, scales_h = lq.lutq_quantize_group64(w, cb, bits, status=st)
+    packed_h = lq.lutq_pack_group64(codes_h, scales_h, bits, status=st)
+    del codes_h, scales_h
+    copies = max(2, int(np.ceil(3 * l2 / packed_h.numel())) + 1)
+    packs_h = [packed_h] + [packed_h.clone() for _ in range(copies - 1)]
+    call_h = lambda i: lq.lutq_gemv_group64(x1, packs_h[i % copies], cb, bits, n, k, y=y1,
+                                            workspace=ws1, status=st)
+    for i in range(4):
+        call_h(i)
+    g_h = capture(call_h, 128)
+    g_h.replay()
+    t_h = time_events(lambda i: g_h.replay(), 8) / 128
+    del g_h
+    y_h = lq.lutq_gemv_group64(x1, packed_h, cb, bits, n, k, workspace=ws1, status=st)
+    mg = 128
+    xg = workloads.activations(mg, k, seed=1).to(dev)
+    yg = torch.empty((mg, n), dtype=torch.float32, device=dev)
+    wsg = lq.new_workspace(mg, n, k, bits, dev)
+    call_g = lambda i: lq.lutq_gemm_group64(xg, packed_h, cb, bits, n, k, y=yg, workspace=wsg,
+                                            status=st)
+    for i in range(3):
+        call_g(i)
+    t_g = time_events(call_g, 20)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    err_h = float(np.linalg.norm(y_h.double().cpu().numpy() - exact) / np.linalg.norm(exact))
+    h_bytes = algorithmic_bytes(1, n, k, bits) + n * (k // 128) * 2   # two scales per 128
+    out["group64"] = {"workload": f"{args.workload}/{args.layer} W[{n},{k}] {args.codebook} "
+                                  f"W{bits} group64 batch1",
+                      "value": h_bytes / t_h / 1e9, "unit": "GB/s", "us": t_h * 1e6,
+                      "frac_of_hbm_peak": h_bytes / t_h / 1e9 / hbm_peak,
+                      "kernel": "lutq::gemv_small_kernel (128-byte scale blocks)",
+                      "gemm_batch128": {"us": t_g * 1e6,
+                                        "tflops": 2.0 * mg * n * k / t_g / 1e12,
+                                        "kernel": "lutq::gemm_kernel (two partials per unit)"},
+                      "rel_error_vs_unquantized": {f"{args.codebook}_group128": err_plain,
+                                                   f"{args.codebook}_group64": err_h}}
+    del packs_h, packed_h, xg, yg, wsg
     # the baselines of the pages' quantizers, same layer, same GEMV: one scale
     # per row, and the tensor-wise asymmetric linear quantizer (levels evenly
     # spaced from min W to max W, one scale for the matrix)
@@ -552,6 +606,7 @@ def run_lutq(args, world, rank, local):
     torch.cuda.synchronize()
     sampler.mark()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hold_stream()
     ev0.record(stream)
     for _ in range(args.steps // chunk):
         g_chunk.replay()
@@ -575,6 +630,7 @@ def run_lutq(args, world, rank, local):
     for i in range(20):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        hold_stream()
         e0.record(stream)
         step(i)
         e1.record(stream)

@@ -49,14 +49,20 @@ constexpr int kTileRows = 128;
 constexpr int kGemmMaxCtas = 256;            // bounds the workspace
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kTmemCols = 512;
-template <int NT>
+template <int NT, bool G64 = false>
 struct GemmCfg {
   // activation stages (shared memory); two at N_tile = 128 leave 32 KB more
   // to L1 (measured 2% faster at batch 128 than three; four: 25% slower)
   static constexpr int XS = NT >= 128 ? 2 : 4;
   static constexpr int XSTAGE = 2 * NT * 128;       // two boxes of NT rows x 128 bytes
-  static constexpr int AS = 4;                      // A stages in tensor memory (64 columns each)
-  static constexpr int DS = NT >= 128 ? 2 : (NT >= 64 ? 3 : 4);  // partial stages (NT columns)
+  // A stages in tensor memory (64 columns each) and partial stages (NT
+  // columns each).  With one scale per group of 64 a unit fills two partial
+  // stages, so the stages go to the partials: at N_tile = 128 two A stages
+  // and three partial stages, below it as many partial stages as fit (at
+  // most 8).
+  static constexpr int AS = (G64 && NT >= 128) ? 2 : 4;
+  static constexpr int DS = G64 ? ((kTmemCols - 64 * AS) / NT < 8 ? (kTmemCols - 64 * AS) / NT : 8)
+                                : (NT >= 128 ? 2 : (NT >= 64 ? 3 : 4));
   static constexpr int DW = NT >= 64 ? 4 : 8;       // dequant warps (8: two per lane quarter)
   static constexpr int NB = DW == 8 ? 4 : 2;        // units of packed words in flight per lane
   static constexpr int KC = 64 * 4 / DW;            // A columns written per dequant warp
@@ -218,7 +224,7 @@ __device__ __forceinline__ void tmem_st_cols32(uint32_t taddr, const uint32_t (&
 template <int BITS, int NT, bool TYPED, bool G64>
 __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, GemmArgs a) {
-  using Cfg = GemmCfg<NT>;
+  using Cfg = GemmCfg<NT, G64>;
   static_assert(!(TYPED && G64), "per-group types use one scale per group of 128");
   // partials per unit (one per scale), the scale block's bytes
   constexpr int H = G64 ? 2 : 1;
@@ -433,6 +439,7 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     float acc[NC];
 #pragma unroll
     for (int j = 0; j < NC; ++j) acc[j] = 0.0f;
+    constexpr int CH = chunk_cols<NC>();
     for (int i = 0; i < n; ++i) {
       const int64_t row = cur.tau * kTileRows + sw * 32 + lane;
       const bool valid = cur.tau * kTileRows + sw * 32 < a.N;
@@ -452,13 +459,12 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
             mbar_wait(bar(B_DF + ds), uint32_t(d / DS) & 1u, abort_flag, kWaitLimitNs);
         if (!__all_sync(0xffffffffu, ok)) goto promote_done;
         tc_fence_after();
-        constexpr int CH = chunk_cols<NC>();
+        const uint32_t tpart = tmem + (uint32_t(sw * 32) << 16) +
+                               uint32_t(Cfg::DCOL + ds * NT + pg * NC);
 #pragma unroll
         for (int c = 0; c < NC / CH; ++c) {
           uint32_t v[32];
-          tmem_ld_cols<NC>(tmem + (uint32_t(sw * 32) << 16) +
-                               uint32_t(Cfg::DCOL + ds * NT + pg * NC + c * CH),
-                           v);
+          tmem_ld_cols<NC>(tpart + uint32_t(c * CH), v);
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < CH; ++j)
@@ -614,7 +620,7 @@ static cudaError_t make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_
 template <int BITS, int NT, bool TYPED, bool G64>
 static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
                              cudaStream_t stream) {
-  using Cfg = GemmCfg<NT>;
+  using Cfg = GemmCfg<NT, G64>;
   static int granted[64] = {0};
   // alignment slack, table, activation stages, barriers and flags (512),
   // the promotion warps' scale rings (two scales per lane and unit with G64)
