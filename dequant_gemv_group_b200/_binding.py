@@ -14,10 +14,14 @@ from typing import Optional, Tuple
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "liblutq.so")
+# LUTQ_LIB_VARIANT=nvtx|bounds loads a tooling build of the same library
+# (see build.py); the default is the product build
+_VARIANT = os.environ.get("LUTQ_LIB_VARIANT") or None
+LIB_PATH = os.path.join(_PKG, "liblutq.so" if _VARIANT is None else f"liblutq_{_VARIANT}.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python dequant_gemv_group_b200/build.py`")
+    raise ImportError(f"{LIB_PATH} is not built; run `python dequant_gemv_group_b200/build.py"
+                      + (f" --variant {_VARIANT}`" if _VARIANT else "`"))
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -27,13 +31,16 @@ LUTQ_OK = 0
 STATUS_NAMES = {
     0: "LUTQ_OK", 1: "LUTQ_ERR_INVALID_ARG", 2: "LUTQ_ERR_SHAPE", 3: "LUTQ_ERR_BITS",
     4: "LUTQ_ERR_ALIGN", 5: "LUTQ_ERR_NONFINITE", 6: "LUTQ_ERR_CODE_RANGE",
-    7: "LUTQ_ERR_TIMEOUT", 8: "LUTQ_ERR_CUDA", 9: "LUTQ_ERR_WORKSPACE",
+    7: "LUTQ_ERR_TIMEOUT", 8: "LUTQ_ERR_CUDA", 9: "LUTQ_ERR_WORKSPACE", 10: "LUTQ_ERR_BOUNDS",
 }
+BUILD_NVTX, BUILD_BOUNDS = 1, 2
 CODEBOOK_KINDS = {"nf4": 0, "logb": 1, "lloyd_max3": 2, "uniform4": 3}
 
 _SIGS = {
     "lutq_status_string": (ctypes.c_char_p, [_i32]),
     "lutq_layout_version": (_i32, []),
+    "lutq_build_flags": (_i32, []),
+    "lutq_selftest_bounds": (_i32, [_vp, _vp]),
     "lutq_packed_bytes": (_i64, [_i64, _i64, _i32]),
     "lutq_codebook": (_i32, [_i32, _i32, _vp]),
     "lutq_quantize": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
@@ -106,6 +113,17 @@ def lutq_status_string(status: int) -> str:
 
 def lutq_layout_version() -> int:
     return lib.lutq_layout_version()
+
+
+def lutq_build_flags() -> int:
+    """BUILD_NVTX | BUILD_BOUNDS bits of the loaded library (0: product build)."""
+    return int(lib.lutq_build_flags())
+
+
+def lutq_selftest_bounds(status: torch.Tensor) -> None:
+    """Run the kernels' index check on an index past its extent (see include/lutq.h)."""
+    _need(status, torch.int32, "status")
+    _check(lib.lutq_selftest_bounds(status.data_ptr(), _stream()), "lutq_selftest_bounds")
 
 
 def lutq_packed_bytes(n: int, k: int, bits: int) -> int:

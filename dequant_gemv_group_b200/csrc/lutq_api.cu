@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include "lutq.h"
+#include "lutq_trace.h"
 #include "lutq_common.cuh"
 
 namespace lutq {
@@ -117,6 +118,7 @@ lutq_status check_product_args(const void* x, int64_t M, int64_t max_m, const vo
 extern "C" {
 
 const char* lutq_status_string(int status) {
+  LUTQ_TRACE_RANGE("lutq_status_string");
   switch (status) {
     case LUTQ_OK: return "LUTQ_OK";
     case LUTQ_ERR_INVALID_ARG: return "LUTQ_ERR_INVALID_ARG: null pointer or invalid value";
@@ -128,13 +130,30 @@ const char* lutq_status_string(int status) {
     case LUTQ_ERR_TIMEOUT: return "LUTQ_ERR_TIMEOUT: bounded wait expired inside a kernel";
     case LUTQ_ERR_CUDA: return "LUTQ_ERR_CUDA: CUDA runtime error";
     case LUTQ_ERR_WORKSPACE: return "LUTQ_ERR_WORKSPACE: workspace missing or too small";
+    case LUTQ_ERR_BOUNDS: return "LUTQ_ERR_BOUNDS: an index outside its buffer (checked build)";
     default: return "unknown lutq status";
   }
 }
 
-int lutq_layout_version(void) { return 2; }
+int lutq_layout_version(void) {
+  LUTQ_TRACE_RANGE("lutq_layout_version");
+  return 2;
+}
+
+int lutq_build_flags(void) {
+  LUTQ_TRACE_RANGE("lutq_build_flags");
+  int flags = 0;
+#ifdef LUTQ_NVTX
+  flags |= LUTQ_BUILD_NVTX;
+#endif
+#ifdef LUTQ_BOUNDS
+  flags |= LUTQ_BUILD_BOUNDS;
+#endif
+  return flags;
+}
 
 int64_t lutq_packed_bytes(int64_t N, int64_t K, int bits) {
+  LUTQ_TRACE_RANGE("lutq_packed_bytes");
   if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK) return -1;
   return (N / lutq::kStrip) * (K / lutq::kGroup) * (lutq::tile_bytes(bits) + lutq::kScaleBytes);
 }
@@ -160,30 +179,35 @@ static lutq_status quantize(const void* W_bf16, int64_t N, int64_t K, const void
 lutq_status lutq_quantize(const void* W_bf16, int64_t N, int64_t K, const void* codebook_bf16,
                           int bits, uint8_t* codes, void* scales_bf16, int32_t* dev_status,
                           void* stream) {
+  LUTQ_TRACE_RANGE("lutq_quantize");
   return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 0);
 }
 
 lutq_status lutq_quantize_rowscale(const void* W_bf16, int64_t N, int64_t K,
                                    const void* codebook_bf16, int bits, uint8_t* codes,
                                    void* scales_bf16, int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_quantize_rowscale");
   return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 1);
 }
 
 lutq_status lutq_quantize_group256(const void* W_bf16, int64_t N, int64_t K,
                                    const void* codebook_bf16, int bits, uint8_t* codes,
                                    void* scales_bf16, int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_quantize_group256");
   return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 3);
 }
 
 lutq_status lutq_quantize_tensorscale(const void* W_bf16, int64_t N, int64_t K,
                                       const void* codebook_bf16, int bits, uint8_t* codes,
                                       void* scales_bf16, int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_quantize_tensorscale");
   return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 2);
 }
 
 lutq_status lutq_quantize_group64(const void* W_bf16, int64_t N, int64_t K,
                                   const void* codebook_bf16, int bits, uint8_t* codes,
                                   void* scales_bf16, int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_quantize_group64");
   return quantize(W_bf16, N, K, codebook_bf16, bits, codes, scales_bf16, dev_status, stream, 4);
 }
 
@@ -203,10 +227,12 @@ static lutq_status pack(const uint8_t* codes, const void* scales_bf16, int64_t N
 
 lutq_status lutq_pack(const uint8_t* codes, const void* scales_bf16, int64_t N, int64_t K,
                       int bits, void* packed, int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_pack");
   return pack(codes, scales_bf16, N, K, bits, packed, dev_status, stream, false);
 }
 
 int64_t lutq_packed_bytes_group64(int64_t N, int64_t K, int bits) {
+  LUTQ_TRACE_RANGE("lutq_packed_bytes_group64");
   if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK) return -1;
   return (N / lutq::kStrip) * (K / lutq::kGroup) *
          (lutq::tile_bytes(bits) + 2 * lutq::kScaleBytes);
@@ -215,10 +241,12 @@ int64_t lutq_packed_bytes_group64(int64_t N, int64_t K, int bits) {
 lutq_status lutq_pack_group64(const uint8_t* codes, const void* scales_bf16, int64_t N,
                               int64_t K, int bits, void* packed, int32_t* dev_status,
                               void* stream) {
+  LUTQ_TRACE_RANGE("lutq_pack_group64");
   return pack(codes, scales_bf16, N, K, bits, packed, dev_status, stream, true);
 }
 
 lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan) {
+  LUTQ_TRACE_RANGE("lutq_gemv_plan");
   if (plan == nullptr || num_sms < 1) return LUTQ_ERR_INVALID_ARG;
   lutq_status st;
   if ((st = check_shape(N, K)) != LUTQ_OK) return st;
@@ -227,11 +255,13 @@ lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan) {
 }
 
 int64_t lutq_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
+  LUTQ_TRACE_RANGE("lutq_workspace_bytes");
   if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK || M < 1) return -1;
   return lutq::workspace_zero_bytes(M, N, K) + lutq::gemm_scratch_bytes(M);
 }
 
 int64_t lutq_workspace_zero_bytes(int64_t M, int64_t N, int64_t K, int bits) {
+  LUTQ_TRACE_RANGE("lutq_workspace_zero_bytes");
   if (check_shape(N, K) != LUTQ_OK || check_bits(bits) != LUTQ_OK || M < 1) return -1;
   return lutq::workspace_zero_bytes(M, N, K);
 }
@@ -240,6 +270,7 @@ lutq_status lutq_gemv(const void* x_bf16, int64_t M, const void* packed,
                       const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
                       void* workspace, int64_t workspace_bytes, int32_t* dev_status,
                       void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemv");
   lutq_status st = check_product_args(x_bf16, M, 16, packed, codebook_bf16, bits, N, K, y,
                                       workspace, workspace_bytes,
                                       lutq_workspace_bytes(M, N, K, bits));
@@ -254,6 +285,7 @@ lutq_status lutq_gemv_out_bf16(const void* x_bf16, int64_t M, const void* packed
                                const void* codebook_bf16, int bits, int64_t N, int64_t K,
                                void* y_bf16, void* workspace, int64_t workspace_bytes,
                                int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemv_out_bf16");
   lutq_status st = check_product_args(x_bf16, M, 16, packed, codebook_bf16, bits, N, K,
                                       static_cast<const float*>(y_bf16), workspace,
                                       workspace_bytes, lutq_workspace_bytes(M, N, K, bits));
@@ -269,6 +301,7 @@ lutq_status lutq_gemm_out_bf16(const void* x_bf16, int64_t M, const void* packed
                                const void* codebook_bf16, int bits, int64_t N, int64_t K,
                                void* y_bf16, void* workspace, int64_t workspace_bytes,
                                int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemm_out_bf16");
   lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, codebook_bf16, bits,
                                       N, K, static_cast<const float*>(y_bf16), workspace,
                                       workspace_bytes, lutq_workspace_bytes(M, N, K, bits));
@@ -284,6 +317,7 @@ lutq_status lutq_gemm(const void* x_bf16, int64_t M, const void* packed,
                       const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
                       void* workspace, int64_t workspace_bytes, int32_t* dev_status,
                       void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemm");
   lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, codebook_bf16, bits,
                                       N, K, y, workspace, workspace_bytes,
                                       lutq_workspace_bytes(M, N, K, bits));
@@ -298,6 +332,7 @@ lutq_status lutq_gemv_group64(const void* x_bf16, int64_t M, const void* packed,
                               const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
                               void* workspace, int64_t workspace_bytes, int32_t* dev_status,
                               void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemv_group64");
   lutq_status st = check_product_args(x_bf16, M, 16, packed, codebook_bf16, bits, N, K, y,
                                       workspace, workspace_bytes,
                                       lutq_workspace_bytes(M, N, K, bits));
@@ -313,6 +348,7 @@ lutq_status lutq_gemm_group64(const void* x_bf16, int64_t M, const void* packed,
                               const void* codebook_bf16, int bits, int64_t N, int64_t K, float* y,
                               void* workspace, int64_t workspace_bytes, int32_t* dev_status,
                               void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemm_group64");
   lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, codebook_bf16, bits,
                                       N, K, y, workspace, workspace_bytes,
                                       lutq_workspace_bytes(M, N, K, bits));
@@ -344,6 +380,7 @@ static lutq_status rht(const void* in, int64_t rows, int64_t K, const int8_t* si
 
 lutq_status lutq_fit_histogram(const void* W_bf16, int64_t N, int64_t K, uint64_t* hist,
                                int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_fit_histogram");
   if (!W_bf16 || !hist) return LUTQ_ERR_INVALID_ARG;
   if (N < 1 || K < lutq::kGroup || K % lutq::kGroup != 0 || N > (int64_t(1) << 31) ||
       K > (int64_t(1) << 31))
@@ -358,11 +395,13 @@ lutq_status lutq_fit_histogram(const void* W_bf16, int64_t N, int64_t K, uint64_
 
 lutq_status lutq_rht_weights(const void* W_bf16, int64_t N, int64_t K, const int8_t* signs,
                              void* W_rot_bf16, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_rht_weights");
   return rht(W_bf16, N, K, signs, W_rot_bf16, false, stream);
 }
 
 lutq_status lutq_rht_activations(const void* x_bf16, int64_t M, int64_t K, const int8_t* signs,
                                  void* x_rot_bf16, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_rht_activations");
   return rht(x_bf16, M, K, signs, x_rot_bf16, true, stream);
 }
 
@@ -370,6 +409,7 @@ lutq_status lutq_gemv_rht(const void* x_bf16, int64_t M, const void* packed,
                           const void* codebook_bf16, const int8_t* signs, int bits, int64_t N,
                           int64_t K, float* y, void* workspace, int64_t workspace_bytes,
                           int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemv_rht");
   if (!signs) return LUTQ_ERR_INVALID_ARG;
   lutq_status st = check_product_args(x_bf16, M, 16, packed, codebook_bf16, bits, N, K, y,
                                       workspace, workspace_bytes,
@@ -384,9 +424,13 @@ lutq_status lutq_gemv_rht(const void* x_bf16, int64_t M, const void* packed,
                                          static_cast<cudaStream_t>(stream)));
 }
 
-int lutq_max_types(int bits) { return check_bits(bits) == LUTQ_OK ? lutq::max_types(bits) : -1; }
+int lutq_max_types(int bits) {
+  LUTQ_TRACE_RANGE("lutq_max_types");
+  return check_bits(bits) == LUTQ_OK ? lutq::max_types(bits) : -1;
+}
 
 int64_t lutq_packed_bytes_typed(int64_t N, int64_t K, int bits) {
+  LUTQ_TRACE_RANGE("lutq_packed_bytes_typed");
   const int64_t body = lutq_packed_bytes(N, K, bits);
   if (body < 0) return -1;
   return body + (N / lutq::kStrip) * (K / lutq::kGroup) * lutq::kTypeBytes;
@@ -396,6 +440,7 @@ lutq_status lutq_quantize_typed(const void* W_bf16, int64_t N, int64_t K,
                                 const void* codebooks_bf16, int types, int bits, uint8_t* codes,
                                 void* scales_bf16, uint8_t* group_types, int32_t* dev_status,
                                 void* stream) {
+  LUTQ_TRACE_RANGE("lutq_quantize_typed");
   if (!W_bf16 || !codebooks_bf16 || !codes || !scales_bf16 || !group_types)
     return LUTQ_ERR_INVALID_ARG;
   lutq_status st = check_bits(bits);
@@ -415,6 +460,7 @@ lutq_status lutq_quantize_typed(const void* W_bf16, int64_t N, int64_t K,
 lutq_status lutq_pack_typed(const uint8_t* codes, const void* scales_bf16,
                             const uint8_t* group_types, int64_t N, int64_t K, int bits,
                             void* packed, int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_pack_typed");
   if (!group_types) return LUTQ_ERR_INVALID_ARG;
   if (!aligned16(group_types)) return LUTQ_ERR_ALIGN;
   lutq_status st = lutq_pack(codes, scales_bf16, N, K, bits, packed, dev_status, stream);
@@ -429,6 +475,7 @@ lutq_status lutq_gemv_typed(const void* x_bf16, int64_t M, const void* packed,
                             const void* codebooks_bf16, int types, int bits, int64_t N, int64_t K,
                             float* y, void* workspace, int64_t workspace_bytes,
                             int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemv_typed");
   lutq_status st = check_product_args(x_bf16, M, 16, packed, codebooks_bf16, bits, N, K, y,
                                       workspace, workspace_bytes,
                                       lutq_workspace_bytes(M, N, K, bits));
@@ -445,6 +492,7 @@ lutq_status lutq_gemm_typed(const void* x_bf16, int64_t M, const void* packed,
                             const void* codebooks_bf16, int types, int bits, int64_t N, int64_t K,
                             float* y, void* workspace, int64_t workspace_bytes,
                             int32_t* dev_status, void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemm_typed");
   lutq_status st = check_product_args(x_bf16, M, int64_t(1) << 30, packed, codebooks_bf16, bits,
                                       N, K, y, workspace, workspace_bytes,
                                       lutq_workspace_bytes(M, N, K, bits));

@@ -14,6 +14,7 @@
 #include <algorithm>
 
 #include "lutq.h"
+#include "lutq_trace.h"
 
 namespace {
 
@@ -108,6 +109,7 @@ std::vector<double> lloyd_max(int n) {
 }  // namespace
 
 extern "C" lutq_status lutq_codebook(int kind, int bits, uint16_t* out_bf16) {
+  LUTQ_TRACE_RANGE("lutq_codebook");
   if (out_bf16 == nullptr) return LUTQ_ERR_INVALID_ARG;
   std::vector<double> lv;
   switch (kind) {
@@ -140,6 +142,7 @@ extern "C" lutq_status lutq_codebook(int kind, int bits, uint16_t* out_bf16) {
 // lutq_quantize_tensorscale writes it), fp64, rounded once to bf16.
 extern "C" lutq_status lutq_codebook_asym_linear(double w_min, double w_max, int bits,
                                                  uint16_t* out_bf16) {
+  LUTQ_TRACE_RANGE("lutq_codebook_asym_linear");
   if (out_bf16 == nullptr) return LUTQ_ERR_INVALID_ARG;
   if (bits != 3 && bits != 4) return LUTQ_ERR_BITS;
   if (!std::isfinite(w_min) || !std::isfinite(w_max) || !(w_min <= w_max))
@@ -164,6 +167,7 @@ extern "C" lutq_status lutq_codebook_asym_linear(double w_min, double w_max, int
 // layer's own weights.
 extern "C" lutq_status lutq_fit_codebook(const uint64_t* hist, int bits, const uint16_t* init_bf16,
                                          int max_iter, uint16_t* out_bf16) {
+  LUTQ_TRACE_RANGE("lutq_fit_codebook");
   constexpr int kHistBins = 16384;
   if (hist == nullptr || init_bf16 == nullptr || out_bf16 == nullptr || max_iter < 0)
     return LUTQ_ERR_INVALID_ARG;

@@ -50,6 +50,20 @@ __device__ __forceinline__ void report(int32_t* dev_status, int code) {
   if (dev_status != nullptr) atomicCAS(dev_status, 0, code);
 }
 
+// Checked builds (-DLUTQ_BOUNDS): LUTQ_IN_BOUNDS(cond, status) is cond, and a
+// false cond is reported as LUTQ_ERR_BOUNDS; the caller skips the access it
+// guards.  Other builds: the constant true, so the check and the skip compile
+// away.
+__device__ __forceinline__ bool bounds_check(bool ok, int32_t* dev_status) {
+  if (!ok) report(dev_status, LUTQ_ERR_BOUNDS);
+  return ok;
+}
+#ifdef LUTQ_BOUNDS
+#define LUTQ_IN_BOUNDS(cond, status) (::lutq::bounds_check(bool(cond), (status)))
+#else
+#define LUTQ_IN_BOUNDS(cond, status) (true)
+#endif
+
 // Store output value i: fp32, or (y_bf16) the fp32 value rounded once to
 // bf16 (round to nearest even; the bf16 output variant of the products).
 __device__ __forceinline__ void store_y(float* y, int y_bf16, int64_t i, float v) {

@@ -94,6 +94,7 @@ struct GemmArgs {
   int64_t ntiles;     // row tiles, ceil(N / 128)
   int64_t U;          // units
   int C;              // CTAs
+  int smem_bytes;     // the block's dynamic shared memory (checked builds)
 };
 
 // CTA c holds units [g_unit_begin(c), g_unit_begin(c+1)).  The host
@@ -155,20 +156,33 @@ __device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t s
   const uint32_t c_lo = g_unit_owner(uint32_t(seg_begin), U, C);
   const uint32_t c_hi = g_unit_owner(uint32_t(seg_end - 1), U, C);
   const int64_t ycol = (bt * kTileRows + c0) * a.N + row;
+  const int64_t ysize = a.M * a.N;
   if (c_lo == c_hi) {
 #pragma unroll
     for (int j = 0; j < NC; ++j)
-      if (c0 + j < mt) store_y(a.y, a.y_bf16, ycol + int64_t(j) * a.N, acc[j]);
+      if (c0 + j < mt && LUTQ_IN_BOUNDS(ycol + int64_t(j) * a.N < ysize, a.dev_status))
+        store_y(a.y, a.y_bf16, ycol + int64_t(j) * a.N, acc[j]);
     return;
   }
   const int64_t cta = blockIdx.x;
   const int slot = (uint32_t(seg) == uint32_t(u0) / uint32_t(a.G)) ? 0 : 1;
+  // checked builds: the partial-sum slot and the counter lie in the workspace
+  const int64_t nparts = int64_t(kGemmMaxCtas) * 2 * 4 * NT * 32;
+  const int64_t ncounters = ((a.M + kTileRows - 1) / kTileRows) * a.ntiles * 4 * kMaxPromoteGroups;
+  const int64_t cidx = (seg * 4 + sw) * kMaxPromoteGroups + pg;
+  (void)ysize;  // read by the checks of checked builds only
+  (void)nparts;
+  (void)ncounters;
+  if (!LUTQ_IN_BOUNDS((((cta * 2 + slot) * 4 + sw) * NT + c0 + NC) * 32 <= nparts &&
+                          cidx < ncounters,
+                      a.dev_status))
+    return;
   float* mine = a.part + (((cta * 2 + slot) * 4 + sw) * NT + c0) * 32;
 #pragma unroll
   for (int j = 0; j < NC; ++j) mine[j * 32 + lane] = acc[j];
   __syncwarp();
   int arrived = 0;
-  int* counter = a.counters + (seg * 4 + sw) * kMaxPromoteGroups + pg;
+  int* counter = a.counters + cidx;
   if (lane == 0) arrived = atom_add_acq_rel_gpu(counter, 1);
   arrived = __shfl_sync(0xffffffffu, arrived, 0);
   if (arrived != int(c_hi - c_lo)) return;
@@ -183,7 +197,8 @@ __device__ void gemm_finish_strip(const GemmArgs& a, float (&acc)[NC], int64_t s
   }
 #pragma unroll
   for (int j = 0; j < NC; ++j)
-    if (c0 + j < mt) store_y(a.y, a.y_bf16, ycol + int64_t(j) * a.N, acc[j]);
+    if (c0 + j < mt && LUTQ_IN_BOUNDS(ycol + int64_t(j) * a.N < ysize, a.dev_status))
+      store_y(a.y, a.y_bf16, ycol + int64_t(j) * a.N, acc[j]);
   if (lane == 0) *counter = 0;
 }
 
@@ -256,6 +271,13 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   uint16_t* cbs = reinterpret_cast<uint16_t*>(misc + 8);
+  // checked builds: table, activation stages, barriers, flags, codebook copy
+  // and the scale rings lie inside the block's dynamic shared memory
+  if (!LUTQ_IN_BOUNDS(bar_sa + 512u + uint32_t(kScaleRingBytes * H) - raw_sa <=
+                          uint32_t(a.smem_bytes) &&
+                          8u * NBAR + 8u + 2u * uint32_t(a.ntypes << BITS) <= 512u,
+                      a.dev_status))
+    return;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -318,7 +340,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     // per-group types: the lane's row is lane (rq = lane & 7, i = lane >> 3)
     // of its strip; its type is bits 2i+1:2i of byte rq of the unit's block
     auto fetch = [&](uint4 (&wd)[NWL], uint32_t& ty) {
-      if (fetched < n && fp.tau * kTileRows + sw * 32 < a.N) {
+      if (fetched < n && fp.tau * kTileRows + sw * 32 < a.N &&
+          LUTQ_IN_BOUNDS((fp.tau * 4 + sw) * a.G + fp.g < (a.N / kStrip) * a.G, a.dev_status)) {
         const int64_t tile = (fp.tau * 4 + sw) * a.G + fp.g;
         const uint8_t* t = a.packed + tile * TB + lane * 16;
 #pragma unroll
@@ -370,7 +393,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         if (TYPED && ((ty >> (2 * (lane >> 3))) & 3u) >= uint32_t(a.ntypes))
           report(a.dev_status, LUTQ_ERR_CODE_RANGE);
         const uint4 h0[2] = {wd[0], wd[DW == 8 ? 1 : (BITS == 4 ? 1 : 2)]};
-        decode_group_half<BITS>(av, h0, DW == 8 ? kh : 0, lut_sa, off_e | sel, off_o | sel);
+        decode_group_half<BITS>(av, h0, DW == 8 ? kh : 0, lut_sa, off_e | sel, off_o | sel,
+                                uint32_t(LUTB), a.dev_status);
       }
       fetch(wd, ty);
       const int as = i % AS;
@@ -384,7 +408,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         const uint32_t ta = tmem + (uint32_t(sw * 32) << 16) + uint32_t(as * 64 + kh * 32);
         tmem_st_cols32(ta, av);
         if (DW == 4) {
-          decode_group_half<BITS>(av, h1, 1, lut_sa, off_e | sel, off_o | sel);
+          decode_group_half<BITS>(av, h1, 1, lut_sa, off_e | sel, off_o | sel, uint32_t(LUTB),
+                                  a.dev_status);
           tmem_st_cols32(ta + 32u, av);
         }
         tmem_wait_st();
@@ -419,7 +444,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     const uint32_t half = uint32_t(scale_slot(lane) >> 1) & 1u;  // which bf16 of the word
     auto issue_scale = [&](const UnitPos& p, int slot, bool live) {
       const int64_t r0 = p.tau * kTileRows + sw * 32;
-      if (live && r0 < a.N) {
+      if (live && r0 < a.N &&
+          LUTQ_IN_BOUNDS((r0 / kStrip) * a.G + p.g < (a.N / kStrip) * a.G, a.dev_status)) {
         const uint8_t* b =
             a.scales + ((r0 / kStrip) * a.G + p.g) * SBB + (scale_slot(lane) & ~3);
 #pragma unroll
@@ -637,6 +663,7 @@ static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
     granted[dev] = smem;
   }
   a.C = int(std::min<int64_t>(std::min<int64_t>(num_sms, kGemmMaxCtas), a.U));
+  a.smem_bytes = smem;
   gemm_kernel<BITS, NT, TYPED, G64><<<unsigned(a.C), Cfg::THREADS, smem, stream>>>(map, a);
   return cudaGetLastError();
 }

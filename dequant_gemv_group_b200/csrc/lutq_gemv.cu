@@ -81,7 +81,13 @@ struct GemvArgs {
   // The grid's first pf_ctas CTAs only bring the packed matrix into L2
   // (the work goes to CTAs pf_ctas .. pf_ctas + C - 1)
   uint32_t pf_ctas;
+  uint32_t smem_bytes;      // the block's dynamic shared memory (checked builds)
 };
+
+// Output value i (< M N) into y; checked builds skip an index outside y.
+__device__ __forceinline__ void put_y(const GemvArgs& a, int64_t i, int M, float v) {
+  if (LUTQ_IN_BOUNDS(i >= 0 && i < int64_t(M) * a.N, a.status)) store_y(a.y, a.y_bf16, i, v);
+}
 
 // Part i of `parts` equal shares of [0, total): [range_begin(i), range_begin(i+1)).
 // The host guarantees total * parts < 2^32, so 32-bit unsigned arithmetic is
@@ -166,7 +172,7 @@ __device__ __forceinline__ void deposit_strip(const GemvArgs& a, const Span& p, 
     for (int i = 0; i < R; ++i)
 #pragma unroll
       for (int m = 0; m < M; ++m)
-        store_y(a.y, a.y_bf16, m * a.N + int64_t(strip) * kStrip + rows[i], vals[i][m]);
+        put_y(a, m * a.N + int64_t(strip) * kStrip + rows[i], M, vals[i][m]);
     return;
   }
   const int sl = (strip == first_strip) ? 0 : 1;
@@ -181,8 +187,11 @@ __device__ __forceinline__ void deposit_strip(const GemvArgs& a, const Span& p, 
 // takes it, writes the sum and clears the slot for the next call.  Both
 // orders give the same fp32 sum (addition of two values commutes), so the
 // result does not depend on timing.
+template <int M>
 __device__ __forceinline__ void exchange_half(unsigned long long* slot, float v,
                                               const GemvArgs& a, int64_t yi) {
+  // one slot per output value of up to 4 batch rows (the workspace's zero part)
+  if (!LUTQ_IN_BOUNDS(yi >= 0 && yi < int64_t(M) * a.N && M <= 4, a.status)) return;
   const unsigned long long mine = (1ull << 32) | __float_as_uint(v);
   const unsigned long long other = atomicExch(slot, mine);
   if (other != 0ull) {
@@ -226,12 +235,12 @@ __device__ void cta_finish(const GemvArgs& a, const Span& p, const float* all_sl
     const int64_t yrow = int64_t(strip) * kStrip + lane;
     if (full && lo >= p.v0 && hi <= p.v1) {
 #pragma unroll
-      for (int m = 0; m < M; ++m) store_y(a.y, a.y_bf16, yrow + m * a.N, sum[m]);
+      for (int m = 0; m < M; ++m) put_y(a, yrow + m * a.N, M, sum[m]);
       continue;
     }
     unsigned long long* xrow = a.xch + yrow;
 #pragma unroll
-    for (int m = 0; m < M; ++m) exchange_half(xrow + m * a.N, sum[m], a, yrow + m * a.N);
+    for (int m = 0; m < M; ++m) exchange_half<M>(xrow + m * a.N, sum[m], a, yrow + m * a.N);
   }
 }
 
@@ -304,18 +313,29 @@ __device__ __forceinline__ void pair_first(float& acc, uint32_t lv, uint32_t xw)
 // independent table loads and accumulator chains are in flight, and each
 // table load serves all M batch rows.  FIRST starts the chains (su is not
 // read).
+// Checked builds compare every table address with the table region's size
+// (lut_limit) and every activation address with the end of the activations
+// (x_end), reporting through st; other builds ignore the three.
+struct Checks {
+  uint32_t lut_limit, x_end;
+  int32_t* st;
+};
+
 template <bool FIRST, int M>
 __device__ __forceinline__ void quad4(float (&su)[4][M], const uint32_t (&idx)[4],
-                                      const uint32_t (&lc)[4], const uint32_t (&xq)[M][4]) {
+                                      const uint32_t (&lc)[4], const uint32_t (&xq)[M][4],
+                                      const Checks& ck) {
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     uint32_t lv[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) {
       // row = byte b of the index word (bits 15:8), column = byte 0 of row
       // i's column word (bits 7:0), table = its byte 1 (bits 23:16; byte 2
       // is zero)
-      lv[i] = lut_ld(__byte_perm(idx[i], lc[i], 0x6504u | (uint32_t(b) << 4)));
+      const uint32_t t = __byte_perm(idx[i], lc[i], 0x6504u | (uint32_t(b) << 4));
+      lv[i] = LUTQ_IN_BOUNDS(t + 4u <= ck.lut_limit, ck.st) ? lut_ld(t) : 0u;
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -331,12 +351,18 @@ __device__ __forceinline__ void quad4(float (&su)[4][M], const uint32_t (&idx)[4
 // Four activation words (8 bf16 values) of each batch row: batch row m's
 // run of the current group starts at xa + m * xstride.
 template <int M>
-__device__ __forceinline__ void load_xq(uint32_t (&xq)[M][4], uint32_t xa, uint32_t xstride) {
+__device__ __forceinline__ void load_xq(uint32_t (&xq)[M][4], uint32_t xa, uint32_t xstride,
+                                        const Checks& ck) {
 #pragma unroll
-  for (int m = 0; m < M; ++m)
+  for (int m = 0; m < M; ++m) {
+    if (!LUTQ_IN_BOUNDS(xa + uint32_t(m) * xstride + 16u <= ck.x_end, ck.st)) {
+      xq[m][0] = xq[m][1] = xq[m][2] = xq[m][3] = 0u;
+      continue;
+    }
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(xq[m][0]), "=r"(xq[m][1]), "=r"(xq[m][2]), "=r"(xq[m][3])
                  : "r"(xa + uint32_t(m) * xstride));
+  }
 }
 
 // Byte offset, inside a tile, of the lane's packed bytes of row rq; rows
@@ -406,20 +432,20 @@ template <int BITS, int M>
 __device__ __forceinline__ void unit_partial(float (&su)[4][M], const uint4 (&wd)[4],
                                              const uint32_t (&lce)[4], const uint32_t (&lco)[4],
                                              uint32_t hi_shift,
-                                             uint32_t xa, uint32_t xstride) {
+                                             uint32_t xa, uint32_t xstride, const Checks& ck) {
   uint32_t xq[M][4];
   if (BITS == 4) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      load_xq<M>(xq, xa + 16u * j, xstride);
+      load_xq<M>(xq, xa + 16u * j, xstride, ck);
       const uint32_t idx[4] = {j == 0 ? wd[0].x : j == 1 ? wd[0].y : j == 2 ? wd[0].z : wd[0].w,
                                j == 0 ? wd[1].x : j == 1 ? wd[1].y : j == 2 ? wd[1].z : wd[1].w,
                                j == 0 ? wd[2].x : j == 1 ? wd[2].y : j == 2 ? wd[2].z : wd[2].w,
                                j == 0 ? wd[3].x : j == 1 ? wd[3].y : j == 2 ? wd[3].z : wd[3].w};
       if (j == 0)
-        quad4<true, M>(su, idx, lce, xq);
+        quad4<true, M>(su, idx, lce, xq, ck);
       else
-        quad4<false, M>(su, idx, lce, xq);
+        quad4<false, M>(su, idx, lce, xq, ck);
     }
   } else {
     // lo u32 j goes with hi u32 j; lo word 1 reads its hi fields two bits up
@@ -433,13 +459,13 @@ __device__ __forceinline__ void unit_partial(float (&su)[4][M], const uint4 (&wd
         e[i] = (l & 0x0F0F0F0Fu) | (h & 0xF0F0F0F0u);
         o[i] = (l & 0xF0F0F0F0u) | (h & 0x0F0F0F0Fu);
       }
-      load_xq<M>(xq, xa + 32u * j, xstride);
+      load_xq<M>(xq, xa + 32u * j, xstride, ck);
       if (j == 0)
-        quad4<true, M>(su, e, lce, xq);
+        quad4<true, M>(su, e, lce, xq, ck);
       else
-        quad4<false, M>(su, e, lce, xq);
-      load_xq<M>(xq, xa + 32u * j + 16u, xstride);
-      quad4<false, M>(su, o, lco, xq);
+        quad4<false, M>(su, e, lce, xq, ck);
+      load_xq<M>(xq, xa + 32u * j + 16u, xstride, ck);
+      quad4<false, M>(su, o, lco, xq, ck);
     }
   }
 }
@@ -564,11 +590,17 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
     if (threadIdx.x == 0) report(a.status, LUTQ_ERR_CUDA);
     return;
   }
+  // checked builds: the window (tables, activations, slots) lies inside the
+  // block's dynamic shared memory
+  if (!LUTQ_IN_BOUNDS(small_end(K, M, kLutRegion) - sbase <= a.smem_bytes, a.status)) return;
 
   auto fetch = [&](uint4 (&wd)[4], uint32_t (&sv)[2], uint32_t& ty) {
+    // checked builds: a unit past the packed matrix is not loaded
+    int live = fn;
+    if (fn > 0 && !LUTQ_IN_BOUNDS(ft < uint32_t(a.U), a.status)) live = 0;
     fetch_unit<BITS>(wd, sv, wide_addr(pk, ft, TB), hi_delta,
-                     wide_addr(psc, ft, uint32_t(SB)), fn);
-    if (TYPED) fetch_type_byte(ty, wide_addr(pty, ft, uint32_t(kTypeBytes)), fn);
+                     wide_addr(psc, ft, uint32_t(SB)), live);
+    if (TYPED) fetch_type_byte(ty, wide_addr(pty, ft, uint32_t(kTypeBytes)), live);
     --fn;
     ++ft;
     if (--fleft == 0) {  // on to the window's first group of the next strip
@@ -665,6 +697,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
 #pragma unroll
   for (int i = 0; i < 4; ++i) rows[i] = rq + 8 * i;
   const uint32_t xstride = K * 2u;
+  const Checks ck = {kLutRegion, kXAt + uint32_t(M) * xstride, a.status};
   // the lane's activations of the window's first group, batch row 0
   const uint32_t xa_w = kXAt + sp.ga * kXGroupBytes + uint32_t(q) * kXChunkBytes;
 
@@ -703,7 +736,7 @@ __global__ void __launch_bounds__(kM1Warps * 32, 1) gemv_small_kernel(GemvArgs a
           report(a.status, LUTQ_ERR_CODE_RANGE);
       }
       float su[4][M];
-      unit_partial<BITS, M>(su, wd, lce, lco, hi_shift, xa, xstride);
+      unit_partial<BITS, M>(su, wd, lce, lco, hi_shift, xa, xstride, ck);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float s = (i & 1) ? bf16_hi_to_f32(sv[i >> 1]) : bf16_lo_to_f32(sv[i >> 1]);
@@ -882,6 +915,7 @@ static cudaError_t launch_small(GemvArgs a, int num_sms, cudaStream_t stream) {
   cfg.gridDim = dim3(unsigned(a.C) + a.pf_ctas);
   cfg.blockDim = dim3(kM1Warps * 32);
   cfg.dynamicSmemBytes = size_t(smem);
+  a.smem_bytes = uint32_t(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -11,6 +11,8 @@
 
 #include <cstdint>
 
+#include "lutq_common.cuh"
+
 namespace lutq {
 
 constexpr int kLutBytes = 256 * 256;  // 64 KB
@@ -112,11 +114,17 @@ __device__ __forceinline__ uint32_t lds32(uint32_t smem_addr) {
   return v;
 }
 
-// Four pair indices (the bytes of idx) -> four bf16x2 code pairs.
+// Four pair indices (the bytes of idx) -> four bf16x2 code pairs.  Checked
+// builds compare each table offset with lut_limit (the table region's size)
+// and report through st; other builds ignore both.
 __device__ __forceinline__ void lookup4(uint32_t* lv, uint32_t idx, uint32_t lut_base,
-                                        uint32_t lane_off) {
+                                        uint32_t lane_off, uint32_t lut_limit = 0x20000u,
+                                        int32_t* st = nullptr) {
 #pragma unroll
-  for (int b = 0; b < 4; ++b) lv[b] = lds32(lut_base + lut_addr(idx, lane_off, b));
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t t = lut_addr(idx, lane_off, b);
+    lv[b] = LUTQ_IN_BOUNDS(t + 4u <= lut_limit, st) ? lds32(lut_base + t) : 0u;
+  }
 }
 
 // The four 32-bit index words of one 3-bit group row, j-th u32 of the two lo
@@ -168,13 +176,15 @@ __device__ __forceinline__ void decode_group_row(uint32_t (&out)[64], const uint
 template <int BITS>
 __device__ __forceinline__ void decode_group_half(uint32_t (&out)[32], const uint4 (&wd)[2],
                                                   int h, uint32_t lut_base, uint32_t off_e,
-                                                  uint32_t off_o) {
+                                                  uint32_t off_o, uint32_t lut_limit = 0x20000u,
+                                                  int32_t* st = nullptr) {
   if (BITS == 4) {
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       const uint32_t v[4] = {wd[w].x, wd[w].y, wd[w].z, wd[w].w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) lookup4(out + 16 * w + 4 * j, v[j], lut_base, off_e);
+      for (int j = 0; j < 4; ++j)
+        lookup4(out + 16 * w + 4 * j, v[j], lut_base, off_e, lut_limit, st);
     }
   } else {
     const uint32_t L[4] = {wd[0].x, wd[0].y, wd[0].z, wd[0].w};
@@ -182,8 +192,10 @@ __device__ __forceinline__ void decode_group_half(uint32_t (&out)[32], const uin
     const uint32_t H[4] = {wd[1].x >> sh, wd[1].y >> sh, wd[1].z >> sh, wd[1].w >> sh};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      lookup4(out + 8 * j, (L[j] & 0x0F0F0F0Fu) | (H[j] & 0xF0F0F0F0u), lut_base, off_e);
-      lookup4(out + 8 * j + 4, (L[j] & 0xF0F0F0F0u) | (H[j] & 0x0F0F0F0Fu), lut_base, off_o);
+      lookup4(out + 8 * j, (L[j] & 0x0F0F0F0Fu) | (H[j] & 0xF0F0F0F0u), lut_base, off_e,
+              lut_limit, st);
+      lookup4(out + 8 * j + 4, (L[j] & 0xF0F0F0F0u) | (H[j] & 0x0F0F0F0Fu), lut_base, off_o,
+              lut_limit, st);
     }
   }
 }

@@ -26,6 +26,7 @@
 #include <cuda_runtime.h>
 
 #include "lutq.h"
+#include "lutq_trace.h"
 #include "lutq_common.cuh"
 
 namespace lutq {
@@ -58,6 +59,7 @@ extern "C" lutq_status lutq_gemv_noalloc(const void* x_bf16, int64_t M, const vo
                                          const void* codebook_bf16, int bits, int64_t N,
                                          int64_t K, float* y, int32_t* dev_status,
                                          void* stream) {
+  LUTQ_TRACE_RANGE("lutq_gemv_noalloc");
   if (!x_bf16 || !packed || !codebook_bf16 || !y) return LUTQ_ERR_INVALID_ARG;
   if (bits != 3 && bits != 4) return LUTQ_ERR_BITS;
   if (N < lutq::kStrip || K < lutq::kGroup || N % lutq::kStrip != 0 || K % lutq::kGroup != 0 ||

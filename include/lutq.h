@@ -51,8 +51,26 @@ typedef enum {
                                product a group type without a table */
   LUTQ_ERR_TIMEOUT = 7,     /* device: a bounded wait inside a kernel expired */
   LUTQ_ERR_CUDA = 8,        /* a CUDA runtime call failed */
-  LUTQ_ERR_WORKSPACE = 9    /* workspace missing or smaller than required */
+  LUTQ_ERR_WORKSPACE = 9,   /* workspace missing or smaller than required */
+  LUTQ_ERR_BOUNDS = 10      /* device, checked builds only (LUTQ_BUILD_BOUNDS): an
+                               index fell outside its buffer; that access was
+                               skipped, so the results are unspecified */
 } lutq_status;
+
+/*
+ * lutq_build_flags - how this library was compiled: a bit mask of
+ * LUTQ_BUILD_NVTX (every C-ABI call opens an NVTX range named after the call,
+ * for Nsight timelines; compiled with -DLUTQ_NVTX) and LUTQ_BUILD_BOUNDS (the
+ * kernels check their global, shared and tensor-memory indices against the
+ * buffers' extents and report LUTQ_ERR_BOUNDS through dev_status instead of
+ * making the access; compiled with -DLUTQ_BOUNDS, slower, for debugging).
+ * The default build returns 0.  No GPU use.
+ *
+ * No counterpart in the paper: these are tooling options of the library.
+ */
+#define LUTQ_BUILD_NVTX 1
+#define LUTQ_BUILD_BOUNDS 2
+int lutq_build_flags(void);
 
 /* Codebook kinds for lutq_codebook. */
 typedef enum {
@@ -339,6 +357,20 @@ lutq_status lutq_gemv_plan(int64_t N, int64_t K, int num_sms, int32_t* plan);
  * 1 .. 1e9.
  */
 lutq_status lutq_selftest_wait_timeout(int32_t* dev_status, int64_t limit_ns, void* stream);
+
+/*
+ * lutq_selftest_bounds - checks the device-side index checks.
+ *
+ * No counterpart in the paper.  Runs one kernel that writes a shared array
+ * through the kernels' index check with an index one past the extent the
+ * check is given (the array itself is larger, so no build makes an access
+ * outside memory).  In a build with LUTQ_BUILD_BOUNDS the check skips the
+ * write and *dev_status (device int32, required) receives LUTQ_ERR_BOUNDS
+ * unless it already held an error; in other builds the check is compiled out
+ * and *dev_status is left as it is.  Asynchronous on `stream`.  Returns
+ * LUTQ_ERR_INVALID_ARG for a NULL dev_status.
+ */
+lutq_status lutq_selftest_bounds(int32_t* dev_status, void* stream);
 
 /*
  * lutq_fit_histogram / lutq_fit_codebook - a codebook fitted to a layer.

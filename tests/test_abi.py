@@ -48,7 +48,7 @@ def test_layout_version_and_sizes(lq):
 
 
 def test_status_strings(lq):
-    for code in range(10):
+    for code in range(11):
         assert lq.lutq_status_string(code).startswith(lq._binding.STATUS_NAMES[code])
     assert "unknown" in lq.lutq_status_string(99)
 
@@ -95,7 +95,8 @@ def test_pack_argument_errors(lq):
     assert f(A, A + 2, 32, 128, 4, A, None, None) == 4            # misaligned scales
 
 
-@pytest.mark.parametrize("name", ["lutq_gemv", "lutq_gemm"])
+@pytest.mark.parametrize("name", ["lutq_gemv", "lutq_gemm", "lutq_gemv_group64",
+                                  "lutq_gemm_group64"])
 def test_product_argument_errors(lq, name):
     f = getattr(lq.lib, name)
     ws = lq.lutq_workspace_bytes(1, 64, 256, 4)
@@ -113,7 +114,7 @@ def test_product_argument_errors(lq, name):
     assert call(n=48) == 2
     assert call(k=200) == 2
     assert call(m=0) == 2
-    if name == "lutq_gemv":
+    if name.startswith("lutq_gemv"):
         assert call(m=17) == 2
     assert call(y=A + 4) == 4
     if ws > 0:
@@ -209,3 +210,42 @@ def test_group256_needs_k_multiple_of_256(lq):
     f = lq.lib.lutq_quantize_group256
     assert f(A, 32, 384, A, 4, A, A, None, None) == 2
     assert f(A, 32, 128, A, 4, A, A, None, None) == 2
+
+
+def test_group64_sizes_and_argument_errors(lq):
+    for n, k, bits in [(4096, 14336, 4), (4096, 4096, 3), (32, 128, 4)]:
+        assert lq.lutq_packed_bytes_group64(n, k, bits) == \
+            lq.lutq_packed_bytes(n, k, bits) + (n // 32) * (k // 128) * 64
+    assert lq.lutq_packed_bytes_group64(33, 128, 4) == -1
+    assert lq.lutq_packed_bytes_group64(32, 128, 2) == -1
+    q, p = lq.lib.lutq_quantize_group64, lq.lib.lutq_pack_group64
+    assert q(None, 32, 128, A, 4, A, A, None, None) == 1
+    assert q(A, 32, 100, A, 4, A, A, None, None) == 2
+    assert q(A, 32, 128, A, 5, A, A, None, None) == 3
+    assert q(A, 32, 128, A, 4, A, A + 2, None, None) == 4
+    assert p(None, A, 32, 128, 4, A, None, None) == 1
+    assert p(A, A, 40, 128, 4, A, None, None) == 2
+    assert p(A, A + 2, 32, 128, 4, A, None, None) == 4
+
+
+def _variant_lib(name):
+    path = os.path.join(ROOT, "dequant_gemv_group_b200", f"liblutq_{name}.so")
+    if not os.path.exists(path):
+        pytest.skip(f"liblutq_{name}.so is not built")
+    return ctypes.CDLL(path)
+
+
+def test_build_flags_of_each_build(lq):
+    # the product build has neither tooling option; the variants one each,
+    # and export the same functions
+    assert lq.lutq_build_flags() == 0
+    declared = _header_functions()
+    for name, flag in (("nvtx", lq.BUILD_NVTX), ("bounds", lq.BUILD_BOUNDS)):
+        lib = _variant_lib(name)
+        assert lib.lutq_build_flags() == flag
+        for fn in declared:
+            assert hasattr(lib, fn), (name, fn)
+
+
+def test_selftest_bounds_argument_error(lq):
+    assert lq.lib.lutq_selftest_bounds(None, None) == 1
