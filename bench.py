@@ -54,6 +54,9 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=5000)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-side", action="store_true", help="skip the GEMM and offline lines")
+    p.add_argument("--table", action="store_true",
+                   help="instead of the JSON line: every workload x layer x codebook x batch, "
+                        "plus batches 17-31 and one scale per group of 64, as a markdown table")
     return p.parse_args()
 
 
@@ -554,6 +557,88 @@ def side_measurements(lq, dev, args):
     return out
 
 
+# batches between the GEMV's 16 and 32 on the 70B-shaped layers, and the
+# group-64 cases of the per-configuration table
+TABLE_EXTRA_BATCHES = {"llama3_70b_mlp": (17, 20, 24, 28, 31)}
+TABLE_GROUP64 = {("llama3_8b_w4_nf4", "down"): (1, 4, 16, 32, 128),
+                 ("llama3_70b_mlp", "gate_up"): (1, 4, 16, 32, 128)}
+
+
+def run_table(args):
+    """Per-configuration table: each product graph-replayed (9 replays of 64
+    calls behind a spin kernel, weights rotating over copies larger than 3x
+    L2); median (p10-p90) microseconds per call, GB/s of algorithmic bytes,
+    percent of 8 TB/s and TFLOP/s, one markdown row each."""
+    import dequant_gemv_group_b200 as lq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    print("| config | layer | W[N,K] | codebook | group | M | call | us median (p10-p90) "
+          "| GB/s | % of 8 TB/s | TFLOP/s |")
+    print("|---|---|---|---|---|---|---|---|---|---|---|")
+
+    def sweep(wname, lay, kind, bits, group, batches, packed, cb):
+        n, k = lay.n, lay.k
+        per = packed.numel()
+        copies = max(2, int(np.ceil(3 * l2 / per)) + 1)
+        packs = [packed] + [packed.clone() for _ in range(copies - 1)]
+        st = lq.new_status(dev)
+        for m in batches:
+            if group == 64:
+                fn = lq.lutq_gemv_group64 if m <= 16 else lq.lutq_gemm_group64
+            else:
+                fn = lq.lutq_gemv if m <= 16 else lq.lutq_gemm
+            x = workloads.activations(m, k, seed=1).to(dev)
+            y = torch.empty((m, n), device=dev)
+            ws = lq.new_workspace(m, n, k, bits, dev)
+            step = lambda i: fn(x, packs[i % copies], cb, bits, n, k, y=y, workspace=ws,
+                                status=st)
+            for i in range(5):
+                step(i)
+            g = capture(step, 64)
+            g.replay()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(9):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                hold_stream()
+                e0.record()
+                g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3 / 64)
+            assert int(st.item()) == 0, (wname, lay.name, m)
+            med, p10, p90 = np.median(ts), np.percentile(ts, 10), np.percentile(ts, 90)
+            gbs = (per + m * k * 2 + m * n * 4) / med / 1e3
+            tf = 2.0 * m * n * k / med / 1e6
+            print(f"| {wname} | {lay.name} | {n}x{k} | {kind} W{bits} | {group} | {m} | "
+                  f"{fn.__name__} | {med:.2f} ({p10:.2f}-{p90:.2f}) | {gbs:.0f} | "
+                  f"{gbs / 80:.1f} | {tf:.1f} |", flush=True)
+            del g, x, y, ws
+        del packs
+
+    for wname, wl in workloads.WORKLOADS.items():
+        for lay in wl.layers:
+            w = lay.weights(seed=0).to(dev)
+            for kind, bits in wl.codebooks:
+                cb = lq.lutq_codebook(kind, bits).to(dev)
+                codes, scales = lq.lutq_quantize(w, cb, bits)
+                packed = lq.lutq_pack(codes, scales, bits)
+                del codes, scales
+                batches = tuple(sorted(set(wl.batches) | set(TABLE_EXTRA_BATCHES.get(wname, ()))))
+                sweep(wname, lay, kind, bits, 128, batches, packed, cb)
+                del packed
+                g64 = TABLE_GROUP64.get((wname, lay.name))
+                if g64 and bits == 4:
+                    codes, scales = lq.lutq_quantize_group64(w, cb, bits)
+                    packed = lq.lutq_pack_group64(codes, scales, bits)
+                    del codes, scales
+                    sweep(wname, lay, kind, bits, 64, g64, packed, cb)
+                    del packed
+            del w
+            torch.cuda.empty_cache()
+
+
 def run_lutq(args, world, rank, local):
     import dequant_gemv_group_b200 as lq
     dev = torch.device("cuda", local)
@@ -731,6 +816,9 @@ def run_lutq(args, world, rank, local):
 
 def main():
     args = parse()
+    if args.table:
+        run_table(args)
+        return
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

@@ -4,22 +4,26 @@
 // dequantization with the matmul; the BitMoD abstract, same listing: the
 // per-group partial sum is rescaled once).
 //
-// Roles of the 10 warps of a CTA (one CTA per SM, persistent):
-//   warps 0-3  dequantize: lane r of warp w owns row 32 w + r of the 128-row
-//              tile; it decodes the row's 128 codes of one group through the
-//              lane-duplicated pair table into 64 bf16 pairs and stores them
-//              into tensor memory (lane = row, column j = codes 2j, 2j+1) as
-//              the A operand of the MMA (W is the M side: swap-AB).
-//   warps 4-7  promote: read the group's fp32 partial D[row, batch] from
-//              tensor memory, add s[row, g] * partial to registers, and write
-//              y (or a split partial) when the row tile's range ends.
-//   warp 8     loads the activations' 128-wide K slice (two 2-D tensor-map
-//              copies, 128-byte swizzle); the dequantize warps load their
-//              rows' packed words themselves, straight into registers.
-//   warp 9     issues tcgen05.mma (for batch tiles of 16 or 32, warps 9 and
-//              10 take alternate units) kind::f16 (A from tensor memory, B from
-//              shared memory, D fp32 in tensor memory), 8 MMAs of K = 16 per
-//              group into a fresh partial, and commits to the mbarriers.
+// Roles of the warps of a CTA (one CTA per SM, persistent; the counts depend
+// on the batch tile N_tile, GemmCfg):
+//   DW dequantize warps (4 at N_tile >= 64, else 8: two per lane quarter,
+//              each taking half of the row's codes): lane r of warp w owns
+//              row 32 (w mod 4) + r of the 128-row tile; it decodes its codes
+//              of one group through the lane-duplicated pair table into bf16
+//              pairs and stores them into tensor memory (lane = row, column
+//              j = codes 2j, 2j+1) as the A operand of the MMA (W is the M
+//              side: swap-AB).  The warps load their rows' packed words
+//              themselves, straight into registers.
+//   4 PG promotion warps (PG = 2 at N_tile = 128, each group owning half of
+//              the batch columns): read the group's fp32 partial D[row, batch]
+//              from tensor memory, add s[row, g] * partial to registers, and
+//              write y (or a split partial) when the row tile's range ends.
+//   1 activation warp: loads the activations' 128-wide K slice (two 2-D
+//              tensor-map copies, 128-byte swizzle, no multicast).
+//   MW MMA warps (2 at N_tile <= 32, taking alternate units; else 1): issue
+//              tcgen05.mma kind::f16 (A from tensor memory, B from shared
+//              memory, D fp32 in tensor memory), 8 MMAs of K = 16 per group
+//              into a fresh partial, and commit to the mbarriers.
 // With one scale per group of 64 (G64) each unit has two partials, one per
 // 64-half (MMAs 0-3 and 4-7, each into its own partial stage), and the
 // promotion warps add s[row, 2g] * first + s[row, 2g + 1] * second.

@@ -1,10 +1,11 @@
-// Fused dequantize-and-multiply GEMV for batches M = 1..16 on the CUDA cores
-// (the FLUTE abstract, "Daily Papers" listing, query "group-128": fuse
+// Fused dequantize-and-multiply GEMV on the CUDA cores for batches M = 1..4
+// (lutq_gemv takes M = 1..16; larger batches go to the tensor-core kernel of
+// lutq_gemm.cu) (the FLUTE abstract, "Daily Papers" listing, query "group-128": fuse
 // dequantization with the product; duplicate and vectorize the lookup table
 // against shared-memory bandwidth limits.  The BitMoD abstract, same listing:
 // rescale each group's partial sum once).
 //
-// Work split (both kernels).  The packed matrix is a sequence of
+// Work split.  The packed matrix is a sequence of
 // U = (N/32) * G units, one unit = (strip of 32 rows, group of 128 codes) =
 // 2048 (4-bit) or 1536 (3-bit) contiguous bytes.  A plan (choose_plan) gives
 // each CTA of a grid of at most one CTA per SM a run of units: whole strips,
@@ -58,7 +59,7 @@ constexpr int kMaxCtas = 512;           // bounds the workspace
 #ifndef LUTQ_M1_WARPS
 #define LUTQ_M1_WARPS 16
 #endif
-constexpr int kM1Warps = LUTQ_M1_WARPS; // warps per CTA, M = 1 kernel
+constexpr int kM1Warps = LUTQ_M1_WARPS; // warps per CTA of the small-batch kernel
 constexpr int kMaxSmemPerBlock = 227 * 1024;
 
 struct GemvArgs {
