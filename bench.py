@@ -664,6 +664,10 @@ def run_lutq(args, world, rank, local):
     ws = lq.new_workspace(m, n, k, bits, dev)
     use_gemm = m > 16
     call = lq.lutq_gemm if use_gemm else lq.lutq_gemv
+    # the kernel that runs the step: lutq_gemv keeps batches of up to 4 on the
+    # CUDA cores when M (K + 2048) <= 80896 (the activations fit its shared
+    # memory, include/lutq.h) and hands the others to the tensor-core kernel
+    cuda_core = (not use_gemm) and m <= 4 and m * (k + 2048) <= 80896
 
     def step(i):
         j = i % copies
@@ -785,9 +789,9 @@ def run_lutq(args, world, rank, local):
                    "steady_state_gbs": nbytes / steady_us / 1e3},
         "roofline": {"bound": "hbm", "achieved": gbs_rank, "peak": hbm_peak, "unit": "GB/s",
                      "frac": gbs_rank / hbm_peak, "peak_source": peak_kind,
-                     "bytes_per_launch": nbytes, "traffic": ncu_traffic(kernel_key,
-                                                                    GEMM_SOURCES if use_gemm else GEMV_SOURCES),
-                     "kernel": "lutq::gemv_small_kernel" if not use_gemm else "lutq::gemm_kernel"},
+                     "bytes_per_launch": nbytes,
+                     "traffic": ncu_traffic(kernel_key, GEMV_SOURCES if cuda_core else GEMM_SOURCES),
+                     "kernel": "lutq::gemv_small_kernel" if cuda_core else "lutq::gemm_kernel"},
         "pct_of_8TBs": gbs_rank / 8000.0,
         "plain_launch_gbs": plain_gbs,
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": m * k * 2,
