@@ -53,7 +53,7 @@ constexpr int kTileRows = 128;
 constexpr int kGemmMaxCtas = 256;            // bounds the workspace
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kTmemCols = 512;
-template <int NT, bool G64 = false>
+template <int NT, bool G64 = false, bool TYPED = false>
 struct GemmCfg {
   // activation stages (shared memory); two at N_tile = 128 leave 32 KB more
   // to L1 (measured 2% faster at batch 128 than three; four: 25% slower)
@@ -64,7 +64,16 @@ struct GemmCfg {
   // stages, so the stages go to the partials: at N_tile = 128 two A stages
   // and three partial stages, below it as many partial stages as fit (at
   // most 8).
-  static constexpr int AS = (G64 && NT >= 128) ? 2 : 4;
+  // TACC: the typed kernel at N_tile = 128 keeps the promotion warps'
+  // running sums in tensor memory (NT columns after the partial stages)
+  // instead of registers.  In registers 64 sums a thread spill under the
+  // 128-register ceiling of 14 warps, and with the typed kernel's larger
+  // table region the spills miss in the L1 that remains (four 4-bit types:
+  // 34% slower than the untyped kernel with register sums, 6% with these);
+  // the untyped kernel, whose spills stay in L1, is 2% faster with
+  // registers.  The sums take two A stages' columns.
+  static constexpr bool TACC = TYPED && NT >= 128 && !G64;
+  static constexpr int AS = ((G64 || TACC) && NT >= 128) ? 2 : 4;
   static constexpr int DS = G64 ? ((kTmemCols - 64 * AS) / NT < 8 ? (kTmemCols - 64 * AS) / NT : 8)
                                 : (NT >= 128 ? 2 : (NT >= 64 ? 3 : 4));
   static constexpr int DW = NT >= 64 ? 4 : 8;       // dequant warps (8: two per lane quarter)
@@ -76,10 +85,14 @@ struct GemmCfg {
   static constexpr int WARPS = DW + 4 * PG + 1 + MW;  // dequant, promote, activation load, MMA
   static constexpr int THREADS = 32 * WARPS;
   static constexpr int DCOL = 64 * AS;              // first partial column
-  static_assert(DCOL + DS * NT <= kTmemCols, "tensor memory columns");
+  static constexpr int ACOL = DCOL + DS * NT;       // first running-sum column (TACC)
+  static_assert(ACOL + (TACC ? NT : 0) <= kTmemCols, "tensor memory columns");
 };
 constexpr int kMaxPromoteGroups = 2;
 constexpr int kScaleRingBytes = 4 * kMaxPromoteGroups * 4 * 32 * 4;  // [warp][SD][lane] u32
+// per-group types: the dequant warps' type words travel through a ring of
+// asynchronous copies, [warp][NB][lane] u32 (at most 8 warps x 4 units)
+constexpr int kTypeRingBytes = 8 * 4 * 32 * 4;
 
 struct GemmArgs {
   const uint8_t* packed;
@@ -243,7 +256,7 @@ __device__ __forceinline__ void tmem_st_cols32(uint32_t taddr, const uint32_t (&
 template <int BITS, int NT, bool TYPED, bool G64>
 __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, GemmArgs a) {
-  using Cfg = GemmCfg<NT, G64>;
+  using Cfg = GemmCfg<NT, G64, TYPED>;
   static_assert(!(TYPED && G64), "per-group types use one scale per group of 128");
   // partials per unit (one per scale), the scale block's bytes
   constexpr int H = G64 ? 2 : 1;
@@ -277,7 +290,8 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
   uint16_t* cbs = reinterpret_cast<uint16_t*>(misc + 8);
   // checked builds: table, activation stages, barriers, flags, codebook copy
   // and the scale rings lie inside the block's dynamic shared memory
-  if (!LUTQ_IN_BOUNDS(bar_sa + 512u + uint32_t(kScaleRingBytes * H) - raw_sa <=
+  if (!LUTQ_IN_BOUNDS(bar_sa + 512u + uint32_t(kScaleRingBytes * H) +
+                              uint32_t(TYPED ? kTypeRingBytes : 0) - raw_sa <=
                           uint32_t(a.smem_bytes) &&
                           8u * NBAR + 8u + 2u * uint32_t(a.ntypes << BITS) <= 512u,
                       a.dev_status))
@@ -342,45 +356,59 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     fp.init(u0, per_bt, a.G);
     int fetched = 0;
     // per-group types: the lane's row is lane (rq = lane & 7, i = lane >> 3)
-    // of its strip; its type is bits 2i+1:2i of byte rq of the unit's block
-    auto fetch = [&](uint4 (&wd)[NWL], uint32_t& ty) {
+    // of its strip; its type is bits 2i+1:2i of byte rq of the unit's block,
+    // i.e. bits 8 (lane & 3) + 2i of the block's 4-byte word lane & 4.  That
+    // word travels through a ring slot per unit in shared memory (one 4-byte
+    // asynchronous copy and one copy group per lane and unit, NB units
+    // ahead): a register load per unit beside the code words made the
+    // kernel 30% slower at N_tile = 16, even with its value read only at the
+    // end.
+    const uint32_t ty_ring =
+        bar_sa + 512u + uint32_t(kScaleRingBytes * H) + uint32_t(warp * NB * 32 + lane) * 4u;
+    auto fetch = [&](uint4 (&wd)[NWL], int slot) {
       if (fetched < n && fp.tau * kTileRows + sw * 32 < a.N &&
           LUTQ_IN_BOUNDS((fp.tau * 4 + sw) * a.G + fp.g < (a.N / kStrip) * a.G, a.dev_status)) {
         const int64_t tile = (fp.tau * 4 + sw) * a.G + fp.g;
         const uint8_t* t = a.packed + tile * TB + lane * 16;
 #pragma unroll
         for (int j = 0; j < NWL; ++j) wd[j] = ld_stream_v4(t + word_of(j) * 512);
-        if (TYPED)  // issued here, with the unit's words (a plain load may sink to its use)
-          asm volatile("ld.global.nc.u8 %0, [%1];"
-                       : "=r"(ty) : "l"(a.types + tile * kTypeBytes + (lane & 7)));
+        if (TYPED)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
+                       ::"r"(ty_ring + uint32_t(slot * 32 * 4)),
+                       "l"(a.types + tile * kTypeBytes + (lane & 4))
+                       : "memory");
       }
+      if (TYPED) asm volatile("cp.async.commit_group;" ::: "memory");
       ++fetched;
       fp.next(a.G, a.ntiles);
     };
     uint4 ring[NB][NWL];
-    uint32_t tyring[NB];
 #pragma unroll
-    for (int t = 0; t < NB; ++t) {
-      tyring[t] = 0;
-      fetch(ring[t], tyring[t]);
-    }
+    for (int t = 0; t < NB; ++t) fetch(ring[t], t);
     UnitPos pos;
     pos.init(u0, per_bt, a.G);
     bool ok = true;
+    bool bad_type = false;  // a stored type without a table in this call
     // the row's table: 4-bit, type bit 0 -> address bit 7 (row half), bit 1
     // -> bit 16; 3-bit, type bit 0 -> bit 16 (through byte 1 of the column
     // word), masked to the table region, so that a type >= ntypes reads an
     // unfilled table inside it, never the activation stages
     auto sel_of = [&](uint32_t ty) -> uint32_t {
       if (!TYPED) return 0u;
-      const uint32_t f = (ty >> (2 * (lane >> 3))) & 3u;
+      const uint32_t f = (ty >> (8 * (lane & 3) + 2 * (lane >> 3))) & 3u;
       return (BITS == 4 ? ((f & 1u) << 7) | ((f >> 1) << 8) : (f & 1u) << 8) &
              ((BITS == 4 ? 0x080u : 0u) | (LUTB > kLutBytes ? 0x100u : 0u));
     };
     // decode unit i from wd, refill wd with unit i + NB, hand the tile to the MMA
-    auto step = [&](uint4 (&wd)[NWL], uint32_t& ty, int i) {
+    auto step = [&](uint4 (&wd)[NWL], int slot, int i) {
       const bool valid = pos.tau * kTileRows + sw * 32 < a.N;
       uint32_t av[32];
+      uint32_t ty = 0;
+      if (TYPED) {
+        // this unit's copy group is complete once at most NB - 1 are pending
+        asm volatile("cp.async.wait_group %0;" ::"n"(NB - 1) : "memory");
+        ty = lds32(ty_ring + uint32_t(slot * 32 * 4));
+      }
       const uint32_t sel = sel_of(ty);
       // a warp that owns the whole row (DW = 4) decodes it in two halves of
       // 32 pairs, storing each before decoding the next (32 registers of
@@ -393,14 +421,14 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         h1[1] = wd[BITS == 4 ? 3 : 2];
       }
       if (valid) {
-        // a stored type without a table in this call is reported
-        if (TYPED && ((ty >> (2 * (lane >> 3))) & 3u) >= uint32_t(a.ntypes))
-          report(a.dev_status, LUTQ_ERR_CODE_RANGE);
+        // a stored type without a table in this call is reported (once, after the loop)
+        if (TYPED)
+          bad_type |= ((ty >> (8 * (lane & 3) + 2 * (lane >> 3))) & 3u) >= uint32_t(a.ntypes);
         const uint4 h0[2] = {wd[0], wd[DW == 8 ? 1 : (BITS == 4 ? 1 : 2)]};
         decode_group_half<BITS>(av, h0, DW == 8 ? kh : 0, lut_sa, off_e | sel, off_o | sel,
                                 uint32_t(LUTB), a.dev_status);
       }
-      fetch(wd, ty);
+      fetch(wd, slot);
       const int as = i % AS;
       ok = mbar_wait(bar(B_AE + as), (uint32_t(i / AS) & 1u) ^ 1u, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -427,8 +455,12 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
 #pragma unroll
       for (int t = 0; t < NB; ++t) {
         if (i + t >= n || !ok) break;
-        step(ring[t], tyring[t], i + t);
+        step(ring[t], t, i + t);
       }
+    }
+    if (TYPED) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      if (bad_type) report(a.dev_status, LUTQ_ERR_CODE_RANGE);
     }
   } else if (warp < W_XLOAD) {
     // ---------------------------------------------------------------- promote
@@ -470,6 +502,10 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
 #pragma unroll
     for (int j = 0; j < NC; ++j) acc[j] = 0.0f;
     constexpr int CH = chunk_cols<NC>();
+    // TACC: the warp's running sums in tensor memory, its lanes and columns
+    // ACOL + pg * NC ..; fresh while the current row tile's range has none
+    const uint32_t tacc = tmem + (uint32_t(sw * 32) << 16) + uint32_t(Cfg::ACOL + pg * NC);
+    bool fresh = true;
     for (int i = 0; i < n; ++i) {
       const int64_t row = cur.tau * kTileRows + sw * 32 + lane;
       const bool valid = cur.tau * kTileRows + sw * 32 < a.N;
@@ -491,20 +527,53 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         tc_fence_after();
         const uint32_t tpart = tmem + (uint32_t(sw * 32) << 16) +
                                uint32_t(Cfg::DCOL + ds * NT + pg * NC);
+        if (Cfg::TACC) {
+          // sum += s * partial, one 32-column chunk at a time; this thread's
+          // stores of the previous unit are complete before it reads back
+          if (!fresh) tmem_wait_st();
 #pragma unroll
-        for (int c = 0; c < NC / CH; ++c) {
-          uint32_t v[32];
-          tmem_ld_cols<NC>(tpart + uint32_t(c * CH), v);
-          tmem_wait_ld();
+          for (int c = 0; c < NC / 32; ++c) {
+            uint32_t v[32], u[32];
+            tmem_ld_32x32b_x32(tpart + uint32_t(c * 32), v);
+            if (!fresh) tmem_ld_32x32b_x32(tacc + uint32_t(c * 32), u);
+            tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < CH; ++j)
-            acc[c * CH + j] = fmaf(s[h], __uint_as_float(v[j]), acc[c * CH + j]);
+            for (int j = 0; j < 32; ++j)
+              u[j] = __float_as_uint(fresh ? s[h] * __uint_as_float(v[j])
+                                           : fmaf(s[h], __uint_as_float(v[j]),
+                                                  __uint_as_float(u[j])));
+            tmem_st_cols32(tacc + uint32_t(c * 32), u);
+          }
+          fresh = false;
+        } else {
+#pragma unroll
+          for (int c = 0; c < NC / CH; ++c) {
+            uint32_t v[32];
+            tmem_ld_cols<NC>(tpart + uint32_t(c * CH), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < CH; ++j)
+              acc[c * CH + j] = fmaf(s[h], __uint_as_float(v[j]), acc[c * CH + j]);
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_DE + ds));
       }
       if (cur.g == a.G - 1 || i == n - 1) {
+        if (Cfg::TACC) {
+          // the range's sums into registers for the strip's write-out
+          tmem_wait_st();
+#pragma unroll
+          for (int c = 0; c < NC / 32; ++c) {
+            uint32_t u[32];
+            tmem_ld_32x32b_x32(tacc + uint32_t(c * 32), u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = __uint_as_float(u[j]);
+          }
+          fresh = true;
+        }
         if (valid)
           gemm_finish_strip<NT, NC>(a, acc, cur.bt * a.ntiles + cur.tau, cur.bt, row, sw, pg, u0,
                                     lane);
@@ -650,12 +719,12 @@ static cudaError_t make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_
 template <int BITS, int NT, bool TYPED, bool G64>
 static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
                              cudaStream_t stream) {
-  using Cfg = GemmCfg<NT, G64>;
+  using Cfg = GemmCfg<NT, G64, TYPED>;
   static int granted[64] = {0};
   // alignment slack, table, activation stages, barriers and flags (512),
   // the promotion warps' scale rings (two scales per lane and unit with G64)
-  const int smem =
-      1024 + a.lut_bytes + Cfg::XS * Cfg::XSTAGE + 512 + kScaleRingBytes * (G64 ? 2 : 1);
+  const int smem = 1024 + a.lut_bytes + Cfg::XS * Cfg::XSTAGE + 512 +
+                   kScaleRingBytes * (G64 ? 2 : 1) + (TYPED ? kTypeRingBytes : 0);
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
