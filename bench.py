@@ -337,6 +337,27 @@ def hold_stream(cycles=200_000):
     torch.cuda._sleep(int(cycles))
 
 
+def time_graph(fn, count, replays=5):
+    """Median device time per call of fn(0) .. fn(count - 1) replayed from an
+    uploaded CUDA graph behind the stream-holding spin (after 3 warm-up calls)."""
+    for i in range(3):
+        fn(i)
+    g = capture(fn, count)
+    g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(replays):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        hold_stream()
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) / 1e3 / count)
+    del g
+    return float(np.median(ts))
+
+
 def time_events(fn, reps):
     """Average device time of fn() over reps calls (CUDA events, current stream)."""
     torch.cuda.synchronize()
@@ -366,10 +387,12 @@ def side_measurements(lq, dev, args):
     x = workloads.activations(m, k, seed=1).to(dev)
     y = torch.empty((m, n), dtype=torch.float32, device=dev)
     ws = lq.new_workspace(m, n, k, bits, dev)
-    call = lambda i: lq.lutq_gemm(x, packed, cb, bits, n, k, y=y, workspace=ws, status=st)
-    for i in range(3):
-        call(i)
-    s = time_events(call, 20)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(2, int(np.ceil(3 * l2 / packed.numel())) + 1)
+    packs_g = [packed] + [packed.clone() for _ in range(copies - 1)]
+    call = lambda i: lq.lutq_gemm(x, packs_g[i % copies], cb, bits, n, k, y=y, workspace=ws,
+                                  status=st)
+    s = time_graph(call, 20)
     assert int(st.item()) == 0
     tflops = 2.0 * m * n * k / s / 1e12
     nbytes = packed.numel() + m * k * 2 + m * n * 4
@@ -381,7 +404,7 @@ def side_measurements(lq, dev, args):
                                 "peak_source": peak_kind + " (bf16 burst)",
                                 "traffic": ncu_traffic(f"gemm_w4_m{m}_{n}x{k}", GEMM_SOURCES)},
                    "kernel": "lutq::gemm_kernel"}
-    del packed, x, y, ws
+    del packed, packs_g, x, y, ws
     # offline steps on the headline layer
     lay = workloads.layer(args.workload, args.layer)
     n, k, bits = lay.n, lay.k, args.bits
@@ -406,7 +429,6 @@ def side_measurements(lq, dev, args):
     codes_r, scales_r = lq.lutq_quantize(wr, cb, bits, status=st)
     packed_r = lq.lutq_pack(codes_r, scales_r, bits, status=st)
     del wr, codes_r, scales_r
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     copies = max(2, int(np.ceil(3 * l2 / packed_r.numel())) + 1)
     packs_r = [packed_r] + [packed_r.clone() for _ in range(copies - 1)]
     call_r = lambda i: lq.lutq_gemv_rht(x1, packs_r[i % copies], cb, signs, bits, n, k, y=y1,
@@ -509,11 +531,9 @@ def side_measurements(lq, dev, args):
     xg = workloads.activations(mg, k, seed=1).to(dev)
     yg = torch.empty((mg, n), dtype=torch.float32, device=dev)
     wsg = lq.new_workspace(mg, n, k, bits, dev)
-    call_g = lambda i: lq.lutq_gemm_group64(xg, packed_h, cb, bits, n, k, y=yg, workspace=wsg,
-                                            status=st)
-    for i in range(3):
-        call_g(i)
-    t_g = time_events(call_g, 20)
+    call_g = lambda i: lq.lutq_gemm_group64(xg, packs_h[i % copies], cb, bits, n, k, y=yg,
+                                            workspace=wsg, status=st)
+    t_g = time_graph(call_g, 20)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     err_h = float(np.linalg.norm(y_h.double().cpu().numpy() - exact) / np.linalg.norm(exact))
