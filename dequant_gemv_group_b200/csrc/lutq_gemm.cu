@@ -7,7 +7,8 @@
 // Roles of the warps of a CTA (one CTA per SM, persistent; the counts depend
 // on the batch tile N_tile, GemmCfg):
 //   DW dequantize warps (4 at N_tile >= 64, else 8: two per lane quarter,
-//              each taking half of the row's codes): lane r of warp w owns
+//              each taking half of the row's codes; 16 quarter-row warps in
+//              the typed 4-bit kernel at N_tile = 16): lane r of warp w owns
 //              row 32 (w mod 4) + r of the 128-row tile; it decodes its codes
 //              of one group through the lane-duplicated pair table into bf16
 //              pairs and stores them into tensor memory (lane = row, column
@@ -53,7 +54,7 @@ constexpr int kTileRows = 128;
 constexpr int kGemmMaxCtas = 256;            // bounds the workspace
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kTmemCols = 512;
-template <int NT, bool G64 = false, bool TYPED = false>
+template <int NT, bool G64 = false, bool TYPED = false, int BITS = 4>
 struct GemmCfg {
   // activation stages (shared memory); two at N_tile = 128 leave 32 KB more
   // to L1 (measured 2% faster at batch 128 than three; four: 25% slower)
@@ -76,8 +77,15 @@ struct GemmCfg {
   static constexpr int AS = ((G64 || TACC) && NT >= 128) ? 2 : 4;
   static constexpr int DS = G64 ? ((kTmemCols - 64 * AS) / NT < 8 ? (kTmemCols - 64 * AS) / NT : 8)
                                 : (NT >= 128 ? 2 : (NT >= 64 ? 3 : 4));
-  static constexpr int DW = NT >= 64 ? 4 : 8;       // dequant warps (8: two per lane quarter)
-  static constexpr int NB = DW == 8 ? 4 : 2;        // units of packed words in flight per lane
+  // dequant warps: 4 (a whole row per lane) at N_tile >= 64; below it 8 (two
+  // per lane quarter, half a row each) or, for the typed kernel with 4-bit
+  // codes at N_tile = 16, 16 (a quarter of a row each: one 16-byte word per
+  // lane and unit).  Measured on the 70B gate/up layer at batch 16: the typed
+  // kernel takes 62.0 us with 16 warps against 67.1 us with 8, while the
+  // untyped kernel takes 53.4 us with 16 against 50.5 us with 8.  At N_tile
+  // = 32 the 23 warps' register share (80) would spill the promotion sums.
+  static constexpr int DW = NT >= 64 ? 4 : (TYPED && BITS == 4 && NT <= 16 ? 16 : 8);
+  static constexpr int NB = DW >= 8 ? 4 : 2;        // units of packed words in flight per lane
   static constexpr int KC = 64 * 4 / DW;            // A columns written per dequant warp
   static constexpr int PG = NT >= 128 ? 2 : 1;      // promotion warp groups
   static constexpr int NC = NT / PG;                // batch columns per promotion warp
@@ -91,8 +99,8 @@ struct GemmCfg {
 constexpr int kMaxPromoteGroups = 2;
 constexpr int kScaleRingBytes = 4 * kMaxPromoteGroups * 4 * 32 * 4;  // [warp][SD][lane] u32
 // per-group types: the dequant warps' type words travel through a ring of
-// asynchronous copies, [warp][NB][lane] u32 (at most 8 warps x 4 units)
-constexpr int kTypeRingBytes = 8 * 4 * 32 * 4;
+// asynchronous copies, [warp][NB][lane] u32 (at most 16 warps x 4 units)
+constexpr int kTypeRingBytes = 16 * 4 * 32 * 4;
 
 struct GemmArgs {
   const uint8_t* packed;
@@ -253,10 +261,21 @@ __device__ __forceinline__ void tmem_st_cols32(uint32_t taddr, const uint32_t (&
       : "memory");
 }
 
+// Each thread of the warp stores v[0..15] to 16 consecutive 32-bit columns of its lane.
+__device__ __forceinline__ void tmem_st_cols16(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
 template <int BITS, int NT, bool TYPED, bool G64>
-__global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
+__global__ void __launch_bounds__(GemmCfg<NT, G64, TYPED, BITS>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, GemmArgs a) {
-  using Cfg = GemmCfg<NT, G64, TYPED>;
+  using Cfg = GemmCfg<NT, G64, TYPED, BITS>;
   static_assert(!(TYPED && G64), "per-group types use one scale per group of 128");
   // partials per unit (one per scale), the scale block's bytes
   constexpr int H = G64 ? 2 : 1;
@@ -346,12 +365,15 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
     // instruction): a 2 KB bulk copy per strip and unit costs the copy
     // engine about as much as 16 KB of data, and would hold the kernel to
     // about a quarter of the HBM bandwidth.
-    const int sw = warp & 3, kh = DW == 8 ? (warp >> 2) : 0;
+    const int sw = warp & 3, kh = DW >= 8 ? (warp >> 2) : 0;
     const uint32_t off_e = uint32_t(lane) * 4u, off_o = 128u + uint32_t(lane) * 4u;
-    constexpr int NWL = DW == 8 ? 2 : WPR;  // 16-byte words per lane and unit
-    // word j of the lane's words: 4-bit, words 2kh, 2kh+1 (DW = 8) or all;
-    // 3-bit, lo word kh and the hi word (DW = 8) or all three
-    auto word_of = [&](int j) { return DW == 8 ? (BITS == 4 ? 2 * kh + j : (j == 0 ? kh : 2)) : j; };
+    static_assert(DW != 16 || BITS == 4, "quarter rows need 4-bit codes");
+    constexpr int NWL = DW == 16 ? 1 : (DW == 8 ? 2 : WPR);  // 16-byte words per lane and unit
+    // word j of the lane's words: 4-bit, word kh (DW = 16), words 2kh, 2kh+1
+    // (DW = 8) or all; 3-bit, lo word kh and the hi word (DW = 8) or all three
+    auto word_of = [&](int j) {
+      return DW == 16 ? kh : DW == 8 ? (BITS == 4 ? 2 * kh + j : (j == 0 ? kh : 2)) : j;
+    };
     UnitPos fp;  // the next unit to fetch
     fp.init(u0, per_bt, a.G);
     int fetched = 0;
@@ -424,9 +446,17 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
         // a stored type without a table in this call is reported (once, after the loop)
         if (TYPED)
           bad_type |= ((ty >> (8 * (lane & 3) + 2 * (lane >> 3))) & 3u) >= uint32_t(a.ntypes);
-        const uint4 h0[2] = {wd[0], wd[DW == 8 ? 1 : (BITS == 4 ? 1 : 2)]};
-        decode_group_half<BITS>(av, h0, DW == 8 ? kh : 0, lut_sa, off_e | sel, off_o | sel,
-                                uint32_t(LUTB), a.dev_status);
+        if (DW == 16) {
+          // a quarter row: the 16 pairs of word kh
+          const uint32_t v[4] = {wd[0].x, wd[0].y, wd[0].z, wd[0].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            lookup4(av + 4 * j, v[j], lut_sa, off_e | sel, uint32_t(LUTB), a.dev_status);
+        } else {
+          const uint4 h0[2] = {wd[0], wd[DW == 8 ? NWL - 1 : (BITS == 4 ? 1 : 2)]};
+          decode_group_half<BITS>(av, h0, DW == 8 ? kh : 0, lut_sa, off_e | sel, off_o | sel,
+                                  uint32_t(LUTB), a.dev_status);
+        }
       }
       fetch(wd, slot);
       const int as = i % AS;
@@ -437,8 +467,12 @@ __global__ void __launch_bounds__(GemmCfg<NT>::THREADS, 1)
       }
       tc_fence_after();
       if (valid) {
-        const uint32_t ta = tmem + (uint32_t(sw * 32) << 16) + uint32_t(as * 64 + kh * 32);
-        tmem_st_cols32(ta, av);
+        const uint32_t ta =
+            tmem + (uint32_t(sw * 32) << 16) + uint32_t(as * 64 + kh * (DW == 16 ? 16 : 32));
+        if (DW == 16)
+          tmem_st_cols16(ta, av);
+        else
+          tmem_st_cols32(ta, av);
         if (DW == 4) {
           decode_group_half<BITS>(av, h1, 1, lut_sa, off_e | sel, off_o | sel, uint32_t(LUTB),
                                   a.dev_status);
@@ -719,7 +753,7 @@ static cudaError_t make_x_map(CUtensorMap* map, const void* x, int64_t M, int64_
 template <int BITS, int NT, bool TYPED, bool G64>
 static cudaError_t launch_nt(const CUtensorMap& map, GemmArgs a, int num_sms,
                              cudaStream_t stream) {
-  using Cfg = GemmCfg<NT, G64, TYPED>;
+  using Cfg = GemmCfg<NT, G64, TYPED, BITS>;
   static int granted[64] = {0};
   // alignment slack, table, activation stages, barriers and flags (512),
   // the promotion warps' scale rings (two scales per lane and unit with G64)
